@@ -1,0 +1,236 @@
+"""Float64 CPU oracle for TriAttention KV-cache pruning (test infrastructure).
+
+This package is the correctness reference for the CUDA library.  Only the
+tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py``
+may import it.  The library under ``rope_aware_kv_b200`` never imports,
+links or calls anything here, and the two share no code.
+
+The arithmetic lives in ``tri_oracle.c`` (plain C, double precision, OpenMP
+over units); this module compiles it with gcc and marshals numpy arrays.
+Every function follows the pages step by step:
+
+* ``calibrate`` -- per-band query centre, mean norm and R_f = |E q_f| / E|q_f|
+  (TriAttention talk announcement, qingkeai.online: S_norm equation and the
+  R_f definition; hyper.ai summary of arXiv 2604.04921, Method section).
+* ``score`` -- de-rotate each post-RoPE key by its position, then the explicit
+  S_trig + S_norm sum averaged over the offsets D (talk page: RoPE rotation,
+  RoPE logit general form, S_trig, S_norm and S~ equations).
+* ``znorm_max`` -- z-score per query head, max over the GQA group (hyper.ai
+  summary, Method section, "normalise then aggregate").
+* ``select`` -- top-B by (score desc, index asc), returned ascending
+  (jaedaily.cn KV-compression tutorial, eviction step).
+* ``prune`` -- all of the above plus the bit-exact gather, over many units.
+
+Parity status: every function is pinned by the ``-m "not gpu"`` tests in
+``tests/test_oracle_pins.py`` against closed forms, brute force and
+invariants; absolute score values at real-model scale are unpinned because the
+pages print no worked example.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "tri_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+F32 = 0
+BF16 = 1
+
+# The pages' constants: theta = 10000 and D = {1, 2, 4, ..., 2^16} (talk page,
+# RoPE rotation and the offset-averaged score S~).
+THETA = 10000.0
+OFFSETS = tuple(1 << i for i in range(17))
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``liboracle.so`` next to its source with gcc (IEEE math, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-Wall", "-Wextra", "-fopenmp", "-shared", "-fPIC",
+               "-o", _LIB, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+    return _LIB
+
+
+def _load():
+    if _lib is None:
+        build()
+        _bind(ctypes.CDLL(_LIB))
+    return _lib
+
+
+def _bind(lib):
+    global _lib
+    P = ctypes.c_void_p
+    i64 = ctypes.c_int64
+    i32 = ctypes.c_int
+    d = ctypes.c_double
+    lib.oracle_calibrate.argtypes = [P, i32, i64, i64, i32, P]
+    lib.oracle_calibrate.restype = i32
+    lib.oracle_score.argtypes = [P, i32, i64, i32, P, i64, P, i32, d, P, i32, P]
+    lib.oracle_score.restype = i32
+    lib.oracle_znorm_max.argtypes = [P, i32, i64, P, P, P, P]
+    lib.oracle_znorm_max.restype = i32
+    lib.oracle_select.argtypes = [P, i64, i64, P, P]
+    lib.oracle_select.restype = i64
+    lib.oracle_prune.argtypes = [P, P, P, i32, i64, i64, i64, i32, i64, i32, P, P, P, d, P,
+                                 i32, i64, P, P, P, P, P, P, P, P, i64, P, i64]
+    lib.oracle_prune.restype = i32
+    lib.oracle_threads.argtypes = []
+    lib.oracle_threads.restype = i32
+    lib.oracle_set_threads.argtypes = [i32]
+    lib.oracle_set_threads.restype = None
+    _lib = lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _elem(a: np.ndarray):
+    """Map a numpy key/query array to (contiguous array, oracle dtype code).
+
+    float32 arrays are float32; uint16 arrays hold raw bfloat16 bit patterns.
+    """
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.float32:
+        return a, F32
+    if a.dtype == np.uint16:
+        return a, BF16
+    raise TypeError(f"oracle takes float32 or raw-bf16 uint16 arrays, got {a.dtype}")
+
+
+class using_library:
+    """Temporarily route every call through another build of the oracle
+    (used by the mutation tests, which compile deliberately broken copies)."""
+
+    def __init__(self, path: str):
+        self.path = path
+        self.saved = None
+
+    def __enter__(self):
+        global _lib
+        self.saved = _load()
+        _lib = None
+        _bind(ctypes.CDLL(self.path))
+        return self
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self.saved
+        return False
+
+
+def threads() -> int:
+    return int(_load().oracle_threads())
+
+
+def set_threads(n: int) -> None:
+    _load().oracle_set_threads(int(n))
+
+
+def calibrate(q: np.ndarray) -> np.ndarray:
+    """q: [H, n_tok, d] pre-RoPE queries -> stats [H, d/2, 4] (re, im, mean|q_f|, R_f)."""
+    q, dt = _elem(q)
+    H, n, d = q.shape
+    out = np.empty((H, d // 2, 4), np.float64)
+    rc = _load().oracle_calibrate(_ptr(q), dt, H, n, d, _ptr(out))
+    if rc:
+        raise ValueError(f"oracle_calibrate failed ({rc})")
+    return out
+
+
+def score(k: np.ndarray, pos: np.ndarray, p_cur: int, stats: np.ndarray,
+          theta: float = THETA, offsets=OFFSETS) -> np.ndarray:
+    """Per-head S~ for one unit: k [n, d] post-RoPE, pos [n], stats [G, d/2, 4] -> [G, n]."""
+    k, dt = _elem(k)
+    n, d = k.shape
+    pos = np.ascontiguousarray(pos, np.int32)
+    st = np.ascontiguousarray(stats, np.float64)
+    G = st.shape[0]
+    off = np.ascontiguousarray(np.asarray(offsets, np.int64))
+    out = np.empty((G, n), np.float64)
+    rc = _load().oracle_score(_ptr(k), dt, n, d, _ptr(pos), int(p_cur), _ptr(st), G,
+                              float(theta), _ptr(off), len(off), _ptr(out))
+    if rc:
+        raise ValueError(f"oracle_score failed ({rc})")
+    return out
+
+
+def znorm_max(raw: np.ndarray):
+    """raw [G, n] -> (z [G, n], final [n], mu [G], sigma [G])."""
+    raw = np.ascontiguousarray(raw, np.float64)
+    G, n = raw.shape
+    z = np.empty((G, n), np.float64)
+    fin = np.empty((n,), np.float64)
+    mu = np.empty((G,), np.float64)
+    sd = np.empty((G,), np.float64)
+    rc = _load().oracle_znorm_max(_ptr(raw), G, n, _ptr(z), _ptr(fin), _ptr(mu), _ptr(sd))
+    if rc:
+        raise ValueError(f"oracle_znorm_max failed ({rc})")
+    return z, fin, mu, sd
+
+
+def select(final: np.ndarray, B: int):
+    """final [n] -> (kept indices ascending [min(B, n)], B-th score)."""
+    fin = np.ascontiguousarray(final, np.float64)
+    n = fin.shape[0]
+    kept = np.empty((max(min(B, n), 1),), np.int32)
+    thr = ctypes.c_double(0.0)
+    m = _load().oracle_select(_ptr(fin), n, int(B), _ptr(kept), ctypes.byref(thr))
+    if m < 0:
+        raise ValueError("oracle_select failed")
+    return kept[:m].copy(), thr.value
+
+
+def prune(k, v, pos, n_seq, n_layers, n_kvheads, G, stats, p_cur, B, n_valid=None,
+          theta=THETA, offsets=OFFSETS, units=None, want_raw=True, want_gather=True):
+    """Whole prune step on [U, cap, d] caches (see tri_oracle.c: oracle_prune).
+
+    stats: [n_layers, n_kvheads*G, d/2, 4] float64.  Returns a dict with
+    raw [U, G, cap], final [U, cap], kept [U, B], n_kept [U], thr [U] and,
+    when ``want_gather``, k_dst / v_dst [U, B, d] and pos_dst [U, B].  Rows of
+    units not in ``units`` are left as NaN / -1 / zero.
+    """
+    k, dt = _elem(k)
+    v2, dtv = _elem(v) if v is not None else (None, dt)
+    if v2 is not None and dtv != dt:
+        raise TypeError("k and v must share a dtype")
+    U, cap, d = k.shape
+    if U != n_seq * n_layers * n_kvheads:
+        raise ValueError("k.shape[0] must equal n_seq * n_layers * n_kvheads")
+    pos = np.ascontiguousarray(pos, np.int32)
+    st = np.ascontiguousarray(stats, np.float64)
+    pc = np.ascontiguousarray(np.asarray(p_cur, np.int64).reshape(-1))
+    nv = None if n_valid is None else np.ascontiguousarray(np.asarray(n_valid, np.int32))
+    off = np.ascontiguousarray(np.asarray(offsets, np.int64))
+    ul = None if units is None else np.ascontiguousarray(np.asarray(units, np.int64))
+    raw = np.full((U, G, cap), np.nan) if want_raw else None
+    fin = np.full((U, cap), np.nan)
+    kept = np.full((U, max(B, 1)), -1, np.int32)
+    nk = np.zeros((U,), np.int64)
+    thr = np.full((U,), np.nan)
+    kd = vd = pd = None
+    if want_gather:
+        kd = np.zeros((U, B, d), k.dtype)
+        vd = np.zeros((U, B, d), k.dtype) if v2 is not None else None
+        pd = np.full((U, B), -1, np.int32)
+    rc = _load().oracle_prune(
+        _ptr(k), _ptr(v2), _ptr(pos), dt, n_seq, n_layers, n_kvheads, G, cap, d, _ptr(nv),
+        _ptr(pc), _ptr(st), float(theta), _ptr(off), len(off), int(B), _ptr(raw), _ptr(fin),
+        _ptr(kept), _ptr(nk), _ptr(thr), _ptr(kd), _ptr(vd), _ptr(pd), B if want_gather else 0,
+        _ptr(ul), 0 if ul is None else len(ul))
+    if rc:
+        raise ValueError(f"oracle_prune failed ({rc})")
+    out = dict(final=fin, kept=kept[:, :B], n_kept=nk, thr=thr)
+    if want_raw:
+        out["raw"] = raw
+    if want_gather:
+        out.update(k_dst=kd, v_dst=vd, pos_dst=pd)
+    return out

@@ -1,0 +1,505 @@
+"""Benchmark of one TriAttention prune step on B200 (libtri, sm_100a).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2]
+                    [--impl reference]
+
+A step is one pass of the whole prune path (fold, score, z-normalise / max,
+top-B select, order-preserving gather of K, V and positions) over every unit
+of the workload.  Units are independent, so at N GPUs every rank prunes its
+own copy of the workload (weak scaling, no collective on the data path) and
+``value`` counts the keys of all ranks over the slowest rank's time.
+
+Default workload: one layer, GQA 28 query / 4 KV heads, 32768 bf16 keys per
+head, budget 2048 (the second workload configuration; the first is the small
+single-head fp32 case the oracle finishes in seconds).  Metric: keys scored
+and pruned per second, plus the achieved HBM bandwidth of the step's
+compulsory bytes (read every key, read the kept values, write the kept keys
+and values, indices and positions) against the measured copy peak.
+
+Timing: W warm-up steps, then K steps captured as one CUDA graph and replayed
+between CUDA events on the launching stream, with a barrier and a device
+synchronise on both sides; the inputs rotate over enough copies that their
+total exceeds the 126 MB L2 (no step reads a cache another step left in L2).
+Per-kernel durations come from events the library records after each of its
+launches inside the same graph.  ``e2e`` repeats the step through the public
+Python API with host (pinned) buffers: the copy of the inputs in and of the
+compacted cache out is inside its timed region.
+
+``--impl reference`` times the float64 CPU oracle (the baseline) on the host
+cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+METRIC = "keys scored+pruned/sec and achieved HBM GB/s (% of measured copy peak) per prune step"
+
+WORKLOAD_TEXT = {
+    "c1": "single head fp32, 4096 keys -> 512, G=1",
+    "c2": "1 layer, GQA 28/4, 32768 bf16 keys per KV head -> 2048",
+    "c3": "windowed decode step, 28 layers x 4 KV heads x 16 seqs, 3200 -> 3072 keys, G=7",
+    "c4": "long prefill compaction, 32 layers x 8 KV heads x 4 seqs, 131072 -> 4096 keys, G=4",
+    "c5": "streaming step, 28 layers x 4 KV heads x 64 seqs, 2176 -> 2048 keys, G=7",
+}
+
+
+def compulsory_bytes(spec) -> int:
+    """Per step: read every valid key, read the kept values, write the kept
+    keys and values, plus 4-byte index and position of every kept row read and
+    written (12 bytes per kept key)."""
+    e = spec.esize
+    m = min(spec.n_valid, spec.B)
+    per_unit = spec.n_valid * spec.d * e + m * spec.d * e + 2 * m * spec.d * e + 12 * m
+    return per_unit * spec.n_units
+
+
+def score_bytes(spec) -> int:
+    """Algorithmic bytes of the score kernel per launch: every valid key read once."""
+    return spec.n_units * spec.n_valid * spec.d * spec.esize
+
+
+def fused_bytes(spec) -> int:
+    return compulsory_bytes(spec)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks (NVML polled in a thread during the timed region)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self.ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread:
+            self._stop.set()
+            self._thread.join()
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        reasons = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
+        med = statistics.median(self.samples) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# the oracle (CPU baseline and reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample(spec, seconds_hint: float = 15.0):
+    """Bounded sample of the workload for the CPU oracle: a few units drawn
+    from the generator on the host, cut to a key count that keeps the run to
+    roughly ``seconds_hint`` seconds.  Returns (inputs, keys, description)."""
+    import oracle
+
+    threads = oracle.threads()
+    n_units = max(1, min(spec.n_units, threads))
+    # ~ 17 offsets x 64 bands x G cosines per key, about 25 ns each
+    per_key = 17 * 64 * spec.G * 25e-9
+    n_keys = int(min(spec.n_valid, max(256, seconds_hint / per_key)))
+    sub = synth.Spec(spec.name + "-sample", 1, 1, n_units, spec.G, n_keys, n_keys,
+                     min(spec.B, max(1, n_keys * spec.B // max(spec.n_valid, 1))), spec.dtype,
+                     min(spec.n_cal, 2048), spec.p_cur, positions="dense", R_range=spec.R_range,
+                     outlier_frac=spec.outlier_frac, stream=spec.stream)
+    wl = synth.make_workload(sub, "cpu")
+    q = synth.calib_queries(sub, wl.hp, 0, "cpu")
+    st = oracle.calibrate(synth.host_elems(q))[None]
+    inputs = dict(k=synth.host_elems(wl.k), v=synth.host_elems(wl.v), pos=wl.pos.numpy(),
+                  p_cur=wl.p_cur.numpy(), stats=st, sub=sub)
+    desc = (f"{n_units} unit(s) x {n_keys} keys (G={spec.G}, B={sub.B}) of {spec.name}, "
+            f"oracle with {min(n_units, threads)} thread(s)")
+    return inputs, n_units * n_keys, desc, min(n_units, threads)
+
+
+def oracle_step(inp):
+    import oracle
+
+    sub = inp["sub"]
+    oracle.prune(inp["k"], inp["v"], inp["pos"], 1, 1, sub.n_kvheads, sub.G, inp["stats"],
+                 inp["p_cur"], sub.B, want_raw=False, want_gather=True)
+
+
+def cpu_baseline(spec):
+    inp, keys, desc, cores = oracle_sample(spec)
+    t0 = time.perf_counter()
+    oracle_step(inp)
+    dt = time.perf_counter() - t0
+    return {"value": keys / dt, "unit": "keys/s", "cores": cores, "kind": "oracle",
+            "sample": desc, "seconds": round(dt, 3)}
+
+
+def run_reference(args, ws, rank):
+    if rank != 0:
+        return
+    spec = synth.SPECS[args.workload]
+    inp, keys, desc, cores = oracle_sample(spec, seconds_hint=0.5)
+    for _ in range(args.warmup):
+        oracle_step(inp)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(inp)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = keys / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "keys/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{args.workload}: {WORKLOAD_TEXT[args.workload]}",
+                   "sample": desc},
+        "cpu_baseline": {"value": value, "unit": "keys/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "keys/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+class StepRunner:
+    """Inputs, destinations and workspace of one prune step, rotated over
+    enough input copies that every step reads from HBM."""
+
+    def __init__(self, spec, device, n_copies=None):
+        import rope_aware_kv_b200 as tri
+
+        self.tri = tri
+        self.spec = spec
+        wl = synth.make_workload(spec, device)
+        self.wl = wl
+        stats = torch.empty((spec.n_layers, spec.n_qheads, 64, 4), dtype=torch.float32,
+                            device=device)
+        for layer in range(spec.n_layers):
+            q = synth.calib_queries(spec, wl.hp, layer, device)
+            tri.tri_calibrate(q, stats=stats[layer])
+            del q
+        self.stats = stats
+        copy_bytes = 2 * wl.k.numel() * wl.k.element_size() + wl.pos.numel() * 4
+        if n_copies is None:
+            n_copies = max(1, math.ceil(4 * L2_BYTES / copy_bytes))
+            free = torch.cuda.mem_get_info()[0]
+            n_copies = max(1, min(n_copies, int(0.5 * free // max(copy_bytes, 1))))
+        self.inputs = [(wl.k, wl.v, wl.pos)]
+        for _ in range(n_copies - 1):
+            self.inputs.append((wl.k.clone(), wl.v.clone(), wl.pos.clone()))
+        U, B = spec.n_units, spec.B
+        m = min(B, spec.cap)
+        self.dst = []
+        for _ in range(n_copies):
+            kd = torch.empty((U, m, spec.d), dtype=wl.k.dtype, device=device)
+            self.dst.append((kd, torch.empty_like(kd),
+                             torch.empty((U, m), dtype=torch.int32, device=device)))
+        self.n_kept = torch.empty((U,), dtype=torch.int32, device=device)
+        self.kept = torch.empty((U, B), dtype=torch.int32, device=device)
+        self.ws = tri.workspace(tri.tri_prune_workspace_bytes(
+            spec.n_seq, spec.n_layers, spec.n_kvheads, spec.G, spec.cap, B))
+        self.cfg = tri.config()
+        self.n_copies = n_copies
+
+    def step(self, i):
+        k, v, pos = self.inputs[i % self.n_copies]
+        kd, vd, pd = self.dst[i % self.n_copies]
+        s = self.spec
+        self.tri.tri_prune(self.cfg, k, v, pos, s.n_seq, s.n_layers, s.n_kvheads, s.G,
+                           self.wl.p_cur, self.stats, s.B, kd, vd, pd, self.n_kept,
+                           n_valid=self.wl.n_valid, kept=self.kept, ws=self.ws)
+
+
+def run_tri(args, ws, rank, local):
+    import rope_aware_kv_b200 as tri
+    from rope_aware_kv_b200 import build as tri_build
+
+    if rank == 0:
+        tri_build.build()
+    barrier(ws)
+    tri.load()
+    spec = synth.SPECS[args.workload]
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    runner = StepRunner(spec, dev)
+    stream = torch.cuda.Stream(device=dev)
+    peak_gbs, peak_kind = measured_peaks()
+
+    with torch.cuda.stream(stream):
+        # Eager warm-up (also initialises the library's static state).
+        for i in range(max(args.warmup, 3)):
+            runner.step(i)
+        torch.cuda.synchronize()
+        tri.tri_set_timing_events(None)
+        runner.step(0)
+        launches = tri.tri_last_launch_count()
+
+        # Per-launch events inside the timed graph.
+        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(launches)]
+               for _ in range(args.steps)]
+        starts = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(args.steps)]
+        for e in starts + [x for row in evs for x in row]:
+            e.record(stream)
+        torch.cuda.synchronize()
+
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+            for i in range(args.steps):
+                starts[i].record(stream)
+                tri.tri_set_timing_events(evs[i])
+                runner.step(args.warmup + i)
+            tri.tri_set_timing_events(None)
+        gw = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gw, stream=stream, capture_error_mode="relaxed"):
+            for i in range(args.warmup):
+                runner.step(i)
+
+    clocks = ClockSampler(local)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    gw.replay()
+    torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+    clocks.start()
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        g.replay()
+        t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(ws)
+    ms_total = t0.elapsed_time(t1)
+    ms_max = max_over_ranks(ms_total, ws)
+    ms_step = ms_max / args.steps
+
+    # Per-kernel durations (first launch includes the workspace memsets).
+    per_launch = np.zeros(launches)
+    for i in range(args.steps):
+        prev = starts[i]
+        for j in range(launches):
+            per_launch[j] += prev.elapsed_time(evs[i][j])
+            prev = evs[i][j]
+    per_launch /= args.steps
+    flags = tri.tri_check_device_error(runner.ws)
+
+    keys_rank = spec.n_units * spec.n_valid
+    value = keys_rank * ws / (ms_step * 1e-3)
+    comp = compulsory_bytes(spec)
+    step_gbs = comp / (ms_step * 1e-3) / 1e9
+
+    # Dominant kernel and its algorithmic bytes.
+    dom = int(np.argmax(per_launch))
+    fused = launches <= 2
+    if fused:
+        dom_name, dom_bytes = "prune_fused_kernel", fused_bytes(spec)
+    else:
+        names = ["fold", "score", "zmax_hist", "radix_pass1", "radix_pass2", "select_count",
+                 "select_compact", "gather"]
+        dom_name = names[dom] if dom < len(names) else f"launch{dom}"
+        gather_bytes = spec.n_units * min(spec.B, spec.n_valid) * (3 * spec.d * spec.esize + 12)
+        byts = {"score": score_bytes(spec), "gather": gather_bytes}
+        dom_bytes = byts.get(dom_name, 0)
+    dom_ms = float(per_launch[dom])
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9 if dom_ms > 0 else 0.0
+
+    e2e = run_e2e(args, runner, stream, spec, ws)
+    cpu = cpu_baseline(spec) if (rank == 0 and ws == 1 and not args.no_cpu_baseline) else None
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "keys/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if spec.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": {
+                "workload": f"{args.workload}: {WORKLOAD_TEXT[args.workload]}",
+                "units": spec.n_units, "keys_per_unit": spec.n_valid, "budget": spec.B,
+                "group": spec.G, "head_dim": spec.d, "parallelism": f"dp{ws} (independent units)",
+                "l2": f"inputs rotated over {runner.n_copies} copies "
+                      f"({runner.n_copies * comp / 2**20:.0f} MiB compulsory > 126 MB L2)",
+                "timing": "one CUDA graph of K steps between CUDA events, max over ranks",
+            },
+            "hbm_gbs": step_gbs, "hbm_frac_of_peak": step_gbs / peak_gbs,
+            "compulsory_bytes_per_step": comp,
+            "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": achieved,
+                         "peak": peak_gbs, "peak_kind": peak_kind, "unit": "GB/s",
+                         "frac": achieved / peak_gbs, "traffic": None,
+                         "algorithmic_bytes": dom_bytes, "ms_per_launch": dom_ms},
+            "per_launch_ms": [round(float(x), 5) for x in per_launch],
+            "gpu_launches": int(launches * args.steps),
+            "device_flags": flags,
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, runner, stream, spec, ws):
+    """The same step through the Python API with host buffers: pinned host
+    inputs copied in, the prune, and the compacted cache copied out."""
+    tri = runner.tri
+    wl = runner.wl
+    hk = wl.k.cpu().pin_memory()
+    hv = wl.v.cpu().pin_memory()
+    hp = wl.pos.cpu().pin_memory()
+    k, v, pos = runner.inputs[0]
+    kd, vd, pd = runner.dst[0]
+    ok = torch.empty(kd.shape, dtype=kd.dtype).pin_memory()
+    ov = torch.empty(vd.shape, dtype=vd.dtype).pin_memory()
+    op = torch.empty(pd.shape, dtype=pd.dtype).pin_memory()
+    steps = max(3, min(args.steps, 20))
+
+    def one():
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        pos.copy_(hp, non_blocking=True)
+        tri.tri_prune(runner.cfg, k, v, pos, spec.n_seq, spec.n_layers, spec.n_kvheads, spec.G,
+                      wl.p_cur, runner.stats, spec.B, kd, vd, pd, runner.n_kept,
+                      n_valid=wl.n_valid, kept=runner.kept, ws=runner.ws)
+        ok.copy_(kd, non_blocking=True)
+        ov.copy_(vd, non_blocking=True)
+        op.copy_(pd, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        one()
+        torch.cuda.synchronize()
+        barrier(ws)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            one()
+        b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b), ws) / steps
+    h2d = hk.numel() * hk.element_size() + hv.numel() * hv.element_size() + hp.numel() * 4
+    d2h = ok.numel() * ok.element_size() + ov.numel() * ov.element_size() + op.numel() * 4
+    return {"value": spec.n_units * spec.n_valid * ws / (ms * 1e-3), "unit": "keys/s",
+            "ms_per_step": ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": steps}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="tri", choices=["tri", "reference"])
+    ap.add_argument("--workload", default="c2", choices=sorted(synth.SPECS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    ws, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, ws, rank)
+        else:
+            run_tri(args, ws, rank, local)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

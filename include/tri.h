@@ -1,0 +1,296 @@
+/*
+ * tri.h -- C ABI of libtri, a B200 (sm_100a) implementation of the KV-cache
+ * pruning hot path of TriAttention ("TriAttention: Efficient Long Reasoning
+ * with Trigonometric KV Compression", arXiv 2604.04921).
+ *
+ * The method, as the pages state it:
+ *   - RoPE rotates each pair (x_2f, x_2f+1) of a d-wide head vector by the
+ *     angle w_f p, w_f = theta^(-2f/d), theta = 10000
+ *     (TriAttention talk announcement, qingkeai.online: RoPE rotation equation;
+ *     hyper.ai summary of arXiv 2604.04921, Method section).
+ *   - Offline calibration collects, per query head and band f, the centre
+ *     E[q_f], the mean norm E[|q_f|] and R_f = |E[q_f]| / E[|q_f|] from
+ *     pre-RoPE queries (talk page: S_norm equation and the R_f definition;
+ *     shibing624 paper reading, "complete scoring framework", step 1).
+ *   - Each cached key k is scored with
+ *         S_trig(k, Delta) = sum_f |E[q_f]| |k_f| cos(w_f Delta + phi_f)
+ *         S_norm(k)        = sum_f (1 - R_f) E[|q_f|] |k_f|
+ *     averaged over the future offsets D = {1, 2, 4, ..., 2^16}
+ *     (talk page: S_trig, S_norm and the offset-averaged score S~).
+ *   - Scores are z-normalised per query head and combined by max over each
+ *     GQA group (hyper.ai summary, Method section, "normalise then aggregate").
+ *   - The top-B keys are kept in their original temporal order and K/V are
+ *     gathered into a compacted cache (jaedaily.cn KV-compression tutorial,
+ *     eviction step: top-k, then sort to keep the temporal order).
+ *   - Scoring and pruning fire once every 128 generated tokens (hyper.ai
+ *     summary, Method section).
+ *
+ * How the library computes S~ (exact algebra, no approximation): with
+ * phi_f = arg E[q_f] - arg k_f, the trigonometric term of band f equals
+ * Re(E[q_f] conj(k_f) e^{i w_f Delta}).  The pre-RoPE key is
+ * k_f = k'_f e^{-i w_f p_k} and Delta = p_cur + delta - p_k, so the key's own
+ * position cancels and the average over D is Re(A_f conj(k'_f)) with
+ * A_f = E[q_f] e^{i w_f p_cur} C_f and C_f = (1/|D|) sum_delta e^{i w_f delta}.
+ * The per-head fold A_f is computed in float64 on the device; the per-key work
+ * is one 128-wide dot product plus 64 band norms per query head, in float32.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Pointers are DEVICE pointers unless a comment says "host".  The caller
+ * allocates every buffer, including the workspace ("ws"); the library
+ * allocates, frees and retains nothing and keeps no state between calls.
+ * Calls are asynchronous on the given CUDA stream ("stream" is a
+ * cudaStream_t passed as void*; NULL is the legacy default stream) and are
+ * safe to capture in a CUDA graph.  Two calls that share a workspace must not
+ * overlap on the GPU.
+ *
+ * Layouts:
+ *   unit u = (seq * n_layers + layer) * n_kvheads + kvh: one KV head's cache.
+ *   K, V:   [U][cap][head_dim] row-major, element type dt, 16-byte aligned.
+ *   pos:    [U][cap] int32 token positions of the cached rows.
+ *   n_valid:[U] int32 number of valid rows of each unit (NULL: every unit
+ *           holds cap rows).  Rows >= n_valid are ignored.
+ *   p_cur:  [n_seq] int64 current position of each sequence (the position of
+ *           the next query).  Future queries sit at p_cur + delta.
+ *   stats:  [n_layers][n_kvheads * G][head_dim/2][4] float32 calibration
+ *           (Re E[q_f], Im E[q_f], E[|q_f|], R_f); query head kvh*G + g
+ *           belongs to KV head kvh (contiguous GQA groups).
+ *
+ * Selection semantics: keys are ranked by final score descending; NaN ranks
+ * below every number; -0.0 equals +0.0; equal scores rank by ascending index.
+ * The kept set is the first min(B, n_valid) keys of that ranking, written in
+ * ascending index order.
+ *
+ * Errors: arguments are validated on the host before anything is launched
+ * (TRI_ERR_INVALID_ARG, TRI_ERR_UNSUPPORTED, TRI_ERR_WORKSPACE); a failed
+ * launch returns TRI_ERR_CUDA.  Conditions only the device can see (n_valid
+ * outside [0, cap], a kept index outside the source cache, a non-finite final
+ * score) set bits in a flag word at the start of the workspace, which each
+ * call clears when it starts; tri_check_device_error reads it.
+ */
+#ifndef TRI_H_
+#define TRI_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum tri_status {
+    TRI_OK = 0,
+    TRI_ERR_INVALID_ARG = 1, /* null / misaligned pointer, bad size or shape */
+    TRI_ERR_UNSUPPORTED = 2, /* valid but not implemented (head_dim, G, dtype) */
+    TRI_ERR_WORKSPACE = 3,   /* ws is NULL or smaller than the *_workspace_bytes query */
+    TRI_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
+    TRI_ERR_DEVICE = 5       /* tri_check_device_error found a device-side flag */
+} tri_status;
+
+typedef enum tri_dtype {
+    TRI_F32 = 0, /* IEEE float32 */
+    TRI_BF16 = 1 /* bfloat16 */
+} tri_dtype;
+
+/* Device flag bits (tri_check_device_error). */
+#define TRI_FLAG_NVALID_RANGE 0x1u /* some n_valid[u] outside [0, cap]; clamped */
+#define TRI_FLAG_INDEX_RANGE 0x2u  /* a kept index outside [0, cap_src) or n_kept > B; row skipped */
+#define TRI_FLAG_NONFINITE 0x4u    /* a final score was NaN (ranked last) */
+#define TRI_FLAG_TIMEOUT 0x8u      /* a bounded wait inside a kernel gave up */
+
+#define TRI_MAX_OFFSETS 64
+#define TRI_MAX_GROUP 8
+
+/* Method parameters.  tri_config_default fills the pages' values. */
+/* Kernel path of tri_prune. */
+#define TRI_PATH_AUTO 0  /* fused kernel when the unit fits in shared memory, else split */
+#define TRI_PATH_FUSED 1 /* one CTA per unit (TRI_ERR_UNSUPPORTED if it does not fit) */
+#define TRI_PATH_SPLIT 2 /* separate score / z-max / select / gather kernels */
+
+typedef struct tri_config {
+    int head_dim;                      /* d; 128 is supported */
+    double theta;                      /* RoPE base, 10000 */
+    int n_offsets;                     /* |D|, 1..TRI_MAX_OFFSETS */
+    int64_t offsets[TRI_MAX_OFFSETS];  /* future offsets delta >= 0 */
+    int path;                          /* TRI_PATH_* (tri_prune only) */
+} tri_config;
+
+/* Fill cfg (host) with head_dim, theta = 10000, D = {2^0, ..., 2^16}
+ * (talk page, offset-averaged score S~) and TRI_PATH_AUTO. */
+void tri_config_default(tri_config* cfg, int head_dim);
+
+/* Human-readable name of a status code (static string). */
+const char* tri_status_str(tri_status s);
+
+/* Library version string (static). */
+const char* tri_version(void);
+
+/* ---------------------------------------------------------------------- */
+/* Calibration (offline, once per model)                                   */
+/* ---------------------------------------------------------------------- */
+
+/* Workspace bytes tri_calibrate needs for n_heads heads of n_tok tokens. */
+size_t tri_calibrate_workspace_bytes(int64_t n_heads, int64_t n_tok, int head_dim);
+
+/*
+ * Per-head, per-band query statistics from pre-RoPE queries
+ * (talk page: R_f = |E[q_f]| / E[|q_f|]; paper reading, offline calibration
+ * on about 10K tokens; hyper.ai summary, R = |E[q]| / E[|q|]).
+ *   q_pre:  [n_heads][n_tok][head_dim] pre-RoPE queries (dt); n_heads is the
+ *           flattened [n_layers][n_qheads].
+ *   stats:  out, [n_heads][head_dim/2][4] float32:
+ *           Re E[q_f], Im E[q_f], E[|q_f|], R_f (R_f = 1 where E[|q_f|] = 0).
+ * Sums are taken in float64 in a fixed order (bitwise deterministic).
+ * Errors: n_heads < 1, n_tok < 1, head_dim != 128 or a null pointer ->
+ * INVALID_ARG / UNSUPPORTED; ws too small -> TRI_ERR_WORKSPACE.
+ */
+tri_status tri_calibrate(const void* q_pre, tri_dtype dt, int64_t n_heads, int64_t n_tok,
+                         int head_dim, float* stats, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Score                                                                   */
+/* ---------------------------------------------------------------------- */
+
+size_t tri_score_workspace_bytes(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G,
+                                 int64_t cap, int head_dim);
+
+/*
+ * Offset-averaged score S~ of every valid key for each query head of its
+ * group, then the GQA "normalise then aggregate" final score (talk page:
+ * S_trig, S_norm, S~; hyper.ai summary, Method section).
+ *   cfg:    host pointer; theta, offsets, head_dim.
+ *   k_post: [U][cap][head_dim] post-RoPE keys (dt), 16-byte aligned.
+ *   G:      query heads per KV head, 1..TRI_MAX_GROUP.
+ *   raw:    out (nullable), [U][G][cap] float32 per-head S~.
+ *   final:  out, [U][cap] float32: max over the group of (S~ - mu_h) / sigma_h,
+ *           with mu_h, sigma_h the mean and population standard deviation of
+ *           head h's S~ over the unit's n_valid keys (z = 0 where sigma_h = 0).
+ * Entries at rows >= n_valid are not written.  Keys' positions are not needed:
+ * the fold cancels them exactly (see the header comment).
+ */
+tri_status tri_score(const tri_config* cfg, const void* k_post, tri_dtype dt, int64_t n_seq,
+                     int64_t n_layers, int64_t n_kvheads, int G, int64_t cap,
+                     const int32_t* n_valid, const int64_t* p_cur, const float* stats, float* raw,
+                     float* final_score, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Top-B selection                                                         */
+/* ---------------------------------------------------------------------- */
+
+size_t tri_select_workspace_bytes(int64_t n_units, int64_t cap, int64_t B);
+
+/*
+ * Keep the top-B keys of each unit by final score, in ascending index order
+ * (talk page: keep only the top-B; tutorial eviction step: top-k then sort).
+ * MSB-first radix select on order-preserving 32-bit keys; ties at the B-th
+ * score go to the lowest indices, so the result is unique and deterministic.
+ *   final:    [U][cap] float32 scores.
+ *   B:        budget >= 1.
+ *   kept_idx: out, [U][B] int32, ascending; slots >= n_kept[u] are set to -1.
+ *   n_kept:   out, [U] int32 = min(B, n_valid[u]).
+ */
+tri_status tri_select_topB(const float* final_score, int64_t n_units, int64_t cap,
+                           const int32_t* n_valid, int64_t B, int32_t* kept_idx, int32_t* n_kept,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Order-preserving compaction                                             */
+/* ---------------------------------------------------------------------- */
+
+size_t tri_compact_workspace_bytes(void);
+
+/*
+ * Gather the kept rows: for r < n_kept[u],
+ *   k_dst[u][r] = k_src[u][kept_idx[u][r]], v_dst likewise, pos_dst likewise
+ * (bit copies; tutorial eviction step: keys[idx], values[idx]).
+ *   k_src, v_src: [U][cap_src][head_dim] (dt); v_src/v_dst may both be NULL.
+ *   pos_src/pos_dst: [U][cap_src] / [U][cap_dst] int32; may both be NULL.
+ *   kept_idx: [U][B]; n_kept: [U].
+ *   k_dst, v_dst: [U][cap_dst][head_dim], cap_dst >= min(B, cap_src); must not
+ *   overlap the sources.
+ * Rows r >= n_kept[u] of the destination are left untouched.
+ */
+tri_status tri_compact(const void* k_src, const void* v_src, const int32_t* pos_src, tri_dtype dt,
+                       int64_t n_units, int64_t cap_src, int head_dim, const int32_t* kept_idx,
+                       const int32_t* n_kept, int64_t B, void* k_dst, void* v_dst,
+                       int32_t* pos_dst, int64_t cap_dst, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* One whole prune step (score + select + compact)                         */
+/* ---------------------------------------------------------------------- */
+
+size_t tri_prune_workspace_bytes(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G,
+                                 int64_t cap, int64_t B, int head_dim);
+
+/*
+ * One prune step over every unit of a batch: score, z-normalise and max,
+ * select the top-B, gather K, V and positions into the destination cache.
+ * Units whose n_valid <= B are copied whole.  Small caches run one fused
+ * kernel per unit; large caches run the split kernels.  Arguments as in the
+ * calls above; kept_idx (nullable, [U][B]) receives the kept indices;
+ * n_kept ([U], required) receives min(B, n_valid[u]), the destination's
+ * n_valid for the next step.
+ */
+tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src,
+                     const int32_t* pos_src, tri_dtype dt, int64_t n_seq, int64_t n_layers,
+                     int64_t n_kvheads, int G, int64_t cap_src, const int32_t* n_valid,
+                     const int64_t* p_cur, const float* stats, int64_t B, void* k_dst,
+                     void* v_dst, int32_t* pos_dst, int64_t cap_dst, int32_t* kept_idx,
+                     int32_t* n_kept, void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Streaming helper: append generated tokens                               */
+/* ---------------------------------------------------------------------- */
+
+/*
+ * Append n_new rows per unit to a cache: rows n_valid[u] .. n_valid[u]+n_new-1
+ * of unit u receive k_new[u][i], v_new[u][i], pos_new[u][i]; n_valid[u] grows by
+ * n_new; p_cur[seq] is set to 1 + the largest appended position of the
+ * sequence's units.  Used by the windowed driver that prunes every 128
+ * generated tokens (hyper.ai summary, Method section).  A unit whose rows
+ * would exceed cap is left unchanged and sets TRI_FLAG_NVALID_RANGE.
+ *   k_new, v_new: [U][n_new][head_dim] (dt); pos_new: [U][n_new] int32.
+ *   n_valid: in/out [U]; p_cur: out [n_seq] (nullable).
+ */
+tri_status tri_append(void* k_cache, void* v_cache, int32_t* pos_cache, tri_dtype dt,
+                      int64_t n_seq, int64_t n_units, int64_t cap, int head_dim,
+                      int32_t* n_valid, int64_t* p_cur, const void* k_new, const void* v_new,
+                      const int32_t* pos_new, int64_t n_new, void* ws, size_t ws_bytes,
+                      void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Launch accounting (profiling)                                           */
+/* ---------------------------------------------------------------------- */
+
+/*
+ * Per-kernel timing for the calling host thread.  events (host array of
+ * cudaEvent_t handles passed as void*, caller-owned, must stay valid while
+ * set) receives one cudaEventRecord on the call's stream right after each
+ * kernel the next calls launch: event i after launch i of each call.  Pass
+ * (NULL, 0) to stop.  Works under stream capture (the records become graph
+ * nodes).  Returns TRI_ERR_INVALID_ARG for n_events < 0 or a NULL array with
+ * n_events > 0.
+ */
+tri_status tri_set_timing_events(void* const* events, int n_events);
+
+/* Number of kernels the most recent tri_* call on this host thread launched
+ * (memsets are not counted). */
+int tri_last_launch_count(void);
+
+/* ---------------------------------------------------------------------- */
+/* Device-side error flag                                                  */
+/* ---------------------------------------------------------------------- */
+
+/*
+ * Synchronise the stream and read the flag word of ws (written by the last
+ * call that used ws).  *flags_out (host, nullable) receives the TRI_FLAG_*
+ * bits.  Returns TRI_OK when no bit is set, TRI_ERR_DEVICE otherwise, or
+ * TRI_ERR_CUDA if the synchronisation fails.
+ */
+tri_status tri_check_device_error(const void* ws, void* stream, uint32_t* flags_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TRI_H_ */

@@ -1,0 +1,544 @@
+// api.cu -- the libtri C ABI (include/tri.h): host-side argument checks,
+// workspace layout, TMA descriptors and kernel dispatch.
+//
+// Nothing here computes any part of the method; every step runs in the
+// kernels of calibrate.cu, score.cu, select.cu, compact.cu and fused.cu.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstring>
+#include <mutex>
+
+#include "tri_internal.cuh"
+#include "tri_launch.h"
+
+using namespace tri;
+
+// Launch accounting for callers that time each kernel (tri_set_timing_events).
+namespace {
+thread_local cudaEvent_t* t_events = nullptr;
+thread_local int t_n_events = 0;
+thread_local int t_launches = 0;
+}  // namespace
+
+void tri::note_launch(cudaStream_t s) {
+    if (t_events && t_launches < t_n_events) {
+        // Under stream capture a plain record only marks a dependency; an
+        // external record becomes an event-record node that can be timed.
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        cudaStreamIsCapturing(s, &cs);
+        if (cs == cudaStreamCaptureStatusActive)
+            cudaEventRecordWithFlags(t_events[t_launches], s, cudaEventRecordExternal);
+        else
+            cudaEventRecord(t_events[t_launches], s);
+    }
+    ++t_launches;
+}
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+// Workspace carving: returns offsets of consecutive, 256-byte aligned regions.
+struct Carve {
+    size_t off = kWsHeader;
+    size_t take(size_t bytes) {
+        const size_t o = off;
+        off = align_up(off + bytes);
+        return o;
+    }
+};
+
+struct DeviceInfo {
+    int sm_count = 0;
+};
+
+DeviceInfo device_info() {
+    static std::mutex mu;
+    static DeviceInfo cache[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(mu);
+    DeviceInfo& d = cache[dev & 63];
+    if (!d.sm_count) cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
+    return d;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D view of a key cache [rows][128] for TMA: boxes of 128 bytes x box_rows
+// rows with the 128-byte swizzle.
+tri_status make_key_map(CUtensorMap* map, const void* k, tri_dtype dt, int64_t rows,
+                        int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return TRI_ERR_CUDA;
+    const int esz = dt == TRI_BF16 ? 2 : 4;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD * esz)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esz), static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(map,
+                          dt == TRI_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                         : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                          2, const_cast<void*>(k), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? TRI_OK : TRI_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3) == 0; }
+bool dtype_ok(tri_dtype dt) { return dt == TRI_BF16 || dt == TRI_F32; }
+
+tri_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TRI_OK : TRI_ERR_CUDA; }
+
+#define TRI_TRY(expr)                              \
+    do {                                           \
+        const tri_status _st = (expr);             \
+        if (_st != TRI_OK) return _st;             \
+    } while (0)
+
+#define TRI_CUDA(expr)                             \
+    do {                                           \
+        if ((expr) != cudaSuccess) return TRI_ERR_CUDA; \
+    } while (0)
+
+tri_status check_cfg(const tri_config* cfg, FoldOffsets* off) {
+    if (!cfg) return TRI_ERR_INVALID_ARG;
+    if (cfg->head_dim != kD) return TRI_ERR_UNSUPPORTED;
+    if (!(cfg->theta > 1.0) || cfg->n_offsets < 1 || cfg->n_offsets > TRI_MAX_OFFSETS)
+        return TRI_ERR_INVALID_ARG;
+    if (cfg->path < TRI_PATH_AUTO || cfg->path > TRI_PATH_SPLIT) return TRI_ERR_INVALID_ARG;
+    off->n = cfg->n_offsets;
+    for (int i = 0; i < cfg->n_offsets; ++i) {
+        if (cfg->offsets[i] < 0) return TRI_ERR_INVALID_ARG;
+        off->v[i] = cfg->offsets[i];
+    }
+    return TRI_OK;
+}
+
+// Shape limits shared by score / prune: grid dimensions and 32-bit TMA row
+// coordinates.
+tri_status check_units(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int64_t cap) {
+    if (n_seq < 1 || n_layers < 1 || n_kvheads < 1 || cap < 1) return TRI_ERR_INVALID_ARG;
+    if (G < 1 || G > kMaxG) return TRI_ERR_UNSUPPORTED;
+    const int64_t U = n_seq * n_layers * n_kvheads;
+    if (U > 65535 || U * cap >= (int64_t(1) << 31) || cap > (int64_t(1) << 30))
+        return TRI_ERR_UNSUPPORTED;
+    return TRI_OK;
+}
+
+// ---- score workspace ----
+struct ScoreWs {
+    size_t wts, raw, partial, counters, mom, total;
+    int64_t tpu;
+};
+
+ScoreWs score_ws(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int64_t cap,
+                 tri_dtype dt, bool own_raw) {
+    ScoreWs w;
+    const int64_t U = n_seq * n_layers * n_kvheads;
+    const int tile = score_tile_keys(dt);
+    w.tpu = (cap + tile - 1) / tile;
+    Carve c;
+    w.wts = c.take(static_cast<size_t>(U * G) * kWHead * 4);
+    w.raw = own_raw ? c.take(static_cast<size_t>(U * G * cap) * 4) : 0;
+    w.partial = c.take(static_cast<size_t>(U * w.tpu * G * 2) * 8);
+    w.counters = c.take(static_cast<size_t>(U) * 4);
+    w.mom = c.take(static_cast<size_t>(U * G) * 8);
+    w.total = c.off;
+    return w;
+}
+
+// ---- select workspace ----
+struct SelectWs {
+    size_t hists, counts, total;
+};
+
+SelectWs select_ws(size_t start, int64_t U, int64_t cap) {
+    SelectWs w;
+    Carve c;
+    c.off = start;
+    w.hists = c.take(static_cast<size_t>(3 * U) * kHistBins0 * 4);
+    const int64_t chunks = (cap + kZChunk - 1) / kZChunk;
+    w.counts = c.take(static_cast<size_t>(U * chunks) * 8);
+    w.total = c.off;
+    return w;
+}
+
+// ---- prune workspace ----
+struct PruneWs {
+    bool fused;
+    ScoreWs sc;
+    size_t fin, kept;
+    SelectWs sel;
+    size_t total;
+};
+
+bool use_fused(tri_dtype dt, int G, int64_t cap, int64_t B) {
+    const size_t smem = fused_smem_bytes(dt, G, cap);
+    const size_t tiles = dt == TRI_BF16 ? 3 * 32768 : 2 * 65536;
+    const int64_t m = B < cap ? B : cap;
+    return smem <= fused_smem_limit() && static_cast<size_t>(kHistBins0 * 4 + m * 4) <= tiles;
+}
+
+PruneWs prune_ws(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int64_t cap,
+                 int64_t B, tri_dtype dt, bool own_kept, int path) {
+    PruneWs w;
+    const int64_t U = n_seq * n_layers * n_kvheads;
+    w.fused = path == TRI_PATH_SPLIT ? false : use_fused(dt, G, cap, B);
+    if (w.fused) {
+        Carve c;
+        w.sc.wts = c.take(static_cast<size_t>(U * G) * kWHead * 4);
+        w.kept = own_kept ? c.take(static_cast<size_t>(U * B) * 4) : 0;
+        w.fin = 0;
+        w.total = c.off;
+        return w;
+    }
+    w.sc = score_ws(n_seq, n_layers, n_kvheads, G, cap, dt, true);
+    Carve c;
+    c.off = w.sc.total;
+    w.fin = c.take(static_cast<size_t>(U * cap) * 4);
+    w.kept = own_kept ? c.take(static_cast<size_t>(U * B) * 4) : 0;
+    w.sel = select_ws(c.off, U, cap);
+    w.total = w.sel.total;
+    return w;
+}
+
+// Every exported call that launches kernels starts a fresh launch count.
+struct LaunchScope {
+    LaunchScope() { t_launches = 0; }
+};
+
+char* ws_at(void* ws, size_t off) { return static_cast<char*>(ws) + off; }
+uint32_t* ws_flag(void* ws) { return reinterpret_cast<uint32_t*>(ws); }
+
+}  // namespace
+
+// ===========================================================================
+// Exported C ABI
+// ===========================================================================
+extern "C" {
+
+void tri_config_default(tri_config* cfg, int head_dim) {
+    if (!cfg) return;
+    std::memset(cfg, 0, sizeof(*cfg));
+    cfg->head_dim = head_dim;
+    cfg->theta = 10000.0;
+    cfg->n_offsets = 17;
+    for (int i = 0; i < 17; ++i) cfg->offsets[i] = int64_t(1) << i;
+}
+
+const char* tri_status_str(tri_status s) {
+    switch (s) {
+        case TRI_OK: return "ok";
+        case TRI_ERR_INVALID_ARG: return "invalid argument";
+        case TRI_ERR_UNSUPPORTED: return "unsupported shape or type";
+        case TRI_ERR_WORKSPACE: return "workspace missing or too small";
+        case TRI_ERR_CUDA: return "CUDA error";
+        case TRI_ERR_DEVICE: return "device-side flag set";
+    }
+    return "unknown status";
+}
+
+const char* tri_version(void) { return "libtri 0.1 sm_100a"; }
+
+size_t tri_calibrate_workspace_bytes(int64_t n_heads, int64_t n_tok, int head_dim) {
+    (void)head_dim;
+    if (n_heads < 1 || n_tok < 1) return kWsHeader;
+    return calibrate_ws_bytes(n_heads, n_tok);
+}
+
+tri_status tri_calibrate(const void* q_pre, tri_dtype dt, int64_t n_heads, int64_t n_tok,
+                         int head_dim, float* stats, void* ws, size_t ws_bytes, void* stream) {
+    LaunchScope scope_;
+    if (!q_pre || !stats || n_heads < 1 || n_tok < 1) return TRI_ERR_INVALID_ARG;
+    if (!dtype_ok(dt)) return TRI_ERR_UNSUPPORTED;
+    if (head_dim != kD) return TRI_ERR_UNSUPPORTED;
+    if (n_heads > 65535) return TRI_ERR_UNSUPPORTED;
+    if (!aligned16(q_pre) || !aligned4(stats)) return TRI_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < calibrate_ws_bytes(n_heads, n_tok) || !aligned16(ws))
+        return TRI_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    TRI_CUDA(cudaMemsetAsync(ws, 0, kWsHeader, s));
+    return cuda_status(launch_calibrate(q_pre, dt, n_heads, n_tok, stats, ws, s));
+}
+
+size_t tri_score_workspace_bytes(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G,
+                                 int64_t cap, int head_dim) {
+    (void)head_dim;
+    if (check_units(n_seq, n_layers, n_kvheads, G, cap) != TRI_OK) return kWsHeader;
+    // Large enough whether or not the caller supplies `raw` (bf16 tiles are
+    // the smaller unit, so the bf16 layout bounds both types).
+    const size_t a = score_ws(n_seq, n_layers, n_kvheads, G, cap, TRI_BF16, true).total;
+    const size_t b = score_ws(n_seq, n_layers, n_kvheads, G, cap, TRI_F32, true).total;
+    return a > b ? a : b;
+}
+
+tri_status tri_score(const tri_config* cfg, const void* k_post, tri_dtype dt, int64_t n_seq,
+                     int64_t n_layers, int64_t n_kvheads, int G, int64_t cap,
+                     const int32_t* n_valid, const int64_t* p_cur, const float* stats, float* raw,
+                     float* final_score, void* ws, size_t ws_bytes, void* stream) {
+    LaunchScope scope_;
+    FoldOffsets off;
+    TRI_TRY(check_cfg(cfg, &off));
+    if (!dtype_ok(dt)) return TRI_ERR_UNSUPPORTED;
+    TRI_TRY(check_units(n_seq, n_layers, n_kvheads, G, cap));
+    if (!k_post || !p_cur || !stats || !final_score) return TRI_ERR_INVALID_ARG;
+    if (!aligned16(k_post) || !aligned4(final_score) || (raw && !aligned4(raw)) ||
+        (n_valid && !aligned4(n_valid)) || !aligned4(stats))
+        return TRI_ERR_INVALID_ARG;
+    const ScoreWs w = score_ws(n_seq, n_layers, n_kvheads, G, cap, dt, raw == nullptr);
+    if (!ws || !aligned16(ws) || ws_bytes < w.total) return TRI_ERR_WORKSPACE;
+    const int64_t U = n_seq * n_layers * n_kvheads;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    CUtensorMap map;
+    TRI_TRY(make_key_map(&map, k_post, dt, U * cap, score_tile_keys(dt)));
+    TRI_CUDA(cudaMemsetAsync(ws, 0, kWsHeader, s));
+    TRI_CUDA(cudaMemsetAsync(ws_at(ws, w.counters), 0, static_cast<size_t>(U) * 4, s));
+    float* wts = reinterpret_cast<float*>(ws_at(ws, w.wts));
+    TRI_CUDA(launch_fold(stats, p_cur, n_seq, n_layers, n_kvheads * G, cfg->theta, off, wts, s));
+    ScoreArgs a;
+    a.n_units = U;
+    a.cap = cap;
+    a.tpu = w.tpu;
+    a.n_valid = n_valid;
+    a.wts = wts;
+    a.raw = raw ? raw : reinterpret_cast<float*>(ws_at(ws, w.raw));
+    a.partial = reinterpret_cast<double*>(ws_at(ws, w.partial));
+    a.counters = reinterpret_cast<uint32_t*>(ws_at(ws, w.counters));
+    a.mom = reinterpret_cast<float2*>(ws_at(ws, w.mom));
+    a.flag = ws_flag(ws);
+    TRI_CUDA(launch_score(dt, G, map, a, device_info().sm_count, s));
+    TRI_CUDA(launch_zmax(G, a.raw, U, cap, n_valid, a.mom, final_score, nullptr, a.flag, s));
+    return TRI_OK;
+}
+
+size_t tri_select_workspace_bytes(int64_t n_units, int64_t cap, int64_t B) {
+    (void)B;
+    if (n_units < 1 || cap < 1) return kWsHeader;
+    return select_ws(kWsHeader, n_units, cap).total;
+}
+
+tri_status tri_select_topB(const float* final_score, int64_t n_units, int64_t cap,
+                           const int32_t* n_valid, int64_t B, int32_t* kept_idx, int32_t* n_kept,
+                           void* ws, size_t ws_bytes, void* stream) {
+    LaunchScope scope_;
+    if (!final_score || !kept_idx || !n_kept || n_units < 1 || cap < 1 || B < 1)
+        return TRI_ERR_INVALID_ARG;
+    if (B > INT32_MAX || n_units > 65535 || cap > (int64_t(1) << 30)) return TRI_ERR_UNSUPPORTED;
+    if (!aligned4(final_score) || !aligned4(kept_idx) || !aligned4(n_kept) ||
+        (n_valid && !aligned4(n_valid)))
+        return TRI_ERR_INVALID_ARG;
+    const SelectWs w = select_ws(kWsHeader, n_units, cap);
+    if (!ws || !aligned16(ws) || ws_bytes < w.total) return TRI_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t* hists = reinterpret_cast<uint32_t*>(ws_at(ws, w.hists));
+    TRI_CUDA(cudaMemsetAsync(ws, 0, w.counts, s));  // header + histograms
+    for (int p = 0; p < 3; ++p)
+        TRI_CUDA(launch_radix_pass(final_score, n_units, cap, n_valid, B, hists, p, ws_flag(ws), s));
+    TRI_CUDA(launch_select_finish(final_score, n_units, cap, n_valid, B, hists,
+                                  reinterpret_cast<uint2*>(ws_at(ws, w.counts)), kept_idx, n_kept,
+                                  s));
+    return TRI_OK;
+}
+
+size_t tri_compact_workspace_bytes(void) { return kWsHeader; }
+
+tri_status tri_compact(const void* k_src, const void* v_src, const int32_t* pos_src, tri_dtype dt,
+                       int64_t n_units, int64_t cap_src, int head_dim, const int32_t* kept_idx,
+                       const int32_t* n_kept, int64_t B, void* k_dst, void* v_dst,
+                       int32_t* pos_dst, int64_t cap_dst, void* ws, size_t ws_bytes,
+                       void* stream) {
+    LaunchScope scope_;
+    if (!k_src || !k_dst || !kept_idx || !n_kept || n_units < 1 || cap_src < 1 || B < 1)
+        return TRI_ERR_INVALID_ARG;
+    if (!dtype_ok(dt) || head_dim != kD) return TRI_ERR_UNSUPPORTED;
+    if ((v_src == nullptr) != (v_dst == nullptr) || (pos_src == nullptr) != (pos_dst == nullptr))
+        return TRI_ERR_INVALID_ARG;
+    if (cap_dst < (B < cap_src ? B : cap_src)) return TRI_ERR_INVALID_ARG;
+    if (!aligned16(k_src) || !aligned16(k_dst) || (v_src && (!aligned16(v_src) || !aligned16(v_dst))))
+        return TRI_ERR_INVALID_ARG;
+    const size_t esz = dt == TRI_BF16 ? 2 : 4;
+    const char* ks = static_cast<const char*>(k_src);
+    const char* kd = static_cast<const char*>(k_dst);
+    const size_t sb = static_cast<size_t>(n_units * cap_src) * kD * esz;
+    const size_t db = static_cast<size_t>(n_units * cap_dst) * kD * esz;
+    if (ks < kd + db && kd < ks + sb) return TRI_ERR_INVALID_ARG;  // overlap
+    if (!ws || ws_bytes < kWsHeader || !aligned16(ws)) return TRI_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    TRI_CUDA(cudaMemsetAsync(ws, 0, kWsHeader, s));
+    return cuda_status(launch_gather(dt, k_src, v_src, pos_src, n_units, cap_src, kept_idx, n_kept,
+                                     B, k_dst, v_dst, pos_dst, cap_dst, ws_flag(ws),
+                                     device_info().sm_count * 8, s));
+}
+
+size_t tri_prune_workspace_bytes(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G,
+                                 int64_t cap, int64_t B, int head_dim) {
+    (void)head_dim;
+    if (check_units(n_seq, n_layers, n_kvheads, G, cap) != TRI_OK || B < 1) return kWsHeader;
+    size_t best = 0;
+    for (tri_dtype dt : {TRI_BF16, TRI_F32}) {
+        const size_t t = prune_ws(n_seq, n_layers, n_kvheads, G, cap, B, dt, true, TRI_PATH_SPLIT).total;
+        if (t > best) best = t;
+    }
+    return best;
+}
+
+tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src,
+                     const int32_t* pos_src, tri_dtype dt, int64_t n_seq, int64_t n_layers,
+                     int64_t n_kvheads, int G, int64_t cap_src, const int32_t* n_valid,
+                     const int64_t* p_cur, const float* stats, int64_t B, void* k_dst,
+                     void* v_dst, int32_t* pos_dst, int64_t cap_dst, int32_t* kept_idx,
+                     int32_t* n_kept, void* ws, size_t ws_bytes, void* stream) {
+    LaunchScope scope_;
+    FoldOffsets off;
+    TRI_TRY(check_cfg(cfg, &off));
+    if (!dtype_ok(dt)) return TRI_ERR_UNSUPPORTED;
+    TRI_TRY(check_units(n_seq, n_layers, n_kvheads, G, cap_src));
+    if (!k_src || !k_dst || !p_cur || !stats || !n_kept || B < 1) return TRI_ERR_INVALID_ARG;
+    if (B > INT32_MAX) return TRI_ERR_UNSUPPORTED;
+    if ((v_src == nullptr) != (v_dst == nullptr) || (pos_src == nullptr) != (pos_dst == nullptr))
+        return TRI_ERR_INVALID_ARG;
+    if (cap_dst < (B < cap_src ? B : cap_src)) return TRI_ERR_INVALID_ARG;
+    if (!aligned16(k_src) || !aligned16(k_dst) ||
+        (v_src && (!aligned16(v_src) || !aligned16(v_dst))) || !aligned4(stats) ||
+        !aligned4(n_kept) || (kept_idx && !aligned4(kept_idx)) || (n_valid && !aligned4(n_valid)))
+        return TRI_ERR_INVALID_ARG;
+    const int64_t U = n_seq * n_layers * n_kvheads;
+    const size_t esz = dt == TRI_BF16 ? 2 : 4;
+    {
+        const char* ks = static_cast<const char*>(k_src);
+        const char* kd = static_cast<const char*>(k_dst);
+        const size_t sb = static_cast<size_t>(U * cap_src) * kD * esz;
+        const size_t db = static_cast<size_t>(U * cap_dst) * kD * esz;
+        if (ks < kd + db && kd < ks + sb) return TRI_ERR_INVALID_ARG;
+    }
+    const PruneWs w =
+        prune_ws(n_seq, n_layers, n_kvheads, G, cap_src, B, dt, kept_idx == nullptr, cfg->path);
+    if (cfg->path == TRI_PATH_FUSED && !w.fused) return TRI_ERR_UNSUPPORTED;
+    if (!ws || !aligned16(ws) || ws_bytes < w.total) return TRI_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float* wts = reinterpret_cast<float*>(ws_at(ws, w.sc.wts));
+    int32_t* kept = kept_idx ? kept_idx : reinterpret_cast<int32_t*>(ws_at(ws, w.kept));
+    uint32_t* flag = ws_flag(ws);
+
+    if (w.fused) {
+        CUtensorMap map;
+        TRI_TRY(make_key_map(&map, k_src, dt, U * cap_src, 128));
+        TRI_CUDA(cudaMemsetAsync(ws, 0, kWsHeader, s));
+        TRI_CUDA(launch_fold(stats, p_cur, n_seq, n_layers, n_kvheads * G, cfg->theta, off, wts, s));
+        FusedArgs a;
+        a.cap = cap_src;
+        a.cap_dst = cap_dst;
+        a.B = B;
+        a.n_valid = n_valid;
+        a.wts = wts;
+        a.k_src = k_src;
+        a.v_src = v_src;
+        a.pos_src = pos_src;
+        a.k_dst = k_dst;
+        a.v_dst = v_dst;
+        a.pos_dst = pos_dst;
+        a.kept = kept_idx;
+        a.n_kept = n_kept;
+        a.flag = flag;
+        return cuda_status(launch_fused(dt, G, map, a, U, s));
+    }
+
+    CUtensorMap map;
+    TRI_TRY(make_key_map(&map, k_src, dt, U * cap_src, score_tile_keys(dt)));
+    // Zero the flag word, the moment counters and the radix histograms.
+    TRI_CUDA(cudaMemsetAsync(ws, 0, kWsHeader, s));
+    TRI_CUDA(cudaMemsetAsync(ws_at(ws, w.sc.counters), 0, static_cast<size_t>(U) * 4, s));
+    TRI_CUDA(cudaMemsetAsync(ws_at(ws, w.sel.hists), 0, w.sel.counts - w.sel.hists, s));
+    TRI_CUDA(launch_fold(stats, p_cur, n_seq, n_layers, n_kvheads * G, cfg->theta, off, wts, s));
+    ScoreArgs a;
+    a.n_units = U;
+    a.cap = cap_src;
+    a.tpu = w.sc.tpu;
+    a.n_valid = n_valid;
+    a.wts = wts;
+    a.raw = reinterpret_cast<float*>(ws_at(ws, w.sc.raw));
+    a.partial = reinterpret_cast<double*>(ws_at(ws, w.sc.partial));
+    a.counters = reinterpret_cast<uint32_t*>(ws_at(ws, w.sc.counters));
+    a.mom = reinterpret_cast<float2*>(ws_at(ws, w.sc.mom));
+    a.flag = flag;
+    const int n_sm = device_info().sm_count;
+    TRI_CUDA(launch_score(dt, G, map, a, n_sm, s));
+    float* fin = reinterpret_cast<float*>(ws_at(ws, w.fin));
+    uint32_t* hists = reinterpret_cast<uint32_t*>(ws_at(ws, w.sel.hists));
+    TRI_CUDA(launch_zmax(G, a.raw, U, cap_src, n_valid, a.mom, fin, hists, flag, s));
+    for (int p = 1; p < 3; ++p)
+        TRI_CUDA(launch_radix_pass(fin, U, cap_src, n_valid, B, hists, p, flag, s));
+    TRI_CUDA(launch_select_finish(fin, U, cap_src, n_valid, B, hists,
+                                  reinterpret_cast<uint2*>(ws_at(ws, w.sel.counts)), kept, n_kept,
+                                  s));
+    return cuda_status(launch_gather(dt, k_src, v_src, pos_src, U, cap_src, kept, n_kept, B, k_dst,
+                                     v_dst, pos_dst, cap_dst, flag, n_sm * 8, s));
+}
+
+tri_status tri_append(void* k_cache, void* v_cache, int32_t* pos_cache, tri_dtype dt,
+                      int64_t n_seq, int64_t n_units, int64_t cap, int head_dim,
+                      int32_t* n_valid, int64_t* p_cur, const void* k_new, const void* v_new,
+                      const int32_t* pos_new, int64_t n_new, void* ws, size_t ws_bytes,
+                      void* stream) {
+    LaunchScope scope_;
+    if (!k_cache || !k_new || !n_valid || n_seq < 1 || n_units < 1 || cap < 1 || n_new < 0)
+        return TRI_ERR_INVALID_ARG;
+    if (!dtype_ok(dt) || head_dim != kD) return TRI_ERR_UNSUPPORTED;
+    if (n_units % n_seq != 0 || n_units > 65535) return TRI_ERR_INVALID_ARG;
+    if ((v_cache == nullptr) != (v_new == nullptr) || (pos_cache == nullptr) != (pos_new == nullptr))
+        return TRI_ERR_INVALID_ARG;
+    if (p_cur && !pos_new) return TRI_ERR_INVALID_ARG;
+    if (!aligned16(k_cache) || !aligned16(k_new) ||
+        (v_cache && (!aligned16(v_cache) || !aligned16(v_new))))
+        return TRI_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < kWsHeader || !aligned16(ws)) return TRI_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    TRI_CUDA(cudaMemsetAsync(ws, 0, kWsHeader, s));
+    if (n_new == 0) return TRI_OK;
+    return cuda_status(launch_append(dt, k_cache, v_cache, pos_cache, n_seq, n_units, cap, n_valid,
+                                     p_cur, k_new, v_new, pos_new, n_new, ws_flag(ws), s));
+}
+
+tri_status tri_set_timing_events(void* const* events, int n_events) {
+    if (n_events < 0 || (n_events > 0 && !events)) return TRI_ERR_INVALID_ARG;
+    t_events = n_events ? reinterpret_cast<cudaEvent_t*>(const_cast<void**>(events)) : nullptr;
+    t_n_events = n_events;
+    return TRI_OK;
+}
+
+int tri_last_launch_count(void) { return t_launches; }
+
+tri_status tri_check_device_error(const void* ws, void* stream, uint32_t* flags_out) {
+    if (!ws) return TRI_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t f = 0;
+    if (cudaMemcpyAsync(&f, ws, sizeof(f), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return TRI_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return TRI_ERR_CUDA;
+    if (flags_out) *flags_out = f;
+    return f ? TRI_ERR_DEVICE : TRI_OK;
+}
+
+}  // extern "C"

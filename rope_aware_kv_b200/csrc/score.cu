@@ -1,0 +1,371 @@
+// score.cu -- fold, fused score and GQA z-max kernels.
+//
+// Score of key k for query head h (talk page: S_trig, S_norm and the
+// offset-averaged S~; hyper.ai summary, Method section):
+//   S~(k) = mean_{delta in D} sum_f |E q_f| |k_f| cos(w_f (p_cur+delta-p_k) + phi_f)
+//         + sum_f (1 - R_f) E|q_f| |k_f|.
+// With k_f = k'_f e^{-i w_f p_k} (the key de-rotated by its position) every
+// trigonometric term is Re(E[q_f] conj(k'_f) e^{i w_f (p_cur+delta)}), so the
+// key position cancels and the mean over D is Re(A_f conj(k'_f)) with
+//   A_f = E[q_f] e^{i w_f p_cur} C_f,   C_f = (1/|D|) sum_delta e^{i w_f delta}.
+// fold_kernel computes A_f (float64, rounded once to float32) and the norm
+// weights c_f = (1 - R_f) E|q_f| per query head; the score kernel then needs,
+// per key and head, one 128-wide dot product with (Re A_f, Im A_f) pairs and
+// one 64-wide dot product of c with the band norms |k'_f| = |k_f|.
+//
+// Data path: keys stream HBM -> shared memory by TMA (128-byte swizzle, one
+// box per 128-byte half row), a producer warp keeps STAGES tiles in flight,
+// four consumer warps compute.  Per-tile float64 moment partials are merged in
+// tile order by the last tile of each unit to finish (an atomic counter; no
+// waiting), so mu and sigma are bitwise reproducible.
+#include "tri_internal.cuh"
+#include "tri_launch.h"
+#include "score_core.cuh"
+
+namespace tri {
+
+// ---------------------------------------------------------------------------
+// Fold: per (seq, layer, query head) weights, chunk-major for the score loop.
+// Record layout per query head: 16 chunks x 12 floats; chunk c covers bands
+// 4c..4c+3: [ReA_4c, ImA_4c, ..., ReA_4c+3, ImA_4c+3, c_4c, ..., c_4c+3].
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(64)
+fold_kernel(const float* __restrict__ stats, const int64_t* __restrict__ p_cur, int64_t n_layers,
+            int64_t n_qheads, double theta, FoldOffsets off, float* __restrict__ wts) {
+    const int f = threadIdx.x;
+    const int64_t q = blockIdx.x;                    // (seq * L + layer) * Hq + qh
+    const int64_t qh = q % n_qheads;
+    const int64_t layer = (q / n_qheads) % n_layers;
+    const int64_t seq = q / (n_qheads * n_layers);
+    const float* st = stats + ((layer * n_qheads + qh) * kF + f) * 4;
+    const double w = pow(theta, -2.0 * static_cast<double>(f) / static_cast<double>(kD));
+    double cre = 0.0, cim = 0.0;
+    for (int i = 0; i < off.n; ++i) {
+        double s, c;
+        sincos(w * static_cast<double>(off.v[i]), &s, &c);
+        cre += c;
+        cim += s;
+    }
+    cre /= off.n;
+    cim /= off.n;
+    double ps, pc;
+    sincos(w * static_cast<double>(p_cur[seq]), &ps, &pc);
+    const double mre = st[0], mim = st[1];
+    // E[q_f] * e^{i w p_cur}
+    const double tre = mre * pc - mim * ps;
+    const double tim = mre * ps + mim * pc;
+    // ... * C_f
+    const double are = tre * cre - tim * cim;
+    const double aim = tre * cim + tim * cre;
+    const double cw = (1.0 - static_cast<double>(st[3])) * static_cast<double>(st[2]);
+    float* rec = wts + q * kWHead + (f >> 2) * kWChunk;
+    const int i = f & 3;
+    rec[2 * i] = static_cast<float>(are);
+    rec[2 * i + 1] = static_cast<float>(aim);
+    rec[8 + i] = static_cast<float>(cw);
+}
+
+// ---------------------------------------------------------------------------
+// Score kernel
+// ---------------------------------------------------------------------------
+template <typename T>
+struct ScoreShape {
+    static constexpr int kRowBytes = kD * static_cast<int>(sizeof(T));  // 256 / 512
+    static constexpr int kBoxes = kRowBytes / 128;                      // 2 / 4
+    static constexpr int kKPT = sizeof(T) == 2 ? 2 : 1;                 // keys per thread
+    static constexpr int kTile = 128 * kKPT;                            // keys per tile
+    static constexpr int kBoxBytes = kTile * 128;
+    static constexpr int kStageBytes = kTile * kRowBytes;               // 64 KB
+    static constexpr int kStages = 3;
+    static constexpr int kConsumers = 128;
+    static constexpr int kThreads = kConsumers + 32;
+};
+
+template <typename T, int G>
+struct ScoreSmem {
+    using S = ScoreShape<T>;
+    alignas(1024) uint8_t tiles[S::kStages][S::kStageBytes];
+    alignas(16) float w[G * kWHead];
+    double red[4][G][2];
+    uint64_t full[S::kStages];
+    uint64_t empty[S::kStages];
+    int last_flag;
+};
+
+template <int G>
+__device__ __forceinline__ void merge_unit_moments(const double* part, int tpu, int n,
+                                                   float2* mom_u) {
+    // Fixed tile order: bitwise reproducible.
+    for (int h = 0; h < G; ++h) {
+        double s1 = 0.0, s2 = 0.0;
+        for (int i = 0; i < tpu; ++i) {
+            s1 += part[(static_cast<int64_t>(i) * G + h) * 2];
+            s2 += part[(static_cast<int64_t>(i) * G + h) * 2 + 1];
+        }
+        float mu = 0.f, inv = 0.f;
+        if (n > 0) {
+            const double m = s1 / n;
+            double var = s2 / n - m * m;
+            if (var < 0.0) var = 0.0;
+            const double sd = sqrt(var);
+            mu = static_cast<float>(m);
+            inv = sd > 0.0 ? static_cast<float>(1.0 / sd) : 0.f;
+            if (!(sd == sd)) inv = __int_as_float(0x7fc00000);  // NaN propagates
+        }
+        mom_u[h] = make_float2(mu, inv);
+    }
+}
+
+template <typename T, int G>
+__global__ void __launch_bounds__(ScoreShape<T>::kThreads, 1)
+score_kernel(const __grid_constant__ CUtensorMap kmap, ScoreArgs a) {
+    using S = ScoreShape<T>;
+    extern __shared__ uint8_t smem_raw[];
+    ScoreSmem<T, G>& sm = *reinterpret_cast<ScoreSmem<T, G>*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x;
+    const int64_t total = a.n_units * a.tpu;
+    const int64_t t_begin = total * blockIdx.x / gridDim.x;
+    const int64_t t_end = total * (blockIdx.x + 1) / gridDim.x;
+
+    if (tid == S::kConsumers) {
+        for (int i = 0; i < S::kStages; ++i) {
+            mbar_init(&sm.full[i], 1);
+            mbar_init(&sm.empty[i], S::kConsumers);
+        }
+        fence_barrier_init();
+        prefetch_tensormap(&kmap);
+    }
+    __syncthreads();
+
+    if (tid >= S::kConsumers) {
+        // Producer warp: one lane issues the TMA loads.
+        if (tid == S::kConsumers) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued[S::kStages] = {};
+            bool ok = true;
+            for (int64_t t = t_begin; t < t_end && ok; ++t) {
+                const int64_t u = t / a.tpu;
+                const int i = static_cast<int>(t % a.tpu);
+                const int n = clamp_nvalid(a.n_valid, u, a.cap, nullptr);
+                if (i * S::kTile >= n) continue;
+                ok = mbar_wait(&sm.empty[stage], phase ^ 1, a.flag);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&sm.full[stage], S::kStageBytes);
+                const int32_t y = static_cast<int32_t>(u * a.cap + static_cast<int64_t>(i) * S::kTile);
+#pragma unroll
+                for (int b = 0; b < S::kBoxes; ++b)
+                    tma_load_2d(sm.tiles[stage] + b * S::kBoxBytes, &kmap, &sm.full[stage],
+                                b * (128 / static_cast<int>(sizeof(T))), y);
+                issued[stage]++;
+                if (++stage == S::kStages) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+            // Every load issued has landed before the CTA may exit.
+            for (int st = 0; st < S::kStages; ++st)
+                if (issued[st]) mbar_wait(&sm.full[st], (issued[st] - 1) & 1, a.flag);
+        }
+        return;
+    }
+
+    // Consumers.
+    int stage = 0;
+    uint32_t phase = 0;
+    int64_t cur_u = -1;
+    for (int64_t t = t_begin; t < t_end; ++t) {
+        const int64_t u = t / a.tpu;
+        const int i = static_cast<int>(t % a.tpu);
+        const int n = clamp_nvalid(a.n_valid, u, a.cap, tid == 0 ? a.flag : nullptr);
+        double m1[G], m2[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) m1[h] = m2[h] = 0.0;
+        if (i * S::kTile < n) {
+            if (u != cur_u) {
+                named_sync(1, S::kConsumers);
+                const float4* src = reinterpret_cast<const float4*>(a.wts + u * G * kWHead);
+                float4* dst = reinterpret_cast<float4*>(sm.w);
+                for (int e = tid; e < G * kWHead / 4; e += S::kConsumers) dst[e] = src[e];
+                named_sync(1, S::kConsumers);
+                cur_u = u;
+            }
+            if (!mbar_wait(&sm.full[stage], phase, a.flag)) break;
+            float s[S::kKPT][G];
+            score_rows<T, G, S::kKPT, S::kBoxBytes>(sm.tiles[stage], sm.w, tid, s);
+            mbar_arrive(&sm.empty[stage]);
+            if (++stage == S::kStages) {
+                stage = 0;
+                phase ^= 1;
+            }
+#pragma unroll
+            for (int k = 0; k < S::kKPT; ++k) {
+                const int j = i * S::kTile + tid + 128 * k;
+                if (j < n) {
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        a.raw[(u * G + h) * a.cap + j] = s[k][h];
+                        const double d = s[k][h];
+                        m1[h] += d;
+                        m2[h] = fma(d, d, m2[h]);
+                    }
+                }
+            }
+        }
+        // Tile moments: warp shuffle, then the 4 warps in order.
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                m1[h] += __shfl_xor_sync(0xffffffffu, m1[h], o);
+                m2[h] += __shfl_xor_sync(0xffffffffu, m2[h], o);
+            }
+        }
+        const int warp = tid >> 5, lane = tid & 31;
+        if (lane == 0) {
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                sm.red[warp][h][0] = m1[h];
+                sm.red[warp][h][1] = m2[h];
+            }
+        }
+        named_sync(1, S::kConsumers);
+        if (tid == 0) {
+            double* part = a.partial + (u * a.tpu + i) * G * 2;
+            for (int h = 0; h < G; ++h) {
+                part[2 * h] = ((sm.red[0][h][0] + sm.red[1][h][0]) + sm.red[2][h][0]) + sm.red[3][h][0];
+                part[2 * h + 1] =
+                    ((sm.red[0][h][1] + sm.red[1][h][1]) + sm.red[2][h][1]) + sm.red[3][h][1];
+            }
+            __threadfence();
+            const uint32_t done = atomicAdd(&a.counters[u], 1u);
+            sm.last_flag = (done == static_cast<uint32_t>(a.tpu) - 1u);
+            if (sm.last_flag) {
+                __threadfence();
+                merge_unit_moments<G>(a.partial + u * a.tpu * G * 2, a.tpu, n, a.mom + u * G);
+                a.counters[u] = 0u;
+            }
+        }
+        named_sync(1, S::kConsumers);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// z-score per head, max over the group, optional first radix histogram.
+// (hyper.ai summary, Method section: GQA normalise-then-aggregate.)
+// ---------------------------------------------------------------------------
+template <int G>
+__global__ void __launch_bounds__(256)
+zmax_kernel(const float* __restrict__ raw, int64_t cap, const int32_t* __restrict__ n_valid,
+            const float2* __restrict__ mom, float* __restrict__ fin, uint32_t* __restrict__ hist0,
+            uint32_t* flag) {
+    __shared__ uint32_t hist[kHistBins0];
+    const int64_t u = blockIdx.y;
+    const int n = clamp_nvalid(n_valid, u, cap, nullptr);
+    const int j0 = blockIdx.x * kZChunk;
+    if (hist0) {
+        for (int b = threadIdx.x; b < kHistBins0; b += blockDim.x) hist[b] = 0;
+        __syncthreads();
+    }
+    float mu[G], inv[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        const float2 m = mom[u * G + h];
+        mu[h] = m.x;
+        inv[h] = m.y;
+    }
+    bool nonfinite = false;
+    const int j1 = min(j0 + kZChunk, n);
+    for (int j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
+        float best = 0.f;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float s = raw[(u * G + h) * cap + j];
+            const float z = (s - mu[h]) * inv[h];
+            best = (h == 0) ? z : fmaxf(best, z);
+        }
+        fin[u * cap + j] = best;
+        if (best != best) nonfinite = true;
+        if (hist0) atomicAdd(&hist[ordered_key(best) >> kShift0], 1u);
+    }
+    if (nonfinite) raise_flag(flag, TRI_FLAG_NONFINITE);
+    if (hist0) {
+        __syncthreads();
+        uint32_t* g = hist0 + u * kHistBins0;
+        for (int b = threadIdx.x; b < kHistBins0; b += blockDim.x)
+            if (hist[b]) atomicAdd(&g[b], hist[b]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host launchers
+// ---------------------------------------------------------------------------
+template <typename T, int G>
+static cudaError_t launch_score_t(const CUtensorMap& map, const ScoreArgs& a, int n_sm,
+                                  cudaStream_t s) {
+    const size_t smem = sizeof(ScoreSmem<T, G>) + 1024;
+    auto kern = score_kernel<T, G>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    const int64_t total = a.n_units * a.tpu;
+    const int grid = static_cast<int>(total < n_sm ? total : n_sm);
+    kern<<<grid, ScoreShape<T>::kThreads, smem, s>>>(map, a);
+    note_launch(s);
+    return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_score_g(int G, const CUtensorMap& map, const ScoreArgs& a, int n_sm,
+                                  cudaStream_t s) {
+    switch (G) {
+        case 1: return launch_score_t<T, 1>(map, a, n_sm, s);
+        case 2: return launch_score_t<T, 2>(map, a, n_sm, s);
+        case 3: return launch_score_t<T, 3>(map, a, n_sm, s);
+        case 4: return launch_score_t<T, 4>(map, a, n_sm, s);
+        case 5: return launch_score_t<T, 5>(map, a, n_sm, s);
+        case 6: return launch_score_t<T, 6>(map, a, n_sm, s);
+        case 7: return launch_score_t<T, 7>(map, a, n_sm, s);
+        case 8: return launch_score_t<T, 8>(map, a, n_sm, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+int score_tile_keys(tri_dtype dt) {
+    return dt == TRI_BF16 ? ScoreShape<__nv_bfloat16>::kTile : ScoreShape<float>::kTile;
+}
+
+cudaError_t launch_fold(const float* stats, const int64_t* p_cur, int64_t n_seq, int64_t n_layers,
+                        int64_t n_qheads, double theta, const FoldOffsets& off, float* wts,
+                        cudaStream_t s) {
+    const int64_t blocks = n_seq * n_layers * n_qheads;
+    fold_kernel<<<static_cast<unsigned>(blocks), 64, 0, s>>>(stats, p_cur, n_layers, n_qheads,
+                                                             theta, off, wts);
+    note_launch(s);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_score(tri_dtype dt, int G, const CUtensorMap& map, const ScoreArgs& a,
+                         int n_sm, cudaStream_t s) {
+    if (dt == TRI_BF16) return launch_score_g<__nv_bfloat16>(G, map, a, n_sm, s);
+    return launch_score_g<float>(G, map, a, n_sm, s);
+}
+
+cudaError_t launch_zmax(int G, const float* raw, int64_t n_units, int64_t cap,
+                        const int32_t* n_valid, const float2* mom, float* fin, uint32_t* hist0,
+                        uint32_t* flag, cudaStream_t s) {
+    dim3 grid(static_cast<unsigned>((cap + kZChunk - 1) / kZChunk), static_cast<unsigned>(n_units));
+    switch (G) {
+#define TRI_ZCASE(g) \
+    case g: zmax_kernel<g><<<grid, 256, 0, s>>>(raw, cap, n_valid, mom, fin, hist0, flag); break;
+        TRI_ZCASE(1) TRI_ZCASE(2) TRI_ZCASE(3) TRI_ZCASE(4)
+        TRI_ZCASE(5) TRI_ZCASE(6) TRI_ZCASE(7) TRI_ZCASE(8)
+#undef TRI_ZCASE
+        default: return cudaErrorInvalidValue;
+    }
+    note_launch(s);
+    return cudaGetLastError();
+}
+
+}  // namespace tri

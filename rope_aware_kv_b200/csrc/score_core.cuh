@@ -1,0 +1,105 @@
+// score_core.cuh -- per-key score arithmetic on a shared-memory key tile.
+//
+// For key k' (post-RoPE) and query head h the folded score is
+//   s_h = sum_f (ReA_hf * x_f + ImA_hf * y_f) + sum_f c_hf * |k'_f|
+// with k'_f = x_f + i y_f the interleaved pair (x_2f, x_2f+1), A_hf the
+// offset-averaged rotated query centre and c_hf = (1 - R_hf) E|q_hf| (see
+// score.cu).  Products are formed with packed float32x2 FMAs: the (x, y) pair
+// of a band against (ReA, ImA), and two band norms against two c weights.
+#pragma once
+
+#include "tri_internal.cuh"
+
+namespace tri {
+
+// Score KPT keys of a tile held in swizzled shared memory.  Row r of box b
+// lives at b * kBoxBytes + r * 128 and its 16-byte chunk j at position
+// (j ^ (r & 7)) (TMA 128-byte swizzle), so 8 consecutive threads reading the
+// same logical chunk of 8 consecutive rows hit 8 different bank groups.
+template <typename T, int G, int KPT, int kBoxBytes>
+__device__ __forceinline__ void score_rows(const uint8_t* tile, const float* w, int tid,
+                                           float (&s)[KPT][G]) {
+    float2 acc[KPT][G];
+#pragma unroll
+    for (int k = 0; k < KPT; ++k)
+#pragma unroll
+        for (int h = 0; h < G; ++h) acc[k][h] = make_float2(0.f, 0.f);
+
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) {
+            float2 xy[KPT][4];
+            float2 nn[KPT][2];
+#pragma unroll
+            for (int k = 0; k < KPT; ++k) {
+                const int r = tid + 128 * k;
+                const uint4 v = *reinterpret_cast<const uint4*>(
+                    tile + (c >> 3) * kBoxBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+                const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+                float n[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float x = bf16_lo(wd[i]), y = bf16_hi(wd[i]);
+                    xy[k][i] = make_float2(x, y);
+                    n[i] = sqrt_approx(fmaf(x, x, y * y));
+                }
+                nn[k][0] = make_float2(n[0], n[1]);
+                nn[k][1] = make_float2(n[2], n[3]);
+            }
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float4* rec = reinterpret_cast<const float4*>(w + h * kWHead + c * kWChunk);
+                const float4 a = rec[0], b = rec[1], cc = rec[2];
+#pragma unroll
+                for (int k = 0; k < KPT; ++k) {
+                    float2 t = acc[k][h];
+                    t = __ffma2_rn(xy[k][0], make_float2(a.x, a.y), t);
+                    t = __ffma2_rn(xy[k][1], make_float2(a.z, a.w), t);
+                    t = __ffma2_rn(xy[k][2], make_float2(b.x, b.y), t);
+                    t = __ffma2_rn(xy[k][3], make_float2(b.z, b.w), t);
+                    t = __ffma2_rn(nn[k][0], make_float2(cc.x, cc.y), t);
+                    t = __ffma2_rn(nn[k][1], make_float2(cc.z, cc.w), t);
+                    acc[k][h] = t;
+                }
+            }
+        }
+    } else {
+        // float32 rows: 32 chunks of 4 floats (2 bands each).
+#pragma unroll 4
+        for (int c = 0; c < 2 * kChunks; ++c) {
+            float2 xy[KPT][2];
+            float2 nn[KPT];
+#pragma unroll
+            for (int k = 0; k < KPT; ++k) {
+                const int r = tid + 128 * k;
+                const float4 v = *reinterpret_cast<const float4*>(
+                    tile + (c >> 3) * kBoxBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+                xy[k][0] = make_float2(v.x, v.y);
+                xy[k][1] = make_float2(v.z, v.w);
+                nn[k] = make_float2(sqrt_approx(fmaf(v.x, v.x, v.y * v.y)),
+                                    sqrt_approx(fmaf(v.z, v.z, v.w * v.w)));
+            }
+            const int half = c & 1;
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float* rec = w + h * kWHead + (c >> 1) * kWChunk;
+                const float4 a = *reinterpret_cast<const float4*>(rec + 4 * half);
+                const float2 cc = *reinterpret_cast<const float2*>(rec + 8 + 2 * half);
+#pragma unroll
+                for (int k = 0; k < KPT; ++k) {
+                    float2 t = acc[k][h];
+                    t = __ffma2_rn(xy[k][0], make_float2(a.x, a.y), t);
+                    t = __ffma2_rn(xy[k][1], make_float2(a.z, a.w), t);
+                    t = __ffma2_rn(nn[k], cc, t);
+                    acc[k][h] = t;
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < KPT; ++k)
+#pragma unroll
+        for (int h = 0; h < G; ++h) s[k][h] = acc[k][h].x + acc[k][h].y;
+}
+
+}  // namespace tri

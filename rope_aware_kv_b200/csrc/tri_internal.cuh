@@ -1,0 +1,149 @@
+// tri_internal.cuh -- device helpers shared by the libtri kernels (sm_100a).
+//
+// Inline PTX wrappers for mbarriers and TMA bulk-tensor loads, the
+// order-preserving float -> uint32 map used by the radix select, the device
+// flag word, and the constants of the supported shape (head_dim 128).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/tri.h"
+
+namespace tri {
+
+constexpr int kD = 128;          // head_dim
+constexpr int kF = kD / 2;       // RoPE bands
+constexpr int kChunks = 16;      // 16-byte chunks of a bf16 row (4 bands each)
+constexpr int kWChunk = 12;      // floats per (head, chunk) weight record: 8 w + 4 c
+constexpr int kWHead = kChunks * kWChunk;  // 192 floats per query head
+constexpr int kMaxG = TRI_MAX_GROUP;
+
+// Flag word at the start of every workspace.
+struct WsHeader {
+    uint32_t flags;
+    uint32_t pad[63];
+};
+constexpr size_t kWsHeader = sizeof(WsHeader);  // 256 bytes
+
+__device__ __forceinline__ void raise_flag(uint32_t* flag, uint32_t bits) {
+    if (flag) atomicOr(flag, bits);
+}
+
+// Order-preserving 32-bit key of a float: a > b  <=>  key(a) > key(b) for
+// numbers; -0.0 and +0.0 share a key; NaN maps to 0, below every number.
+__device__ __forceinline__ uint32_t ordered_key(float x) {
+    if (x != x) return 0u;
+    uint32_t u = __float_as_uint(x);
+    if (u == 0x80000000u) u = 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for the phase with the given parity to complete, giving up after
+// kWaitLimitNs nanoseconds (a TMA tile lands in microseconds; the limit only
+// exists so that a fault elsewhere can never hang the GPU).  Returns false on
+// timeout and raises TRI_FLAG_TIMEOUT.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            raise_flag(flag, TRI_FLAG_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// TMA (bulk tensor copies, no multicast)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t x, int32_t y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cta.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// Named barrier among `count` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Approximate IEEE sqrt (max relative error ~2^-23, PTX sqrt.approx).
+__device__ __forceinline__ float sqrt_approx(float x) {
+    float r;
+    asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// bf16 pair in one 32-bit word: low half is the even element.
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ int clamp_nvalid(const int32_t* n_valid, int64_t u, int64_t cap,
+                                            uint32_t* flag) {
+    if (!n_valid) return static_cast<int>(cap);
+    int n = n_valid[u];
+    if (n < 0 || n > cap) {
+        raise_flag(flag, TRI_FLAG_NVALID_RANGE);
+        n = n < 0 ? 0 : static_cast<int>(cap);
+    }
+    return n;
+}
+
+}  // namespace tri

@@ -1,0 +1,97 @@
+// tri_launch.h -- host-side launch interfaces between the libtri translation
+// units (not part of the public C ABI, which is include/tri.h).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/tri.h"
+
+namespace tri {
+
+constexpr int kZChunk = 2048;      // keys per CTA in the z-max / radix / compaction kernels
+constexpr int kHistBins0 = 2048;   // bins of the first (and largest) radix digit
+constexpr int kShift0 = 21;        // the first digit is key bits 31..21
+
+struct FoldOffsets {
+    int n;
+    int64_t v[TRI_MAX_OFFSETS];
+};
+
+struct ScoreArgs {
+    int64_t n_units;
+    int64_t cap;
+    int64_t tpu;                 // tiles per unit
+    const int32_t* n_valid;
+    const float* wts;            // fold output, [U*G][192]
+    float* raw;                  // [U][G][cap]
+    double* partial;             // [U][tpu][G][2]
+    uint32_t* counters;          // [U], zero on entry
+    float2* mom;                 // [U][G] (mu, 1/sigma)
+    uint32_t* flag;
+};
+
+struct FusedArgs {
+    int64_t cap;
+    int64_t cap_dst;
+    int64_t B;
+    const int32_t* n_valid;
+    const float* wts;            // [U*G][192]
+    const void* k_src;
+    const void* v_src;
+    const int32_t* pos_src;
+    void* k_dst;
+    void* v_dst;
+    int32_t* pos_dst;
+    int32_t* kept;               // [U][B] or null
+    int32_t* n_kept;             // [U]
+    uint32_t* flag;
+};
+
+// api.cu: call after every kernel launch (counts launches and records the
+// caller's timing event for that launch, if any).
+void note_launch(cudaStream_t s);
+
+// calibrate.cu
+size_t calibrate_ws_bytes(int64_t n_heads, int64_t n_tok);
+cudaError_t launch_calibrate(const void* q, tri_dtype dt, int64_t n_heads, int64_t n_tok,
+                             float* stats, void* ws, cudaStream_t s);
+
+// score.cu
+int score_tile_keys(tri_dtype dt);
+cudaError_t launch_fold(const float* stats, const int64_t* p_cur, int64_t n_seq, int64_t n_layers,
+                        int64_t n_qheads, double theta, const FoldOffsets& off, float* wts,
+                        cudaStream_t s);
+cudaError_t launch_score(tri_dtype dt, int G, const CUtensorMap& map, const ScoreArgs& a,
+                         int n_sm, cudaStream_t s);
+cudaError_t launch_zmax(int G, const float* raw, int64_t n_units, int64_t cap,
+                        const int32_t* n_valid, const float2* mom, float* fin, uint32_t* hist0,
+                        uint32_t* flag, cudaStream_t s);
+
+// select.cu
+cudaError_t launch_radix_pass(const float* fin, int64_t n_units, int64_t cap,
+                              const int32_t* n_valid, int64_t B, uint32_t* hists, int pass,
+                              uint32_t* flag, cudaStream_t s);
+cudaError_t launch_select_finish(const float* fin, int64_t n_units, int64_t cap,
+                                 const int32_t* n_valid, int64_t B, const uint32_t* hists,
+                                 uint2* counts, int32_t* kept, int32_t* n_kept, cudaStream_t s);
+
+// compact.cu
+cudaError_t launch_gather(tri_dtype dt, const void* k_src, const void* v_src,
+                          const int32_t* pos_src, int64_t n_units, int64_t cap_src,
+                          const int32_t* kept, const int32_t* n_kept, int64_t B, void* k_dst,
+                          void* v_dst, int32_t* pos_dst, int64_t cap_dst, uint32_t* flag,
+                          int n_blocks, cudaStream_t s);
+cudaError_t launch_append(tri_dtype dt, void* k_cache, void* v_cache, int32_t* pos_cache,
+                          int64_t n_seq, int64_t n_units, int64_t cap, int32_t* n_valid,
+                          int64_t* p_cur, const void* k_new, const void* v_new,
+                          const int32_t* pos_new, int64_t n_new, uint32_t* flag, cudaStream_t s);
+
+// fused.cu
+size_t fused_smem_bytes(tri_dtype dt, int G, int64_t cap);
+size_t fused_smem_limit();
+cudaError_t launch_fused(tri_dtype dt, int G, const CUtensorMap& map, const FusedArgs& a,
+                         int64_t n_units, cudaStream_t s);
+
+}  // namespace tri

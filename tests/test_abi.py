@@ -1,0 +1,105 @@
+"""The C-ABI library builds, loads and exports every symbol include/tri.h
+declares; host-side argument checks answer without touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import rope_aware_kv_b200 as tri
+from rope_aware_kv_b200 import build as tri_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tri.h")
+GOLDEN = os.path.join(ROOT, "tests", "golden", "page_constants.txt")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    tri_build.build()
+    return tri.load()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(tri_[a-zA-Z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("tri_calibrate", "tri_score", "tri_select_topB", "tri_compact", "tri_prune"):
+        assert n in names
+    assert set(names) == set(tri.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_library_is_sm100a_only(lib):
+    assert b"sm_100a" in lib.tri_version()
+
+
+def test_default_config_matches_the_pages(lib):
+    vals = {}
+    for line in open(GOLDEN):
+        line = line.split("#", 1)[0].strip()
+        if line:
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip()
+    cfg = tri.config()
+    assert cfg.theta == float(vals["theta"])
+    assert [cfg.offsets[i] for i in range(cfg.n_offsets)] == [int(x) for x in vals["offsets"].split()]
+    assert cfg.head_dim == 128 and cfg.path == tri.PATH_AUTO
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert lib.tri_status_str(code).decode() == tri.STATUS[code]
+
+
+def test_workspace_queries(lib):
+    small = lib.tri_prune_workspace_bytes(1, 1, 4, 7, 4096, 512, 128)
+    big = lib.tri_prune_workspace_bytes(1, 1, 4, 7, 32768, 2048, 128)
+    assert 256 < small < big
+    assert lib.tri_score_workspace_bytes(1, 1, 4, 7, 32768, 128) >= 4 * 7 * 32768 * 4
+    assert lib.tri_select_workspace_bytes(4, 32768, 2048) >= 3 * 4 * 2048 * 4
+    assert lib.tri_compact_workspace_bytes() == 256
+    assert lib.tri_calibrate_workspace_bytes(28, 10240, 128) > 256
+
+
+def _prune_status(lib, cfg, **over):
+    args = dict(k_src=16, v_src=16, pos_src=16, dt=tri.TRI_BF16, n_seq=1, n_layers=1, n_kvheads=4,
+                G=7, cap=4096, n_valid=None, p_cur=16, stats=16, B=512, k_dst=1 << 40,
+                v_dst=1 << 41, pos_dst=16, cap_dst=512, kept=None, n_kept=16, ws=None, ws_bytes=0)
+    args.update(over)
+    P = lambda v: None if v is None else ctypes.c_void_p(v)
+    return lib.tri_prune(ctypes.byref(cfg) if cfg is not None else None, P(args["k_src"]),
+                         P(args["v_src"]), P(args["pos_src"]), args["dt"], args["n_seq"],
+                         args["n_layers"], args["n_kvheads"], args["G"], args["cap"],
+                         P(args["n_valid"]), P(args["p_cur"]), P(args["stats"]), args["B"],
+                         P(args["k_dst"]), P(args["v_dst"]), P(args["pos_dst"]), args["cap_dst"],
+                         P(args["kept"]), P(args["n_kept"]), P(args["ws"]), args["ws_bytes"], None)
+
+
+def test_host_validation_without_gpu(lib):
+    """Bad arguments are refused on the host before anything is launched."""
+    cfg = tri.config()
+    assert _prune_status(lib, None) == 1                      # no config
+    assert _prune_status(lib, cfg, G=9) == 2                  # group too large
+    assert _prune_status(lib, cfg, G=0) == 2
+    assert _prune_status(lib, cfg, dt=7) == 2                 # unknown dtype
+    assert _prune_status(lib, cfg, B=0) == 1                  # empty budget
+    assert _prune_status(lib, cfg, k_src=18) == 1             # misaligned keys
+    assert _prune_status(lib, cfg, v_dst=None) == 1           # v_src without v_dst
+    assert _prune_status(lib, cfg, cap_dst=100) == 1          # destination too small
+    assert _prune_status(lib, cfg, k_dst=16 + 4096) == 1      # destination overlaps source
+    bad = tri.config(head_dim=64)
+    assert _prune_status(lib, bad) == 2
+    cfg2 = tri.config()
+    cfg2.n_offsets = 0
+    assert _prune_status(lib, cfg2) == 1
+    cfg3 = tri.config(path=7)
+    assert _prune_status(lib, cfg3) == 1

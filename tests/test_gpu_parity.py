@@ -1,0 +1,345 @@
+"""GPU parity: every libtri entry point against the float64 oracle on the
+same seeded inputs.  Calls go through the C ABI (ctypes binding).
+
+Small cases span several key tiles and a ragged tail; the workload configs
+run at their full sizes in the launch configuration the benchmark times, with
+the oracle checking every unit where it finishes in seconds and a fixed
+sample of units otherwise.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import rope_aware_kv_b200 as tri
+import synth
+from rope_aware_kv_b200 import build as tri_build
+from tests import gpu_helpers as H
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    tri_build.build()
+    tri.load()
+    oracle.build()
+    yield
+    torch.cuda.empty_cache()
+
+
+def _spec(dtype="bf16", G=3, n_seq=2, n_layers=2, n_kvheads=2, cap=700, B=300, n_cal=3000,
+          positions="dense", p_cur=None, R_range=(0.6, 1.0), stream=11, **kw):
+    return synth.Spec("t", n_seq, n_layers, n_kvheads, G, cap, cap, B, dtype, n_cal,
+                      p_cur if p_cur is not None else cap, positions=positions, R_range=R_range,
+                      stream=stream, **kw)
+
+
+def _ragged_nvalid(spec, B):
+    U = spec.n_units
+    choices = [spec.cap, spec.cap - 1, 0, 1, B, B + 1, 255, 256, 257, 513, spec.cap // 2]
+    nv = np.array([choices[u % len(choices)] for u in range(U)], np.int32)
+    return np.clip(nv, 0, spec.cap)
+
+
+# ---------------------------------------------------------------------------
+# calibration
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_calibrate_parity(dtype):
+    spec = _spec(dtype=dtype, G=3, n_layers=2, n_kvheads=1, n_cal=3000)
+    wl = synth.make_workload(spec, "cuda")
+    gst, ost = H.stats_for(spec, wl)
+    g = gst.cpu().numpy().astype(np.float64)
+    scale = ost[..., 2:3]
+    assert np.max(np.abs(g[..., :3] - ost[..., :3]) / scale) < 1e-6
+    assert np.max(np.abs(g[..., 3] - ost[..., 3])) < 1e-6
+
+
+# ---------------------------------------------------------------------------
+# score
+# ---------------------------------------------------------------------------
+def _score_case(spec, n_valid=None):
+    wl = synth.make_workload(spec, "cuda")
+    gst, ost = H.stats_for(spec, wl)
+    nv = torch.as_tensor(n_valid if n_valid is not None else wl.n_valid.cpu().numpy(),
+                         dtype=torch.int32, device="cuda")
+    raw = torch.full((spec.n_units, spec.G, spec.cap), float("nan"), device="cuda")
+    cfg = tri.config()
+    _, fin = tri.tri_score(cfg, wl.k, spec.n_seq, spec.n_layers, spec.n_kvheads, spec.G, wl.p_cur,
+                           gst, n_valid=nv, raw=raw)
+    torch.cuda.synchronize()
+    return wl, ost, nv.cpu().numpy(), raw.cpu().numpy(), fin.cpu().numpy()
+
+
+@pytest.mark.parametrize("dtype,G", [("bf16", 1), ("bf16", 3), ("bf16", 7), ("bf16", 8),
+                                     ("f32", 1), ("f32", 4)])
+def test_score_parity_ragged(dtype, G):
+    spec = _spec(dtype=dtype, G=G, cap=700)
+    nv = _ragged_nvalid(spec, 300)
+    wl, ost, nv, raw, fin = _score_case(spec, nv)
+    o = oracle.prune(synth.host_elems(wl.k), None, wl.pos.cpu().numpy(), spec.n_seq,
+                     spec.n_layers, spec.n_kvheads, G, ost, wl.p_cur.cpu().numpy(), 300,
+                     n_valid=nv, want_gather=False)
+    for u in range(spec.n_units):
+        n = int(nv[u])
+        assert H.check_raw(raw[u], o["raw"][u], n) <= H.RAW_RTOL
+        assert H.check_final(fin[u], o["final"][u], n) <= H.Z_RTOL
+
+
+@pytest.mark.parametrize("name", ["c1", "c2"])
+def test_score_parity_config(name):
+    spec = synth.SPECS[name]
+    wl, ost, nv, raw, fin = _score_case(spec)
+    o = oracle.prune(synth.host_elems(wl.k), None, wl.pos.cpu().numpy(), spec.n_seq,
+                     spec.n_layers, spec.n_kvheads, spec.G, ost, wl.p_cur.cpu().numpy(), spec.B,
+                     n_valid=nv, want_gather=False)
+    for u in range(spec.n_units):
+        n = int(nv[u])
+        assert H.check_raw(raw[u], o["raw"][u], n) <= H.RAW_RTOL
+        assert H.check_final(fin[u], o["final"][u], n) <= H.Z_RTOL
+
+
+# ---------------------------------------------------------------------------
+# select
+# ---------------------------------------------------------------------------
+def _select_inputs(U, cap, seed):
+    rng = np.random.default_rng(seed)
+    x = rng.normal(size=(U, cap)).astype(np.float32)
+    # Heavy ties and special values in some units.
+    x[1] = np.round(x[1] * 2) / 2
+    x[2, ::7] = np.nan
+    x[2, 1::7] = -0.0
+    x[2, 2::7] = 0.0
+    x[3] = 1.5
+    x[4, : cap // 2] = -np.inf
+    return x
+
+
+@pytest.mark.parametrize("B", [1, 7, 100, 2048, 4999, 5000, 6000])
+def test_select_parity(B):
+    U, cap = 6, 5000
+    x = _select_inputs(U, cap, B)
+    nv = np.array([cap, cap, cap, cap, cap, 3001], np.int32)
+    fin = torch.as_tensor(x, device="cuda")
+    kept, nk = tri.tri_select_topB(fin, B, n_valid=torch.as_tensor(nv, device="cuda"))
+    kept, nk = kept.cpu().numpy(), nk.cpu().numpy()
+    for u in range(U):
+        n = int(nv[u])
+        ok, _ = oracle.select(x[u, :n].astype(np.float64), B)
+        assert nk[u] == len(ok)
+        np.testing.assert_array_equal(kept[u, :len(ok)], ok)
+        assert np.all(kept[u, len(ok):] == -1)
+
+
+def test_select_large_units_exact():
+    """Several CTAs per unit (the split path's chunking) with quantised ties."""
+    U, cap, B = 3, 131072 + 77, 4096
+    rng = np.random.default_rng(5)
+    x = (np.round(rng.normal(size=(U, cap)) * 64) / 64).astype(np.float32)
+    fin = torch.as_tensor(x, device="cuda")
+    kept, nk = tri.tri_select_topB(fin, B)
+    kept = kept.cpu().numpy()
+    for u in range(U):
+        ok, _ = oracle.select(x[u].astype(np.float64), B)
+        np.testing.assert_array_equal(kept[u], ok)
+
+
+# ---------------------------------------------------------------------------
+# compact
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_compact_bitwise(dtype):
+    U, cap, B = 5, 1000, 333
+    g = torch.Generator(device="cuda").manual_seed(3)
+    k = torch.randn((U, cap, 128), generator=g, device="cuda").to(dtype)
+    v = torch.randn((U, cap, 128), generator=g, device="cuda").to(dtype)
+    pos = torch.randint(0, 1 << 30, (U, cap), generator=g, device="cuda", dtype=torch.int32)
+    rng = np.random.default_rng(4)
+    kept = np.full((U, B), -1, np.int32)
+    nk = np.array([B, B, 0, 1, 200], np.int32)
+    for u in range(U):
+        kept[u, :nk[u]] = np.sort(rng.choice(cap, nk[u], replace=False))
+    kd = torch.zeros((U, B, 128), dtype=dtype, device="cuda")
+    vd = torch.zeros_like(kd)
+    pd = torch.full((U, B), -7, dtype=torch.int32, device="cuda")
+    tri.tri_compact(k, v, pos, torch.as_tensor(kept, device="cuda"), torch.as_tensor(nk, device="cuda"),
+                    kd, vd, pd)
+    torch.cuda.synchronize()
+    for u in range(U):
+        m = int(nk[u])
+        assert H.rows_equal(kd[u, :m], k[u], kept[u, :m])
+        assert H.rows_equal(vd[u, :m], v[u], kept[u, :m])
+        assert torch.equal(pd[u, :m].cpu(), pos[u].cpu()[torch.as_tensor(kept[u, :m], dtype=torch.long)])
+        assert torch.all(pd[u, m:] == -7)
+
+
+# ---------------------------------------------------------------------------
+# prune (score + select + compact)
+# ---------------------------------------------------------------------------
+def _run_prune(spec, wl, gst, B, path=tri.PATH_AUTO, n_valid=None, cap_dst=None):
+    U = spec.n_units
+    cap_dst = cap_dst or B
+    nv = n_valid if n_valid is not None else wl.n_valid
+    kd = torch.zeros((U, cap_dst, 128), dtype=wl.k.dtype, device="cuda")
+    vd = torch.zeros_like(kd)
+    pd = torch.full((U, cap_dst), -1, dtype=torch.int32, device="cuda")
+    kept = torch.empty((U, B), dtype=torch.int32, device="cuda")
+    nk = torch.empty((U,), dtype=torch.int32, device="cuda")
+    ws = tri.workspace(tri.tri_prune_workspace_bytes(spec.n_seq, spec.n_layers, spec.n_kvheads,
+                                                     spec.G, spec.cap, B))
+    tri.tri_prune(tri.config(path=path), wl.k, wl.v, wl.pos, spec.n_seq, spec.n_layers,
+                  spec.n_kvheads, spec.G, wl.p_cur, gst, B, kd, vd, pd, nk, n_valid=nv, kept=kept,
+                  ws=ws)
+    flags = tri.tri_check_device_error(ws)
+    return dict(k=kd, v=vd, pos=pd, kept=kept.cpu().numpy(), n_kept=nk.cpu().numpy(), flags=flags)
+
+
+def _check_prune(spec, wl, ost, out, B, nv, units):
+    if len(units) == spec.n_units:
+        o = oracle.prune(synth.host_elems(wl.k), None, wl.pos.cpu().numpy(), spec.n_seq,
+                         spec.n_layers, spec.n_kvheads, spec.G, ost, wl.p_cur.cpu().numpy(), B,
+                         n_valid=nv, want_gather=False, want_raw=False)
+    else:
+        o = _oracle_units(spec, wl, ost, B, nv, units)
+    exempt = 0
+    for u in units:
+        n = int(nv[u])
+        m = min(n, B)
+        assert out["n_kept"][u] == m
+        gk = out["kept"][u, :m]
+        exempt += H.check_kept(gk, o["final"][u], o["kept"][u], n, B)
+        assert np.all(out["kept"][u, m:] == -1)
+        assert H.rows_equal(out["k"][u, :m], wl.k[u], gk)
+        assert H.rows_equal(out["v"][u, :m], wl.v[u], gk)
+        assert np.array_equal(out["pos"][u, :m].cpu().numpy(), wl.pos[u].cpu().numpy()[gk])
+    return exempt
+
+
+def _oracle_units(spec, wl, ost, B, nv, units):
+    """Oracle on a sample of units without copying the whole cache to the host."""
+    U, cap = spec.n_units, spec.cap
+    fin = np.full((U, cap), np.nan)
+    kept = np.full((U, B), -1, np.int32)
+    idx = torch.as_tensor(list(units), device="cuda")
+    kk = synth.host_elems(wl.k[idx])
+    pp = wl.pos[idx].cpu().numpy()
+    pc = wl.p_cur.cpu().numpy()
+    Lh = spec.n_layers * spec.n_kvheads
+    for i, u in enumerate(units):
+        seq, layer, kvh = u // Lh, (u // spec.n_kvheads) % spec.n_layers, u % spec.n_kvheads
+        st = ost[layer:layer + 1, kvh * spec.G:(kvh + 1) * spec.G]
+        o = oracle.prune(kk[i:i + 1], None, pp[i:i + 1], 1, 1, 1, spec.G, st, pc[seq:seq + 1], B,
+                         n_valid=nv[u:u + 1], want_gather=False, want_raw=False)
+        fin[u] = o["final"][0]
+        kept[u] = o["kept"][0]
+    return dict(final=fin, kept=kept)
+
+
+@pytest.mark.parametrize("path", [tri.PATH_FUSED, tri.PATH_SPLIT])
+@pytest.mark.parametrize("dtype,G", [("bf16", 7), ("bf16", 4), ("bf16", 1), ("f32", 2)])
+def test_prune_parity_ragged(path, dtype, G):
+    B = 300
+    spec = _spec(dtype=dtype, G=G, cap=700, B=B)
+    wl = synth.make_workload(spec, "cuda")
+    gst, ost = H.stats_for(spec, wl)
+    nv = _ragged_nvalid(spec, B)
+    out = _run_prune(spec, wl, gst, B, path=path, n_valid=torch.as_tensor(nv, device="cuda"))
+    assert out["flags"] == 0
+    exempt = _check_prune(spec, wl, ost, out, B, nv, list(range(spec.n_units)))
+    assert exempt <= 2 * spec.n_units
+
+
+def test_prune_paths_agree_bitwise():
+    """The fused and split kernels compute the same scores in the same order,
+    so their kept sets and gathered rows are identical."""
+    B = 900
+    spec = _spec(dtype="bf16", G=7, cap=3200, B=B, n_seq=2, n_layers=2, n_kvheads=4,
+                 positions="scattered", p_cur=32768)
+    wl = synth.make_workload(spec, "cuda")
+    gst, _ = H.stats_for(spec, wl)
+    a = _run_prune(spec, wl, gst, B, path=tri.PATH_FUSED)
+    b = _run_prune(spec, wl, gst, B, path=tri.PATH_SPLIT)
+    np.testing.assert_array_equal(a["kept"], b["kept"])
+    assert torch.equal(a["k"], b["k"]) and torch.equal(a["v"], b["v"])
+
+
+@pytest.mark.parametrize("name,sample", [("c1", None), ("c2", None), ("c3", 24)])
+def test_prune_parity_config(name, sample):
+    spec = synth.SPECS[name]
+    wl = synth.make_workload(spec, "cuda")
+    gst, ost = H.stats_for(spec, wl)
+    out = _run_prune(spec, wl, gst, spec.B)
+    assert out["flags"] == 0
+    nv = wl.n_valid.cpu().numpy()
+    if sample is None:
+        units = list(range(spec.n_units))
+    else:
+        units = sorted(set(np.linspace(0, spec.n_units - 1, sample).astype(int).tolist()))
+    exempt = _check_prune(spec, wl, ost, out, spec.B, nv, units)
+    assert exempt <= 2 * len(units)
+
+
+def test_prune_deterministic():
+    spec = synth.SPECS["c2"]
+    wl = synth.make_workload(spec, "cuda")
+    gst, _ = H.stats_for(spec, wl)
+    a = _run_prune(spec, wl, gst, spec.B)
+    b = _run_prune(spec, wl, gst, spec.B)
+    np.testing.assert_array_equal(a["kept"], b["kept"])
+    assert torch.equal(a["k"], b["k"]) and torch.equal(a["v"], b["v"]) and torch.equal(a["pos"], b["pos"])
+
+
+# ---------------------------------------------------------------------------
+# edge cases
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("path", [tri.PATH_FUSED, tri.PATH_SPLIT])
+def test_identical_keys_keep_lowest_indices(path):
+    """All keys equal: every head has sigma = 0, every z is 0, all scores tie,
+    and the lowest B indices are kept."""
+    spec = _spec(dtype="bf16", G=3, cap=1000, B=123)
+    wl = synth.make_workload(spec, "cuda")
+    wl.k[:] = wl.k[:, :1]
+    gst, _ = H.stats_for(spec, wl)
+    out = _run_prune(spec, wl, gst, 123, path=path)
+    assert np.all(out["kept"] == np.arange(123)[None, :])
+
+
+@pytest.mark.parametrize("path", [tri.PATH_FUSED, tri.PATH_SPLIT])
+def test_nan_key_poisons_unit_and_flags(path):
+    """A NaN key makes that unit's moments NaN: every final score is NaN,
+    NaN ranks last and ties go to the lowest indices; the flag is raised.
+    Other units are unaffected."""
+    B = 50
+    spec = _spec(dtype="bf16", G=2, cap=400, B=B)
+    wl = synth.make_workload(spec, "cuda")
+    wl.k[1, 17, 5] = float("nan")
+    gst, ost = H.stats_for(spec, wl)
+    out = _run_prune(spec, wl, gst, B, path=path)
+    assert out["flags"] & tri.FLAG_NONFINITE
+    assert np.array_equal(out["kept"][1], np.arange(B))
+    o = _oracle_units(spec, wl, ost, B, wl.n_valid.cpu().numpy(), [0, 1])
+    np.testing.assert_array_equal(o["kept"][1], np.arange(B))
+    H.check_kept(out["kept"][0], o["final"][0], o["kept"][0], spec.cap, B)
+
+
+def test_nvalid_out_of_range_is_flagged_and_clamped():
+    spec = _spec(dtype="bf16", G=2, cap=400, B=50)
+    wl = synth.make_workload(spec, "cuda")
+    gst, _ = H.stats_for(spec, wl)
+    nv = torch.full((spec.n_units,), 400, dtype=torch.int32, device="cuda")
+    nv[3] = 401
+    out = _run_prune(spec, wl, gst, 50, n_valid=nv)
+    assert out["flags"] & tri.FLAG_NVALID_RANGE
+    assert out["n_kept"][3] == 50
+
+
+def test_budget_at_least_cache_keeps_everything():
+    spec = _spec(dtype="bf16", G=7, cap=512, B=512)
+    wl = synth.make_workload(spec, "cuda")
+    gst, _ = H.stats_for(spec, wl)
+    out = _run_prune(spec, wl, gst, 600, cap_dst=600)
+    assert np.all(out["n_kept"] == 512)
+    assert np.all(out["kept"][:, :512] == np.arange(512)[None])
+    assert np.all(out["kept"][:, 512:] == -1)
+    assert torch.equal(out["k"][:, :512], wl.k)

@@ -50,10 +50,11 @@ gather_kernel(const uint4* __restrict__ k_src, const uint4* __restrict__ v_src,
             if (g < total) {
                 const int64_t u = g / B;
                 const int64_t r = g - u * B;
-                int nk = n_kept[u];
-                if (nk > B) {
+                int64_t nk = n_kept[u];
+                const int64_t lim = B < cap_dst ? B : cap_dst;
+                if (nk > lim || nk < 0) {
                     if (lane == 0 && r == 0) raise_flag(flag, TRI_FLAG_INDEX_RANGE);
-                    nk = static_cast<int>(B);
+                    nk = nk < 0 ? 0 : lim;
                 }
                 if (r < nk) {
                     const int32_t j = kept[g];

@@ -92,27 +92,46 @@ struct ScoreSmem {
     int last_flag;
 };
 
+// Merge the per-tile moment partials of one unit, by one warp: lane l sums
+// tiles l, l+32, ... in order, then a fixed shuffle tree; lane 0's result is
+// used, so the merge is bitwise reproducible.
 template <int G>
 __device__ __forceinline__ void merge_unit_moments(const double* part, int tpu, int n,
                                                    float2* mom_u) {
-    // Fixed tile order: bitwise reproducible.
+    const int lane = threadIdx.x & 31;
+    double s1[G], s2[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) s1[h] = s2[h] = 0.0;
+    for (int i = lane; i < tpu; i += 32) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            s1[h] += part[(static_cast<int64_t>(i) * G + h) * 2];
+            s2[h] += part[(static_cast<int64_t>(i) * G + h) * 2 + 1];
+        }
+    }
+#pragma unroll
     for (int h = 0; h < G; ++h) {
-        double s1 = 0.0, s2 = 0.0;
-        for (int i = 0; i < tpu; ++i) {
-            s1 += part[(static_cast<int64_t>(i) * G + h) * 2];
-            s2 += part[(static_cast<int64_t>(i) * G + h) * 2 + 1];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            s1[h] += __shfl_down_sync(0xffffffffu, s1[h], o);
+            s2[h] += __shfl_down_sync(0xffffffffu, s2[h], o);
         }
-        float mu = 0.f, inv = 0.f;
-        if (n > 0) {
-            const double m = s1 / n;
-            double var = s2 / n - m * m;
-            if (var < 0.0) var = 0.0;
-            const double sd = sqrt(var);
-            mu = static_cast<float>(m);
-            inv = sd > 0.0 ? static_cast<float>(1.0 / sd) : 0.f;
-            if (!(sd == sd)) inv = __int_as_float(0x7fc00000);  // NaN propagates
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            float mu = 0.f, inv = 0.f;
+            if (n > 0) {
+                const double m = s1[h] / n;
+                double var = s2[h] / n - m * m;
+                if (var < 0.0) var = 0.0;
+                const double sd = sqrt(var);
+                mu = static_cast<float>(m);
+                inv = sd > 0.0 ? static_cast<float>(1.0 / sd) : 0.f;
+                if (!(sd == sd)) inv = __int_as_float(0x7fc00000);  // NaN propagates
+            }
+            mom_u[h] = make_float2(mu, inv);
         }
-        mom_u[h] = make_float2(mu, inv);
     }
 }
 
@@ -241,11 +260,14 @@ score_kernel(const __grid_constant__ CUtensorMap kmap, ScoreArgs a) {
             __threadfence();
             const uint32_t done = atomicAdd(&a.counters[u], 1u);
             sm.last_flag = (done == static_cast<uint32_t>(a.tpu) - 1u);
-            if (sm.last_flag) {
-                __threadfence();
-                merge_unit_moments<G>(a.partial + u * a.tpu * G * 2, a.tpu, n, a.mom + u * G);
-                a.counters[u] = 0u;
-            }
+        }
+        named_sync(1, S::kConsumers);
+        if (sm.last_flag && warp == 0) {
+            // The last tile of the unit to finish merges every tile's partial.
+            __threadfence();
+            merge_unit_moments<G>(a.partial + u * a.tpu * G * 2, static_cast<int>(a.tpu), n,
+                                  a.mom + u * G);
+            if (lane == 0) a.counters[u] = 0u;
         }
         named_sync(1, S::kConsumers);
     }
@@ -276,18 +298,28 @@ zmax_kernel(const float* __restrict__ raw, int64_t cap, const int32_t* __restric
         inv[h] = m.y;
     }
     bool nonfinite = false;
-    const int j1 = min(j0 + kZChunk, n);
-    for (int j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
-        float best = 0.f;
+    constexpr int kPer = kZChunk / 256;  // keys per thread
+    float sv[kPer][G];
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
-            const float s = raw[(u * G + h) * cap + j];
-            const float z = (s - mu[h]) * inv[h];
-            best = (h == 0) ? z : fmaxf(best, z);
+    for (int i = 0; i < kPer; ++i) {
+        const int j = j0 + threadIdx.x + 256 * i;
+#pragma unroll
+        for (int h = 0; h < G; ++h) sv[i][h] = (j < n) ? raw[(u * G + h) * cap + j] : 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        const int j = j0 + threadIdx.x + 256 * i;
+        if (j < n) {
+            float best = 0.f;
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float z = (sv[i][h] - mu[h]) * inv[h];
+                best = (h == 0) ? z : fmaxf(best, z);
+            }
+            fin[u * cap + j] = best;
+            if (best != best) nonfinite = true;
+            if (hist0) atomicAdd(&hist[ordered_key(best) >> kShift0], 1u);
         }
-        fin[u * cap + j] = best;
-        if (best != best) nonfinite = true;
-        if (hist0) atomicAdd(&hist[ordered_key(best) >> kShift0], 1u);
     }
     if (nonfinite) raise_flag(flag, TRI_FLAG_NONFINITE);
     if (hist0) {

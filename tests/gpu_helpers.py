@@ -57,7 +57,8 @@ def check_final(gpu_fin, ora_fin, n):
 
 
 def check_kept(gpu_kept, ora_fin, ora_kept, n, B):
-    """Compare kept sets with the exempt band; returns the number of exempt keys."""
+    """Compare kept sets with the exempt band.  Returns the number of keys on
+    which the two sets differ (all of them inside the band)."""
     m = min(n, B)
     gk = np.asarray(gpu_kept[:m])
     assert len(gk) == m
@@ -81,7 +82,7 @@ def check_kept(gpu_kept, ora_fin, ora_kept, n, B):
     diff = gset != oset
     assert not np.any(diff & ~band), (
         f"kept sets differ outside the exempt band at {np.nonzero(diff & ~band)[0][:10]}")
-    return int(band.sum())
+    return int(diff.sum())
 
 
 def rows_equal(dst, src, idx):

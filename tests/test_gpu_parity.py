@@ -202,18 +202,18 @@ def _check_prune(spec, wl, ost, out, B, nv, units):
                          n_valid=nv, want_gather=False, want_raw=False)
     else:
         o = _oracle_units(spec, wl, ost, B, nv, units)
-    exempt = 0
+    mismatched = 0
     for u in units:
         n = int(nv[u])
         m = min(n, B)
         assert out["n_kept"][u] == m
         gk = out["kept"][u, :m]
-        exempt += H.check_kept(gk, o["final"][u], o["kept"][u], n, B)
+        mismatched += H.check_kept(gk, o["final"][u], o["kept"][u], n, B)
         assert np.all(out["kept"][u, m:] == -1)
         assert H.rows_equal(out["k"][u, :m], wl.k[u], gk)
         assert H.rows_equal(out["v"][u, :m], wl.v[u], gk)
         assert np.array_equal(out["pos"][u, :m].cpu().numpy(), wl.pos[u].cpu().numpy()[gk])
-    return exempt
+    return mismatched
 
 
 def _oracle_units(spec, wl, ost, B, nv, units):
@@ -246,8 +246,8 @@ def test_prune_parity_ragged(path, dtype, G):
     nv = _ragged_nvalid(spec, B)
     out = _run_prune(spec, wl, gst, B, path=path, n_valid=torch.as_tensor(nv, device="cuda"))
     assert out["flags"] == 0
-    exempt = _check_prune(spec, wl, ost, out, B, nv, list(range(spec.n_units)))
-    assert exempt <= 2 * spec.n_units
+    mismatched = _check_prune(spec, wl, ost, out, B, nv, list(range(spec.n_units)))
+    assert mismatched <= 2 * spec.n_units
 
 
 def test_prune_paths_agree_bitwise():
@@ -276,8 +276,8 @@ def test_prune_parity_config(name, sample):
         units = list(range(spec.n_units))
     else:
         units = sorted(set(np.linspace(0, spec.n_units - 1, sample).astype(int).tolist()))
-    exempt = _check_prune(spec, wl, ost, out, spec.B, nv, units)
-    assert exempt <= 2 * len(units)
+    mismatched = _check_prune(spec, wl, ost, out, spec.B, nv, units)
+    assert mismatched <= 2 * len(units)
 
 
 def test_prune_deterministic():

@@ -195,10 +195,14 @@ struct PruneWs {
 };
 
 bool use_fused(tri_dtype dt, int G, int64_t cap, int64_t B) {
-    const size_t smem = fused_smem_bytes(dt, G, cap);
-    const size_t tiles = dt == TRI_BF16 ? 3 * 32768 : 2 * 65536;
-    const int64_t m = B < cap ? B : cap;
-    return smem <= fused_smem_limit() && static_cast<size_t>(kHistBins0 * 4 + m * 4) <= tiles;
+    return fused_smem_bytes(dt, G, cap, B) <= fused_smem_limit();
+}
+
+// CTAs of the persistent fused kernel: one per SM (its shared memory allows
+// no more), never more than the units.
+int64_t fused_ctas(int64_t U) {
+    const int64_t sms = device_info().sm_count > 0 ? device_info().sm_count : 148;
+    return U < sms ? U : sms;
 }
 
 PruneWs prune_ws(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int64_t cap,
@@ -209,6 +213,7 @@ PruneWs prune_ws(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int6
     if (w.fused) {
         Carve c;
         w.sc.wts = c.take(static_cast<size_t>(U * G) * kWHead * 4);
+        w.sc.raw = c.take(static_cast<size_t>(fused_ctas(U) * G * cap) * 4);
         w.kept = own_kept ? c.take(static_cast<size_t>(U * B) * 4) : 0;
         w.fin = 0;
         w.total = c.off;
@@ -398,8 +403,10 @@ size_t tri_prune_workspace_bytes(int64_t n_seq, int64_t n_layers, int64_t n_kvhe
     if (check_units(n_seq, n_layers, n_kvheads, G, cap) != TRI_OK || B < 1) return kWsHeader;
     size_t best = 0;
     for (tri_dtype dt : {TRI_BF16, TRI_F32}) {
-        const size_t t = prune_ws(n_seq, n_layers, n_kvheads, G, cap, B, dt, true, TRI_PATH_SPLIT).total;
-        if (t > best) best = t;
+        for (int path : {TRI_PATH_AUTO, TRI_PATH_SPLIT}) {
+            const size_t t = prune_ws(n_seq, n_layers, n_kvheads, G, cap, B, dt, true, path).total;
+            if (t > best) best = t;
+        }
     }
     return best;
 }
@@ -444,10 +451,11 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
 
     if (w.fused) {
         CUtensorMap map;
-        TRI_TRY(make_key_map(&map, k_src, dt, U * cap_src, 128));
+        TRI_TRY(make_key_map(&map, k_src, dt, U * cap_src, fused_tile_keys(dt)));
         TRI_CUDA(cudaMemsetAsync(ws, 0, kWsHeader, s));
         TRI_CUDA(launch_fold(stats, p_cur, n_seq, n_layers, n_kvheads * G, cfg->theta, off, wts, s));
         FusedArgs a;
+        a.n_units = U;
         a.cap = cap_src;
         a.cap_dst = cap_dst;
         a.B = B;
@@ -461,8 +469,9 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
         a.pos_dst = pos_dst;
         a.kept = kept_idx;
         a.n_kept = n_kept;
+        a.scratch = reinterpret_cast<float*>(ws_at(ws, w.sc.raw));
         a.flag = flag;
-        return cuda_status(launch_fused(dt, G, map, a, U, s));
+        return cuda_status(launch_fused(dt, G, map, a, static_cast<int>(fused_ctas(U)), s));
     }
 
     CUtensorMap map;

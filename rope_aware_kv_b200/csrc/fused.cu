@@ -1,18 +1,30 @@
-// fused.cu -- one prune step of a small cache in a single kernel, one CTA per
-// unit: score -> z-score / max -> radix select -> ordered gather.
+// fused.cu -- one prune step of small caches in a single persistent kernel:
+// each CTA takes whole units (one KV head's cache) in turn and runs
+// score -> z-score / max -> radix select -> ordered gather on each.
 //
 // Every phase follows the same definitions as the split kernels (score.cu,
 // select.cu, compact.cu): the folded S~ per query head (talk page: S_trig,
 // S_norm, S~), z-score per head and max over the GQA group (hyper.ai summary,
 // Method section), top-B by (score desc, index asc) kept in temporal order
-// (jaedaily.cn tutorial, eviction step).  Here the per-head scores of the unit
-// stay in shared memory, the moments need no second launch, and the three
-// radix passes run on shared-memory histograms.  Only the key reads, the kept
-// V reads and the K/V/position writes touch HBM (the kept K rows are re-read,
-// usually from L2).
+// (jaedaily.cn tutorial, eviction step).
 //
-// Shared memory: [key tiles][G weight records][G x cap scores][barriers ...].
-// After scoring, the tile area is reused for the histogram and the kept list.
+// Per unit:
+//   score   a producer lane streams 128-key tiles (32 KB) into a 4-stage TMA
+//           ring; the four math warps form two pairs, each pair scores one
+//           tile with every lane on 4 keys and the GQA heads split between
+//           the pair's two warps (so one broadcast weight load feeds 4 keys);
+//           per-head scores go to a per-CTA float32 scratch that stays in L2,
+//           float64 moments stay in registers.
+//   z-max   fixed-order moment merge, final = max_h z_h into shared memory,
+//           first radix digit histogram.
+//   select  two more radix digits on shared-memory histograms, then the
+//           ordered compaction of kept indices (warp ballots).
+//   gather  kept rows form runs of consecutive indices; one lane moves each
+//           run piece (<= 16 KB) of K and of V with cp.async.bulk through an
+//           8-stage shared-memory ring (global -> shared -> global), keeping
+//           up to 7 pieces in flight; the other lanes copy positions.
+// HBM traffic per unit is the compulsory bytes plus the re-read of kept K
+// rows (often from L2).
 #include "select_core.cuh"
 #include "score_core.cuh"
 #include "tri_internal.cuh"
@@ -22,317 +34,457 @@ namespace tri {
 
 template <typename T>
 struct FusedShape {
-    static constexpr int kRowBytes = kD * static_cast<int>(sizeof(T));
+    static constexpr int kRowBytes = kD * static_cast<int>(sizeof(T));  // 256 / 512
     static constexpr int kBoxes = kRowBytes / 128;
-    static constexpr int kTile = 128;                      // keys per tile, one per consumer
+    static constexpr int kKPT = sizeof(T) == 2 ? 4 : 2;                 // keys per lane
+    static constexpr int kTile = 32 * kKPT;                             // keys per tile
     static constexpr int kBoxBytes = kTile * 128;
-    static constexpr int kStageBytes = kTile * kRowBytes;  // 32 KB bf16 / 64 KB f32
-    static constexpr int kStages = sizeof(T) == 2 ? 3 : 2;
-    static constexpr int kTilesBytes = kStages * kStageBytes;
-    static constexpr int kConsumers = 128;
-    static constexpr int kThreads = kConsumers + 32;
+    static constexpr int kStageBytes = kTile * kRowBytes;               // 32 KB
+    static constexpr int kStages = 4;
+    static constexpr int kRegionA = kStages * kStageBytes;              // 128 KB
+    static constexpr int kMath = 128;
+    static constexpr int kThreads = kMath + 32;
     static constexpr int kWarps = kThreads / 32;
-    static constexpr int kVec = kRowBytes / 16;            // 16-byte vectors per row
+    static constexpr int kGStage = 16384;                               // gather piece buffer
+    static constexpr int kGStages = kRegionA / kGStage;                 // 8
+    static constexpr int kGRows = kGStage / kRowBytes;                  // rows per piece
 };
 
 struct FusedLayout {
-    size_t w, sc, bars, red, mom, misc, total;
+    size_t w, fin, kidx, bars, red, misc, total;
 };
 
 template <typename T>
-__host__ __device__ inline FusedLayout fused_layout(int G, int64_t cap) {
+__host__ __device__ inline FusedLayout fused_layout(int G, int64_t cap, int64_t B) {
     using S = FusedShape<T>;
     FusedLayout L;
-    const int64_t capP = (cap + 3) & ~int64_t(3);
-    L.w = S::kTilesBytes;
-    L.sc = L.w + static_cast<size_t>(G) * kWHead * 4;
-    L.bars = L.sc + static_cast<size_t>(G) * capP * 4;
-    L.bars = (L.bars + 15) & ~size_t(15);
-    L.red = L.bars + 2 * S::kStages * 8;
-    L.mom = L.red + static_cast<size_t>(4) * G * 2 * 8;
-    L.misc = L.mom + static_cast<size_t>(G) * 8;
-    L.total = L.misc + 128 + 1024;  // + state / warp counts, + alignment slack
+    const int64_t capP = (cap + 4) & ~int64_t(3);
+    const int64_t m = B < cap ? B : cap;
+    L.w = S::kRegionA;
+    L.fin = L.w + static_cast<size_t>(G) * kWHead * 4;
+    L.kidx = L.fin + static_cast<size_t>(capP) * 4;
+    L.bars = L.kidx + ((static_cast<size_t>(m) * 4 + 15) & ~size_t(15));
+    L.red = L.bars + (2 * S::kStages + S::kGStages) * 8;
+    L.misc = L.red + static_cast<size_t>(4) * kMaxG * 2 * 8;
+    L.total = L.misc + 256 + 1024;  // state and warp counts; alignment slack
     return L;
 }
+
+// Head split between the two warps of a pair.
+template <int G>
+struct HeadSplit {
+    static constexpr int kA = (G + 1) / 2;
+    static constexpr int kB = G - kA;
+};
 
 template <typename T, int G>
 __global__ void __launch_bounds__(FusedShape<T>::kThreads, 1)
 prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
     using S = FusedShape<T>;
+    constexpr int GA = HeadSplit<G>::kA;
+    constexpr int GB = HeadSplit<G>::kB;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const FusedLayout L = fused_layout<T>(G, a.cap);
-    const int64_t capP = (a.cap + 3) & ~int64_t(3);
-    uint8_t* tiles = base;
+    const FusedLayout L = fused_layout<T>(G, a.cap, a.B);
+    uint8_t* regA = base;
     float* w = reinterpret_cast<float*>(base + L.w);
-    float* sc = reinterpret_cast<float*>(base + L.sc);
+    float* fin = reinterpret_cast<float*>(base + L.fin);
+    int32_t* kidx = reinterpret_cast<int32_t*>(base + L.kidx);
     uint64_t* full = reinterpret_cast<uint64_t*>(base + L.bars);
     uint64_t* empty = full + S::kStages;
-    double* red = reinterpret_cast<double*>(base + L.red);      // [4][G][2]
-    float2* mom = reinterpret_cast<float2*>(base + L.mom);       // [G]
+    uint64_t* gfull = empty + S::kStages;
+    double* red = reinterpret_cast<double*>(base + L.red);  // [4 warps][kMaxG][2]
     SelState* st = reinterpret_cast<SelState*>(base + L.misc);
-    uint32_t* wcnt = reinterpret_cast<uint32_t*>(base + L.misc + 32);  // [kWarps][2]
-    uint32_t* hist = reinterpret_cast<uint32_t*>(tiles);               // after scoring
-    int32_t* kidx = reinterpret_cast<int32_t*>(tiles + kHistBins0 * 4);
+    float2* mom = reinterpret_cast<float2*>(base + L.misc + 16);            // [kMaxG]
+    uint32_t* wcnt = reinterpret_cast<uint32_t*>(base + L.misc + 16 + 64);  // [kWarps][2]
+    int32_t* nchunks = reinterpret_cast<int32_t*>(base + L.misc + 16 + 64 + 48);
+    int32_t* abort_flag = nchunks + 1;
+    uint32_t* hist = reinterpret_cast<uint32_t*>(regA);  // between scoring and gathering
+    int32_t* chunk_r = reinterpret_cast<int32_t*>(fin);  // after the compaction
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const int64_t u = blockIdx.x;
-    const int n = clamp_nvalid(a.n_valid, u, a.cap, tid == 0 ? a.flag : nullptr);
     const int64_t B = a.B;
-    const int m = static_cast<int>(n < B ? n : B);
-    const bool keep_all = n <= B;
+    float* scratch = a.scratch + static_cast<int64_t>(blockIdx.x) * G * a.cap;
 
-    if (!keep_all) {
-        // ---------------- Phase A: scores into shared memory ----------------
-        if (tid == S::kConsumers) {
-            for (int i = 0; i < S::kStages; ++i) {
-                mbar_init(&full[i], 1);
-                mbar_init(&empty[i], S::kConsumers);
+    if (tid == S::kMath) {
+        for (int i = 0; i < S::kStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 64);
+        }
+        for (int i = 0; i < S::kGStages; ++i) mbar_init(&gfull[i], 1);
+        fence_barrier_init();
+        prefetch_tensormap(&kmap);
+        *abort_flag = 0;
+    }
+    __syncthreads();
+
+    uint32_t tiles_done = 0;   // running tile count (TMA ring position) of this CTA
+    uint32_t pieces_done = 0;  // running gather-piece count (gather ring position)
+
+    for (int64_t u = blockIdx.x; u < a.n_units; u += gridDim.x) {
+        if (*abort_flag) break;  // a bounded wait gave up: stop cleanly
+        const int n = clamp_nvalid(a.n_valid, u, a.cap, tid == 0 ? a.flag : nullptr);
+        const int m = static_cast<int>(n < B ? n : B);
+        const bool keep_all = n <= B;
+        const int n_tiles = keep_all ? 0 : (n + S::kTile - 1) / S::kTile;
+
+        if (!keep_all) {
+            // ---------------- score ----------------
+            if (tid < S::kMath) {
+                const float4* src = reinterpret_cast<const float4*>(a.wts + u * G * kWHead);
+                float4* dst = reinterpret_cast<float4*>(w);
+                for (int e = tid; e < G * kWHead / 4; e += S::kMath) dst[e] = src[e];
             }
-            fence_barrier_init();
-            prefetch_tensormap(&kmap);
-        }
-        {
-            const float4* src = reinterpret_cast<const float4*>(a.wts + u * G * kWHead);
-            float4* dst = reinterpret_cast<float4*>(w);
-            for (int e = tid; e < G * kWHead / 4; e += S::kThreads) dst[e] = src[e];
-        }
-        __syncthreads();
-        const int n_tiles = (n + S::kTile - 1) / S::kTile;
-        if (tid >= S::kConsumers) {
-            if (tid == S::kConsumers) {
-                int stage = 0;
-                uint32_t phase = 0;
-                uint32_t issued[S::kStages] = {};
-                for (int i = 0; i < n_tiles; ++i) {
-                    if (!mbar_wait(&empty[stage], phase ^ 1, a.flag)) break;
-                    mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
-                    const int32_t y = static_cast<int32_t>(u * a.cap + static_cast<int64_t>(i) * S::kTile);
+            __syncthreads();
+            if (tid >= S::kMath) {
+                if (tid == S::kMath) {
+                    for (int i = 0; i < n_tiles; ++i) {
+                        const uint32_t tc = tiles_done + i;
+                        const int stage = tc % S::kStages;
+                        if (!mbar_wait(&empty[stage], ((tc / S::kStages) & 1) ^ 1, a.flag)) {
+                            *abort_flag = 1;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
+                        const int32_t y =
+                            static_cast<int32_t>(u * a.cap + static_cast<int64_t>(i) * S::kTile);
 #pragma unroll
-                    for (int b = 0; b < S::kBoxes; ++b)
-                        tma_load_2d(tiles + stage * S::kStageBytes + b * S::kBoxBytes, &kmap,
-                                    &full[stage], b * (128 / static_cast<int>(sizeof(T))), y);
-                    issued[stage]++;
-                    if (++stage == S::kStages) {
-                        stage = 0;
-                        phase ^= 1;
+                        for (int b = 0; b < S::kBoxes; ++b)
+                            tma_load_2d(regA + stage * S::kStageBytes + b * S::kBoxBytes, &kmap,
+                                        &full[stage], b * (128 / static_cast<int>(sizeof(T))), y);
                     }
                 }
-                for (int s2 = 0; s2 < S::kStages; ++s2)
-                    if (issued[s2]) mbar_wait(&full[s2], (issued[s2] - 1) & 1, a.flag);
-            }
-        } else {
-            double m1[G], m2[G];
+            } else {
+                const int pair = warp >> 1, half = warp & 1;
+                const int hb = half == 0 ? 0 : GA;
+                const int gh = half == 0 ? GA : GB;
+                double m1[GA], m2[GA];
 #pragma unroll
-            for (int h = 0; h < G; ++h) m1[h] = m2[h] = 0.0;
-            int stage = 0;
-            uint32_t phase = 0;
-            for (int i = 0; i < n_tiles; ++i) {
-                if (!mbar_wait(&full[stage], phase, a.flag)) break;
-                float s[1][G];
-                score_rows<T, G, 1, S::kBoxBytes>(tiles + stage * S::kStageBytes, w, tid, s);
-                mbar_arrive(&empty[stage]);
-                if (++stage == S::kStages) {
-                    stage = 0;
-                    phase ^= 1;
+                for (int h = 0; h < GA; ++h) m1[h] = m2[h] = 0.0;
+                for (int i = pair; i < n_tiles; i += 2) {
+                    const uint32_t tc = tiles_done + i;
+                    const int stage = tc % S::kStages;
+                    if (!mbar_wait(&full[stage], (tc / S::kStages) & 1, a.flag)) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                    const uint8_t* tile = regA + stage * S::kStageBytes;
+                    float s[S::kKPT][GA];
+                    if (half == 0) {
+                        score_rows<T, GA, S::kKPT, S::kBoxBytes, 32>(tile, w, lane, s);
+                    } else {
+                        if constexpr (GB > 0) {
+                            float sb[S::kKPT][GB];
+                            score_rows<T, GB, S::kKPT, S::kBoxBytes, 32>(tile, w + GA * kWHead,
+                                                                          lane, sb);
+#pragma unroll
+                            for (int k = 0; k < S::kKPT; ++k) {
+#pragma unroll
+                                for (int h = 0; h < GA; ++h) s[k][h] = 0.f;
+#pragma unroll
+                                for (int h = 0; h < GB; ++h) s[k][h] = sb[k][h];
+                            }
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < S::kKPT; ++k)
+#pragma unroll
+                                for (int h = 0; h < GA; ++h) s[k][h] = 0.f;
+                        }
+                    }
+                    mbar_arrive(&empty[stage]);
+#pragma unroll
+                    for (int k = 0; k < S::kKPT; ++k) {
+                        const int j = i * S::kTile + lane + 32 * k;
+                        if (j < n) {
+#pragma unroll
+                            for (int h = 0; h < GA; ++h) {
+                                if (h < gh) {
+                                    scratch[static_cast<int64_t>(hb + h) * a.cap + j] = s[k][h];
+                                    const double d = s[k][h];
+                                    m1[h] += d;
+                                    m2[h] = fma(d, d, m2[h]);
+                                }
+                            }
+                        }
+                    }
                 }
-                const int j = i * S::kTile + tid;
-                if (j < n) {
 #pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        sc[h * capP + j] = s[0][h];
-                        const double d = s[0][h];
-                        m1[h] += d;
-                        m2[h] = fma(d, d, m2[h]);
+                for (int h = 0; h < GA; ++h) {
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) {
+                        m1[h] += __shfl_down_sync(0xffffffffu, m1[h], o);
+                        m2[h] += __shfl_down_sync(0xffffffffu, m2[h], o);
+                    }
+                    if (lane == 0) {
+                        red[(warp * kMaxG + h) * 2] = m1[h];
+                        red[(warp * kMaxG + h) * 2 + 1] = m2[h];
                     }
                 }
             }
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    m1[h] += __shfl_xor_sync(0xffffffffu, m1[h], o);
-                    m2[h] += __shfl_xor_sync(0xffffffffu, m2[h], o);
-                }
-                if (lane == 0) {
-                    red[(warp * G + h) * 2] = m1[h];
-                    red[(warp * G + h) * 2 + 1] = m2[h];
-                }
+            __syncthreads();
+            if (*abort_flag) break;
+            // ---------------- moments (fixed order: pair 0 then pair 1) ----------------
+            if (tid < G) {
+                const int h = tid;
+                const int half = h < GA ? 0 : 1;
+                const int hh = h < GA ? h : h - GA;
+                const double s1 =
+                    red[(half * kMaxG + hh) * 2] + red[((2 + half) * kMaxG + hh) * 2];
+                const double s2 =
+                    red[(half * kMaxG + hh) * 2 + 1] + red[((2 + half) * kMaxG + hh) * 2 + 1];
+                const double mu = s1 / n;
+                double var = s2 / n - mu * mu;
+                if (var < 0.0) var = 0.0;
+                const double sd = sqrt(var);
+                float inv = sd > 0.0 ? static_cast<float>(1.0 / sd) : 0.f;
+                if (!(sd == sd)) inv = __int_as_float(0x7fc00000);
+                mom[h] = make_float2(static_cast<float>(mu), inv);
             }
-        }
-        __syncthreads();
-        // ---------------- Phase B: moments (fixed order) ----------------
-        if (tid < G) {
-            const int h = tid;
-            const double s1 = ((red[(0 * G + h) * 2] + red[(1 * G + h) * 2]) + red[(2 * G + h) * 2]) +
-                              red[(3 * G + h) * 2];
-            const double s2 = ((red[(0 * G + h) * 2 + 1] + red[(1 * G + h) * 2 + 1]) +
-                               red[(2 * G + h) * 2 + 1]) + red[(3 * G + h) * 2 + 1];
-            const double mu = s1 / n;
-            double var = s2 / n - mu * mu;
-            if (var < 0.0) var = 0.0;
-            const double sd = sqrt(var);
-            float inv = sd > 0.0 ? static_cast<float>(1.0 / sd) : 0.f;
-            if (!(sd == sd)) inv = __int_as_float(0x7fc00000);
-            mom[h] = make_float2(static_cast<float>(mu), inv);
-        }
-        for (int b = tid; b < kHistBins0; b += S::kThreads) hist[b] = 0;
-        __syncthreads();
-        // ---------------- Phase C: final score + first digit ----------------
-        {
-            float mu[G], inv[G];
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-                mu[h] = mom[h].x;
-                inv[h] = mom[h].y;
-            }
-            bool nonfinite = false;
-            for (int j = tid; j < n; j += S::kThreads) {
-                float best = 0.f;
+            for (int b = tid; b < kHistBins0; b += S::kThreads) hist[b] = 0;
+            __syncthreads();
+            // ---------------- final score + first digit ----------------
+            {
+                float mu[G], inv[G];
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
-                    const float z = (sc[h * capP + j] - mu[h]) * inv[h];
-                    best = (h == 0) ? z : fmaxf(best, z);
+                    mu[h] = mom[h].x;
+                    inv[h] = mom[h].y;
                 }
-                sc[j] = best;
-                if (best != best) nonfinite = true;
-                atomicAdd(&hist[ordered_key(best) >> pass_shift(0)], 1u);
+                bool nonfinite = false;
+                constexpr int kU = 4;
+                for (int j0 = tid; j0 < n; j0 += S::kThreads * kU) {
+                    float sv[kU][G];
+#pragma unroll
+                    for (int q = 0; q < kU; ++q) {
+                        const int j = j0 + q * S::kThreads;
+#pragma unroll
+                        for (int h = 0; h < G; ++h)
+                            sv[q][h] = j < n ? scratch[static_cast<int64_t>(h) * a.cap + j] : 0.f;
+                    }
+#pragma unroll
+                    for (int q = 0; q < kU; ++q) {
+                        const int j = j0 + q * S::kThreads;
+                        if (j < n) {
+                            float best = 0.f;
+#pragma unroll
+                            for (int h = 0; h < G; ++h) {
+                                const float z = (sv[q][h] - mu[h]) * inv[h];
+                                best = (h == 0) ? z : fmaxf(best, z);
+                            }
+                            fin[j] = best;
+                            if (best != best) nonfinite = true;
+                            atomicAdd(&hist[ordered_key(best) >> pass_shift(0)], 1u);
+                        }
+                    }
+                }
+                if (nonfinite) raise_flag(a.flag, TRI_FLAG_NONFINITE);
             }
-            if (nonfinite) raise_flag(a.flag, TRI_FLAG_NONFINITE);
-        }
-        __syncthreads();
-        // ---------------- Phase D: radix passes 1 and 2 ----------------
-        if (warp == 0) {
-            uint32_t bin, above;
-            warp_find_bin(hist, 1 << pass_bits(0), static_cast<uint32_t>(B), bin, above);
-            if (lane == 0) {
-                st->prefix = bin;
-                st->k = static_cast<uint32_t>(B) - above;
-                st->gt = above;
-                st->keep_all = 0;
-            }
-        }
-        __syncthreads();
-        for (int p = 1; p < 3; ++p) {
-            const int nb = 1 << pass_bits(p);
-            for (int b = tid; b < nb; b += S::kThreads) hist[b] = 0;
             __syncthreads();
-            const uint32_t prefix = st->prefix;
-            const int shift = pass_shift(p);
-            const int hi_shift = shift + pass_bits(p);
-            for (int j = tid; j < n; j += S::kThreads) {
-                const uint32_t key = ordered_key(sc[j]);
-                if ((key >> hi_shift) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
-            }
-            __syncthreads();
+            // ---------------- radix passes 1 and 2 ----------------
             if (warp == 0) {
                 uint32_t bin, above;
-                warp_find_bin(hist, nb, st->k, bin, above);
+                warp_find_bin(hist, 1 << pass_bits(0), static_cast<uint32_t>(B), bin, above);
                 if (lane == 0) {
-                    st->prefix = (prefix << pass_bits(p)) | bin;
-                    st->k -= above;
-                    st->gt += above;
+                    st->prefix = bin;
+                    st->k = static_cast<uint32_t>(B) - above;
+                    st->gt = above;
+                    st->keep_all = 0;
                 }
             }
             __syncthreads();
-        }
-        // ---------------- Phase E: ordered compaction of indices ----------------
-        {
-            const uint32_t T = st->prefix, kt = st->k;
-            const int seg = ((n + S::kWarps * 32 - 1) / (S::kWarps * 32)) * 32;
-            const int j0 = warp * seg;
-            const int j1 = min(j0 + seg, n);
-            uint32_t gt = 0, eq = 0;
-            for (int j = j0 + lane; j - lane < j1; j += 32) {
-                const bool valid = j < j1;
-                const uint32_t key = valid ? ordered_key(sc[j]) : 0u;
-                gt += __popc(__ballot_sync(0xffffffffu, valid && key > T));
-                eq += __popc(__ballot_sync(0xffffffffu, valid && key == T));
-            }
-            if (lane == 0) {
-                wcnt[2 * warp] = gt;
-                wcnt[2 * warp + 1] = eq;
-            }
-            __syncthreads();
-            uint32_t pos = 0, ties = 0;
-            for (int v = 0; v < warp; ++v) {
-                const uint32_t take = ties < kt ? min(wcnt[2 * v + 1], kt - ties) : 0u;
-                pos += wcnt[2 * v] + take;
-                ties += wcnt[2 * v + 1];
-            }
-            const uint32_t lt = (1u << lane) - 1u;
-            for (int j = j0 + lane; j - lane < j1; j += 32) {
-                const bool valid = j < j1;
-                const uint32_t key = valid ? ordered_key(sc[j]) : 0u;
-                const bool is_eq = valid && key == T;
-                const uint32_t beq = __ballot_sync(0xffffffffu, is_eq);
-                const uint32_t my_tie = ties + __popc(beq & lt);
-                const bool keep = valid && (key > T || (is_eq && my_tie < kt));
-                const uint32_t bk = __ballot_sync(0xffffffffu, keep);
-                if (keep) {
-                    const uint32_t r = pos + __popc(bk & lt);
-                    if (r < static_cast<uint32_t>(m)) kidx[r] = j;
+            for (int p = 1; p < 3; ++p) {
+                const int nb = 1 << pass_bits(p);
+                for (int b = tid; b < nb; b += S::kThreads) hist[b] = 0;
+                __syncthreads();
+                const uint32_t prefix = st->prefix;
+                const int shift = pass_shift(p);
+                const int hi_shift = shift + pass_bits(p);
+                for (int j = tid; j < n; j += S::kThreads) {
+                    const uint32_t key = ordered_key(fin[j]);
+                    if ((key >> hi_shift) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
                 }
-                pos += __popc(bk);
-                ties += __popc(beq);
+                __syncthreads();
+                if (warp == 0) {
+                    uint32_t bin, above;
+                    warp_find_bin(hist, nb, st->k, bin, above);
+                    if (lane == 0) {
+                        st->prefix = (prefix << pass_bits(p)) | bin;
+                        st->k -= above;
+                        st->gt += above;
+                    }
+                }
+                __syncthreads();
             }
+            // ---------------- ordered compaction of indices ----------------
+            {
+                const uint32_t Tk = st->prefix, kt = st->k;
+                const int seg = ((n + S::kWarps * 32 - 1) / (S::kWarps * 32)) * 32;
+                const int j0 = warp * seg;
+                const int j1 = min(j0 + seg, n);
+                uint32_t gt = 0, eq = 0;
+                for (int j = j0 + lane; j - lane < j1; j += 32) {
+                    const bool valid = j < j1;
+                    const uint32_t key = valid ? ordered_key(fin[j]) : 0u;
+                    gt += __popc(__ballot_sync(0xffffffffu, valid && key > Tk));
+                    eq += __popc(__ballot_sync(0xffffffffu, valid && key == Tk));
+                }
+                if (lane == 0) {
+                    wcnt[2 * warp] = gt;
+                    wcnt[2 * warp + 1] = eq;
+                }
+                __syncthreads();
+                uint32_t pos = 0, ties = 0;
+                for (int v = 0; v < warp; ++v) {
+                    const uint32_t take = ties < kt ? min(wcnt[2 * v + 1], kt - ties) : 0u;
+                    pos += wcnt[2 * v] + take;
+                    ties += wcnt[2 * v + 1];
+                }
+                const uint32_t lt = (1u << lane) - 1u;
+                for (int j = j0 + lane; j - lane < j1; j += 32) {
+                    const bool valid = j < j1;
+                    const uint32_t key = valid ? ordered_key(fin[j]) : 0u;
+                    const bool is_eq = valid && key == Tk;
+                    const uint32_t beq = __ballot_sync(0xffffffffu, is_eq);
+                    const uint32_t my_tie = ties + __popc(beq & lt);
+                    const bool keep = valid && (key > Tk || (is_eq && my_tie < kt));
+                    const uint32_t bk = __ballot_sync(0xffffffffu, keep);
+                    if (keep) {
+                        const uint32_t r = pos + __popc(bk & lt);
+                        if (r < static_cast<uint32_t>(m)) kidx[r] = j;
+                    }
+                    pos += __popc(bk);
+                    ties += __popc(beq);
+                }
+            }
+        } else {
+            for (int r = tid; r < m; r += S::kThreads) kidx[r] = r;
         }
         __syncthreads();
-    }
 
-    // ---------------- Phase F: gather rows (and the kept list) ----------------
-    if (a.kept) {
-        int32_t* out = a.kept + u * B;
-        for (int r = tid; r < B; r += S::kThreads)
-            out[r] = r < m ? (keep_all ? r : kidx[r]) : -1;
-    }
-    if (tid == 0) a.n_kept[u] = m;
-    {
-        constexpr int kVec = S::kVec;
-        constexpr int kRows = S::kThreads / kVec;  // rows per pass (10 bf16 / 5 f32)
-        constexpr int kUnroll = 8;
-        const int l = tid % kVec;
-        const int rs = tid / kVec;
-        const uint4* ks = static_cast<const uint4*>(a.k_src);
-        const uint4* vs = static_cast<const uint4*>(a.v_src);
-        uint4* kd = static_cast<uint4*>(a.k_dst);
-        uint4* vd = static_cast<uint4*>(a.v_dst);
-        for (int r0 = 0; r0 < m; r0 += kRows * kUnroll) {
-            uint4 kv[kUnroll], vv[kUnroll];
-            int src[kUnroll];
-#pragma unroll
-            for (int q = 0; q < kUnroll; ++q) {
-                const int r = r0 + q * kRows + rs;
-                src[q] = (rs < kRows && r < m) ? (keep_all ? r : kidx[r]) : -1;
-                if (src[q] >= n) {  // cannot happen when the selection is consistent
-                    raise_flag(a.flag, TRI_FLAG_INDEX_RANGE);
-                    src[q] = -1;
+        // ---------------- gather ----------------
+        // Piece boundaries: the start of a run of consecutive source rows, or
+        // a row index that is a multiple of kGRows (no piece exceeds a buffer).
+        {
+            const int seg = ((m + S::kWarps * 32 - 1) / (S::kWarps * 32)) * 32;
+            const int r0 = warp * seg;
+            const int r1 = min(r0 + seg, m);
+            uint32_t cnt = 0;
+            for (int r = r0 + lane; r - lane < r1; r += 32) {
+                bool start = false;
+                if (r < r1) {
+                    const int32_t j = kidx[r];
+                    const int32_t jp = r > 0 ? kidx[r - 1] : -2;
+                    start = (r % S::kGRows == 0) || j != jp + 1;
                 }
-                if (src[q] >= 0) {
-                    const int64_t row = u * a.cap + src[q];
-                    kv[q] = ks[row * kVec + l];
-                    if (vs) vv[q] = vs[row * kVec + l];
-                }
+                cnt += __popc(__ballot_sync(0xffffffffu, start));
             }
-#pragma unroll
-            for (int q = 0; q < kUnroll; ++q) {
-                if (src[q] >= 0) {
-                    const int r = r0 + q * kRows + rs;
-                    const int64_t drow = u * a.cap_dst + r;
-                    kd[drow * kVec + l] = kv[q];
-                    if (vd) vd[drow * kVec + l] = vv[q];
-                    if (a.pos_dst && l == 0) a.pos_dst[drow] = a.pos_src[u * a.cap + src[q]];
+            if (lane == 0) wcnt[2 * warp] = cnt;
+            __syncthreads();
+            uint32_t pos = 0;
+            for (int v = 0; v < warp; ++v) pos += wcnt[2 * v];
+            if (warp == S::kWarps - 1 && lane == 0) *nchunks = static_cast<int>(pos + cnt);
+            const uint32_t lt = (1u << lane) - 1u;
+            for (int r = r0 + lane; r - lane < r1; r += 32) {
+                bool start = false;
+                if (r < r1) {
+                    const int32_t j = kidx[r];
+                    const int32_t jp = r > 0 ? kidx[r - 1] : -2;
+                    start = (r % S::kGRows == 0) || j != jp + 1;
                 }
+                const uint32_t b = __ballot_sync(0xffffffffu, start);
+                if (start) chunk_r[pos + __popc(b & lt)] = r;
+                pos += __popc(b);
             }
         }
+        fence_proxy_async();
+        __syncthreads();
+        const int n_chunks = *nchunks;
+        const int npc = a.v_src ? 2 * n_chunks : n_chunks;  // K (and V) piece per chunk
+        if (tid == S::kMath) {
+            const char* ks = static_cast<const char*>(a.k_src);
+            const char* vs = static_cast<const char*>(a.v_src);
+            char* kd = static_cast<char*>(a.k_dst);
+            char* vd = static_cast<char*>(a.v_dst);
+            auto piece = [&](int p, const char*& src, char*& dst, uint32_t& bytes) {
+                const int c = a.v_src ? (p >> 1) : p;
+                const bool is_v = a.v_src && (p & 1);
+                const int r = chunk_r[c];
+                const int rend = (c + 1 < n_chunks) ? chunk_r[c + 1] : m;
+                int32_t j = kidx[r];
+                bool ok = j >= 0 && j + (rend - r) <= n && rend > r && rend - r <= S::kGRows;
+                if (!ok) {  // cannot happen when the selection is consistent
+                    raise_flag(a.flag, TRI_FLAG_INDEX_RANGE);
+                    j = 0;
+                }
+                const int64_t srow = u * a.cap + j;
+                const int64_t drow = u * a.cap_dst + r;
+                src = (is_v ? vs : ks) + srow * S::kRowBytes;
+                dst = (is_v ? vd : kd) + drow * S::kRowBytes;
+                bytes = ok ? static_cast<uint32_t>((rend - r) * S::kRowBytes) : 0u;
+            };
+            uint8_t* gbuf = regA;
+            int issued = 0;
+            for (; issued < npc && issued < S::kGStages - 1; ++issued) {
+                const char* src;
+                char* dst;
+                uint32_t bytes;
+                piece(issued, src, dst, bytes);
+                const int sb = (pieces_done + issued) % S::kGStages;
+                mbar_arrive_expect_tx(&gfull[sb], bytes);
+                if (bytes) bulk_load(gbuf + sb * S::kGStage, src, bytes, &gfull[sb]);
+            }
+            for (int p = 0; p < npc; ++p) {
+                const uint32_t pc = pieces_done + p;
+                const int sb = pc % S::kGStages;
+                if (!mbar_wait(&gfull[sb], (pc / S::kGStages) & 1, a.flag)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                const char* src;
+                char* dst;
+                uint32_t bytes;
+                piece(p, src, dst, bytes);
+                if (bytes) bulk_store(dst, gbuf + sb * S::kGStage, bytes);
+                bulk_commit();
+                // Every store but the newest has finished reading its buffer,
+                // so the buffer of piece p - 1 can take piece p + kGStages - 1.
+                bulk_wait_read<1>();
+                if (issued < npc) {
+                    piece(issued, src, dst, bytes);
+                    const int sn = (pieces_done + issued) % S::kGStages;
+                    mbar_arrive_expect_tx(&gfull[sn], bytes);
+                    if (bytes) bulk_load(gbuf + sn * S::kGStage, src, bytes, &gfull[sn]);
+                    ++issued;
+                }
+            }
+            bulk_wait_all();
+        } else {
+            // Positions and the kept list.
+            const int nt = S::kThreads - 32;
+            const int t = tid < S::kMath ? tid : tid - 32;
+            for (int r = t; r < m; r += nt) {
+                const int32_t j = kidx[r];
+                if (a.pos_dst && j >= 0 && j < n) a.pos_dst[u * a.cap_dst + r] = a.pos_src[u * a.cap + j];
+            }
+            if (a.kept)
+                for (int r = t; r < B; r += nt) a.kept[u * B + r] = r < m ? kidx[r] : -1;
+            if (t == 0) a.n_kept[u] = m;
+        }
+        tiles_done += n_tiles;
+        pieces_done += npc;
+        fence_proxy_async();
+        __syncthreads();
     }
 }
 
-size_t fused_smem_bytes(tri_dtype dt, int G, int64_t cap) {
-    return dt == TRI_BF16 ? fused_layout<__nv_bfloat16>(G, cap).total
-                          : fused_layout<float>(G, cap).total;
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+size_t fused_smem_bytes(tri_dtype dt, int G, int64_t cap, int64_t B) {
+    return dt == TRI_BF16 ? fused_layout<__nv_bfloat16>(G, cap, B).total
+                          : fused_layout<float>(G, cap, B).total;
 }
 
 size_t fused_smem_limit() {
@@ -345,39 +497,43 @@ size_t fused_smem_limit() {
     return static_cast<size_t>(lim);
 }
 
+int fused_tile_keys(tri_dtype dt) {
+    return dt == TRI_BF16 ? FusedShape<__nv_bfloat16>::kTile : FusedShape<float>::kTile;
+}
+
 template <typename T, int G>
-static cudaError_t launch_fused_t(const CUtensorMap& map, const FusedArgs& a, int64_t n_units,
+static cudaError_t launch_fused_t(const CUtensorMap& map, const FusedArgs& a, int n_ctas,
                                   cudaStream_t s) {
-    const size_t smem = fused_layout<T>(G, a.cap).total;
+    const size_t smem = fused_layout<T>(G, a.cap, a.B).total;
     auto kern = prune_fused_kernel<T, G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<static_cast<unsigned>(n_units), FusedShape<T>::kThreads, smem, s>>>(map, a);
+    kern<<<n_ctas, FusedShape<T>::kThreads, smem, s>>>(map, a);
     note_launch(s);
     return cudaGetLastError();
 }
 
 template <typename T>
-static cudaError_t launch_fused_g(int G, const CUtensorMap& map, const FusedArgs& a,
-                                  int64_t n_units, cudaStream_t s) {
+static cudaError_t launch_fused_g(int G, const CUtensorMap& map, const FusedArgs& a, int n_ctas,
+                                  cudaStream_t s) {
     switch (G) {
-        case 1: return launch_fused_t<T, 1>(map, a, n_units, s);
-        case 2: return launch_fused_t<T, 2>(map, a, n_units, s);
-        case 3: return launch_fused_t<T, 3>(map, a, n_units, s);
-        case 4: return launch_fused_t<T, 4>(map, a, n_units, s);
-        case 5: return launch_fused_t<T, 5>(map, a, n_units, s);
-        case 6: return launch_fused_t<T, 6>(map, a, n_units, s);
-        case 7: return launch_fused_t<T, 7>(map, a, n_units, s);
-        case 8: return launch_fused_t<T, 8>(map, a, n_units, s);
+        case 1: return launch_fused_t<T, 1>(map, a, n_ctas, s);
+        case 2: return launch_fused_t<T, 2>(map, a, n_ctas, s);
+        case 3: return launch_fused_t<T, 3>(map, a, n_ctas, s);
+        case 4: return launch_fused_t<T, 4>(map, a, n_ctas, s);
+        case 5: return launch_fused_t<T, 5>(map, a, n_ctas, s);
+        case 6: return launch_fused_t<T, 6>(map, a, n_ctas, s);
+        case 7: return launch_fused_t<T, 7>(map, a, n_ctas, s);
+        case 8: return launch_fused_t<T, 8>(map, a, n_ctas, s);
     }
     return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_fused(tri_dtype dt, int G, const CUtensorMap& map, const FusedArgs& a,
-                         int64_t n_units, cudaStream_t s) {
-    if (dt == TRI_BF16) return launch_fused_g<__nv_bfloat16>(G, map, a, n_units, s);
-    return launch_fused_g<float>(G, map, a, n_units, s);
+                         int n_ctas, cudaStream_t s) {
+    if (dt == TRI_BF16) return launch_fused_g<__nv_bfloat16>(G, map, a, n_ctas, s);
+    return launch_fused_g<float>(G, map, a, n_ctas, s);
 }
 
 }  // namespace tri

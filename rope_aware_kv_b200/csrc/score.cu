@@ -28,41 +28,66 @@ namespace tri {
 // Fold: per (seq, layer, query head) weights, chunk-major for the score loop.
 // Record layout per query head: 16 chunks x 12 floats; chunk c covers bands
 // 4c..4c+3: [ReA_4c, ImA_4c, ..., ReA_4c+3, ImA_4c+3, c_4c, ..., c_4c+3].
+// One block per (sequence, group of kFoldHeads query heads): the block first
+// forms C_f = mean_delta e^{i w_f delta} (256 threads, each a quarter of the
+// offsets of one band, merged in a fixed order) and e^{i w_f p_cur}, then
+// A_f = E[q_f] e^{i w_f p_cur} C_f for every head of its group, in float64.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(64)
+constexpr int kFoldHeads = 64;
+
+__global__ void __launch_bounds__(256)
 fold_kernel(const float* __restrict__ stats, const int64_t* __restrict__ p_cur, int64_t n_layers,
             int64_t n_qheads, double theta, FoldOffsets off, float* __restrict__ wts) {
-    const int f = threadIdx.x;
-    const int64_t q = blockIdx.x;                    // (seq * L + layer) * Hq + qh
-    const int64_t qh = q % n_qheads;
-    const int64_t layer = (q / n_qheads) % n_layers;
-    const int64_t seq = q / (n_qheads * n_layers);
-    const float* st = stats + ((layer * n_qheads + qh) * kF + f) * 4;
-    const double w = pow(theta, -2.0 * static_cast<double>(f) / static_cast<double>(kD));
-    double cre = 0.0, cim = 0.0;
-    for (int i = 0; i < off.n; ++i) {
-        double s, c;
-        sincos(w * static_cast<double>(off.v[i]), &s, &c);
-        cre += c;
-        cim += s;
+    __shared__ double part[4][kF][2];
+    __shared__ double cf[kF][2], ef[kF][2];
+    const int t = threadIdx.x;
+    const int64_t seq = blockIdx.x;
+    {
+        const int f = t & (kF - 1), q = t >> 6;
+        const double w = pow(theta, -2.0 * static_cast<double>(f) / static_cast<double>(kD));
+        double cre = 0.0, cim = 0.0;
+        for (int i = q; i < off.n; i += 4) {
+            double sn, cs;
+            sincos(w * static_cast<double>(off.v[i]), &sn, &cs);
+            cre += cs;
+            cim += sn;
+        }
+        part[q][f][0] = cre;
+        part[q][f][1] = cim;
+        if (q == 0) {
+            double ps, pc;
+            sincos(w * static_cast<double>(p_cur[seq]), &ps, &pc);
+            ef[f][0] = pc;
+            ef[f][1] = ps;
+        }
     }
-    cre /= off.n;
-    cim /= off.n;
-    double ps, pc;
-    sincos(w * static_cast<double>(p_cur[seq]), &ps, &pc);
-    const double mre = st[0], mim = st[1];
-    // E[q_f] * e^{i w p_cur}
-    const double tre = mre * pc - mim * ps;
-    const double tim = mre * ps + mim * pc;
-    // ... * C_f
-    const double are = tre * cre - tim * cim;
-    const double aim = tre * cim + tim * cre;
-    const double cw = (1.0 - static_cast<double>(st[3])) * static_cast<double>(st[2]);
-    float* rec = wts + q * kWHead + (f >> 2) * kWChunk;
-    const int i = f & 3;
-    rec[2 * i] = static_cast<float>(are);
-    rec[2 * i + 1] = static_cast<float>(aim);
-    rec[8 + i] = static_cast<float>(cw);
+    __syncthreads();
+    if (t < kF) {
+        const double inv = 1.0 / off.n;
+        cf[t][0] = (((part[0][t][0] + part[1][t][0]) + part[2][t][0]) + part[3][t][0]) * inv;
+        cf[t][1] = (((part[0][t][1] + part[1][t][1]) + part[2][t][1]) + part[3][t][1]) * inv;
+    }
+    __syncthreads();
+    const int64_t LH = n_layers * n_qheads;
+    const int64_t h0 = static_cast<int64_t>(blockIdx.y) * kFoldHeads;
+    const int64_t h1 = h0 + kFoldHeads < LH ? h0 + kFoldHeads : LH;
+    for (int64_t e = h0 * kF + t; e < h1 * kF; e += blockDim.x) {
+        const int64_t lh = e / kF;  // layer * Hq + qh
+        const int f = static_cast<int>(e % kF);
+        const float* st = stats + (lh * kF + f) * 4;
+        const double mre = st[0], mim = st[1];
+        const double tre = mre * ef[f][0] - mim * ef[f][1];  // E[q_f] e^{i w p_cur}
+        const double tim = mre * ef[f][1] + mim * ef[f][0];
+        const double are = tre * cf[f][0] - tim * cf[f][1];  // ... * C_f
+        const double aim = tre * cf[f][1] + tim * cf[f][0];
+        const double cw = (1.0 - static_cast<double>(st[3])) * static_cast<double>(st[2]);
+        const int64_t q = seq * LH + lh;  // (seq * L + layer) * Hq + qh
+        float* rec = wts + q * kWHead + (f >> 2) * kWChunk;
+        const int i = f & 3;
+        rec[2 * i] = static_cast<float>(are);
+        rec[2 * i + 1] = static_cast<float>(aim);
+        rec[8 + i] = static_cast<float>(cw);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -212,7 +237,7 @@ score_kernel(const __grid_constant__ CUtensorMap kmap, ScoreArgs a) {
             }
             if (!mbar_wait(&sm.full[stage], phase, a.flag)) break;
             float s[S::kKPT][G];
-            score_rows<T, G, S::kKPT, S::kBoxBytes>(sm.tiles[stage], sm.w, tid, s);
+            score_rows<T, G, S::kKPT, S::kBoxBytes, 128>(sm.tiles[stage], sm.w, tid, s);
             mbar_arrive(&sm.empty[stage]);
             if (++stage == S::kStages) {
                 stage = 0;
@@ -371,9 +396,9 @@ int score_tile_keys(tri_dtype dt) {
 cudaError_t launch_fold(const float* stats, const int64_t* p_cur, int64_t n_seq, int64_t n_layers,
                         int64_t n_qheads, double theta, const FoldOffsets& off, float* wts,
                         cudaStream_t s) {
-    const int64_t blocks = n_seq * n_layers * n_qheads;
-    fold_kernel<<<static_cast<unsigned>(blocks), 64, 0, s>>>(stats, p_cur, n_layers, n_qheads,
-                                                             theta, off, wts);
+    const int64_t groups = (n_layers * n_qheads + kFoldHeads - 1) / kFoldHeads;
+    dim3 grid(static_cast<unsigned>(n_seq), static_cast<unsigned>(groups));
+    fold_kernel<<<grid, 256, 0, s>>>(stats, p_cur, n_layers, n_qheads, theta, off, wts);
     note_launch(s);
     return cudaGetLastError();
 }

@@ -16,8 +16,10 @@ namespace tri {
 // lives at b * kBoxBytes + r * 128 and its 16-byte chunk j at position
 // (j ^ (r & 7)) (TMA 128-byte swizzle), so 8 consecutive threads reading the
 // same logical chunk of 8 consecutive rows hit 8 different bank groups.
-template <typename T, int G, int KPT, int kBoxBytes>
-__device__ __forceinline__ void score_rows(const uint8_t* tile, const float* w, int tid,
+// Rows first_row + kRowStride * k (k < KPT) of the tile; w points at the
+// weight record of the first of the G heads scored here.
+template <typename T, int G, int KPT, int kBoxBytes, int kRowStride>
+__device__ __forceinline__ void score_rows(const uint8_t* tile, const float* w, int first_row,
                                            float (&s)[KPT][G]) {
     float2 acc[KPT][G];
 #pragma unroll
@@ -32,7 +34,7 @@ __device__ __forceinline__ void score_rows(const uint8_t* tile, const float* w, 
             float2 nn[KPT][2];
 #pragma unroll
             for (int k = 0; k < KPT; ++k) {
-                const int r = tid + 128 * k;
+                const int r = first_row + kRowStride * k;
                 const uint4 v = *reinterpret_cast<const uint4*>(
                     tile + (c >> 3) * kBoxBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
                 const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
@@ -71,7 +73,7 @@ __device__ __forceinline__ void score_rows(const uint8_t* tile, const float* w, 
             float2 nn[KPT];
 #pragma unroll
             for (int k = 0; k < KPT; ++k) {
-                const int r = tid + 128 * k;
+                const int r = first_row + kRowStride * k;
                 const float4 v = *reinterpret_cast<const float4*>(
                     tile + (c >> 3) * kBoxBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
                 xy[k][0] = make_float2(v.x, v.y);

@@ -33,6 +33,7 @@ struct ScoreArgs {
 };
 
 struct FusedArgs {
+    int64_t n_units;
     int64_t cap;
     int64_t cap_dst;
     int64_t B;
@@ -46,6 +47,7 @@ struct FusedArgs {
     int32_t* pos_dst;
     int32_t* kept;               // [U][B] or null
     int32_t* n_kept;             // [U]
+    float* scratch;              // [grid][G][cap] per-CTA score scratch
     uint32_t* flag;
 };
 
@@ -89,9 +91,10 @@ cudaError_t launch_append(tri_dtype dt, void* k_cache, void* v_cache, int32_t* p
                           const int32_t* pos_new, int64_t n_new, uint32_t* flag, cudaStream_t s);
 
 // fused.cu
-size_t fused_smem_bytes(tri_dtype dt, int G, int64_t cap);
+size_t fused_smem_bytes(tri_dtype dt, int G, int64_t cap, int64_t B);
 size_t fused_smem_limit();
+int fused_tile_keys(tri_dtype dt);
 cudaError_t launch_fused(tri_dtype dt, int G, const CUtensorMap& map, const FusedArgs& a,
-                         int64_t n_units, cudaStream_t s);
+                         int n_ctas, cudaStream_t s);
 
 }  // namespace tri

@@ -45,9 +45,11 @@ struct FusedShape {
     static constexpr int kMath = 128;
     static constexpr int kThreads = kMath + 32;
     static constexpr int kWarps = kThreads / 32;
-    static constexpr int kGStage = 16384;                               // gather piece buffer
-    static constexpr int kGStages = kRegionA / kGStage;                 // 8
+    static constexpr int kGStage = 8192;                                // gather piece buffer
+    static constexpr int kGStages = kRegionA / kGStage;                 // 16
+    static constexpr int kGLead = kGStages / 2;                         // loads issued ahead
     static constexpr int kGRows = kGStage / kRowBytes;                  // rows per piece
+    static constexpr int kMinBulkRows = 4;  // shorter runs are copied by threads
 };
 
 struct FusedLayout {
@@ -402,68 +404,97 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
         __syncthreads();
         const int n_chunks = *nchunks;
         const int npc = a.v_src ? 2 * n_chunks : n_chunks;  // K (and V) piece per chunk
+        // Piece p: chunk p / 2 (p with V), rows [chunk_r[c], chunk_r[c + 1]).
+        auto chunk_rows = [&](int c, int& r, int& len, int32_t& j) -> bool {
+            r = chunk_r[c];
+            const int rend = (c + 1 < n_chunks) ? chunk_r[c + 1] : m;
+            len = rend - r;
+            j = kidx[r];
+            return j >= 0 && j + len <= n && len > 0 && len <= S::kGRows;
+        };
         if (tid == S::kMath) {
+            // Bulk-copy engine for pieces of at least kMinBulkRows rows: loads
+            // run kGLead pieces ahead of stores; a buffer is refilled once the
+            // store that read it kGLead pieces earlier has finished reading.
             const char* ks = static_cast<const char*>(a.k_src);
             const char* vs = static_cast<const char*>(a.v_src);
             char* kd = static_cast<char*>(a.k_dst);
             char* vd = static_cast<char*>(a.v_dst);
-            auto piece = [&](int p, const char*& src, char*& dst, uint32_t& bytes) {
-                const int c = a.v_src ? (p >> 1) : p;
-                const bool is_v = a.v_src && (p & 1);
-                const int r = chunk_r[c];
-                const int rend = (c + 1 < n_chunks) ? chunk_r[c + 1] : m;
-                int32_t j = kidx[r];
-                bool ok = j >= 0 && j + (rend - r) <= n && rend > r && rend - r <= S::kGRows;
-                if (!ok) {  // cannot happen when the selection is consistent
-                    raise_flag(a.flag, TRI_FLAG_INDEX_RANGE);
-                    j = 0;
-                }
-                const int64_t srow = u * a.cap + j;
-                const int64_t drow = u * a.cap_dst + r;
-                src = (is_v ? vs : ks) + srow * S::kRowBytes;
-                dst = (is_v ? vd : kd) + drow * S::kRowBytes;
-                bytes = ok ? static_cast<uint32_t>((rend - r) * S::kRowBytes) : 0u;
-            };
             uint8_t* gbuf = regA;
-            int issued = 0;
-            for (; issued < npc && issued < S::kGStages - 1; ++issued) {
-                const char* src;
-                char* dst;
-                uint32_t bytes;
-                piece(issued, src, dst, bytes);
-                const int sb = (pieces_done + issued) % S::kGStages;
-                mbar_arrive_expect_tx(&gfull[sb], bytes);
-                if (bytes) bulk_load(gbuf + sb * S::kGStage, src, bytes, &gfull[sb]);
-            }
-            for (int p = 0; p < npc; ++p) {
-                const uint32_t pc = pieces_done + p;
+            uint32_t ld = 0, stq = 0;  // bulk pieces loaded / stored in this unit
+            int pl = 0;                // next piece index to consider for loading
+            auto next_load = [&]() {
+                for (; pl < npc; ++pl) {
+                    const int c = a.v_src ? (pl >> 1) : pl;
+                    const bool is_v = a.v_src && (pl & 1);
+                    int r, len;
+                    int32_t j;
+                    const bool ok = chunk_rows(c, r, len, j);
+                    if (!ok) {  // cannot happen when the selection is consistent
+                        if (len > 0) raise_flag(a.flag, TRI_FLAG_INDEX_RANGE);
+                        continue;
+                    }
+                    if (len < S::kMinBulkRows) continue;
+                    const uint32_t pc = pieces_done + ld;
+                    const int sb = pc % S::kGStages;
+                    const uint32_t bytes = static_cast<uint32_t>(len * S::kRowBytes);
+                    mbar_arrive_expect_tx(&gfull[sb], bytes);
+                    bulk_load(gbuf + sb * S::kGStage,
+                              (is_v ? vs : ks) + (u * a.cap + j) * S::kRowBytes, bytes, &gfull[sb]);
+                    ++ld;
+                    ++pl;
+                    return;
+                }
+            };
+            for (int q = 0; q < S::kGLead; ++q) next_load();
+            int ps = 0;  // next piece index to consider for storing
+            for (; ps < npc; ++ps) {
+                const int c = a.v_src ? (ps >> 1) : ps;
+                const bool is_v = a.v_src && (ps & 1);
+                int r, len;
+                int32_t j;
+                if (!chunk_rows(c, r, len, j) || len < S::kMinBulkRows) continue;
+                const uint32_t pc = pieces_done + stq;
                 const int sb = pc % S::kGStages;
                 if (!mbar_wait(&gfull[sb], (pc / S::kGStages) & 1, a.flag)) {
                     *abort_flag = 1;
                     break;
                 }
-                const char* src;
-                char* dst;
-                uint32_t bytes;
-                piece(p, src, dst, bytes);
-                if (bytes) bulk_store(dst, gbuf + sb * S::kGStage, bytes);
+                bulk_store((is_v ? vd : kd) + (u * a.cap_dst + r) * S::kRowBytes,
+                           gbuf + sb * S::kGStage, static_cast<uint32_t>(len * S::kRowBytes));
                 bulk_commit();
-                // Every store but the newest has finished reading its buffer,
-                // so the buffer of piece p - 1 can take piece p + kGStages - 1.
-                bulk_wait_read<1>();
-                if (issued < npc) {
-                    piece(issued, src, dst, bytes);
-                    const int sn = (pieces_done + issued) % S::kGStages;
-                    mbar_arrive_expect_tx(&gfull[sn], bytes);
-                    if (bytes) bulk_load(gbuf + sn * S::kGStage, src, bytes, &gfull[sn]);
-                    ++issued;
-                }
+                ++stq;
+                // Stores up to stq - kGLead have read their buffers; the next
+                // load reuses the buffer of store stq - kGLead.
+                bulk_wait_read<S::kGLead - 1>();
+                next_load();
             }
             bulk_wait_all();
+            nchunks[2] = static_cast<int32_t>(ld);  // ring advance, read by all threads
         } else {
-            // Positions and the kept list.
+            // Short runs of K / V rows (vector copies), positions, kept list.
             const int nt = S::kThreads - 32;
             const int t = tid < S::kMath ? tid : tid - 32;
+            constexpr int kVec = S::kRowBytes / 16;
+            const uint4* ks = static_cast<const uint4*>(a.k_src);
+            const uint4* vs = static_cast<const uint4*>(a.v_src);
+            uint4* kd = static_cast<uint4*>(a.k_dst);
+            uint4* vd = static_cast<uint4*>(a.v_dst);
+            for (int c = t / kVec; c < n_chunks; c += nt / kVec) {
+                int r, len;
+                int32_t j;
+                if (!chunk_rows(c, r, len, j) || len >= S::kMinBulkRows) continue;
+                const int l = t % kVec;
+                for (int q = 0; q < len; ++q) {
+                    const int64_t srow = u * a.cap + j + q;
+                    const int64_t drow = u * a.cap_dst + r + q;
+                    const uint4 kv = ks[srow * kVec + l];
+                    uint4 vv;
+                    if (vs) vv = vs[srow * kVec + l];
+                    kd[drow * kVec + l] = kv;
+                    if (vd) vd[drow * kVec + l] = vv;
+                }
+            }
             for (int r = t; r < m; r += nt) {
                 const int32_t j = kidx[r];
                 if (a.pos_dst && j >= 0 && j < n) a.pos_dst[u * a.cap_dst + r] = a.pos_src[u * a.cap + j];
@@ -472,8 +503,9 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
                 for (int r = t; r < B; r += nt) a.kept[u * B + r] = r < m ? kidx[r] : -1;
             if (t == 0) a.n_kept[u] = m;
         }
+        __syncthreads();
         tiles_done += n_tiles;
-        pieces_done += npc;
+        pieces_done += static_cast<uint32_t>(nchunks[2]);
         fence_proxy_async();
         __syncthreads();
     }

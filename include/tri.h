@@ -277,6 +277,18 @@ tri_status tri_set_timing_events(void* const* events, int n_events);
  * (memsets are not counted). */
 int tri_last_launch_count(void);
 
+/*
+ * Phase tracing for the calling host thread.  When device_buf (device
+ * memory, caller-owned, at least n_units * 512 bytes) is set, the fused
+ * kernel of tri_prune writes %globaltimer nanoseconds into
+ * device_buf[(u * 8 + p) * 8 + w] (uint64): lane 0 of warp w records phase
+ * point p of unit u just before the barrier that ends the phase, so a phase
+ * ends at the largest w entry.  p = 0: start of the unit; 1: scored;
+ * 2: z-max done; 3: selected; 4: gathered.  Units a call does not reach
+ * through the fused kernel are left untouched.  Pass (NULL, 0) to stop.
+ */
+tri_status tri_set_phase_trace(void* device_buf, size_t bytes);
+
 /* ---------------------------------------------------------------------- */
 /* Device-side error flag                                                  */
 /* ---------------------------------------------------------------------- */

@@ -52,7 +52,7 @@ EXPORTS = (
     "tri_compact_workspace_bytes", "tri_compact",
     "tri_prune_workspace_bytes", "tri_prune",
     "tri_append", "tri_check_device_error",
-    "tri_set_timing_events", "tri_last_launch_count",
+    "tri_set_timing_events", "tri_last_launch_count", "tri_set_phase_trace",
 )
 
 
@@ -106,6 +106,7 @@ def load(path: Optional[str] = None):
         "tri_check_device_error": (i32, [P, P, u32p]),
         "tri_set_timing_events": (i32, [ctypes.POINTER(ctypes.c_void_p), i32]),
         "tri_last_launch_count": (i32, []),
+        "tri_set_phase_trace": (i32, [P, sz]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -298,6 +299,15 @@ def tri_set_timing_events(events: Optional[Sequence["torch.cuda.Event"]]):
     arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
     _timing_keep = (arr, list(events))
     _check("tri_set_timing_events", load().tri_set_timing_events(arr, len(events)))
+
+
+def tri_set_phase_trace(buf: Optional[torch.Tensor]):
+    """Per-unit phase timestamps of the fused kernel into buf (int64 CUDA
+    tensor of at least 8 * units entries), or None to stop."""
+    if buf is None:
+        _check("tri_set_phase_trace", load().tri_set_phase_trace(None, 0))
+    else:
+        _check("tri_set_phase_trace", load().tri_set_phase_trace(_ptr(buf), buf.numel() * buf.element_size()))
 
 
 def tri_last_launch_count() -> int:

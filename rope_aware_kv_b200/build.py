@@ -48,8 +48,11 @@ def _stale() -> bool:
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False, jobs: int = 8) -> str:
-    if not force and not _stale():
+def build(force: bool = False, verbose: bool = False, jobs: int = 8, out: str = LIB,
+          defines=()) -> str:
+    """Compile the library to ``out`` (default: the in-tree libtri.so); extra
+    ``-D`` defines select compile-time variants of the kernels."""
+    if out == LIB and not defines and not force and not _stale():
         return LIB
     nvcc = _nvcc()
     tmp = tempfile.mkdtemp(prefix="tri_build_")
@@ -58,7 +61,8 @@ def build(force: bool = False, verbose: bool = False, jobs: int = 8) -> str:
         procs = []
         for src in sources():
             obj = os.path.join(tmp, os.path.basename(src) + ".o")
-            cmd = [nvcc, *ARCH, *FLAGS, "-I", INCLUDE, "-c", src, "-o", obj]
+            cmd = [nvcc, *ARCH, *FLAGS, *[f"-D{d}" for d in defines], "-I", INCLUDE, "-c", src,
+                   "-o", obj]
             if verbose:
                 cmd += ["-Xptxas", "-v"]
             procs.append((src, subprocess.Popen(cmd, stdout=subprocess.PIPE,
@@ -67,12 +71,12 @@ def build(force: bool = False, verbose: bool = False, jobs: int = 8) -> str:
             if len(procs) >= jobs:
                 _drain(procs, verbose)
         _drain(procs, verbose)
-        out = LIB + ".tmp"
-        subprocess.run([nvcc, *ARCH, "-shared", "-o", out, *objs], check=True)
-        os.replace(out, LIB)
+        tmp_out = out + ".tmp"
+        subprocess.run([nvcc, *ARCH, "-shared", "-o", tmp_out, *objs], check=True)
+        os.replace(tmp_out, out)
     finally:
         shutil.rmtree(tmp, ignore_errors=True)
-    return LIB
+    return out
 
 
 def _drain(procs, verbose):

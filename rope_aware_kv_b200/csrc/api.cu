@@ -21,6 +21,17 @@ thread_local int t_n_events = 0;
 thread_local int t_launches = 0;
 }  // namespace
 
+namespace {
+thread_local uint64_t* t_trace = nullptr;
+thread_local size_t t_trace_bytes = 0;
+}  // namespace
+
+uint64_t* tri::phase_trace_buffer(int64_t n_units) {
+    if (!t_trace || t_trace_bytes < static_cast<size_t>(n_units) * kTracePoints * kTraceWarps * 8)
+        return nullptr;
+    return t_trace;
+}
+
 void tri::note_launch(cudaStream_t s) {
     if (t_events && t_launches < t_n_events) {
         // Under stream capture a plain record only marks a dependency; an
@@ -470,6 +481,7 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
         a.kept = kept_idx;
         a.n_kept = n_kept;
         a.scratch = reinterpret_cast<float*>(ws_at(ws, w.sc.raw));
+        a.trace = phase_trace_buffer(U);
         a.flag = flag;
         return cuda_status(launch_fused(dt, G, map, a, static_cast<int>(fused_ctas(U)), s));
     }
@@ -538,6 +550,13 @@ tri_status tri_set_timing_events(void* const* events, int n_events) {
 }
 
 int tri_last_launch_count(void) { return t_launches; }
+
+tri_status tri_set_phase_trace(void* device_buf, size_t bytes) {
+    if (bytes && !device_buf) return TRI_ERR_INVALID_ARG;
+    t_trace = static_cast<uint64_t*>(device_buf);
+    t_trace_bytes = device_buf ? bytes : 0;
+    return TRI_OK;
+}
 
 tri_status tri_check_device_error(const void* ws, void* stream, uint32_t* flags_out) {
     if (!ws) return TRI_ERR_INVALID_ARG;

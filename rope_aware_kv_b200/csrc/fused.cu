@@ -19,10 +19,9 @@
 //           first radix digit histogram.
 //   select  two more radix digits on shared-memory histograms, then the
 //           ordered compaction of kept indices (warp ballots).
-//   gather  kept rows form runs of consecutive indices; one lane moves each
-//           run piece (<= 16 KB) of K and of V with cp.async.bulk through an
-//           8-stage shared-memory ring (global -> shared -> global), keeping
-//           up to 7 pieces in flight; the other lanes copy positions.
+//   gather  every thread copies 16-byte pieces of kept K and V rows with
+//           deep memory-level parallelism (loads of 16 rows in flight before
+//           their stores), plus positions and the kept list.
 // HBM traffic per unit is the compulsory bytes plus the re-read of kept K
 // rows (often from L2).
 #include "select_core.cuh"
@@ -45,11 +44,7 @@ struct FusedShape {
     static constexpr int kMath = 128;
     static constexpr int kThreads = kMath + 32;
     static constexpr int kWarps = kThreads / 32;
-    static constexpr int kGStage = 8192;                                // gather piece buffer
-    static constexpr int kGStages = kRegionA / kGStage;                 // 16
-    static constexpr int kGLead = kGStages / 2;                         // loads issued ahead
-    static constexpr int kGRows = kGStage / kRowBytes;                  // rows per piece
-    static constexpr int kMinBulkRows = 4;  // shorter runs are copied by threads
+    static constexpr int kGatherBatch = sizeof(T) == 2 ? 16 : 8;        // rows per thread per batch
 };
 
 struct FusedLayout {
@@ -66,7 +61,7 @@ __host__ __device__ inline FusedLayout fused_layout(int G, int64_t cap, int64_t 
     L.fin = L.w + static_cast<size_t>(G) * kWHead * 4;
     L.kidx = L.fin + static_cast<size_t>(capP) * 4;
     L.bars = L.kidx + ((static_cast<size_t>(m) * 4 + 15) & ~size_t(15));
-    L.red = L.bars + (2 * S::kStages + S::kGStages) * 8;
+    L.red = L.bars + (2 * S::kStages) * 8;
     L.misc = L.red + static_cast<size_t>(4) * kMaxG * 2 * 8;
     L.total = L.misc + 256 + 1024;  // state and warp counts; alignment slack
     return L;
@@ -78,6 +73,14 @@ struct HeadSplit {
     static constexpr int kA = (G + 1) / 2;
     static constexpr int kB = G - kA;
 };
+
+// Phase trace: lane 0 of every warp records %globaltimer just before the
+// barrier that ends phase i of unit u (the phase ends at the latest warp);
+// slot i = 0 marks the start of the unit.
+__device__ __forceinline__ void trace_point(const FusedArgs& a, int64_t u, int i) {
+    if (a.trace && (threadIdx.x & 31) == 0)
+        a.trace[(u * kTracePoints + i) * kTraceWarps + (threadIdx.x >> 5)] = globaltimer_ns();
+}
 
 template <typename T, int G>
 __global__ void __launch_bounds__(FusedShape<T>::kThreads, 1)
@@ -95,15 +98,12 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
     int32_t* kidx = reinterpret_cast<int32_t*>(base + L.kidx);
     uint64_t* full = reinterpret_cast<uint64_t*>(base + L.bars);
     uint64_t* empty = full + S::kStages;
-    uint64_t* gfull = empty + S::kStages;
     double* red = reinterpret_cast<double*>(base + L.red);  // [4 warps][kMaxG][2]
     SelState* st = reinterpret_cast<SelState*>(base + L.misc);
     float2* mom = reinterpret_cast<float2*>(base + L.misc + 16);            // [kMaxG]
     uint32_t* wcnt = reinterpret_cast<uint32_t*>(base + L.misc + 16 + 64);  // [kWarps][2]
-    int32_t* nchunks = reinterpret_cast<int32_t*>(base + L.misc + 16 + 64 + 48);
-    int32_t* abort_flag = nchunks + 1;
+    int32_t* abort_flag = reinterpret_cast<int32_t*>(base + L.misc + 16 + 64 + 48);
     uint32_t* hist = reinterpret_cast<uint32_t*>(regA);  // between scoring and gathering
-    int32_t* chunk_r = reinterpret_cast<int32_t*>(fin);  // after the compaction
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -115,7 +115,6 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], 64);
         }
-        for (int i = 0; i < S::kGStages; ++i) mbar_init(&gfull[i], 1);
         fence_barrier_init();
         prefetch_tensormap(&kmap);
         *abort_flag = 0;
@@ -123,7 +122,6 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
     __syncthreads();
 
     uint32_t tiles_done = 0;   // running tile count (TMA ring position) of this CTA
-    uint32_t pieces_done = 0;  // running gather-piece count (gather ring position)
 
     for (int64_t u = blockIdx.x; u < a.n_units; u += gridDim.x) {
         if (*abort_flag) break;  // a bounded wait gave up: stop cleanly
@@ -131,6 +129,7 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
         const int m = static_cast<int>(n < B ? n : B);
         const bool keep_all = n <= B;
         const int n_tiles = keep_all ? 0 : (n + S::kTile - 1) / S::kTile;
+        trace_point(a, u, 0);
 
         if (!keep_all) {
             // ---------------- score ----------------
@@ -225,6 +224,7 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
                     }
                 }
             }
+            trace_point(a, u, 1);
             __syncthreads();
             if (*abort_flag) break;
             // ---------------- moments (fixed order: pair 0 then pair 1) ----------------
@@ -283,6 +283,7 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
                 }
                 if (nonfinite) raise_flag(a.flag, TRI_FLAG_NONFINITE);
             }
+            trace_point(a, u, 2);
             __syncthreads();
             // ---------------- radix passes 1 and 2 ----------------
             if (warp == 0) {
@@ -363,149 +364,65 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
         } else {
             for (int r = tid; r < m; r += S::kThreads) kidx[r] = r;
         }
+        trace_point(a, u, 3);
         __syncthreads();
 
         // ---------------- gather ----------------
-        // Piece boundaries: the start of a run of consecutive source rows, or
-        // a row index that is a multiple of kGRows (no piece exceeds a buffer).
+        // Every thread moves 16-byte pieces of kept rows: kGRowsPerThread rows
+        // of K and of V in flight per thread (loads first, then stores), so
+        // about 80 KB of loads are in flight per SM; a store frees its
+        // registers at once, so only the load latency limits the rate.
         {
-            const int seg = ((m + S::kWarps * 32 - 1) / (S::kWarps * 32)) * 32;
-            const int r0 = warp * seg;
-            const int r1 = min(r0 + seg, m);
-            uint32_t cnt = 0;
-            for (int r = r0 + lane; r - lane < r1; r += 32) {
-                bool start = false;
-                if (r < r1) {
-                    const int32_t j = kidx[r];
-                    const int32_t jp = r > 0 ? kidx[r - 1] : -2;
-                    start = (r % S::kGRows == 0) || j != jp + 1;
-                }
-                cnt += __popc(__ballot_sync(0xffffffffu, start));
-            }
-            if (lane == 0) wcnt[2 * warp] = cnt;
-            __syncthreads();
-            uint32_t pos = 0;
-            for (int v = 0; v < warp; ++v) pos += wcnt[2 * v];
-            if (warp == S::kWarps - 1 && lane == 0) *nchunks = static_cast<int>(pos + cnt);
-            const uint32_t lt = (1u << lane) - 1u;
-            for (int r = r0 + lane; r - lane < r1; r += 32) {
-                bool start = false;
-                if (r < r1) {
-                    const int32_t j = kidx[r];
-                    const int32_t jp = r > 0 ? kidx[r - 1] : -2;
-                    start = (r % S::kGRows == 0) || j != jp + 1;
-                }
-                const uint32_t b = __ballot_sync(0xffffffffu, start);
-                if (start) chunk_r[pos + __popc(b & lt)] = r;
-                pos += __popc(b);
-            }
-        }
-        fence_proxy_async();
-        __syncthreads();
-        const int n_chunks = *nchunks;
-        const int npc = a.v_src ? 2 * n_chunks : n_chunks;  // K (and V) piece per chunk
-        // Piece p: chunk p / 2 (p with V), rows [chunk_r[c], chunk_r[c + 1]).
-        auto chunk_rows = [&](int c, int& r, int& len, int32_t& j) -> bool {
-            r = chunk_r[c];
-            const int rend = (c + 1 < n_chunks) ? chunk_r[c + 1] : m;
-            len = rend - r;
-            j = kidx[r];
-            return j >= 0 && j + len <= n && len > 0 && len <= S::kGRows;
-        };
-        if (tid == S::kMath) {
-            // Bulk-copy engine for pieces of at least kMinBulkRows rows: loads
-            // run kGLead pieces ahead of stores; a buffer is refilled once the
-            // store that read it kGLead pieces earlier has finished reading.
-            const char* ks = static_cast<const char*>(a.k_src);
-            const char* vs = static_cast<const char*>(a.v_src);
-            char* kd = static_cast<char*>(a.k_dst);
-            char* vd = static_cast<char*>(a.v_dst);
-            uint8_t* gbuf = regA;
-            uint32_t ld = 0, stq = 0;  // bulk pieces loaded / stored in this unit
-            int pl = 0;                // next piece index to consider for loading
-            auto next_load = [&]() {
-                for (; pl < npc; ++pl) {
-                    const int c = a.v_src ? (pl >> 1) : pl;
-                    const bool is_v = a.v_src && (pl & 1);
-                    int r, len;
-                    int32_t j;
-                    const bool ok = chunk_rows(c, r, len, j);
-                    if (!ok) {  // cannot happen when the selection is consistent
-                        if (len > 0) raise_flag(a.flag, TRI_FLAG_INDEX_RANGE);
-                        continue;
-                    }
-                    if (len < S::kMinBulkRows) continue;
-                    const uint32_t pc = pieces_done + ld;
-                    const int sb = pc % S::kGStages;
-                    const uint32_t bytes = static_cast<uint32_t>(len * S::kRowBytes);
-                    mbar_arrive_expect_tx(&gfull[sb], bytes);
-                    bulk_load(gbuf + sb * S::kGStage,
-                              (is_v ? vs : ks) + (u * a.cap + j) * S::kRowBytes, bytes, &gfull[sb]);
-                    ++ld;
-                    ++pl;
-                    return;
-                }
-            };
-            for (int q = 0; q < S::kGLead; ++q) next_load();
-            int ps = 0;  // next piece index to consider for storing
-            for (; ps < npc; ++ps) {
-                const int c = a.v_src ? (ps >> 1) : ps;
-                const bool is_v = a.v_src && (ps & 1);
-                int r, len;
-                int32_t j;
-                if (!chunk_rows(c, r, len, j) || len < S::kMinBulkRows) continue;
-                const uint32_t pc = pieces_done + stq;
-                const int sb = pc % S::kGStages;
-                if (!mbar_wait(&gfull[sb], (pc / S::kGStages) & 1, a.flag)) {
-                    *abort_flag = 1;
-                    break;
-                }
-                bulk_store((is_v ? vd : kd) + (u * a.cap_dst + r) * S::kRowBytes,
-                           gbuf + sb * S::kGStage, static_cast<uint32_t>(len * S::kRowBytes));
-                bulk_commit();
-                ++stq;
-                // Stores up to stq - kGLead have read their buffers; the next
-                // load reuses the buffer of store stq - kGLead.
-                bulk_wait_read<S::kGLead - 1>();
-                next_load();
-            }
-            bulk_wait_all();
-            nchunks[2] = static_cast<int32_t>(ld);  // ring advance, read by all threads
-        } else {
-            // Short runs of K / V rows (vector copies), positions, kept list.
-            const int nt = S::kThreads - 32;
-            const int t = tid < S::kMath ? tid : tid - 32;
             constexpr int kVec = S::kRowBytes / 16;
+            constexpr int kGroups = S::kThreads / kVec;  // rows per pass
+            constexpr int kBatch = S::kGatherBatch;
+            const int l = tid % kVec;
+            const int g = tid / kVec;
             const uint4* ks = static_cast<const uint4*>(a.k_src);
             const uint4* vs = static_cast<const uint4*>(a.v_src);
             uint4* kd = static_cast<uint4*>(a.k_dst);
             uint4* vd = static_cast<uint4*>(a.v_dst);
-            for (int c = t / kVec; c < n_chunks; c += nt / kVec) {
-                int r, len;
-                int32_t j;
-                if (!chunk_rows(c, r, len, j) || len >= S::kMinBulkRows) continue;
-                const int l = t % kVec;
-                for (int q = 0; q < len; ++q) {
-                    const int64_t srow = u * a.cap + j + q;
-                    const int64_t drow = u * a.cap_dst + r + q;
-                    const uint4 kv = ks[srow * kVec + l];
-                    uint4 vv;
-                    if (vs) vv = vs[srow * kVec + l];
-                    kd[drow * kVec + l] = kv;
-                    if (vd) vd[drow * kVec + l] = vv;
+            if (g < kGroups) {
+                for (int r0 = 0; r0 < m; r0 += kGroups * kBatch) {
+                    uint4 kv[kBatch], vv[kBatch];
+                    int32_t jj[kBatch];
+#pragma unroll
+                    for (int q = 0; q < kBatch; ++q) {
+                        const int r = r0 + q * kGroups + g;
+                        int32_t j = r < m ? kidx[r] : -1;
+                        if (j >= n) {  // cannot happen when the selection is consistent
+                            raise_flag(a.flag, TRI_FLAG_INDEX_RANGE);
+                            j = -1;
+                        }
+                        jj[q] = j;
+                    }
+#pragma unroll
+                    for (int q = 0; q < kBatch; ++q) {
+                        if (jj[q] >= 0) {
+                            const int64_t srow = u * a.cap + jj[q];
+                            kv[q] = ld_stream(ks + srow * kVec + l);
+                            if (vs) vv[q] = ld_stream(vs + srow * kVec + l);
+                        }
+                    }
+#pragma unroll
+                    for (int q = 0; q < kBatch; ++q) {
+                        if (jj[q] >= 0) {
+                            const int r = r0 + q * kGroups + g;
+                            const int64_t drow = u * a.cap_dst + r;
+                            st_stream(kd + drow * kVec + l, kv[q]);
+                            if (vd) st_stream(vd + drow * kVec + l, vv[q]);
+                            if (a.pos_dst && l == 0) a.pos_dst[drow] = a.pos_src[u * a.cap + jj[q]];
+                        }
+                    }
                 }
             }
-            for (int r = t; r < m; r += nt) {
-                const int32_t j = kidx[r];
-                if (a.pos_dst && j >= 0 && j < n) a.pos_dst[u * a.cap_dst + r] = a.pos_src[u * a.cap + j];
-            }
             if (a.kept)
-                for (int r = t; r < B; r += nt) a.kept[u * B + r] = r < m ? kidx[r] : -1;
-            if (t == 0) a.n_kept[u] = m;
+                for (int r = tid; r < B; r += S::kThreads) a.kept[u * B + r] = r < m ? kidx[r] : -1;
+            if (tid == 0) a.n_kept[u] = m;
         }
+        trace_point(a, u, 4);
         __syncthreads();
         tiles_done += n_tiles;
-        pieces_done += static_cast<uint32_t>(nchunks[2]);
         fence_proxy_async();
         __syncthreads();
     }

@@ -10,7 +10,15 @@
 
 #include "tri_internal.cuh"
 
+// Unroll factor of the 16-chunk loop: full unrolling lets the compiler hoist
+// shared-memory loads, partial unrolling keeps the instruction footprint small.
+#ifndef TRI_SCORE_UNROLL
+#define TRI_SCORE_UNROLL 4
+#endif
+
 namespace tri {
+
+constexpr int kScoreUnroll = TRI_SCORE_UNROLL;
 
 // Score KPT keys of a tile held in swizzled shared memory.  Row r of box b
 // lives at b * kBoxBytes + r * 128 and its 16-byte chunk j at position
@@ -28,7 +36,7 @@ __device__ __forceinline__ void score_rows(const uint8_t* tile, const float* w, 
         for (int h = 0; h < G; ++h) acc[k][h] = make_float2(0.f, 0.f);
 
     if constexpr (sizeof(T) == 2) {
-#pragma unroll
+#pragma unroll kScoreUnroll
         for (int c = 0; c < kChunks; ++c) {
             float2 xy[KPT][4];
             float2 nn[KPT][2];

@@ -48,8 +48,15 @@ struct FusedArgs {
     int32_t* kept;               // [U][B] or null
     int32_t* n_kept;             // [U]
     float* scratch;              // [grid][G][cap] per-CTA score scratch
+    uint64_t* trace;             // [U][kTracePoints] phase timestamps, or null
     uint32_t* flag;
 };
+
+constexpr int kTracePoints = 8;  // per unit: start, scored, z-max, selected, gathered
+constexpr int kTraceWarps = 8;   // one slot per warp of the fused kernel
+
+// api.cu: the caller's phase-trace buffer for the next launches (or null).
+uint64_t* phase_trace_buffer(int64_t n_units);
 
 // api.cu: call after every kernel launch (counts launches and records the
 // caller's timing event for that launch, if any).

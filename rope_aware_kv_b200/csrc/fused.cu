@@ -19,9 +19,11 @@
 //           first radix digit histogram.
 //   select  two more radix digits on shared-memory histograms, then the
 //           ordered compaction of kept indices (warp ballots).
-//   gather  every thread copies 16-byte pieces of kept K and V rows with
-//           deep memory-level parallelism (loads of 16 rows in flight before
-//           their stores), plus positions and the kept list.
+//   gather  kept rows form runs of consecutive indices; one lane streams
+//           each run piece (<= 8 KB) of K and of V into a 16-buffer shared
+//           ring with cp.async.bulk (up to 128 KB of loads in flight), and the
+//           math warps copy landed pieces to the destination with 16-byte
+//           stores, freeing each buffer as soon as it is read.
 // HBM traffic per unit is the compulsory bytes plus the re-read of kept K
 // rows (often from L2).
 #include "select_core.cuh"
@@ -44,7 +46,9 @@ struct FusedShape {
     static constexpr int kMath = 128;
     static constexpr int kThreads = kMath + 32;
     static constexpr int kWarps = kThreads / 32;
-    static constexpr int kGatherBatch = sizeof(T) == 2 ? 16 : 8;        // rows per thread per batch
+    static constexpr int kGStage = 8192;                                // gather piece buffer
+    static constexpr int kGStages = kRegionA / kGStage;                 // 16
+    static constexpr int kGRows = kGStage / kRowBytes;                  // rows per piece
 };
 
 struct FusedLayout {
@@ -61,7 +65,7 @@ __host__ __device__ inline FusedLayout fused_layout(int G, int64_t cap, int64_t 
     L.fin = L.w + static_cast<size_t>(G) * kWHead * 4;
     L.kidx = L.fin + static_cast<size_t>(capP) * 4;
     L.bars = L.kidx + ((static_cast<size_t>(m) * 4 + 15) & ~size_t(15));
-    L.red = L.bars + (2 * S::kStages) * 8;
+    L.red = L.bars + (2 * S::kStages + 2 * S::kGStages) * 8;
     L.misc = L.red + static_cast<size_t>(4) * kMaxG * 2 * 8;
     L.total = L.misc + 256 + 1024;  // state and warp counts; alignment slack
     return L;
@@ -98,12 +102,16 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
     int32_t* kidx = reinterpret_cast<int32_t*>(base + L.kidx);
     uint64_t* full = reinterpret_cast<uint64_t*>(base + L.bars);
     uint64_t* empty = full + S::kStages;
+    uint64_t* gfull = empty + S::kStages;
+    uint64_t* gempty = gfull + S::kGStages;
     double* red = reinterpret_cast<double*>(base + L.red);  // [4 warps][kMaxG][2]
     SelState* st = reinterpret_cast<SelState*>(base + L.misc);
     float2* mom = reinterpret_cast<float2*>(base + L.misc + 16);            // [kMaxG]
     uint32_t* wcnt = reinterpret_cast<uint32_t*>(base + L.misc + 16 + 64);  // [kWarps][2]
-    int32_t* abort_flag = reinterpret_cast<int32_t*>(base + L.misc + 16 + 64 + 48);
+    int32_t* nchunks = reinterpret_cast<int32_t*>(base + L.misc + 16 + 64 + 48);
+    int32_t* abort_flag = nchunks + 1;
     uint32_t* hist = reinterpret_cast<uint32_t*>(regA);  // between scoring and gathering
+    int32_t* chunk_r = reinterpret_cast<int32_t*>(fin);  // after the compaction
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -115,6 +123,10 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], 64);
         }
+        for (int i = 0; i < S::kGStages; ++i) {
+            mbar_init(&gfull[i], 1);
+            mbar_init(&gempty[i], 32);
+        }
         fence_barrier_init();
         prefetch_tensormap(&kmap);
         *abort_flag = 0;
@@ -122,6 +134,7 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
     __syncthreads();
 
     uint32_t tiles_done = 0;   // running tile count (TMA ring position) of this CTA
+    uint32_t pieces_done = 0;  // running gather-piece count (gather ring position)
 
     for (int64_t u = blockIdx.x; u < a.n_units; u += gridDim.x) {
         if (*abort_flag) break;  // a bounded wait gave up: stop cleanly
@@ -368,61 +381,115 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
         __syncthreads();
 
         // ---------------- gather ----------------
-        // Every thread moves 16-byte pieces of kept rows: kGRowsPerThread rows
-        // of K and of V in flight per thread (loads first, then stores), so
-        // about 80 KB of loads are in flight per SM; a store frees its
-        // registers at once, so only the load latency limits the rate.
+        // Kept rows form runs of consecutive source rows; a piece is a run cut
+        // at row indices that are multiples of kGRows (<= 8 KB).  The engine
+        // lane streams K and V pieces into a 16-buffer shared-memory ring with
+        // cp.async.bulk (no registers or L1 miss slots held, up to 128 KB in
+        // flight); math warp (piece % 4) copies each landed piece to the
+        // destination with 16-byte stores and frees its buffer at once.
         {
+            const int seg = ((m + S::kWarps * 32 - 1) / (S::kWarps * 32)) * 32;
+            const int r0 = warp * seg;
+            const int r1 = min(r0 + seg, m);
+            uint32_t cnt = 0;
+            for (int r = r0 + lane; r - lane < r1; r += 32) {
+                bool start = false;
+                if (r < r1) {
+                    const int32_t j = kidx[r];
+                    const int32_t jp = r > 0 ? kidx[r - 1] : -2;
+                    start = (r % S::kGRows == 0) || j != jp + 1;
+                }
+                cnt += __popc(__ballot_sync(0xffffffffu, start));
+            }
+            if (lane == 0) wcnt[2 * warp] = cnt;
+            __syncthreads();
+            uint32_t pos = 0;
+            for (int v = 0; v < warp; ++v) pos += wcnt[2 * v];
+            if (warp == S::kWarps - 1 && lane == 0) *nchunks = static_cast<int>(pos + cnt);
+            const uint32_t lt = (1u << lane) - 1u;
+            for (int r = r0 + lane; r - lane < r1; r += 32) {
+                bool start = false;
+                if (r < r1) {
+                    const int32_t j = kidx[r];
+                    const int32_t jp = r > 0 ? kidx[r - 1] : -2;
+                    start = (r % S::kGRows == 0) || j != jp + 1;
+                }
+                const uint32_t b = __ballot_sync(0xffffffffu, start);
+                if (start) chunk_r[pos + __popc(b & lt)] = r;
+                pos += __popc(b);
+            }
+        }
+        fence_proxy_async();
+        __syncthreads();
+        const int n_chunks = *nchunks;
+        const int npc = a.v_src ? 2 * n_chunks : n_chunks;  // K (and V) piece per chunk
+        auto chunk_rows = [&](int c, int& r, int& len, int32_t& j) -> bool {
+            r = chunk_r[c];
+            const int rend = (c + 1 < n_chunks) ? chunk_r[c + 1] : m;
+            len = rend - r;
+            j = kidx[r];
+            return j >= 0 && j + len <= n && len > 0 && len <= S::kGRows;
+        };
+        if (tid == S::kMath) {
+            // Engine: bulk loads only.
+            const char* ks = static_cast<const char*>(a.k_src);
+            const char* vs = static_cast<const char*>(a.v_src);
+            for (int p = 0; p < npc; ++p) {
+                const uint32_t pc = pieces_done + p;
+                const int sb = pc % S::kGStages;
+                if (!mbar_wait(&gempty[sb], ((pc / S::kGStages) & 1) ^ 1, a.flag)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                const int c = a.v_src ? (p >> 1) : p;
+                const bool is_v = a.v_src && (p & 1);
+                int r, len;
+                int32_t j;
+                if (!chunk_rows(c, r, len, j)) {  // cannot happen when the selection is consistent
+                    raise_flag(a.flag, TRI_FLAG_INDEX_RANGE);
+                    mbar_arrive_expect_tx(&gfull[sb], 0);
+                    continue;
+                }
+                const uint32_t bytes = static_cast<uint32_t>(len * S::kRowBytes);
+                mbar_arrive_expect_tx(&gfull[sb], bytes);
+                bulk_load(regA + sb * S::kGStage, (is_v ? vs : ks) + (u * a.cap + j) * S::kRowBytes,
+                          bytes, &gfull[sb]);
+            }
+        } else if (tid < S::kMath) {
+            // Math warps: drain pieces warp, warp + 4, ... to global memory.
             constexpr int kVec = S::kRowBytes / 16;
-            constexpr int kGroups = S::kThreads / kVec;  // rows per pass
-            constexpr int kBatch = S::kGatherBatch;
-            const int l = tid % kVec;
-            const int g = tid / kVec;
-            const uint4* ks = static_cast<const uint4*>(a.k_src);
-            const uint4* vs = static_cast<const uint4*>(a.v_src);
             uint4* kd = static_cast<uint4*>(a.k_dst);
             uint4* vd = static_cast<uint4*>(a.v_dst);
-            if (g < kGroups) {
-                for (int r0 = 0; r0 < m; r0 += kGroups * kBatch) {
-                    uint4 kv[kBatch], vv[kBatch];
-                    int32_t jj[kBatch];
-#pragma unroll
-                    for (int q = 0; q < kBatch; ++q) {
-                        const int r = r0 + q * kGroups + g;
-                        int32_t j = r < m ? kidx[r] : -1;
-                        if (j >= n) {  // cannot happen when the selection is consistent
-                            raise_flag(a.flag, TRI_FLAG_INDEX_RANGE);
-                            j = -1;
-                        }
-                        jj[q] = j;
-                    }
-#pragma unroll
-                    for (int q = 0; q < kBatch; ++q) {
-                        if (jj[q] >= 0) {
-                            const int64_t srow = u * a.cap + jj[q];
-                            kv[q] = ld_stream(ks + srow * kVec + l);
-                            if (vs) vv[q] = ld_stream(vs + srow * kVec + l);
-                        }
-                    }
-#pragma unroll
-                    for (int q = 0; q < kBatch; ++q) {
-                        if (jj[q] >= 0) {
-                            const int r = r0 + q * kGroups + g;
-                            const int64_t drow = u * a.cap_dst + r;
-                            st_stream(kd + drow * kVec + l, kv[q]);
-                            if (vd) st_stream(vd + drow * kVec + l, vv[q]);
-                            if (a.pos_dst && l == 0) a.pos_dst[drow] = a.pos_src[u * a.cap + jj[q]];
-                        }
-                    }
+            for (int p = warp; p < npc; p += 4) {
+                const uint32_t pc = pieces_done + p;
+                const int sb = pc % S::kGStages;
+                if (!mbar_wait(&gfull[sb], (pc / S::kGStages) & 1, a.flag)) {
+                    *abort_flag = 1;
+                    break;
                 }
+                const int c = a.v_src ? (p >> 1) : p;
+                const bool is_v = a.v_src && (p & 1);
+                int r, len;
+                int32_t j;
+                if (chunk_rows(c, r, len, j)) {
+                    const uint4* buf = reinterpret_cast<const uint4*>(regA + sb * S::kGStage);
+                    uint4* dst = (is_v ? vd : kd) + (u * a.cap_dst + r) * kVec;
+                    const int nv = len * kVec;
+                    for (int e = lane; e < nv; e += 32) st_stream(dst + e, buf[e]);
+                    if (!is_v && a.pos_dst && lane < len)
+                        a.pos_dst[u * a.cap_dst + r + lane] = a.pos_src[u * a.cap + j + lane];
+                }
+                __syncwarp();
+                mbar_arrive(&gempty[sb]);
             }
-            if (a.kept)
-                for (int r = tid; r < B; r += S::kThreads) a.kept[u * B + r] = r < m ? kidx[r] : -1;
-            if (tid == 0) a.n_kept[u] = m;
         }
+        if (a.kept)
+            for (int r = tid; r < B; r += S::kThreads) a.kept[u * B + r] = r < m ? kidx[r] : -1;
+        if (tid == 0) a.n_kept[u] = m;
         trace_point(a, u, 4);
         __syncthreads();
         tiles_done += n_tiles;
+        pieces_done += static_cast<uint32_t>(npc);
         fence_proxy_async();
         __syncthreads();
     }

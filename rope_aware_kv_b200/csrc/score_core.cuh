@@ -112,4 +112,69 @@ __device__ __forceinline__ void score_rows(const uint8_t* tile, const float* w, 
         for (int h = 0; h < G; ++h) s[k][h] = acc[k][h].x + acc[k][h].y;
 }
 
+// Partial scores over half of the bands (bf16 rows): chunks 8*half .. 8*half+7,
+// i.e. TMA box `half` of the tile, for all G heads.  Two warps that each take
+// one half of the same keys produce the full score as the sum of their parts.
+template <typename T, int G, int KPT, int kBoxBytes, int kRowStride, int kHalf>
+__device__ __forceinline__ void score_rows_half_t(const uint8_t* tile, const float* w,
+                                                  int first_row, float (&s)[KPT][G]) {
+    static_assert(sizeof(T) == 2, "band split is for bfloat16 rows");
+    float2 acc[KPT][G];
+#pragma unroll
+    for (int k = 0; k < KPT; ++k)
+#pragma unroll
+        for (int h = 0; h < G; ++h) acc[k][h] = make_float2(0.f, 0.f);
+#pragma unroll kScoreUnroll
+    for (int cc = 0; cc < 8; ++cc) {
+        const int c = kHalf * 8 + cc;
+        float2 xy[KPT][4];
+        float2 nn[KPT][2];
+#pragma unroll
+        for (int k = 0; k < KPT; ++k) {
+            const int r = first_row + kRowStride * k;
+            const uint4 v = *reinterpret_cast<const uint4*>(tile + kHalf * kBoxBytes + r * 128 +
+                                                            ((cc ^ (r & 7)) << 4));
+            const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+            float n[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float x = bf16_lo(wd[i]), y = bf16_hi(wd[i]);
+                xy[k][i] = make_float2(x, y);
+                n[i] = sqrt_approx(fmaf(x, x, y * y));
+            }
+            nn[k][0] = make_float2(n[0], n[1]);
+            nn[k][1] = make_float2(n[2], n[3]);
+        }
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float4* rec = reinterpret_cast<const float4*>(w + h * kWHead + c * kWChunk);
+            const float4 a = rec[0], b = rec[1], cw = rec[2];
+#pragma unroll
+            for (int k = 0; k < KPT; ++k) {
+                float2 t = acc[k][h];
+                t = __ffma2_rn(xy[k][0], make_float2(a.x, a.y), t);
+                t = __ffma2_rn(xy[k][1], make_float2(a.z, a.w), t);
+                t = __ffma2_rn(xy[k][2], make_float2(b.x, b.y), t);
+                t = __ffma2_rn(xy[k][3], make_float2(b.z, b.w), t);
+                t = __ffma2_rn(nn[k][0], make_float2(cw.x, cw.y), t);
+                t = __ffma2_rn(nn[k][1], make_float2(cw.z, cw.w), t);
+                acc[k][h] = t;
+            }
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < KPT; ++k)
+#pragma unroll
+        for (int h = 0; h < G; ++h) s[k][h] = acc[k][h].x + acc[k][h].y;
+}
+
+template <typename T, int G, int KPT, int kBoxBytes, int kRowStride>
+__device__ __forceinline__ void score_rows_half(const uint8_t* tile, const float* w, int first_row,
+                                                int half, float (&s)[KPT][G]) {
+    if (half == 0)
+        score_rows_half_t<T, G, KPT, kBoxBytes, kRowStride, 0>(tile, w, first_row, s);
+    else
+        score_rows_half_t<T, G, KPT, kBoxBytes, kRowStride, 1>(tile, w, first_row, s);
+}
+
 }  // namespace tri

@@ -84,7 +84,8 @@ typedef enum tri_status {
     TRI_ERR_UNSUPPORTED = 2, /* valid but not implemented (head_dim, G, dtype) */
     TRI_ERR_WORKSPACE = 3,   /* ws is NULL or smaller than the *_workspace_bytes query */
     TRI_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
-    TRI_ERR_DEVICE = 5       /* tri_check_device_error found a device-side flag */
+    TRI_ERR_DEVICE = 5,      /* tri_check_device_error found a device-side flag */
+    TRI_ERR_SCRATCH_LIMIT = 6 /* the request needs more than the static scratch holds */
 } tri_status;
 
 typedef enum tri_dtype {
@@ -192,6 +193,37 @@ size_t tri_select_workspace_bytes(int64_t n_units, int64_t cap, int64_t B);
 tri_status tri_select_topB(const float* final_score, int64_t n_units, int64_t cap,
                            const int32_t* n_valid, int64_t B, int32_t* kept_idx, int32_t* n_kept,
                            void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * tri_select_topB without a workspace, for callers that cannot allocate
+ * device memory (a serving engine whose memory manager owns all device memory
+ * and hands a plugin only its inputs and outputs; a latency-critical path
+ * where cudaMalloc, which may synchronise the device or fail, is forbidden).
+ * The pages have no counterpart: this is an integration variant of the
+ * selection above and returns exactly its results.
+ *
+ * The scratch (radix histograms and per-chunk counts) lives in a statically
+ * allocated device array of tri_select_static_scratch_bytes() bytes (1 MiB)
+ * that every GPU which loads the library reserves until the process exits.
+ * Arguments, layouts and results are those of tri_select_topB.  A request
+ * whose scratch would not fit (3 * 8 KiB per unit plus 8 bytes per 2048 keys
+ * per unit, plus 256 bytes) returns TRI_ERR_SCRATCH_LIMIT before anything is
+ * launched; e.g. 40 units of up to 131072 keys fit.  Nothing is allocated:
+ * no cudaMalloc, cudaFree or allocating library call.
+ *
+ * The first call on a device looks up the array's device address with that
+ * device current (cudaGetSymbolAddress) and remembers it; make that first call
+ * before capturing any stream on the device.  Every call shares the one array
+ * and clears what must start at zero itself, so calls whose executions overlap
+ * on the GPU (different streams, or different host threads) race and must be
+ * serialised by the caller.  Device-side flags are not reported.
+ */
+tri_status tri_select_topB_static(const float* final_score, int64_t n_units, int64_t cap,
+                                  const int32_t* n_valid, int64_t B, int32_t* kept_idx,
+                                  int32_t* n_kept, void* stream);
+
+/* Size in bytes of the static scratch array of tri_select_topB_static. */
+size_t tri_select_static_scratch_bytes(void);
 
 /* ---------------------------------------------------------------------- */
 /* Order-preserving compaction                                             */

@@ -29,7 +29,8 @@ TRI_F32 = 0
 TRI_BF16 = 1
 
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape or type",
-          3: "workspace missing or too small", 4: "CUDA error", 5: "device-side flag set"}
+          3: "workspace missing or too small", 4: "CUDA error", 5: "device-side flag set",
+          6: "request exceeds the static scratch"}
 
 FLAG_NVALID_RANGE = 0x1
 FLAG_INDEX_RANGE = 0x2
@@ -53,6 +54,7 @@ EXPORTS = (
     "tri_prune_workspace_bytes", "tri_prune",
     "tri_append", "tri_check_device_error",
     "tri_set_timing_events", "tri_last_launch_count", "tri_set_phase_trace",
+    "tri_select_topB_static", "tri_select_static_scratch_bytes",
 )
 
 
@@ -107,6 +109,8 @@ def load(path: Optional[str] = None):
         "tri_set_timing_events": (i32, [ctypes.POINTER(ctypes.c_void_p), i32]),
         "tri_last_launch_count": (i32, []),
         "tri_set_phase_trace": (i32, [P, sz]),
+        "tri_select_topB_static": (i32, [P, i64, i64, P, i64, P, P, P]),
+        "tri_select_static_scratch_bytes": (sz, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -235,6 +239,23 @@ def tri_select_topB(final: torch.Tensor, B: int, n_valid: Optional[torch.Tensor]
     _check("tri_select_topB", load().tri_select_topB(
         _ptr(final), U, cap, _ptr(n_valid), B, _ptr(kept), _ptr(n_kept), _ptr(ws), ws.numel(),
         _stream(stream)))
+    return kept, n_kept
+
+
+def tri_select_topB_static(final: torch.Tensor, B: int, n_valid: Optional[torch.Tensor] = None,
+                           kept: Optional[torch.Tensor] = None,
+                           n_kept: Optional[torch.Tensor] = None, stream=None):
+    """tri_select_topB with the library's static device scratch instead of a
+    workspace (for callers that cannot allocate device memory; see tri.h).
+    Overlapping calls race on the shared scratch."""
+    U, cap = final.shape
+    dev = final.device
+    if kept is None:
+        kept = torch.empty((U, B), dtype=torch.int32, device=dev)
+    if n_kept is None:
+        n_kept = torch.empty((U,), dtype=torch.int32, device=dev)
+    _check("tri_select_topB_static", load().tri_select_topB_static(
+        _ptr(final), U, cap, _ptr(n_valid), B, _ptr(kept), _ptr(n_kept), _stream(stream)))
     return kept, n_kept
 
 

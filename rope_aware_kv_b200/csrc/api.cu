@@ -272,6 +272,7 @@ const char* tri_status_str(tri_status s) {
         case TRI_ERR_WORKSPACE: return "workspace missing or too small";
         case TRI_ERR_CUDA: return "CUDA error";
         case TRI_ERR_DEVICE: return "device-side flag set";
+        case TRI_ERR_SCRATCH_LIMIT: return "request exceeds the static scratch";
     }
     return "unknown status";
 }

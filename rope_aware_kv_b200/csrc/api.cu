@@ -205,8 +205,17 @@ struct PruneWs {
     size_t total;
 };
 
-bool use_fused(tri_dtype dt, int G, int64_t cap, int64_t B) {
-    return fused_smem_bytes(dt, G, cap, B) <= fused_smem_limit();
+// Deepest TMA ring (4..6 stages of 32 KB) the fused kernel fits in shared
+// memory, or 0 when even 4 stages do not fit.
+int fused_stages(tri_dtype dt, int G, int64_t cap, int64_t B) {
+    for (int st = fused_max_stages(); st >= 4; --st)
+        if (fused_smem_bytes(dt, G, cap, B, st) <= fused_smem_limit()) return st;
+    return 0;
+}
+
+bool use_fused(tri_dtype dt, int G, int64_t cap, int64_t B, int path) {
+    const int st = fused_stages(dt, G, cap, B);
+    return path == TRI_PATH_FUSED ? st >= 4 : st >= 5;
 }
 
 // CTAs of the persistent fused kernel: one per SM (its shared memory allows
@@ -220,7 +229,7 @@ PruneWs prune_ws(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int6
                  int64_t B, tri_dtype dt, bool own_kept, int path) {
     PruneWs w;
     const int64_t U = n_seq * n_layers * n_kvheads;
-    w.fused = path == TRI_PATH_SPLIT ? false : use_fused(dt, G, cap, B);
+    w.fused = path == TRI_PATH_SPLIT ? false : use_fused(dt, G, cap, B, path);
     if (w.fused) {
         Carve c;
         w.sc.wts = c.take(static_cast<size_t>(U * G) * kWHead * 4);
@@ -468,6 +477,7 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
         TRI_CUDA(launch_fold(stats, p_cur, n_seq, n_layers, n_kvheads * G, cfg->theta, off, wts, s));
         FusedArgs a;
         a.n_units = U;
+        a.stages = fused_stages(dt, G, cap_src, B);
         a.cap = cap_src;
         a.cap_dst = cap_dst;
         a.B = B;

@@ -9,12 +9,11 @@
 // (jaedaily.cn tutorial, eviction step).
 //
 // Per unit:
-//   score   a producer lane streams 128-key tiles (32 KB) into a 4-stage TMA
-//           ring; the four math warps form two pairs, each pair scores one
-//           tile with every lane on 4 keys and the GQA heads split between
-//           the pair's two warps (so one broadcast weight load feeds 4 keys);
-//           per-head scores go to a per-CTA float32 scratch that stays in L2,
-//           float64 moments stay in registers.
+//   score   a producer lane streams 128-key tiles (32 KB) into a TMA ring of
+//           4 to 6 stages; each of the four math warps scores whole tiles,
+//           every lane on 4 keys for all GQA heads (so one broadcast weight
+//           load feeds 4 keys); per-head scores go to a per-CTA float32
+//           scratch that stays in L2, float64 moments stay in registers.
 //   z-max   fixed-order moment merge, final = max_h z_h into shared memory,
 //           first radix digit histogram.
 //   select  two more radix digits on shared-memory histograms, then the
@@ -41,13 +40,12 @@ struct FusedShape {
     static constexpr int kTile = 32 * kKPT;                             // keys per tile
     static constexpr int kBoxBytes = kTile * 128;
     static constexpr int kStageBytes = kTile * kRowBytes;               // 32 KB
-    static constexpr int kStages = 4;
-    static constexpr int kRegionA = kStages * kStageBytes;              // 128 KB
+    static constexpr int kMaxStages = 6;                                // TMA ring depth (runtime)
     static constexpr int kMath = 128;
     static constexpr int kThreads = kMath + 32;
     static constexpr int kWarps = kThreads / 32;
     static constexpr int kGStage = 8192;                                // gather piece buffer
-    static constexpr int kGStages = kRegionA / kGStage;                 // 16
+    static constexpr int kMaxGStages = kMaxStages * kStageBytes / kGStage;
     static constexpr int kGRows = kGStage / kRowBytes;                  // rows per piece
 };
 
@@ -56,27 +54,20 @@ struct FusedLayout {
 };
 
 template <typename T>
-__host__ __device__ inline FusedLayout fused_layout(int G, int64_t cap, int64_t B) {
+__host__ __device__ inline FusedLayout fused_layout(int G, int64_t cap, int64_t B, int stages) {
     using S = FusedShape<T>;
     FusedLayout L;
     const int64_t capP = (cap + 4) & ~int64_t(3);
     const int64_t m = B < cap ? B : cap;
-    L.w = S::kRegionA;
+    L.w = static_cast<size_t>(stages) * S::kStageBytes;
     L.fin = L.w + static_cast<size_t>(G) * kWHead * 4;
     L.kidx = L.fin + static_cast<size_t>(capP) * 4;
     L.bars = L.kidx + ((static_cast<size_t>(m) * 4 + 15) & ~size_t(15));
-    L.red = L.bars + (2 * S::kStages + 2 * S::kGStages) * 8;
+    L.red = L.bars + (2 * S::kMaxStages + 2 * S::kMaxGStages) * 8;
     L.misc = L.red + static_cast<size_t>(4) * kMaxG * 2 * 8;
     L.total = L.misc + 256 + 1024;  // state and warp counts; alignment slack
     return L;
 }
-
-// Head split between the two warps of a pair.
-template <int G>
-struct HeadSplit {
-    static constexpr int kA = (G + 1) / 2;
-    static constexpr int kB = G - kA;
-};
 
 // Phase trace: lane 0 of every warp records %globaltimer just before the
 // barrier that ends phase i of unit u (the phase ends at the latest warp);
@@ -90,20 +81,20 @@ template <typename T, int G>
 __global__ void __launch_bounds__(FusedShape<T>::kThreads, 1)
 prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
     using S = FusedShape<T>;
-    constexpr int GA = HeadSplit<G>::kA;
-    constexpr int GB = HeadSplit<G>::kB;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const FusedLayout L = fused_layout<T>(G, a.cap, a.B);
+    const int n_stages = a.stages;
+    const int n_gstages = n_stages * S::kStageBytes / S::kGStage;
+    const FusedLayout L = fused_layout<T>(G, a.cap, a.B, n_stages);
     uint8_t* regA = base;
     float* w = reinterpret_cast<float*>(base + L.w);
     float* fin = reinterpret_cast<float*>(base + L.fin);
     int32_t* kidx = reinterpret_cast<int32_t*>(base + L.kidx);
     uint64_t* full = reinterpret_cast<uint64_t*>(base + L.bars);
-    uint64_t* empty = full + S::kStages;
-    uint64_t* gfull = empty + S::kStages;
-    uint64_t* gempty = gfull + S::kGStages;
+    uint64_t* empty = full + S::kMaxStages;
+    uint64_t* gfull = empty + S::kMaxStages;
+    uint64_t* gempty = gfull + S::kMaxGStages;
     double* red = reinterpret_cast<double*>(base + L.red);  // [4 warps][kMaxG][2]
     SelState* st = reinterpret_cast<SelState*>(base + L.misc);
     float2* mom = reinterpret_cast<float2*>(base + L.misc + 16);            // [kMaxG]
@@ -119,11 +110,11 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
     float* scratch = a.scratch + static_cast<int64_t>(blockIdx.x) * G * a.cap;
 
     if (tid == S::kMath) {
-        for (int i = 0; i < S::kStages; ++i) {
+        for (int i = 0; i < n_stages; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 64);
+            mbar_init(&empty[i], 32);
         }
-        for (int i = 0; i < S::kGStages; ++i) {
+        for (int i = 0; i < n_gstages; ++i) {
             mbar_init(&gfull[i], 1);
             mbar_init(&gempty[i], 32);
         }
@@ -156,8 +147,8 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
                 if (tid == S::kMath) {
                     for (int i = 0; i < n_tiles; ++i) {
                         const uint32_t tc = tiles_done + i;
-                        const int stage = tc % S::kStages;
-                        if (!mbar_wait(&empty[stage], ((tc / S::kStages) & 1) ^ 1, a.flag)) {
+                        const int stage = tc % n_stages;
+                        if (!mbar_wait(&empty[stage], ((tc / n_stages) & 1) ^ 1, a.flag)) {
                             *abort_flag = 1;
                             break;
                         }
@@ -171,61 +162,38 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
                     }
                 }
             } else {
-                const int pair = warp >> 1, half = warp & 1;
-                const int hb = half == 0 ? 0 : GA;
-                const int gh = half == 0 ? GA : GB;
-                double m1[GA], m2[GA];
+                // Math warp w scores tiles w, w + 4, ... with all G heads.
+                double m1[G], m2[G];
 #pragma unroll
-                for (int h = 0; h < GA; ++h) m1[h] = m2[h] = 0.0;
-                for (int i = pair; i < n_tiles; i += 2) {
+                for (int h = 0; h < G; ++h) m1[h] = m2[h] = 0.0;
+                for (int i = warp; i < n_tiles; i += 4) {
                     const uint32_t tc = tiles_done + i;
-                    const int stage = tc % S::kStages;
-                    if (!mbar_wait(&full[stage], (tc / S::kStages) & 1, a.flag)) {
+                    const int stage = tc % n_stages;
+                    if (!mbar_wait(&full[stage], (tc / n_stages) & 1, a.flag)) {
                         *abort_flag = 1;
                         break;
                     }
-                    const uint8_t* tile = regA + stage * S::kStageBytes;
-                    float s[S::kKPT][GA];
-                    if (half == 0) {
-                        score_rows<T, GA, S::kKPT, S::kBoxBytes, 32>(tile, w, lane, s);
-                    } else {
-                        if constexpr (GB > 0) {
-                            float sb[S::kKPT][GB];
-                            score_rows<T, GB, S::kKPT, S::kBoxBytes, 32>(tile, w + GA * kWHead,
-                                                                          lane, sb);
-#pragma unroll
-                            for (int k = 0; k < S::kKPT; ++k) {
-#pragma unroll
-                                for (int h = 0; h < GA; ++h) s[k][h] = 0.f;
-#pragma unroll
-                                for (int h = 0; h < GB; ++h) s[k][h] = sb[k][h];
-                            }
-                        } else {
-#pragma unroll
-                            for (int k = 0; k < S::kKPT; ++k)
-#pragma unroll
-                                for (int h = 0; h < GA; ++h) s[k][h] = 0.f;
-                        }
-                    }
+                    float s[S::kKPT][G];
+                    score_rows<T, G, S::kKPT, S::kBoxBytes, 32>(regA + stage * S::kStageBytes, w,
+                                                                 lane, s);
+                    __syncwarp();
                     mbar_arrive(&empty[stage]);
 #pragma unroll
                     for (int k = 0; k < S::kKPT; ++k) {
                         const int j = i * S::kTile + lane + 32 * k;
                         if (j < n) {
 #pragma unroll
-                            for (int h = 0; h < GA; ++h) {
-                                if (h < gh) {
-                                    scratch[static_cast<int64_t>(hb + h) * a.cap + j] = s[k][h];
-                                    const double d = s[k][h];
-                                    m1[h] += d;
-                                    m2[h] = fma(d, d, m2[h]);
-                                }
+                            for (int h = 0; h < G; ++h) {
+                                scratch[static_cast<int64_t>(h) * a.cap + j] = s[k][h];
+                                const double d = s[k][h];
+                                m1[h] += d;
+                                m2[h] = fma(d, d, m2[h]);
                             }
                         }
                     }
                 }
 #pragma unroll
-                for (int h = 0; h < GA; ++h) {
+                for (int h = 0; h < G; ++h) {
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) {
                         m1[h] += __shfl_down_sync(0xffffffffu, m1[h], o);
@@ -240,15 +208,13 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
             trace_point(a, u, 1);
             __syncthreads();
             if (*abort_flag) break;
-            // ---------------- moments (fixed order: pair 0 then pair 1) ----------------
+            // ---------------- moments (fixed order: warps 0..3) ----------------
             if (tid < G) {
                 const int h = tid;
-                const int half = h < GA ? 0 : 1;
-                const int hh = h < GA ? h : h - GA;
-                const double s1 =
-                    red[(half * kMaxG + hh) * 2] + red[((2 + half) * kMaxG + hh) * 2];
-                const double s2 =
-                    red[(half * kMaxG + hh) * 2 + 1] + red[((2 + half) * kMaxG + hh) * 2 + 1];
+                const double s1 = ((red[(0 * kMaxG + h) * 2] + red[(1 * kMaxG + h) * 2]) +
+                                   red[(2 * kMaxG + h) * 2]) + red[(3 * kMaxG + h) * 2];
+                const double s2 = ((red[(0 * kMaxG + h) * 2 + 1] + red[(1 * kMaxG + h) * 2 + 1]) +
+                                   red[(2 * kMaxG + h) * 2 + 1]) + red[(3 * kMaxG + h) * 2 + 1];
                 const double mu = s1 / n;
                 double var = s2 / n - mu * mu;
                 if (var < 0.0) var = 0.0;
@@ -436,8 +402,8 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
             const char* vs = static_cast<const char*>(a.v_src);
             for (int p = 0; p < npc; ++p) {
                 const uint32_t pc = pieces_done + p;
-                const int sb = pc % S::kGStages;
-                if (!mbar_wait(&gempty[sb], ((pc / S::kGStages) & 1) ^ 1, a.flag)) {
+                const int sb = pc % n_gstages;
+                if (!mbar_wait(&gempty[sb], ((pc / n_gstages) & 1) ^ 1, a.flag)) {
                     *abort_flag = 1;
                     break;
                 }
@@ -462,8 +428,8 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
             uint4* vd = static_cast<uint4*>(a.v_dst);
             for (int p = warp; p < npc; p += 4) {
                 const uint32_t pc = pieces_done + p;
-                const int sb = pc % S::kGStages;
-                if (!mbar_wait(&gfull[sb], (pc / S::kGStages) & 1, a.flag)) {
+                const int sb = pc % n_gstages;
+                if (!mbar_wait(&gfull[sb], (pc / n_gstages) & 1, a.flag)) {
                     *abort_flag = 1;
                     break;
                 }
@@ -498,10 +464,12 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-size_t fused_smem_bytes(tri_dtype dt, int G, int64_t cap, int64_t B) {
-    return dt == TRI_BF16 ? fused_layout<__nv_bfloat16>(G, cap, B).total
-                          : fused_layout<float>(G, cap, B).total;
+size_t fused_smem_bytes(tri_dtype dt, int G, int64_t cap, int64_t B, int stages) {
+    return dt == TRI_BF16 ? fused_layout<__nv_bfloat16>(G, cap, B, stages).total
+                          : fused_layout<float>(G, cap, B, stages).total;
 }
+
+int fused_max_stages() { return FusedShape<float>::kMaxStages; }
 
 size_t fused_smem_limit() {
     static int lim = 0;
@@ -520,7 +488,7 @@ int fused_tile_keys(tri_dtype dt) {
 template <typename T, int G>
 static cudaError_t launch_fused_t(const CUtensorMap& map, const FusedArgs& a, int n_ctas,
                                   cudaStream_t s) {
-    const size_t smem = fused_layout<T>(G, a.cap, a.B).total;
+    const size_t smem = fused_layout<T>(G, a.cap, a.B, a.stages).total;
     auto kern = prune_fused_kernel<T, G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));

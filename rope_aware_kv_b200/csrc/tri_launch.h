@@ -34,6 +34,7 @@ struct ScoreArgs {
 
 struct FusedArgs {
     int64_t n_units;
+    int stages;                  // TMA ring depth, 4..6
     int64_t cap;
     int64_t cap_dst;
     int64_t B;
@@ -98,7 +99,8 @@ cudaError_t launch_append(tri_dtype dt, void* k_cache, void* v_cache, int32_t* p
                           const int32_t* pos_new, int64_t n_new, uint32_t* flag, cudaStream_t s);
 
 // fused.cu
-size_t fused_smem_bytes(tri_dtype dt, int G, int64_t cap, int64_t B);
+size_t fused_smem_bytes(tri_dtype dt, int G, int64_t cap, int64_t B, int stages);
+int fused_max_stages();
 size_t fused_smem_limit();
 int fused_tile_keys(tri_dtype dt);
 cudaError_t launch_fused(tri_dtype dt, int G, const CUtensorMap& map, const FusedArgs& a,

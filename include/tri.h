@@ -104,9 +104,10 @@ typedef enum tri_dtype {
 
 /* Method parameters.  tri_config_default fills the pages' values. */
 /* Kernel path of tri_prune. */
-#define TRI_PATH_AUTO 0  /* fused kernel when the unit fits in shared memory, else split */
+#define TRI_PATH_AUTO 0  /* fused for many small units, coop for few units, else split */
 #define TRI_PATH_FUSED 1 /* one CTA per unit (TRI_ERR_UNSUPPORTED if it does not fit) */
 #define TRI_PATH_SPLIT 2 /* separate score / z-max / select / gather kernels */
+#define TRI_PATH_COOP 3  /* each unit split over several CTAs of one kernel (few large units) */
 
 typedef struct tri_config {
     int head_dim;                      /* d; 128 is supported */
@@ -257,8 +258,10 @@ size_t tri_prune_workspace_bytes(int64_t n_seq, int64_t n_layers, int64_t n_kvhe
 /*
  * One prune step over every unit of a batch: score, z-normalise and max,
  * select the top-B, gather K, V and positions into the destination cache.
- * Units whose n_valid <= B are copied whole.  Small caches run one fused
- * kernel per unit; large caches run the split kernels.  Arguments as in the
+ * Units whose n_valid <= B are copied whole.  Many small caches run one
+ * persistent fused kernel (whole units per CTA); a few caches (fewer than
+ * half the SMs) run one kernel with each unit split over several CTAs;
+ * otherwise the split kernels run (cfg->path can force a path).  Arguments as in the
  * calls above; kept_idx (nullable, [U][B]) receives the kept indices;
  * n_kept ([U], required) receives min(B, n_valid[u]), the destination's
  * n_valid for the next step.

@@ -43,6 +43,7 @@ HEAD_DIM = 128
 PATH_AUTO = 0
 PATH_FUSED = 1
 PATH_SPLIT = 2
+PATH_COOP = 3
 
 # Symbols include/tri.h declares (checked by the ABI tests).
 EXPORTS = (

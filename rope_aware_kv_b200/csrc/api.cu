@@ -138,7 +138,7 @@ tri_status check_cfg(const tri_config* cfg, FoldOffsets* off) {
     if (cfg->head_dim != kD) return TRI_ERR_UNSUPPORTED;
     if (!(cfg->theta > 1.0) || cfg->n_offsets < 1 || cfg->n_offsets > TRI_MAX_OFFSETS)
         return TRI_ERR_INVALID_ARG;
-    if (cfg->path < TRI_PATH_AUTO || cfg->path > TRI_PATH_SPLIT) return TRI_ERR_INVALID_ARG;
+    if (cfg->path < TRI_PATH_AUTO || cfg->path > TRI_PATH_COOP) return TRI_ERR_INVALID_ARG;
     off->n = cfg->n_offsets;
     for (int i = 0; i < cfg->n_offsets; ++i) {
         if (cfg->offsets[i] < 0) return TRI_ERR_INVALID_ARG;
@@ -197,12 +197,21 @@ SelectWs select_ws(size_t start, int64_t U, int64_t cap) {
 }
 
 // ---- prune workspace ----
+struct CoopPlan {
+    bool ok = false;
+    int ctas_per_unit = 0, stages = 0;
+    int64_t keys_max = 0;
+};
+
 struct PruneWs {
-    bool fused;
+    bool fused = false;
+    bool coop = false;
+    CoopPlan cp;
     ScoreWs sc;
-    size_t fin, kept;
+    size_t fin = 0, kept = 0;
     SelectWs sel;
-    size_t total;
+    size_t partial = 0, hists = 0, counts = 0, bar = 0, zero_end = 0;
+    size_t total = 0;
 };
 
 // Deepest TMA ring (4..6 stages of 32 KB) the fused kernel fits in shared
@@ -218,18 +227,71 @@ bool use_fused(tri_dtype dt, int G, int64_t cap, int64_t B, int path) {
     return path == TRI_PATH_FUSED ? st >= 4 : st >= 5;
 }
 
+int64_t sm_count_or_default() {
+    const int64_t sms = device_info().sm_count;
+    return sms > 0 ? sms : 148;
+}
+
 // CTAs of the persistent fused kernel: one per SM (its shared memory allows
 // no more), never more than the units.
 int64_t fused_ctas(int64_t U) {
-    const int64_t sms = device_info().sm_count > 0 ? device_info().sm_count : 148;
+    const int64_t sms = sm_count_or_default();
     return U < sms ? U : sms;
+}
+
+// Cooperative plan: C = floor(SMs / U) CTAs per unit (at most one per key
+// tile), each with the deepest TMA ring its keys leave room for.
+CoopPlan coop_plan(tri_dtype dt, int G, int64_t U, int64_t cap) {
+    CoopPlan p;
+    const int64_t sms = sm_count_or_default();
+    const int64_t tile = coop_tile_keys(dt);
+    const int64_t tiles = (cap + tile - 1) / tile;
+    int64_t C = sms / U;
+    if (C > tiles) C = tiles;
+    if (C < 2) return p;
+    p.keys_max = ((tiles + C - 1) / C) * tile;
+    for (int st = coop_max_stages(); st >= 2; --st) {
+        if (coop_smem_bytes(dt, G, p.keys_max, st) <= fused_smem_limit()) {
+            p.stages = st;
+            break;
+        }
+    }
+    if (!p.stages) return p;
+    p.ctas_per_unit = static_cast<int>(C);
+    p.ok = true;
+    return p;
 }
 
 PruneWs prune_ws(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int64_t cap,
                  int64_t B, tri_dtype dt, bool own_kept, int path) {
     PruneWs w;
     const int64_t U = n_seq * n_layers * n_kvheads;
-    w.fused = path == TRI_PATH_SPLIT ? false : use_fused(dt, G, cap, B, path);
+    const int64_t sms = sm_count_or_default();
+    const bool fused_ok = path != TRI_PATH_SPLIT && path != TRI_PATH_COOP &&
+                          use_fused(dt, G, cap, B, path);
+    const CoopPlan cp = (path == TRI_PATH_AUTO || path == TRI_PATH_COOP)
+                            ? coop_plan(dt, G, U, cap)
+                            : CoopPlan();
+    const bool want_coop =
+        path == TRI_PATH_COOP || (path == TRI_PATH_AUTO && cp.ok && (U < sms || !fused_ok));
+    if (want_coop && cp.ok) {
+        w.coop = true;
+        w.cp = cp;
+        const int64_t grid = U * cp.ctas_per_unit;
+        Carve c;
+        w.sc.wts = c.take(static_cast<size_t>(U * G) * kWHead * 4);
+        w.sc.raw = c.take(static_cast<size_t>(grid * G * cp.keys_max) * 4);
+        w.partial = c.take(static_cast<size_t>(grid * G * 2) * 8);
+        w.counts = c.take(static_cast<size_t>(grid) * 8);
+        w.kept = own_kept ? c.take(static_cast<size_t>(U * B) * 4) : 0;
+        w.hists = c.take(static_cast<size_t>(3 * U) * kHistBins0 * 4);
+        w.bar = c.take(static_cast<size_t>(U) * 4);
+        w.zero_end = c.off;
+        w.total = c.off;
+        return w;
+    }
+    if (path == TRI_PATH_COOP) return w;  // not possible: tri_prune reports it
+    w.fused = fused_ok;
     if (w.fused) {
         Carve c;
         w.sc.wts = c.take(static_cast<size_t>(U * G) * kWHead * 4);
@@ -424,7 +486,7 @@ size_t tri_prune_workspace_bytes(int64_t n_seq, int64_t n_layers, int64_t n_kvhe
     if (check_units(n_seq, n_layers, n_kvheads, G, cap) != TRI_OK || B < 1) return kWsHeader;
     size_t best = 0;
     for (tri_dtype dt : {TRI_BF16, TRI_F32}) {
-        for (int path : {TRI_PATH_AUTO, TRI_PATH_SPLIT}) {
+        for (int path : {TRI_PATH_AUTO, TRI_PATH_SPLIT, TRI_PATH_COOP}) {
             const size_t t = prune_ws(n_seq, n_layers, n_kvheads, G, cap, B, dt, true, path).total;
             if (t > best) best = t;
         }
@@ -464,11 +526,46 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
     const PruneWs w =
         prune_ws(n_seq, n_layers, n_kvheads, G, cap_src, B, dt, kept_idx == nullptr, cfg->path);
     if (cfg->path == TRI_PATH_FUSED && !w.fused) return TRI_ERR_UNSUPPORTED;
+    if (cfg->path == TRI_PATH_COOP && !w.coop) return TRI_ERR_UNSUPPORTED;
     if (!ws || !aligned16(ws) || ws_bytes < w.total) return TRI_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     float* wts = reinterpret_cast<float*>(ws_at(ws, w.sc.wts));
     int32_t* kept = kept_idx ? kept_idx : reinterpret_cast<int32_t*>(ws_at(ws, w.kept));
     uint32_t* flag = ws_flag(ws);
+
+    if (w.coop) {
+        CUtensorMap map;
+        TRI_TRY(make_key_map(&map, k_src, dt, U * cap_src, coop_tile_keys(dt)));
+        TRI_CUDA(cudaMemsetAsync(ws, 0, kWsHeader, s));
+        TRI_CUDA(cudaMemsetAsync(ws_at(ws, w.hists), 0, w.zero_end - w.hists, s));
+        TRI_CUDA(launch_fold(stats, p_cur, n_seq, n_layers, n_kvheads * G, cfg->theta, off, wts, s));
+        CoopArgs a;
+        a.n_units = U;
+        a.cap = cap_src;
+        a.cap_dst = cap_dst;
+        a.B = B;
+        a.keys_max = w.cp.keys_max;
+        a.stages = w.cp.stages;
+        a.ctas_per_unit = w.cp.ctas_per_unit;
+        a.n_valid = n_valid;
+        a.wts = wts;
+        a.k_src = k_src;
+        a.v_src = v_src;
+        a.pos_src = pos_src;
+        a.k_dst = k_dst;
+        a.v_dst = v_dst;
+        a.pos_dst = pos_dst;
+        a.kept = kept_idx;
+        a.n_kept = n_kept;
+        a.scratch = reinterpret_cast<float*>(ws_at(ws, w.sc.raw));
+        a.partial = reinterpret_cast<double*>(ws_at(ws, w.partial));
+        a.hists = reinterpret_cast<uint32_t*>(ws_at(ws, w.hists));
+        a.counts = reinterpret_cast<uint2*>(ws_at(ws, w.counts));
+        a.bar = reinterpret_cast<uint32_t*>(ws_at(ws, w.bar));
+        a.flag = flag;
+        return cuda_status(
+            launch_coop(dt, G, map, a, static_cast<int>(U * w.cp.ctas_per_unit), s));
+    }
 
     if (w.fused) {
         CUtensorMap map;

@@ -1,0 +1,531 @@
+// coop.cu -- one prune step of a few large caches in a single kernel: every
+// unit (one KV head's cache) is split over C consecutive CTAs, one per SM, and
+// the CTAs of a unit meet at five unit-wide barriers.
+//
+// Same definitions as the other paths: the folded S~ per query head (talk
+// page: S_trig, S_norm, S~), z-score per head and max over the GQA group
+// (hyper.ai summary, Method section), top-B by (score desc, index asc) kept
+// in temporal order (jaedaily.cn tutorial, eviction step).
+//
+//   phase 1  score the CTA's tiles (TMA ring, one math warp per 128-key tile,
+//            all heads) into an L2-resident per-CTA scratch; float64 moment
+//            partial per CTA                                   -> barrier 1
+//   phase 2  fixed-order merge of the unit's partials; final = max_h z_h of
+//            the CTA's keys into shared memory; digit-0 histogram added to
+//            the unit's global histogram                       -> barrier 2
+//   phase 3  digit-1 histogram of the keys in the digit-0 bin  -> barrier 3
+//   phase 4  digit-2 histogram                                 -> barrier 4
+//   phase 5  the CTA's counts above / equal to the threshold   -> barrier 5
+//   phase 6  fixed-order prefix over the unit's CTAs, ordered compaction of
+//            the CTA's kept keys, gather of their K / V / position rows.
+//
+// A barrier is an atomic arrival counter per unit (zeroed by the host before
+// the launch) and a bounded spin on it; every CTA of the grid is resident (one
+// per SM, grid <= SMs), and a spin that exceeds its time limit raises
+// TRI_FLAG_TIMEOUT and makes the CTA skip the remaining phases, so a fault
+// elsewhere cannot hang the GPU.
+#include "select_core.cuh"
+#include "score_core.cuh"
+#include "tri_internal.cuh"
+#include "tri_launch.h"
+
+namespace tri {
+
+template <typename T>
+struct CoopShape {
+    static constexpr int kRowBytes = kD * static_cast<int>(sizeof(T));
+    static constexpr int kBoxes = kRowBytes / 128;
+    static constexpr int kKPT = sizeof(T) == 2 ? 4 : 2;
+    static constexpr int kTile = 32 * kKPT;
+    static constexpr int kBoxBytes = kTile * 128;
+    static constexpr int kStageBytes = kTile * kRowBytes;  // 32 KB
+    static constexpr int kMaxStages = 6;
+    static constexpr int kMath = 128;
+    static constexpr int kThreads = kMath + 32;
+    static constexpr int kWarps = kThreads / 32;
+};
+
+struct CoopLayout {
+    size_t w, fin, list, bars, red, misc, total;
+};
+
+template <typename T>
+__host__ __device__ inline CoopLayout coop_layout(int G, int64_t keys_max, int stages) {
+    using S = CoopShape<T>;
+    CoopLayout L;
+    const int64_t kp = (keys_max + 3) & ~int64_t(3);
+    L.w = static_cast<size_t>(stages) * S::kStageBytes;
+    L.fin = L.w + static_cast<size_t>(G) * kWHead * 4;
+    L.list = L.fin + static_cast<size_t>(kp) * 4;
+    L.bars = L.list + static_cast<size_t>(kp) * 8;
+    L.red = L.bars + 2 * S::kMaxStages * 8;
+    L.misc = L.red + static_cast<size_t>(4) * kMaxG * 2 * 8;
+    L.total = L.misc + kHistBins0 * 4 + 512 + 1024;  // histogram, state; alignment slack
+    return L;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Unit-wide barrier: arrive on the unit's counter, wait (bounded) until
+// `target` arrivals.  Returns false, for every thread of the CTA, if this or
+// an earlier barrier gave up.
+__device__ __forceinline__ bool unit_barrier(uint32_t* ctr, uint32_t target, uint32_t* flag,
+                                             int* abort_flag) {
+    __threadfence();  // this thread's global writes before the arrival
+    __syncthreads();
+    if (threadIdx.x == 0 && !*abort_flag) {
+        __threadfence();
+        atomicAdd(ctr, 1u);
+        const uint64_t t0 = globaltimer_ns();
+        while (ld_acquire_u32(ctr) < target) {
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                raise_flag(flag, TRI_FLAG_TIMEOUT);
+                *abort_flag = 1;
+                break;
+            }
+            __nanosleep(64);
+        }
+        __threadfence();
+    }
+    __syncthreads();
+    return !*abort_flag;
+}
+
+template <typename T, int G>
+__global__ void __launch_bounds__(CoopShape<T>::kThreads, 1)
+prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
+    using S = CoopShape<T>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const CoopLayout L = coop_layout<T>(G, a.keys_max, a.stages);
+    uint8_t* ring = base;
+    float* w = reinterpret_cast<float*>(base + L.w);
+    float* fin = reinterpret_cast<float*>(base + L.fin);
+    int2* list = reinterpret_cast<int2*>(base + L.list);
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + L.bars);
+    uint64_t* empty = full + S::kMaxStages;
+    double* red = reinterpret_cast<double*>(base + L.red);  // [4 warps][kMaxG][2]
+    uint32_t* hist = reinterpret_cast<uint32_t*>(base + L.misc);
+    SelState* st = reinterpret_cast<SelState*>(base + L.misc + kHistBins0 * 4);
+    float2* mom = reinterpret_cast<float2*>(base + L.misc + kHistBins0 * 4 + 16);   // [kMaxG]
+    uint32_t* wcnt = reinterpret_cast<uint32_t*>(base + L.misc + kHistBins0 * 4 + 80);  // [5][2]
+    uint32_t* bases = wcnt + 16;                                            // [2]
+    int* abort_flag = reinterpret_cast<int*>(bases + 4);
+    int* nlist = abort_flag + 1;
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int C = a.ctas_per_unit;
+    const int64_t u = blockIdx.x / C;
+    const int c = blockIdx.x % C;
+    const int64_t B = a.B;
+    const int n = clamp_nvalid(a.n_valid, u, a.cap, (tid == 0 && c == 0) ? a.flag : nullptr);
+    const int m = static_cast<int>(n < B ? n : B);
+    const bool keep_all = n <= B;
+    const int T_u = (n + S::kTile - 1) / S::kTile;
+    const int t0 = static_cast<int>(static_cast<int64_t>(c) * T_u / C);
+    const int t1 = static_cast<int>(static_cast<int64_t>(c + 1) * T_u / C);
+    const int j0 = t0 * S::kTile;                       // first key of this CTA
+    const int j1 = min(t1 * S::kTile, n);               // one past the last
+    const int nk = max(j1 - j0, 0);
+    float* scratch = a.scratch + static_cast<int64_t>(blockIdx.x) * G * a.keys_max;
+    uint32_t* ctr = a.bar + u;
+
+    if (tid == 0) {
+        *abort_flag = 0;
+        *nlist = 0;
+    }
+    if (keep_all) {
+        // Every valid key is kept: rows j0..j1-1 go to the same rows.
+        __syncthreads();
+        if (a.kept) {
+            for (int j = j0 + tid; j < j1; j += S::kThreads) a.kept[u * B + j] = j;
+            if (c == C - 1)
+                for (int64_t r = m + tid; r < B; r += S::kThreads) a.kept[u * B + r] = -1;
+        }
+        for (int j = tid; j < nk; j += S::kThreads) list[j] = make_int2(j0 + j, j0 + j);
+        if (tid == 0) *nlist = nk;
+        if (c == 0 && tid == 0) a.n_kept[u] = m;
+    } else {
+        // ---------------- phase 1: score ----------------
+        if (tid == S::kMath) {
+            for (int i = 0; i < a.stages; ++i) {
+                mbar_init(&full[i], 1);
+                mbar_init(&empty[i], 32);
+            }
+            fence_barrier_init();
+            prefetch_tensormap(&kmap);
+        }
+        {
+            const float4* src = reinterpret_cast<const float4*>(a.wts + u * G * kWHead);
+            float4* dst = reinterpret_cast<float4*>(w);
+            for (int e = tid; e < G * kWHead / 4; e += S::kThreads) dst[e] = src[e];
+        }
+        __syncthreads();
+        const int nt = t1 - t0;
+        if (tid >= S::kMath) {
+            if (tid == S::kMath) {
+                for (int l = 0; l < nt; ++l) {
+                    const int stage = l % a.stages;
+                    if (!mbar_wait(&empty[stage], ((l / a.stages) & 1) ^ 1, a.flag)) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
+                    const int32_t y = static_cast<int32_t>(u * a.cap + static_cast<int64_t>(t0 + l) * S::kTile);
+#pragma unroll
+                    for (int b = 0; b < S::kBoxes; ++b)
+                        tma_load_2d(ring + stage * S::kStageBytes + b * S::kBoxBytes, &kmap,
+                                    &full[stage], b * (128 / static_cast<int>(sizeof(T))), y);
+                }
+            }
+        } else {
+            double m1[G], m2[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) m1[h] = m2[h] = 0.0;
+            for (int l = warp; l < nt; l += 4) {
+                const int stage = l % a.stages;
+                if (!mbar_wait(&full[stage], (l / a.stages) & 1, a.flag)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                float s[S::kKPT][G];
+                score_rows<T, G, S::kKPT, S::kBoxBytes, 32>(ring + stage * S::kStageBytes, w, lane, s);
+                __syncwarp();
+                mbar_arrive(&empty[stage]);
+#pragma unroll
+                for (int k = 0; k < S::kKPT; ++k) {
+                    const int jl = l * S::kTile + lane + 32 * k;  // local key index
+                    if (j0 + jl < n) {
+#pragma unroll
+                        for (int h = 0; h < G; ++h) {
+                            scratch[static_cast<int64_t>(h) * a.keys_max + jl] = s[k][h];
+                            const double d = s[k][h];
+                            m1[h] += d;
+                            m2[h] = fma(d, d, m2[h]);
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    m1[h] += __shfl_down_sync(0xffffffffu, m1[h], o);
+                    m2[h] += __shfl_down_sync(0xffffffffu, m2[h], o);
+                }
+                if (lane == 0) {
+                    red[(warp * kMaxG + h) * 2] = m1[h];
+                    red[(warp * kMaxG + h) * 2 + 1] = m2[h];
+                }
+            }
+        }
+        __syncthreads();
+        if (tid < G) {
+            const int h = tid;
+            double* part = a.partial + ((u * C + c) * G + h) * 2;
+            part[0] = ((red[(0 * kMaxG + h) * 2] + red[(1 * kMaxG + h) * 2]) +
+                       red[(2 * kMaxG + h) * 2]) + red[(3 * kMaxG + h) * 2];
+            part[1] = ((red[(0 * kMaxG + h) * 2 + 1] + red[(1 * kMaxG + h) * 2 + 1]) +
+                       red[(2 * kMaxG + h) * 2 + 1]) + red[(3 * kMaxG + h) * 2 + 1];
+        }
+        if (!unit_barrier(ctr, 1u * C, a.flag, abort_flag)) return;
+
+        // ---------------- phase 2: moments, final, digit 0 ----------------
+        // Warp w merges heads w, w + 5, ...: lane l sums CTAs l, l + 32, ...
+        // in order, then a fixed shuffle tree; lane 0's value is used.
+        for (int h = warp; h < G; h += S::kWarps) {
+            double s1 = 0.0, s2 = 0.0;
+            for (int cc = lane; cc < C; cc += 32) {
+                const double* part = a.partial + ((u * C + cc) * G + h) * 2;
+                s1 += part[0];
+                s2 += part[1];
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                s1 += __shfl_down_sync(0xffffffffu, s1, o);
+                s2 += __shfl_down_sync(0xffffffffu, s2, o);
+            }
+            if (lane == 0) {
+                const double mu = s1 / n;
+                double var = s2 / n - mu * mu;
+                if (var < 0.0) var = 0.0;
+                const double sd = sqrt(var);
+                float inv = sd > 0.0 ? static_cast<float>(1.0 / sd) : 0.f;
+                if (!(sd == sd)) inv = __int_as_float(0x7fc00000);
+                mom[h] = make_float2(static_cast<float>(mu), inv);
+            }
+        }
+        for (int b = tid; b < kHistBins0; b += S::kThreads) hist[b] = 0;
+        __syncthreads();
+        {
+            float mu[G], inv[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                mu[h] = mom[h].x;
+                inv[h] = mom[h].y;
+            }
+            bool nonfinite = false;
+            for (int jl = tid; jl < nk; jl += S::kThreads) {
+                float sv[G];
+#pragma unroll
+                for (int h = 0; h < G; ++h) sv[h] = scratch[static_cast<int64_t>(h) * a.keys_max + jl];
+                float best = 0.f;
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float z = (sv[h] - mu[h]) * inv[h];
+                    best = (h == 0) ? z : fmaxf(best, z);
+                }
+                fin[jl] = best;
+                if (best != best) nonfinite = true;
+                atomicAdd(&hist[ordered_key(best) >> pass_shift(0)], 1u);
+            }
+            if (nonfinite) raise_flag(a.flag, TRI_FLAG_NONFINITE);
+        }
+        __syncthreads();
+        {
+            uint32_t* g = a.hists + u * kHistBins0;
+            for (int b = tid; b < kHistBins0; b += S::kThreads)
+                if (hist[b]) atomicAdd(&g[b], hist[b]);
+        }
+        if (!unit_barrier(ctr, 2u * C, a.flag, abort_flag)) return;
+
+        // ---------------- phases 3 and 4: digits 1 and 2 ----------------
+        if (warp == 0) {
+            uint32_t bin, above;
+            warp_find_bin(a.hists + u * kHistBins0, 1 << pass_bits(0), static_cast<uint32_t>(B),
+                          bin, above);
+            if (lane == 0) {
+                st->prefix = bin;
+                st->k = static_cast<uint32_t>(B) - above;
+                st->gt = above;
+                st->keep_all = 0;
+            }
+        }
+        for (int p = 1; p < 3; ++p) {
+            const int nb = 1 << pass_bits(p);
+            for (int b = tid; b < nb; b += S::kThreads) hist[b] = 0;
+            __syncthreads();
+            const uint32_t prefix = st->prefix;
+            const int shift = pass_shift(p);
+            const int hi_shift = shift + pass_bits(p);
+            for (int jl = tid; jl < nk; jl += S::kThreads) {
+                const uint32_t key = ordered_key(fin[jl]);
+                if ((key >> hi_shift) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+            }
+            __syncthreads();
+            uint32_t* g = a.hists + (static_cast<int64_t>(p) * a.n_units + u) * kHistBins0;
+            for (int b = tid; b < nb; b += S::kThreads)
+                if (hist[b]) atomicAdd(&g[b], hist[b]);
+            if (!unit_barrier(ctr, (2u + p) * C, a.flag, abort_flag)) return;
+            if (warp == 0) {
+                uint32_t bin, above;
+                warp_find_bin(g, nb, st->k, bin, above);
+                if (lane == 0) {
+                    st->prefix = (prefix << pass_bits(p)) | bin;
+                    st->k -= above;
+                    st->gt += above;
+                }
+            }
+            __syncthreads();
+        }
+
+        // ---------------- phase 5: the CTA's counts ----------------
+        const uint32_t Tk = st->prefix, kt = st->k;
+        {
+            uint32_t gt = 0, eq = 0;
+            for (int jl = tid; jl < nk; jl += S::kThreads) {
+                const uint32_t key = ordered_key(fin[jl]);
+                gt += key > Tk;
+                eq += key == Tk;
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                gt += __shfl_xor_sync(0xffffffffu, gt, o);
+                eq += __shfl_xor_sync(0xffffffffu, eq, o);
+            }
+            if (lane == 0) {
+                wcnt[2 * warp] = gt;
+                wcnt[2 * warp + 1] = eq;
+            }
+            __syncthreads();
+            if (tid == 0) {
+                uint32_t g2 = 0, e2 = 0;
+                for (int v = 0; v < S::kWarps; ++v) {
+                    g2 += wcnt[2 * v];
+                    e2 += wcnt[2 * v + 1];
+                }
+                a.counts[u * C + c] = make_uint2(g2, e2);
+            }
+        }
+        if (!unit_barrier(ctr, 5u * C, a.flag, abort_flag)) return;
+
+        // ---------------- phase 6: ordered compaction ----------------
+        if (warp == 0) {
+            uint32_t gsum = 0, esum = 0;
+            for (int cc = lane; cc < c; cc += 32) {
+                const uint2 v = a.counts[u * C + cc];
+                gsum += v.x;
+                esum += v.y;
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                gsum += __shfl_xor_sync(0xffffffffu, gsum, o);
+                esum += __shfl_xor_sync(0xffffffffu, esum, o);
+            }
+            if (lane == 0) {
+                bases[0] = gsum + min(esum, kt);  // kept before this CTA
+                bases[1] = esum;                  // ties before this CTA
+            }
+        }
+        __syncthreads();
+        {
+            const int seg = ((nk + S::kWarps * 32 - 1) / (S::kWarps * 32)) * 32;
+            const int l0 = warp * seg;
+            const int l1 = min(l0 + seg, nk);
+            uint32_t gt = 0, eq = 0;
+            for (int jl = l0 + lane; jl - lane < l1; jl += 32) {
+                const bool valid = jl < l1;
+                const uint32_t key = valid ? ordered_key(fin[jl]) : 0u;
+                gt += __popc(__ballot_sync(0xffffffffu, valid && key > Tk));
+                eq += __popc(__ballot_sync(0xffffffffu, valid && key == Tk));
+            }
+            if (lane == 0) {
+                wcnt[2 * warp] = gt;
+                wcnt[2 * warp + 1] = eq;
+            }
+            __syncthreads();
+            uint32_t pos = bases[0], ties = bases[1];
+            uint32_t lpos = 0;  // kept before this warp within the CTA
+            for (int v = 0; v < warp; ++v) {
+                const uint32_t take = ties < kt ? min(wcnt[2 * v + 1], kt - ties) : 0u;
+                lpos += wcnt[2 * v] + take;
+                ties += wcnt[2 * v + 1];
+            }
+            pos += lpos;
+            const uint32_t lt = (1u << lane) - 1u;
+            for (int jl = l0 + lane; jl - lane < l1; jl += 32) {
+                const bool valid = jl < l1;
+                const uint32_t key = valid ? ordered_key(fin[jl]) : 0u;
+                const bool is_eq = valid && key == Tk;
+                const uint32_t beq = __ballot_sync(0xffffffffu, is_eq);
+                const uint32_t my_tie = ties + __popc(beq & lt);
+                const bool keep = valid && (key > Tk || (is_eq && my_tie < kt));
+                const uint32_t bk = __ballot_sync(0xffffffffu, keep);
+                if (keep) {
+                    const uint32_t r = pos + __popc(bk & lt);
+                    const uint32_t lr = lpos + __popc(bk & lt);
+                    if (r < static_cast<uint32_t>(m) && lr < static_cast<uint32_t>(nk)) {
+                        list[lr] = make_int2(j0 + jl, static_cast<int>(r));
+                        if (a.kept) a.kept[u * B + r] = j0 + jl;
+                    }
+                }
+                pos += __popc(bk);
+                lpos += __popc(bk);
+                ties += __popc(beq);
+            }
+            if (warp == S::kWarps - 1 && lane == 0) *nlist = static_cast<int>(lpos);
+        }
+        if (c == 0 && tid == 0) a.n_kept[u] = m;
+    }
+    __syncthreads();
+
+    // ---------------- gather of this CTA's kept rows ----------------
+    {
+        constexpr int kVec = S::kRowBytes / 16;
+        constexpr int kGroups = S::kThreads / kVec;
+        constexpr int kBatch = 8;
+        const int cnt = *nlist;
+        const int l = tid % kVec;
+        const int g = tid / kVec;
+        const uint4* ks = static_cast<const uint4*>(a.k_src);
+        const uint4* vs = static_cast<const uint4*>(a.v_src);
+        uint4* kd = static_cast<uint4*>(a.k_dst);
+        uint4* vd = static_cast<uint4*>(a.v_dst);
+        if (g < kGroups) {
+            for (int e0 = 0; e0 < cnt; e0 += kGroups * kBatch) {
+                uint4 kv[kBatch], vv[kBatch];
+                int2 jr[kBatch];
+#pragma unroll
+                for (int q = 0; q < kBatch; ++q) {
+                    const int e = e0 + q * kGroups + g;
+                    jr[q] = e < cnt ? list[e] : make_int2(-1, -1);
+                    if (jr[q].x >= n || jr[q].y >= m) jr[q].x = -1;  // cannot happen
+                }
+#pragma unroll
+                for (int q = 0; q < kBatch; ++q) {
+                    if (jr[q].x >= 0) {
+                        const int64_t srow = u * a.cap + jr[q].x;
+                        kv[q] = ld_stream(ks + srow * kVec + l);
+                        if (vs) vv[q] = ld_stream(vs + srow * kVec + l);
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < kBatch; ++q) {
+                    if (jr[q].x >= 0) {
+                        const int64_t drow = u * a.cap_dst + jr[q].y;
+                        st_stream(kd + drow * kVec + l, kv[q]);
+                        if (vd) st_stream(vd + drow * kVec + l, vv[q]);
+                        if (a.pos_dst && l == 0) a.pos_dst[drow] = a.pos_src[u * a.cap + jr[q].x];
+                    }
+                }
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+size_t coop_smem_bytes(tri_dtype dt, int G, int64_t keys_max, int stages) {
+    return dt == TRI_BF16 ? coop_layout<__nv_bfloat16>(G, keys_max, stages).total
+                          : coop_layout<float>(G, keys_max, stages).total;
+}
+
+int coop_tile_keys(tri_dtype dt) {
+    return dt == TRI_BF16 ? CoopShape<__nv_bfloat16>::kTile : CoopShape<float>::kTile;
+}
+
+int coop_max_stages() { return CoopShape<float>::kMaxStages; }
+
+template <typename T, int G>
+static cudaError_t launch_coop_t(const CUtensorMap& map, const CoopArgs& a, int n_ctas,
+                                 cudaStream_t s) {
+    const size_t smem = coop_layout<T>(G, a.keys_max, a.stages).total;
+    auto kern = prune_coop_kernel<T, G>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    kern<<<n_ctas, CoopShape<T>::kThreads, smem, s>>>(map, a);
+    note_launch(s);
+    return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_coop_g(int G, const CUtensorMap& map, const CoopArgs& a, int n_ctas,
+                                 cudaStream_t s) {
+    switch (G) {
+        case 1: return launch_coop_t<T, 1>(map, a, n_ctas, s);
+        case 2: return launch_coop_t<T, 2>(map, a, n_ctas, s);
+        case 3: return launch_coop_t<T, 3>(map, a, n_ctas, s);
+        case 4: return launch_coop_t<T, 4>(map, a, n_ctas, s);
+        case 5: return launch_coop_t<T, 5>(map, a, n_ctas, s);
+        case 6: return launch_coop_t<T, 6>(map, a, n_ctas, s);
+        case 7: return launch_coop_t<T, 7>(map, a, n_ctas, s);
+        case 8: return launch_coop_t<T, 8>(map, a, n_ctas, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_coop(tri_dtype dt, int G, const CUtensorMap& map, const CoopArgs& a,
+                        int n_ctas, cudaStream_t s) {
+    if (dt == TRI_BF16) return launch_coop_g<__nv_bfloat16>(G, map, a, n_ctas, s);
+    return launch_coop_g<float>(G, map, a, n_ctas, s);
+}
+
+}  // namespace tri

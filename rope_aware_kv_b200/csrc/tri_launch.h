@@ -53,6 +53,32 @@ struct FusedArgs {
     uint32_t* flag;
 };
 
+struct CoopArgs {
+    int64_t n_units;
+    int64_t cap;
+    int64_t cap_dst;
+    int64_t B;
+    int64_t keys_max;            // most keys one CTA takes
+    int stages;                  // TMA ring depth
+    int ctas_per_unit;           // C
+    const int32_t* n_valid;
+    const float* wts;            // [U*G][192]
+    const void* k_src;
+    const void* v_src;
+    const int32_t* pos_src;
+    void* k_dst;
+    void* v_dst;
+    int32_t* pos_dst;
+    int32_t* kept;               // [U][B] or null
+    int32_t* n_kept;             // [U]
+    float* scratch;              // [grid][G][keys_max]
+    double* partial;             // [U][C][G][2]
+    uint32_t* hists;             // [3][U][2048], zero on entry
+    uint2* counts;               // [U][C]
+    uint32_t* bar;               // [U], zero on entry
+    uint32_t* flag;
+};
+
 constexpr int kTracePoints = 8;  // per unit: start, scored, z-max, selected, gathered
 constexpr int kTraceWarps = 8;   // one slot per warp of the fused kernel
 
@@ -97,6 +123,13 @@ cudaError_t launch_append(tri_dtype dt, void* k_cache, void* v_cache, int32_t* p
                           int64_t n_seq, int64_t n_units, int64_t cap, int32_t* n_valid,
                           int64_t* p_cur, const void* k_new, const void* v_new,
                           const int32_t* pos_new, int64_t n_new, uint32_t* flag, cudaStream_t s);
+
+// coop.cu
+size_t coop_smem_bytes(tri_dtype dt, int G, int64_t keys_max, int stages);
+int coop_tile_keys(tri_dtype dt);
+int coop_max_stages();
+cudaError_t launch_coop(tri_dtype dt, int G, const CUtensorMap& map, const CoopArgs& a,
+                        int n_ctas, cudaStream_t s);
 
 // fused.cu
 size_t fused_smem_bytes(tri_dtype dt, int G, int64_t cap, int64_t B, int stages);

@@ -236,7 +236,7 @@ def _oracle_units(spec, wl, ost, B, nv, units):
     return dict(final=fin, kept=kept)
 
 
-@pytest.mark.parametrize("path", [tri.PATH_FUSED, tri.PATH_SPLIT])
+@pytest.mark.parametrize("path", [tri.PATH_FUSED, tri.PATH_SPLIT, tri.PATH_COOP])
 @pytest.mark.parametrize("dtype,G", [("bf16", 7), ("bf16", 4), ("bf16", 1), ("f32", 2)])
 def test_prune_parity_ragged(path, dtype, G):
     B = 300
@@ -261,11 +261,13 @@ def test_prune_paths_agree():
     gst, _ = H.stats_for(spec, wl)
     a = _run_prune(spec, wl, gst, B, path=tri.PATH_FUSED)
     b = _run_prune(spec, wl, gst, B, path=tri.PATH_SPLIT)
+    c = _run_prune(spec, wl, gst, B, path=tri.PATH_COOP)
     for u in range(spec.n_units):
-        diff = np.setxor1d(a["kept"][u], b["kept"][u])
-        assert len(diff) <= 2
-        assert H.rows_equal(a["k"][u], wl.k[u], a["kept"][u])
-        assert H.rows_equal(b["v"][u], wl.v[u], b["kept"][u])
+        for other in (b, c):
+            diff = np.setxor1d(a["kept"][u], other["kept"][u])
+            assert len(diff) <= 2
+            assert H.rows_equal(other["k"][u], wl.k[u], other["kept"][u])
+            assert H.rows_equal(other["v"][u], wl.v[u], other["kept"][u])
 
 
 @pytest.mark.parametrize("name,sample", [("c1", None), ("c2", None), ("c3", 24)])
@@ -284,12 +286,13 @@ def test_prune_parity_config(name, sample):
     assert mismatched <= 2 * len(units)
 
 
-def test_prune_deterministic():
+@pytest.mark.parametrize("path", [tri.PATH_AUTO, tri.PATH_SPLIT])
+def test_prune_deterministic(path):
     spec = synth.SPECS["c2"]
     wl = synth.make_workload(spec, "cuda")
     gst, _ = H.stats_for(spec, wl)
-    a = _run_prune(spec, wl, gst, spec.B)
-    b = _run_prune(spec, wl, gst, spec.B)
+    a = _run_prune(spec, wl, gst, spec.B, path=path)
+    b = _run_prune(spec, wl, gst, spec.B, path=path)
     np.testing.assert_array_equal(a["kept"], b["kept"])
     assert torch.equal(a["k"], b["k"]) and torch.equal(a["v"], b["v"]) and torch.equal(a["pos"], b["pos"])
 
@@ -297,7 +300,7 @@ def test_prune_deterministic():
 # ---------------------------------------------------------------------------
 # edge cases
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("path", [tri.PATH_FUSED, tri.PATH_SPLIT])
+@pytest.mark.parametrize("path", [tri.PATH_FUSED, tri.PATH_SPLIT, tri.PATH_COOP])
 def test_identical_keys_keep_lowest_indices(path):
     """All keys equal: every head has sigma = 0, every z is 0, all scores tie,
     and the lowest B indices are kept."""
@@ -309,7 +312,7 @@ def test_identical_keys_keep_lowest_indices(path):
     assert np.all(out["kept"] == np.arange(123)[None, :])
 
 
-@pytest.mark.parametrize("path", [tri.PATH_FUSED, tri.PATH_SPLIT])
+@pytest.mark.parametrize("path", [tri.PATH_FUSED, tri.PATH_SPLIT, tri.PATH_COOP])
 def test_nan_key_poisons_unit_and_flags(path):
     """A NaN key makes that unit's moments NaN: every final score is NaN,
     NaN ranks last and ties go to the lowest indices; the flag is raised.

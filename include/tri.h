@@ -319,8 +319,11 @@ int tri_last_launch_count(void);
  * device_buf[(u * 8 + p) * 8 + w] (uint64): lane 0 of warp w records phase
  * point p of unit u just before the barrier that ends the phase, so a phase
  * ends at the largest w entry.  p = 0: start of the unit; 1: scored;
- * 2: z-max done; 3: selected; 4: gathered.  Units a call does not reach
- * through the fused kernel are left untouched.  Pass (NULL, 0) to stop.
+ * 2: z-max done; 3: selected; 4: gathered.  The cooperative kernel (a few
+ * units, each split over several CTAs) indexes by CTA instead of unit and
+ * needs grid * 512 bytes: points 0 start, 1 scored, 2 after the first unit
+ * barrier, 3 z-max done, 4 after the second barrier, 5 after the last
+ * barrier, 6 compaction done, 7 gather done.  Pass (NULL, 0) to stop.
  */
 tri_status tri_set_phase_trace(void* device_buf, size_t bytes);
 

@@ -562,6 +562,7 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
         a.hists = reinterpret_cast<uint32_t*>(ws_at(ws, w.hists));
         a.counts = reinterpret_cast<uint2*>(ws_at(ws, w.counts));
         a.bar = reinterpret_cast<uint32_t*>(ws_at(ws, w.bar));
+        a.trace = phase_trace_buffer(U * w.cp.ctas_per_unit);
         a.flag = flag;
         return cuda_status(
             launch_coop(dt, G, map, a, static_cast<int>(U * w.cp.ctas_per_unit), s));

@@ -95,6 +95,13 @@ __device__ __forceinline__ bool unit_barrier(uint32_t* ctr, uint32_t target, uin
     return !*abort_flag;
 }
 
+// Phase trace by CTA: lane 0 of every warp records %globaltimer at point i.
+__device__ __forceinline__ void coop_trace(const CoopArgs& a, int i) {
+    if (a.trace && (threadIdx.x & 31) == 0)
+        a.trace[(static_cast<int64_t>(blockIdx.x) * kTracePoints + i) * kTraceWarps +
+                (threadIdx.x >> 5)] = globaltimer_ns();
+}
+
 template <typename T, int G>
 __global__ void __launch_bounds__(CoopShape<T>::kThreads, 1)
 prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
@@ -140,6 +147,7 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
         *abort_flag = 0;
         *nlist = 0;
     }
+    coop_trace(a, 0);
     if (keep_all) {
         // Every valid key is kept: rows j0..j1-1 go to the same rows.
         __syncthreads();
@@ -234,7 +242,9 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
             part[1] = ((red[(0 * kMaxG + h) * 2 + 1] + red[(1 * kMaxG + h) * 2 + 1]) +
                        red[(2 * kMaxG + h) * 2 + 1]) + red[(3 * kMaxG + h) * 2 + 1];
         }
+        coop_trace(a, 1);
         if (!unit_barrier(ctr, 1u * C, a.flag, abort_flag)) return;
+        coop_trace(a, 2);
 
         // ---------------- phase 2: moments, final, digit 0 ----------------
         // Warp w merges heads w, w + 5, ...: lane l sums CTAs l, l + 32, ...
@@ -293,7 +303,9 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
             for (int b = tid; b < kHistBins0; b += S::kThreads)
                 if (hist[b]) atomicAdd(&g[b], hist[b]);
         }
+        coop_trace(a, 3);
         if (!unit_barrier(ctr, 2u * C, a.flag, abort_flag)) return;
+        coop_trace(a, 4);
 
         // ---------------- phases 3 and 4: digits 1 and 2 ----------------
         if (warp == 0) {
@@ -364,6 +376,7 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
             }
         }
         if (!unit_barrier(ctr, 5u * C, a.flag, abort_flag)) return;
+        coop_trace(a, 5);
 
         // ---------------- phase 6: ordered compaction ----------------
         if (warp == 0) {
@@ -433,6 +446,7 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
         }
         if (c == 0 && tid == 0) a.n_kept[u] = m;
     }
+    coop_trace(a, 6);
     __syncthreads();
 
     // ---------------- gather of this CTA's kept rows ----------------
@@ -477,6 +491,7 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
             }
         }
     }
+    coop_trace(a, 7);
 }
 
 // ---------------------------------------------------------------------------

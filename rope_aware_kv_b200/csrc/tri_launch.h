@@ -53,6 +53,9 @@ struct FusedArgs {
     uint32_t* flag;
 };
 
+constexpr int kTracePoints = 8;  // phase points per unit (fused) or CTA (coop)
+constexpr int kTraceWarps = 8;   // one slot per warp
+
 struct CoopArgs {
     int64_t n_units;
     int64_t cap;
@@ -76,11 +79,10 @@ struct CoopArgs {
     uint32_t* hists;             // [3][U][2048], zero on entry
     uint2* counts;               // [U][C]
     uint32_t* bar;               // [U], zero on entry
+    uint64_t* trace;             // [grid][kTracePoints][kTraceWarps] or null
     uint32_t* flag;
 };
 
-constexpr int kTracePoints = 8;  // per unit: start, scored, z-max, selected, gathered
-constexpr int kTraceWarps = 8;   // one slot per warp of the fused kernel
 
 // api.cu: the caller's phase-trace buffer for the next launches (or null).
 uint64_t* phase_trace_buffer(int64_t n_units);

@@ -400,10 +400,13 @@ def run_tri(args, ws, rank, local):
     step_gbs = comp / (ms_step * 1e-3) / 1e9
 
     # Dominant kernel and its algorithmic bytes.
+    path = tri.tri_prune_path(spec.n_seq, spec.n_layers, spec.n_kvheads, spec.G, spec.cap, spec.B,
+                              spec.torch_dtype)
     dom = int(np.argmax(per_launch))
-    fused = launches <= 2
-    if fused:
-        dom_name, dom_bytes = "prune_fused_kernel", fused_bytes(spec)
+    if path in (tri.PATH_FUSED, tri.PATH_COOP):
+        names = ["fold", "prune_fused_kernel" if path == tri.PATH_FUSED else "prune_coop_kernel"]
+        dom_name = names[dom] if dom < len(names) else f"launch{dom}"
+        dom_bytes = fused_bytes(spec) if dom == 1 else 0
     else:
         names = ["fold", "score", "zmax_hist", "radix_pass1", "radix_pass2", "select_count",
                  "select_compact", "gather"]
@@ -440,6 +443,7 @@ def run_tri(args, ws, rank, local):
                          "frac": achieved / peak_gbs, "traffic": None,
                          "algorithmic_bytes": dom_bytes, "ms_per_launch": dom_ms},
             "per_launch_ms": [round(float(x), 5) for x in per_launch],
+            "path": {tri.PATH_FUSED: "fused", tri.PATH_COOP: "coop"}.get(path, "split"),
             "evented_ms_per_step": ev_step,
             "gpu_launches": int(launches * args.steps),
             "device_flags": flags,

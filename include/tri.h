@@ -273,6 +273,12 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
                      void* v_dst, int32_t* pos_dst, int64_t cap_dst, int32_t* kept_idx,
                      int32_t* n_kept, void* ws, size_t ws_bytes, void* stream);
 
+/* The kernel path (TRI_PATH_FUSED, TRI_PATH_COOP or TRI_PATH_SPLIT) that
+ * tri_prune takes for these shapes on the current device when cfg->path is
+ * `path`; -1 when `path` cannot serve them or the shapes are invalid. */
+int tri_prune_path(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int64_t cap,
+                   int64_t B, tri_dtype dt, int path);
+
 /* ---------------------------------------------------------------------- */
 /* Streaming helper: append generated tokens                               */
 /* ---------------------------------------------------------------------- */

@@ -55,7 +55,7 @@ EXPORTS = (
     "tri_prune_workspace_bytes", "tri_prune",
     "tri_append", "tri_check_device_error",
     "tri_set_timing_events", "tri_last_launch_count", "tri_set_phase_trace",
-    "tri_select_topB_static", "tri_select_static_scratch_bytes",
+    "tri_select_topB_static", "tri_select_static_scratch_bytes", "tri_prune_path",
 )
 
 
@@ -112,6 +112,7 @@ def load(path: Optional[str] = None):
         "tri_set_phase_trace": (i32, [P, sz]),
         "tri_select_topB_static": (i32, [P, i64, i64, P, i64, P, P, P]),
         "tri_select_static_scratch_bytes": (sz, []),
+        "tri_prune_path": (i32, [i64, i64, i64, i32, i64, i64, i32, i32]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -277,6 +278,13 @@ def tri_compact(k_src: torch.Tensor, v_src: Optional[torch.Tensor], pos_src: Opt
 
 def tri_prune_workspace_bytes(n_seq, n_layers, n_kvheads, G, cap, B, head_dim=HEAD_DIM) -> int:
     return load().tri_prune_workspace_bytes(n_seq, n_layers, n_kvheads, G, cap, B, head_dim)
+
+
+def tri_prune_path(n_seq, n_layers, n_kvheads, G, cap, B, dtype=torch.bfloat16,
+                   path: int = PATH_AUTO) -> int:
+    """Kernel path tri_prune takes for these shapes (PATH_FUSED / COOP / SPLIT)."""
+    dt = TRI_BF16 if dtype == torch.bfloat16 else TRI_F32
+    return int(load().tri_prune_path(n_seq, n_layers, n_kvheads, G, cap, B, dt, path))
 
 
 def tri_prune(cfg: TriConfig, k_src: torch.Tensor, v_src: Optional[torch.Tensor],

@@ -494,6 +494,17 @@ size_t tri_prune_workspace_bytes(int64_t n_seq, int64_t n_layers, int64_t n_kvhe
     return best;
 }
 
+int tri_prune_path(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int64_t cap,
+                   int64_t B, tri_dtype dt, int path) {
+    if (check_units(n_seq, n_layers, n_kvheads, G, cap) != TRI_OK || B < 1 || !dtype_ok(dt))
+        return -1;
+    const PruneWs w = prune_ws(n_seq, n_layers, n_kvheads, G, cap, B, dt, false, path);
+    if (w.coop) return TRI_PATH_COOP;
+    if (w.fused) return TRI_PATH_FUSED;
+    if (path == TRI_PATH_FUSED || path == TRI_PATH_COOP) return -1;
+    return TRI_PATH_SPLIT;
+}
+
 tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src,
                      const int32_t* pos_src, tri_dtype dt, int64_t n_seq, int64_t n_layers,
                      int64_t n_kvheads, int G, int64_t cap_src, const int32_t* n_valid,

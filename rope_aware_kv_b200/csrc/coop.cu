@@ -281,19 +281,31 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
                 inv[h] = mom[h].y;
             }
             bool nonfinite = false;
-            for (int jl = tid; jl < nk; jl += S::kThreads) {
-                float sv[G];
+            constexpr int kU = 4;
+            for (int j0l = tid; j0l < nk; j0l += S::kThreads * kU) {
+                float sv[kU][G];
 #pragma unroll
-                for (int h = 0; h < G; ++h) sv[h] = scratch[static_cast<int64_t>(h) * a.keys_max + jl];
-                float best = 0.f;
+                for (int q = 0; q < kU; ++q) {
+                    const int jl = j0l + q * S::kThreads;
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    const float z = (sv[h] - mu[h]) * inv[h];
-                    best = (h == 0) ? z : fmaxf(best, z);
+                    for (int h = 0; h < G; ++h)
+                        sv[q][h] = jl < nk ? scratch[static_cast<int64_t>(h) * a.keys_max + jl] : 0.f;
                 }
-                fin[jl] = best;
-                if (best != best) nonfinite = true;
-                atomicAdd(&hist[ordered_key(best) >> pass_shift(0)], 1u);
+#pragma unroll
+                for (int q = 0; q < kU; ++q) {
+                    const int jl = j0l + q * S::kThreads;
+                    if (jl < nk) {
+                        float best = 0.f;
+#pragma unroll
+                        for (int h = 0; h < G; ++h) {
+                            const float z = (sv[q][h] - mu[h]) * inv[h];
+                            best = (h == 0) ? z : fmaxf(best, z);
+                        }
+                        fin[jl] = best;
+                        if (best != best) nonfinite = true;
+                        atomicAdd(&hist[ordered_key(best) >> pass_shift(0)], 1u);
+                    }
+                }
             }
             if (nonfinite) raise_flag(a.flag, TRI_FLAG_NONFINITE);
         }
@@ -308,10 +320,17 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
         coop_trace(a, 4);
 
         // ---------------- phases 3 and 4: digits 1 and 2 ----------------
+        // The unit's histogram is read once into shared memory by every
+        // thread (16-byte loads), then scanned by one warp.
+        {
+            const uint4* g = reinterpret_cast<const uint4*>(a.hists + u * kHistBins0);
+            uint4* h4 = reinterpret_cast<uint4*>(hist);
+            for (int b = tid; b < kHistBins0 / 4; b += S::kThreads) h4[b] = ld_cg_u4(g + b);
+        }
+        __syncthreads();
         if (warp == 0) {
             uint32_t bin, above;
-            warp_find_bin(a.hists + u * kHistBins0, 1 << pass_bits(0), static_cast<uint32_t>(B),
-                          bin, above);
+            warp_find_bin(hist, 1 << pass_bits(0), static_cast<uint32_t>(B), bin, above);
             if (lane == 0) {
                 st->prefix = bin;
                 st->k = static_cast<uint32_t>(B) - above;
@@ -319,6 +338,7 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
                 st->keep_all = 0;
             }
         }
+        __syncthreads();
         for (int p = 1; p < 3; ++p) {
             const int nb = 1 << pass_bits(p);
             for (int b = tid; b < nb; b += S::kThreads) hist[b] = 0;
@@ -335,9 +355,15 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
             for (int b = tid; b < nb; b += S::kThreads)
                 if (hist[b]) atomicAdd(&g[b], hist[b]);
             if (!unit_barrier(ctr, (2u + p) * C, a.flag, abort_flag)) return;
+            {
+                const uint4* g4 = reinterpret_cast<const uint4*>(g);
+                uint4* h4 = reinterpret_cast<uint4*>(hist);
+                for (int b = tid; b < nb / 4; b += S::kThreads) h4[b] = ld_cg_u4(g4 + b);
+            }
+            __syncthreads();
             if (warp == 0) {
                 uint32_t bin, above;
-                warp_find_bin(g, nb, st->k, bin, above);
+                warp_find_bin(hist, nb, st->k, bin, above);
                 if (lane == 0) {
                     st->prefix = (prefix << pass_bits(p)) | bin;
                     st->k -= above;

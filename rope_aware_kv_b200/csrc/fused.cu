@@ -145,6 +145,8 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
             __syncthreads();
             if (tid >= S::kMath) {
                 if (tid == S::kMath) {
+                    // Keys stay in L2 for the kept-row re-read of the gather.
+                    const uint64_t keep_pol = policy_evict_last();
                     for (int i = 0; i < n_tiles; ++i) {
                         const uint32_t tc = tiles_done + i;
                         const int stage = tc % n_stages;
@@ -157,8 +159,9 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
                             static_cast<int32_t>(u * a.cap + static_cast<int64_t>(i) * S::kTile);
 #pragma unroll
                         for (int b = 0; b < S::kBoxes; ++b)
-                            tma_load_2d(regA + stage * S::kStageBytes + b * S::kBoxBytes, &kmap,
-                                        &full[stage], b * (128 / static_cast<int>(sizeof(T))), y);
+                            tma_load_2d_hint(regA + stage * S::kStageBytes + b * S::kBoxBytes,
+                                             &kmap, &full[stage],
+                                             b * (128 / static_cast<int>(sizeof(T))), y, keep_pol);
                     }
                 }
             } else {
@@ -397,7 +400,8 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
             return j >= 0 && j + len <= n && len > 0 && len <= S::kGRows;
         };
         if (tid == S::kMath) {
-            // Engine: bulk loads only.
+            // Engine: bulk loads only (last use of these rows: evict first).
+            const uint64_t last_use = policy_evict_first();
             const char* ks = static_cast<const char*>(a.k_src);
             const char* vs = static_cast<const char*>(a.v_src);
             for (int p = 0; p < npc; ++p) {
@@ -418,11 +422,29 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
                 }
                 const uint32_t bytes = static_cast<uint32_t>(len * S::kRowBytes);
                 mbar_arrive_expect_tx(&gfull[sb], bytes);
-                bulk_load(regA + sb * S::kGStage, (is_v ? vs : ks) + (u * a.cap + j) * S::kRowBytes,
-                          bytes, &gfull[sb]);
+                bulk_load_hint(regA + sb * S::kGStage,
+                               (is_v ? vs : ks) + (u * a.cap + j) * S::kRowBytes, bytes, &gfull[sb],
+                               last_use);
             }
         } else if (tid < S::kMath) {
-            // Math warps: drain pieces warp, warp + 4, ... to global memory.
+            // Math warps: positions of the kept rows (8 loads in flight per
+            // thread), then drain pieces warp, warp + 4, ... to global memory.
+            if (a.pos_dst) {
+                for (int r0 = tid; r0 < m; r0 += S::kMath * 8) {
+                    int32_t pv[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const int r = r0 + q * S::kMath;
+                        const int32_t j = r < m ? kidx[r] : -1;
+                        pv[q] = (j >= 0 && j < n) ? a.pos_src[u * a.cap + j] : 0;
+                    }
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const int r = r0 + q * S::kMath;
+                        if (r < m) a.pos_dst[u * a.cap_dst + r] = pv[q];
+                    }
+                }
+            }
             constexpr int kVec = S::kRowBytes / 16;
             uint4* kd = static_cast<uint4*>(a.k_dst);
             uint4* vd = static_cast<uint4*>(a.v_dst);
@@ -442,8 +464,6 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
                     uint4* dst = (is_v ? vd : kd) + (u * a.cap_dst + r) * kVec;
                     const int nv = len * kVec;
                     for (int e = lane; e < nv; e += 32) st_stream(dst + e, buf[e]);
-                    if (!is_v && a.pos_dst && lane < len)
-                        a.pos_dst[u * a.cap_dst + r + lane] = a.pos_src[u * a.cap + j + lane];
                 }
                 __syncwarp();
                 mbar_arrive(&gempty[sb]);

@@ -279,14 +279,14 @@ PruneWs prune_ws(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int6
         w.cp = cp;
         const int64_t grid = U * cp.ctas_per_unit;
         Carve c;
-        w.sc.wts = c.take(static_cast<size_t>(U * G) * kWHead * 4);
+        w.hists = c.take(static_cast<size_t>(3 * U) * kHistBins0 * 4);
+        w.bar = c.take(static_cast<size_t>(U) * 4);
+        w.zero_end = c.off;
+        w.sc.wts = c.take(256);
         w.sc.raw = c.take(static_cast<size_t>(grid * G * cp.keys_max) * 4);
         w.partial = c.take(static_cast<size_t>(grid * G * 2) * 8);
         w.counts = c.take(static_cast<size_t>(grid) * 8);
         w.kept = own_kept ? c.take(static_cast<size_t>(U * B) * 4) : 0;
-        w.hists = c.take(static_cast<size_t>(3 * U) * kHistBins0 * 4);
-        w.bar = c.take(static_cast<size_t>(U) * 4);
-        w.zero_end = c.off;
         w.total = c.off;
         return w;
     }
@@ -294,7 +294,7 @@ PruneWs prune_ws(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int6
     w.fused = fused_ok;
     if (w.fused) {
         Carve c;
-        w.sc.wts = c.take(static_cast<size_t>(U * G) * kWHead * 4);
+        w.sc.wts = c.take(256);
         w.sc.raw = c.take(static_cast<size_t>(fused_ctas(U) * G * cap) * 4);
         w.kept = own_kept ? c.take(static_cast<size_t>(U * B) * 4) : 0;
         w.fin = 0;
@@ -522,7 +522,7 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
         return TRI_ERR_INVALID_ARG;
     if (cap_dst < (B < cap_src ? B : cap_src)) return TRI_ERR_INVALID_ARG;
     if (!aligned16(k_src) || !aligned16(k_dst) ||
-        (v_src && (!aligned16(v_src) || !aligned16(v_dst))) || !aligned4(stats) ||
+        (v_src && (!aligned16(v_src) || !aligned16(v_dst))) || !aligned16(stats) ||
         !aligned4(n_kept) || (kept_idx && !aligned4(kept_idx)) || (n_valid && !aligned4(n_valid)))
         return TRI_ERR_INVALID_ARG;
     const int64_t U = n_seq * n_layers * n_kvheads;
@@ -547,11 +547,16 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
     if (w.coop) {
         CUtensorMap map;
         TRI_TRY(make_key_map(&map, k_src, dt, U * cap_src, coop_tile_keys(dt)));
-        TRI_CUDA(cudaMemsetAsync(ws, 0, kWsHeader, s));
-        TRI_CUDA(cudaMemsetAsync(ws_at(ws, w.hists), 0, w.zero_end - w.hists, s));
-        TRI_CUDA(launch_fold(stats, p_cur, n_seq, n_layers, n_kvheads * G, cfg->theta, off, wts, s));
+        // One memset: the flag word, the unit histograms and barrier counters.
+        TRI_CUDA(cudaMemsetAsync(ws, 0, w.zero_end, s));
         CoopArgs a;
         a.n_units = U;
+        a.stats = stats;
+        a.p_cur = p_cur;
+        a.n_layers = n_layers;
+        a.n_kvheads = n_kvheads;
+        a.theta = cfg->theta;
+        a.off = off;
         a.cap = cap_src;
         a.cap_dst = cap_dst;
         a.B = B;
@@ -559,7 +564,6 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
         a.stages = w.cp.stages;
         a.ctas_per_unit = w.cp.ctas_per_unit;
         a.n_valid = n_valid;
-        a.wts = wts;
         a.k_src = k_src;
         a.v_src = v_src;
         a.pos_src = pos_src;
@@ -583,15 +587,19 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
         CUtensorMap map;
         TRI_TRY(make_key_map(&map, k_src, dt, U * cap_src, fused_tile_keys(dt)));
         TRI_CUDA(cudaMemsetAsync(ws, 0, kWsHeader, s));
-        TRI_CUDA(launch_fold(stats, p_cur, n_seq, n_layers, n_kvheads * G, cfg->theta, off, wts, s));
         FusedArgs a;
+        a.stats = stats;
+        a.p_cur = p_cur;
+        a.n_layers = n_layers;
+        a.n_kvheads = n_kvheads;
+        a.theta = cfg->theta;
+        a.off = off;
         a.n_units = U;
         a.stages = fused_stages(dt, G, cap_src, B);
         a.cap = cap_src;
         a.cap_dst = cap_dst;
         a.B = B;
         a.n_valid = n_valid;
-        a.wts = wts;
         a.k_src = k_src;
         a.v_src = v_src;
         a.pos_src = pos_src;

@@ -25,6 +25,7 @@
 // TRI_FLAG_TIMEOUT and makes the CTA skip the remaining phases, so a fault
 // elsewhere cannot hang the GPU.
 #include "select_core.cuh"
+#include "fold_core.cuh"
 #include "score_core.cuh"
 #include "tri_internal.cuh"
 #include "tri_launch.h"
@@ -60,7 +61,8 @@ __host__ __device__ inline CoopLayout coop_layout(int G, int64_t keys_max, int s
     L.bars = L.list + static_cast<size_t>(kp) * 8;
     L.red = L.bars + 2 * S::kMaxStages * 8;
     L.misc = L.red + static_cast<size_t>(4) * kMaxG * 2 * 8;
-    L.total = L.misc + kHistBins0 * 4 + 512 + 1024;  // histogram, state; alignment slack
+    // histogram, state; alignment slack; static shared memory (fold)
+    L.total = L.misc + kHistBins0 * 4 + 512 + 1024 + kFoldStaticBytes;
     return L;
 }
 
@@ -169,16 +171,26 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
             fence_barrier_init();
             prefetch_tensormap(&kmap);
         }
-        {
-            const float4* src = reinterpret_cast<const float4*>(a.wts + u * G * kWHead);
-            float4* dst = reinterpret_cast<float4*>(w);
-            for (int e = tid; e < G * kWHead / 4; e += S::kThreads) dst[e] = src[e];
-        }
-        __syncthreads();
+        __syncthreads();  // barriers initialised before the producer starts
         const int nt = t1 - t0;
+        __shared__ FoldShared fs;
+        if (tid == S::kMath) {
+            // Issue the first tile loads before the fold so they overlap it.
+            for (int l = 0; l < nt && l < a.stages; ++l) {
+                mbar_arrive_expect_tx(&full[l], S::kStageBytes);
+                const int32_t y =
+                    static_cast<int32_t>(u * a.cap + static_cast<int64_t>(t0 + l) * S::kTile);
+#pragma unroll
+                for (int b = 0; b < S::kBoxes; ++b)
+                    tma_load_2d(ring + l * S::kStageBytes + b * S::kBoxBytes, &kmap, &full[l],
+                                b * (128 / static_cast<int>(sizeof(T))), y);
+            }
+        }
+        fold_prepare(fs, a.off, a.theta);
+        fold_unit<G>(fs, w, a.stats, a.p_cur, u, a.n_layers, a.n_kvheads);
         if (tid >= S::kMath) {
             if (tid == S::kMath) {
-                for (int l = 0; l < nt; ++l) {
+                for (int l = a.stages; l < nt; ++l) {  // the first stages were issued above
                     const int stage = l % a.stages;
                     if (!mbar_wait(&empty[stage], ((l / a.stages) & 1) ^ 1, a.flag)) {
                         *abort_flag = 1;
@@ -537,7 +549,8 @@ int coop_max_stages() { return CoopShape<float>::kMaxStages; }
 template <typename T, int G>
 static cudaError_t launch_coop_t(const CUtensorMap& map, const CoopArgs& a, int n_ctas,
                                  cudaStream_t s) {
-    const size_t smem = coop_layout<T>(G, a.keys_max, a.stages).total;
+    // Dynamic part only; the static fold factors are within kFoldStaticBytes.
+    const size_t smem = coop_layout<T>(G, a.keys_max, a.stages).total - kFoldStaticBytes;
     auto kern = prune_coop_kernel<T, G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));

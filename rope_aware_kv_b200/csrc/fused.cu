@@ -26,6 +26,7 @@
 // HBM traffic per unit is the compulsory bytes plus the re-read of kept K
 // rows (often from L2).
 #include "select_core.cuh"
+#include "fold_core.cuh"
 #include "score_core.cuh"
 #include "tri_internal.cuh"
 #include "tri_launch.h"
@@ -65,7 +66,8 @@ __host__ __device__ inline FusedLayout fused_layout(int G, int64_t cap, int64_t 
     L.bars = L.kidx + ((static_cast<size_t>(m) * 4 + 15) & ~size_t(15));
     L.red = L.bars + (2 * S::kMaxStages + 2 * S::kMaxGStages) * 8;
     L.misc = L.red + static_cast<size_t>(4) * kMaxG * 2 * 8;
-    L.total = L.misc + 256 + 1024;  // state and warp counts; alignment slack
+    // state and warp counts; alignment slack; static shared memory (fold)
+    L.total = L.misc + 256 + 1024 + kFoldStaticBytes;
     return L;
 }
 
@@ -122,7 +124,8 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
         prefetch_tensormap(&kmap);
         *abort_flag = 0;
     }
-    __syncthreads();
+    __shared__ FoldShared fs;
+    fold_prepare(fs, a.off, a.theta);
 
     uint32_t tiles_done = 0;   // running tile count (TMA ring position) of this CTA
     uint32_t pieces_done = 0;  // running gather-piece count (gather ring position)
@@ -137,12 +140,7 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
 
         if (!keep_all) {
             // ---------------- score ----------------
-            if (tid < S::kMath) {
-                const float4* src = reinterpret_cast<const float4*>(a.wts + u * G * kWHead);
-                float4* dst = reinterpret_cast<float4*>(w);
-                for (int e = tid; e < G * kWHead / 4; e += S::kMath) dst[e] = src[e];
-            }
-            __syncthreads();
+            fold_unit<G>(fs, w, a.stats, a.p_cur, u, a.n_layers, a.n_kvheads);
             if (tid >= S::kMath) {
                 if (tid == S::kMath) {
                     // Keys stay in L2 for the kept-row re-read of the gather.
@@ -508,7 +506,8 @@ int fused_tile_keys(tri_dtype dt) {
 template <typename T, int G>
 static cudaError_t launch_fused_t(const CUtensorMap& map, const FusedArgs& a, int n_ctas,
                                   cudaStream_t s) {
-    const size_t smem = fused_layout<T>(G, a.cap, a.B, a.stages).total;
+    // Dynamic part only; the static fold factors are within kFoldStaticBytes.
+    const size_t smem = fused_layout<T>(G, a.cap, a.B, a.stages).total - kFoldStaticBytes;
     auto kern = prune_fused_kernel<T, G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));

@@ -19,6 +19,10 @@ struct FoldOffsets {
     int64_t v[TRI_MAX_OFFSETS];
 };
 
+// Static shared memory of the fused and cooperative kernels (the fold's
+// per-band factors), counted in their shared-memory budgets.
+constexpr size_t kFoldStaticBytes = 4096;
+
 struct ScoreArgs {
     int64_t n_units;
     int64_t cap;
@@ -35,11 +39,17 @@ struct ScoreArgs {
 struct FusedArgs {
     int64_t n_units;
     int stages;                  // TMA ring depth, 4..6
+    // fold inputs (the kernel forms the per-head weights itself)
+    const float* stats;          // [L][Hkv*G][64][4]
+    const int64_t* p_cur;        // [n_seq]
+    int64_t n_layers;
+    int64_t n_kvheads;
+    double theta;
+    FoldOffsets off;
     int64_t cap;
     int64_t cap_dst;
     int64_t B;
     const int32_t* n_valid;
-    const float* wts;            // [U*G][192]
     const void* k_src;
     const void* v_src;
     const int32_t* pos_src;
@@ -58,6 +68,12 @@ constexpr int kTraceWarps = 8;   // one slot per warp
 
 struct CoopArgs {
     int64_t n_units;
+    const float* stats;          // fold inputs, as in FusedArgs
+    const int64_t* p_cur;
+    int64_t n_layers;
+    int64_t n_kvheads;
+    double theta;
+    FoldOffsets off;
     int64_t cap;
     int64_t cap_dst;
     int64_t B;
@@ -65,7 +81,6 @@ struct CoopArgs {
     int stages;                  // TMA ring depth
     int ctas_per_unit;           // C
     const int32_t* n_valid;
-    const float* wts;            // [U*G][192]
     const void* k_src;
     const void* v_src;
     const int32_t* pos_src;

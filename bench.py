@@ -404,9 +404,9 @@ def run_tri(args, ws, rank, local):
                               spec.torch_dtype)
     dom = int(np.argmax(per_launch))
     if path in (tri.PATH_FUSED, tri.PATH_COOP):
-        names = ["fold", "prune_fused_kernel" if path == tri.PATH_FUSED else "prune_coop_kernel"]
-        dom_name = names[dom] if dom < len(names) else f"launch{dom}"
-        dom_bytes = fused_bytes(spec) if dom == 1 else 0
+        # One launch per step: the whole path in one kernel.
+        dom_name = "prune_fused_kernel" if path == tri.PATH_FUSED else "prune_coop_kernel"
+        dom_bytes = fused_bytes(spec)
     else:
         names = ["fold", "score", "zmax_hist", "radix_pass1", "radix_pass2", "select_count",
                  "select_compact", "gather"]

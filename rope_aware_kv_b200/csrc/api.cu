@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstring>
 #include <mutex>
 
@@ -145,6 +146,26 @@ tri_status check_cfg(const tri_config* cfg, FoldOffsets* off) {
         off->v[i] = cfg->offsets[i];
     }
     return TRI_OK;
+}
+
+// w_f = theta^(-2f/d) and C_f = (1/|D|) sum_delta e^{i w_f delta} in float64
+// (talk page: RoPE frequencies and the offset-averaged score S~).  These
+// depend on the configuration only.
+FoldConst fold_const(const tri_config* cfg) {
+    FoldConst fc;
+    for (int f = 0; f < kF; ++f) {
+        const double w = std::pow(cfg->theta, -2.0 * f / static_cast<double>(kD));
+        double cre = 0.0, cim = 0.0;
+        for (int i = 0; i < cfg->n_offsets; ++i) {
+            const double a = w * static_cast<double>(cfg->offsets[i]);
+            cre += std::cos(a);
+            cim += std::sin(a);
+        }
+        fc.omega[f] = w;
+        fc.cf[f][0] = cre / cfg->n_offsets;
+        fc.cf[f][1] = cim / cfg->n_offsets;
+    }
+    return fc;
 }
 
 // Shape limits shared by score / prune: grid dimensions and 32-bit TMA row
@@ -555,8 +576,7 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
         a.p_cur = p_cur;
         a.n_layers = n_layers;
         a.n_kvheads = n_kvheads;
-        a.theta = cfg->theta;
-        a.off = off;
+        a.fc = fold_const(cfg);
         a.cap = cap_src;
         a.cap_dst = cap_dst;
         a.B = B;
@@ -592,8 +612,7 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
         a.p_cur = p_cur;
         a.n_layers = n_layers;
         a.n_kvheads = n_kvheads;
-        a.theta = cfg->theta;
-        a.off = off;
+        a.fc = fold_const(cfg);
         a.n_units = U;
         a.stages = fused_stages(dt, G, cap_src, B);
         a.cap = cap_src;

@@ -186,8 +186,7 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
                                 b * (128 / static_cast<int>(sizeof(T))), y);
             }
         }
-        fold_prepare(fs, a.off, a.theta);
-        fold_unit<G>(fs, w, a.stats, a.p_cur, u, a.n_layers, a.n_kvheads);
+        fold_unit<G>(fs, a.fc, w, a.stats, a.p_cur, u, a.n_layers, a.n_kvheads);
         if (tid >= S::kMath) {
             if (tid == S::kMath) {
                 for (int l = a.stages; l < nt; ++l) {  // the first stages were issued above

@@ -3,9 +3,9 @@
 // A_f = E[q_f] e^{i w_f p_cur} C_f with C_f = (1/|D|) sum_delta e^{i w_f delta}
 // and c_f = (1 - R_f) E|q_f| (talk page: S_trig, S_norm and the
 // offset-averaged S~; the key position cancels, see score.cu).  The
-// config-only factors w_f and C_f are formed once per CTA; each unit then
-// needs 64 phases e^{i w_f p_cur} and G x 64 complex products, all in
-// float64, rounded once to the float32 weight records the score loop reads
+// config-only factors w_f and C_f arrive as a kernel parameter (FoldConst);
+// each unit needs 64 phases e^{i w_f p_cur} and G x 64 complex products, all
+// in float64, rounded once to the float32 weight records the score loop reads
 // (16 chunks x 12 floats per head: 4 bands' (Re A, Im A) pairs, then their c).
 #pragma once
 
@@ -15,46 +15,23 @@
 namespace tri {
 
 struct FoldShared {
-    double omega[kF];
-    double cf[kF][2];
-    double ef[kF][2];
+    double ef[64][2];
 };
 static_assert(sizeof(FoldShared) <= kFoldStaticBytes, "fold factors exceed their budget");
-
-// w_f and C_f for the CTA: thread f < 64 sums the |D| phasors of band f in
-// offset order.  Every thread must call it; a __syncthreads follows inside.
-__device__ __forceinline__ void fold_prepare(FoldShared& fs, const FoldOffsets& off,
-                                             double theta) {
-    const int f = threadIdx.x;
-    if (f < kF) {
-        const double w = pow(theta, -2.0 * static_cast<double>(f) / static_cast<double>(kD));
-        double cre = 0.0, cim = 0.0;
-        for (int i = 0; i < off.n; ++i) {
-            double sn, cs;
-            sincos(w * static_cast<double>(off.v[i]), &sn, &cs);
-            cre += cs;
-            cim += sn;
-        }
-        fs.omega[f] = w;
-        fs.cf[f][0] = cre / off.n;
-        fs.cf[f][1] = cim / off.n;
-    }
-    __syncthreads();
-}
 
 // Weight records of the G query heads of unit u into w (shared memory).
 // Two __syncthreads inside; every thread of the CTA must call it.
 template <int G>
-__device__ __forceinline__ void fold_unit(FoldShared& fs, float* w, const float* stats,
-                                          const int64_t* p_cur, int64_t u, int64_t n_layers,
-                                          int64_t n_kvheads) {
+__device__ __forceinline__ void fold_unit(FoldShared& fs, const FoldConst& fc, float* w,
+                                          const float* stats, const int64_t* p_cur, int64_t u,
+                                          int64_t n_layers, int64_t n_kvheads) {
     const int t = threadIdx.x;
     const int64_t kvh = u % n_kvheads;
     const int64_t layer = (u / n_kvheads) % n_layers;
     const int64_t seq = u / (n_kvheads * n_layers);
     if (t < kF) {
         double ps, pc;
-        sincos(fs.omega[t] * static_cast<double>(p_cur[seq]), &ps, &pc);
+        sincos(fc.omega[t] * static_cast<double>(p_cur[seq]), &ps, &pc);
         fs.ef[t][0] = pc;
         fs.ef[t][1] = ps;
     }
@@ -66,8 +43,8 @@ __device__ __forceinline__ void fold_unit(FoldShared& fs, float* w, const float*
         const double mre = st.x, mim = st.y;
         const double tre = mre * fs.ef[f][0] - mim * fs.ef[f][1];
         const double tim = mre * fs.ef[f][1] + mim * fs.ef[f][0];
-        const double are = tre * fs.cf[f][0] - tim * fs.cf[f][1];
-        const double aim = tre * fs.cf[f][1] + tim * fs.cf[f][0];
+        const double are = tre * fc.cf[f][0] - tim * fc.cf[f][1];
+        const double aim = tre * fc.cf[f][1] + tim * fc.cf[f][0];
         const double cw = (1.0 - static_cast<double>(st.w)) * static_cast<double>(st.z);
         float* rec = w + h * kWHead + (f >> 2) * kWChunk;
         const int i = f & 3;

@@ -125,7 +125,6 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
         *abort_flag = 0;
     }
     __shared__ FoldShared fs;
-    fold_prepare(fs, a.off, a.theta);
 
     uint32_t tiles_done = 0;   // running tile count (TMA ring position) of this CTA
     uint32_t pieces_done = 0;  // running gather-piece count (gather ring position)
@@ -140,12 +139,30 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
 
         if (!keep_all) {
             // ---------------- score ----------------
-            fold_unit<G>(fs, w, a.stats, a.p_cur, u, a.n_layers, a.n_kvheads);
+            // The first tiles of the unit are requested before the fold so
+            // that their loads overlap it (every ring stage is free here).
+            const int pre = n_tiles < n_stages ? n_tiles : n_stages;
+            if (tid == S::kMath) {
+                const uint64_t keep_pol = policy_evict_last();
+                for (int i = 0; i < pre; ++i) {
+                    const uint32_t tc = tiles_done + i;
+                    const int stage = tc % n_stages;
+                    mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
+                    const int32_t y =
+                        static_cast<int32_t>(u * a.cap + static_cast<int64_t>(i) * S::kTile);
+#pragma unroll
+                    for (int b = 0; b < S::kBoxes; ++b)
+                        tma_load_2d_hint(regA + stage * S::kStageBytes + b * S::kBoxBytes, &kmap,
+                                         &full[stage], b * (128 / static_cast<int>(sizeof(T))), y,
+                                         keep_pol);
+                }
+            }
+            fold_unit<G>(fs, a.fc, w, a.stats, a.p_cur, u, a.n_layers, a.n_kvheads);
             if (tid >= S::kMath) {
                 if (tid == S::kMath) {
                     // Keys stay in L2 for the kept-row re-read of the gather.
                     const uint64_t keep_pol = policy_evict_last();
-                    for (int i = 0; i < n_tiles; ++i) {
+                    for (int i = pre; i < n_tiles; ++i) {
                         const uint32_t tc = tiles_done + i;
                         const int stage = tc % n_stages;
                         if (!mbar_wait(&empty[stage], ((tc / n_stages) & 1) ^ 1, a.flag)) {

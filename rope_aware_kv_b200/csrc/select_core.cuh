@@ -18,38 +18,60 @@ __host__ __device__ __forceinline__ int pass_shift(int p) { return p == 0 ? 21 :
 
 // Descending search in one histogram by a single warp: the bin b* such that
 // (sum of bins above b*) < k <= (sum of bins >= b*).  Returns b* and the sum
-// above it.
+// above it.  Lane l owns the l-th highest slice of nbins / 32 bins (read with
+// 16-byte loads; hist must be 16-byte aligned); after a warp scan of the slice
+// sums, all lanes scan the slice that holds b* together.
 __device__ __forceinline__ void warp_find_bin(const uint32_t* hist, int nbins, uint32_t k,
                                               uint32_t& bin, uint32_t& above) {
     const int lane = threadIdx.x & 31;
-    const int per = nbins / 32;
-    // Lane 0 owns the highest bins.
-    const int hi = nbins - lane * per;  // exclusive
+    const int per = nbins / 32;                 // 64 or 32
+    const int hi = nbins - lane * per;          // exclusive top of this lane's slice
+    const uint4* h4 = reinterpret_cast<const uint4*>(hist + (hi - per));
     uint32_t sum = 0;
-    for (int b = hi - 1; b >= hi - per; --b) sum += hist[b];
-    uint32_t excl = sum;
+#pragma unroll 4
+    for (int i = 0; i < per / 4; ++i) {
+        const uint4 v = h4[i];
+        sum += (v.x + v.y) + (v.z + v.w);
+    }
+    uint32_t incl = sum;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t v = __shfl_up_sync(0xffffffffu, excl, o);
-        if (lane >= o) excl += v;
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
     }
-    excl -= sum;  // exclusive prefix (bins above this lane's slice)
-    const bool mine = (excl < k) && (k <= excl + sum);
+    const uint32_t excl = incl - sum;           // bins above this lane's slice
+    const bool mine = (excl < k) && (k <= incl);
     const uint32_t who = __ballot_sync(0xffffffffu, mine);
     const int src = who ? (__ffs(who) - 1) : 31;
-    uint32_t b_out = 0, a_out = 0;
-    if (lane == src) {
-        uint32_t acc = excl;
-        int b = hi - 1;
-        for (; b > hi - per; --b) {
-            if (acc + hist[b] >= k) break;
-            acc += hist[b];
-        }
-        b_out = static_cast<uint32_t>(b);
-        a_out = acc;
+    const uint32_t base = __shfl_sync(0xffffffffu, excl, src);
+    // Slice of lane src, top bin first: lane l takes q consecutive bins.
+    const int q = per / 32;                     // 2 or 1
+    const int top = nbins - src * per - 1;
+    uint32_t v0 = hist[top - lane * q];
+    uint32_t v1 = q > 1 ? hist[top - lane * q - 1] : 0u;
+    const uint32_t loc = v0 + v1;
+    uint32_t inc2 = loc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, inc2, o);
+        if (lane >= o) inc2 += v;
     }
-    bin = __shfl_sync(0xffffffffu, b_out, src);
-    above = __shfl_sync(0xffffffffu, a_out, src);
+    const uint32_t exc2 = inc2 - loc;
+    const bool hit = (base + exc2 < k) && (k <= base + inc2);
+    const uint32_t who2 = __ballot_sync(0xffffffffu, hit);
+    const int t = who2 ? (__ffs(who2) - 1) : 31;
+    uint32_t b_out = 0, a_out = 0;
+    if (lane == t) {
+        if (base + exc2 + v0 >= k || q == 1) {
+            b_out = static_cast<uint32_t>(top - lane * q);
+            a_out = base + exc2;
+        } else {
+            b_out = static_cast<uint32_t>(top - lane * q - 1);
+            a_out = base + exc2 + v0;
+        }
+    }
+    bin = __shfl_sync(0xffffffffu, b_out, t);
+    above = __shfl_sync(0xffffffffu, a_out, t);
 }
 
 }  // namespace tri

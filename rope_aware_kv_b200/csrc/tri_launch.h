@@ -19,8 +19,16 @@ struct FoldOffsets {
     int64_t v[TRI_MAX_OFFSETS];
 };
 
+// Config-only fold factors (RoPE frequencies w_f and the offset-averaged
+// phasor C_f = (1/|D|) sum_delta e^{i w_f delta}), formed once per call by the
+// host code of the library in float64 and passed as a kernel parameter.
+struct FoldConst {
+    double omega[64];
+    double cf[64][2];
+};
+
 // Static shared memory of the fused and cooperative kernels (the fold's
-// per-band factors), counted in their shared-memory budgets.
+// per-unit phases), counted in their shared-memory budgets.
 constexpr size_t kFoldStaticBytes = 4096;
 
 struct ScoreArgs {
@@ -44,8 +52,7 @@ struct FusedArgs {
     const int64_t* p_cur;        // [n_seq]
     int64_t n_layers;
     int64_t n_kvheads;
-    double theta;
-    FoldOffsets off;
+    FoldConst fc;
     int64_t cap;
     int64_t cap_dst;
     int64_t B;
@@ -72,8 +79,7 @@ struct CoopArgs {
     const int64_t* p_cur;
     int64_t n_layers;
     int64_t n_kvheads;
-    double theta;
-    FoldOffsets off;
+    FoldConst fc;
     int64_t cap;
     int64_t cap_dst;
     int64_t B;

@@ -125,6 +125,7 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
         *abort_flag = 0;
     }
     __shared__ FoldShared fs;
+    __syncthreads();  // barriers and the abort flag initialised before anyone reads them
 
     uint32_t tiles_done = 0;   // running tile count (TMA ring position) of this CTA
     uint32_t pieces_done = 0;  // running gather-piece count (gather ring position)

@@ -47,8 +47,9 @@ __device__ __forceinline__ void warp_find_bin(const uint32_t* hist, int nbins, u
     // Slice of lane src, top bin first: lane l takes q consecutive bins.
     const int q = per / 32;                     // 2 or 1
     const int top = nbins - src * per - 1;
-    uint32_t v0 = hist[top - lane * q];
-    uint32_t v1 = q > 1 ? hist[top - lane * q - 1] : 0u;
+    const int i0 = top - lane * q;               // >= 0 for every lane
+    const uint32_t v0 = hist[i0];
+    const uint32_t v1 = q > 1 ? hist[i0 - 1] : 0u;  // i0 >= 1 whenever q == 2
     const uint32_t loc = v0 + v1;
     uint32_t inc2 = loc;
 #pragma unroll

@@ -1,7 +1,7 @@
 """Benchmark of one TriAttention prune step on B200 (libtri, sm_100a).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2]
-                    [--impl reference]
+                    [--impl reference] [--n-seq S] [--no-cpu-baseline]
 
 A step is one pass of the whole prune path (fold, score, z-normalise / max,
 top-B select, order-preserving gather of K, V and positions) over every unit
@@ -77,6 +77,34 @@ def score_bytes(spec) -> int:
 
 def fused_bytes(spec) -> int:
     return compulsory_bytes(spec)
+
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
+# kernel per launch, from one ncu capture each (summaries under profiles/),
+# keyed by workload and kernel, with the hash of the kernel sources it was
+# taken on: once the sources change, ``traffic`` is reported as null until the
+# kernel is captured again.  "scale" multiplies a capture of a smaller case of
+# the workload up to one full launch (traffic grows with the units processed).
+TRAFFIC = {}
+
+
+def kernel_sources_hash() -> str:
+    import hashlib
+
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "rope_aware_kv_b200", "csrc")
+    for name in sorted(os.listdir(d)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(d, name), "rb") as fh:
+                h.update(name.encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload: str, kernel: str, n_seq_override: int):
+    rec = TRAFFIC.get((workload, kernel))
+    if rec is None or n_seq_override or rec["src"] != kernel_sources_hash():
+        return None
+    return rec["bytes_per_launch"]
 
 
 def measured_peaks():
@@ -315,6 +343,8 @@ def run_tri(args, ws, rank, local):
     barrier(ws)
     tri.load()
     spec = synth.SPECS[args.workload]
+    if args.n_seq:
+        spec = spec.scaled(n_seq=args.n_seq)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     runner = StepRunner(spec, dev)
@@ -429,7 +459,8 @@ def run_tri(args, ws, rank, local):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if spec.dtype == "bf16" else "f32", "data": "synthetic",
             "config": {
-                "workload": f"{args.workload}: {WORKLOAD_TEXT[args.workload]}",
+                "workload": f"{args.workload}: {WORKLOAD_TEXT[args.workload]}" + (
+                    f" (cut to {spec.n_seq} sequence(s))" if args.n_seq else ""),
                 "units": spec.n_units, "keys_per_unit": spec.n_valid, "budget": spec.B,
                 "group": spec.G, "head_dim": spec.d, "parallelism": f"dp{ws} (independent units)",
                 "l2": f"inputs rotated over {runner.n_copies} copies "
@@ -440,7 +471,8 @@ def run_tri(args, ws, rank, local):
             "compulsory_bytes_per_step": comp,
             "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": achieved,
                          "peak": peak_gbs, "peak_kind": peak_kind, "unit": "GB/s",
-                         "frac": achieved / peak_gbs, "traffic": None,
+                         "frac": achieved / peak_gbs,
+                         "traffic": measured_traffic(args.workload, dom_name, args.n_seq),
                          "algorithmic_bytes": dom_bytes, "ms_per_launch": dom_ms},
             "per_launch_ms": [round(float(x), 5) for x in per_launch],
             "path": {tri.PATH_FUSED: "fused", tri.PATH_COOP: "coop"}.get(path, "split"),
@@ -507,6 +539,9 @@ def main():
     ap.add_argument("--impl", default="tri", choices=["tri", "reference"])
     ap.add_argument("--workload", default="c2", choices=sorted(synth.SPECS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--n-seq", type=int, default=0,
+                    help="run the workload with this many sequences instead (a smaller case "
+                         "of the same kernel for profiler captures; not a bench line)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

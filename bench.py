@@ -85,7 +85,12 @@ def fused_bytes(spec) -> int:
 # taken on: once the sources change, ``traffic`` is reported as null until the
 # kernel is captured again.  "scale" multiplies a capture of a smaller case of
 # the workload up to one full launch (traffic grows with the units processed).
-TRAFFIC = {}
+TRAFFIC = {
+    # profiles/prune_coop_kernel_c2_full.txt
+    ("c2", "prune_coop_kernel"): {"bytes_per_launch": 36259584, "src": "00d04262a9971991"},
+    # profiles/prune_fused_kernel_c3-2seq_full.txt: 224 of 1792 units captured, x 8
+    ("c3", "prune_fused_kernel"): {"bytes_per_launch": 6274965504, "src": "00d04262a9971991"},
+}
 
 
 def kernel_sources_hash() -> str:

@@ -231,7 +231,8 @@ struct PruneWs {
     ScoreWs sc;
     size_t fin = 0, kept = 0;
     SelectWs sel;
-    size_t partial = 0, hists = 0, counts = 0, bar = 0, zero_end = 0;
+    size_t partial = 0, hists = 0, counts = 0, bar = 0, zero_end = 0, hists_key = 0, cand = 0,
+           cand_count = 0;
     size_t total = 0;
 };
 
@@ -269,6 +270,7 @@ CoopPlan coop_plan(tri_dtype dt, int G, int64_t U, int64_t cap) {
     const int64_t tiles = (cap + tile - 1) / tile;
     int64_t C = sms / U;
     if (C > tiles) C = tiles;
+    if (C > kMaxCtasPerUnit) C = kMaxCtasPerUnit;
     if (C < 2) return p;
     p.keys_max = ((tiles + C - 1) / C) * tile;
     for (int st = coop_max_stages(); st >= 2; --st) {
@@ -300,9 +302,12 @@ PruneWs prune_ws(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int6
         w.cp = cp;
         const int64_t grid = U * cp.ctas_per_unit;
         Carve c;
-        w.hists = c.take(static_cast<size_t>(3 * U) * kHistBins0 * 4);
+        w.hists = c.take(static_cast<size_t>(U) * kHistBins0 * 4);
         w.bar = c.take(static_cast<size_t>(U) * 4);
+        w.cand_count = c.take(static_cast<size_t>(U) * 4);
         w.zero_end = c.off;
+        w.hists_key = c.take(static_cast<size_t>(3 * U) * kHistBins0 * 4);
+        w.cand = c.take(static_cast<size_t>(U) * kCandMax * 8);
         w.sc.wts = c.take(256);
         w.sc.raw = c.take(static_cast<size_t>(grid * G * cp.keys_max) * 4);
         w.partial = c.take(static_cast<size_t>(grid * G * 2) * 8);
@@ -595,8 +600,11 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
         a.scratch = reinterpret_cast<float*>(ws_at(ws, w.sc.raw));
         a.partial = reinterpret_cast<double*>(ws_at(ws, w.partial));
         a.hists = reinterpret_cast<uint32_t*>(ws_at(ws, w.hists));
+        a.hists_key = reinterpret_cast<uint32_t*>(ws_at(ws, w.hists_key));
         a.counts = reinterpret_cast<uint2*>(ws_at(ws, w.counts));
         a.bar = reinterpret_cast<uint32_t*>(ws_at(ws, w.bar));
+        a.cand_count = reinterpret_cast<uint32_t*>(ws_at(ws, w.cand_count));
+        a.cand = reinterpret_cast<int2*>(ws_at(ws, w.cand));
         a.trace = phase_trace_buffer(U * w.cp.ctas_per_unit);
         a.flag = flag;
         return cuda_status(

@@ -1,6 +1,6 @@
 // coop.cu -- one prune step of a few large caches in a single kernel: every
 // unit (one KV head's cache) is split over C consecutive CTAs, one per SM, and
-// the CTAs of a unit meet at five unit-wide barriers.
+// the CTAs of a unit meet at three unit-wide barriers.
 //
 // Same definitions as the other paths: the folded S~ per query head (talk
 // page: S_trig, S_norm, S~), z-score per head and max over the GQA group
@@ -11,13 +11,19 @@
 //            all heads) into an L2-resident per-CTA scratch; float64 moment
 //            partial per CTA                                   -> barrier 1
 //   phase 2  fixed-order merge of the unit's partials; final = max_h z_h of
-//            the CTA's keys into shared memory; digit-0 histogram added to
-//            the unit's global histogram                       -> barrier 2
-//   phase 3  digit-1 histogram of the keys in the digit-0 bin  -> barrier 3
-//   phase 4  digit-2 histogram                                 -> barrier 4
-//   phase 5  the CTA's counts above / equal to the threshold   -> barrier 5
-//   phase 6  fixed-order prefix over the unit's CTAs, ordered compaction of
-//            the CTA's kept keys, gather of their K / V / position rows.
+//            the CTA's keys into shared memory; histogram of the linear
+//            z-bins of final added to the unit's global one    -> barrier 2
+//   phase 3  the z-bin b0 of the B-th key; the CTA's count of keys above b0
+//            and its keys inside b0 (the candidates) appended to a unit-wide
+//            list                                              -> barrier 3
+//   phase 4  every CTA ranks all candidates itself (a three-digit radix
+//            select of their full keys in shared memory) and derives how many
+//            rows and ties the CTAs before it keep: no further barrier
+//   phase 5  ordered compaction of the CTA's kept keys, gather of their
+//            K / V / position rows.
+// If more than kCandMax keys share b0 (many equal scores), phase 4 falls back
+// to unit-wide histograms of the same three digits over the keys of b0 and
+// per-CTA counts, with barriers 4 to 7.
 //
 // A barrier is an atomic arrival counter per unit (zeroed by the host before
 // the launch) and a bounded spin on it; every CTA of the grid is resident (one
@@ -45,6 +51,10 @@ struct CoopShape {
     static constexpr int kThreads = kMath + 32;
     static constexpr int kWarps = kThreads / 32;
 };
+
+static_assert(static_cast<size_t>(kCandMax) * 8 <= 2 * CoopShape<float>::kStageBytes &&
+                  static_cast<size_t>(kCandMax) * 8 <= 2 * CoopShape<__nv_bfloat16>::kStageBytes,
+              "the candidate list must fit a two-stage TMA ring");
 
 struct CoopLayout {
     size_t w, fin, list, bars, red, misc, total;
@@ -262,10 +272,18 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
         // in order, then a fixed shuffle tree; lane 0's value is used.
         for (int h = warp; h < G; h += S::kWarps) {
             double s1 = 0.0, s2 = 0.0;
-            for (int cc = lane; cc < C; cc += 32) {
-                const double* part = a.partial + ((u * C + cc) * G + h) * 2;
-                s1 += part[0];
-                s2 += part[1];
+            double2 pv[kMaxCtasPerUnit / 32];
+#pragma unroll
+            for (int q = 0; q < kMaxCtasPerUnit / 32; ++q) {
+                const int cc = lane + 32 * q;
+                pv[q] = cc < C ? __ldcg(reinterpret_cast<const double2*>(
+                                     a.partial + ((u * C + cc) * G + h) * 2))
+                               : make_double2(0.0, 0.0);
+            }
+#pragma unroll
+            for (int q = 0; q < kMaxCtasPerUnit / 32; ++q) {
+                s1 += pv[q].x;
+                s2 += pv[q].y;
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
@@ -314,7 +332,7 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
                         }
                         fin[jl] = best;
                         if (best != best) nonfinite = true;
-                        atomicAdd(&hist[ordered_key(best) >> pass_shift(0)], 1u);
+                        atomicAdd(&hist[zbin(best)], 1u);
                     }
                 }
             }
@@ -330,77 +348,140 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
         if (!unit_barrier(ctr, 2u * C, a.flag, abort_flag)) return;
         coop_trace(a, 4);
 
-        // ---------------- phases 3 and 4: digits 1 and 2 ----------------
-        // The unit's histogram is read once into shared memory by every
-        // thread (16-byte loads), then scanned by one warp.
-        {
-            const uint4* g = reinterpret_cast<const uint4*>(a.hists + u * kHistBins0);
-            uint4* h4 = reinterpret_cast<uint4*>(hist);
-            for (int b = tid; b < kHistBins0 / 4; b += S::kThreads) h4[b] = ld_cg_u4(g + b);
-        }
+        // ---------------- phase 3: threshold bin, candidates ----------------
+        // Every CTA reads the unit's z-bin histogram and finds the bin b0 that
+        // holds the B-th key.  Keys above b0 are kept; the keys in b0 (the
+        // candidates) go to a unit-wide list in global memory, so that after
+        // one more barrier every CTA can finish the selection on its own.
+        copy_l2_to_shared(reinterpret_cast<uint4*>(hist),
+                          reinterpret_cast<const uint4*>(a.hists + u * kHistBins0),
+                          kHistBins0 / 4);
         __syncthreads();
+        uint32_t* zb0 = bases + 2;  // the threshold z-bin
         if (warp == 0) {
             uint32_t bin, above;
-            warp_find_bin(hist, 1 << pass_bits(0), static_cast<uint32_t>(B), bin, above);
+            warp_find_bin(hist, kZBins, static_cast<uint32_t>(B), bin, above);
             if (lane == 0) {
-                st->prefix = bin;
-                st->k = static_cast<uint32_t>(B) - above;
+                *zb0 = bin;
+                st->prefix = 0;
+                st->k = static_cast<uint32_t>(B) - above;  // to take from bin b0
                 st->gt = above;
                 st->keep_all = 0;
             }
         }
-        __syncthreads();
-        for (int p = 1; p < 3; ++p) {
-            const int nb = 1 << pass_bits(p);
-            for (int b = tid; b < nb; b += S::kThreads) hist[b] = 0;
-            __syncthreads();
-            const uint32_t prefix = st->prefix;
-            const int shift = pass_shift(p);
-            const int hi_shift = shift + pass_bits(p);
-            for (int jl = tid; jl < nk; jl += S::kThreads) {
-                const uint32_t key = ordered_key(fin[jl]);
-                if ((key >> hi_shift) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
-            }
-            __syncthreads();
-            uint32_t* g = a.hists + (static_cast<int64_t>(p) * a.n_units + u) * kHistBins0;
-            for (int b = tid; b < nb; b += S::kThreads)
-                if (hist[b]) atomicAdd(&g[b], hist[b]);
-            if (!unit_barrier(ctr, (2u + p) * C, a.flag, abort_flag)) return;
-            {
-                const uint4* g4 = reinterpret_cast<const uint4*>(g);
-                uint4* h4 = reinterpret_cast<uint4*>(hist);
-                for (int b = tid; b < nb / 4; b += S::kThreads) h4[b] = ld_cg_u4(g4 + b);
-            }
-            __syncthreads();
-            if (warp == 0) {
-                uint32_t bin, above;
-                warp_find_bin(hist, nb, st->k, bin, above);
-                if (lane == 0) {
-                    st->prefix = (prefix << pass_bits(p)) | bin;
-                    st->k -= above;
-                    st->gt += above;
-                }
-            }
-            __syncthreads();
-        }
-
-        // ---------------- phase 5: the CTA's counts ----------------
-        const uint32_t Tk = st->prefix, kt = st->k;
+        // This CTA's share of the unit's three full-key digit histograms,
+        // which only the overflow path accumulates into (after barrier 3).
         {
-            uint32_t gt = 0, eq = 0;
-            for (int jl = tid; jl < nk; jl += S::kThreads) {
-                const uint32_t key = ordered_key(fin[jl]);
-                gt += key > Tk;
-                eq += key == Tk;
+            const int z0 = (c * kHistBins0) / C, z1 = ((c + 1) * kHistBins0) / C;
+            for (int p = 0; p < 3; ++p) {
+                uint32_t* g = a.hists_key + (static_cast<int64_t>(p) * a.n_units + u) * kHistBins0;
+                for (int b = z0 + tid; b < z1; b += S::kThreads) g[b] = 0u;
             }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                gt += __shfl_xor_sync(0xffffffffu, gt, o);
-                eq += __shfl_xor_sync(0xffffffffu, eq, o);
+        }
+        __syncthreads();
+        const uint32_t b0 = *zb0;
+        // Warp w owns the contiguous keys [l0, l1) of this CTA (here and in
+        // the ordered compaction).
+        const int seg = ((nk + S::kWarps * 32 - 1) / (S::kWarps * 32)) * 32;
+        const int l0 = warp * seg;
+        const int l1 = min(l0 + seg, nk);
+        const uint32_t lt = (1u << lane) - 1u;
+        {
+            uint32_t above = 0, cands = 0;
+            for (int jl = l0 + lane; jl - lane < l1; jl += 32) {
+                const bool valid = jl < l1;
+                const uint32_t bin = valid ? zbin(fin[jl]) : 0u;
+                above += __popc(__ballot_sync(0xffffffffu, valid && bin > b0));
+                cands += __popc(__ballot_sync(0xffffffffu, valid && bin == b0));
             }
             if (lane == 0) {
-                wcnt[2 * warp] = gt;
-                wcnt[2 * warp + 1] = eq;
+                wcnt[2 * warp] = above;
+                wcnt[2 * warp + 1] = cands;
+            }
+            __syncthreads();
+            if (tid == 0) {
+                uint32_t ab = 0, cn = 0;
+                for (int v = 0; v < S::kWarps; ++v) {
+                    ab += wcnt[2 * v];
+                    cn += wcnt[2 * v + 1];
+                }
+                bases[0] = atomicAdd(&a.cand_count[u], cn);  // this CTA's first slot
+                a.counts[u * C + c] = make_uint2(ab, cn);
+            }
+            __syncthreads();
+            uint32_t slot = bases[0];
+            for (int v = 0; v < warp; ++v) slot += wcnt[2 * v + 1];
+            int2* out = a.cand + u * kCandMax;
+            for (int jl = l0 + lane; jl - lane < l1; jl += 32) {
+                const bool valid = jl < l1;
+                const float f = valid ? fin[jl] : 0.f;
+                const bool is_c = valid && zbin(f) == b0;
+                const uint32_t bc = __ballot_sync(0xffffffffu, is_c);
+                const uint32_t r = slot + __popc(bc & lt);
+                if (is_c && r < static_cast<uint32_t>(kCandMax))
+                    out[r] = make_int2(static_cast<int>(ordered_key(f)), j0 + jl);
+                slot += __popc(bc);
+            }
+        }
+        if (!unit_barrier(ctr, 3u * C, a.flag, abort_flag)) return;
+
+        // ---------------- phase 4: the threshold key ----------------
+        // Three radix digits of the full key (11, 11, 10 bits) find the
+        // k-th largest key of bin b0 and how many of its ties are kept.
+        const uint32_t n_cand = ld_acquire_u32(a.cand_count + u);
+        if (n_cand <= static_cast<uint32_t>(kCandMax)) {
+            // Over the candidates, by every CTA in its own shared memory (the
+            // TMA ring is free after scoring).
+            int2* cs = reinterpret_cast<int2*>(ring);
+            const int nc = static_cast<int>(n_cand);
+            // Pairs of entries; an odd count also copies the unused slot nc.
+            copy_l2_to_shared(reinterpret_cast<uint4*>(cs),
+                              reinterpret_cast<const uint4*>(a.cand + u * kCandMax), (nc + 1) / 2);
+            for (int p = 0; p < 3; ++p) {
+                const int nb = 1 << pass_bits(p);
+                for (int b = tid; b < nb; b += S::kThreads) hist[b] = 0;
+                __syncthreads();
+                const uint32_t prefix = st->prefix;
+                const int shift = pass_shift(p);
+                const int hi_shift = shift + pass_bits(p);
+                for (int i = tid; i < nc; i += S::kThreads) {
+                    const uint32_t key = static_cast<uint32_t>(cs[i].x);
+                    if (p == 0 || (key >> hi_shift) == prefix)
+                        atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+                }
+                __syncthreads();
+                if (warp == 0) {
+                    uint32_t bin, above;
+                    warp_find_bin(hist, nb, st->k, bin, above);
+                    if (lane == 0) {
+                        st->prefix = (prefix << pass_bits(p)) | bin;
+                        st->k -= above;
+                        st->gt += above;
+                    }
+                }
+                __syncthreads();
+            }
+            // Kept rows and threshold ties in the CTAs before this one: their
+            // keys above b0 (the published counts), their candidates above the
+            // threshold key, and their ties up to the number taken.
+            const uint32_t Tk = st->prefix, kt = st->k;
+            uint32_t gs = 0, es = 0;
+            for (int i = tid; i < nc; i += S::kThreads) {
+                const int2 e = cs[i];
+                if (e.y < j0) {
+                    gs += static_cast<uint32_t>(e.x) > Tk;
+                    es += static_cast<uint32_t>(e.x) == Tk;
+                }
+            }
+            for (int cc = tid; cc < c; cc += S::kThreads) gs += __ldcg(a.counts + u * C + cc).x;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                gs += __shfl_xor_sync(0xffffffffu, gs, o);
+                es += __shfl_xor_sync(0xffffffffu, es, o);
+            }
+            if (lane == 0) {
+                wcnt[2 * warp] = gs;
+                wcnt[2 * warp + 1] = es;
             }
             __syncthreads();
             if (tid == 0) {
@@ -409,35 +490,97 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
                     g2 += wcnt[2 * v];
                     e2 += wcnt[2 * v + 1];
                 }
-                a.counts[u * C + c] = make_uint2(g2, e2);
+                bases[0] = g2 + min(e2, kt);  // kept before this CTA
+                bases[1] = e2;                // ties before this CTA
             }
-        }
-        if (!unit_barrier(ctr, 5u * C, a.flag, abort_flag)) return;
-        coop_trace(a, 5);
-
-        // ---------------- phase 6: ordered compaction ----------------
-        if (warp == 0) {
-            uint32_t gsum = 0, esum = 0;
-            for (int cc = lane; cc < c; cc += 32) {
-                const uint2 v = a.counts[u * C + cc];
-                gsum += v.x;
-                esum += v.y;
+        } else {
+            // Overflow: more than kCandMax keys share bin b0 (many equal
+            // scores).  The same digits as unit-wide histograms over the keys
+            // of bin b0, then the CTAs' counts above / equal to the threshold.
+            for (int p = 0; p < 3; ++p) {
+                const int nb = 1 << pass_bits(p);
+                for (int b = tid; b < nb; b += S::kThreads) hist[b] = 0;
+                __syncthreads();
+                const uint32_t prefix = st->prefix;
+                const int shift = pass_shift(p);
+                const int hi_shift = shift + pass_bits(p);
+                for (int jl = tid; jl < nk; jl += S::kThreads) {
+                    const float f = fin[jl];
+                    const uint32_t key = ordered_key(f);
+                    if (zbin(f) == b0 && (p == 0 || (key >> hi_shift) == prefix))
+                        atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+                }
+                __syncthreads();
+                uint32_t* g = a.hists_key + (static_cast<int64_t>(p) * a.n_units + u) * kHistBins0;
+                for (int b = tid; b < nb; b += S::kThreads)
+                    if (hist[b]) atomicAdd(&g[b], hist[b]);
+                if (!unit_barrier(ctr, (4u + p) * C, a.flag, abort_flag)) return;
+                copy_l2_to_shared(reinterpret_cast<uint4*>(hist),
+                                  reinterpret_cast<const uint4*>(g), nb / 4);
+                __syncthreads();
+                if (warp == 0) {
+                    uint32_t bin, above;
+                    warp_find_bin(hist, nb, st->k, bin, above);
+                    if (lane == 0) {
+                        st->prefix = (prefix << pass_bits(p)) | bin;
+                        st->k -= above;
+                        st->gt += above;
+                    }
+                }
+                __syncthreads();
             }
+            const uint32_t Tk = st->prefix, kt = st->k;
+            {
+                uint32_t gt = 0, eq = 0;
+                for (int jl = tid; jl < nk; jl += S::kThreads) {
+                    const uint32_t key = ordered_key(fin[jl]);
+                    gt += key > Tk;
+                    eq += key == Tk;
+                }
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                gsum += __shfl_xor_sync(0xffffffffu, gsum, o);
-                esum += __shfl_xor_sync(0xffffffffu, esum, o);
+                for (int o = 16; o > 0; o >>= 1) {
+                    gt += __shfl_xor_sync(0xffffffffu, gt, o);
+                    eq += __shfl_xor_sync(0xffffffffu, eq, o);
+                }
+                if (lane == 0) {
+                    wcnt[2 * warp] = gt;
+                    wcnt[2 * warp + 1] = eq;
+                }
+                __syncthreads();
+                if (tid == 0) {
+                    uint32_t g2 = 0, e2 = 0;
+                    for (int v = 0; v < S::kWarps; ++v) {
+                        g2 += wcnt[2 * v];
+                        e2 += wcnt[2 * v + 1];
+                    }
+                    a.counts[u * C + c] = make_uint2(g2, e2);
+                }
             }
-            if (lane == 0) {
-                bases[0] = gsum + min(esum, kt);  // kept before this CTA
-                bases[1] = esum;                  // ties before this CTA
+            if (!unit_barrier(ctr, 7u * C, a.flag, abort_flag)) return;
+            if (warp == 0) {
+                uint32_t gsum = 0, esum = 0;
+                for (int cc = lane; cc < c; cc += 32) {
+                    const uint2 v = __ldcg(a.counts + u * C + cc);
+                    gsum += v.x;
+                    esum += v.y;
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    gsum += __shfl_xor_sync(0xffffffffu, gsum, o);
+                    esum += __shfl_xor_sync(0xffffffffu, esum, o);
+                }
+                if (lane == 0) {
+                    bases[0] = gsum + min(esum, kt);  // kept before this CTA
+                    bases[1] = esum;                  // ties before this CTA
+                }
             }
         }
+        coop_trace(a, 5);
+        const uint32_t Tk = st->prefix, kt = st->k;
         __syncthreads();
+
+        // ---------------- phase 5: ordered compaction ----------------
         {
-            const int seg = ((nk + S::kWarps * 32 - 1) / (S::kWarps * 32)) * 32;
-            const int l0 = warp * seg;
-            const int l1 = min(l0 + seg, nk);
             uint32_t gt = 0, eq = 0;
             for (int jl = l0 + lane; jl - lane < l1; jl += 32) {
                 const bool valid = jl < l1;
@@ -458,7 +601,6 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
                 ties += wcnt[2 * v + 1];
             }
             pos += lpos;
-            const uint32_t lt = (1u << lane) - 1u;
             for (int jl = l0 + lane; jl - lane < l1; jl += 32) {
                 const bool valid = jl < l1;
                 const uint32_t key = valid ? ordered_key(fin[jl]) : 0u;

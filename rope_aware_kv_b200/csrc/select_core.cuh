@@ -12,6 +12,18 @@ struct SelState {
     int keep_all;     // n_valid <= B: every valid key is kept
 };
 
+// Linear bin of a standardised score: 2048 bins of width 1/64 over
+// [-16, 16), both ends open, NaN in the lowest bin.  Non-decreasing in the
+// selection order (NaN lowest, -0 = +0), so the keys above the bin of the
+// B-th key are all kept; at the thresholds z-scores reach (|z| of a few
+// units) a bin holds far fewer keys than a bin of the key's top 11 bits.
+constexpr int kZBins = 2048;
+__device__ __forceinline__ uint32_t zbin(float z) {
+    if (!(z == z)) return 0u;
+    const float t = floorf((z + 16.0f) * 64.0f);
+    return t < 0.f ? 0u : (t > 2047.f ? 2047u : static_cast<uint32_t>(t));
+}
+
 // Digit p of the 32-bit key: bits [pass_shift(p), pass_shift(p) + pass_bits(p)).
 __host__ __device__ __forceinline__ int pass_bits(int p) { return p < 2 ? 11 : 10; }
 __host__ __device__ __forceinline__ int pass_shift(int p) { return p == 0 ? 21 : (p == 1 ? 10 : 0); }

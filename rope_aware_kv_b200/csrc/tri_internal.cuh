@@ -217,6 +217,26 @@ __device__ __forceinline__ uint4 ld_cg_u4(const uint4* p) {
     return v;
 }
 
+// Copy n16 16-byte words that other CTAs wrote in this launch from global
+// memory (through L2, bypassing L1) to shared memory, every thread of the CTA
+// keeping up to 8 loads in flight.
+__device__ __forceinline__ void copy_l2_to_shared(uint4* dst, const uint4* src, int n16) {
+    const int tid = threadIdx.x, nthr = blockDim.x;
+    for (int base = 0; base < n16; base += 8 * nthr) {
+        uint4 v[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int i = base + q * nthr + tid;
+            if (i < n16) v[q] = ld_cg_u4(src + i);
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int i = base + q * nthr + tid;
+            if (i < n16) dst[i] = v[q];
+        }
+    }
+}
+
 // Named barrier among `count` threads (a multiple of 32) of the CTA.
 __device__ __forceinline__ void named_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");

@@ -73,6 +73,12 @@ struct FusedArgs {
 constexpr int kTracePoints = 8;  // phase points per unit (fused) or CTA (coop)
 constexpr int kTraceWarps = 8;   // one slot per warp
 
+// Threshold-bin candidates one unit of the cooperative path can exchange
+// (8 bytes each; staged in the CTA's TMA ring of at least 2 x 32 KB).
+constexpr int kCandMax = 8192;
+// Most CTAs the cooperative path splits one unit over (a multiple of 32).
+constexpr int kMaxCtasPerUnit = 160;
+
 struct CoopArgs {
     int64_t n_units;
     const float* stats;          // fold inputs, as in FusedArgs
@@ -97,9 +103,12 @@ struct CoopArgs {
     int32_t* n_kept;             // [U]
     float* scratch;              // [grid][G][keys_max]
     double* partial;             // [U][C][G][2]
-    uint32_t* hists;             // [3][U][2048], zero on entry
+    uint32_t* hists;             // [U][2048] z-bin histograms, zero on entry
+    uint32_t* hists_key;         // [3][U][2048] full-key digits (zeroed in the kernel)
     uint2* counts;               // [U][C]
     uint32_t* bar;               // [U], zero on entry
+    uint32_t* cand_count;        // [U], zero on entry
+    int2* cand;                  // [U][kCandMax] (ordered key, key index)
     uint64_t* trace;             // [grid][kTracePoints][kTraceWarps] or null
     uint32_t* flag;
 };

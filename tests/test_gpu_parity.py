@@ -312,6 +312,34 @@ def test_identical_keys_keep_lowest_indices(path):
     assert np.all(out["kept"] == np.arange(123)[None, :])
 
 
+@pytest.mark.parametrize("path", [tri.PATH_COOP, tri.PATH_SPLIT])
+def test_threshold_tie_group_beyond_candidate_list(path):
+    """Keys alternate between two vectors, so with one head the z-scores take
+    two values and the B-th key sits in a group of 9000 equal scores: more
+    than the cooperative kernel's candidate list holds (8192), which sends it
+    down its unit-wide radix path.  The keys of a group are equal, so their
+    scores are equal (the key position cancels); the lowest-index keys of
+    the higher group are kept.  The oracle evaluates each key's score at its
+    own position and so differs inside a group only by float64 rounding: it
+    fixes which group is higher, and that each group's scores agree."""
+    B = 5000
+    spec = _spec(dtype="bf16", G=1, n_seq=1, n_layers=1, n_kvheads=2, cap=18000, B=B)
+    wl = synth.make_workload(spec, "cuda")
+    wl.k[:, 0::2] = wl.k[:, :1]
+    wl.k[:, 1::2] = wl.k[:, 1:2]
+    gst, ost = H.stats_for(spec, wl)
+    out = _run_prune(spec, wl, gst, B, path=path)
+    assert out["flags"] == 0
+    o = _oracle_units(spec, wl, ost, B, wl.n_valid.cpu().numpy(), list(range(spec.n_units)))
+    for u in range(spec.n_units):
+        even, odd = o["final"][u, 0::2], o["final"][u, 1::2]
+        assert np.ptp(even) <= 1e-9 and np.ptp(odd) <= 1e-9 and abs(even[0] - odd[0]) > 1.0
+        first = 0 if even[0] > odd[0] else 1
+        np.testing.assert_array_equal(out["kept"][u], first + 2 * np.arange(B))
+        assert H.rows_equal(out["k"][u], wl.k[u], out["kept"][u])
+        assert H.rows_equal(out["v"][u], wl.v[u], out["kept"][u])
+
+
 @pytest.mark.parametrize("path", [tri.PATH_FUSED, tri.PATH_SPLIT, tri.PATH_COOP])
 def test_nan_key_poisons_unit_and_flags(path):
     """A NaN key makes that unit's moments NaN: every final score is NaN,

@@ -7,7 +7,7 @@
 // (hyper.ai summary, Method section), top-B by (score desc, index asc) kept
 // in temporal order (jaedaily.cn tutorial, eviction step).
 //
-//   phase 1  score the CTA's tiles (TMA ring, one math warp per 128-key tile,
+//   phase 1  score the CTA's tiles (TMA ring, seven math warps, one per 128-key tile,
 //            all heads) into an L2-resident per-CTA scratch; float64 moment
 //            partial per CTA                                   -> barrier 1
 //   phase 2  fixed-order merge of the unit's partials; final = max_h z_h of
@@ -47,9 +47,17 @@ struct CoopShape {
     static constexpr int kBoxBytes = kTile * 128;
     static constexpr int kStageBytes = kTile * kRowBytes;  // 32 KB
     static constexpr int kMaxStages = 6;
-    static constexpr int kMath = 128;
+    static constexpr int kMathWarps = 7;          // + one producer warp: 256 threads
+    static constexpr int kMath = 32 * kMathWarps;
     static constexpr int kThreads = kMath + 32;
     static constexpr int kWarps = kThreads / 32;
+    // Tile-landed barriers indexed by the tile number, not the ring stage (a
+    // math warp takes every kMathWarps-th tile and so skips phases of a
+    // stage's barrier): a warp waiting for tile t has finished tile
+    // t - kMathWarps, so tiles up to t - kMathWarps - 1 - stages are consumed,
+    // including t - kTileBars, the previous use of its barrier.
+    static constexpr int kTileBars = 16;
+    static_assert(kTileBars >= kMathWarps + 1 + kMaxStages, "tile barriers too few");
 };
 
 static_assert(static_cast<size_t>(kCandMax) * 8 <= 2 * CoopShape<float>::kStageBytes &&
@@ -69,8 +77,8 @@ __host__ __device__ inline CoopLayout coop_layout(int G, int64_t keys_max, int s
     L.fin = L.w + static_cast<size_t>(G) * kWHead * 4;
     L.list = L.fin + static_cast<size_t>(kp) * 4;
     L.bars = L.list + static_cast<size_t>(kp) * 8;
-    L.red = L.bars + 2 * S::kMaxStages * 8;
-    L.misc = L.red + static_cast<size_t>(4) * kMaxG * 2 * 8;
+    L.red = L.bars + (S::kTileBars + S::kMaxStages) * 8;
+    L.misc = L.red + static_cast<size_t>(S::kMathWarps) * kMaxG * 2 * 8;
     // histogram, state; alignment slack; static shared memory (fold)
     L.total = L.misc + kHistBins0 * 4 + 512 + 1024 + kFoldStaticBytes;
     return L;
@@ -126,13 +134,13 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
     float* w = reinterpret_cast<float*>(base + L.w);
     float* fin = reinterpret_cast<float*>(base + L.fin);
     int2* list = reinterpret_cast<int2*>(base + L.list);
-    uint64_t* full = reinterpret_cast<uint64_t*>(base + L.bars);
-    uint64_t* empty = full + S::kMaxStages;
-    double* red = reinterpret_cast<double*>(base + L.red);  // [4 warps][kMaxG][2]
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + L.bars);  // [kTileBars] tile landed
+    uint64_t* empty = full + S::kTileBars;                         // [stages] stage free
+    double* red = reinterpret_cast<double*>(base + L.red);  // [math warps][kMaxG][2]
     uint32_t* hist = reinterpret_cast<uint32_t*>(base + L.misc);
     SelState* st = reinterpret_cast<SelState*>(base + L.misc + kHistBins0 * 4);
     float2* mom = reinterpret_cast<float2*>(base + L.misc + kHistBins0 * 4 + 16);   // [kMaxG]
-    uint32_t* wcnt = reinterpret_cast<uint32_t*>(base + L.misc + kHistBins0 * 4 + 80);  // [5][2]
+    uint32_t* wcnt = reinterpret_cast<uint32_t*>(base + L.misc + kHistBins0 * 4 + 80);  // [kWarps][2]
     uint32_t* bases = wcnt + 16;                                            // [2]
     int* abort_flag = reinterpret_cast<int*>(bases + 4);
     int* nlist = abort_flag + 1;
@@ -174,10 +182,8 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
     } else {
         // ---------------- phase 1: score ----------------
         if (tid == S::kMath) {
-            for (int i = 0; i < a.stages; ++i) {
-                mbar_init(&full[i], 1);
-                mbar_init(&empty[i], 32);
-            }
+            for (int i = 0; i < S::kTileBars; ++i) mbar_init(&full[i], 1);
+            for (int i = 0; i < a.stages; ++i) mbar_init(&empty[i], 32);
             fence_barrier_init();
             prefetch_tensormap(&kmap);
         }
@@ -187,12 +193,13 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
         if (tid == S::kMath) {
             // Issue the first tile loads before the fold so they overlap it.
             for (int l = 0; l < nt && l < a.stages; ++l) {
-                mbar_arrive_expect_tx(&full[l], S::kStageBytes);
+                mbar_arrive_expect_tx(&full[l % S::kTileBars], S::kStageBytes);
                 const int32_t y =
                     static_cast<int32_t>(u * a.cap + static_cast<int64_t>(t0 + l) * S::kTile);
 #pragma unroll
                 for (int b = 0; b < S::kBoxes; ++b)
-                    tma_load_2d(ring + l * S::kStageBytes + b * S::kBoxBytes, &kmap, &full[l],
+                    tma_load_2d(ring + l * S::kStageBytes + b * S::kBoxBytes, &kmap,
+                                &full[l % S::kTileBars],
                                 b * (128 / static_cast<int>(sizeof(T))), y);
             }
         }
@@ -205,21 +212,22 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
                         *abort_flag = 1;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
+                    mbar_arrive_expect_tx(&full[l % S::kTileBars], S::kStageBytes);
                     const int32_t y = static_cast<int32_t>(u * a.cap + static_cast<int64_t>(t0 + l) * S::kTile);
 #pragma unroll
                     for (int b = 0; b < S::kBoxes; ++b)
                         tma_load_2d(ring + stage * S::kStageBytes + b * S::kBoxBytes, &kmap,
-                                    &full[stage], b * (128 / static_cast<int>(sizeof(T))), y);
+                                    &full[l % S::kTileBars],
+                                    b * (128 / static_cast<int>(sizeof(T))), y);
                 }
             }
         } else {
             double m1[G], m2[G];
 #pragma unroll
             for (int h = 0; h < G; ++h) m1[h] = m2[h] = 0.0;
-            for (int l = warp; l < nt; l += 4) {
+            for (int l = warp; l < nt; l += S::kMathWarps) {
                 const int stage = l % a.stages;
-                if (!mbar_wait(&full[stage], (l / a.stages) & 1, a.flag)) {
+                if (!mbar_wait(&full[l % S::kTileBars], (l / S::kTileBars) & 1, a.flag)) {
                     *abort_flag = 1;
                     break;
                 }
@@ -258,10 +266,14 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
         if (tid < G) {
             const int h = tid;
             double* part = a.partial + ((u * C + c) * G + h) * 2;
-            part[0] = ((red[(0 * kMaxG + h) * 2] + red[(1 * kMaxG + h) * 2]) +
-                       red[(2 * kMaxG + h) * 2]) + red[(3 * kMaxG + h) * 2];
-            part[1] = ((red[(0 * kMaxG + h) * 2 + 1] + red[(1 * kMaxG + h) * 2 + 1]) +
-                       red[(2 * kMaxG + h) * 2 + 1]) + red[(3 * kMaxG + h) * 2 + 1];
+            double s1 = 0.0, s2 = 0.0;  // fixed order: math warps 0, 1, ...
+#pragma unroll
+            for (int v = 0; v < S::kMathWarps; ++v) {
+                s1 += red[(v * kMaxG + h) * 2];
+                s2 += red[(v * kMaxG + h) * 2 + 1];
+            }
+            part[0] = s1;
+            part[1] = s2;
         }
         coop_trace(a, 1);
         if (!unit_barrier(ctr, 1u * C, a.flag, abort_flag)) return;

@@ -10,7 +10,7 @@
 //
 // Per unit:
 //   score   a producer lane streams 128-key tiles (32 KB) into a TMA ring of
-//           4 to 6 stages; each of the four math warps scores whole tiles,
+//           4 to 6 stages; each of the seven math warps scores whole tiles,
 //           every lane on 4 keys for all GQA heads (so one broadcast weight
 //           load feeds 4 keys); per-head scores go to a per-CTA float32
 //           scratch that stays in L2, float64 moments stay in registers.
@@ -18,11 +18,12 @@
 //           first radix digit histogram.
 //   select  two more radix digits on shared-memory histograms, then the
 //           ordered compaction of kept indices (warp ballots).
-//   gather  kept rows form runs of consecutive indices; one lane streams
-//           each run piece (<= 8 KB) of K and of V into a 16-buffer shared
-//           ring with cp.async.bulk (up to 128 KB of loads in flight), and the
-//           math warps copy landed pieces to the destination with 16-byte
-//           stores, freeing each buffer as soon as it is read.
+//   gather  kept rows form runs of consecutive indices; one lane fills 8 KB
+//           shared buffers, each with kGRows consecutive destination rows of K
+//           or V, by one cp.async.bulk per run piece (the whole TMA ring, up
+//           to 192 KB of loads, in flight), and the math warps copy landed
+//           buffers to the destination with 16-byte stores, freeing each
+//           buffer as soon as it is read.
 // HBM traffic per unit is the compulsory bytes plus the re-read of kept K
 // rows (often from L2).
 #include "select_core.cuh"
@@ -42,12 +43,26 @@ struct FusedShape {
     static constexpr int kBoxBytes = kTile * 128;
     static constexpr int kStageBytes = kTile * kRowBytes;               // 32 KB
     static constexpr int kMaxStages = 6;                                // TMA ring depth (runtime)
-    static constexpr int kMath = 128;
+    static constexpr int kMathWarps = 7;  // + one producer / copy-engine warp: 256 threads
+    static constexpr int kMath = 32 * kMathWarps;
     static constexpr int kThreads = kMath + 32;
     static constexpr int kWarps = kThreads / 32;
     static constexpr int kGStage = 8192;                                // gather piece buffer
     static constexpr int kMaxGStages = kMaxStages * kStageBytes / kGStage;
     static constexpr int kGRows = kGStage / kRowBytes;                  // rows per piece
+    // "Landed" barriers are indexed by the running tile / piece count, not by
+    // the ring stage.  A math warp takes every kMathWarps-th tile, so it skips
+    // phases of a stage's barrier; a parity wait on a barrier that is more
+    // than one phase behind would pass at once.  When a warp waits for tile t
+    // it has finished tile t - kMathWarps, so every tile up to
+    // t - kMathWarps - 1 - stages has been consumed; with kTileBars >=
+    // kMathWarps + 1 + kMaxStages the previous use of barrier t % kTileBars
+    // (tile t - kTileBars) is among them, and the wait is exact.  Same for
+    // gather pieces with kPieceBars >= kMathWarps + 1 + kMaxGStages.
+    static constexpr int kTileBars = 16;
+    static constexpr int kPieceBars = 32;
+    static_assert(kTileBars >= kMathWarps + 1 + kMaxStages, "tile barriers too few");
+    static_assert(kPieceBars >= kMathWarps + 1 + kMaxGStages, "piece barriers too few");
 };
 
 struct FusedLayout {
@@ -64,8 +79,8 @@ __host__ __device__ inline FusedLayout fused_layout(int G, int64_t cap, int64_t 
     L.fin = L.w + static_cast<size_t>(G) * kWHead * 4;
     L.kidx = L.fin + static_cast<size_t>(capP) * 4;
     L.bars = L.kidx + ((static_cast<size_t>(m) * 4 + 15) & ~size_t(15));
-    L.red = L.bars + (2 * S::kMaxStages + 2 * S::kMaxGStages) * 8;
-    L.misc = L.red + static_cast<size_t>(4) * kMaxG * 2 * 8;
+    L.red = L.bars + (S::kTileBars + S::kMaxStages + S::kPieceBars + S::kMaxGStages) * 8;
+    L.misc = L.red + static_cast<size_t>(FusedShape<T>::kMathWarps) * kMaxG * 2 * 8;
     // state and warp counts; alignment slack; static shared memory (fold)
     L.total = L.misc + 256 + 1024 + kFoldStaticBytes;
     return L;
@@ -93,15 +108,15 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
     float* w = reinterpret_cast<float*>(base + L.w);
     float* fin = reinterpret_cast<float*>(base + L.fin);
     int32_t* kidx = reinterpret_cast<int32_t*>(base + L.kidx);
-    uint64_t* full = reinterpret_cast<uint64_t*>(base + L.bars);
-    uint64_t* empty = full + S::kMaxStages;
-    uint64_t* gfull = empty + S::kMaxStages;
-    uint64_t* gempty = gfull + S::kMaxGStages;
-    double* red = reinterpret_cast<double*>(base + L.red);  // [4 warps][kMaxG][2]
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + L.bars);  // [kTileBars] tile landed
+    uint64_t* empty = full + S::kTileBars;                         // [stages] stage free
+    uint64_t* gfull = empty + S::kMaxStages;                       // [kPieceBars] piece landed
+    uint64_t* gempty = gfull + S::kPieceBars;                      // [gather stages] buffer free
+    double* red = reinterpret_cast<double*>(base + L.red);  // [math warps][kMaxG][2]
     SelState* st = reinterpret_cast<SelState*>(base + L.misc);
     float2* mom = reinterpret_cast<float2*>(base + L.misc + 16);            // [kMaxG]
     uint32_t* wcnt = reinterpret_cast<uint32_t*>(base + L.misc + 16 + 64);  // [kWarps][2]
-    int32_t* nchunks = reinterpret_cast<int32_t*>(base + L.misc + 16 + 64 + 48);
+    int32_t* nchunks = reinterpret_cast<int32_t*>(base + L.misc + 16 + 64 + 8 * S::kWarps);
     int32_t* abort_flag = nchunks + 1;
     uint32_t* hist = reinterpret_cast<uint32_t*>(regA);  // between scoring and gathering
     int32_t* chunk_r = reinterpret_cast<int32_t*>(fin);  // after the compaction
@@ -112,14 +127,10 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
     float* scratch = a.scratch + static_cast<int64_t>(blockIdx.x) * G * a.cap;
 
     if (tid == S::kMath) {
-        for (int i = 0; i < n_stages; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 32);
-        }
-        for (int i = 0; i < n_gstages; ++i) {
-            mbar_init(&gfull[i], 1);
-            mbar_init(&gempty[i], 32);
-        }
+        for (int i = 0; i < S::kTileBars; ++i) mbar_init(&full[i], 1);
+        for (int i = 0; i < n_stages; ++i) mbar_init(&empty[i], 32);
+        for (int i = 0; i < S::kPieceBars; ++i) mbar_init(&gfull[i], 1);
+        for (int i = 0; i < n_gstages; ++i) mbar_init(&gempty[i], 32);
         fence_barrier_init();
         prefetch_tensormap(&kmap);
         *abort_flag = 0;
@@ -148,13 +159,14 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
                 for (int i = 0; i < pre; ++i) {
                     const uint32_t tc = tiles_done + i;
                     const int stage = tc % n_stages;
-                    mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
+                    uint64_t* landed = &full[tc % S::kTileBars];
+                    mbar_arrive_expect_tx(landed, S::kStageBytes);
                     const int32_t y =
                         static_cast<int32_t>(u * a.cap + static_cast<int64_t>(i) * S::kTile);
 #pragma unroll
                     for (int b = 0; b < S::kBoxes; ++b)
                         tma_load_2d_hint(regA + stage * S::kStageBytes + b * S::kBoxBytes, &kmap,
-                                         &full[stage], b * (128 / static_cast<int>(sizeof(T))), y,
+                                         landed, b * (128 / static_cast<int>(sizeof(T))), y,
                                          keep_pol);
                 }
             }
@@ -170,25 +182,26 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
                             *abort_flag = 1;
                             break;
                         }
-                        mbar_arrive_expect_tx(&full[stage], S::kStageBytes);
+                        uint64_t* landed = &full[tc % S::kTileBars];
+                        mbar_arrive_expect_tx(landed, S::kStageBytes);
                         const int32_t y =
                             static_cast<int32_t>(u * a.cap + static_cast<int64_t>(i) * S::kTile);
 #pragma unroll
                         for (int b = 0; b < S::kBoxes; ++b)
                             tma_load_2d_hint(regA + stage * S::kStageBytes + b * S::kBoxBytes,
-                                             &kmap, &full[stage],
+                                             &kmap, landed,
                                              b * (128 / static_cast<int>(sizeof(T))), y, keep_pol);
                     }
                 }
             } else {
-                // Math warp w scores tiles w, w + 4, ... with all G heads.
+                // Math warp w scores tiles w, w + kMathWarps, ... with all G heads.
                 double m1[G], m2[G];
 #pragma unroll
                 for (int h = 0; h < G; ++h) m1[h] = m2[h] = 0.0;
-                for (int i = warp; i < n_tiles; i += 4) {
+                for (int i = warp; i < n_tiles; i += S::kMathWarps) {
                     const uint32_t tc = tiles_done + i;
                     const int stage = tc % n_stages;
-                    if (!mbar_wait(&full[stage], (tc / n_stages) & 1, a.flag)) {
+                    if (!mbar_wait(&full[tc % S::kTileBars], (tc / S::kTileBars) & 1, a.flag)) {
                         *abort_flag = 1;
                         break;
                     }
@@ -227,13 +240,15 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
             trace_point(a, u, 1);
             __syncthreads();
             if (*abort_flag) break;
-            // ---------------- moments (fixed order: warps 0..3) ----------------
+            // ---------------- moments (fixed order: math warps 0, 1, ...) ----------------
             if (tid < G) {
                 const int h = tid;
-                const double s1 = ((red[(0 * kMaxG + h) * 2] + red[(1 * kMaxG + h) * 2]) +
-                                   red[(2 * kMaxG + h) * 2]) + red[(3 * kMaxG + h) * 2];
-                const double s2 = ((red[(0 * kMaxG + h) * 2 + 1] + red[(1 * kMaxG + h) * 2 + 1]) +
-                                   red[(2 * kMaxG + h) * 2 + 1]) + red[(3 * kMaxG + h) * 2 + 1];
+                double s1 = 0.0, s2 = 0.0;
+#pragma unroll
+                for (int v = 0; v < S::kMathWarps; ++v) {
+                    s1 += red[(v * kMaxG + h) * 2];
+                    s2 += red[(v * kMaxG + h) * 2 + 1];
+                }
                 const double mu = s1 / n;
                 double var = s2 / n - mu * mu;
                 if (var < 0.0) var = 0.0;
@@ -367,11 +382,13 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
 
         // ---------------- gather ----------------
         // Kept rows form runs of consecutive source rows; a piece is a run cut
-        // at row indices that are multiples of kGRows (<= 8 KB).  The engine
-        // lane streams K and V pieces into a 16-buffer shared-memory ring with
-        // cp.async.bulk (no registers or L1 miss slots held, up to 128 KB in
-        // flight); math warp (piece % 4) copies each landed piece to the
-        // destination with 16-byte stores and frees its buffer at once.
+        // at destination rows that are multiples of kGRows.  Buffer q of the
+        // shared-memory ring (8 KB) receives destination rows [q kGRows,
+        // (q + 1) kGRows): the engine lane issues one cp.async.bulk per piece
+        // inside it, all completing on the buffer's barrier, so every buffer
+        // in flight is full (no registers or L1 miss slots held); math warp
+        // (slot % kMathWarps) copies each landed buffer to its contiguous
+        // destination rows with 16-byte stores and frees it at once.
         {
             const int seg = ((m + S::kWarps * 32 - 1) / (S::kWarps * 32)) * 32;
             const int r0 = warp * seg;
@@ -407,44 +424,65 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
         fence_proxy_async();
         __syncthreads();
         const int n_chunks = *nchunks;
-        const int npc = a.v_src ? 2 * n_chunks : n_chunks;  // K (and V) piece per chunk
-        auto chunk_rows = [&](int c, int& r, int& len, int32_t& j) -> bool {
-            r = chunk_r[c];
-            const int rend = (c + 1 < n_chunks) ? chunk_r[c + 1] : m;
-            len = rend - r;
-            j = kidx[r];
-            return j >= 0 && j + len <= n && len > 0 && len <= S::kGRows;
-        };
-        if (tid == S::kMath) {
-            // Engine: bulk loads only (last use of these rows: evict first).
+        // A buffer holds kGRows consecutive destination rows, gathered from
+        // the pieces (runs) that start inside them; K and V of buffer q are
+        // slots 2q and 2q + 1.
+        const int n_buf = (m + S::kGRows - 1) / S::kGRows;
+        const int npc = a.v_src ? 2 * n_buf : n_buf;
+        if (tid >= S::kMath) {
+            // Engine warp: for each buffer, lane l issues the bulk loads of
+            // the buffer's l-th piece (a buffer of kGRows rows holds at most
+            // kGRows <= 32 pieces).  Last use of these rows: evict first.
             const uint64_t last_use = policy_evict_first();
             const char* ks = static_cast<const char*>(a.k_src);
             const char* vs = static_cast<const char*>(a.v_src);
-            for (int p = 0; p < npc; ++p) {
-                const uint32_t pc = pieces_done + p;
-                const int sb = pc % n_gstages;
-                if (!mbar_wait(&gempty[sb], ((pc / n_gstages) & 1) ^ 1, a.flag)) {
-                    *abort_flag = 1;
-                    break;
+            const int halves = a.v_src ? 2 : 1;
+            int c0 = 0;  // first piece of the current buffer
+            for (int q = 0; q < n_buf; ++q) {
+                const int rq0 = q * S::kGRows;
+                const int rq1 = min(rq0 + S::kGRows, m);
+                const int c = c0 + lane;
+                const bool mine = c < n_chunks && chunk_r[c] < rq1;
+                const int r = mine ? chunk_r[c] : 0;
+                const int rend = mine ? ((c + 1 < n_chunks) ? chunk_r[c + 1] : m) : 0;
+                const int32_t j = mine ? kidx[r] : 0;
+                const bool ok =
+                    mine && r >= rq0 && rend <= rq1 && rend > r && j >= 0 && j + (rend - r) <= n;
+                if (mine && !ok) raise_flag(a.flag, TRI_FLAG_INDEX_RANGE);  // cannot happen
+                uint32_t bytes = ok ? static_cast<uint32_t>((rend - r) * S::kRowBytes) : 0u;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
+                const int n_mine = __popc(__ballot_sync(0xffffffffu, mine));
+                bool stop = false;
+                for (int half = 0; half < halves; ++half) {
+                    const uint32_t pc = pieces_done + (a.v_src ? 2 * q + half : q);
+                    const int sb = pc % n_gstages;
+                    uint64_t* landed = &gfull[pc % S::kPieceBars];
+                    if (lane == 0) {
+                        if (!mbar_wait(&gempty[sb], ((pc / n_gstages) & 1) ^ 1, a.flag)) {
+                            *abort_flag = 1;
+                        } else {
+                            mbar_arrive_expect_tx(landed, bytes);
+                        }
+                    }
+                    __syncwarp();
+                    if (*abort_flag) {
+                        stop = true;
+                        break;
+                    }
+                    if (ok)
+                        bulk_load_hint(regA + sb * S::kGStage + (r - rq0) * S::kRowBytes,
+                                       (half ? vs : ks) + (u * a.cap + j) * S::kRowBytes,
+                                       static_cast<uint32_t>((rend - r) * S::kRowBytes), landed,
+                                       last_use);
                 }
-                const int c = a.v_src ? (p >> 1) : p;
-                const bool is_v = a.v_src && (p & 1);
-                int r, len;
-                int32_t j;
-                if (!chunk_rows(c, r, len, j)) {  // cannot happen when the selection is consistent
-                    raise_flag(a.flag, TRI_FLAG_INDEX_RANGE);
-                    mbar_arrive_expect_tx(&gfull[sb], 0);
-                    continue;
-                }
-                const uint32_t bytes = static_cast<uint32_t>(len * S::kRowBytes);
-                mbar_arrive_expect_tx(&gfull[sb], bytes);
-                bulk_load_hint(regA + sb * S::kGStage,
-                               (is_v ? vs : ks) + (u * a.cap + j) * S::kRowBytes, bytes, &gfull[sb],
-                               last_use);
+                if (stop) break;
+                c0 += n_mine;
             }
         } else if (tid < S::kMath) {
             // Math warps: positions of the kept rows (8 loads in flight per
-            // thread), then drain pieces warp, warp + 4, ... to global memory.
+            // thread), then drain pieces warp, warp + kMathWarps, ... to global
+            // memory.
             if (a.pos_dst) {
                 for (int r0 = tid; r0 < m; r0 += S::kMath * 8) {
                     int32_t pv[8];
@@ -464,23 +502,21 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
             constexpr int kVec = S::kRowBytes / 16;
             uint4* kd = static_cast<uint4*>(a.k_dst);
             uint4* vd = static_cast<uint4*>(a.v_dst);
-            for (int p = warp; p < npc; p += 4) {
+            for (int p = warp; p < npc; p += S::kMathWarps) {
                 const uint32_t pc = pieces_done + p;
                 const int sb = pc % n_gstages;
-                if (!mbar_wait(&gfull[sb], (pc / n_gstages) & 1, a.flag)) {
+                if (!mbar_wait(&gfull[pc % S::kPieceBars], (pc / S::kPieceBars) & 1, a.flag)) {
                     *abort_flag = 1;
                     break;
                 }
-                const int c = a.v_src ? (p >> 1) : p;
+                const int q = a.v_src ? (p >> 1) : p;
                 const bool is_v = a.v_src && (p & 1);
-                int r, len;
-                int32_t j;
-                if (chunk_rows(c, r, len, j)) {
-                    const uint4* buf = reinterpret_cast<const uint4*>(regA + sb * S::kGStage);
-                    uint4* dst = (is_v ? vd : kd) + (u * a.cap_dst + r) * kVec;
-                    const int nv = len * kVec;
-                    for (int e = lane; e < nv; e += 32) st_stream(dst + e, buf[e]);
-                }
+                const int rq0 = q * S::kGRows;
+                const int len = min(S::kGRows, m - rq0);
+                const uint4* buf = reinterpret_cast<const uint4*>(regA + sb * S::kGStage);
+                uint4* dst = (is_v ? vd : kd) + (u * a.cap_dst + rq0) * kVec;
+                const int nv = len * kVec;
+                for (int e = lane; e < nv; e += 32) st_stream(dst + e, buf[e]);
                 __syncwarp();
                 mbar_arrive(&gempty[sb]);
             }

@@ -63,6 +63,12 @@ struct FusedShape {
     static constexpr int kPieceBars = 32;
     static_assert(kTileBars >= kMathWarps + 1 + kMaxStages, "tile barriers too few");
     static_assert(kPieceBars >= kMathWarps + 1 + kMaxGStages, "piece barriers too few");
+    // Dense gather (most rows kept): 16 KB buffers of kDRows source rows.
+    static constexpr int kDStage = 16384;
+    static constexpr int kMaxDStages = kMaxStages * kStageBytes / kDStage;
+    static constexpr int kDRows = kDStage / kRowBytes;  // 64 / 32, a multiple of 32
+    static_assert(kDRows % 32 == 0, "dense chunks are whole 32-key groups");
+    static_assert(kPieceBars >= kMathWarps + 1 + kMaxDStages, "dense barriers too few");
 };
 
 struct FusedLayout {
@@ -79,7 +85,8 @@ __host__ __device__ inline FusedLayout fused_layout(int G, int64_t cap, int64_t 
     L.fin = L.w + static_cast<size_t>(G) * kWHead * 4;
     L.kidx = L.fin + static_cast<size_t>(capP) * 4;
     L.bars = L.kidx + ((static_cast<size_t>(m) * 4 + 15) & ~size_t(15));
-    L.red = L.bars + (S::kTileBars + S::kMaxStages + S::kPieceBars + S::kMaxGStages) * 8;
+    L.red = L.bars + (S::kTileBars + S::kMaxStages + 2 * S::kPieceBars + S::kMaxGStages +
+                      S::kMaxDStages) * 8;
     L.misc = L.red + static_cast<size_t>(FusedShape<T>::kMathWarps) * kMaxG * 2 * 8;
     // state and warp counts; alignment slack; static shared memory (fold)
     L.total = L.misc + 256 + 1024 + kFoldStaticBytes;
@@ -103,6 +110,7 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int n_stages = a.stages;
     const int n_gstages = n_stages * S::kStageBytes / S::kGStage;
+    const int n_dstages = n_stages * S::kStageBytes / S::kDStage;
     const FusedLayout L = fused_layout<T>(G, a.cap, a.B, n_stages);
     uint8_t* regA = base;
     float* w = reinterpret_cast<float*>(base + L.w);
@@ -112,6 +120,8 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
     uint64_t* empty = full + S::kTileBars;                         // [stages] stage free
     uint64_t* gfull = empty + S::kMaxStages;                       // [kPieceBars] piece landed
     uint64_t* gempty = gfull + S::kPieceBars;                      // [gather stages] buffer free
+    uint64_t* dfull = gempty + S::kMaxGStages;                     // dense: [kPieceBars] landed
+    uint64_t* dempty = dfull + S::kPieceBars;                      // dense: [stages] free
     double* red = reinterpret_cast<double*>(base + L.red);  // [math warps][kMaxG][2]
     SelState* st = reinterpret_cast<SelState*>(base + L.misc);
     float2* mom = reinterpret_cast<float2*>(base + L.misc + 16);            // [kMaxG]
@@ -131,6 +141,8 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
         for (int i = 0; i < n_stages; ++i) mbar_init(&empty[i], 32);
         for (int i = 0; i < S::kPieceBars; ++i) mbar_init(&gfull[i], 1);
         for (int i = 0; i < n_gstages; ++i) mbar_init(&gempty[i], 32);
+        for (int i = 0; i < S::kPieceBars; ++i) mbar_init(&dfull[i], 1);
+        for (int i = 0; i < n_dstages; ++i) mbar_init(&dempty[i], 32);
         fence_barrier_init();
         prefetch_tensormap(&kmap);
         *abort_flag = 0;
@@ -140,6 +152,7 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
 
     uint32_t tiles_done = 0;   // running tile count (TMA ring position) of this CTA
     uint32_t pieces_done = 0;  // running gather-piece count (gather ring position)
+    uint32_t dense_done = 0;   // running dense-chunk count (dense ring position)
 
     for (int64_t u = blockIdx.x; u < a.n_units; u += gridDim.x) {
         if (*abort_flag) break;  // a bounded wait gave up: stop cleanly
@@ -381,144 +394,265 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
         __syncthreads();
 
         // ---------------- gather ----------------
-        // Kept rows form runs of consecutive source rows; a piece is a run cut
-        // at destination rows that are multiples of kGRows.  Buffer q of the
-        // shared-memory ring (8 KB) receives destination rows [q kGRows,
-        // (q + 1) kGRows): the engine lane issues one cp.async.bulk per piece
-        // inside it, all completing on the buffer's barrier, so every buffer
-        // in flight is full (no registers or L1 miss slots held); math warp
-        // (slot % kMathWarps) copies each landed buffer to its contiguous
-        // destination rows with 16-byte stores and frees it at once.
-        {
-            const int seg = ((m + S::kWarps * 32 - 1) / (S::kWarps * 32)) * 32;
-            const int r0 = warp * seg;
-            const int r1 = min(r0 + seg, m);
-            uint32_t cnt = 0;
-            for (int r = r0 + lane; r - lane < r1; r += 32) {
-                bool start = false;
-                if (r < r1) {
-                    const int32_t j = kidx[r];
-                    const int32_t jp = r > 0 ? kidx[r - 1] : -2;
-                    start = (r % S::kGRows == 0) || j != jp + 1;
-                }
-                cnt += __popc(__ballot_sync(0xffffffffu, start));
-            }
-            if (lane == 0) wcnt[2 * warp] = cnt;
+        // Two ways, chosen per unit.
+        //  dense (at least 3/4 of the rows kept): the ring holds 16 KB chunks
+        //    of kDRows consecutive source rows, one cp.async.bulk each (the
+        //    few dropped rows are read too); the copying warp stores each
+        //    kept row of a landed chunk at its destination rank, from a
+        //    per-32-key keep mask and the rank of the group's first kept row.
+        //  runs (otherwise): kept rows form runs of consecutive source rows;
+        //    a piece is a run cut at destination rows that are multiples of
+        //    kGRows.  Buffer q (8 KB) receives destination rows [q kGRows,
+        //    (q + 1) kGRows): the engine warp issues one cp.async.bulk per
+        //    piece inside it (lane l takes the l-th piece), all completing on
+        //    the buffer's barrier, so every buffer in flight is full.
+        // Either way, loads hold no registers or L1 miss slots, and math warp
+        // (slot % kMathWarps) copies each landed buffer out with 16-byte
+        // stores, freeing it as soon as it is read.
+        const bool dense = 4 * static_cast<int64_t>(m) >= 3 * static_cast<int64_t>(n);
+        const int n_groups = (n + 31) / 32;
+        uint32_t* kmask = reinterpret_cast<uint32_t*>(fin);  // dense: after the compaction
+        uint32_t* kbase = kmask + n_groups;
+        if (dense) {
+            for (int g = tid; g < n_groups; g += S::kThreads) kmask[g] = 0u;
             __syncthreads();
-            uint32_t pos = 0;
-            for (int v = 0; v < warp; ++v) pos += wcnt[2 * v];
-            if (warp == S::kWarps - 1 && lane == 0) *nchunks = static_cast<int>(pos + cnt);
-            const uint32_t lt = (1u << lane) - 1u;
-            for (int r = r0 + lane; r - lane < r1; r += 32) {
-                bool start = false;
-                if (r < r1) {
-                    const int32_t j = kidx[r];
-                    const int32_t jp = r > 0 ? kidx[r - 1] : -2;
-                    start = (r % S::kGRows == 0) || j != jp + 1;
+            for (int r = tid; r < m; r += S::kThreads) {
+                const int32_t j = kidx[r];
+                if (j < 0 || j >= n) continue;  // cannot happen
+                atomicOr(&kmask[j >> 5], 1u << (j & 31));
+                if (r == 0 || (kidx[r - 1] >> 5) != (j >> 5)) kbase[j >> 5] = static_cast<uint32_t>(r);
+            }
+        } else {
+            {
+                const int seg = ((m + S::kWarps * 32 - 1) / (S::kWarps * 32)) * 32;
+                const int r0 = warp * seg;
+                const int r1 = min(r0 + seg, m);
+                uint32_t cnt = 0;
+                for (int r = r0 + lane; r - lane < r1; r += 32) {
+                    bool start = false;
+                    if (r < r1) {
+                        const int32_t j = kidx[r];
+                        const int32_t jp = r > 0 ? kidx[r - 1] : -2;
+                        start = (r % S::kGRows == 0) || j != jp + 1;
+                    }
+                    cnt += __popc(__ballot_sync(0xffffffffu, start));
                 }
-                const uint32_t b = __ballot_sync(0xffffffffu, start);
-                if (start) chunk_r[pos + __popc(b & lt)] = r;
-                pos += __popc(b);
+                if (lane == 0) wcnt[2 * warp] = cnt;
+                __syncthreads();
+                uint32_t pos = 0;
+                for (int v = 0; v < warp; ++v) pos += wcnt[2 * v];
+                if (warp == S::kWarps - 1 && lane == 0) *nchunks = static_cast<int>(pos + cnt);
+                const uint32_t lt = (1u << lane) - 1u;
+                for (int r = r0 + lane; r - lane < r1; r += 32) {
+                    bool start = false;
+                    if (r < r1) {
+                        const int32_t j = kidx[r];
+                        const int32_t jp = r > 0 ? kidx[r - 1] : -2;
+                        start = (r % S::kGRows == 0) || j != jp + 1;
+                    }
+                    const uint32_t b = __ballot_sync(0xffffffffu, start);
+                    if (start) chunk_r[pos + __popc(b & lt)] = r;
+                    pos += __popc(b);
+                }
             }
         }
         fence_proxy_async();
         __syncthreads();
-        const int n_chunks = *nchunks;
-        // A buffer holds kGRows consecutive destination rows, gathered from
-        // the pieces (runs) that start inside them; K and V of buffer q are
-        // slots 2q and 2q + 1.
-        const int n_buf = (m + S::kGRows - 1) / S::kGRows;
-        const int npc = a.v_src ? 2 * n_buf : n_buf;
-        if (tid >= S::kMath) {
-            // Engine warp: for each buffer, lane l issues the bulk loads of
-            // the buffer's l-th piece (a buffer of kGRows rows holds at most
-            // kGRows <= 32 pieces).  Last use of these rows: evict first.
-            const uint64_t last_use = policy_evict_first();
-            const char* ks = static_cast<const char*>(a.k_src);
-            const char* vs = static_cast<const char*>(a.v_src);
-            const int halves = a.v_src ? 2 : 1;
-            int c0 = 0;  // first piece of the current buffer
-            for (int q = 0; q < n_buf; ++q) {
-                const int rq0 = q * S::kGRows;
-                const int rq1 = min(rq0 + S::kGRows, m);
-                const int c = c0 + lane;
-                const bool mine = c < n_chunks && chunk_r[c] < rq1;
-                const int r = mine ? chunk_r[c] : 0;
-                const int rend = mine ? ((c + 1 < n_chunks) ? chunk_r[c + 1] : m) : 0;
-                const int32_t j = mine ? kidx[r] : 0;
-                const bool ok =
-                    mine && r >= rq0 && rend <= rq1 && rend > r && j >= 0 && j + (rend - r) <= n;
-                if (mine && !ok) raise_flag(a.flag, TRI_FLAG_INDEX_RANGE);  // cannot happen
-                uint32_t bytes = ok ? static_cast<uint32_t>((rend - r) * S::kRowBytes) : 0u;
+        // Math warps copy the positions of the kept rows first (8 loads in
+        // flight per thread).
+        auto copy_positions = [&]() {
+            if (!a.pos_dst) return;
+            for (int r0 = tid; r0 < m; r0 += S::kMath * 8) {
+                int32_t pv[8];
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
-                const int n_mine = __popc(__ballot_sync(0xffffffffu, mine));
-                bool stop = false;
-                for (int half = 0; half < halves; ++half) {
-                    const uint32_t pc = pieces_done + (a.v_src ? 2 * q + half : q);
-                    const int sb = pc % n_gstages;
-                    uint64_t* landed = &gfull[pc % S::kPieceBars];
-                    if (lane == 0) {
-                        if (!mbar_wait(&gempty[sb], ((pc / n_gstages) & 1) ^ 1, a.flag)) {
-                            *abort_flag = 1;
-                        } else {
-                            mbar_arrive_expect_tx(landed, bytes);
-                        }
-                    }
-                    __syncwarp();
-                    if (*abort_flag) {
-                        stop = true;
+                for (int q = 0; q < 8; ++q) {
+                    const int r = r0 + q * S::kMath;
+                    const int32_t j = r < m ? kidx[r] : -1;
+                    pv[q] = (j >= 0 && j < n) ? a.pos_src[u * a.cap + j] : 0;
+                }
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int r = r0 + q * S::kMath;
+                    if (r < m) a.pos_dst[u * a.cap_dst + r] = pv[q];
+                }
+            }
+        };
+        constexpr int kVec = S::kRowBytes / 16;
+        uint4* kd = static_cast<uint4*>(a.k_dst);
+        uint4* vd = static_cast<uint4*>(a.v_dst);
+        int npc = 0;
+        if (dense) {
+            const int n_dchunks = (n + S::kDRows - 1) / S::kDRows;
+            npc = a.v_src ? 2 * n_dchunks : n_dchunks;  // K (and V) slot per chunk
+            if (tid == S::kMath) {
+                const uint64_t last_use = policy_evict_first();
+                for (int p = 0; p < npc; ++p) {
+                    const uint32_t pc = dense_done + p;
+                    const int sb = pc % n_dstages;
+                    if (!mbar_wait(&dempty[sb], ((pc / n_dstages) & 1) ^ 1, a.flag)) {
+                        *abort_flag = 1;
                         break;
                     }
-                    if (ok)
-                        bulk_load_hint(regA + sb * S::kGStage + (r - rq0) * S::kRowBytes,
-                                       (half ? vs : ks) + (u * a.cap + j) * S::kRowBytes,
-                                       static_cast<uint32_t>((rend - r) * S::kRowBytes), landed,
-                                       last_use);
+                    const int c = a.v_src ? (p >> 1) : p;
+                    const bool is_v = a.v_src && (p & 1);
+                    const int row0 = c * S::kDRows;
+                    const int rows = min(S::kDRows, n - row0);
+                    bool any = false;
+                    for (int g = row0 >> 5; g < ((row0 + rows + 31) >> 5); ++g) any |= kmask[g] != 0u;
+                    const uint32_t bytes = any ? static_cast<uint32_t>(rows * S::kRowBytes) : 0u;
+                    uint64_t* landed = &dfull[pc % S::kPieceBars];
+                    mbar_arrive_expect_tx(landed, bytes);
+                    if (bytes)
+                        bulk_load_hint(regA + sb * S::kDStage,
+                                       static_cast<const char*>(is_v ? a.v_src : a.k_src) +
+                                           (u * a.cap + row0) * S::kRowBytes,
+                                       bytes, landed, last_use);
                 }
-                if (stop) break;
-                c0 += n_mine;
-            }
-        } else if (tid < S::kMath) {
-            // Math warps: positions of the kept rows (8 loads in flight per
-            // thread), then drain pieces warp, warp + kMathWarps, ... to global
-            // memory.
-            if (a.pos_dst) {
-                for (int r0 = tid; r0 < m; r0 += S::kMath * 8) {
-                    int32_t pv[8];
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const int r = r0 + q * S::kMath;
-                        const int32_t j = r < m ? kidx[r] : -1;
-                        pv[q] = (j >= 0 && j < n) ? a.pos_src[u * a.cap + j] : 0;
+            } else if (tid < S::kMath) {
+                copy_positions();
+                for (int p = warp; p < npc; p += S::kMathWarps) {
+                    const uint32_t pc = dense_done + p;
+                    const int sb = pc % n_dstages;
+                    if (!mbar_wait(&dfull[pc % S::kPieceBars], (pc / S::kPieceBars) & 1, a.flag)) {
+                        *abort_flag = 1;
+                        break;
                     }
+                    const int c = a.v_src ? (p >> 1) : p;
+                    const bool is_v = a.v_src && (p & 1);
+                    const int row0 = c * S::kDRows;
+                    const int nv = min(S::kDRows, n - row0) * kVec;
+                    const uint4* buf = reinterpret_cast<const uint4*>(regA + sb * S::kDStage);
+                    uint4* dst = (is_v ? vd : kd) + u * a.cap_dst * kVec;
+                    // Rounds of 8 loads in flight per lane; the buffer is freed
+                    // once its last round is read.
+                    constexpr int kRound = 8;
+                    constexpr int kRounds = S::kDStage / 16 / 32 / kRound;
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const int r = r0 + q * S::kMath;
-                        if (r < m) a.pos_dst[u * a.cap_dst + r] = pv[q];
+                    for (int h = 0; h < kRounds; ++h) {
+                        uint4 v[kRound];
+#pragma unroll
+                        for (int i = 0; i < kRound; ++i) {
+                            const int e = lane + 32 * (h * kRound + i);
+                            if (e < nv) v[i] = buf[e];
+                        }
+                        if (h == kRounds - 1) {
+                            __syncwarp();
+                            mbar_arrive(&dempty[sb]);
+                        }
+#pragma unroll
+                        for (int i = 0; i < kRound; ++i) {
+                            const int e = lane + 32 * (h * kRound + i);
+                            if (e < nv) {
+                                const int j = row0 + e / kVec;
+                                const uint32_t mask = kmask[j >> 5];
+                                const uint32_t bit = 1u << (j & 31);
+                                if (mask & bit) {
+                                    const uint32_t r = kbase[j >> 5] + __popc(mask & (bit - 1u));
+                                    st_stream(dst + static_cast<int64_t>(r) * kVec + e % kVec, v[i]);
+                                }
+                            }
+                        }
                     }
                 }
             }
-            constexpr int kVec = S::kRowBytes / 16;
-            uint4* kd = static_cast<uint4*>(a.k_dst);
-            uint4* vd = static_cast<uint4*>(a.v_dst);
-            for (int p = warp; p < npc; p += S::kMathWarps) {
-                const uint32_t pc = pieces_done + p;
-                const int sb = pc % n_gstages;
-                if (!mbar_wait(&gfull[pc % S::kPieceBars], (pc / S::kPieceBars) & 1, a.flag)) {
-                    *abort_flag = 1;
-                    break;
+        } else {
+            const int n_chunks = *nchunks;
+            // A buffer holds kGRows consecutive destination rows, gathered from
+            // the pieces (runs) that start inside them; K and V of buffer q are
+            // slots 2q and 2q + 1.
+            const int n_buf = (m + S::kGRows - 1) / S::kGRows;
+            npc = a.v_src ? 2 * n_buf : n_buf;
+            if (tid >= S::kMath) {
+                // Engine warp: for each buffer, lane l issues the bulk loads of
+                // the buffer's l-th piece (a buffer of kGRows rows holds at most
+                // kGRows <= 32 pieces).  Last use of these rows: evict first.
+                const uint64_t last_use = policy_evict_first();
+                const char* ks = static_cast<const char*>(a.k_src);
+                const char* vs = static_cast<const char*>(a.v_src);
+                const int halves = a.v_src ? 2 : 1;
+                int c0 = 0;  // first piece of the current buffer
+                for (int q = 0; q < n_buf; ++q) {
+                    const int rq0 = q * S::kGRows;
+                    const int rq1 = min(rq0 + S::kGRows, m);
+                    const int c = c0 + lane;
+                    const bool mine = c < n_chunks && chunk_r[c] < rq1;
+                    const int r = mine ? chunk_r[c] : 0;
+                    const int rend = mine ? ((c + 1 < n_chunks) ? chunk_r[c + 1] : m) : 0;
+                    const int32_t j = mine ? kidx[r] : 0;
+                    const bool ok =
+                        mine && r >= rq0 && rend <= rq1 && rend > r && j >= 0 && j + (rend - r) <= n;
+                    if (mine && !ok) raise_flag(a.flag, TRI_FLAG_INDEX_RANGE);  // cannot happen
+                    uint32_t bytes = ok ? static_cast<uint32_t>((rend - r) * S::kRowBytes) : 0u;
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
+                    const int n_mine = __popc(__ballot_sync(0xffffffffu, mine));
+                    bool stop = false;
+                    for (int half = 0; half < halves; ++half) {
+                        const uint32_t pc = pieces_done + (a.v_src ? 2 * q + half : q);
+                        const int sb = pc % n_gstages;
+                        uint64_t* landed = &gfull[pc % S::kPieceBars];
+                        if (lane == 0) {
+                            if (!mbar_wait(&gempty[sb], ((pc / n_gstages) & 1) ^ 1, a.flag)) {
+                                *abort_flag = 1;
+                            } else {
+                                mbar_arrive_expect_tx(landed, bytes);
+                            }
+                        }
+                        __syncwarp();
+                        if (*abort_flag) {
+                            stop = true;
+                            break;
+                        }
+                        if (ok)
+                            bulk_load_hint(regA + sb * S::kGStage + (r - rq0) * S::kRowBytes,
+                                           (half ? vs : ks) + (u * a.cap + j) * S::kRowBytes,
+                                           static_cast<uint32_t>((rend - r) * S::kRowBytes), landed,
+                                           last_use);
+                    }
+                    if (stop) break;
+                    c0 += n_mine;
                 }
-                const int q = a.v_src ? (p >> 1) : p;
-                const bool is_v = a.v_src && (p & 1);
-                const int rq0 = q * S::kGRows;
-                const int len = min(S::kGRows, m - rq0);
-                const uint4* buf = reinterpret_cast<const uint4*>(regA + sb * S::kGStage);
-                uint4* dst = (is_v ? vd : kd) + (u * a.cap_dst + rq0) * kVec;
-                const int nv = len * kVec;
-                for (int e = lane; e < nv; e += 32) st_stream(dst + e, buf[e]);
-                __syncwarp();
-                mbar_arrive(&gempty[sb]);
+            } else if (tid < S::kMath) {
+                // Math warps: positions of the kept rows (8 loads in flight per
+                // thread), then drain pieces warp, warp + kMathWarps, ... to global
+                // memory.
+                copy_positions();
+                for (int p = warp; p < npc; p += S::kMathWarps) {
+                    const uint32_t pc = pieces_done + p;
+                    const int sb = pc % n_gstages;
+                    if (!mbar_wait(&gfull[pc % S::kPieceBars], (pc / S::kPieceBars) & 1, a.flag)) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                    const int q = a.v_src ? (p >> 1) : p;
+                    const bool is_v = a.v_src && (p & 1);
+                    const int rq0 = q * S::kGRows;
+                    const int len = min(S::kGRows, m - rq0);
+                    const uint4* buf = reinterpret_cast<const uint4*>(regA + sb * S::kGStage);
+                    uint4* dst = (is_v ? vd : kd) + (u * a.cap_dst + rq0) * kVec;
+                    const int nv = len * kVec;
+                    // Two halves through registers (8 loads in flight per lane);
+                    // the buffer is freed once its second half is read.
+                    constexpr int kHalf = S::kGStage / 16 / 32 / 2;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint4 v[kHalf];
+#pragma unroll
+                        for (int i = 0; i < kHalf; ++i) {
+                            const int e = lane + 32 * (h * kHalf + i);
+                            if (e < nv) v[i] = buf[e];
+                        }
+                        if (h == 1) {
+                            __syncwarp();
+                            mbar_arrive(&gempty[sb]);
+                        }
+#pragma unroll
+                        for (int i = 0; i < kHalf; ++i) {
+                            const int e = lane + 32 * (h * kHalf + i);
+                            if (e < nv) st_stream(dst + e, v[i]);
+                        }
+                    }
+                }
             }
         }
         if (a.kept)
@@ -527,7 +661,10 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
         trace_point(a, u, 4);
         __syncthreads();
         tiles_done += n_tiles;
-        pieces_done += static_cast<uint32_t>(npc);
+        if (dense)
+            dense_done += static_cast<uint32_t>(npc);
+        else
+            pieces_done += static_cast<uint32_t>(npc);
         fence_proxy_async();
         __syncthreads();
     }

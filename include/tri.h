@@ -286,7 +286,7 @@ int tri_prune_path(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, in
 /*
  * Append n_new rows per unit to a cache: rows n_valid[u] .. n_valid[u]+n_new-1
  * of unit u receive k_new[u][i], v_new[u][i], pos_new[u][i]; n_valid[u] grows by
- * n_new; p_cur[seq] is set to 1 + the largest appended position of the
+ * n_new; p_cur[seq] is set to 1 + the largest position in pos_new of the
  * sequence's units.  Used by the windowed driver that prunes every 128
  * generated tokens (hyper.ai summary, Method section).  A unit whose rows
  * would exceed cap is left unchanged and sets TRI_FLAG_NVALID_RANGE.

@@ -679,11 +679,13 @@ tri_status tri_append(void* k_cache, void* v_cache, int32_t* pos_cache, tri_dtyp
                       const int32_t* pos_new, int64_t n_new, void* ws, size_t ws_bytes,
                       void* stream) {
     LaunchScope scope_;
-    if (!k_cache || !k_new || !n_valid || n_seq < 1 || n_units < 1 || cap < 1 || n_new < 0)
+    if (!k_cache || !n_valid || n_seq < 1 || n_units < 1 || cap < 1 || n_new < 0)
         return TRI_ERR_INVALID_ARG;
+    if (n_new > 0 && !k_new) return TRI_ERR_INVALID_ARG;  // nothing is read when n_new == 0
     if (!dtype_ok(dt) || head_dim != kD) return TRI_ERR_UNSUPPORTED;
     if (n_units % n_seq != 0 || n_units > 65535) return TRI_ERR_INVALID_ARG;
-    if ((v_cache == nullptr) != (v_new == nullptr) || (pos_cache == nullptr) != (pos_new == nullptr))
+    if (n_new > 0 && ((v_cache == nullptr) != (v_new == nullptr) ||
+                      (pos_cache == nullptr) != (pos_new == nullptr)))
         return TRI_ERR_INVALID_ARG;
     if (p_cur && !pos_new) return TRI_ERR_INVALID_ARG;
     if (!aligned16(k_cache) || !aligned16(k_new) ||

@@ -170,10 +170,11 @@ cudaError_t launch_append(tri_dtype dt, void* k_cache, void* v_cache, int32_t* p
             static_cast<const uint4*>(k_new), static_cast<const uint4*>(v_new), pos_new, n_new, flag);
         note_launch(s);
     }
-    if (p_cur && pos_new && n_new > 0)
+    if (p_cur && pos_new && n_new > 0) {
         append_pcur_kernel<<<static_cast<unsigned>(n_seq), 256, 0, s>>>(p_cur, n_units / n_seq,
                                                                          pos_new, n_new);
         note_launch(s);
+    }
     return cudaGetLastError();
 }
 

@@ -217,22 +217,31 @@ def _check_prune(spec, wl, ost, out, B, nv, units):
 
 
 def _oracle_units(spec, wl, ost, B, nv, units):
-    """Oracle on a sample of units without copying the whole cache to the host."""
+    """Oracle on a sample of units without copying the whole cache to the host:
+    the sampled units that share a current position go to one oracle call as
+    a stack of single-head "layers" (each with its own statistics), so the
+    oracle's threads run over them."""
     U, cap = spec.n_units, spec.cap
     fin = np.full((U, cap), np.nan)
     kept = np.full((U, B), -1, np.int32)
-    idx = torch.as_tensor(list(units), device="cuda")
-    kk = synth.host_elems(wl.k[idx])
-    pp = wl.pos[idx].cpu().numpy()
     pc = wl.p_cur.cpu().numpy()
     Lh = spec.n_layers * spec.n_kvheads
-    for i, u in enumerate(units):
-        seq, layer, kvh = u // Lh, (u // spec.n_kvheads) % spec.n_layers, u % spec.n_kvheads
-        st = ost[layer:layer + 1, kvh * spec.G:(kvh + 1) * spec.G]
-        o = oracle.prune(kk[i:i + 1], None, pp[i:i + 1], 1, 1, 1, spec.G, st, pc[seq:seq + 1], B,
-                         n_valid=nv[u:u + 1], want_gather=False, want_raw=False)
-        fin[u] = o["final"][0]
-        kept[u] = o["kept"][0]
+    by_pcur = {}
+    for u in units:
+        by_pcur.setdefault(int(pc[u // Lh]), []).append(u)
+    for p_cur, us in by_pcur.items():
+        idx = torch.as_tensor(us, device=wl.k.device)
+        kk = synth.host_elems(wl.k[idx])
+        pp = wl.pos[idx].cpu().numpy()
+        st = np.stack([ost[(u // spec.n_kvheads) % spec.n_layers,
+                           (u % spec.n_kvheads) * spec.G:(u % spec.n_kvheads + 1) * spec.G]
+                       for u in us])
+        o = oracle.prune(kk, None, pp, 1, len(us), 1, spec.G, st, np.asarray([p_cur]), B,
+                         n_valid=np.asarray([nv[u] for u in us]), want_gather=False,
+                         want_raw=False)
+        for i, u in enumerate(us):
+            fin[u] = o["final"][i]
+            kept[u] = o["kept"][i]
     return dict(final=fin, kept=kept)
 
 
@@ -270,8 +279,12 @@ def test_prune_paths_agree():
             assert H.rows_equal(other["v"][u], wl.v[u], other["kept"][u])
 
 
-@pytest.mark.parametrize("name,sample", [("c1", None), ("c2", None), ("c3", 24)])
+@pytest.mark.parametrize("name,sample", [("c1", None), ("c2", None), ("c3", 24), ("c5", 16),
+                                         ("c4", 4)])
 def test_prune_parity_config(name, sample):
+    """Every workload configuration at its full size, in the launch the bench
+    times (the path tri_prune picks); units sampled where the oracle would
+    take too long on all of them."""
     spec = synth.SPECS[name]
     wl = synth.make_workload(spec, "cuda")
     gst, ost = H.stats_for(spec, wl)

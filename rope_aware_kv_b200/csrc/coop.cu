@@ -92,10 +92,12 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
 
 // Unit-wide barrier: arrive on the unit's counter, wait (bounded) until
 // `target` arrivals.  Returns false, for every thread of the CTA, if this or
-// an earlier barrier gave up.
+// an earlier barrier gave up.  The CTA barrier orders every thread's writes
+// before thread 0's device-scope fence and arrival (the fence is cumulative),
+// and thread 0's fence after the wait orders the other CTAs' writes before
+// everything that follows the second CTA barrier.
 __device__ __forceinline__ bool unit_barrier(uint32_t* ctr, uint32_t target, uint32_t* flag,
                                              int* abort_flag) {
-    __threadfence();  // this thread's global writes before the arrival
     __syncthreads();
     if (threadIdx.x == 0 && !*abort_flag) {
         __threadfence();
@@ -449,29 +451,50 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
             // Pairs of entries; an odd count also copies the unused slot nc.
             copy_l2_to_shared(reinterpret_cast<uint4*>(cs),
                               reinterpret_cast<const uint4*>(a.cand + u * kCandMax), (nc + 1) / 2);
-            for (int p = 0; p < 3; ++p) {
-                const int nb = 1 << pass_bits(p);
-                for (int b = tid; b < nb; b += S::kThreads) hist[b] = 0;
-                __syncthreads();
-                const uint32_t prefix = st->prefix;
-                const int shift = pass_shift(p);
-                const int hi_shift = shift + pass_bits(p);
-                for (int i = tid; i < nc; i += S::kThreads) {
-                    const uint32_t key = static_cast<uint32_t>(cs[i].x);
-                    if (p == 0 || (key >> hi_shift) == prefix)
-                        atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+            if (nc <= S::kThreads) {
+                // Few candidates: thread i ranks candidate i against all of
+                // them by (key desc, index asc); rank k0 - 1 is the threshold.
+                const uint32_t k0 = st->k;
+                __syncthreads();  // the list is staged and k0 read before st changes
+                const int2 me = tid < nc ? cs[tid] : make_int2(0, 0);
+                const uint32_t mk = static_cast<uint32_t>(me.x);
+                uint32_t above = 0, rank = 0;
+                for (int i = 0; i < nc; ++i) {
+                    const int2 e = cs[i];
+                    const uint32_t ek = static_cast<uint32_t>(e.x);
+                    above += ek > mk;
+                    rank += (ek > mk) || (ek == mk && e.y < me.y);
+                }
+                if (tid < nc && rank == k0 - 1) {
+                    st->prefix = mk;
+                    st->k = k0 - above;  // ties of the threshold key that are kept
                 }
                 __syncthreads();
-                if (warp == 0) {
-                    uint32_t bin, above;
-                    warp_find_bin(hist, nb, st->k, bin, above);
-                    if (lane == 0) {
-                        st->prefix = (prefix << pass_bits(p)) | bin;
-                        st->k -= above;
-                        st->gt += above;
+            } else {
+                for (int p = 0; p < 3; ++p) {
+                    const int nb = 1 << pass_bits(p);
+                    for (int b = tid; b < nb; b += S::kThreads) hist[b] = 0;
+                    __syncthreads();
+                    const uint32_t prefix = st->prefix;
+                    const int shift = pass_shift(p);
+                    const int hi_shift = shift + pass_bits(p);
+                    for (int i = tid; i < nc; i += S::kThreads) {
+                        const uint32_t key = static_cast<uint32_t>(cs[i].x);
+                        if (p == 0 || (key >> hi_shift) == prefix)
+                            atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
                     }
+                    __syncthreads();
+                    if (warp == 0) {
+                        uint32_t bin, above;
+                        warp_find_bin(hist, nb, st->k, bin, above);
+                        if (lane == 0) {
+                            st->prefix = (prefix << pass_bits(p)) | bin;
+                            st->k -= above;
+                            st->gt += above;
+                        }
+                    }
+                    __syncthreads();
                 }
-                __syncthreads();
             }
             // Kept rows and threshold ties in the CTAs before this one: their
             // keys above b0 (the published counts), their candidates above the

@@ -15,9 +15,10 @@
 //           load feeds 4 keys); per-head scores go to a per-CTA float32
 //           scratch that stays in L2, float64 moments stay in registers.
 //   z-max   fixed-order moment merge, final = max_h z_h into shared memory,
-//           first radix digit histogram.
-//   select  two more radix digits on shared-memory histograms, then the
-//           ordered compaction of kept indices (warp ballots).
+//           histogram of its linear z-bins.
+//   select  the keys in the z-bin of the B-th key are listed and ranked
+//           (directly, or by a three-digit radix of their full keys), then
+//           the ordered compaction of kept indices (warp ballots).
 //   gather  kept rows form runs of consecutive indices; one lane fills 8 KB
 //           shared buffers, each with kGRows consecutive destination rows of K
 //           or V, by one cp.async.bulk per run piece (the whole TMA ring, up
@@ -303,7 +304,7 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
                             }
                             fin[j] = best;
                             if (best != best) nonfinite = true;
-                            atomicAdd(&hist[ordered_key(best) >> pass_shift(0)], 1u);
+                            atomicAdd(&hist[zbin(best)], 1u);
                         }
                     }
                 }
@@ -311,40 +312,102 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
             }
             trace_point(a, u, 2);
             __syncthreads();
-            // ---------------- radix passes 1 and 2 ----------------
+            // ---------------- threshold ----------------
+            // The z-bin b0 of the B-th key; the keys in b0 (the candidates)
+            // go to a list in the free TMA ring, and the B-th key is found
+            // among them: by direct ranking when there are at most one per
+            // thread, else by a three-digit radix select of their full keys;
+            // if they do not fit the list, by the same radix over the keys of
+            // b0 in place.
+            uint32_t* zb0 = reinterpret_cast<uint32_t*>(base + L.misc + 152);
+            int32_t* ncand = reinterpret_cast<int32_t*>(base + L.misc + 156);
             if (warp == 0) {
                 uint32_t bin, above;
-                warp_find_bin(hist, 1 << pass_bits(0), static_cast<uint32_t>(B), bin, above);
+                warp_find_bin(hist, kZBins, static_cast<uint32_t>(B), bin, above);
                 if (lane == 0) {
-                    st->prefix = bin;
-                    st->k = static_cast<uint32_t>(B) - above;
+                    *zb0 = bin;
+                    *ncand = 0;
+                    st->prefix = 0;
+                    st->k = static_cast<uint32_t>(B) - above;  // to take from bin b0
                     st->gt = above;
                     st->keep_all = 0;
                 }
             }
             __syncthreads();
-            for (int p = 1; p < 3; ++p) {
-                const int nb = 1 << pass_bits(p);
-                for (int b = tid; b < nb; b += S::kThreads) hist[b] = 0;
-                __syncthreads();
-                const uint32_t prefix = st->prefix;
-                const int shift = pass_shift(p);
-                const int hi_shift = shift + pass_bits(p);
-                for (int j = tid; j < n; j += S::kThreads) {
-                    const uint32_t key = ordered_key(fin[j]);
-                    if ((key >> hi_shift) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+            const uint32_t b0 = *zb0;
+            int2* cand = reinterpret_cast<int2*>(regA + kHistBins0 * 4);
+            const int cand_cap =
+                static_cast<int>((static_cast<size_t>(n_stages) * S::kStageBytes - kHistBins0 * 4) / 8);
+            {
+                const uint32_t lt = (1u << lane) - 1u;
+                for (int j0 = warp * 32; j0 < n; j0 += S::kWarps * 32) {
+                    const int j = j0 + lane;
+                    const float f = j < n ? fin[j] : 0.f;
+                    const bool is_c = j < n && zbin(f) == b0;
+                    const uint32_t bc = __ballot_sync(0xffffffffu, is_c);
+                    if (bc == 0u) continue;
+                    int slot = 0;
+                    if (lane == 0) slot = atomicAdd(ncand, __popc(bc));
+                    slot = __shfl_sync(0xffffffffu, slot, 0);
+                    const int r = slot + __popc(bc & lt);
+                    if (is_c && r < cand_cap) cand[r] = make_int2(static_cast<int>(ordered_key(f)), j);
+                }
+            }
+            __syncthreads();
+            const int nc = *ncand;
+            if (nc <= S::kThreads) {
+                const uint32_t k0 = st->k;
+                __syncthreads();  // k0 read before st changes
+                const int2 me = tid < nc ? cand[tid] : make_int2(0, 0);
+                const uint32_t mk = static_cast<uint32_t>(me.x);
+                uint32_t above = 0, rank = 0;
+                for (int i = 0; i < nc; ++i) {
+                    const int2 e = cand[i];
+                    const uint32_t ek = static_cast<uint32_t>(e.x);
+                    above += ek > mk;
+                    rank += (ek > mk) || (ek == mk && e.y < me.y);
+                }
+                if (tid < nc && rank == k0 - 1) {
+                    st->prefix = mk;
+                    st->k = k0 - above;  // ties of the threshold key that are kept
                 }
                 __syncthreads();
-                if (warp == 0) {
-                    uint32_t bin, above;
-                    warp_find_bin(hist, nb, st->k, bin, above);
-                    if (lane == 0) {
-                        st->prefix = (prefix << pass_bits(p)) | bin;
-                        st->k -= above;
-                        st->gt += above;
+            } else {
+                const bool listed = nc <= cand_cap;
+                for (int p = 0; p < 3; ++p) {
+                    const int nb = 1 << pass_bits(p);
+                    for (int b = tid; b < nb; b += S::kThreads) hist[b] = 0;
+                    __syncthreads();
+                    const uint32_t prefix = st->prefix;
+                    const int shift = pass_shift(p);
+                    const int hi_shift = shift + pass_bits(p);
+                    const int cnt = listed ? nc : n;
+                    for (int i = tid; i < cnt; i += S::kThreads) {
+                        uint32_t key;
+                        bool in_bin;
+                        if (listed) {
+                            key = static_cast<uint32_t>(cand[i].x);
+                            in_bin = true;
+                        } else {
+                            const float f = fin[i];
+                            key = ordered_key(f);
+                            in_bin = zbin(f) == b0;
+                        }
+                        if (in_bin && (p == 0 || (key >> hi_shift) == prefix))
+                            atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
                     }
+                    __syncthreads();
+                    if (warp == 0) {
+                        uint32_t bin, above;
+                        warp_find_bin(hist, nb, st->k, bin, above);
+                        if (lane == 0) {
+                            st->prefix = (prefix << pass_bits(p)) | bin;
+                            st->k -= above;
+                            st->gt += above;
+                        }
+                    }
+                    __syncthreads();
                 }
-                __syncthreads();
             }
             // ---------------- ordered compaction of indices ----------------
             {

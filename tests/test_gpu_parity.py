@@ -353,6 +353,23 @@ def test_threshold_tie_group_beyond_candidate_list(path):
         assert H.rows_equal(out["v"][u], wl.v[u], out["kept"][u])
 
 
+@pytest.mark.parametrize("path", [tri.PATH_FUSED, tri.PATH_COOP, tri.PATH_SPLIT])
+def test_identical_keys_beyond_every_candidate_list(path):
+    """17000 equal keys (sigma = 0, every score 0, one z-bin): more than the
+    fused kernel's candidate list in a four-stage ring (15360) and the
+    cooperative kernel's (8192), so both rank the tie in place; the lowest B
+    indices are kept."""
+    B = 6000
+    spec = _spec(dtype="bf16", G=1, n_seq=1, n_layers=1, n_kvheads=1, cap=17000, B=B)
+    wl = synth.make_workload(spec, "cuda")
+    wl.k[:] = wl.k[:, :1]
+    gst, _ = H.stats_for(spec, wl)
+    out = _run_prune(spec, wl, gst, B, path=path)
+    assert out["flags"] == 0
+    np.testing.assert_array_equal(out["kept"][0], np.arange(B))
+    assert H.rows_equal(out["v"][0], wl.v[0], np.arange(B))
+
+
 @pytest.mark.parametrize("path", [tri.PATH_FUSED, tri.PATH_SPLIT, tri.PATH_COOP])
 def test_nan_key_poisons_unit_and_flags(path):
     """A NaN key makes that unit's moments NaN: every final score is NaN,

@@ -204,6 +204,15 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
                                 &full[l % S::kTileBars],
                                 b * (128 / static_cast<int>(sizeof(T))), y);
             }
+            // The CTA's other tiles are requested into L2 at once.
+            const char* kunit = static_cast<const char*>(a.k_src) + u * a.cap * S::kRowBytes;
+            const uint64_t pol = policy_evict_last();
+            for (int l = a.stages; l < nt; ++l) {
+                const int t = t0 + l;
+                const int rows = min(S::kTile, static_cast<int>(a.cap) - t * S::kTile);
+                prefetch_l2_bulk(kunit + static_cast<int64_t>(t) * S::kStageBytes,
+                                 static_cast<uint32_t>(rows * S::kRowBytes), pol);
+            }
         }
         fold_unit<G>(fs, a.fc, w, a.stats, a.p_cur, u, a.n_layers, a.n_kvheads);
         if (tid >= S::kMath) {

@@ -33,6 +33,12 @@
 #include "tri_internal.cuh"
 #include "tri_launch.h"
 
+// How many key tiles ahead of its shared-memory ring the fused kernel asks
+// L2 to fetch (0: no prefetch).
+#ifndef TRI_PREFETCH_TILES
+#define TRI_PREFETCH_TILES 6
+#endif
+
 namespace tri {
 
 template <typename T>
@@ -51,18 +57,27 @@ struct FusedShape {
     static constexpr int kGStage = 8192;                                // gather piece buffer
     static constexpr int kMaxGStages = kMaxStages * kStageBytes / kGStage;
     static constexpr int kGRows = kGStage / kRowBytes;                  // rows per piece
-    // "Landed" barriers are indexed by the running tile / piece count, not by
-    // the ring stage.  A math warp takes every kMathWarps-th tile, so it skips
-    // phases of a stage's barrier; a parity wait on a barrier that is more
-    // than one phase behind would pass at once.  When a warp waits for tile t
-    // it has finished tile t - kMathWarps, so every tile up to
-    // t - kMathWarps - 1 - stages has been consumed; with kTileBars >=
-    // kMathWarps + 1 + kMaxStages the previous use of barrier t % kTileBars
-    // (tile t - kTileBars) is among them, and the wait is exact.  Same for
-    // gather pieces with kPieceBars >= kMathWarps + 1 + kMaxGStages.
-    static constexpr int kTileBars = 16;
+    // The score ring holds half tiles (16 KB: one 128-byte TMA box of bf16
+    // rows, two of float32 rows), so a warp frees the first half of its tile
+    // while it scores the second.  Half h of tile t is ring slot 2t + h.
+    static constexpr int kHalfBoxes = kBoxes / 2;
+    static constexpr int kHalfBytes = kStageBytes / 2;
+    static constexpr int kHalfChunks = kHalfBoxes * 8;                   // 16-byte chunks per half
+    static constexpr int kMaxHStages = 2 * kMaxStages;
+    static constexpr int kPrefetchTiles = TRI_PREFETCH_TILES;  // L2 prefetch distance, tiles
+    // "Landed" barriers are indexed by the running half-tile / piece count,
+    // not by the ring stage.  A math warp takes every kMathWarps-th tile, so
+    // it skips phases of a stage's barrier; a parity wait on a barrier that is
+    // more than one phase behind would pass at once.  When a warp waits for a
+    // half of tile t it has finished tile t - kMathWarps, so every half up to
+    // 2 (t - kMathWarps) - half stages has been consumed; with kHalfBars >=
+    // 2 kMathWarps + 1 + kMaxHStages the previous use of the half's barrier
+    // (kHalfBars halves earlier) is among them, and the wait is exact.  Same
+    // for gather pieces with kPieceBars >= kMathWarps + 1 + kMaxGStages.
+    static constexpr int kHalfBars = 32;
     static constexpr int kPieceBars = 32;
-    static_assert(kTileBars >= kMathWarps + 1 + kMaxStages, "tile barriers too few");
+    static_assert(kBoxes % 2 == 0, "a tile splits into two halves of whole boxes");
+    static_assert(kHalfBars >= 2 * kMathWarps + 1 + kMaxHStages, "half-tile barriers too few");
     static_assert(kPieceBars >= kMathWarps + 1 + kMaxGStages, "piece barriers too few");
     // Dense gather (most rows kept): 16 KB buffers of kDRows source rows.
     static constexpr int kDStage = 16384;
@@ -86,7 +101,7 @@ __host__ __device__ inline FusedLayout fused_layout(int G, int64_t cap, int64_t 
     L.fin = L.w + static_cast<size_t>(G) * kWHead * 4;
     L.kidx = L.fin + static_cast<size_t>(capP) * 4;
     L.bars = L.kidx + ((static_cast<size_t>(m) * 4 + 15) & ~size_t(15));
-    L.red = L.bars + (S::kTileBars + S::kMaxStages + 2 * S::kPieceBars + S::kMaxGStages +
+    L.red = L.bars + (S::kHalfBars + S::kMaxHStages + 2 * S::kPieceBars + S::kMaxGStages +
                       S::kMaxDStages) * 8;
     L.misc = L.red + static_cast<size_t>(FusedShape<T>::kMathWarps) * kMaxG * 2 * 8;
     // state and warp counts; alignment slack; static shared memory (fold)
@@ -110,6 +125,7 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
     uint8_t* base = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int n_stages = a.stages;
+    const int n_hstages = 2 * n_stages;  // half-tile slots of the score ring
     const int n_gstages = n_stages * S::kStageBytes / S::kGStage;
     const int n_dstages = n_stages * S::kStageBytes / S::kDStage;
     const FusedLayout L = fused_layout<T>(G, a.cap, a.B, n_stages);
@@ -117,9 +133,9 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
     float* w = reinterpret_cast<float*>(base + L.w);
     float* fin = reinterpret_cast<float*>(base + L.fin);
     int32_t* kidx = reinterpret_cast<int32_t*>(base + L.kidx);
-    uint64_t* full = reinterpret_cast<uint64_t*>(base + L.bars);  // [kTileBars] tile landed
-    uint64_t* empty = full + S::kTileBars;                         // [stages] stage free
-    uint64_t* gfull = empty + S::kMaxStages;                       // [kPieceBars] piece landed
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + L.bars);  // [kHalfBars] half landed
+    uint64_t* empty = full + S::kHalfBars;                         // [half stages] stage free
+    uint64_t* gfull = empty + S::kMaxHStages;                      // [kPieceBars] piece landed
     uint64_t* gempty = gfull + S::kPieceBars;                      // [gather stages] buffer free
     uint64_t* dfull = gempty + S::kMaxGStages;                     // dense: [kPieceBars] landed
     uint64_t* dempty = dfull + S::kPieceBars;                      // dense: [stages] free
@@ -138,8 +154,8 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
     float* scratch = a.scratch + static_cast<int64_t>(blockIdx.x) * G * a.cap;
 
     if (tid == S::kMath) {
-        for (int i = 0; i < S::kTileBars; ++i) mbar_init(&full[i], 1);
-        for (int i = 0; i < n_stages; ++i) mbar_init(&empty[i], 32);
+        for (int i = 0; i < S::kHalfBars; ++i) mbar_init(&full[i], 1);
+        for (int i = 0; i < n_hstages; ++i) mbar_init(&empty[i], 32);
         for (int i = 0; i < S::kPieceBars; ++i) mbar_init(&gfull[i], 1);
         for (int i = 0; i < n_gstages; ++i) mbar_init(&gempty[i], 32);
         for (int i = 0; i < S::kPieceBars; ++i) mbar_init(&dfull[i], 1);
@@ -165,46 +181,52 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
 
         if (!keep_all) {
             // ---------------- score ----------------
-            // The first tiles of the unit are requested before the fold so
-            // that their loads overlap it (every ring stage is free here).
-            const int pre = n_tiles < n_stages ? n_tiles : n_stages;
+            // The first half tiles of the unit are requested before the fold
+            // so that their loads overlap it (every ring slot is free here).
+            // Keys stay in L2 for the kept-row re-read of the gather.
+            const int n_halves = 2 * n_tiles;
+            const int pre = n_halves < n_hstages ? n_halves : n_hstages;
+            auto issue_half = [&](int hh, uint64_t pol) {  // hh: half index within the unit
+                const uint32_t hc = 2 * tiles_done + hh;
+                uint64_t* landed = &full[hc % S::kHalfBars];
+                mbar_arrive_expect_tx(landed, S::kHalfBytes);
+                const int32_t y =
+                    static_cast<int32_t>(u * a.cap + static_cast<int64_t>(hh >> 1) * S::kTile);
+#pragma unroll
+                for (int b = 0; b < S::kHalfBoxes; ++b)
+                    tma_load_2d_hint(regA + (hc % n_hstages) * S::kHalfBytes + b * S::kBoxBytes,
+                                     &kmap, landed,
+                                     ((hh & 1) * S::kHalfBoxes + b) * (128 / static_cast<int>(sizeof(T))),
+                                     y, pol);
+            };
+            // Tiles beyond the ring are requested into L2 kPrefetchTiles ahead
+            // of their load into shared memory, so that far more bytes are in
+            // flight than the ring holds (most of it is being scored).
+            const char* kunit = static_cast<const char*>(a.k_src) + u * a.cap * S::kRowBytes;
+            auto prefetch_tile = [&](int t, uint64_t pol) {
+                if (S::kPrefetchTiles == 0 || t >= n_tiles) return;
+                const int rows = min(S::kTile, static_cast<int>(a.cap) - t * S::kTile);
+                prefetch_l2_bulk(kunit + static_cast<int64_t>(t) * S::kStageBytes,
+                                 static_cast<uint32_t>(rows * S::kRowBytes), pol);
+            };
             if (tid == S::kMath) {
                 const uint64_t keep_pol = policy_evict_last();
-                for (int i = 0; i < pre; ++i) {
-                    const uint32_t tc = tiles_done + i;
-                    const int stage = tc % n_stages;
-                    uint64_t* landed = &full[tc % S::kTileBars];
-                    mbar_arrive_expect_tx(landed, S::kStageBytes);
-                    const int32_t y =
-                        static_cast<int32_t>(u * a.cap + static_cast<int64_t>(i) * S::kTile);
-#pragma unroll
-                    for (int b = 0; b < S::kBoxes; ++b)
-                        tma_load_2d_hint(regA + stage * S::kStageBytes + b * S::kBoxBytes, &kmap,
-                                         landed, b * (128 / static_cast<int>(sizeof(T))), y,
-                                         keep_pol);
-                }
+                for (int hh = 0; hh < pre; ++hh) issue_half(hh, keep_pol);
+                for (int t = pre / 2; t < pre / 2 + S::kPrefetchTiles; ++t) prefetch_tile(t, keep_pol);
             }
             fold_unit<G>(fs, a.fc, w, a.stats, a.p_cur, u, a.n_layers, a.n_kvheads);
             if (tid >= S::kMath) {
                 if (tid == S::kMath) {
-                    // Keys stay in L2 for the kept-row re-read of the gather.
                     const uint64_t keep_pol = policy_evict_last();
-                    for (int i = pre; i < n_tiles; ++i) {
-                        const uint32_t tc = tiles_done + i;
-                        const int stage = tc % n_stages;
-                        if (!mbar_wait(&empty[stage], ((tc / n_stages) & 1) ^ 1, a.flag)) {
+                    for (int hh = pre; hh < n_halves; ++hh) {
+                        const uint32_t hc = 2 * tiles_done + hh;
+                        const int slot = hc % n_hstages;
+                        if (!mbar_wait(&empty[slot], ((hc / n_hstages) & 1) ^ 1, a.flag)) {
                             *abort_flag = 1;
                             break;
                         }
-                        uint64_t* landed = &full[tc % S::kTileBars];
-                        mbar_arrive_expect_tx(landed, S::kStageBytes);
-                        const int32_t y =
-                            static_cast<int32_t>(u * a.cap + static_cast<int64_t>(i) * S::kTile);
-#pragma unroll
-                        for (int b = 0; b < S::kBoxes; ++b)
-                            tma_load_2d_hint(regA + stage * S::kStageBytes + b * S::kBoxBytes,
-                                             &kmap, landed,
-                                             b * (128 / static_cast<int>(sizeof(T))), y, keep_pol);
+                        issue_half(hh, keep_pol);
+                        if ((hh & 1) == 0) prefetch_tile(hh / 2 + S::kPrefetchTiles, keep_pol);
                     }
                 }
             } else {
@@ -213,17 +235,29 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
 #pragma unroll
                 for (int h = 0; h < G; ++h) m1[h] = m2[h] = 0.0;
                 for (int i = warp; i < n_tiles; i += S::kMathWarps) {
-                    const uint32_t tc = tiles_done + i;
-                    const int stage = tc % n_stages;
-                    if (!mbar_wait(&full[tc % S::kTileBars], (tc / S::kTileBars) & 1, a.flag)) {
+                    float2 acc[S::kKPT][G];
+                    score_acc_zero<G, S::kKPT>(acc);
+                    bool ok = true;
+#pragma unroll 1
+                    for (int half = 0; half < 2; ++half) {
+                        const uint32_t hc = 2 * (tiles_done + i) + half;
+                        const int slot = hc % n_hstages;
+                        if (!mbar_wait(&full[hc % S::kHalfBars], (hc / S::kHalfBars) & 1, a.flag)) {
+                            ok = false;
+                            break;
+                        }
+                        score_rows_acc<T, G, S::kKPT, S::kBoxBytes, 32>(
+                            regA + slot * S::kHalfBytes, half * S::kHalfChunks,
+                            (half + 1) * S::kHalfChunks, w, lane, acc);
+                        __syncwarp();
+                        mbar_arrive(&empty[slot]);
+                    }
+                    if (!ok) {
                         *abort_flag = 1;
                         break;
                     }
                     float s[S::kKPT][G];
-                    score_rows<T, G, S::kKPT, S::kBoxBytes, 32>(regA + stage * S::kStageBytes, w,
-                                                                 lane, s);
-                    __syncwarp();
-                    mbar_arrive(&empty[stage]);
+                    score_acc_final<G, S::kKPT>(acc, s);
 #pragma unroll
                     for (int k = 0; k < S::kKPT; ++k) {
                         const int j = i * S::kTile + lane + 32 * k;

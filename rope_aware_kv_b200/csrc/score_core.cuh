@@ -20,31 +20,33 @@ namespace tri {
 
 constexpr int kScoreUnroll = TRI_SCORE_UNROLL;
 
-// Score KPT keys of a tile held in swizzled shared memory.  Row r of box b
-// lives at b * kBoxBytes + r * 128 and its 16-byte chunk j at position
-// (j ^ (r & 7)) (TMA 128-byte swizzle), so 8 consecutive threads reading the
-// same logical chunk of 8 consecutive rows hit 8 different bank groups.
-// Rows first_row + kRowStride * k (k < KPT) of the tile; w points at the
-// weight record of the first of the G heads scored here.
-template <typename T, int G, int KPT, int kBoxBytes, int kRowStride>
-__device__ __forceinline__ void score_rows(const uint8_t* tile, const float* w, int first_row,
-                                           float (&s)[KPT][G]) {
-    float2 acc[KPT][G];
-#pragma unroll
-    for (int k = 0; k < KPT; ++k)
-#pragma unroll
-        for (int h = 0; h < G; ++h) acc[k][h] = make_float2(0.f, 0.f);
+// Chunks (16 bytes: 4 bf16 bands or 2 float32 bands) per key row.
+template <typename T>
+__host__ __device__ constexpr int row_chunks() { return sizeof(T) == 2 ? kChunks : 2 * kChunks; }
 
+// Accumulate chunks [c0, c1) of KPT keys into acc.  The keys live in
+// swizzled shared memory as 128-byte TMA boxes: chunk c of row r is at
+// boxes + ((c >> 3) - (c0 >> 3)) * kBoxBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4)
+// (TMA 128-byte swizzle: 8 consecutive threads reading the same logical
+// chunk of 8 consecutive rows hit 8 different bank groups), so `boxes` may
+// hold the whole tile (c0 = 0) or only the boxes from c0 on.  Rows
+// first_row + kRowStride * k (k < KPT); w points at the weight record of the
+// first of the G heads scored here.  Scoring a tile in parts accumulates in
+// the same order as scoring it whole.
+template <typename T, int G, int KPT, int kBoxBytes, int kRowStride>
+__device__ __forceinline__ void score_rows_acc(const uint8_t* boxes, int c0, int c1, const float* w,
+                                               int first_row, float2 (&acc)[KPT][G]) {
+    const int box0 = c0 >> 3;
     if constexpr (sizeof(T) == 2) {
 #pragma unroll kScoreUnroll
-        for (int c = 0; c < kChunks; ++c) {
+        for (int c = c0; c < c1; ++c) {
             float2 xy[KPT][4];
             float2 nn[KPT][2];
 #pragma unroll
             for (int k = 0; k < KPT; ++k) {
                 const int r = first_row + kRowStride * k;
                 const uint4 v = *reinterpret_cast<const uint4*>(
-                    tile + (c >> 3) * kBoxBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+                    boxes + ((c >> 3) - box0) * kBoxBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
                 const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
                 float n[4];
 #pragma unroll
@@ -76,14 +78,14 @@ __device__ __forceinline__ void score_rows(const uint8_t* tile, const float* w, 
     } else {
         // float32 rows: 32 chunks of 4 floats (2 bands each).
 #pragma unroll 4
-        for (int c = 0; c < 2 * kChunks; ++c) {
+        for (int c = c0; c < c1; ++c) {
             float2 xy[KPT][2];
             float2 nn[KPT];
 #pragma unroll
             for (int k = 0; k < KPT; ++k) {
                 const int r = first_row + kRowStride * k;
                 const float4 v = *reinterpret_cast<const float4*>(
-                    tile + (c >> 3) * kBoxBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+                    boxes + ((c >> 3) - box0) * kBoxBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
                 xy[k][0] = make_float2(v.x, v.y);
                 xy[k][1] = make_float2(v.z, v.w);
                 nn[k] = make_float2(sqrt_approx(fmaf(v.x, v.x, v.y * v.y)),
@@ -106,75 +108,32 @@ __device__ __forceinline__ void score_rows(const uint8_t* tile, const float* w, 
             }
         }
     }
-#pragma unroll
-    for (int k = 0; k < KPT; ++k)
-#pragma unroll
-        for (int h = 0; h < G; ++h) s[k][h] = acc[k][h].x + acc[k][h].y;
 }
 
-// Partial scores over half of the bands (bf16 rows): chunks 8*half .. 8*half+7,
-// i.e. TMA box `half` of the tile, for all G heads.  Two warps that each take
-// one half of the same keys produce the full score as the sum of their parts.
-template <typename T, int G, int KPT, int kBoxBytes, int kRowStride, int kHalf>
-__device__ __forceinline__ void score_rows_half_t(const uint8_t* tile, const float* w,
-                                                  int first_row, float (&s)[KPT][G]) {
-    static_assert(sizeof(T) == 2, "band split is for bfloat16 rows");
-    float2 acc[KPT][G];
+template <int G, int KPT>
+__device__ __forceinline__ void score_acc_zero(float2 (&acc)[KPT][G]) {
 #pragma unroll
     for (int k = 0; k < KPT; ++k)
 #pragma unroll
         for (int h = 0; h < G; ++h) acc[k][h] = make_float2(0.f, 0.f);
-#pragma unroll kScoreUnroll
-    for (int cc = 0; cc < 8; ++cc) {
-        const int c = kHalf * 8 + cc;
-        float2 xy[KPT][4];
-        float2 nn[KPT][2];
-#pragma unroll
-        for (int k = 0; k < KPT; ++k) {
-            const int r = first_row + kRowStride * k;
-            const uint4 v = *reinterpret_cast<const uint4*>(tile + kHalf * kBoxBytes + r * 128 +
-                                                            ((cc ^ (r & 7)) << 4));
-            const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
-            float n[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float x = bf16_lo(wd[i]), y = bf16_hi(wd[i]);
-                xy[k][i] = make_float2(x, y);
-                n[i] = sqrt_approx(fmaf(x, x, y * y));
-            }
-            nn[k][0] = make_float2(n[0], n[1]);
-            nn[k][1] = make_float2(n[2], n[3]);
-        }
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-            const float4* rec = reinterpret_cast<const float4*>(w + h * kWHead + c * kWChunk);
-            const float4 a = rec[0], b = rec[1], cw = rec[2];
-#pragma unroll
-            for (int k = 0; k < KPT; ++k) {
-                float2 t = acc[k][h];
-                t = __ffma2_rn(xy[k][0], make_float2(a.x, a.y), t);
-                t = __ffma2_rn(xy[k][1], make_float2(a.z, a.w), t);
-                t = __ffma2_rn(xy[k][2], make_float2(b.x, b.y), t);
-                t = __ffma2_rn(xy[k][3], make_float2(b.z, b.w), t);
-                t = __ffma2_rn(nn[k][0], make_float2(cw.x, cw.y), t);
-                t = __ffma2_rn(nn[k][1], make_float2(cw.z, cw.w), t);
-                acc[k][h] = t;
-            }
-        }
-    }
+}
+
+template <int G, int KPT>
+__device__ __forceinline__ void score_acc_final(const float2 (&acc)[KPT][G], float (&s)[KPT][G]) {
 #pragma unroll
     for (int k = 0; k < KPT; ++k)
 #pragma unroll
         for (int h = 0; h < G; ++h) s[k][h] = acc[k][h].x + acc[k][h].y;
 }
 
+// Score KPT keys of a whole tile (all chunks) into s.
 template <typename T, int G, int KPT, int kBoxBytes, int kRowStride>
-__device__ __forceinline__ void score_rows_half(const uint8_t* tile, const float* w, int first_row,
-                                                int half, float (&s)[KPT][G]) {
-    if (half == 0)
-        score_rows_half_t<T, G, KPT, kBoxBytes, kRowStride, 0>(tile, w, first_row, s);
-    else
-        score_rows_half_t<T, G, KPT, kBoxBytes, kRowStride, 1>(tile, w, first_row, s);
+__device__ __forceinline__ void score_rows(const uint8_t* tile, const float* w, int first_row,
+                                           float (&s)[KPT][G]) {
+    float2 acc[KPT][G];
+    score_acc_zero<G, KPT>(acc);
+    score_rows_acc<T, G, KPT, kBoxBytes, kRowStride>(tile, 0, row_chunks<T>(), w, first_row, acc);
+    score_acc_final<G, KPT>(acc, s);
 }
 
 }  // namespace tri

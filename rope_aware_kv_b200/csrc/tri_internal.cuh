@@ -150,6 +150,15 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint
 }
 
 // global -> shared with an L2 cache policy:
+// Ask L2 to fetch [gsrc, gsrc + bytes) ahead of its use (16-byte aligned,
+// a multiple of 16 bytes); nothing lands in shared memory.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* gsrc, uint32_t bytes, uint64_t policy) {
+    asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;" ::"l"(
+                     reinterpret_cast<uint64_t>(gsrc)),
+                 "r"(bytes), "l"(policy)
+                 : "memory");
+}
+
 __device__ __forceinline__ void bulk_load_hint(void* smem_dst, const void* gsrc, uint32_t bytes,
                                                uint64_t* bar, uint64_t policy) {
     asm volatile(

@@ -7,9 +7,10 @@
 // (hyper.ai summary, Method section), top-B by (score desc, index asc) kept
 // in temporal order (jaedaily.cn tutorial, eviction step).
 //
-//   phase 1  score the CTA's tiles (TMA ring, seven math warps, one per 128-key tile,
-//            all heads) into an L2-resident per-CTA scratch; float64 moment
-//            partial per CTA                                   -> barrier 1
+//   phase 1  score the CTA's tiles (a TMA ring of half tiles; seven math
+//            warps, each on whole 128-key tiles with all heads) into an
+//            L2-resident per-CTA scratch; float64 moment partial per CTA
+//                                                              -> barrier 1
 //   phase 2  fixed-order merge of the unit's partials; final = max_h z_h of
 //            the CTA's keys into shared memory; histogram of the linear
 //            z-bins of final added to the unit's global one    -> barrier 2
@@ -51,13 +52,22 @@ struct CoopShape {
     static constexpr int kMath = 32 * kMathWarps;
     static constexpr int kThreads = kMath + 32;
     static constexpr int kWarps = kThreads / 32;
-    // Tile-landed barriers indexed by the tile number, not the ring stage (a
-    // math warp takes every kMathWarps-th tile and so skips phases of a
-    // stage's barrier): a warp waiting for tile t has finished tile
-    // t - kMathWarps, so tiles up to t - kMathWarps - 1 - stages are consumed,
-    // including t - kTileBars, the previous use of its barrier.
-    static constexpr int kTileBars = 16;
-    static_assert(kTileBars >= kMathWarps + 1 + kMaxStages, "tile barriers too few");
+    // The ring holds half tiles (one TMA box of bf16 rows, two of float32):
+    // half h of the CTA's tile l is slot 2l + h, so a warp frees the first
+    // half of its tile while it scores the second.
+    static constexpr int kHalfBoxes = kBoxes / 2;
+    static constexpr int kHalfBytes = kStageBytes / 2;
+    static constexpr int kHalfChunks = kHalfBoxes * 8;
+    static constexpr int kMaxHStages = 2 * kMaxStages;
+    // Half-landed barriers indexed by the half number, not the ring slot (a
+    // math warp takes every kMathWarps-th tile and so skips phases of a slot's
+    // barrier): a warp waiting for a half of tile l has finished tile
+    // l - kMathWarps, so every half up to 2 (l - kMathWarps) - slots has been
+    // consumed, including the previous use of its barrier (kHalfBars halves
+    // earlier).
+    static constexpr int kHalfBars = 32;
+    static_assert(kBoxes % 2 == 0, "a tile splits into two halves of whole boxes");
+    static_assert(kHalfBars >= 2 * kMathWarps + 1 + kMaxHStages, "half barriers too few");
 };
 
 static_assert(static_cast<size_t>(kCandMax) * 8 <= 2 * CoopShape<float>::kStageBytes &&
@@ -77,7 +87,7 @@ __host__ __device__ inline CoopLayout coop_layout(int G, int64_t keys_max, int s
     L.fin = L.w + static_cast<size_t>(G) * kWHead * 4;
     L.list = L.fin + static_cast<size_t>(kp) * 4;
     L.bars = L.list + static_cast<size_t>(kp) * 8;
-    L.red = L.bars + (S::kTileBars + S::kMaxStages) * 8;
+    L.red = L.bars + (S::kHalfBars + S::kMaxHStages) * 8;
     L.misc = L.red + static_cast<size_t>(S::kMathWarps) * kMaxG * 2 * 8;
     // histogram, state; alignment slack; static shared memory (fold)
     L.total = L.misc + kHistBins0 * 4 + 512 + 1024 + kFoldStaticBytes;
@@ -136,8 +146,8 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
     float* w = reinterpret_cast<float*>(base + L.w);
     float* fin = reinterpret_cast<float*>(base + L.fin);
     int2* list = reinterpret_cast<int2*>(base + L.list);
-    uint64_t* full = reinterpret_cast<uint64_t*>(base + L.bars);  // [kTileBars] tile landed
-    uint64_t* empty = full + S::kTileBars;                         // [stages] stage free
+    uint64_t* full = reinterpret_cast<uint64_t*>(base + L.bars);  // [kHalfBars] half landed
+    uint64_t* empty = full + S::kHalfBars;                         // [half slots] slot free
     double* red = reinterpret_cast<double*>(base + L.red);  // [math warps][kMaxG][2]
     uint32_t* hist = reinterpret_cast<uint32_t*>(base + L.misc);
     SelState* st = reinterpret_cast<SelState*>(base + L.misc + kHistBins0 * 4);
@@ -184,30 +194,34 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
     } else {
         // ---------------- phase 1: score ----------------
         if (tid == S::kMath) {
-            for (int i = 0; i < S::kTileBars; ++i) mbar_init(&full[i], 1);
-            for (int i = 0; i < a.stages; ++i) mbar_init(&empty[i], 32);
+            for (int i = 0; i < S::kHalfBars; ++i) mbar_init(&full[i], 1);
+            for (int i = 0; i < 2 * a.stages; ++i) mbar_init(&empty[i], 32);
             fence_barrier_init();
             prefetch_tensormap(&kmap);
         }
         __syncthreads();  // barriers initialised before the producer starts
         const int nt = t1 - t0;
+        const int n_hslots = 2 * a.stages;
+        const int n_halves = 2 * nt;
+        const int pre = n_halves < n_hslots ? n_halves : n_hslots;
         __shared__ FoldShared fs;
-        if (tid == S::kMath) {
-            // Issue the first tile loads before the fold so they overlap it.
-            for (int l = 0; l < nt && l < a.stages; ++l) {
-                mbar_arrive_expect_tx(&full[l % S::kTileBars], S::kStageBytes);
-                const int32_t y =
-                    static_cast<int32_t>(u * a.cap + static_cast<int64_t>(t0 + l) * S::kTile);
+        auto issue_half = [&](int hh) {
+            uint64_t* landed = &full[hh % S::kHalfBars];
+            mbar_arrive_expect_tx(landed, S::kHalfBytes);
+            const int32_t y =
+                static_cast<int32_t>(u * a.cap + static_cast<int64_t>(t0 + (hh >> 1)) * S::kTile);
 #pragma unroll
-                for (int b = 0; b < S::kBoxes; ++b)
-                    tma_load_2d(ring + l * S::kStageBytes + b * S::kBoxBytes, &kmap,
-                                &full[l % S::kTileBars],
-                                b * (128 / static_cast<int>(sizeof(T))), y);
-            }
+            for (int b = 0; b < S::kHalfBoxes; ++b)
+                tma_load_2d(ring + (hh % n_hslots) * S::kHalfBytes + b * S::kBoxBytes, &kmap, landed,
+                            ((hh & 1) * S::kHalfBoxes + b) * (128 / static_cast<int>(sizeof(T))), y);
+        };
+        if (tid == S::kMath) {
+            // Issue the first half tiles before the fold so they overlap it.
+            for (int hh = 0; hh < pre; ++hh) issue_half(hh);
             // The CTA's other tiles are requested into L2 at once.
             const char* kunit = static_cast<const char*>(a.k_src) + u * a.cap * S::kRowBytes;
             const uint64_t pol = policy_evict_last();
-            for (int l = a.stages; l < nt; ++l) {
+            for (int l = pre / 2; l < nt; ++l) {
                 const int t = t0 + l;
                 const int rows = min(S::kTile, static_cast<int>(a.cap) - t * S::kTile);
                 prefetch_l2_bulk(kunit + static_cast<int64_t>(t) * S::kStageBytes,
@@ -217,19 +231,12 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
         fold_unit<G>(fs, a.fc, w, a.stats, a.p_cur, u, a.n_layers, a.n_kvheads);
         if (tid >= S::kMath) {
             if (tid == S::kMath) {
-                for (int l = a.stages; l < nt; ++l) {  // the first stages were issued above
-                    const int stage = l % a.stages;
-                    if (!mbar_wait(&empty[stage], ((l / a.stages) & 1) ^ 1, a.flag)) {
+                for (int hh = pre; hh < n_halves; ++hh) {  // the first slots were issued above
+                    if (!mbar_wait(&empty[hh % n_hslots], ((hh / n_hslots) & 1) ^ 1, a.flag)) {
                         *abort_flag = 1;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[l % S::kTileBars], S::kStageBytes);
-                    const int32_t y = static_cast<int32_t>(u * a.cap + static_cast<int64_t>(t0 + l) * S::kTile);
-#pragma unroll
-                    for (int b = 0; b < S::kBoxes; ++b)
-                        tma_load_2d(ring + stage * S::kStageBytes + b * S::kBoxBytes, &kmap,
-                                    &full[l % S::kTileBars],
-                                    b * (128 / static_cast<int>(sizeof(T))), y);
+                    issue_half(hh);
                 }
             }
         } else {
@@ -237,15 +244,28 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
 #pragma unroll
             for (int h = 0; h < G; ++h) m1[h] = m2[h] = 0.0;
             for (int l = warp; l < nt; l += S::kMathWarps) {
-                const int stage = l % a.stages;
-                if (!mbar_wait(&full[l % S::kTileBars], (l / S::kTileBars) & 1, a.flag)) {
+                float2 acc[S::kKPT][G];
+                score_acc_zero<G, S::kKPT>(acc);
+                bool ok = true;
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    const int hh = 2 * l + half;
+                    if (!mbar_wait(&full[hh % S::kHalfBars], (hh / S::kHalfBars) & 1, a.flag)) {
+                        ok = false;
+                        break;
+                    }
+                    score_rows_acc<T, G, S::kKPT, S::kBoxBytes, 32>(
+                        ring + (hh % n_hslots) * S::kHalfBytes, half * S::kHalfChunks,
+                        (half + 1) * S::kHalfChunks, w, lane, acc);
+                    __syncwarp();
+                    mbar_arrive(&empty[hh % n_hslots]);
+                }
+                if (!ok) {
                     *abort_flag = 1;
                     break;
                 }
                 float s[S::kKPT][G];
-                score_rows<T, G, S::kKPT, S::kBoxBytes, 32>(ring + stage * S::kStageBytes, w, lane, s);
-                __syncwarp();
-                mbar_arrive(&empty[stage]);
+                score_acc_final<G, S::kKPT>(acc, s);
 #pragma unroll
                 for (int k = 0; k < S::kKPT; ++k) {
                     const int jl = l * S::kTile + lane + 32 * k;  // local key index

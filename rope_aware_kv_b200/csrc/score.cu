@@ -14,10 +14,12 @@
 // one 64-wide dot product of c with the band norms |k'_f| = |k_f|.
 //
 // Data path: keys stream HBM -> shared memory by TMA (128-byte swizzle, one
-// box per 128-byte half row), a producer warp keeps STAGES tiles in flight,
-// four consumer warps compute.  Per-tile float64 moment partials are merged in
-// tile order by the last tile of each unit to finish (an atomic counter; no
-// waiting), so mu and sigma are bitwise reproducible.
+// box per 128-byte part of a row) into a ring of half tiles kept full by a
+// producer lane; seven math warps each score whole 128-key tiles (4 keys per
+// lane, all heads), the tiles of a CTA's range taken round robin within each
+// unit.  Each tile's float64 moment partial (a warp reduction) is merged in
+// tile order by the warp that finishes the unit's last tile (an atomic
+// counter; no waiting), so mu and sigma are bitwise reproducible.
 #include "tri_internal.cuh"
 #include "tri_launch.h"
 #include "score_core.cuh"
@@ -97,24 +99,36 @@ template <typename T>
 struct ScoreShape {
     static constexpr int kRowBytes = kD * static_cast<int>(sizeof(T));  // 256 / 512
     static constexpr int kBoxes = kRowBytes / 128;                      // 2 / 4
-    static constexpr int kKPT = sizeof(T) == 2 ? 2 : 1;                 // keys per thread
-    static constexpr int kTile = 128 * kKPT;                            // keys per tile
+    static constexpr int kKPT = sizeof(T) == 2 ? 4 : 2;                 // keys per lane
+    static constexpr int kTile = 32 * kKPT;                             // keys per tile
     static constexpr int kBoxBytes = kTile * 128;
-    static constexpr int kStageBytes = kTile * kRowBytes;               // 64 KB
-    static constexpr int kStages = 3;
-    static constexpr int kConsumers = 128;
-    static constexpr int kThreads = kConsumers + 32;
+    static constexpr int kStageBytes = kTile * kRowBytes;               // 32 KB
+    static constexpr int kHalfBoxes = kBoxes / 2;
+    static constexpr int kHalfBytes = kStageBytes / 2;                  // 16 KB
+    static constexpr int kHalfChunks = kHalfBoxes * 8;
+    static constexpr int kHSlots = 12;                                  // 192 KB ring
+    static constexpr int kMathWarps = 7;
+    static constexpr int kMath = 32 * kMathWarps;
+    static constexpr int kThreads = kMath + 32;
+    // Half-landed barriers indexed by the running half count (a warp takes
+    // every kMathWarps-th tile of a unit and skips phases of a slot's
+    // barrier).  A warp waiting for a half of tile t has finished tile
+    // t - kMathWarps of the same unit, or (its first tile of a unit) every
+    // tile before the unit was consumed at the unit's CTA barrier; either
+    // way the previous use of the barrier, kHalfBars halves earlier, was
+    // consumed when kHalfBars >= 2 kMathWarps + 1 + kHSlots.
+    static constexpr int kHalfBars = 32;
+    static_assert(kHalfBars >= 2 * kMathWarps + 1 + kHSlots, "half barriers too few");
 };
 
 template <typename T, int G>
 struct ScoreSmem {
     using S = ScoreShape<T>;
-    alignas(1024) uint8_t tiles[S::kStages][S::kStageBytes];
+    alignas(1024) uint8_t ring[S::kHSlots][S::kHalfBytes];
     alignas(16) float w[G * kWHead];
-    double red[4][G][2];
-    uint64_t full[S::kStages];
-    uint64_t empty[S::kStages];
-    int last_flag;
+    uint64_t full[S::kHalfBars];
+    uint64_t empty[S::kHSlots];
+    int abort;  // a bounded wait gave up: every thread stops at the next unit
 };
 
 // Merge the per-tile moment partials of one unit, by one warp: lane l sums
@@ -168,134 +182,147 @@ score_kernel(const __grid_constant__ CUtensorMap kmap, ScoreArgs a) {
     ScoreSmem<T, G>& sm = *reinterpret_cast<ScoreSmem<T, G>*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    // This CTA's tiles: a contiguous range of the flattened (unit, tile) list.
     const int64_t total = a.n_units * a.tpu;
     const int64_t t_begin = total * blockIdx.x / gridDim.x;
     const int64_t t_end = total * (blockIdx.x + 1) / gridDim.x;
 
-    if (tid == S::kConsumers) {
-        for (int i = 0; i < S::kStages; ++i) {
-            mbar_init(&sm.full[i], 1);
-            mbar_init(&sm.empty[i], S::kConsumers);
-        }
+    if (tid == S::kMath) {
+        for (int i = 0; i < S::kHalfBars; ++i) mbar_init(&sm.full[i], 1);
+        for (int i = 0; i < S::kHSlots; ++i) mbar_init(&sm.empty[i], 32);
         fence_barrier_init();
         prefetch_tensormap(&kmap);
+        sm.abort = 0;
     }
     __syncthreads();
 
-    if (tid >= S::kConsumers) {
-        // Producer warp: one lane issues the TMA loads.
-        if (tid == S::kConsumers) {
-            int stage = 0;
-            uint32_t phase = 0;
-            uint32_t issued[S::kStages] = {};
-            bool ok = true;
-            for (int64_t t = t_begin; t < t_end && ok; ++t) {
-                const int64_t u = t / a.tpu;
-                const int i = static_cast<int>(t % a.tpu);
-                const int n = clamp_nvalid(a.n_valid, u, a.cap, nullptr);
-                if (i * S::kTile >= n) continue;
-                ok = mbar_wait(&sm.empty[stage], phase ^ 1, a.flag);
-                if (!ok) break;
-                mbar_arrive_expect_tx(&sm.full[stage], S::kStageBytes);
-                const int32_t y = static_cast<int32_t>(u * a.cap + static_cast<int64_t>(i) * S::kTile);
+    // Units of the range in order; tiles i0 <= i < i1 of unit u, empty tiles
+    // (beyond n_valid) skipped.  hbase counts the halves before the unit.
+    const int64_t u_first = t_begin / a.tpu;
+    const int64_t u_last = t_end > t_begin ? (t_end - 1) / a.tpu : u_first - 1;
+    uint32_t hbase = 0;
+    for (int64_t u = u_first; u <= u_last; ++u) {
+        const int n = clamp_nvalid(a.n_valid, u, a.cap, tid == 0 ? a.flag : nullptr);
+        const int64_t lo = u * a.tpu > t_begin ? u * a.tpu : t_begin;
+        const int64_t hi = (u + 1) * a.tpu < t_end ? (u + 1) * a.tpu : t_end;
+        const int i0 = static_cast<int>(lo - u * a.tpu);
+        const int ntv = (n + S::kTile - 1) / S::kTile;  // tiles with keys
+        const int i1 = min(static_cast<int>(hi - u * a.tpu), ntv);
+        const int nt = i1 > i0 ? i1 - i0 : 0;
+        if (nt == 0) continue;
+        // Weights of the unit (every earlier tile is consumed past this barrier).
+        __syncthreads();
+        if (sm.abort) break;
+        {
+            const float4* src = reinterpret_cast<const float4*>(a.wts + u * G * kWHead);
+            float4* dst = reinterpret_cast<float4*>(sm.w);
+            for (int e = tid; e < G * kWHead / 4; e += S::kThreads) dst[e] = src[e];
+        }
+        __syncthreads();
+        if (tid >= S::kMath) {
+            if (tid == S::kMath) {
+                for (int hh = 0; hh < 2 * nt; ++hh) {
+                    const uint32_t hc = hbase + hh;
+                    const int slot = hc % S::kHSlots;
+                    if (sm.abort ||
+                        !mbar_wait(&sm.empty[slot], ((hc / S::kHSlots) & 1) ^ 1, a.flag)) {
+                        sm.abort = 1;
+                        break;
+                    }
+                    uint64_t* landed = &sm.full[hc % S::kHalfBars];
+                    mbar_arrive_expect_tx(landed, S::kHalfBytes);
+                    const int32_t y = static_cast<int32_t>(
+                        u * a.cap + static_cast<int64_t>(i0 + (hh >> 1)) * S::kTile);
 #pragma unroll
-                for (int b = 0; b < S::kBoxes; ++b)
-                    tma_load_2d(sm.tiles[stage] + b * S::kBoxBytes, &kmap, &sm.full[stage],
-                                b * (128 / static_cast<int>(sizeof(T))), y);
-                issued[stage]++;
-                if (++stage == S::kStages) {
-                    stage = 0;
-                    phase ^= 1;
+                    for (int b = 0; b < S::kHalfBoxes; ++b)
+                        tma_load_2d(sm.ring[slot] + b * S::kBoxBytes, &kmap, landed,
+                                    ((hh & 1) * S::kHalfBoxes + b) *
+                                        (128 / static_cast<int>(sizeof(T))),
+                                    y);
                 }
             }
-            // Every load issued has landed before the CTA may exit.
-            for (int st = 0; st < S::kStages; ++st)
-                if (issued[st]) mbar_wait(&sm.full[st], (issued[st] - 1) & 1, a.flag);
-        }
-        return;
-    }
-
-    // Consumers.
-    int stage = 0;
-    uint32_t phase = 0;
-    int64_t cur_u = -1;
-    for (int64_t t = t_begin; t < t_end; ++t) {
-        const int64_t u = t / a.tpu;
-        const int i = static_cast<int>(t % a.tpu);
-        const int n = clamp_nvalid(a.n_valid, u, a.cap, tid == 0 ? a.flag : nullptr);
-        double m1[G], m2[G];
+        } else {
+            for (int k = warp; k < nt; k += S::kMathWarps) {
+                const int i = i0 + k;
+                float2 acc[S::kKPT][G];
+                score_acc_zero<G, S::kKPT>(acc);
+                bool ok = true;
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    const uint32_t hc = hbase + 2 * k + half;
+                    const int slot = hc % S::kHSlots;
+                    if (!mbar_wait(&sm.full[hc % S::kHalfBars], (hc / S::kHalfBars) & 1, a.flag)) {
+                        ok = false;
+                        break;
+                    }
+                    score_rows_acc<T, G, S::kKPT, S::kBoxBytes, 32>(
+                        sm.ring[slot], half * S::kHalfChunks, (half + 1) * S::kHalfChunks, sm.w,
+                        lane, acc);
+                    __syncwarp();
+                    mbar_arrive(&sm.empty[slot]);
+                }
+                if (!ok) {
+                    sm.abort = 1;
+                    break;
+                }
+                float s[S::kKPT][G];
+                score_acc_final<G, S::kKPT>(acc, s);
+                double m1[G], m2[G];
 #pragma unroll
-        for (int h = 0; h < G; ++h) m1[h] = m2[h] = 0.0;
-        if (i * S::kTile < n) {
-            if (u != cur_u) {
-                named_sync(1, S::kConsumers);
-                const float4* src = reinterpret_cast<const float4*>(a.wts + u * G * kWHead);
-                float4* dst = reinterpret_cast<float4*>(sm.w);
-                for (int e = tid; e < G * kWHead / 4; e += S::kConsumers) dst[e] = src[e];
-                named_sync(1, S::kConsumers);
-                cur_u = u;
-            }
-            if (!mbar_wait(&sm.full[stage], phase, a.flag)) break;
-            float s[S::kKPT][G];
-            score_rows<T, G, S::kKPT, S::kBoxBytes, 128>(sm.tiles[stage], sm.w, tid, s);
-            mbar_arrive(&sm.empty[stage]);
-            if (++stage == S::kStages) {
-                stage = 0;
-                phase ^= 1;
-            }
+                for (int h = 0; h < G; ++h) m1[h] = m2[h] = 0.0;
 #pragma unroll
-            for (int k = 0; k < S::kKPT; ++k) {
-                const int j = i * S::kTile + tid + 128 * k;
-                if (j < n) {
+                for (int kk = 0; kk < S::kKPT; ++kk) {
+                    const int j = i * S::kTile + lane + 32 * kk;
+                    if (j < n) {
 #pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        a.raw[(u * G + h) * a.cap + j] = s[k][h];
-                        const double d = s[k][h];
-                        m1[h] += d;
-                        m2[h] = fma(d, d, m2[h]);
+                        for (int h = 0; h < G; ++h) {
+                            a.raw[(u * G + h) * a.cap + j] = s[kk][h];
+                            const double d = s[kk][h];
+                            m1[h] += d;
+                            m2[h] = fma(d, d, m2[h]);
+                        }
                     }
                 }
-            }
-        }
-        // Tile moments: warp shuffle, then the 4 warps in order.
 #pragma unroll
-        for (int h = 0; h < G; ++h) {
+                for (int h = 0; h < G; ++h) {
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                m1[h] += __shfl_xor_sync(0xffffffffu, m1[h], o);
-                m2[h] += __shfl_xor_sync(0xffffffffu, m2[h], o);
-            }
-        }
-        const int warp = tid >> 5, lane = tid & 31;
-        if (lane == 0) {
+                    for (int o = 16; o > 0; o >>= 1) {
+                        m1[h] += __shfl_xor_sync(0xffffffffu, m1[h], o);
+                        m2[h] += __shfl_xor_sync(0xffffffffu, m2[h], o);
+                    }
+                }
+                uint32_t done = 0;
+                if (lane == 0) {
+                    double* part = a.partial + (u * a.tpu + i) * G * 2;
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
-                sm.red[warp][h][0] = m1[h];
-                sm.red[warp][h][1] = m2[h];
+                    for (int h = 0; h < G; ++h) {
+                        part[2 * h] = m1[h];
+                        part[2 * h + 1] = m2[h];
+                    }
+                    __threadfence();
+                    done = atomicAdd(&a.counters[u], 1u);
+                }
+                done = __shfl_sync(0xffffffffu, done, 0);
+                if (done == static_cast<uint32_t>(ntv) - 1u) {
+                    // The last tile of the unit: merge every tile's partial.
+                    __threadfence();
+                    merge_unit_moments<G>(a.partial + u * a.tpu * G * 2, ntv, n, a.mom + u * G);
+                    if (lane == 0) a.counters[u] = 0u;
+                }
             }
         }
-        named_sync(1, S::kConsumers);
-        if (tid == 0) {
-            double* part = a.partial + (u * a.tpu + i) * G * 2;
-            for (int h = 0; h < G; ++h) {
-                part[2 * h] = ((sm.red[0][h][0] + sm.red[1][h][0]) + sm.red[2][h][0]) + sm.red[3][h][0];
-                part[2 * h + 1] =
-                    ((sm.red[0][h][1] + sm.red[1][h][1]) + sm.red[2][h][1]) + sm.red[3][h][1];
-            }
-            __threadfence();
-            const uint32_t done = atomicAdd(&a.counters[u], 1u);
-            sm.last_flag = (done == static_cast<uint32_t>(a.tpu) - 1u);
-        }
-        named_sync(1, S::kConsumers);
-        if (sm.last_flag && warp == 0) {
-            // The last tile of the unit to finish merges every tile's partial.
-            __threadfence();
-            merge_unit_moments<G>(a.partial + u * a.tpu * G * 2, static_cast<int>(a.tpu), n,
-                                  a.mom + u * G);
-            if (lane == 0) a.counters[u] = 0u;
-        }
-        named_sync(1, S::kConsumers);
+        hbase += 2 * nt;
     }
+    // Every load issued has landed before the CTA may exit: the math warps
+    // consumed them all, unless a wait gave up; then loads still in flight
+    // are given time to land.
+    __syncthreads();
+    if (sm.abort && tid == 0) {
+        const uint64_t t0 = globaltimer_ns();
+        while (globaltimer_ns() - t0 < 100000) __nanosleep(1000);
+    }
+    __syncthreads();
 }
 
 // ---------------------------------------------------------------------------

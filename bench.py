@@ -87,9 +87,9 @@ def fused_bytes(spec) -> int:
 # the workload up to one full launch (traffic grows with the units processed).
 TRAFFIC = {
     # profiles/prune_coop_kernel_c2_full.txt
-    ("c2", "prune_coop_kernel"): {"bytes_per_launch": 36259584, "src": "00d04262a9971991"},
+    ("c2", "prune_coop_kernel"): {"bytes_per_launch": 36241664, "src": "beba6fb151a885f1"},
     # profiles/prune_fused_kernel_c3-2seq_full.txt: 224 of 1792 units captured, x 8
-    ("c3", "prune_fused_kernel"): {"bytes_per_launch": 6274965504, "src": "00d04262a9971991"},
+    ("c3", "prune_fused_kernel"): {"bytes_per_launch": 6438772736, "src": "beba6fb151a885f1"},
 }
 
 

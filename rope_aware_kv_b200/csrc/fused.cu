@@ -9,24 +9,26 @@
 // (jaedaily.cn tutorial, eviction step).
 //
 // Per unit:
-//   score   a producer lane streams 128-key tiles (32 KB) into a TMA ring of
-//           4 to 6 stages; each of the seven math warps scores whole tiles,
-//           every lane on 4 keys for all GQA heads (so one broadcast weight
-//           load feeds 4 keys); per-head scores go to a per-CTA float32
-//           scratch that stays in L2, float64 moments stay in registers.
+//   score   a producer lane streams 128-key tiles (32 KB, as two 16 KB halves
+//           of one TMA box each) into a ring of 8 to 12 half slots and asks L2
+//           for the tiles after them; each of the seven math warps scores
+//           whole tiles, every lane on 4 keys for all GQA heads (so one
+//           broadcast weight load feeds 4 keys); per-head scores go to a
+//           per-CTA float32 scratch that stays in L2, float64 moments stay in
+//           registers.
 //   z-max   fixed-order moment merge, final = max_h z_h into shared memory,
 //           histogram of its linear z-bins.
 //   select  the keys in the z-bin of the B-th key are listed and ranked
 //           (directly, or by a three-digit radix of their full keys), then
 //           the ordered compaction of kept indices (warp ballots).
-//   gather  kept rows form runs of consecutive indices; one lane fills 8 KB
-//           shared buffers, each with kGRows consecutive destination rows of K
-//           or V, by one cp.async.bulk per run piece (the whole TMA ring, up
-//           to 192 KB of loads, in flight), and the math warps copy landed
-//           buffers to the destination with 16-byte stores, freeing each
-//           buffer as soon as it is read.
+//   gather  with most rows kept, 16 KB chunks of consecutive source rows are
+//           bulk-loaded and each kept row stored at its rank; otherwise the
+//           runs of kept rows fill 8 KB buffers of consecutive destination
+//           rows (one cp.async.bulk per run).  The whole ring is in flight;
+//           the math warps copy landed buffers out with 16-byte stores and
+//           free each as soon as it is read.
 // HBM traffic per unit is the compulsory bytes plus the re-read of kept K
-// rows (often from L2).
+// rows (mostly from L2) and, for chunks, the dropped rows among them.
 #include "select_core.cuh"
 #include "fold_core.cuh"
 #include "score_core.cuh"

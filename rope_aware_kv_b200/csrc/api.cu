@@ -432,6 +432,7 @@ tri_status tri_score(const tri_config* cfg, const void* k_post, tri_dtype dt, in
     float* wts = reinterpret_cast<float*>(ws_at(ws, w.wts));
     TRI_CUDA(launch_fold(stats, p_cur, n_seq, n_layers, n_kvheads * G, cfg->theta, off, wts, s));
     ScoreArgs a;
+    a.keys = k_post;
     a.n_units = U;
     a.cap = cap;
     a.tpu = w.tpu;
@@ -649,6 +650,7 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
     TRI_CUDA(cudaMemsetAsync(ws_at(ws, w.sel.hists), 0, w.sel.counts - w.sel.hists, s));
     TRI_CUDA(launch_fold(stats, p_cur, n_seq, n_layers, n_kvheads * G, cfg->theta, off, wts, s));
     ScoreArgs a;
+    a.keys = k_src;
     a.n_units = U;
     a.cap = cap_src;
     a.tpu = w.sc.tpu;

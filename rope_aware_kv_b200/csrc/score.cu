@@ -24,6 +24,12 @@
 #include "tri_launch.h"
 #include "score_core.cuh"
 
+// How many key tiles ahead of its shared-memory ring the score kernel asks
+// L2 to fetch (0: no prefetch).
+#ifndef TRI_PREFETCH_TILES
+#define TRI_PREFETCH_TILES 6
+#endif
+
 namespace tri {
 
 // ---------------------------------------------------------------------------
@@ -119,6 +125,7 @@ struct ScoreShape {
     // consumed when kHalfBars >= 2 kMathWarps + 1 + kHSlots.
     static constexpr int kHalfBars = 32;
     static_assert(kHalfBars >= 2 * kMathWarps + 1 + kHSlots, "half barriers too few");
+    static constexpr int kPrefetchTiles = TRI_PREFETCH_TILES;
 };
 
 template <typename T, int G>
@@ -222,7 +229,21 @@ score_kernel(const __grid_constant__ CUtensorMap kmap, ScoreArgs a) {
         __syncthreads();
         if (tid >= S::kMath) {
             if (tid == S::kMath) {
+                // Tiles are also requested into L2 kPrefetchTiles ahead of
+                // their load into the ring (TRI_PREFETCH_TILES, 0: none).
+                const char* kunit = static_cast<const char*>(a.keys) + u * a.cap * S::kRowBytes;
+                const uint64_t pol = policy_evict_first();
+                auto prefetch_tile = [&](int k) {
+                    if (S::kPrefetchTiles == 0 || k >= nt) return;
+                    const int t = i0 + k;
+                    const int rows = min(S::kTile, static_cast<int>(a.cap) - t * S::kTile);
+                    prefetch_l2_bulk(kunit + static_cast<int64_t>(t) * S::kStageBytes,
+                                     static_cast<uint32_t>(rows * S::kRowBytes), pol);
+                };
+                for (int k = S::kHSlots / 2; k < S::kHSlots / 2 + S::kPrefetchTiles; ++k)
+                    prefetch_tile(k);
                 for (int hh = 0; hh < 2 * nt; ++hh) {
+                    if ((hh & 1) == 0 && hh >= S::kHSlots) prefetch_tile(hh / 2 + S::kPrefetchTiles);
                     const uint32_t hc = hbase + hh;
                     const int slot = hc % S::kHSlots;
                     if (sm.abort ||

@@ -32,6 +32,7 @@ struct FoldConst {
 constexpr size_t kFoldStaticBytes = 4096;
 
 struct ScoreArgs {
+    const void* keys;            // [U][cap][128] (for L2 prefetch; loads go through the map)
     int64_t n_units;
     int64_t cap;
     int64_t tpu;                 // tiles per unit

@@ -116,9 +116,9 @@ def kernel_sources_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def measured_traffic(workload: str, kernel: str, n_seq_override: int):
+def measured_traffic(workload: str, kernel: str, cut: bool):
     rec = TRAFFIC.get((workload, kernel))
-    if rec is None or n_seq_override or rec["src"] != kernel_sources_hash():
+    if rec is None or cut or rec["src"] != kernel_sources_hash():
         return None
     return rec["bytes_per_launch"]
 
@@ -361,6 +361,8 @@ def run_tri(args, ws, rank, local):
     spec = synth.SPECS[args.workload]
     if args.n_seq:
         spec = spec.scaled(n_seq=args.n_seq)
+    if args.n_layers:
+        spec = spec.scaled(n_layers=args.n_layers)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     runner = StepRunner(spec, dev)
@@ -476,7 +478,8 @@ def run_tri(args, ws, rank, local):
             "dtype": "bf16" if spec.dtype == "bf16" else "f32", "data": "synthetic",
             "config": {
                 "workload": f"{args.workload}: {WORKLOAD_TEXT[args.workload]}" + (
-                    f" (cut to {spec.n_seq} sequence(s))" if args.n_seq else ""),
+                    f" (cut to {spec.n_seq} sequence(s) x {spec.n_layers} layer(s))"
+                    if (args.n_seq or args.n_layers) else ""),
                 "units": spec.n_units, "keys_per_unit": spec.n_valid, "budget": spec.B,
                 "group": spec.G, "head_dim": spec.d, "parallelism": f"dp{ws} (independent units)",
                 "l2": f"inputs rotated over {runner.n_copies} copies "
@@ -488,7 +491,8 @@ def run_tri(args, ws, rank, local):
             "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": achieved,
                          "peak": peak_gbs, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": achieved / peak_gbs,
-                         "traffic": measured_traffic(args.workload, dom_name, args.n_seq),
+                         "traffic": measured_traffic(args.workload, dom_name,
+                                                     bool(args.n_seq or args.n_layers)),
                          "algorithmic_bytes": dom_bytes, "ms_per_launch": dom_ms},
             "per_launch_ms": [round(float(x), 5) for x in per_launch],
             "path": {tri.PATH_FUSED: "fused", tri.PATH_COOP: "coop"}.get(path, "split"),
@@ -558,6 +562,8 @@ def main():
     ap.add_argument("--n-seq", type=int, default=0,
                     help="run the workload with this many sequences instead (a smaller case "
                          "of the same kernel for profiler captures; not a bench line)")
+    ap.add_argument("--n-layers", type=int, default=0,
+                    help="run the workload with this many layers instead (as --n-seq)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

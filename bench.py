@@ -87,9 +87,11 @@ def fused_bytes(spec) -> int:
 # the workload up to one full launch (traffic grows with the units processed).
 TRAFFIC = {
     # profiles/prune_coop_kernel_c2_full.txt
-    ("c2", "prune_coop_kernel"): {"bytes_per_launch": 36241664, "src": "165fa8a312e9a19d"},
+    ("c2", "prune_coop_kernel"): {"bytes_per_launch": 36226304, "src": "a87ada92f3060ee5"},
     # profiles/prune_fused_kernel_c3-2seq_full.txt: 224 of 1792 units captured, x 8
-    ("c3", "prune_fused_kernel"): {"bytes_per_launch": 6438772736, "src": "165fa8a312e9a19d"},
+    ("c3", "prune_fused_kernel"): {"bytes_per_launch": 6429958144, "src": "a87ada92f3060ee5"},
+    # profiles/score_kernel_c4-1seq-2layers_full.txt: 16 of 1024 units captured, x 64
+    ("c4", "score_kernel"): {"bytes_per_launch": 39339245568, "src": "a87ada92f3060ee5"},
 }
 
 
@@ -456,11 +458,12 @@ def run_tri(args, ws, rank, local):
         dom_name = "prune_fused_kernel" if path == tri.PATH_FUSED else "prune_coop_kernel"
         dom_bytes = fused_bytes(spec)
     else:
-        names = ["fold", "score", "zmax_hist", "radix_pass1", "radix_pass2", "select_count",
-                 "select_compact", "gather"]
+        names = ["fold_kernel", "score_kernel", "zmax_kernel", "radix_pass_kernel",
+                 "radix_pass_kernel", "select_count_kernel", "select_compact_kernel",
+                 "gather_kernel"]
         dom_name = names[dom] if dom < len(names) else f"launch{dom}"
         gather_bytes = spec.n_units * min(spec.B, spec.n_valid) * (3 * spec.d * spec.esize + 12)
-        byts = {"score": score_bytes(spec), "gather": gather_bytes}
+        byts = {"score_kernel": score_bytes(spec), "gather_kernel": gather_bytes}
         dom_bytes = byts.get(dom_name, 0)
     # The breakdown graph's events stretch each step a little; scale the
     # dominant kernel's interval by the plain graph's step time.

@@ -328,8 +328,9 @@ int tri_last_launch_count(void);
  * 2: z-max done; 3: selected; 4: gathered.  The cooperative kernel (a few
  * units, each split over several CTAs) indexes by CTA instead of unit and
  * needs grid * 512 bytes: points 0 start, 1 scored, 2 after the first unit
- * barrier, 3 z-max done, 4 after the second barrier, 5 after the last
- * barrier, 6 compaction done, 7 gather done.  Pass (NULL, 0) to stop.
+ * barrier, 3 z-max done, 4 after the second barrier, 5 threshold known (past
+ * the third barrier), 6 compaction done, 7 gather done.  Pass (NULL, 0) to
+ * stop.
  */
 tri_status tri_set_phase_trace(void* device_buf, size_t bytes);
 

@@ -87,11 +87,11 @@ def fused_bytes(spec) -> int:
 # the workload up to one full launch (traffic grows with the units processed).
 TRAFFIC = {
     # profiles/prune_coop_kernel_c2_full.txt
-    ("c2", "prune_coop_kernel"): {"bytes_per_launch": 36226304, "src": "a87ada92f3060ee5"},
+    ("c2", "prune_coop_kernel"): {"bytes_per_launch": 36226304, "src": "2885885db7594c5c"},
     # profiles/prune_fused_kernel_c3-2seq_full.txt: 224 of 1792 units captured, x 8
-    ("c3", "prune_fused_kernel"): {"bytes_per_launch": 6429958144, "src": "a87ada92f3060ee5"},
+    ("c3", "prune_fused_kernel"): {"bytes_per_launch": 6429958144, "src": "58689953c672b152"},
     # profiles/score_kernel_c4-1seq-2layers_full.txt: 16 of 1024 units captured, x 64
-    ("c4", "score_kernel"): {"bytes_per_launch": 39339245568, "src": "a87ada92f3060ee5"},
+    ("c4", "score_kernel"): {"bytes_per_launch": 39339245568, "src": "be9b26c9e0f73f28"},
 }
 
 
@@ -106,21 +106,44 @@ def _code_only(text: str) -> str:
     return " ".join(text.split())
 
 
-def kernel_sources_hash() -> str:
-    import hashlib
+# Translation unit of each kernel whose traffic is recorded.
+KERNEL_SOURCE = {
+    "prune_coop_kernel": "coop.cu",
+    "prune_fused_kernel": "fused.cu",
+    "score_kernel": "score.cu",
+}
 
-    h = hashlib.sha256()
+
+def kernel_sources_hash(kernel: str = "") -> str:
+    """Hash of the code (comments stripped) a kernel is compiled from: its
+    translation unit and every local header it includes, transitively; with
+    no kernel named, of every source file."""
+    import hashlib
+    import re
+
     d = os.path.join(ROOT, "rope_aware_kv_b200", "csrc")
-    for name in sorted(os.listdir(d)):
-        if name.endswith((".cu", ".cuh", ".h")):
+    if kernel in KERNEL_SOURCE:
+        files, todo = set(), [KERNEL_SOURCE[kernel]]
+        while todo:
+            name = todo.pop()
+            if name in files or not os.path.exists(os.path.join(d, name)):
+                continue
+            files.add(name)
             with open(os.path.join(d, name), encoding="utf-8") as fh:
-                h.update(name.encode() + b"\0" + _code_only(fh.read()).encode())
+                todo += re.findall(r'#include\s+"([^"/]+)"', fh.read())
+        names = sorted(files)
+    else:
+        names = sorted(n for n in os.listdir(d) if n.endswith((".cu", ".cuh", ".h")))
+    h = hashlib.sha256()
+    for name in names:
+        with open(os.path.join(d, name), encoding="utf-8") as fh:
+            h.update(name.encode() + b"\0" + _code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 
 def measured_traffic(workload: str, kernel: str, cut: bool):
     rec = TRAFFIC.get((workload, kernel))
-    if rec is None or cut or rec["src"] != kernel_sources_hash():
+    if rec is None or cut or rec["src"] != kernel_sources_hash(kernel):
         return None
     return rec["bytes_per_launch"]
 

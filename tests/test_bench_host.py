@@ -28,9 +28,25 @@ def test_source_hash_ignores_comments_only():
 def test_traffic_reported_only_for_the_captured_sources(monkeypatch):
     key = ("c2", "prune_coop_kernel")
     rec = bench.TRAFFIC[key]
-    monkeypatch.setattr(bench, "kernel_sources_hash", lambda: rec["src"])
+    monkeypatch.setattr(bench, "kernel_sources_hash", lambda *k: rec["src"])
     assert bench.measured_traffic(*key, False) == rec["bytes_per_launch"]
     assert bench.measured_traffic(*key, True) is None          # a cut workload
     assert bench.measured_traffic("c2", "other_kernel", False) is None
-    monkeypatch.setattr(bench, "kernel_sources_hash", lambda: "0" * 16)
+    monkeypatch.setattr(bench, "kernel_sources_hash", lambda *k: "0" * 16)
     assert bench.measured_traffic(*key, False) is None          # sources changed
+
+
+def test_kernel_hash_covers_its_own_sources_only(tmp_path, monkeypatch):
+    csrc = tmp_path / "rope_aware_kv_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "coop.cu").write_text('#include "common.cuh"\nint coop;\n')
+    (csrc / "fused.cu").write_text('#include "common.cuh"\nint fused;\n')
+    (csrc / "common.cuh").write_text("int shared;\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    coop0, fused0 = (bench.kernel_sources_hash("prune_coop_kernel"),
+                     bench.kernel_sources_hash("prune_fused_kernel"))
+    (csrc / "fused.cu").write_text('#include "common.cuh"\nint fused2;\n')
+    assert bench.kernel_sources_hash("prune_coop_kernel") == coop0
+    assert bench.kernel_sources_hash("prune_fused_kernel") != fused0
+    (csrc / "common.cuh").write_text("int shared2;\n")
+    assert bench.kernel_sources_hash("prune_coop_kernel") != coop0

@@ -149,6 +149,25 @@ size_t tri_calibrate_workspace_bytes(int64_t n_heads, int64_t n_tok, int head_di
 tri_status tri_calibrate(const void* q_pre, tri_dtype dt, int64_t n_heads, int64_t n_tok,
                          int head_dim, float* stats, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * Calibration split for data-parallel shards of the calibration tokens: each
+ * shard reduces its tokens to float64 sums, the shards' sums are added (an
+ * all-reduce over the ranks), and the statistics are formed from the totals.
+ * Not in the pages (they calibrate offline on one batch); the statistics
+ * equal tri_calibrate's on all tokens up to float64 rounding of the sum order.
+ *   tri_calibrate_sums: q_pre as in tri_calibrate; sums: out,
+ *     [n_heads][head_dim/2][3] float64 = (sum Re q_f, sum Im q_f, sum |q_f|)
+ *     over the shard's n_tok tokens; workspace as tri_calibrate's.
+ *   tri_calibrate_finish: sums: [n_heads][head_dim/2][3] float64 totals;
+ *     n_tok_total: tokens summed (>= 1); stats: out, as tri_calibrate's.
+ * Errors as tri_calibrate.
+ */
+tri_status tri_calibrate_sums(const void* q_pre, tri_dtype dt, int64_t n_heads, int64_t n_tok,
+                              int head_dim, double* sums, void* ws, size_t ws_bytes,
+                              void* stream);
+tri_status tri_calibrate_finish(const double* sums, int64_t n_heads, int64_t n_tok_total,
+                                int head_dim, float* stats, void* stream);
+
 /* ---------------------------------------------------------------------- */
 /* Score                                                                   */
 /* ---------------------------------------------------------------------- */

@@ -48,7 +48,7 @@ PATH_COOP = 3
 # Symbols include/tri.h declares (checked by the ABI tests).
 EXPORTS = (
     "tri_config_default", "tri_status_str", "tri_version",
-    "tri_calibrate_workspace_bytes", "tri_calibrate",
+    "tri_calibrate_workspace_bytes", "tri_calibrate", "tri_calibrate_sums", "tri_calibrate_finish",
     "tri_score_workspace_bytes", "tri_score",
     "tri_select_workspace_bytes", "tri_select_topB",
     "tri_compact_workspace_bytes", "tri_compact",
@@ -95,6 +95,8 @@ def load(path: Optional[str] = None):
         "tri_version": (ctypes.c_char_p, []),
         "tri_calibrate_workspace_bytes": (sz, [i64, i64, i32]),
         "tri_calibrate": (i32, [P, i32, i64, i64, i32, P, P, sz, P]),
+        "tri_calibrate_sums": (i32, [P, i32, i64, i64, i32, P, P, sz, P]),
+        "tri_calibrate_finish": (i32, [P, i64, i64, i32, P, P]),
         "tri_score_workspace_bytes": (sz, [i64, i64, i64, i32, i64, i32]),
         "tri_score": (i32, [ctypes.POINTER(TriConfig), P, i32, i64, i64, i64, i32, i64, P, P, P, P,
                             P, P, sz, P]),
@@ -199,6 +201,52 @@ def tri_calibrate(q_pre: torch.Tensor, stats: Optional[torch.Tensor] = None,
     _check("tri_calibrate", load().tri_calibrate(_ptr(q_pre), _dt(q_pre), H, n_tok, d, _ptr(stats),
                                                 _ptr(ws), ws.numel(), _stream(stream)))
     return stats
+
+
+def tri_calibrate_sums(q_pre: torch.Tensor, sums: Optional[torch.Tensor] = None,
+                       ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """q_pre [..., n_tok, d] (one shard's tokens) -> float64 sums [..., d/2, 3]."""
+    *lead, n_tok, d = q_pre.shape
+    H = 1
+    for x in lead:
+        H *= x
+    if sums is None:
+        sums = torch.empty((*lead, d // 2, 3), dtype=torch.float64, device=q_pre.device)
+    need = tri_calibrate_workspace_bytes(H, n_tok, d)
+    if ws is None:
+        ws = workspace(need, q_pre.device)
+    _check("tri_calibrate_sums", load().tri_calibrate_sums(
+        _ptr(q_pre), _dt(q_pre), H, n_tok, d, _ptr(sums), _ptr(ws), ws.numel(), _stream(stream)))
+    return sums
+
+
+def tri_calibrate_finish(sums: torch.Tensor, n_tok_total: int,
+                         stats: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """float64 sums [..., d/2, 3] over n_tok_total tokens -> stats [..., d/2, 4]."""
+    *lead, F, _ = sums.shape
+    H = 1
+    for x in lead:
+        H *= x
+    if stats is None:
+        stats = torch.empty((*lead, F, 4), dtype=torch.float32, device=sums.device)
+    _check("tri_calibrate_finish", load().tri_calibrate_finish(
+        _ptr(sums), H, int(n_tok_total), 2 * F, _ptr(stats), _stream(stream)))
+    return stats
+
+
+def calibrate_data_parallel(q_shard: torch.Tensor, group=None) -> torch.Tensor:
+    """Calibration over the calibration tokens of all data-parallel ranks:
+    each rank reduces its own shard q_shard [..., n_tok_rank, d] to float64
+    sums, one all-reduce adds the sums and the token counts over the process
+    group, and every rank forms the same statistics [..., d/2, 4]."""
+    import torch.distributed as dist
+
+    sums = tri_calibrate_sums(q_shard)
+    n = torch.tensor([q_shard.shape[-2]], dtype=torch.float64, device=sums.device)
+    both = torch.cat([sums.reshape(-1), n])
+    dist.all_reduce(both, op=dist.ReduceOp.SUM, group=group)
+    total = int(round(both[-1].item()))
+    return tri_calibrate_finish(both[:-1].reshape(sums.shape).contiguous(), total)
 
 
 def tri_score_workspace_bytes(n_seq, n_layers, n_kvheads, G, cap, head_dim=HEAD_DIM) -> int:

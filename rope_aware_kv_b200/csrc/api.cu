@@ -12,6 +12,7 @@
 
 #include "tri_internal.cuh"
 #include "tri_launch.h"
+#include "calibrate_dp.h"
 
 using namespace tri;
 
@@ -395,6 +396,33 @@ tri_status tri_calibrate(const void* q_pre, tri_dtype dt, int64_t n_heads, int64
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     TRI_CUDA(cudaMemsetAsync(ws, 0, kWsHeader, s));
     return cuda_status(launch_calibrate(q_pre, dt, n_heads, n_tok, stats, ws, s));
+}
+
+tri_status tri_calibrate_sums(const void* q_pre, tri_dtype dt, int64_t n_heads, int64_t n_tok,
+                              int head_dim, double* sums, void* ws, size_t ws_bytes,
+                              void* stream) {
+    LaunchScope scope_;
+    if (!q_pre || !sums || n_heads < 1 || n_tok < 1) return TRI_ERR_INVALID_ARG;
+    if (!dtype_ok(dt)) return TRI_ERR_UNSUPPORTED;
+    if (head_dim != kD) return TRI_ERR_UNSUPPORTED;
+    if (n_heads > 65535) return TRI_ERR_UNSUPPORTED;
+    if (!aligned16(q_pre) || (reinterpret_cast<uintptr_t>(sums) & 7)) return TRI_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < calibrate_ws_bytes(n_heads, n_tok) || !aligned16(ws))
+        return TRI_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    TRI_CUDA(cudaMemsetAsync(ws, 0, kWsHeader, s));
+    return cuda_status(launch_calibrate_sums(q_pre, dt, n_heads, n_tok, sums, ws, s));
+}
+
+tri_status tri_calibrate_finish(const double* sums, int64_t n_heads, int64_t n_tok_total,
+                                int head_dim, float* stats, void* stream) {
+    LaunchScope scope_;
+    if (!sums || !stats || n_heads < 1 || n_tok_total < 1) return TRI_ERR_INVALID_ARG;
+    if (head_dim != kD) return TRI_ERR_UNSUPPORTED;
+    if (n_heads > 65535) return TRI_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(sums) & 7) || !aligned4(stats)) return TRI_ERR_INVALID_ARG;
+    return cuda_status(launch_calibrate_finish(sums, n_heads, n_tok_total, stats,
+                                               static_cast<cudaStream_t>(stream)));
 }
 
 size_t tri_score_workspace_bytes(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G,

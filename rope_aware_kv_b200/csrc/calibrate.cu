@@ -12,6 +12,7 @@
 // the result is bitwise reproducible.
 #include "tri_internal.cuh"
 #include "tri_launch.h"
+#include "calibrate_dp.h"
 
 namespace tri {
 
@@ -85,6 +86,65 @@ calib_merge_kernel(const double* __restrict__ part, int n_chunks, int64_t n_tok,
     s[1] = static_cast<float>(mim);
     s[2] = static_cast<float>(mn);
     s[3] = static_cast<float>(R);
+}
+
+// Data-parallel calibration: the chunk partials of a shard summed in chunk
+// order into float64 totals, and statistics formed from (all-reduced) totals.
+__global__ void __launch_bounds__(64)
+calib_sum_kernel(const double* __restrict__ part, int n_chunks, double* __restrict__ sums) {
+    const int f = threadIdx.x;
+    const int64_t h = blockIdx.x;
+    double a = 0.0, b = 0.0, c = 0.0;
+    for (int i = 0; i < n_chunks; ++i) {
+        const double* o = part + ((h * n_chunks + i) * 64 + f) * 3;
+        a += o[0];
+        b += o[1];
+        c += o[2];
+    }
+    double* o = sums + (h * 64 + f) * 3;
+    o[0] = a;
+    o[1] = b;
+    o[2] = c;
+}
+
+__global__ void __launch_bounds__(64)
+calib_finish_kernel(const double* __restrict__ sums, int64_t n_tok, float* __restrict__ stats) {
+    const int f = threadIdx.x;
+    const int64_t h = blockIdx.x;
+    const double* o = sums + (h * 64 + f) * 3;
+    const double inv = 1.0 / static_cast<double>(n_tok);
+    const double mre = o[0] * inv, mim = o[1] * inv, mn = o[2] * inv;
+    const double R = (mn > 0.0) ? sqrt(mre * mre + mim * mim) / mn : 1.0;
+    float* s = stats + (h * 64 + f) * 4;
+    s[0] = static_cast<float>(mre);
+    s[1] = static_cast<float>(mim);
+    s[2] = static_cast<float>(mn);
+    s[3] = static_cast<float>(R);
+}
+
+cudaError_t launch_calibrate_sums(const void* q, tri_dtype dt, int64_t n_heads, int64_t n_tok,
+                                  double* sums, void* ws, cudaStream_t s) {
+    const int n_chunks = static_cast<int>((n_tok + kCalChunk - 1) / kCalChunk);
+    double* part = reinterpret_cast<double*>(static_cast<char*>(ws) + kWsHeader);
+    dim3 grid(n_chunks, static_cast<unsigned>(n_heads));
+    if (dt == TRI_BF16) {
+        calib_partial_kernel<__nv_bfloat16><<<grid, kCalThreads, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(q), n_tok, n_chunks, part);
+    } else {
+        calib_partial_kernel<float><<<grid, kCalThreads, 0, s>>>(static_cast<const float*>(q),
+                                                                  n_tok, n_chunks, part);
+    }
+    note_launch(s);
+    calib_sum_kernel<<<static_cast<unsigned>(n_heads), 64, 0, s>>>(part, n_chunks, sums);
+    note_launch(s);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_calibrate_finish(const double* sums, int64_t n_heads, int64_t n_tok,
+                                    float* stats, cudaStream_t s) {
+    calib_finish_kernel<<<static_cast<unsigned>(n_heads), 64, 0, s>>>(sums, n_tok, stats);
+    note_launch(s);
+    return cudaGetLastError();
 }
 
 size_t calibrate_ws_bytes(int64_t n_heads, int64_t n_tok) {

@@ -103,3 +103,22 @@ def test_host_validation_without_gpu(lib):
     assert _prune_status(lib, cfg2) == 1
     cfg3 = tri.config(path=7)
     assert _prune_status(lib, cfg3) == 1
+
+
+def test_calibration_split_validation_without_gpu(lib):
+    """The data-parallel calibration entry points refuse bad arguments on
+    the host (fake, never dereferenced addresses)."""
+    q, sums, stats, ws = 4096, 8192, 12288, 16384
+    wsb = tri.tri_calibrate_workspace_bytes(2, 100)
+    assert lib.tri_calibrate_sums(None, 0, 2, 100, 128, sums, ws, wsb, None) == 1
+    assert lib.tri_calibrate_sums(q, 0, 2, 100, 128, None, ws, wsb, None) == 1
+    assert lib.tri_calibrate_sums(q, 0, 0, 100, 128, sums, ws, wsb, None) == 1
+    assert lib.tri_calibrate_sums(q, 0, 2, 100, 64, sums, ws, wsb, None) == 2
+    assert lib.tri_calibrate_sums(q, 7, 2, 100, 128, sums, ws, wsb, None) == 2
+    assert lib.tri_calibrate_sums(q + 4, 0, 2, 100, 128, sums, ws, wsb, None) == 1
+    assert lib.tri_calibrate_sums(q, 0, 2, 100, 128, sums + 4, ws, wsb, None) == 1
+    assert lib.tri_calibrate_sums(q, 0, 2, 100, 128, sums, ws, 16, None) == 3
+    assert lib.tri_calibrate_finish(None, 2, 100, 128, stats, None) == 1
+    assert lib.tri_calibrate_finish(sums, 2, 0, 128, stats, None) == 1
+    assert lib.tri_calibrate_finish(sums, 2, 100, 64, stats, None) == 2
+    assert lib.tri_calibrate_finish(sums + 4, 2, 100, 128, stats, None) == 1

@@ -56,6 +56,54 @@ def test_calibrate_parity(dtype):
     assert np.max(np.abs(g[..., 3] - ost[..., 3])) < 1e-6
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_calibrate_from_shard_sums(dtype):
+    """Calibration tokens split over data-parallel shards (uneven, one shard
+    smaller than a reduction chunk): the shards' float64 sums, added as an
+    all-reduce would, give the statistics of the whole batch (oracle and
+    tri_calibrate)."""
+    spec = _spec(dtype=dtype, G=3, n_layers=2, n_kvheads=1, n_cal=3000)
+    wl = synth.make_workload(spec, "cuda")
+    q = synth.calib_queries(spec, wl.hp, 1, "cuda")          # [Hq, 3000, 128]
+    whole = tri.tri_calibrate(q)
+    cuts = [0, 700, 1337, 1337 + 500, 3000]
+    total = sum(tri.tri_calibrate_sums(q[:, a:b].contiguous())
+                for a, b in zip(cuts[:-1], cuts[1:]))
+    stats = tri.tri_calibrate_finish(total, q.shape[1]).cpu().numpy().astype(np.float64)
+    ost = oracle.calibrate(synth.host_elems(q))
+    scale = ost[..., 2:3]
+    assert np.max(np.abs(stats[..., :3] - ost[..., :3]) / scale) < 1e-6
+    assert np.max(np.abs(stats[..., 3] - ost[..., 3])) < 1e-6
+    w = whole.cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(stats[..., :3] - w[..., :3]) / w[..., 2:3]) < 1e-6
+    assert np.max(np.abs(stats[..., 3] - w[..., 3])) < 1e-6
+
+
+def test_calibrate_data_parallel_over_nccl_one_rank():
+    """The data-parallel helper through a real NCCL all-reduce (one rank on
+    this GPU): the statistics equal tri_calibrate's."""
+    import os
+    import socket
+
+    import torch.distributed as dist
+
+    spec = _spec(dtype="bf16", G=3, n_layers=1, n_kvheads=1, n_cal=2048)
+    wl = synth.make_workload(spec, "cuda")
+    q = synth.calib_queries(spec, wl.hp, 0, "cuda")
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1)
+    try:
+        got = tri.calibrate_data_parallel(q)
+    finally:
+        dist.destroy_process_group()
+    ref = tri.tri_calibrate(q).cpu().numpy().astype(np.float64)
+    got = got.cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(got[..., :3] - ref[..., :3]) / ref[..., 2:3]) < 1e-6
+    assert np.max(np.abs(got[..., 3] - ref[..., 3])) < 1e-6
+
+
 # ---------------------------------------------------------------------------
 # score
 # ---------------------------------------------------------------------------

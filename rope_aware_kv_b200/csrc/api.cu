@@ -55,6 +55,12 @@ constexpr size_t kAlign = 256;
 size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
 // Workspace carving: returns offsets of consecutive, 256-byte aligned regions.
+bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
+    const char* pa = static_cast<const char*>(a);
+    const char* pb = static_cast<const char*>(b);
+    return pa < pb + bn && pb < pa + an;
+}
+
 struct Carve {
     size_t off = kWsHeader;
     size_t take(size_t bytes) {
@@ -583,11 +589,20 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
     const int64_t U = n_seq * n_layers * n_kvheads;
     const size_t esz = dt == TRI_BF16 ? 2 : 4;
     {
-        const char* ks = static_cast<const char*>(k_src);
-        const char* kd = static_cast<const char*>(k_dst);
+        // No destination may overlap a source (the gather reads the sources
+        // while it writes the destinations).
         const size_t sb = static_cast<size_t>(U * cap_src) * kD * esz;
         const size_t db = static_cast<size_t>(U * cap_dst) * kD * esz;
-        if (ks < kd + db && kd < ks + sb) return TRI_ERR_INVALID_ARG;
+        const size_t spb = static_cast<size_t>(U * cap_src) * 4;
+        const size_t dpb = static_cast<size_t>(U * cap_dst) * 4;
+        const void* src[3] = {k_src, v_src, pos_src};
+        const size_t sn[3] = {sb, sb, spb};
+        const void* dst[3] = {k_dst, v_dst, pos_dst};
+        const size_t dn[3] = {db, db, dpb};
+        for (int i = 0; i < 3; ++i)
+            for (int j = 0; j < 3; ++j)
+                if (src[i] && dst[j] && overlaps(src[i], sn[i], dst[j], dn[j]))
+                    return TRI_ERR_INVALID_ARG;
     }
     const PruneWs w =
         prune_ws(n_seq, n_layers, n_kvheads, G, cap_src, B, dt, kept_idx == nullptr, cfg->path);

@@ -71,9 +71,10 @@ def test_workspace_queries(lib):
 
 
 def _prune_status(lib, cfg, **over):
-    args = dict(k_src=16, v_src=16, pos_src=16, dt=tri.TRI_BF16, n_seq=1, n_layers=1, n_kvheads=4,
-                G=7, cap=4096, n_valid=None, p_cur=16, stats=16, B=512, k_dst=1 << 40,
-                v_dst=1 << 41, pos_dst=16, cap_dst=512, kept=None, n_kept=16, ws=None, ws_bytes=0)
+    args = dict(k_src=1 << 36, v_src=1 << 37, pos_src=1 << 38, dt=tri.TRI_BF16, n_seq=1,
+                n_layers=1, n_kvheads=4, G=7, cap=4096, n_valid=None, p_cur=16, stats=16, B=512,
+                k_dst=1 << 40, v_dst=1 << 41, pos_dst=1 << 42, cap_dst=512, kept=None, n_kept=16,
+                ws=None, ws_bytes=0)
     args.update(over)
     P = lambda v: None if v is None else ctypes.c_void_p(v)
     return lib.tri_prune(ctypes.byref(cfg) if cfg is not None else None, P(args["k_src"]),
@@ -92,10 +93,14 @@ def test_host_validation_without_gpu(lib):
     assert _prune_status(lib, cfg, G=0) == 2
     assert _prune_status(lib, cfg, dt=7) == 2                 # unknown dtype
     assert _prune_status(lib, cfg, B=0) == 1                  # empty budget
-    assert _prune_status(lib, cfg, k_src=18) == 1             # misaligned keys
+    assert _prune_status(lib, cfg, k_src=(1 << 36) + 2) == 1  # misaligned keys
     assert _prune_status(lib, cfg, v_dst=None) == 1           # v_src without v_dst
     assert _prune_status(lib, cfg, cap_dst=100) == 1          # destination too small
-    assert _prune_status(lib, cfg, k_dst=16 + 4096) == 1      # destination overlaps source
+    assert _prune_status(lib, cfg) == 3                       # well formed: no workspace
+    assert _prune_status(lib, cfg, k_dst=(1 << 36) + 4096) == 1  # K destination overlaps K
+    assert _prune_status(lib, cfg, v_dst=(1 << 37) + 256) == 1   # V destination overlaps V
+    assert _prune_status(lib, cfg, k_dst=(1 << 37) + 512) == 1   # K destination overlaps V
+    assert _prune_status(lib, cfg, pos_dst=(1 << 38) + 64) == 1  # positions overlap
     bad = tri.config(head_dim=64)
     assert _prune_status(lib, bad) == 2
     cfg2 = tri.config()

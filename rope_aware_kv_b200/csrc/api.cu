@@ -61,6 +61,25 @@ bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
     return pa < pb + bn && pb < pa + an;
 }
 
+// Whether any destination (K, V, positions; null ones skipped) overlaps any
+// source: the gather reads the sources while it writes the destinations.
+bool gather_buffers_overlap(const void* k_src, const void* v_src, const void* pos_src,
+                            const void* k_dst, const void* v_dst, const void* pos_dst,
+                            int64_t n_units, int64_t cap_src, int64_t cap_dst, size_t esz) {
+    const size_t sb = static_cast<size_t>(n_units * cap_src) * kD * esz;
+    const size_t db = static_cast<size_t>(n_units * cap_dst) * kD * esz;
+    const size_t spb = static_cast<size_t>(n_units * cap_src) * 4;
+    const size_t dpb = static_cast<size_t>(n_units * cap_dst) * 4;
+    const void* src[3] = {k_src, v_src, pos_src};
+    const size_t sn[3] = {sb, sb, spb};
+    const void* dst[3] = {k_dst, v_dst, pos_dst};
+    const size_t dn[3] = {db, db, dpb};
+    for (int i = 0; i < 3; ++i)
+        for (int j = 0; j < 3; ++j)
+            if (src[i] && dst[j] && overlaps(src[i], sn[i], dst[j], dn[j])) return true;
+    return false;
+}
+
 struct Carve {
     size_t off = kWsHeader;
     size_t take(size_t bytes) {
@@ -528,11 +547,9 @@ tri_status tri_compact(const void* k_src, const void* v_src, const int32_t* pos_
     if (!aligned16(k_src) || !aligned16(k_dst) || (v_src && (!aligned16(v_src) || !aligned16(v_dst))))
         return TRI_ERR_INVALID_ARG;
     const size_t esz = dt == TRI_BF16 ? 2 : 4;
-    const char* ks = static_cast<const char*>(k_src);
-    const char* kd = static_cast<const char*>(k_dst);
-    const size_t sb = static_cast<size_t>(n_units * cap_src) * kD * esz;
-    const size_t db = static_cast<size_t>(n_units * cap_dst) * kD * esz;
-    if (ks < kd + db && kd < ks + sb) return TRI_ERR_INVALID_ARG;  // overlap
+    if (gather_buffers_overlap(k_src, v_src, pos_src, k_dst, v_dst, pos_dst, n_units, cap_src,
+                               cap_dst, esz))
+        return TRI_ERR_INVALID_ARG;
     if (!ws || ws_bytes < kWsHeader || !aligned16(ws)) return TRI_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     TRI_CUDA(cudaMemsetAsync(ws, 0, kWsHeader, s));
@@ -588,22 +605,9 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
         return TRI_ERR_INVALID_ARG;
     const int64_t U = n_seq * n_layers * n_kvheads;
     const size_t esz = dt == TRI_BF16 ? 2 : 4;
-    {
-        // No destination may overlap a source (the gather reads the sources
-        // while it writes the destinations).
-        const size_t sb = static_cast<size_t>(U * cap_src) * kD * esz;
-        const size_t db = static_cast<size_t>(U * cap_dst) * kD * esz;
-        const size_t spb = static_cast<size_t>(U * cap_src) * 4;
-        const size_t dpb = static_cast<size_t>(U * cap_dst) * 4;
-        const void* src[3] = {k_src, v_src, pos_src};
-        const size_t sn[3] = {sb, sb, spb};
-        const void* dst[3] = {k_dst, v_dst, pos_dst};
-        const size_t dn[3] = {db, db, dpb};
-        for (int i = 0; i < 3; ++i)
-            for (int j = 0; j < 3; ++j)
-                if (src[i] && dst[j] && overlaps(src[i], sn[i], dst[j], dn[j]))
-                    return TRI_ERR_INVALID_ARG;
-    }
+    if (gather_buffers_overlap(k_src, v_src, pos_src, k_dst, v_dst, pos_dst, U, cap_src, cap_dst,
+                               esz))
+        return TRI_ERR_INVALID_ARG;
     const PruneWs w =
         prune_ws(n_seq, n_layers, n_kvheads, G, cap_src, B, dt, kept_idx == nullptr, cfg->path);
     if (cfg->path == TRI_PATH_FUSED && !w.fused) return TRI_ERR_UNSUPPORTED;

@@ -564,7 +564,7 @@ size_t tri_prune_workspace_bytes(int64_t n_seq, int64_t n_layers, int64_t n_kvhe
     if (check_units(n_seq, n_layers, n_kvheads, G, cap) != TRI_OK || B < 1) return kWsHeader;
     size_t best = 0;
     for (tri_dtype dt : {TRI_BF16, TRI_F32}) {
-        for (int path : {TRI_PATH_AUTO, TRI_PATH_SPLIT, TRI_PATH_COOP}) {
+        for (int path : {TRI_PATH_AUTO, TRI_PATH_FUSED, TRI_PATH_SPLIT, TRI_PATH_COOP}) {
             const size_t t = prune_ws(n_seq, n_layers, n_kvheads, G, cap, B, dt, true, path).total;
             if (t > best) best = t;
         }

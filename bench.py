@@ -1,7 +1,8 @@
 """Benchmark of one TriAttention prune step on B200 (libtri, sm_100a).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c2]
-                    [--impl reference] [--n-seq S] [--no-cpu-baseline]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c4]
+                    [--impl reference] [--n-seq S] [--n-layers L]
+                    [--no-cpu-baseline] [--no-sub]
 
 A step is one pass of the whole prune path (fold, score, z-normalise / max,
 top-B select, order-preserving gather of K, V and positions) over every unit
@@ -9,10 +10,13 @@ of the workload.  Units are independent, so at N GPUs every rank prunes its
 own copy of the workload (weak scaling, no collective on the data path) and
 ``value`` counts the keys of all ranks over the slowest rank's time.
 
-Default workload: one layer, GQA 28 query / 4 KV heads, 32768 bf16 keys per
-head, budget 2048 (the second workload configuration; the first is the small
-single-head fp32 case the oracle finishes in seconds).  Metric: keys scored
-and pruned per second, plus the achieved HBM bandwidth of the step's
+Default workload: the long-prefill compaction (32 layers x 8 KV heads x 4
+sequences, GQA 32/8, 131072 bf16 keys per head, budget 4096), the largest
+configuration that fits one GPU.  The same line carries driver-timed
+sub-records of the other 32K-token configurations (one layer of 4 KV heads
+at 32768 keys; the windowed decode step; the streaming step), each with its
+time per step, keys/s and fraction of the HBM roofline.  Metric: keys
+scored and pruned per second, plus the achieved HBM bandwidth of the step's
 compulsory bytes (read every key, read the kept values, write the kept keys
 and values, indices and positions) against the measured copy peak.
 
@@ -254,14 +258,15 @@ def max_over_ranks(x: float, ws: int) -> float:
 # ---------------------------------------------------------------------------
 # the oracle (CPU baseline and reference arm)
 # ---------------------------------------------------------------------------
-def oracle_sample(spec, seconds_hint: float = 15.0):
-    """Bounded sample of the workload for the CPU oracle: a few units drawn
-    from the generator on the host, cut to a key count that keeps the run to
-    roughly ``seconds_hint`` seconds.  Returns (inputs, keys, description)."""
+def oracle_sample(spec, seconds_hint: float = 8.0, units=None):
+    """Bounded sample of the workload for the CPU oracle: ``units`` units (one
+    per oracle thread by default) drawn from the generator on the host, cut
+    to a key count that keeps each unit to roughly ``seconds_hint`` seconds of
+    one core.  Returns (inputs, keys, description, units)."""
     import oracle
 
     threads = oracle.threads()
-    n_units = max(1, min(spec.n_units, threads))
+    n_units = max(1, min(spec.n_units, units if units is not None else threads))
     # ~ 17 offsets x 64 bands x G cosines per key, about 25 ns each
     per_key = 17 * 64 * spec.G * 25e-9
     n_keys = int(min(spec.n_valid, max(256, seconds_hint / per_key)))
@@ -274,9 +279,9 @@ def oracle_sample(spec, seconds_hint: float = 15.0):
     st = oracle.calibrate(synth.host_elems(q))[None]
     inputs = dict(k=synth.host_elems(wl.k), v=synth.host_elems(wl.v), pos=wl.pos.numpy(),
                   p_cur=wl.p_cur.numpy(), stats=st, sub=sub)
-    desc = (f"{n_units} unit(s) x {n_keys} keys (G={spec.G}, B={sub.B}) of {spec.name}, "
-            f"oracle with {min(n_units, threads)} thread(s)")
-    return inputs, n_units * n_keys, desc, min(n_units, threads)
+    desc = (f"sampled: {n_units} unit(s) x {n_keys} keys (G={spec.G}, B={sub.B}) of "
+            f"{spec.name}")
+    return inputs, n_units * n_keys, desc, n_units
 
 
 def oracle_step(inp):
@@ -288,19 +293,39 @@ def oracle_step(inp):
 
 
 def cpu_baseline(spec):
-    inp, keys, desc, cores = oracle_sample(spec)
+    """The float64 oracle on the host cores, on a sample of the workload: one
+    unit per thread with every thread, then one unit on one thread."""
+    import oracle
+
+    threads = oracle.threads()
+    inp, keys, desc, n_units = oracle_sample(spec)
     t0 = time.perf_counter()
     oracle_step(inp)
-    dt = time.perf_counter() - t0
-    return {"value": keys / dt, "unit": "keys/s", "cores": cores, "kind": "oracle",
-            "sample": desc, "seconds": round(dt, 3)}
+    dt_all = time.perf_counter() - t0
+    inp1, keys1, desc1, _ = oracle_sample(spec, units=1)
+    oracle.set_threads(1)
+    try:
+        t0 = time.perf_counter()
+        oracle_step(inp1)
+        dt_one = time.perf_counter() - t0
+    finally:
+        oracle.set_threads(threads)
+    return {"value": keys / dt_all, "unit": "keys/s", "cores": os.cpu_count(),
+            "threads": min(n_units, threads), "kind": "oracle",
+            "sample": desc + f", oracle on {min(n_units, threads)} thread(s)",
+            "seconds": round(dt_all, 3),
+            "single_thread": {"value": keys1 / dt_one, "unit": "keys/s", "threads": 1,
+                              "sample": desc1 + ", oracle on 1 thread",
+                              "seconds": round(dt_one, 3)}}
 
 
 def run_reference(args, ws, rank):
     if rank != 0:
         return
+    import oracle
+
     spec = synth.SPECS[args.workload]
-    inp, keys, desc, cores = oracle_sample(spec, seconds_hint=0.5)
+    inp, keys, desc, n_units = oracle_sample(spec, seconds_hint=0.5)
     for _ in range(args.warmup):
         oracle_step(inp)
     t0 = time.perf_counter()
@@ -308,6 +333,8 @@ def run_reference(args, ws, rank):
         oracle_step(inp)
     dt = (time.perf_counter() - t0) / args.steps
     value = keys / dt
+    threads = min(n_units, oracle.threads())
+    desc = desc + f", oracle on {threads} thread(s)"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "keys/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -315,8 +342,8 @@ def run_reference(args, ws, rank):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": f"{args.workload}: {WORKLOAD_TEXT[args.workload]}",
                    "sample": desc},
-        "cpu_baseline": {"value": value, "unit": "keys/s", "cores": cores, "kind": "oracle",
-                         "sample": desc},
+        "cpu_baseline": {"value": value, "unit": "keys/s", "cores": os.cpu_count(),
+                         "threads": threads, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "keys/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -375,25 +402,31 @@ class StepRunner:
                            n_valid=self.wl.n_valid, kept=self.kept, ws=self.ws)
 
 
-def run_tri(args, ws, rank, local):
+KERNEL_NAMES = {
+    "pipe_small": ["prune_pipe_kernel"],
+    "pipe_big": ["fold_kernel", "prune_pipe_kernel"],
+    "fused": ["prune_fused_kernel"],
+    "coop": ["prune_coop_kernel"],
+    "split": ["fold_kernel", "score_kernel", "zmax_kernel", "radix_pass_kernel",
+              "radix_pass_kernel", "select_count_kernel", "select_compact_kernel",
+              "gather_kernel"],
+}
+
+
+def path_name(tri, spec):
+    path = tri.tri_prune_path(spec.n_seq, spec.n_layers, spec.n_kvheads, spec.G, spec.cap,
+                              spec.B, spec.torch_dtype)
+    if path == tri.PATH_PIPE:
+        return "pipe_small" if tri.tri_last_launch_count() == 1 else "pipe_big"
+    return {tri.PATH_FUSED: "fused", tri.PATH_COOP: "coop"}.get(path, "split")
+
+
+def time_workload(args, spec, dev, stream, ws, steps):
+    """Time `steps` prune steps of spec as one CUDA graph (max over ranks) and
+    break the step down per launch.  Returns (runner, record)."""
     import rope_aware_kv_b200 as tri
-    from rope_aware_kv_b200 import build as tri_build
 
-    if rank == 0:
-        tri_build.build()
-    barrier(ws)
-    tri.load()
-    spec = synth.SPECS[args.workload]
-    if args.n_seq:
-        spec = spec.scaled(n_seq=args.n_seq)
-    if args.n_layers:
-        spec = spec.scaled(n_layers=args.n_layers)
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
     runner = StepRunner(spec, dev)
-    stream = torch.cuda.Stream(device=dev)
-    peak_gbs, peak_kind = measured_peaks()
-
     with torch.cuda.stream(stream):
         # Eager warm-up (also initialises the library's static state).
         for i in range(max(args.warmup, 3)):
@@ -402,11 +435,12 @@ def run_tri(args, ws, rank, local):
         tri.tri_set_timing_events(None)
         runner.step(0)
         launches = tri.tri_last_launch_count()
+        pname = path_name(tri, spec)
 
         # Per-launch events inside the timed graph.
         evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(launches)]
-               for _ in range(args.steps)]
-        starts = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(args.steps)]
+               for _ in range(steps)]
+        starts = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(steps)]
         for e in starts + [x for row in evs for x in row]:
             e.record(stream)
         torch.cuda.synchronize()
@@ -414,12 +448,12 @@ def run_tri(args, ws, rank, local):
         # Timed graph: K steps, nothing but the library's own launches.
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
-            for i in range(args.steps):
+            for i in range(steps):
                 runner.step(args.warmup + i)
         # Breakdown graph: the same K steps with an event after every launch.
         ge = torch.cuda.CUDAGraph()
         with torch.cuda.graph(ge, stream=stream, capture_error_mode="relaxed"):
-            for i in range(args.steps):
+            for i in range(steps):
                 starts[i].record(stream)
                 tri.tri_set_timing_events(evs[i])
                 runner.step(args.warmup + i)
@@ -429,7 +463,7 @@ def run_tri(args, ws, rank, local):
             for i in range(args.warmup):
                 runner.step(i)
 
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     gw.replay()
@@ -446,7 +480,7 @@ def run_tri(args, ws, rank, local):
     barrier(ws)
     ms_total = t0.elapsed_time(t1)
     ms_max = max_over_ranks(ms_total, ws)
-    ms_step = ms_max / args.steps
+    ms_step = ms_max / steps
 
     # Per-kernel durations from the breakdown graph (an interval runs from the
     # previous launch's event to this launch's event; the first launch's
@@ -457,77 +491,132 @@ def run_tri(args, ws, rank, local):
     torch.cuda.synchronize()
     per_launch = np.zeros(launches)
     ev_total = 0.0
-    for i in range(args.steps):
+    for i in range(steps):
         prev = starts[i]
         for j in range(launches):
             per_launch[j] += prev.elapsed_time(evs[i][j])
             prev = evs[i][j]
         ev_total += starts[i].elapsed_time(evs[i][-1])
-    per_launch /= args.steps
-    ev_step = ev_total / args.steps
+    per_launch /= steps
+    ev_step = ev_total / steps
     flags = tri.tri_check_device_error(runner.ws)
-
-    keys_rank = spec.n_units * spec.n_valid
-    value = keys_rank * ws / (ms_step * 1e-3)
+    del g, ge, gw
+    peak_gbs, peak_kind = measured_peaks()
     comp = compulsory_bytes(spec)
-    step_gbs = comp / (ms_step * 1e-3) / 1e9
+    keys_rank = spec.n_units * spec.n_valid
+    rec = {
+        "workload": f"{spec.name}: {WORKLOAD_TEXT.get(spec.name, spec.name)}",
+        "path": pname, "ms_per_step": ms_step, "value": keys_rank * ws / (ms_step * 1e-3),
+        "unit": "keys/s", "hbm_gbs": comp / (ms_step * 1e-3) / 1e9,
+        "frac": comp / (ms_step * 1e-3) / 1e9 / peak_gbs, "peak_gbs": peak_gbs,
+        "peak_kind": peak_kind, "compulsory_bytes_per_step": comp, "steps": steps,
+        "launches_per_step": launches, "device_flags": flags,
+        "per_launch_ms": [round(float(x), 5) for x in per_launch],
+        "evented_ms_per_step": ev_step, "clocks": clk,
+        "l2": f"inputs rotated over {runner.n_copies} copies "
+              f"({runner.n_copies * comp / 2**20:.0f} MiB compulsory > 126 MB L2)",
+    }
+    return runner, rec
 
-    # Dominant kernel and its algorithmic bytes.
-    path = tri.tri_prune_path(spec.n_seq, spec.n_layers, spec.n_kvheads, spec.G, spec.cap, spec.B,
-                              spec.torch_dtype)
+
+def dominant(spec, rec, ms_step):
+    """The dominant kernel of a step, its algorithmic bytes and its time."""
+    names = KERNEL_NAMES[rec["path"]]
+    per_launch = rec["per_launch_ms"]
     dom = int(np.argmax(per_launch))
-    if path in (tri.PATH_FUSED, tri.PATH_COOP):
-        # One launch per step: the whole path in one kernel.
-        dom_name = "prune_fused_kernel" if path == tri.PATH_FUSED else "prune_coop_kernel"
-        dom_bytes = fused_bytes(spec)
+    dom_name = names[dom] if dom < len(names) else f"launch{dom}"
+    if dom_name in ("prune_pipe_kernel", "prune_fused_kernel", "prune_coop_kernel"):
+        # One kernel runs the whole path: the step's compulsory bytes.
+        dom_bytes = compulsory_bytes(spec)
     else:
-        names = ["fold_kernel", "score_kernel", "zmax_kernel", "radix_pass_kernel",
-                 "radix_pass_kernel", "select_count_kernel", "select_compact_kernel",
-                 "gather_kernel"]
-        dom_name = names[dom] if dom < len(names) else f"launch{dom}"
         gather_bytes = spec.n_units * min(spec.B, spec.n_valid) * (3 * spec.d * spec.esize + 12)
-        byts = {"score_kernel": score_bytes(spec), "gather_kernel": gather_bytes}
-        dom_bytes = byts.get(dom_name, 0)
+        dom_bytes = {"score_kernel": score_bytes(spec), "gather_kernel": gather_bytes}.get(dom_name, 0)
     # The breakdown graph's events stretch each step a little; scale the
     # dominant kernel's interval by the plain graph's step time.
-    dom_ms = float(per_launch[dom]) * (ms_step / ev_step if ev_step > 0 else 1.0)
-    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9 if dom_ms > 0 else 0.0
+    ev = rec["evented_ms_per_step"]
+    dom_ms = float(per_launch[dom]) * (ms_step / ev if ev > 0 else 1.0)
+    return dom_name, dom_bytes, dom_ms
 
+
+SUB_WORKLOADS = ("c2", "c3", "c5")
+
+
+def run_tri(args, ws, rank, local):
+    import rope_aware_kv_b200 as tri
+    from rope_aware_kv_b200 import build as tri_build
+
+    if rank == 0:
+        tri_build.build()
+    barrier(ws)
+    tri.load()
+    spec = synth.SPECS[args.workload]
+    if args.n_seq:
+        spec = spec.scaled(n_seq=args.n_seq)
+    if args.n_layers:
+        spec = spec.scaled(n_layers=args.n_layers)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    peak_gbs, peak_kind = measured_peaks()
+
+    runner, rec = time_workload(args, spec, dev, stream, ws, args.steps)
+    ms_step = rec["ms_per_step"]
+    dom_name, dom_bytes, dom_ms = dominant(spec, rec, ms_step)
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9 if dom_ms > 0 else 0.0
     e2e = run_e2e(args, runner, stream, spec, ws)
+    launches = rec["launches_per_step"]
+    del runner
+    torch.cuda.empty_cache()
+
+    # Driver-timed sub-records of the other 32K-token configurations.
+    subs = {}
+    if not (args.no_sub or args.n_seq or args.n_layers):
+        for name in SUB_WORKLOADS:
+            if name == args.workload:
+                continue
+            r2, srec = time_workload(args, synth.SPECS[name], dev, stream, ws,
+                                     min(args.steps, 50))
+            dn, db, dms = dominant(synth.SPECS[name], srec, srec["ms_per_step"])
+            srec["roofline"] = {"kernel": dn, "achieved": db / (dms * 1e-3) / 1e9 if dms > 0 else 0,
+                                "algorithmic_bytes": db, "ms_per_launch": dms}
+            subs[name] = srec
+            del r2
+            torch.cuda.empty_cache()
+
     cpu = cpu_baseline(spec) if (rank == 0 and ws == 1 and not args.no_cpu_baseline) else None
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": "keys/s", "n_gpus": ws,
+            "metric": METRIC, "value": rec["value"], "unit": "keys/s", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if spec.dtype == "bf16" else "f32", "data": "synthetic",
             "config": {
-                "workload": f"{args.workload}: {WORKLOAD_TEXT[args.workload]}" + (
+                "workload": rec["workload"] + (
                     f" (cut to {spec.n_seq} sequence(s) x {spec.n_layers} layer(s))"
                     if (args.n_seq or args.n_layers) else ""),
                 "units": spec.n_units, "keys_per_unit": spec.n_valid, "budget": spec.B,
                 "group": spec.G, "head_dim": spec.d, "parallelism": f"dp{ws} (independent units)",
-                "l2": f"inputs rotated over {runner.n_copies} copies "
-                      f"({runner.n_copies * comp / 2**20:.0f} MiB compulsory > 126 MB L2)",
+                "l2": rec["l2"],
                 "timing": "one CUDA graph of K steps between CUDA events, max over ranks",
             },
-            "hbm_gbs": step_gbs, "hbm_frac_of_peak": step_gbs / peak_gbs,
-            "compulsory_bytes_per_step": comp,
+            "hbm_gbs": rec["hbm_gbs"], "hbm_frac_of_peak": rec["frac"],
+            "compulsory_bytes_per_step": rec["compulsory_bytes_per_step"],
             "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": achieved,
                          "peak": peak_gbs, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": achieved / peak_gbs,
                          "traffic": measured_traffic(args.workload, dom_name,
                                                      bool(args.n_seq or args.n_layers)),
                          "algorithmic_bytes": dom_bytes, "ms_per_launch": dom_ms},
-            "per_launch_ms": [round(float(x), 5) for x in per_launch],
-            "path": {tri.PATH_FUSED: "fused", tri.PATH_COOP: "coop"}.get(path, "split"),
-            "evented_ms_per_step": ev_step,
+            "per_launch_ms": rec["per_launch_ms"],
+            "path": rec["path"],
+            "evented_ms_per_step": rec["evented_ms_per_step"],
             "gpu_launches": int(launches * args.steps),
-            "device_flags": flags,
-            "clocks": clk,
+            "device_flags": rec["device_flags"],
+            "clocks": rec["clocks"],
             "e2e": e2e,
             "cpu_baseline": cpu,
+            "sub_workloads": subs,
         }
         print(json.dumps(line), flush=True)
 
@@ -537,15 +626,19 @@ def run_e2e(args, runner, stream, spec, ws):
     inputs copied in, the prune, and the compacted cache copied out."""
     tri = runner.tri
     wl = runner.wl
-    hk = wl.k.cpu().pin_memory()
-    hv = wl.v.cpu().pin_memory()
-    hp = wl.pos.cpu().pin_memory()
+    hk = torch.empty(wl.k.shape, dtype=wl.k.dtype, pin_memory=True)
+    hv = torch.empty(wl.v.shape, dtype=wl.v.dtype, pin_memory=True)
+    hp = torch.empty(wl.pos.shape, dtype=wl.pos.dtype, pin_memory=True)
+    hk.copy_(wl.k)
+    hv.copy_(wl.v)
+    hp.copy_(wl.pos)
     k, v, pos = runner.inputs[0]
     kd, vd, pd = runner.dst[0]
     ok = torch.empty(kd.shape, dtype=kd.dtype).pin_memory()
     ov = torch.empty(vd.shape, dtype=vd.dtype).pin_memory()
     op = torch.empty(pd.shape, dtype=pd.dtype).pin_memory()
-    steps = max(3, min(args.steps, 20))
+    big = hk.numel() * hk.element_size() > (8 << 30)
+    steps = 3 if big else max(3, min(args.steps, 20))
 
     def one():
         k.copy_(hk, non_blocking=True)
@@ -583,8 +676,10 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="tri", choices=["tri", "reference"])
-    ap.add_argument("--workload", default="c2", choices=sorted(synth.SPECS))
+    ap.add_argument("--workload", default="c4", choices=sorted(synth.SPECS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sub", action="store_true",
+                    help="time the chosen workload only (no sub-records of the others)")
     ap.add_argument("--n-seq", type=int, default=0,
                     help="run the workload with this many sequences instead (a smaller case "
                          "of the same kernel for profiler captures; not a bench line)")

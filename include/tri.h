@@ -38,7 +38,10 @@
  * --------------------------------
  * Pointers are DEVICE pointers unless a comment says "host".  The caller
  * allocates every buffer, including the workspace ("ws"); the library
- * allocates, frees and retains nothing and keeps no state between calls.
+ * allocates, frees and retains nothing and keeps no state between calls,
+ * except three per-host-thread profiling settings (tri_set_timing_events,
+ * tri_set_phase_trace, tri_last_launch_count) and the cached device address
+ * of tri_select_topB_static's static scratch.
  * Calls are asynchronous on the given CUDA stream ("stream" is a
  * cudaStream_t passed as void*; NULL is the legacy default stream) and are
  * safe to capture in a CUDA graph.  Two calls that share a workspace must not
@@ -104,10 +107,11 @@ typedef enum tri_dtype {
 
 /* Method parameters.  tri_config_default fills the pages' values. */
 /* Kernel path of tri_prune. */
-#define TRI_PATH_AUTO 0  /* fused for many small units, coop for few units, else split */
+#define TRI_PATH_AUTO 0  /* coop for fewer units than SMs, else pipe, else split */
 #define TRI_PATH_FUSED 1 /* one CTA per unit (TRI_ERR_UNSUPPORTED if it does not fit) */
 #define TRI_PATH_SPLIT 2 /* separate score / z-max / select / gather kernels */
 #define TRI_PATH_COOP 3  /* each unit split over several CTAs of one kernel (few large units) */
+#define TRI_PATH_PIPE 4  /* persistent kernel, gather of one unit overlapping the next's score */
 
 typedef struct tri_config {
     int head_dim;                      /* d; 128 is supported */
@@ -231,9 +235,11 @@ tri_status tri_select_topB(const float* final_score, int64_t n_units, int64_t ca
  * launched; e.g. 40 units of up to 131072 keys fit.  Nothing is allocated:
  * no cudaMalloc, cudaFree or allocating library call.
  *
- * The first call on a device looks up the array's device address with that
- * device current (cudaGetSymbolAddress) and remembers it; make that first call
- * before capturing any stream on the device.  Every call shares the one array
+ * Each call made outside stream capture looks up the array's device address
+ * with the device current (cudaGetSymbolAddress) and remembers it for calls
+ * made while a stream is being captured, so the first call on a device (and
+ * the first after a cudaDeviceReset) must come before any stream capture on
+ * it; a captured call with no earlier uncaptured call returns TRI_ERR_CUDA.  Every call shares the one array
  * and clears what must start at zero itself, so calls whose executions overlap
  * on the GPU (different streams, or different host threads) race and must be
  * serialised by the caller.  Device-side flags are not reported.
@@ -277,22 +283,29 @@ size_t tri_prune_workspace_bytes(int64_t n_seq, int64_t n_layers, int64_t n_kvhe
 /*
  * One prune step over every unit of a batch: score, z-normalise and max,
  * select the top-B, gather K, V and positions into the destination cache.
- * Units whose n_valid <= B are copied whole.  Many small caches run one
- * persistent fused kernel (whole units per CTA); a few caches (fewer than
- * half the SMs) run one kernel with each unit split over several CTAs;
- * otherwise the split kernels run (cfg->path can force a path).  Arguments as in the
+ * Units whose n_valid <= B are copied whole.  With fewer units than SMs, one
+ * kernel splits each unit over several CTAs (TRI_PATH_COOP); otherwise one
+ * persistent kernel scores, selects and gathers, the gather of each unit
+ * overlapping the scoring of the next (TRI_PATH_PIPE; a unit too large for
+ * one CTA is scored in chunks by many CTAs and selected by the CTA that
+ * completes it); the separate kernels of tri_score / tri_select_topB /
+ * tri_compact (TRI_PATH_SPLIT) and the earlier whole-unit fused kernel
+ * (TRI_PATH_FUSED) can be forced through cfg->path.  Arguments as in the
  * calls above; kept_idx (nullable, [U][B]) receives the kept indices;
  * n_kept ([U], required) receives min(B, n_valid[u]), the destination's
- * n_valid for the next step.
+ * n_valid for the next step; final_score (nullable, [U][cap_src] float32)
+ * receives the final scores of tri_score for every unit with n_valid > B
+ * (rows of units that are copied whole may be left unwritten).
  */
 tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src,
                      const int32_t* pos_src, tri_dtype dt, int64_t n_seq, int64_t n_layers,
                      int64_t n_kvheads, int G, int64_t cap_src, const int32_t* n_valid,
                      const int64_t* p_cur, const float* stats, int64_t B, void* k_dst,
                      void* v_dst, int32_t* pos_dst, int64_t cap_dst, int32_t* kept_idx,
-                     int32_t* n_kept, void* ws, size_t ws_bytes, void* stream);
+                     int32_t* n_kept, float* final_score, void* ws, size_t ws_bytes,
+                     void* stream);
 
-/* The kernel path (TRI_PATH_FUSED, TRI_PATH_COOP or TRI_PATH_SPLIT) that
+/* The kernel path (TRI_PATH_PIPE, TRI_PATH_COOP, TRI_PATH_FUSED or TRI_PATH_SPLIT) that
  * tri_prune takes for these shapes on the current device when cfg->path is
  * `path`; -1 when `path` cannot serve them or the shapes are invalid. */
 int tri_prune_path(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int64_t cap,

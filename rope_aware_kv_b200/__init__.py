@@ -44,6 +44,7 @@ PATH_AUTO = 0
 PATH_FUSED = 1
 PATH_SPLIT = 2
 PATH_COOP = 3
+PATH_PIPE = 4
 
 # Symbols include/tri.h declares (checked by the ABI tests).
 EXPORTS = (
@@ -106,7 +107,7 @@ def load(path: Optional[str] = None):
         "tri_compact": (i32, [P, P, P, i32, i64, i64, i32, P, P, i64, P, P, P, i64, P, sz, P]),
         "tri_prune_workspace_bytes": (sz, [i64, i64, i64, i32, i64, i64, i32]),
         "tri_prune": (i32, [ctypes.POINTER(TriConfig), P, P, P, i32, i64, i64, i64, i32, i64, P, P,
-                            P, i64, P, P, P, i64, P, P, P, sz, P]),
+                            P, i64, P, P, P, i64, P, P, P, P, sz, P]),
         "tri_append": (i32, [P, P, P, i32, i64, i64, i64, i32, P, P, P, P, P, i64, P, sz, P]),
         "tri_check_device_error": (i32, [P, P, u32p]),
         "tri_set_timing_events": (i32, [ctypes.POINTER(ctypes.c_void_p), i32]),
@@ -330,7 +331,7 @@ def tri_prune_workspace_bytes(n_seq, n_layers, n_kvheads, G, cap, B, head_dim=HE
 
 def tri_prune_path(n_seq, n_layers, n_kvheads, G, cap, B, dtype=torch.bfloat16,
                    path: int = PATH_AUTO) -> int:
-    """Kernel path tri_prune takes for these shapes (PATH_FUSED / COOP / SPLIT)."""
+    """Kernel path tri_prune takes for these shapes (PATH_PIPE / COOP / FUSED / SPLIT)."""
     dt = TRI_BF16 if dtype == torch.bfloat16 else TRI_F32
     return int(load().tri_prune_path(n_seq, n_layers, n_kvheads, G, cap, B, dt, path))
 
@@ -340,8 +341,11 @@ def tri_prune(cfg: TriConfig, k_src: torch.Tensor, v_src: Optional[torch.Tensor]
               p_cur: torch.Tensor, stats: torch.Tensor, B: int, k_dst: torch.Tensor,
               v_dst: Optional[torch.Tensor], pos_dst: Optional[torch.Tensor],
               n_kept: torch.Tensor, n_valid: Optional[torch.Tensor] = None,
-              kept: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, stream=None):
-    """One prune step: score, select the top-B, gather into the destination cache."""
+              kept: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, stream=None,
+              final: Optional[torch.Tensor] = None):
+    """One prune step: score, select the top-B, gather into the destination
+    cache.  ``final`` (optional, [U, cap_src] float32) receives the final
+    scores of the units that were pruned."""
     U, cap_src, d = k_src.shape
     cap_dst = k_dst.shape[1]
     if ws is None:
@@ -350,7 +354,8 @@ def tri_prune(cfg: TriConfig, k_src: torch.Tensor, v_src: Optional[torch.Tensor]
     _check("tri_prune", load().tri_prune(
         ctypes.byref(cfg), _ptr(k_src), _ptr(v_src), _ptr(pos_src), _dt(k_src), n_seq, n_layers,
         n_kvheads, G, cap_src, _ptr(n_valid), _ptr(p_cur), _ptr(stats), B, _ptr(k_dst), _ptr(v_dst),
-        _ptr(pos_dst), cap_dst, _ptr(kept), _ptr(n_kept), _ptr(ws), ws.numel(), _stream(stream)))
+        _ptr(pos_dst), cap_dst, _ptr(kept), _ptr(n_kept), _ptr(final), _ptr(ws), ws.numel(),
+        _stream(stream)))
 
 
 def tri_append(k_cache, v_cache, pos_cache, n_seq: int, n_valid: torch.Tensor,

@@ -34,6 +34,23 @@ uint64_t* tri::phase_trace_buffer(int64_t n_units) {
     return t_trace;
 }
 
+void tri::begin_launches() { t_launches = 0; }
+
+SelectWs tri::select_ws(size_t start, int64_t U, int64_t cap) {
+    SelectWs w;
+    size_t off = start;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = (off + bytes + 255) & ~size_t(255);
+        return o;
+    };
+    w.hists = take(static_cast<size_t>(3 * U) * kHistBins0 * 4);
+    const int64_t chunks = (cap + kZChunk - 1) / kZChunk;
+    w.counts = take(static_cast<size_t>(U * chunks) * 8);
+    w.total = off;
+    return w;
+}
+
 void tri::note_launch(cudaStream_t s) {
     if (t_events && t_launches < t_n_events) {
         // Under stream capture a plain record only marks a dependency; an
@@ -123,22 +140,26 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 2-D view of a key cache [rows][128] for TMA: boxes of 128 bytes x box_rows
-// rows with the 128-byte swizzle.
+// 2-D view of a key cache [rows][128] for TMA: boxes of box_bytes (128, 64
+// or 32) bytes x box_rows rows, swizzled with the same span.
 tri_status make_key_map(CUtensorMap* map, const void* k, tri_dtype dt, int64_t rows,
-                        int box_rows) {
+                        int box_rows, int box_bytes = 128) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return TRI_ERR_CUDA;
     const int esz = dt == TRI_BF16 ? 2 : 4;
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(rows)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kD * esz)};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esz), static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(box_bytes / esz),
+                               static_cast<cuuint32_t>(box_rows)};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = fn(map,
                           dt == TRI_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                          : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
                           2, const_cast<void*>(k), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          box_bytes == 32   ? CU_TENSOR_MAP_SWIZZLE_32B
+                          : box_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                            : CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? TRI_OK : TRI_ERR_CUDA;
 }
@@ -165,7 +186,7 @@ tri_status check_cfg(const tri_config* cfg, FoldOffsets* off) {
     if (cfg->head_dim != kD) return TRI_ERR_UNSUPPORTED;
     if (!(cfg->theta > 1.0) || cfg->n_offsets < 1 || cfg->n_offsets > TRI_MAX_OFFSETS)
         return TRI_ERR_INVALID_ARG;
-    if (cfg->path < TRI_PATH_AUTO || cfg->path > TRI_PATH_COOP) return TRI_ERR_INVALID_ARG;
+    if (cfg->path < TRI_PATH_AUTO || cfg->path > TRI_PATH_PIPE) return TRI_ERR_INVALID_ARG;
     off->n = cfg->n_offsets;
     for (int i = 0; i < cfg->n_offsets; ++i) {
         if (cfg->offsets[i] < 0) return TRI_ERR_INVALID_ARG;
@@ -227,21 +248,6 @@ ScoreWs score_ws(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int6
     return w;
 }
 
-// ---- select workspace ----
-struct SelectWs {
-    size_t hists, counts, total;
-};
-
-SelectWs select_ws(size_t start, int64_t U, int64_t cap) {
-    SelectWs w;
-    Carve c;
-    c.off = start;
-    w.hists = c.take(static_cast<size_t>(3 * U) * kHistBins0 * 4);
-    const int64_t chunks = (cap + kZChunk - 1) / kZChunk;
-    w.counts = c.take(static_cast<size_t>(U * chunks) * 8);
-    w.total = c.off;
-    return w;
-}
 
 // ---- prune workspace ----
 struct CoopPlan {
@@ -250,10 +256,21 @@ struct CoopPlan {
     int64_t keys_max = 0;
 };
 
+struct PipePlan {
+    bool ok = false;
+    bool big = false;   // large-unit mode (chunks, last-arriver selection)
+    int gslots = 0;     // gather buffers
+    int64_t grid = 0;
+    int64_t cpu = 0;    // chunks per unit (large mode)
+};
+
 struct PruneWs {
     bool fused = false;
     bool coop = false;
+    bool pipe = false;
     CoopPlan cp;
+    PipePlan pp;
+    size_t queue = 0, counters = 0, wts = 0, raw = 0, fin_scratch = 0;
     ScoreWs sc;
     size_t fin = 0, kept = 0;
     SelectWs sel;
@@ -311,11 +328,66 @@ CoopPlan coop_plan(tri_dtype dt, int G, int64_t U, int64_t cap) {
     return p;
 }
 
+// Pipelined kernel: the small-unit mode when a unit's final scores fit its
+// idle rings (uint16 indices), else the large-unit mode; either needs its
+// shared-memory layout to fit one CTA.
+PipePlan pipe_plan(tri_dtype dt, int G, int64_t U, int64_t cap, int64_t B) {
+    PipePlan p;
+    const int64_t sms = sm_count_or_default();
+    const bool small = pipe_small_fits(dt, cap);
+    const int e = pipe_engine_warps();
+    for (int g = pipe_max_gslots() / e * e; g >= pipe_min_gslots(); g -= e) {
+        if (pipe_smem_bytes(dt, G, cap, B, !small, g) <= fused_smem_limit()) {
+            p.gslots = g;
+            break;
+        }
+    }
+    if (!p.gslots) return p;
+    p.ok = true;
+    p.big = !small;
+    if (small) {
+        p.grid = U < sms ? U : sms;
+    } else {
+        const int64_t ck = pipe_chunk_keys(dt);
+        p.cpu = (cap + ck - 1) / ck;
+        const int64_t items = U * p.cpu;
+        p.grid = items < sms ? items : sms;
+    }
+    return p;
+}
+
 PruneWs prune_ws(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int64_t cap,
                  int64_t B, tri_dtype dt, bool own_kept, int path) {
     PruneWs w;
     const int64_t U = n_seq * n_layers * n_kvheads;
     const int64_t sms = sm_count_or_default();
+    if (path == TRI_PATH_PIPE || path == TRI_PATH_AUTO) {
+        const PipePlan pp = pipe_plan(dt, G, U, cap, B);
+        const CoopPlan cp0 = path == TRI_PATH_AUTO ? coop_plan(dt, G, U, cap) : CoopPlan();
+        const bool take = pp.ok && (path == TRI_PATH_PIPE || !(cp0.ok && U < sms));
+        if (take) {
+            w.pipe = true;
+            w.pp = pp;
+            Carve c;
+            w.queue = c.take(4);
+            w.counters = c.take(static_cast<size_t>(U) * 4);
+            w.zero_end = c.off;
+            // Score rows are padded to a multiple of 32 keys (16-byte groups).
+            const int64_t capP = (cap + 31) & ~int64_t(31);
+            if (pp.big) {
+                w.wts = c.take(static_cast<size_t>(U * G) * kWHead * 4);
+                w.raw = c.take(static_cast<size_t>(U * G * capP) * 4);
+                w.partial = c.take(static_cast<size_t>(U * pp.cpu * G * 2) * 8);
+                w.fin_scratch = c.take(static_cast<size_t>(pp.grid * capP) * 4);
+            } else {
+                w.raw = c.take(static_cast<size_t>(pp.grid * G * capP) * 4);
+            }
+            w.kept = own_kept ? c.take(static_cast<size_t>(U * B) * 4) : 0;
+            w.total = c.off;
+            return w;
+        }
+        if (path == TRI_PATH_PIPE) return w;  // not possible: tri_prune reports it
+    }
     const bool fused_ok = path != TRI_PATH_SPLIT && path != TRI_PATH_COOP &&
                           use_fused(dt, G, cap, B, path);
     const CoopPlan cp = (path == TRI_PATH_AUTO || path == TRI_PATH_COOP)
@@ -365,7 +437,7 @@ PruneWs prune_ws(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int6
 
 // Every exported call that launches kernels starts a fresh launch count.
 struct LaunchScope {
-    LaunchScope() { t_launches = 0; }
+    LaunchScope() { begin_launches(); }
 };
 
 char* ws_at(void* ws, size_t off) { return static_cast<char*>(ws) + off; }
@@ -564,7 +636,8 @@ size_t tri_prune_workspace_bytes(int64_t n_seq, int64_t n_layers, int64_t n_kvhe
     if (check_units(n_seq, n_layers, n_kvheads, G, cap) != TRI_OK || B < 1) return kWsHeader;
     size_t best = 0;
     for (tri_dtype dt : {TRI_BF16, TRI_F32}) {
-        for (int path : {TRI_PATH_AUTO, TRI_PATH_FUSED, TRI_PATH_SPLIT, TRI_PATH_COOP}) {
+        for (int path : {TRI_PATH_AUTO, TRI_PATH_FUSED, TRI_PATH_SPLIT, TRI_PATH_COOP,
+                         TRI_PATH_PIPE}) {
             const size_t t = prune_ws(n_seq, n_layers, n_kvheads, G, cap, B, dt, true, path).total;
             if (t > best) best = t;
         }
@@ -577,9 +650,10 @@ int tri_prune_path(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, in
     if (check_units(n_seq, n_layers, n_kvheads, G, cap) != TRI_OK || B < 1 || !dtype_ok(dt))
         return -1;
     const PruneWs w = prune_ws(n_seq, n_layers, n_kvheads, G, cap, B, dt, false, path);
+    if (w.pipe) return TRI_PATH_PIPE;
     if (w.coop) return TRI_PATH_COOP;
     if (w.fused) return TRI_PATH_FUSED;
-    if (path == TRI_PATH_FUSED || path == TRI_PATH_COOP) return -1;
+    if (path == TRI_PATH_FUSED || path == TRI_PATH_COOP || path == TRI_PATH_PIPE) return -1;
     return TRI_PATH_SPLIT;
 }
 
@@ -588,7 +662,8 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
                      int64_t n_kvheads, int G, int64_t cap_src, const int32_t* n_valid,
                      const int64_t* p_cur, const float* stats, int64_t B, void* k_dst,
                      void* v_dst, int32_t* pos_dst, int64_t cap_dst, int32_t* kept_idx,
-                     int32_t* n_kept, void* ws, size_t ws_bytes, void* stream) {
+                     int32_t* n_kept, float* final_score, void* ws, size_t ws_bytes,
+                     void* stream) {
     LaunchScope scope_;
     FoldOffsets off;
     TRI_TRY(check_cfg(cfg, &off));
@@ -601,7 +676,8 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
     if (cap_dst < (B < cap_src ? B : cap_src)) return TRI_ERR_INVALID_ARG;
     if (!aligned16(k_src) || !aligned16(k_dst) ||
         (v_src && (!aligned16(v_src) || !aligned16(v_dst))) || !aligned16(stats) ||
-        !aligned4(n_kept) || (kept_idx && !aligned4(kept_idx)) || (n_valid && !aligned4(n_valid)))
+        !aligned4(n_kept) || (kept_idx && !aligned4(kept_idx)) || (n_valid && !aligned4(n_valid)) ||
+        (final_score && !aligned4(final_score)))
         return TRI_ERR_INVALID_ARG;
     const int64_t U = n_seq * n_layers * n_kvheads;
     const size_t esz = dt == TRI_BF16 ? 2 : 4;
@@ -612,11 +688,56 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
         prune_ws(n_seq, n_layers, n_kvheads, G, cap_src, B, dt, kept_idx == nullptr, cfg->path);
     if (cfg->path == TRI_PATH_FUSED && !w.fused) return TRI_ERR_UNSUPPORTED;
     if (cfg->path == TRI_PATH_COOP && !w.coop) return TRI_ERR_UNSUPPORTED;
+    if (cfg->path == TRI_PATH_PIPE && !w.pipe) return TRI_ERR_UNSUPPORTED;
     if (!ws || !aligned16(ws) || ws_bytes < w.total) return TRI_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     float* wts = reinterpret_cast<float*>(ws_at(ws, w.sc.wts));
     int32_t* kept = kept_idx ? kept_idx : reinterpret_cast<int32_t*>(ws_at(ws, w.kept));
     uint32_t* flag = ws_flag(ws);
+
+    if (w.pipe) {
+        CUtensorMap map;
+        TRI_TRY(make_key_map(&map, k_src, dt, U * cap_src, pipe_tile_keys(dt),
+                             pipe_slice_bytes(w.pp.big)));
+        // One memset: the flag word, the work-item queue and the unit counters.
+        TRI_CUDA(cudaMemsetAsync(ws, 0, w.zero_end, s));
+        PipeArgs a;
+        a.n_units = U;
+        a.gslots = w.pp.gslots;
+        a.cap = cap_src;
+        a.cap_dst = cap_dst;
+        a.B = B;
+        a.n_valid = n_valid;
+        a.stats = stats;
+        a.p_cur = p_cur;
+        a.n_layers = n_layers;
+        a.n_kvheads = n_kvheads;
+        a.fc = fold_const(cfg);
+        a.wts = nullptr;
+        a.k_src = k_src;
+        a.v_src = v_src;
+        a.pos_src = pos_src;
+        a.k_dst = k_dst;
+        a.v_dst = v_dst;
+        a.pos_dst = pos_dst;
+        a.kept = kept_idx;
+        a.n_kept = n_kept;
+        a.final_out = final_score;
+        a.raw = reinterpret_cast<float*>(ws_at(ws, w.raw));
+        a.fin_scratch = w.pp.big ? reinterpret_cast<float*>(ws_at(ws, w.fin_scratch)) : nullptr;
+        a.partial = w.pp.big ? reinterpret_cast<double*>(ws_at(ws, w.partial)) : nullptr;
+        a.counters = reinterpret_cast<uint32_t*>(ws_at(ws, w.counters));
+        a.queue = reinterpret_cast<uint32_t*>(ws_at(ws, w.queue));
+        a.trace = w.pp.big ? nullptr : phase_trace_buffer(U);
+        a.flag = flag;
+        if (w.pp.big) {
+            float* pw = reinterpret_cast<float*>(ws_at(ws, w.wts));
+            TRI_CUDA(launch_fold(stats, p_cur, n_seq, n_layers, n_kvheads * G, cfg->theta, off, pw,
+                                 s));
+            a.wts = pw;
+        }
+        return cuda_status(launch_pipe(dt, G, w.pp.big, map, a, static_cast<int>(w.pp.grid), s));
+    }
 
     if (w.coop) {
         CUtensorMap map;
@@ -645,6 +766,7 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
         a.pos_dst = pos_dst;
         a.kept = kept_idx;
         a.n_kept = n_kept;
+        a.final_out = final_score;
         a.scratch = reinterpret_cast<float*>(ws_at(ws, w.sc.raw));
         a.partial = reinterpret_cast<double*>(ws_at(ws, w.partial));
         a.hists = reinterpret_cast<uint32_t*>(ws_at(ws, w.hists));
@@ -683,6 +805,7 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
         a.pos_dst = pos_dst;
         a.kept = kept_idx;
         a.n_kept = n_kept;
+        a.final_out = final_score;
         a.scratch = reinterpret_cast<float*>(ws_at(ws, w.sc.raw));
         a.trace = phase_trace_buffer(U);
         a.flag = flag;
@@ -710,7 +833,7 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
     a.flag = flag;
     const int n_sm = device_info().sm_count;
     TRI_CUDA(launch_score(dt, G, map, a, n_sm, s));
-    float* fin = reinterpret_cast<float*>(ws_at(ws, w.fin));
+    float* fin = final_score ? final_score : reinterpret_cast<float*>(ws_at(ws, w.fin));
     uint32_t* hists = reinterpret_cast<uint32_t*>(ws_at(ws, w.sel.hists));
     TRI_CUDA(launch_zmax(G, a.raw, U, cap_src, n_valid, a.mom, fin, hists, flag, s));
     for (int p = 1; p < 3; ++p)

@@ -374,6 +374,7 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
                             best = (h == 0) ? z : fmaxf(best, z);
                         }
                         fin[jl] = best;
+                        if (a.final_out) a.final_out[u * a.cap + j0 + jl] = best;
                         if (best != best) nonfinite = true;
                         atomicAdd(&hist[zbin(best)], 1u);
                     }
@@ -760,8 +761,22 @@ static cudaError_t launch_coop_t(const CUtensorMap& map, const CoopArgs& a, int 
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<n_ctas, CoopShape<T>::kThreads, smem, s>>>(map, a);
+    // The CTAs of a unit wait for one another at unit barriers, so all of
+    // them must be resident at once: a cooperative launch guarantees it or
+    // fails here, instead of leaving CTAs to time out at the barriers.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(n_ctas));
+    cfg.blockDim = dim3(CoopShape<T>::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, map, a);
     note_launch(s);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

@@ -19,25 +19,34 @@ struct FoldShared {
 };
 static_assert(sizeof(FoldShared) <= kFoldStaticBytes, "fold factors exceed their budget");
 
-// Weight records of the G query heads of unit u into w (shared memory).
-// Two __syncthreads inside; every thread of the CTA must call it.
+// Weight records of the G query heads of unit u into w (shared memory),
+// computed by the first nthreads threads of the CTA: with bar_id 0 they are
+// all of its threads (two __syncthreads inside), otherwise the named barrier
+// bar_id synchronises exactly those threads.
 template <int G>
-__device__ __forceinline__ void fold_unit(FoldShared& fs, const FoldConst& fc, float* w,
-                                          const float* stats, const int64_t* p_cur, int64_t u,
-                                          int64_t n_layers, int64_t n_kvheads) {
+__device__ __forceinline__ void fold_unit_sync(FoldShared& fs, const FoldConst& fc, float* w,
+                                               const float* stats, const int64_t* p_cur,
+                                               int64_t u, int64_t n_layers, int64_t n_kvheads,
+                                               int bar_id, int nthreads) {
     const int t = threadIdx.x;
     const int64_t kvh = u % n_kvheads;
     const int64_t layer = (u / n_kvheads) % n_layers;
     const int64_t seq = u / (n_kvheads * n_layers);
+    auto sync = [&]() {
+        if (bar_id == 0)
+            __syncthreads();
+        else
+            named_sync(bar_id, nthreads);
+    };
     if (t < kF) {
         double ps, pc;
         sincos(fc.omega[t] * static_cast<double>(p_cur[seq]), &ps, &pc);
         fs.ef[t][0] = pc;
         fs.ef[t][1] = ps;
     }
-    __syncthreads();
+    sync();
     const float* st_base = stats + ((layer * n_kvheads + kvh) * G) * kF * 4;
-    for (int e = t; e < G * kF; e += blockDim.x) {
+    for (int e = t; e < G * kF; e += nthreads) {
         const int h = e / kF, f = e % kF;
         const float4 st = *reinterpret_cast<const float4*>(st_base + (h * kF + f) * 4);
         const double mre = st.x, mim = st.y;
@@ -52,7 +61,16 @@ __device__ __forceinline__ void fold_unit(FoldShared& fs, const FoldConst& fc, f
         rec[2 * i + 1] = static_cast<float>(aim);
         rec[8 + i] = static_cast<float>(cw);
     }
-    __syncthreads();
+    sync();
+}
+
+// Every thread of the CTA computes the fold (two __syncthreads inside).
+template <int G>
+__device__ __forceinline__ void fold_unit(FoldShared& fs, const FoldConst& fc, float* w,
+                                          const float* stats, const int64_t* p_cur, int64_t u,
+                                          int64_t n_layers, int64_t n_kvheads) {
+    fold_unit_sync<G>(fs, fc, w, stats, p_cur, u, n_layers, n_kvheads, 0,
+                      static_cast<int>(blockDim.x));
 }
 
 }  // namespace tri

@@ -339,6 +339,7 @@ prune_fused_kernel(const __grid_constant__ CUtensorMap kmap, FusedArgs a) {
                                 best = (h == 0) ? z : fmaxf(best, z);
                             }
                             fin[j] = best;
+                            if (a.final_out) a.final_out[u * a.cap + j] = best;
                             if (best != best) nonfinite = true;
                             atomicAdd(&hist[zbin(best)], 1u);
                         }

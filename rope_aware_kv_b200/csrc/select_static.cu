@@ -23,21 +23,25 @@ constexpr size_t kStaticScratchBytes = size_t(1) << 20;
 
 static __device__ __align__(256) uint8_t g_select_scratch[kStaticScratchBytes];
 
-constexpr size_t kAlign = 256;
-size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
-
-// Device address of g_select_scratch on the current device, looked up once
-// per device with that device current.
-tri_status scratch_address(void** out) {
+// Device address of g_select_scratch on the current device.  Looked up with
+// that device current on every call made outside stream capture (so a
+// context re-created after cudaDeviceReset is followed), and remembered per
+// device for calls made while the stream is being captured, which must come
+// after one uncaptured call on that device.
+tri_status scratch_address(cudaStream_t s, void** out) {
     static std::mutex mu;
     static void* addr[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return TRI_ERR_CUDA;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) return TRI_ERR_CUDA;
     std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
+    if (cs == cudaStreamCaptureStatusNone) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess || !p) return TRI_ERR_CUDA;
         addr[dev] = p;
+    } else if (!addr[dev]) {
+        return TRI_ERR_CUDA;  // first call on this device under capture
     }
     *out = addr[dev];
     return TRI_OK;
@@ -58,18 +62,16 @@ extern "C" tri_status tri_select_topB_static(const float* final_score, int64_t n
     if (!aligned4(final_score) || !aligned4(kept_idx) || !aligned4(n_kept) ||
         (n_valid && !aligned4(n_valid)))
         return TRI_ERR_INVALID_ARG;
-    // Same layout as tri_select_topB's workspace: flag word, three radix
+    tri::begin_launches();
+    // The layout of tri_select_topB's workspace: flag word, three radix
     // histograms per unit, per-chunk counts.
-    const size_t hists = tri::kWsHeader;
-    const size_t counts =
-        align_up(hists + static_cast<size_t>(3 * n_units) * tri::kHistBins0 * 4);
-    const int64_t chunks = (cap + tri::kZChunk - 1) / tri::kZChunk;
-    const size_t need = align_up(counts + static_cast<size_t>(n_units * chunks) * 8);
-    if (need > kStaticScratchBytes) return TRI_ERR_SCRATCH_LIMIT;
-    void* ws = nullptr;
-    const tri_status st = scratch_address(&ws);
-    if (st != TRI_OK) return st;
+    const tri::SelectWs lay = tri::select_ws(tri::kWsHeader, n_units, cap);
+    if (lay.total > kStaticScratchBytes) return TRI_ERR_SCRATCH_LIMIT;
+    const size_t hists = lay.hists, counts = lay.counts;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    void* ws = nullptr;
+    const tri_status st = scratch_address(s, &ws);
+    if (st != TRI_OK) return st;
     char* base = static_cast<char*>(ws);
     // The histograms accumulate with atomics: zero them (and the flag word).
     if (cudaMemsetAsync(base, 0, counts, s) != cudaSuccess) return TRI_ERR_CUDA;

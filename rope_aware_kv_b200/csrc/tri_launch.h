@@ -66,8 +66,42 @@ struct FusedArgs {
     int32_t* pos_dst;
     int32_t* kept;               // [U][B] or null
     int32_t* n_kept;             // [U]
+    float* final_out;            // [U][cap] final scores, or null
     float* scratch;              // [grid][G][cap] per-CTA score scratch
     uint64_t* trace;             // [U][kTracePoints] phase timestamps, or null
+    uint32_t* flag;
+};
+
+// The pipelined kernel (pipe.cu).
+struct PipeArgs {
+    int64_t n_units;
+    int gslots;                  // gather buffers (shared memory permitting)
+    int64_t cap;
+    int64_t cap_dst;
+    int64_t B;
+    const int32_t* n_valid;
+    // fold inputs of the small-unit mode (the kernel forms the weights itself)
+    const float* stats;          // [L][Hkv*G][64][4]
+    const int64_t* p_cur;        // [n_seq]
+    int64_t n_layers;
+    int64_t n_kvheads;
+    FoldConst fc;
+    const float* wts;            // large-unit mode: fold output [U*G][192]
+    const void* k_src;
+    const void* v_src;
+    const int32_t* pos_src;
+    void* k_dst;
+    void* v_dst;
+    int32_t* pos_dst;
+    int32_t* kept;               // [U][B] or null
+    int32_t* n_kept;             // [U]
+    float* final_out;            // [U][cap] or null
+    float* raw;                  // small: [grid][G][cap]; large: [U][G][cap]
+    float* fin_scratch;          // large: [grid][cap] (when final_out is null)
+    double* partial;             // large: [U][chunks][G][2]
+    uint32_t* counters;          // large: [U], zero on entry
+    uint32_t* queue;             // large: work-item counter, zero on entry
+    uint64_t* trace;             // [U][kTracePoints][kTraceWarps] or null (small mode)
     uint32_t* flag;
 };
 
@@ -102,6 +136,7 @@ struct CoopArgs {
     int32_t* pos_dst;
     int32_t* kept;               // [U][B] or null
     int32_t* n_kept;             // [U]
+    float* final_out;            // [U][cap] final scores, or null
     float* scratch;              // [grid][G][keys_max]
     double* partial;             // [U][C][G][2]
     uint32_t* hists;             // [U][2048] z-bin histograms, zero on entry
@@ -114,6 +149,18 @@ struct CoopArgs {
     uint32_t* flag;
 };
 
+
+// api.cu: byte offsets of the selection's scratch from `start` (the flag
+// word comes first): three radix histograms per unit, then per-chunk
+// counts.  Shared by tri_select_topB and its static-scratch variant.
+struct SelectWs {
+    size_t hists, counts, total;
+};
+SelectWs select_ws(size_t start, int64_t n_units, int64_t cap);
+
+// api.cu: every exported call that launches kernels starts a fresh launch
+// count for tri_last_launch_count.
+void begin_launches();
 
 // api.cu: the caller's phase-trace buffer for the next launches (or null).
 uint64_t* phase_trace_buffer(int64_t n_units);
@@ -171,5 +218,17 @@ size_t fused_smem_limit();
 int fused_tile_keys(tri_dtype dt);
 cudaError_t launch_fused(tri_dtype dt, int G, const CUtensorMap& map, const FusedArgs& a,
                          int n_ctas, cudaStream_t s);
+
+// pipe.cu
+size_t pipe_smem_bytes(tri_dtype dt, int G, int64_t cap, int64_t B, bool big, int gslots);
+int pipe_min_gslots();
+int pipe_max_gslots();
+bool pipe_small_fits(tri_dtype dt, int64_t cap);
+int pipe_slice_bytes(bool big);
+int pipe_engine_warps();
+int pipe_tile_keys(tri_dtype dt);
+int pipe_chunk_keys(tri_dtype dt);
+cudaError_t launch_pipe(tri_dtype dt, int G, bool big, const CUtensorMap& map, const PipeArgs& a,
+                        int n_ctas, cudaStream_t s);
 
 }  // namespace tri

@@ -74,7 +74,7 @@ def _prune_status(lib, cfg, **over):
     args = dict(k_src=1 << 36, v_src=1 << 37, pos_src=1 << 38, dt=tri.TRI_BF16, n_seq=1,
                 n_layers=1, n_kvheads=4, G=7, cap=4096, n_valid=None, p_cur=16, stats=16, B=512,
                 k_dst=1 << 40, v_dst=1 << 41, pos_dst=1 << 42, cap_dst=512, kept=None, n_kept=16,
-                ws=None, ws_bytes=0)
+                final=None, ws=None, ws_bytes=0)
     args.update(over)
     P = lambda v: None if v is None else ctypes.c_void_p(v)
     return lib.tri_prune(ctypes.byref(cfg) if cfg is not None else None, P(args["k_src"]),
@@ -82,7 +82,8 @@ def _prune_status(lib, cfg, **over):
                          args["n_layers"], args["n_kvheads"], args["G"], args["cap"],
                          P(args["n_valid"]), P(args["p_cur"]), P(args["stats"]), args["B"],
                          P(args["k_dst"]), P(args["v_dst"]), P(args["pos_dst"]), args["cap_dst"],
-                         P(args["kept"]), P(args["n_kept"]), P(args["ws"]), args["ws_bytes"], None)
+                         P(args["kept"]), P(args["n_kept"]), P(args["final"]), P(args["ws"]),
+                         args["ws_bytes"], None)
 
 
 def test_host_validation_without_gpu(lib):
@@ -101,6 +102,8 @@ def test_host_validation_without_gpu(lib):
     assert _prune_status(lib, cfg, v_dst=(1 << 37) + 256) == 1   # V destination overlaps V
     assert _prune_status(lib, cfg, k_dst=(1 << 37) + 512) == 1   # K destination overlaps V
     assert _prune_status(lib, cfg, pos_dst=(1 << 38) + 64) == 1  # positions overlap
+    assert _prune_status(lib, cfg, final=(1 << 43) + 2) == 1     # misaligned final scores
+    assert _prune_status(lib, cfg, final=1 << 43) == 3           # well formed: no workspace
     bad = tri.config(head_dim=64)
     assert _prune_status(lib, bad) == 2
     cfg2 = tri.config()
@@ -108,6 +111,7 @@ def test_host_validation_without_gpu(lib):
     assert _prune_status(lib, cfg2) == 1
     cfg3 = tri.config(path=7)
     assert _prune_status(lib, cfg3) == 1
+    assert _prune_status(lib, tri.config(path=tri.PATH_PIPE)) in (2, 3)  # no device here: 2
 
 
 def test_calibration_split_validation_without_gpu(lib):

@@ -39,6 +39,10 @@ MUTANTS = [
     ("gather off by one", "const int64_t src = u * cap + kp[rr];",
      "const int64_t src = u * cap + kp[rr] + (kp[rr] + 1 < n ? 1 : 0);"),
     ("mean norm uses |mean|", "sn += hypot(x, y);", "sn += fabs(x) + fabs(y);"),
+    ("head max keeps a leading NaN", "for (int h = 1; h < G; ++h) m = fmax(m, z[(int64_t)h * n + j]);",
+     "for (int h = 1; h < G; ++h) m = (z[(int64_t)h * n + j] > m) ? z[(int64_t)h * n + j] : m;"),
+    ("head max takes a later NaN", "for (int h = 1; h < G; ++h) m = fmax(m, z[(int64_t)h * n + j]);",
+     "for (int h = 1; h < G; ++h) m = (m > z[(int64_t)h * n + j]) ? m : z[(int64_t)h * n + j];"),
 ]
 
 PIN_TESTS = [
@@ -49,6 +53,7 @@ PIN_TESTS = [
     lambda: pins.test_offset_fold_equals_direct_sum(),
     lambda: pins.test_linear_offsets_geometric_closed_form(),
     lambda: pins.test_znorm_population_moments_and_max(),
+    lambda: pins.test_znorm_max_skips_a_nan_head(),
     lambda: [pins.test_select_matches_brute_force(s) for s in range(12)],
     lambda: pins.test_select_order_and_threshold(),
     lambda: [pins.test_prune_gather_is_bitwise_and_ascending(dt) for dt in ("f32", "bf16")],

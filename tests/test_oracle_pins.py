@@ -203,6 +203,26 @@ def test_znorm_population_moments_and_max():
     assert np.all([fin[j] in z[:, j] for j in range(raw.shape[1])])
 
 
+def test_znorm_max_skips_a_nan_head():
+    """Reading of the head maximum (the pages are silent on NaN): a head whose
+    scores are NaN (its moments are NaN, so every z of it is NaN) is skipped
+    by the maximum, wherever it sits in the group; the final score is NaN
+    only when every head is NaN.  Expected values are the largest finite z
+    of each key, formed here from the z the oracle returns."""
+    rng = np.random.default_rng(16)
+    for nan_head in (0, 2):
+        raw = rng.normal(size=(3, 50)) * np.array([[1.0], [2.0], [0.5]])
+        raw[nan_head, 7] = np.nan  # one NaN score poisons that head's moments
+        z, fin, mu, sd = oracle.znorm_max(raw)
+        assert np.isnan(mu[nan_head]) and np.all(np.isnan(z[nan_head]))
+        others = [h for h in range(3) if h != nan_head]
+        assert not np.any(np.isnan(fin))
+        np.testing.assert_array_equal(fin, np.max(z[others], axis=0))
+    raw = np.full((2, 5), np.nan)
+    _, fin, _, _ = oracle.znorm_max(raw)
+    assert np.all(np.isnan(fin))
+
+
 def _brute_force_topB(vals, B):
     n = len(vals)
     m = min(B, n)

@@ -271,6 +271,7 @@ struct PruneWs {
     CoopPlan cp;
     PipePlan pp;
     size_t queue = 0, counters = 0, wts = 0, raw = 0, fin_scratch = 0;
+    size_t zcand = 0, zcount = 0, zstate = 0;  // split path: z-bin selection
     ScoreWs sc;
     size_t fin = 0, kept = 0;
     SelectWs sel;
@@ -335,6 +336,7 @@ PipePlan pipe_plan(tri_dtype dt, int G, int64_t U, int64_t cap, int64_t B) {
     PipePlan p;
     const int64_t sms = sm_count_or_default();
     const bool small = pipe_small_fits(dt, cap);
+    if (!small && !pipe_big_fits(cap)) return p;
     const int e = pipe_engine_warps();
     for (int g = pipe_max_gslots() / e * e; g >= pipe_min_gslots(); g -= e) {
         if (pipe_smem_bytes(dt, G, cap, B, !small, g) <= fused_smem_limit()) {
@@ -364,7 +366,10 @@ PruneWs prune_ws(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int6
     if (path == TRI_PATH_PIPE || path == TRI_PATH_AUTO) {
         const PipePlan pp = pipe_plan(dt, G, U, cap, B);
         const CoopPlan cp0 = path == TRI_PATH_AUTO ? coop_plan(dt, G, U, cap) : CoopPlan();
-        const bool take = pp.ok && (path == TRI_PATH_PIPE || !(cp0.ok && U < sms));
+        // AUTO takes the pipelined kernel for units that fit one CTA (whole
+        // units per CTA); units scored in chunks run faster on the split
+        // kernels.
+        const bool take = pp.ok && (path == TRI_PATH_PIPE || (!pp.big && !(cp0.ok && U < sms)));
         if (take) {
             w.pipe = true;
             w.pp = pp;
@@ -431,7 +436,11 @@ PruneWs prune_ws(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int6
     w.fin = c.take(static_cast<size_t>(U * cap) * 4);
     w.kept = own_kept ? c.take(static_cast<size_t>(U * B) * 4) : 0;
     w.sel = select_ws(c.off, U, cap);
-    w.total = w.sel.total;
+    c.off = w.sel.total;
+    w.zcand = c.take(static_cast<size_t>(U) * kCandMax * 8);
+    w.zcount = c.take(static_cast<size_t>(U) * 4);
+    w.zstate = c.take(static_cast<size_t>(U) * zsel_state_bytes());
+    w.total = c.off;
     return w;
 }
 
@@ -569,7 +578,7 @@ tri_status tri_score(const tri_config* cfg, const void* k_post, tri_dtype dt, in
     a.mom = reinterpret_cast<float2*>(ws_at(ws, w.mom));
     a.flag = ws_flag(ws);
     TRI_CUDA(launch_score(dt, G, map, a, device_info().sm_count, s));
-    TRI_CUDA(launch_zmax(G, a.raw, U, cap, n_valid, a.mom, final_score, nullptr, a.flag, s));
+    TRI_CUDA(launch_zmax(G, a.raw, U, cap, n_valid, a.mom, final_score, nullptr, 0, a.flag, s));
     return TRI_OK;
 }
 
@@ -818,6 +827,7 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
     TRI_CUDA(cudaMemsetAsync(ws, 0, kWsHeader, s));
     TRI_CUDA(cudaMemsetAsync(ws_at(ws, w.sc.counters), 0, static_cast<size_t>(U) * 4, s));
     TRI_CUDA(cudaMemsetAsync(ws_at(ws, w.sel.hists), 0, w.sel.counts - w.sel.hists, s));
+    TRI_CUDA(cudaMemsetAsync(ws_at(ws, w.zcount), 0, static_cast<size_t>(U) * 4, s));
     TRI_CUDA(launch_fold(stats, p_cur, n_seq, n_layers, n_kvheads * G, cfg->theta, off, wts, s));
     ScoreArgs a;
     a.keys = k_src;
@@ -835,12 +845,12 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
     TRI_CUDA(launch_score(dt, G, map, a, n_sm, s));
     float* fin = final_score ? final_score : reinterpret_cast<float*>(ws_at(ws, w.fin));
     uint32_t* hists = reinterpret_cast<uint32_t*>(ws_at(ws, w.sel.hists));
-    TRI_CUDA(launch_zmax(G, a.raw, U, cap_src, n_valid, a.mom, fin, hists, flag, s));
-    for (int p = 1; p < 3; ++p)
-        TRI_CUDA(launch_radix_pass(fin, U, cap_src, n_valid, B, hists, p, flag, s));
-    TRI_CUDA(launch_select_finish(fin, U, cap_src, n_valid, B, hists,
-                                  reinterpret_cast<uint2*>(ws_at(ws, w.sel.counts)), kept, n_kept,
-                                  s));
+    TRI_CUDA(launch_zmax(G, a.raw, U, cap_src, n_valid, a.mom, fin, hists, 1, flag, s));
+    TRI_CUDA(launch_zselect(fin, U, cap_src, n_valid, B, hists,
+                            reinterpret_cast<uint2*>(ws_at(ws, w.sel.counts)),
+                            reinterpret_cast<int2*>(ws_at(ws, w.zcand)),
+                            reinterpret_cast<uint32_t*>(ws_at(ws, w.zcount)), ws_at(ws, w.zstate), kept,
+                            n_kept, s));
     return cuda_status(launch_gather(dt, k_src, v_src, pos_src, U, cap_src, kept, n_kept, B, k_dst,
                                      v_dst, pos_dst, cap_dst, flag, n_sm * 8, s));
 }

@@ -96,10 +96,15 @@ struct PipeShape {
     static constexpr int kGGap = 1;
     static constexpr int kHand = 2;                // index buffers (units handed to the engine)
     static_assert(kGRows <= 32, "one lane per destination row of a gather piece");
-    static_assert(kMinGSlots >= (kGGap + 2) * kEngWarps, "gather ring too shallow");
+    static_assert(kMinGSlots >= (kGGap + 1) * kEngWarps, "gather ring too shallow");
+    static_assert(kEngWarps <= 2, "run-start scratch for two engine warps");
 };
 
 constexpr int kPipeCand = 1024;   // threshold-bin candidates listed in shared memory
+// Large units merge their chunks' moment partials in the idle rings, after
+// the histogram and the candidate list.
+constexpr int kPartOff = 16384;
+
 // Tiles per work item of a large unit: a multiple of the math warps' count.
 constexpr int kChunkTiles = 6 * PipeShape<float>::kMathWarps;
 
@@ -134,7 +139,7 @@ __host__ __device__ inline PipeLayout pipe_layout(int G, int64_t cap, int64_t B,
     L.kidx = o;
     o += SS::kHand * ((static_cast<size_t>(m) * (big ? 4 : 2) + 15) & ~size_t(15));
     L.smask = o;
-    o += SS::kHand * ((static_cast<size_t>((m + SS::kGRows - 1) / SS::kGRows) * 4 + 15) & ~size_t(15));
+    o += SS::kHand * ((static_cast<size_t>((m + SS::kGRows - 1) / SS::kGRows) * 8 + 15) & ~size_t(15));
     L.bars = o;
     o += (SS::kMathWarps * SB::kQ * 2 + SS::kMaxGSlots + 2 * SS::kHand) * 8;
     L.red = o;
@@ -172,6 +177,7 @@ struct PipeMisc {
     int32_t hdr_m[PipeShape<float>::kHand];
     uint32_t gdst_rows[PipeShape<float>::kMaxGSlots];  // engine: rows of each gather buffer
     int64_t gdst[PipeShape<float>::kMaxGSlots];        // engine: destination byte offset
+    int32_t runst[2][64];                              // engine: start row of each run
 };
 static_assert(sizeof(PipeMisc) <= 1024, "misc state exceeds its budget");
 
@@ -191,20 +197,6 @@ __device__ __forceinline__ void bulk_store_hint(void* gdst, const void* smem_src
                      "l"(reinterpret_cast<uint64_t>(gdst)),
                  "r"(smem_u32(smem_src)), "r"(bytes), "l"(policy)
                  : "memory");
-}
-
-// Drop lines from L2 without writing them back (scratch no longer needed):
-// every whole 128-byte line inside [p, p + bytes), by the math threads.
-__device__ __forceinline__ void discard_l2(const void* p) {
-    asm volatile("discard.global.L2 [%0], 128;" ::"l"(reinterpret_cast<uint64_t>(p)) : "memory");
-}
-__device__ __forceinline__ void discard_range(const void* p, int64_t bytes, int tid, int nthr) {
-    const uintptr_t b = reinterpret_cast<uintptr_t>(p);
-    const uintptr_t lo = (b + 127) & ~uintptr_t(127);
-    const uintptr_t hi = (b + static_cast<uintptr_t>(bytes)) & ~uintptr_t(127);
-    for (uintptr_t a = lo + static_cast<uintptr_t>(tid) * 128; a < hi;
-         a += static_cast<uintptr_t>(nthr) * 128)
-        discard_l2(reinterpret_cast<const void*>(a));
 }
 
 // Score KPT keys (rows lane + 32 k of the tile) on the chunks of one slice
@@ -322,6 +314,123 @@ __device__ __forceinline__ float f4at(const float4& v, int i) {
 // Round a key count up to the padded row length of the score scratch.
 __host__ __device__ __forceinline__ int64_t pipe_pad(int64_t n) { return (n + 31) & ~int64_t(31); }
 
+// Rank the listed threshold-bin candidates (at most kPipeCand): the B-th
+// key's full 32-bit key T into ms->st.prefix and the number of its ties that
+// are kept into ms->st.k.  Directly (one candidate per thread) when they are
+// few, else by a three-digit radix of their keys.  Every math thread calls it.
+__device__ __forceinline__ void rank_listed(int nc, uint32_t* hist, const int2* cand, PipeMisc* ms) {
+    using S = PipeShape<float>;
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    if (nc <= S::kMath) {
+        const uint32_t k0 = ms->st.k;
+        math_sync();  // k0 read before st changes
+        const int2 me = tid < nc ? cand[tid] : make_int2(0, 0);
+        const uint32_t mk = static_cast<uint32_t>(me.x);
+        uint32_t above = 0, rank = 0;
+        for (int i = 0; i < nc; ++i) {
+            const int2 e = cand[i];
+            const uint32_t ek = static_cast<uint32_t>(e.x);
+            above += ek > mk;
+            rank += (ek > mk) || (ek == mk && e.y < me.y);
+        }
+        if (tid < nc && rank == k0 - 1) {
+            ms->st.prefix = mk;
+            ms->st.k = k0 - above;  // ties of the threshold key that are kept
+        }
+        math_sync();
+        return;
+    }
+    for (int p = 0; p < 3; ++p) {
+        const int nb = 1 << pass_bits(p);
+        for (int b = tid; b < nb; b += S::kMath) hist[b] = 0;
+        math_sync();
+        const uint32_t prefix = ms->st.prefix;
+        const int shift = pass_shift(p);
+        const int hi_shift = shift + pass_bits(p);
+        for (int i = tid; i < nc; i += S::kMath) {
+            const uint32_t key = static_cast<uint32_t>(cand[i].x);
+            if (p == 0 || (key >> hi_shift) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+        }
+        math_sync();
+        if (warp == 0) {
+            uint32_t bin, above;
+            warp_find_bin(hist, nb, ms->st.k, bin, above);
+            if (lane == 0) {
+                ms->st.prefix = (prefix << pass_bits(p)) | bin;
+                ms->st.k -= above;
+                ms->st.gt += above;
+            }
+        }
+        math_sync();
+    }
+}
+
+// The z-bin b0 holding the B-th key, and the selection state that follows
+// from it (warp 0), from a unit's z-bin histogram.
+__device__ __forceinline__ void threshold_bin(const uint32_t* hist, int64_t B, PipeMisc* ms) {
+    const int lane = threadIdx.x & 31;
+    uint32_t bin, above;
+    warp_find_bin(hist, kZBins, static_cast<uint32_t>(B), bin, above);
+    if (lane == 0) {
+        ms->zb0 = bin;
+        ms->ncand = 0;
+        ms->st.prefix = 0;
+        ms->st.k = static_cast<uint32_t>(B) - above;  // to take from bin b0
+        ms->st.gt = above;
+        ms->st.keep_all = 0;
+    }
+}
+
+// Ordered write of one 128-key block of final scores v (lane l holds keys
+// 4l .. 4l + 3 of the block, the first at index jb): every key above T and
+// the ties of T while fewer than kt have been taken; pos / ties run on.
+template <typename Idx>
+__device__ __forceinline__ void write_block(const float4& v, int jb, int valid_to, uint32_t Tk,
+                                            uint32_t kt, int m, uint32_t& pos, uint32_t& ties,
+                                            Idx* kidx) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t lt = (1u << lane) - 1u;
+    uint32_t gtm = 0, eqm = 0;  // 4-bit masks of this lane's keys
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t key = ordered_key(f4at(v, i));
+        const bool valid = jb + i < valid_to;
+        gtm |= (valid && key > Tk) ? (1u << i) : 0u;
+        eqm |= (valid && key == Tk) ? (1u << i) : 0u;
+    }
+    // Keys are ordered lane-major: ties before this lane's keys.
+    uint32_t eq_before = 0, eq_total = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t bal = __ballot_sync(0xffffffffu, (eqm >> i) & 1u);
+        eq_before += __popc(bal & lt);
+        eq_total += __popc(bal);
+    }
+    uint32_t keepm = gtm;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t my_tie = ties + eq_before + __popc(eqm & ((1u << i) - 1u));
+        if (((eqm >> i) & 1u) && my_tie < kt) keepm |= 1u << i;
+    }
+    uint32_t keep_before = 0, keep_total = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t bal = __ballot_sync(0xffffffffu, (keepm >> i) & 1u);
+        keep_before += __popc(bal & lt);
+        keep_total += __popc(bal);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if ((keepm >> i) & 1u) {
+            const uint32_t r = pos + keep_before + __popc(keepm & ((1u << i) - 1u));
+            if (r < static_cast<uint32_t>(m)) kidx[r] = static_cast<Idx>(jb + i);
+        }
+    }
+    pos += keep_total;
+    ties += eq_total;
+}
+
 // Selection of one unit by the math threads, from its final scores (padded
 // row, 16-byte groups) and their z-bin histogram.
 //   1. the z-bin b0 of the B-th key (a descending scan of the histogram);
@@ -335,25 +444,14 @@ __host__ __device__ __forceinline__ int64_t pipe_pad(int64_t n) { return (n + 31
 //      threshold key T and the first (B - above) keys equal to T.
 // Loads keep 4 groups of 4 keys in flight per lane.
 template <typename Fin, typename Idx>
-__device__ __noinline__ void select_unit(const Fin fin, int n, int64_t B, int m, uint32_t* hist,
+__device__ __forceinline__ void select_unit(const Fin fin, int n, int64_t B, int m, uint32_t* hist,
                                          int2* cand, PipeMisc* ms, Idx* kidx) {
     using S = PipeShape<float>;
-    constexpr int kLook = 4;  // 128-key blocks whose loads are in flight at once
+    // 128-key blocks whose loads are in flight at once.
+    constexpr int kLook = 4;
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const uint32_t lt = (1u << lane) - 1u;
-    if (warp == 0) {
-        uint32_t bin, above;
-        warp_find_bin(hist, kZBins, static_cast<uint32_t>(B), bin, above);
-        if (lane == 0) {
-            ms->zb0 = bin;
-            ms->ncand = 0;
-            ms->st.prefix = 0;
-            ms->st.k = static_cast<uint32_t>(B) - above;  // to take from bin b0
-            ms->st.gt = above;
-            ms->st.keep_all = 0;
-        }
-    }
+    if (warp == 0) threshold_bin(hist, B, ms);
     if (tid < S::kMathWarps * 2) ms->wadd[tid >> 1][tid & 1] = 0u;
     math_sync();
     const uint32_t b0 = ms->zb0;
@@ -394,24 +492,10 @@ __device__ __noinline__ void select_unit(const Fin fin, int n, int64_t B, int m,
     math_sync();
     const int nc = ms->ncand;
     const bool listed = nc <= kPipeCand;
-    if (nc <= S::kMath) {
-        const uint32_t k0 = ms->st.k;
-        math_sync();  // k0 read before st changes
-        const int2 me = tid < nc ? cand[tid] : make_int2(0, 0);
-        const uint32_t mk = static_cast<uint32_t>(me.x);
-        uint32_t above = 0, rank = 0;
-        for (int i = 0; i < nc; ++i) {
-            const int2 e = cand[i];
-            const uint32_t ek = static_cast<uint32_t>(e.x);
-            above += ek > mk;
-            rank += (ek > mk) || (ek == mk && e.y < me.y);
-        }
-        if (tid < nc && rank == k0 - 1) {
-            ms->st.prefix = mk;
-            ms->st.k = k0 - above;  // ties of the threshold key that are kept
-        }
-        math_sync();
+    if (listed) {
+        rank_listed(nc, hist, cand, ms);
     } else {
+        // Too many keys share b0 to list: the same radix in place over them.
         for (int p = 0; p < 3; ++p) {
             const int nb = 1 << pass_bits(p);
             for (int b = tid; b < nb; b += S::kMath) hist[b] = 0;
@@ -419,22 +503,14 @@ __device__ __noinline__ void select_unit(const Fin fin, int n, int64_t B, int m,
             const uint32_t prefix = ms->st.prefix;
             const int shift = pass_shift(p);
             const int hi_shift = shift + pass_bits(p);
-            if (listed) {
-                for (int i = tid; i < nc; i += S::kMath) {
-                    const uint32_t key = static_cast<uint32_t>(cand[i].x);
-                    if (p == 0 || (key >> hi_shift) == prefix)
-                        atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
-                }
-            } else {
-                for (int g = tid; 4 * g < n; g += S::kMath) {
-                    const float4 v = fin.get4(4 * g);
+            for (int g = tid; 4 * g < n; g += S::kMath) {
+                const float4 v = fin.get4(4 * g);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float f = f4at(v, i);
-                        const uint32_t key = ordered_key(f);
-                        if (4 * g + i < n && zbin(f) == b0 && (p == 0 || (key >> hi_shift) == prefix))
-                            atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
-                    }
+                for (int i = 0; i < 4; ++i) {
+                    const float f = f4at(v, i);
+                    const uint32_t key = ordered_key(f);
+                    if (4 * g + i < n && zbin(f) == b0 && (p == 0 || (key >> hi_shift) == prefix))
+                        atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
                 }
             }
             math_sync();
@@ -511,45 +587,7 @@ __device__ __noinline__ void select_unit(const Fin fin, int n, int64_t B, int m,
 #pragma unroll
         for (int q = 0; q < kLook; ++q) {
             if (bb + q >= blk1) break;
-            const int jb = ((bb + q) << 7) + 4 * lane;  // this lane's first key
-            uint32_t gtm = 0, eqm = 0;                   // 4-bit masks of this lane's keys
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint32_t key = ordered_key(f4at(v[q], i));
-                const bool valid = jb + i < n;
-                gtm |= (valid && key > Tk) ? (1u << i) : 0u;
-                eqm |= (valid && key == Tk) ? (1u << i) : 0u;
-            }
-            // Keys are ordered lane-major: ties before this lane's keys.
-            uint32_t eq_before = 0, eq_total = 0;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint32_t bal = __ballot_sync(0xffffffffu, (eqm >> i) & 1u);
-                eq_before += __popc(bal & lt);
-                eq_total += __popc(bal);
-            }
-            uint32_t keepm = gtm;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint32_t my_tie = ties + eq_before + __popc(eqm & ((1u << i) - 1u));
-                if (((eqm >> i) & 1u) && my_tie < kt) keepm |= 1u << i;
-            }
-            uint32_t keep_before = 0, keep_total = 0;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint32_t bal = __ballot_sync(0xffffffffu, (keepm >> i) & 1u);
-                keep_before += __popc(bal & lt);
-                keep_total += __popc(bal);
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                if ((keepm >> i) & 1u) {
-                    const uint32_t r = pos + keep_before + __popc(keepm & ((1u << i) - 1u));
-                    if (r < static_cast<uint32_t>(m)) kidx[r] = static_cast<Idx>(jb + i);
-                }
-            }
-            pos += keep_total;
-            ties += eq_total;
+            write_block(v[q], ((bb + q) << 7) + 4 * lane, n, Tk, kt, m, pos, ties, kidx);
         }
     }
 }
@@ -559,7 +597,7 @@ __device__ __noinline__ void select_unit(const Fin fin, int n, int64_t B, int m,
 // into final_out, when given), the z-bin histogram into hist (zeroed by the
 // caller), NaN flagged.  Groups of 4 keys move as 16-byte accesses.
 template <int G, typename Fin>
-__device__ __noinline__ void zmax_unit(const float* raw, int64_t ldr, int n, const PipeMisc* ms,
+__device__ __forceinline__ void zmax_unit(const float* raw, int64_t ldr, int n, const PipeMisc* ms,
                                        const Fin fin, float* final_out, uint32_t* hist,
                                        uint32_t* flag) {
     using S = PipeShape<float>;
@@ -571,6 +609,7 @@ __device__ __noinline__ void zmax_unit(const float* raw, int64_t ldr, int n, con
         inv[h] = ms->mom[h].y;
     }
     bool nonfinite = false;
+    // Groups of 4 keys in flight per thread: 16-byte loads of every head.
     constexpr int kU = G <= 4 ? 2 : 1;
     const int n4 = (n + 3) >> 2;
     for (int g0 = tid; g0 < n4; g0 += S::kMath * kU) {
@@ -629,19 +668,21 @@ __device__ __forceinline__ void pipe_trace(const PipeArgs& a, int64_t u, int p, 
 // ---------------------------------------------------------------------------
 // The gather engine (kEngWarps warps).
 //
-// Pieces: destination rows [kGRows q, kGRows (q + 1)) of a unit, of K and of
-// V together in one buffer; engine warp e takes pieces e, e + kEngWarps, ...
-// of every unit, through its own share of the buffers.  Loading a piece:
-// lane l takes destination row kGRows q + l; the math warps have marked the
-// rows that start a run of consecutive source rows (the piece's run-start
-// mask), and each starting lane issues one bulk load of its run for K and
-// one for V, all completing on the buffer's barrier.  Up to (buffers - kGGap)
-// pieces load while older ones are stored with one bulk store for K and one
-// for V, so loads, stores and the next unit's loads overlap.
+// Pieces: destination rows [kGRows q, kGRows (q + 1)) of a unit (32 bf16 or
+// 16 float32 rows), of K and of V together in one 16 KB buffer; engine warp
+// e takes pieces e, e + kEngWarps, ... of every unit, through its own share
+// of the buffers.  The math warps have marked the rows of each piece that
+// start a run of consecutive source rows (the piece's run-start mask).  Loading a piece: lane o takes bulk load o, the K (o even) or V (o
+// odd) rows of run o / 2, so one instruction issues up to 32 loads, all
+// completing on the buffer's barrier (a bulk-copy instruction costs its warp
+// a few hundred cycles whatever its size, its lanes little more).
+// Up to (buffers - kGGap) pieces load while older ones are stored, K by lane
+// 0 and V by lane 1 of one instruction, so loads, stores and the next unit's
+// loads overlap.
 // ---------------------------------------------------------------------------
 template <typename T, typename Idx>
 __device__ void pipe_engine(const PipeArgs& a, int eng, uint8_t* gbuf, int gs, const Idx* kidx_base,
-                            size_t kidx_stride, const uint32_t* smask_base, size_t smask_stride,
+                            size_t kidx_stride, const uint64_t* smask_base, size_t smask_stride,
                             uint64_t* gfull, uint64_t* kready, uint64_t* kfree, PipeMisc* ms) {
     using S = PipeShape<T>;
     const int lane = threadIdx.x & 31;
@@ -657,18 +698,18 @@ __device__ void pipe_engine(const PipeArgs& a, int eng, uint8_t* gbuf, int gs, c
     int64_t u = 0;
     int m = 0, P = 0, q = 0;
     const Idx* kx = nullptr;
-    const uint32_t* smask = nullptr;
+    const uint64_t* smask = nullptr;
 
     // Store the oldest loaded piece.  Returns false if its wait gave up.
     auto store_one = [&]() -> bool {
         const int sl = stored % gs;
         if (!warp_wait(&gfull[sl], (stored / gs) & 1, a.flag)) return false;
-        if (lane == 0) {
+        if (lane < (has_v ? 2 : 1)) {
             const int g = eng * gs + sl;
             const int64_t off = ms->gdst[g];
             const uint32_t bytes = ms->gdst_rows[g] * S::kRowBytes;
-            bulk_store_hint(kd + off, gbuf + sl * S::kGSlotBytes, bytes, pol);
-            if (has_v) bulk_store_hint(vd + off, gbuf + sl * S::kGSlotBytes + S::kGHalf, bytes, pol);
+            bulk_store_hint((lane ? vd : kd) + off, gbuf + sl * S::kGSlotBytes + lane * S::kGHalf, bytes,
+                            pol);
             bulk_commit();
         }
         __syncwarp();
@@ -719,15 +760,22 @@ __device__ void pipe_engine(const PipeArgs& a, int eng, uint8_t* gbuf, int gs, c
             // be done reading it: stored >= issued - ahead + 1, so at least
             // gs - ahead = kGGap stores were committed after it, and it is
             // complete once no more than the kGGap newest are pending.
-            if (issued >= static_cast<uint32_t>(gs) && lane == 0) bulk_wait_read<S::kGGap>();
+            if (issued >= static_cast<uint32_t>(gs) && lane < (has_v ? 2 : 1))
+                bulk_wait_read<S::kGGap>();  // lanes 0 and 1 each track their own stores
             __syncwarp();
             const int r0 = q * S::kGRows;
             const int rows = min(S::kGRows, m - r0);
-            const uint32_t starts = smask[q];
-            const int32_t j = lane < rows ? static_cast<int32_t>(kx[r0 + lane]) : 0;
-            const bool start = (starts >> lane) & 1u;
-            const uint32_t later = starts & ~((2u << lane) - 1u);  // run starts after this lane
-            const int end = later ? __ffs(later) - 1 : rows;
+            // Only the piece's own rows, and its first row always starts a
+            // run: the runs then partition the piece exactly, whatever the mask.
+            const uint64_t row_mask = rows >= 64 ? ~0ull : ((1ull << rows) - 1ull);
+            const uint64_t starts = (smask[q] & row_mask) | 1ull;
+            const int n_runs = __popcll(starts);
+            int32_t* rs = ms->runst[eng];
+#pragma unroll
+            for (int hb = 0; hb < 2; ++hb) {
+                const int bit = lane + 32 * hb;
+                if ((starts >> bit) & 1ull) rs[__popcll(starts & ((1ull << bit) - 1ull))] = bit;
+            }
             uint64_t* landed = &gfull[sl];
             if (lane == 0) {
                 mbar_arrive_expect_tx(landed, static_cast<uint32_t>(rows * S::kRowBytes * (has_v ? 2 : 1)));
@@ -735,21 +783,30 @@ __device__ void pipe_engine(const PipeArgs& a, int eng, uint8_t* gbuf, int gs, c
                 ms->gdst_rows[eng * gs + sl] = static_cast<uint32_t>(rows);
             }
             __syncwarp();
-            if (start) {
-                // A run that would leave the source cache (cannot happen) lands
-                // copies of row 0 instead, so that the barrier completes.
-                const bool ok = j >= 0 && j + (end - lane) <= a.cap;
-                if (!ok) raise_flag(a.flag, TRI_FLAG_INDEX_RANGE);
-                uint8_t* buf = gbuf + sl * S::kGSlotBytes + lane * S::kRowBytes;
-                for (int l = 0; l < (ok ? 1 : end - lane); ++l) {
-                    const int64_t src_row = u * a.cap + (ok ? j : 0);
-                    const uint32_t len = static_cast<uint32_t>((ok ? end - lane : 1) * S::kRowBytes);
-                    bulk_load_hint(buf + l * S::kRowBytes, ks + src_row * S::kRowBytes, len, landed, pol);
-                    if (has_v)
-                        bulk_load_hint(buf + S::kGHalf + l * S::kRowBytes, vs + src_row * S::kRowBytes,
-                                       len, landed, pol);
+            uint8_t* buf = gbuf + sl * S::kGSlotBytes;
+            const int n_ops = n_runs * (has_v ? 2 : 1);
+            for (int o = lane; o - lane < n_ops; o += 32) {
+                if (o < n_ops) {
+                    const int r = has_v ? (o >> 1) : o;
+                    const int t = has_v ? (o & 1) : 0;
+                    const int l0 = rs[r];
+                    const int l1 = r + 1 < n_runs ? rs[r + 1] : rows;
+                    const int32_t j = static_cast<int32_t>(kx[r0 + l0]);
+                    // A run that would leave the source cache (cannot happen)
+                    // lands copies of row 0 instead, so that the barrier completes.
+                    const bool ok = j >= 0 && j + (l1 - l0) <= a.cap;
+                    if (!ok) raise_flag(a.flag, TRI_FLAG_INDEX_RANGE);
+                    const char* src = (t ? vs : ks) + (u * a.cap + (ok ? j : 0)) * S::kRowBytes;
+                    uint8_t* dst = buf + t * S::kGHalf + l0 * S::kRowBytes;
+                    if (ok) {
+                        bulk_load_hint(dst, src, static_cast<uint32_t>((l1 - l0) * S::kRowBytes), landed, pol);
+                    } else {
+                        for (int l = 0; l < l1 - l0; ++l)
+                            bulk_load_hint(dst + l * S::kRowBytes, src, S::kRowBytes, landed, pol);
+                    }
                 }
             }
+            __syncwarp();  // the run starts are read before the next piece rewrites them
             ++issued;
             q += S::kEngWarps;
             if (q >= P) {
@@ -772,7 +829,7 @@ __device__ void pipe_engine(const PipeArgs& a, int eng, uint8_t* gbuf, int gs, c
         if (done) break;
     }
     if (failed) ms->abort = 1;
-    if (lane == 0) bulk_wait_all();
+    if (lane < 2) bulk_wait_all();
     if (failed) {
         // Loads still in flight into the buffers: give them time to land.
         const uint64_t t0 = globaltimer_ns();
@@ -804,12 +861,12 @@ prune_pipe_kernel(const __grid_constant__ CUtensorMap kmap, PipeArgs a) {
     uint32_t* hist = reinterpret_cast<uint32_t*>(base + L.hist);  // aliases the rings
     int2* cand = reinterpret_cast<int2*>(base + L.cand);          // aliases the rings
     Idx* kidx = reinterpret_cast<Idx*>(base + L.kidx);
-    uint32_t* smask = reinterpret_cast<uint32_t*>(base + L.smask);
+    uint64_t* smask = reinterpret_cast<uint64_t*>(base + L.smask);
     const int64_t m_max = a.B < a.cap ? a.B : a.cap;
     const size_t kidx_stride =
         ((static_cast<size_t>(m_max) * sizeof(Idx) + 15) & ~size_t(15)) / sizeof(Idx);
     const size_t smask_stride =
-        ((static_cast<size_t>((m_max + S::kGRows - 1) / S::kGRows) * 4 + 15) & ~size_t(15)) / 4;
+        ((static_cast<size_t>((m_max + S::kGRows - 1) / S::kGRows) * 8 + 15) & ~size_t(15)) / 8;
     uint64_t* full = reinterpret_cast<uint64_t*>(base + L.bars);  // [warp][kQ]
     uint64_t* gfull = full + S::kMathWarps * PipeShape<T, true>::kQ * 2;  // [gslots]
     uint64_t* kready = gfull + S::kMaxGSlots;                       // [kHand]
@@ -970,16 +1027,27 @@ prune_pipe_kernel(const __grid_constant__ CUtensorMap kmap, PipeArgs a) {
         math_sync();
         if (ms->stop) return false;
         Idx* kx = kidx + slot * kidx_stride;
-        uint32_t* sm = smask + slot * smask_stride;
+        uint64_t* sm = smask + slot * smask_stride;
         fill(kx);
         math_sync();
         const int P = (m + S::kGRows - 1) / S::kGRows;
         for (int q = warp; q < P; q += S::kMathWarps) {
-            const int r = q * S::kGRows + lane;
-            const bool valid = lane < S::kGRows && r < m;
-            const int32_t j = valid ? static_cast<int32_t>(kx[r]) : 0;
-            const int32_t jp = __shfl_up_sync(0xffffffffu, j, 1);
-            const uint32_t st = __ballot_sync(0xffffffffu, valid && (lane == 0 || j != jp + 1));
+            // Rows q kGRows + lane (and + 32): a row starts a run unless its
+            // source row follows that of the row before it in the piece.
+            const int ra = q * S::kGRows + lane;
+            const bool va = lane < S::kGRows && ra < m;
+            const int32_t ja = va ? static_cast<int32_t>(kx[ra]) : 0;
+            const int32_t pa = __shfl_up_sync(0xffffffffu, ja, 1);
+            uint64_t st = __ballot_sync(0xffffffffu, va && (lane == 0 || ja != pa + 1));
+            if (S::kGRows > 32) {
+                const int rb = ra + 32;
+                const bool vb = rb < m;
+                const int32_t jb = vb ? static_cast<int32_t>(kx[rb]) : 0;
+                int32_t pb = __shfl_up_sync(0xffffffffu, jb, 1);
+                const int32_t last_a = __shfl_sync(0xffffffffu, ja, 31);
+                if (lane == 0) pb = last_a;
+                st |= static_cast<uint64_t>(__ballot_sync(0xffffffffu, vb && jb != pb + 1)) << 32;
+            }
             if (lane == 0) sm[q] = st;
         }
         math_sync();
@@ -1069,8 +1137,6 @@ prune_pipe_kernel(const __grid_constant__ CUtensorMap kmap, PipeArgs a) {
                 zmax_unit<G>(raw, capP, n, ms, FinShared{fin_s},
                              a.final_out ? a.final_out + u * a.cap : nullptr, hist, a.flag);
                 math_sync();
-                // The unit's per-head scores are dead: drop them from L2 unwritten.
-                discard_range(raw, static_cast<int64_t>(G) * capP * 4, tid, S::kMath);
                 pipe_trace(a, u, 2, warp);
                 // This warp's first tile of the next unit into L2.
                 const int64_t un = u + gridDim.x;
@@ -1187,24 +1253,29 @@ prune_pipe_kernel(const __grid_constant__ CUtensorMap kmap, PipeArgs a) {
             if (!ms->last) continue;
             __threadfence();
             // This CTA completed unit u: moments in chunk order, final
-            // scores, selection, hand-off.
-            if (tid < G) {
-                double s1 = 0.0, s2 = 0.0;
+            // scores, selection, hand-off.  The chunks' partials are loaded
+            // at once (into the idle rings) and summed in chunk order.
+            {
+                double* pp = reinterpret_cast<double*>(ring + kPartOff);
                 const double* part = a.partial + u * cpu * G * 2;
-                for (int cc = 0; cc < chunks; ++cc) {
-                    s1 += __ldcg(part + (cc * G + tid) * 2);
-                    s2 += __ldcg(part + (cc * G + tid) * 2 + 1);
+                for (int e = tid; e < chunks * G * 2; e += S::kMath) pp[e] = __ldcg(part + e);
+                math_sync();
+                if (tid < G) {
+                    double s1 = 0.0, s2 = 0.0;
+                    for (int cc = 0; cc < chunks; ++cc) {
+                        s1 += pp[(cc * G + tid) * 2];
+                        s2 += pp[(cc * G + tid) * 2 + 1];
+                    }
+                    ms->mom[tid] = moments_from_sums(s1, s2, n);
                 }
-                ms->mom[tid] = moments_from_sums(s1, s2, n);
             }
             if (tid == 0) a.counters[u] = 0u;
             for (int b = tid; b < kZBins; b += S::kMath) hist[b] = 0;
             math_sync();
             float* fin_g = a.fin_scratch + static_cast<int64_t>(blockIdx.x) * capP;
-            zmax_unit<G>(raw, capP, n, ms, FinGlobal{fin_g},
-                         a.final_out ? a.final_out + u * a.cap : nullptr, hist, a.flag);
+            float* fo = a.final_out ? a.final_out + u * a.cap : nullptr;
+            zmax_unit<G>(raw, capP, n, ms, FinGlobal{fin_g}, fo, hist, a.flag);
             math_sync();
-            discard_range(raw, static_cast<int64_t>(G) * capP * 4, tid, S::kMath);
             const bool ok = handoff(u, m, [&](Idx* kx) {
                 select_unit(FinGlobal{fin_g}, n, B, m, hist, cand, ms, kx);
             });
@@ -1212,7 +1283,6 @@ prune_pipe_kernel(const __grid_constant__ CUtensorMap kmap, PipeArgs a) {
                 failed = true;
                 break;
             }
-            discard_range(fin_g, static_cast<int64_t>(n) * 4, tid, S::kMath);
         }
     }
     if (failed) ms->abort = 1;
@@ -1245,6 +1315,14 @@ int pipe_chunk_keys(tri_dtype dt) { return pipe_tile_keys(dt) * kChunkTiles; }
 
 bool pipe_small_fits(tri_dtype dt, int64_t cap) {
     return dt == TRI_BF16 ? pipe_small_unit<__nv_bfloat16>(cap) : pipe_small_unit<float>(cap);
+}
+
+bool pipe_big_fits(int64_t cap) {
+    // The chunks' moment partials of one unit fit the rings after the
+    // histogram and candidates.
+    using S = PipeShape<float, true>;
+    const int64_t chunks = (cap + kChunkTiles * S::kTile - 1) / (kChunkTiles * S::kTile);
+    return kPartOff + chunks * kMaxG * 16 <= static_cast<int64_t>(S::kMathWarps) * S::kQ * S::kSlotBytes;
 }
 
 int pipe_slice_bytes(bool big) { return big ? PipeShape<float, true>::kSliceBytes

@@ -23,6 +23,7 @@
 #include "tri_internal.cuh"
 #include "tri_launch.h"
 #include "score_core.cuh"
+#include "select_core.cuh"
 
 // How many key tiles ahead of its shared-memory ring the score kernel asks
 // L2 to fetch (0: no prefetch).
@@ -354,7 +355,7 @@ template <int G>
 __global__ void __launch_bounds__(256)
 zmax_kernel(const float* __restrict__ raw, int64_t cap, const int32_t* __restrict__ n_valid,
             const float2* __restrict__ mom, float* __restrict__ fin, uint32_t* __restrict__ hist0,
-            uint32_t* flag) {
+            int zbins, uint32_t* flag) {
     __shared__ uint32_t hist[kHistBins0];
     const int64_t u = blockIdx.y;
     const int n = clamp_nvalid(n_valid, u, cap, nullptr);
@@ -391,7 +392,7 @@ zmax_kernel(const float* __restrict__ raw, int64_t cap, const int32_t* __restric
             }
             fin[u * cap + j] = best;
             if (best != best) nonfinite = true;
-            if (hist0) atomicAdd(&hist[ordered_key(best) >> kShift0], 1u);
+            if (hist0) atomicAdd(&hist[zbins ? zbin(best) : (ordered_key(best) >> kShift0)], 1u);
         }
     }
     if (nonfinite) raise_flag(flag, TRI_FLAG_NONFINITE);
@@ -459,11 +460,11 @@ cudaError_t launch_score(tri_dtype dt, int G, const CUtensorMap& map, const Scor
 
 cudaError_t launch_zmax(int G, const float* raw, int64_t n_units, int64_t cap,
                         const int32_t* n_valid, const float2* mom, float* fin, uint32_t* hist0,
-                        uint32_t* flag, cudaStream_t s) {
+                        int zbins, uint32_t* flag, cudaStream_t s) {
     dim3 grid(static_cast<unsigned>((cap + kZChunk - 1) / kZChunk), static_cast<unsigned>(n_units));
     switch (G) {
 #define TRI_ZCASE(g) \
-    case g: zmax_kernel<g><<<grid, 256, 0, s>>>(raw, cap, n_valid, mom, fin, hist0, flag); break;
+    case g: zmax_kernel<g><<<grid, 256, 0, s>>>(raw, cap, n_valid, mom, fin, hist0, zbins, flag); break;
         TRI_ZCASE(1) TRI_ZCASE(2) TRI_ZCASE(3) TRI_ZCASE(4)
         TRI_ZCASE(5) TRI_ZCASE(6) TRI_ZCASE(7) TRI_ZCASE(8)
 #undef TRI_ZCASE

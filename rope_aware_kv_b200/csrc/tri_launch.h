@@ -181,9 +181,20 @@ cudaError_t launch_fold(const float* stats, const int64_t* p_cur, int64_t n_seq,
                         cudaStream_t s);
 cudaError_t launch_score(tri_dtype dt, int G, const CUtensorMap& map, const ScoreArgs& a,
                          int n_sm, cudaStream_t s);
+// hist0 (nullable): per-unit histogram of the final scores, of their z-bins
+// (zbins != 0) or of their first radix digit.
 cudaError_t launch_zmax(int G, const float* raw, int64_t n_units, int64_t cap,
                         const int32_t* n_valid, const float2* mom, float* fin, uint32_t* hist0,
-                        uint32_t* flag, cudaStream_t s);
+                        int zbins, uint32_t* flag, cudaStream_t s);
+
+// zselect.cu: top-B by z-bins on the split path (zhist from launch_zmax with
+// zbins; counts [U][chunks] and cand [U][kCandMax] scratch, cand_count [U]
+// zero on entry, state [U] of zsel_state_bytes()).
+size_t zsel_state_bytes();
+cudaError_t launch_zselect(const float* fin, int64_t n_units, int64_t cap, const int32_t* n_valid,
+                           int64_t B, const uint32_t* zhist, uint2* counts, int2* cand,
+                           uint32_t* cand_count, void* state, int32_t* kept, int32_t* n_kept,
+                           cudaStream_t s);
 
 // select.cu
 cudaError_t launch_radix_pass(const float* fin, int64_t n_units, int64_t cap,
@@ -224,6 +235,7 @@ size_t pipe_smem_bytes(tri_dtype dt, int G, int64_t cap, int64_t B, bool big, in
 int pipe_min_gslots();
 int pipe_max_gslots();
 bool pipe_small_fits(tri_dtype dt, int64_t cap);
+bool pipe_big_fits(int64_t cap);
 int pipe_slice_bytes(bool big);
 int pipe_engine_warps();
 int pipe_tile_keys(tri_dtype dt);

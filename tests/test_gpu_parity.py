@@ -381,7 +381,7 @@ def test_prune_parity_config(name, sample):
 
 def test_prune_default_paths():
     """The path tri_prune takes for each workload configuration."""
-    want = {"c1": tri.PATH_COOP, "c2": tri.PATH_COOP, "c3": tri.PATH_PIPE, "c4": tri.PATH_PIPE,
+    want = {"c1": tri.PATH_COOP, "c2": tri.PATH_COOP, "c3": tri.PATH_PIPE, "c4": tri.PATH_SPLIT,
             "c5": tri.PATH_PIPE}
     for name, path in want.items():
         s = synth.SPECS[name]

@@ -21,6 +21,10 @@ Every function follows the pages step by step:
   (jaedaily.cn KV-compression tutorial, eviction step).
 * ``prune`` -- all of the above plus the bit-exact gather, over many units.
 
+Method variants (``variant`` bits, protection and per-layer budgets of
+``prune``; ``calibrate`` with positions and pairing) follow the pages'
+ablations and alternatives, see ``tri_oracle.c``.
+
 Parity status: every function is pinned by the ``-m "not gpu"`` tests in
 ``tests/test_oracle_pins.py`` against closed forms, brute force and
 invariants; absolute score values at real-model scale are unpinned because the
@@ -45,6 +49,12 @@ BF16 = 1
 # RoPE rotation and the offset-averaged score S~).
 THETA = 10000.0
 OFFSETS = tuple(1 << i for i in range(17))
+
+# Variant bits (tri_oracle.c: ORA_VAR_*).
+VAR_NO_TRIG = 1
+VAR_NO_R = 2
+VAR_MAX_OFFSET = 4
+VAR_HALF_SPLIT = 8
 
 _lib = None
 
@@ -73,14 +83,18 @@ def _bind(lib):
     d = ctypes.c_double
     lib.oracle_calibrate.argtypes = [P, i32, i64, i64, i32, P]
     lib.oracle_calibrate.restype = i32
-    lib.oracle_score.argtypes = [P, i32, i64, i32, P, i64, P, i32, d, P, i32, P]
+    lib.oracle_calibrate_ex.argtypes = [P, i32, i64, i64, i32, P, d, i32, P]
+    lib.oracle_calibrate_ex.restype = i32
+    lib.oracle_select_protected.argtypes = [P, i64, i64, i64, i64, P, P]
+    lib.oracle_select_protected.restype = i64
+    lib.oracle_score.argtypes = [P, i32, i64, i32, P, i64, P, i32, d, P, i32, i32, P]
     lib.oracle_score.restype = i32
     lib.oracle_znorm_max.argtypes = [P, i32, i64, P, P, P, P]
     lib.oracle_znorm_max.restype = i32
     lib.oracle_select.argtypes = [P, i64, i64, P, P]
     lib.oracle_select.restype = i64
     lib.oracle_prune.argtypes = [P, P, P, i32, i64, i64, i64, i32, i64, i32, P, P, P, d, P,
-                                 i32, i64, P, P, P, P, P, P, P, P, i64, P, i64]
+                                 i32, i64, P, P, P, P, P, P, P, P, i64, P, i64, i32, i64, i64, P]
     lib.oracle_prune.restype = i32
     lib.oracle_threads.argtypes = []
     lib.oracle_threads.restype = i32
@@ -135,19 +149,27 @@ def set_threads(n: int) -> None:
     _load().oracle_set_threads(int(n))
 
 
-def calibrate(q: np.ndarray) -> np.ndarray:
-    """q: [H, n_tok, d] pre-RoPE queries -> stats [H, d/2, 4] (re, im, mean|q_f|, R_f)."""
+def calibrate(q: np.ndarray, pos=None, theta: float = THETA, half: bool = False) -> np.ndarray:
+    """q: [H, n_tok, d] queries -> stats [H, d/2, 4] (re, im, mean|q_f|, R_f).
+
+    Pre-RoPE queries by default; with ``pos`` ([n_tok] positions) the queries
+    are post-RoPE and are rotated back first.  ``half``: half-split bands."""
     q, dt = _elem(q)
     H, n, d = q.shape
     out = np.empty((H, d // 2, 4), np.float64)
-    rc = _load().oracle_calibrate(_ptr(q), dt, H, n, d, _ptr(out))
+    if pos is None and not half:
+        rc = _load().oracle_calibrate(_ptr(q), dt, H, n, d, _ptr(out))
+    else:
+        pp = None if pos is None else np.ascontiguousarray(np.asarray(pos, np.int32))
+        rc = _load().oracle_calibrate_ex(_ptr(q), dt, H, n, d, _ptr(pp), float(theta),
+                                         1 if half else 0, _ptr(out))
     if rc:
         raise ValueError(f"oracle_calibrate failed ({rc})")
     return out
 
 
 def score(k: np.ndarray, pos: np.ndarray, p_cur: int, stats: np.ndarray,
-          theta: float = THETA, offsets=OFFSETS) -> np.ndarray:
+          theta: float = THETA, offsets=OFFSETS, variant: int = 0) -> np.ndarray:
     """Per-head S~ for one unit: k [n, d] post-RoPE, pos [n], stats [G, d/2, 4] -> [G, n]."""
     k, dt = _elem(k)
     n, d = k.shape
@@ -157,7 +179,7 @@ def score(k: np.ndarray, pos: np.ndarray, p_cur: int, stats: np.ndarray,
     off = np.ascontiguousarray(np.asarray(offsets, np.int64))
     out = np.empty((G, n), np.float64)
     rc = _load().oracle_score(_ptr(k), dt, n, d, _ptr(pos), int(p_cur), _ptr(st), G,
-                              float(theta), _ptr(off), len(off), _ptr(out))
+                              float(theta), _ptr(off), len(off), int(variant), _ptr(out))
     if rc:
         raise ValueError(f"oracle_score failed ({rc})")
     return out
@@ -189,8 +211,23 @@ def select(final: np.ndarray, B: int):
     return kept[:m].copy(), thr.value
 
 
+def select_protected(final: np.ndarray, B: int, n_sink: int, n_recent: int):
+    """Top-B with the first n_sink and last n_recent keys always kept ->
+    (kept ascending, score of the last unprotected key kept)."""
+    fin = np.ascontiguousarray(final, np.float64)
+    n = fin.shape[0]
+    kept = np.empty((max(min(B, n), 1),), np.int32)
+    thr = ctypes.c_double(0.0)
+    m = _load().oracle_select_protected(_ptr(fin), n, int(B), int(n_sink), int(n_recent),
+                                        _ptr(kept), ctypes.byref(thr))
+    if m < 0:
+        raise ValueError("oracle_select_protected failed")
+    return kept[:m].copy(), thr.value
+
+
 def prune(k, v, pos, n_seq, n_layers, n_kvheads, G, stats, p_cur, B, n_valid=None,
-          theta=THETA, offsets=OFFSETS, units=None, want_raw=True, want_gather=True):
+          theta=THETA, offsets=OFFSETS, units=None, want_raw=True, want_gather=True,
+          variant=0, n_sink=0, n_recent=0, layer_budget=None):
     """Whole prune step on [U, cap, d] caches (see tri_oracle.c: oracle_prune).
 
     stats: [n_layers, n_kvheads*G, d/2, 4] float64.  Returns a dict with
@@ -211,6 +248,7 @@ def prune(k, v, pos, n_seq, n_layers, n_kvheads, G, stats, p_cur, B, n_valid=Non
     nv = None if n_valid is None else np.ascontiguousarray(np.asarray(n_valid, np.int32))
     off = np.ascontiguousarray(np.asarray(offsets, np.int64))
     ul = None if units is None else np.ascontiguousarray(np.asarray(units, np.int64))
+    lb = None if layer_budget is None else np.ascontiguousarray(np.asarray(layer_budget, np.int64))
     raw = np.full((U, G, cap), np.nan) if want_raw else None
     fin = np.full((U, cap), np.nan)
     kept = np.full((U, max(B, 1)), -1, np.int32)
@@ -225,7 +263,8 @@ def prune(k, v, pos, n_seq, n_layers, n_kvheads, G, stats, p_cur, B, n_valid=Non
         _ptr(k), _ptr(v2), _ptr(pos), dt, n_seq, n_layers, n_kvheads, G, cap, d, _ptr(nv),
         _ptr(pc), _ptr(st), float(theta), _ptr(off), len(off), int(B), _ptr(raw), _ptr(fin),
         _ptr(kept), _ptr(nk), _ptr(thr), _ptr(kd), _ptr(vd), _ptr(pd), B if want_gather else 0,
-        _ptr(ul), 0 if ul is None else len(ul))
+        _ptr(ul), 0 if ul is None else len(ul), int(variant), int(n_sink), int(n_recent),
+        _ptr(lb))
     if rc:
         raise ValueError(f"oracle_prune failed ({rc})")
     out = dict(final=fin, kept=kept[:, :B], n_kept=nk, thr=thr)

@@ -44,6 +44,24 @@
  *   - ties at the B-th score go to the lowest index;
  *   - R_f = 1 when E[|q_f|] = 0 (the norm weight (1-R_f)E|q_f| is 0 anyway).
  *
+ * Method variants (each off by default; the pages name them as ablations or
+ * alternatives, the readings are listed in the design notes):
+ *   ORA_VAR_NO_TRIG     S_trig left out, the score is S_norm alone (shibing624
+ *                       paper reading, ablation section: without S_trig);
+ *   ORA_VAR_NO_R        the norm weight without the concentration factor,
+ *                       E[|q_f|] instead of (1 - R_f) E[|q_f|] (same section:
+ *                       without the R weighting);
+ *   ORA_VAR_MAX_OFFSET  the maximum over the offsets of S_trig + S_norm
+ *                       instead of their mean (same page, future-offset
+ *                       paragraph: the maximum is the key's score);
+ *   ORA_VAR_HALF_SPLIT  band f pairs components (x_f, x_{f+d/2}) instead of
+ *                       (x_2f, x_2f+1) (the rotate-half RoPE layout);
+ *   protection          the n_sink first and n_recent last keys of a unit are
+ *                       always kept (jaedaily.cn tutorial, streaming section:
+ *                       the most recent tokens are protected from eviction);
+ *   layer budgets       a budget per layer instead of one B (same tutorial,
+ *                       budget paragraph: pyramid-shaped budgets per layer).
+ *
  * Element types: 0 = float32, 1 = bfloat16 (upper half of a float32).  Both
  * decode exactly to double.
  */
@@ -58,6 +76,11 @@
 #define ORA_F32 0
 #define ORA_BF16 1
 
+#define ORA_VAR_NO_TRIG 1
+#define ORA_VAR_NO_R 2
+#define ORA_VAR_MAX_OFFSET 4
+#define ORA_VAR_HALF_SPLIT 8
+
 #define ORA_OK 0
 #define ORA_EINVAL 1
 #define ORA_ENOMEM 2
@@ -70,6 +93,20 @@ static double ora_decode(const void* base, int dtype, int64_t i) {
     float f;
     memcpy(&f, &bits, sizeof f);
     return (double)f;
+}
+
+/* Components (x, y) of band f of the d-vector starting at element `row`:
+ * interleaved (x_2f, x_2f+1) as the talk page's RoPE matrix pairs them, or
+ * half-split (x_f, x_{f+d/2}) for the rotate-half layout. */
+static void ora_band(const void* base, int dtype, int64_t row, int f, int d, int half,
+                     double* x, double* y) {
+    if (half) {
+        *x = ora_decode(base, dtype, row + f);
+        *y = ora_decode(base, dtype, row + f + d / 2);
+    } else {
+        *x = ora_decode(base, dtype, row + 2 * f);
+        *y = ora_decode(base, dtype, row + 2 * f + 1);
+    }
 }
 
 /* RoPE angular frequency of band f: w_f = theta^(-2f/d) (talk page, RoPE
@@ -95,22 +132,37 @@ void oracle_set_threads(int n) {
 }
 
 /*
- * Calibration.  q: pre-RoPE queries [n_heads][n_tok][d]; stats out:
+ * Calibration.  q: queries [n_heads][n_tok][d]; stats out:
  * [n_heads][d/2][4] = (Re E[q_f], Im E[q_f], E[|q_f|], R_f).
+ * Pre-RoPE queries are averaged as they are.  Post-RoPE queries (qpos
+ * non-NULL: the position of each token, [n_tok], shared by the heads) are
+ * first rotated back by -w_f p, the inverse of the talk page's RoPE matrix,
+ * which gives the pre-RoPE band (shibing624 paper reading, Q/K concentration
+ * section: the centres live in the pre-RoPE space).  `half` selects the
+ * half-split band pairing.  The same statistics of keys are the K centres.
  */
-int oracle_calibrate(const void* q, int dtype, int64_t n_heads, int64_t n_tok, int d,
-                     double* stats) {
+int oracle_calibrate_ex(const void* q, int dtype, int64_t n_heads, int64_t n_tok, int d,
+                        const int32_t* qpos, double theta, int half, double* stats) {
     if (!q || !stats || n_heads < 0 || n_tok <= 0 || d <= 0 || (d & 1)) return ORA_EINVAL;
     const int F = d / 2;
     int64_t h;
 #pragma omp parallel for schedule(dynamic)
     for (h = 0; h < n_heads; ++h) {
         for (int f = 0; f < F; ++f) {
+            const double w = ora_omega(theta, f, d);
             double sx = 0.0, sy = 0.0, sn = 0.0;
             for (int64_t n = 0; n < n_tok; ++n) {
                 const int64_t row = (h * n_tok + n) * (int64_t)d;
-                const double x = ora_decode(q, dtype, row + 2 * f);
-                const double y = ora_decode(q, dtype, row + 2 * f + 1);
+                double x, y;
+                ora_band(q, dtype, row, f, d, half, &x, &y);
+                if (qpos) {
+                    const double a = w * (double)qpos[n];
+                    const double c = cos(a), sn_ = sin(a);
+                    const double xr = c * x + sn_ * y;
+                    const double yr = -sn_ * x + c * y;
+                    x = xr;
+                    y = yr;
+                }
                 sx += x;
                 sy += y;
                 sn += hypot(x, y);
@@ -129,6 +181,12 @@ int oracle_calibrate(const void* q, int dtype, int64_t n_heads, int64_t n_tok, i
     return ORA_OK;
 }
 
+/* Calibration of pre-RoPE queries with interleaved bands. */
+int oracle_calibrate(const void* q, int dtype, int64_t n_heads, int64_t n_tok, int d,
+                     double* stats) {
+    return oracle_calibrate_ex(q, dtype, n_heads, n_tok, d, NULL, 10000.0, 0, stats);
+}
+
 /*
  * Score one unit (one KV head's cache) for the G query heads of its group,
  * in the pages' unfolded form.
@@ -140,17 +198,21 @@ int oracle_calibrate(const void* q, int dtype, int64_t n_heads, int64_t n_tok, i
  */
 static void ora_score_unit(const void* k, int dtype, int64_t n, int d, const int32_t* pos,
                            int64_t p_cur, const double* stats, int G, double theta,
-                           const int64_t* offsets, int n_off, double* raw, double* kmag,
-                           double* karg, const double* omega) {
+                           const int64_t* offsets, int n_off, int variant, double* raw,
+                           double* kmag, double* karg, const double* omega) {
     const int F = d / 2;
+    const int half = (variant & ORA_VAR_HALF_SPLIT) != 0;
+    const int use_trig = (variant & ORA_VAR_NO_TRIG) == 0;
+    const int use_r = (variant & ORA_VAR_NO_R) == 0;
+    const int use_max = (variant & ORA_VAR_MAX_OFFSET) != 0;
     double qmag[512], qarg[512], qnw[512];
     (void)theta;
     for (int64_t j = 0; j < n; ++j) {
         const double pj = (double)pos[j];
         /* De-rotate: k_f = R(-w_f p_j) k'_f, the inverse of the RoPE matrix. */
         for (int f = 0; f < F; ++f) {
-            const double xr = ora_decode(k, dtype, j * d + 2 * f);
-            const double yr = ora_decode(k, dtype, j * d + 2 * f + 1);
+            double xr, yr;
+            ora_band(k, dtype, j * d, f, d, half, &xr, &yr);
             const double a = omega[f] * pj;
             const double c = cos(a), s = sin(a);
             const double x = c * xr + s * yr;
@@ -165,20 +227,21 @@ static void ora_score_unit(const void* k, int dtype, int64_t n, int d, const int
             for (int f = 0; f < F; ++f) {
                 qmag[f] = hypot(st[f * 4 + 0], st[f * 4 + 1]);
                 qarg[f] = atan2(st[f * 4 + 1], st[f * 4 + 0]);
-                qnw[f] = (1.0 - st[f * 4 + 3]) * st[f * 4 + 2];
+                qnw[f] = (use_r ? 1.0 - st[f * 4 + 3] : 1.0) * st[f * 4 + 2];
             }
-            double total = 0.0;
+            double total = 0.0, best = -INFINITY;
             for (int o = 0; o < n_off; ++o) {
                 const double Delta = (double)(p_cur - (int64_t)pos[j] + offsets[o]);
                 double s_trig = 0.0, s_norm = 0.0;
                 for (int f = 0; f < F; ++f) {
                     const double phi = qarg[f] - karg[f];
-                    s_trig += qmag[f] * kmag[f] * cos(omega[f] * Delta + phi);
+                    if (use_trig) s_trig += qmag[f] * kmag[f] * cos(omega[f] * Delta + phi);
                     s_norm += qnw[f] * kmag[f];
                 }
                 total += s_trig + s_norm;
+                if (s_trig + s_norm > best) best = s_trig + s_norm;
             }
-            raw[(int64_t)h * n + j] = total / (double)n_off;
+            raw[(int64_t)h * n + j] = use_max ? best : total / (double)n_off;
         }
     }
 }
@@ -257,6 +320,42 @@ int64_t oracle_select(const double* fin, int64_t n, int64_t B, int32_t* kept, do
 }
 
 /*
+ * Top-B selection with protected keys: every key j < n_sink or
+ * j >= n - n_recent is kept, the lowest indices of them when they alone are
+ * more than B; the places left go to the other keys in the order of
+ * oracle_select.  threshold out (optional): the score of the last unprotected
+ * key kept, NaN when none is.  Returns the number kept, or -1.
+ */
+int64_t oracle_select_protected(const double* fin, int64_t n, int64_t B, int64_t n_sink,
+                                int64_t n_recent, int32_t* kept, double* threshold) {
+    if (n < 0 || B < 0 || n_sink < 0 || n_recent < 0) return -1;
+    const int64_t m = (B < n) ? B : n;
+    if (threshold) *threshold = NAN;
+    if (n == 0) return 0;
+    int64_t p = 0;
+    for (int64_t j = 0; j < n && p < m; ++j)
+        if (j < n_sink || j >= n - n_recent) kept[p++] = (int32_t)j;
+    if (p == m) return m;
+    ora_item* it = (ora_item*)malloc((size_t)n * sizeof(ora_item));
+    if (!it) return -1;
+    int64_t c = 0;
+    for (int64_t j = 0; j < n; ++j) {
+        if (j < n_sink || j >= n - n_recent) continue;
+        it[c].v = fin[j];
+        it[c].idx = (int32_t)j;
+        it[c].nan = isnan(fin[j]) ? 1 : 0;
+        ++c;
+    }
+    qsort(it, (size_t)c, sizeof(ora_item), ora_cmp_rank);
+    const int64_t rest = m - p;
+    for (int64_t r = 0; r < rest; ++r) kept[p + r] = it[r].idx;
+    if (threshold && rest > 0) *threshold = it[rest - 1].v;
+    free(it);
+    qsort(kept, (size_t)m, sizeof(int32_t), ora_cmp_i32);
+    return m;
+}
+
+/*
  * Whole prune step over a batch of units, one unit at a time per thread.
  * Unit u = (seq * n_layers + layer) * n_kvheads + kvh; its query heads are
  * kvh*G .. kvh*G+G-1 of that layer.
@@ -273,17 +372,24 @@ int64_t oracle_select(const double* fin, int64_t n, int64_t B, int32_t* kept, do
  *   thr:        [U] B-th score (optional)
  *   k_dst, v_dst, pos_dst: [U][cap_dst][d] gathered rows (optional)
  *   unit_list:  subset of units to process (NULL: all), n_list entries
+ *   variant:    ORA_VAR_* bits (0: the method as the pages' main text states it)
+ *   n_sink, n_recent: protected first / last keys of each unit (0: none)
+ *   layer_budget: [n_layers] budget of each layer's units, at most B (NULL: B)
  */
 int oracle_prune(const void* k, const void* v, const int32_t* pos, int dtype, int64_t n_seq,
                  int64_t n_layers, int64_t n_kvheads, int G, int64_t cap, int d,
                  const int32_t* n_valid, const int64_t* p_cur, const double* stats, double theta,
                  const int64_t* offsets, int n_off, int64_t B, double* raw, double* fin,
                  int32_t* kept, int64_t* n_kept, double* thr, void* k_dst, void* v_dst,
-                 int32_t* pos_dst, int64_t cap_dst, const int64_t* unit_list, int64_t n_list) {
+                 int32_t* pos_dst, int64_t cap_dst, const int64_t* unit_list, int64_t n_list,
+                 int variant, int64_t n_sink, int64_t n_recent, const int64_t* layer_budget) {
     if (!k || !pos || !p_cur || !stats || !offsets || n_off <= 0 || G <= 0 || cap < 0 || d <= 0 ||
-        d > 1024 || (d & 1) || B < 0)
+        d > 1024 || (d & 1) || B < 0 || n_sink < 0 || n_recent < 0)
         return ORA_EINVAL;
     if ((k_dst || v_dst || pos_dst) && cap_dst < ((B < cap) ? B : cap)) return ORA_EINVAL;
+    if (layer_budget)
+        for (int64_t l = 0; l < n_layers; ++l)
+            if (layer_budget[l] < 0 || layer_budget[l] > B) return ORA_EINVAL;
     const int F = d / 2;
     const int64_t U = n_seq * n_layers * n_kvheads;
     const int64_t count = unit_list ? n_list : U;
@@ -321,10 +427,13 @@ int oracle_prune(const void* k, const void* v, const int32_t* pos, int dtype, in
             const double* st = stats + ((layer * n_kvheads + kvh) * (int64_t)G) * F * 4;
             const void* ku = (const char*)k + (size_t)(u * cap * d) * esize;
             ora_score_unit(ku, dtype, n, d, pos + u * cap, p_cur[seq], st, G, theta, offsets,
-                           n_off, r, kmag, karg, omega);
+                           n_off, variant, r, kmag, karg, omega);
             ora_znorm_max(r, G, n, z, fn, NULL, NULL);
             double t;
-            const int64_t m = oracle_select(fn, n, B, kp, &t);
+            const int64_t Bu = layer_budget ? layer_budget[layer] : B;
+            const int64_t m = (n_sink > 0 || n_recent > 0)
+                                  ? oracle_select_protected(fn, n, Bu, n_sink, n_recent, kp, &t)
+                                  : oracle_select(fn, n, Bu, kp, &t);
             if (raw)
                 for (int h = 0; h < G; ++h)
                     memcpy(raw + (u * G + h) * cap, r + (int64_t)h * n, (size_t)n * sizeof(double));
@@ -358,7 +467,7 @@ int oracle_prune(const void* k, const void* v, const int32_t* pos, int dtype, in
 /* Score only (per-head S~) for one unit; exposed for the pins. */
 int oracle_score(const void* k, int dtype, int64_t n, int d, const int32_t* pos, int64_t p_cur,
                  const double* stats, int G, double theta, const int64_t* offsets, int n_off,
-                 double* raw) {
+                 int variant, double* raw) {
     if (!k || !pos || !stats || !offsets || !raw || n < 0 || G <= 0 || d <= 0 || d > 1024 ||
         (d & 1) || n_off <= 0)
         return ORA_EINVAL;
@@ -373,8 +482,8 @@ int oracle_score(const void* k, int dtype, int64_t n, int d, const int32_t* pos,
         return ORA_ENOMEM;
     }
     for (int f = 0; f < F; ++f) omega[f] = ora_omega(theta, f, d);
-    ora_score_unit(k, dtype, n, d, pos, p_cur, stats, G, theta, offsets, n_off, raw, kmag, karg,
-                   omega);
+    ora_score_unit(k, dtype, n, d, pos, p_cur, stats, G, theta, offsets, n_off, variant, raw,
+                   kmag, karg, omega);
     free(omega);
     free(kmag);
     free(karg);

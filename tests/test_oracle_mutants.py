@@ -13,6 +13,7 @@ import pytest
 
 import oracle
 from tests import test_oracle_pins as pins
+from tests import test_oracle_variants as var
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "tri_oracle.c")
 
@@ -20,15 +21,32 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "tri_oracle.c")
 MUTANTS = [
     ("omega exponent -f/d", "pow(theta, -2.0 * (double)f / (double)d)",
      "pow(theta, -1.0 * (double)f / (double)d)"),
-    ("half-split pairing", "const double yr = ora_decode(k, dtype, j * d + 2 * f + 1);",
-     "const double yr = ora_decode(k, dtype, j * d + (2 * f + 1 + d / 2) % d);"),
+    ("half-split pairing", "*y = ora_decode(base, dtype, row + 2 * f + 1);",
+     "*y = ora_decode(base, dtype, row + (2 * f + 1 + d / 2) % d);"),
     ("phase sign", "const double phi = qarg[f] - karg[f];", "const double phi = karg[f] - qarg[f];"),
     ("de-rotation direction", "const double x = c * xr + s * yr;", "const double x = c * xr - s * yr;"),
     ("Delta sign", "(double)(p_cur - (int64_t)pos[j] + offsets[o])",
      "(double)((int64_t)pos[j] - p_cur + offsets[o])"),
-    ("no 1/|D|", "raw[(int64_t)h * n + j] = total / (double)n_off;", "raw[(int64_t)h * n + j] = total;"),
-    ("R weight on the wrong side", "qnw[f] = (1.0 - st[f * 4 + 3]) * st[f * 4 + 2];",
-     "qnw[f] = st[f * 4 + 3] * st[f * 4 + 2];"),
+    ("no 1/|D|", "use_max ? best : total / (double)n_off;", "use_max ? best : total;"),
+    ("R weight on the wrong side", "(use_r ? 1.0 - st[f * 4 + 3] : 1.0)",
+     "(use_r ? st[f * 4 + 3] : 1.0)"),
+    # method variants
+    ("no-trig keeps S_trig", "if (use_trig) s_trig +=", "if (1) s_trig +="),
+    ("no-R keeps the R factor", "(use_r ? 1.0 - st[f * 4 + 3] : 1.0)",
+     "(1.0 - st[f * 4 + 3])"),
+    ("max over offsets takes the min", "if (s_trig + s_norm > best) best = s_trig + s_norm;",
+     "if (best == -INFINITY || s_trig + s_norm < best) best = s_trig + s_norm;"),
+    ("max over offsets drops S_norm", "if (s_trig + s_norm > best) best = s_trig + s_norm;",
+     "if (s_trig > best) best = s_trig;"),
+    ("half-split pairs f with f + d/2 - 1", "*y = ora_decode(base, dtype, row + f + d / 2);",
+     "*y = ora_decode(base, dtype, row + (f + d / 2 - 1 + d) % d);"),
+    ("post-RoPE calibration rotates forward", "const double xr = c * x + sn_ * y;",
+     "const double xr = c * x - sn_ * y;"),
+    ("recent window one short", "if (j < n_sink || j >= n - n_recent) kept[p++] = (int32_t)j;",
+     "if (j < n_sink || j > n - n_recent) kept[p++] = (int32_t)j;"),
+    ("protected keys ignored", "const int64_t rest = m - p;", "const int64_t rest = m - p; p = 0;"),
+    ("layer budget of the next layer", "const int64_t Bu = layer_budget ? layer_budget[layer] : B;",
+     "const int64_t Bu = layer_budget ? layer_budget[(layer + 1) % n_layers] : B;"),
     ("sample sigma", "sqrt(ss / (double)n)", "sqrt(ss / (double)(n > 1 ? n - 1 : 1))"),
     ("mean over heads", "for (int h = 1; h < G; ++h) m = fmax(m, z[(int64_t)h * n + j]);",
      "for (int h = 1; h < G; ++h) m += z[(int64_t)h * n + j]; m /= G;"),
@@ -58,6 +76,17 @@ PIN_TESTS = [
     lambda: pins.test_select_order_and_threshold(),
     lambda: [pins.test_prune_gather_is_bitwise_and_ascending(dt) for dt in ("f32", "bf16")],
     lambda: pins.test_unit_phasor_MRL_matches_R(),
+    lambda: var.test_no_trig_is_blind_to_band_phases(),
+    lambda: var.test_no_trig_with_concentrated_queries_is_zero(),
+    lambda: var.test_no_r_score_bounds(),
+    lambda: var.test_no_r_equals_default_for_centreless_queries(),
+    lambda: [var.test_max_over_offsets_equals_explicit_rope_logit_max(o)
+             for o in [(1,), (3, 1000), oracle.OFFSETS]],
+    lambda: var.test_max_over_offsets_bounds_the_mean(),
+    lambda: var.test_half_split_is_a_relabelling_of_interleaved(),
+    lambda: var.test_post_rope_calibration_recovers_pre_rope_stats(),
+    lambda: [var.test_protected_selection_matches_brute_force(s) for s in range(8)],
+    lambda: var.test_layer_budgets_equal_single_budget_runs(),
 ]
 
 

@@ -20,6 +20,9 @@ Every function follows the pages step by step:
 * ``select`` -- top-B by (score desc, index asc), returned ascending
   (jaedaily.cn KV-compression tutorial, eviction step).
 * ``prune`` -- all of the above plus the bit-exact gather, over many units.
+* ``decode_attention`` -- softmax attention of the next token's queries over
+  the kept keys, renormalised over them (jaedaily.cn tutorial, compression
+  objective), the consumer of the compacted cache.
 
 Method variants (``variant`` bits, protection and per-layer budgets of
 ``prune``; ``calibrate`` with positions and pairing) follow the pages'
@@ -96,6 +99,8 @@ def _bind(lib):
     lib.oracle_prune.argtypes = [P, P, P, i32, i64, i64, i64, i32, i64, i32, P, P, P, d, P,
                                  i32, i64, P, P, P, P, P, P, P, P, i64, P, i64, i32, i64, i64, P]
     lib.oracle_prune.restype = i32
+    lib.oracle_decode_attention.argtypes = [P, P, P, i32, i64, i32, i64, i32, P, d, P]
+    lib.oracle_decode_attention.restype = i32
     lib.oracle_threads.argtypes = []
     lib.oracle_threads.restype = i32
     lib.oracle_set_threads.argtypes = [i32]
@@ -272,4 +277,25 @@ def prune(k, v, pos, n_seq, n_layers, n_kvheads, G, stats, p_cur, B, n_valid=Non
         out["raw"] = raw
     if want_gather:
         out.update(k_dst=kd, v_dst=vd, pos_dst=pd)
+    return out
+
+
+def decode_attention(q, k, v, n_valid=None, scale=None):
+    """Attention of one query token per head over a cache (tri_oracle.c:
+    oracle_decode_attention).  q [U, G, d], k / v [U, cap, d] (float32 or raw
+    bf16 uint16, one type) -> out [U, G, d] float64."""
+    q, dt = _elem(q)
+    k, dtk = _elem(k)
+    v, dtv = _elem(v)
+    if not dt == dtk == dtv:
+        raise TypeError("q, k and v must share a dtype")
+    U, G, d = q.shape
+    cap = k.shape[1]
+    nv = None if n_valid is None else np.ascontiguousarray(np.asarray(n_valid, np.int32))
+    sc = 1.0 / np.sqrt(d) if scale is None else float(scale)
+    out = np.empty((U, G, d), np.float64)
+    rc = _load().oracle_decode_attention(_ptr(q), _ptr(k), _ptr(v), dt, U, G, cap, d, _ptr(nv),
+                                         sc, _ptr(out))
+    if rc:
+        raise ValueError(f"oracle_decode_attention failed ({rc})")
     return out

@@ -497,3 +497,65 @@ int oracle_znorm_max(const double* raw, int G, int64_t n, double* z, double* fin
     ora_znorm_max(raw, G, n, z, fin, mu, sd);
     return ORA_OK;
 }
+
+/*
+ * Decode attention of one new query token over a (compacted) cache, one unit
+ * at a time (jaedaily.cn tutorial, KV-compression objective: the output over
+ * the kept subset S is sum_{j in S} a_j v_j with the softmax weights
+ * a_j = exp(q.k_j / sqrt(d)) / sum_{j' in S} exp(q.k_j' / sqrt(d)),
+ * renormalised over S).  scale multiplies the dot products (1/sqrt(d) for
+ * the usual attention; any positive value).
+ *   q:   [U][G][d] post-RoPE query of the current token for the G query heads
+ *        of each unit (float32 or bf16 codes, like k and v)
+ *   k,v: [U][cap][d] cache rows; the first n_valid[u] are attended
+ *   out: [U][G][d] double
+ * A unit with no valid key gives zeros.  The maximum score is subtracted
+ * before exponentiating (the value is the same in exact arithmetic).
+ */
+int oracle_decode_attention(const void* q, const void* k, const void* v, int dtype,
+                            int64_t n_units, int G, int64_t cap, int d, const int32_t* n_valid,
+                            double scale, double* out) {
+    if (!q || !k || !v || !out || n_units < 0 || G <= 0 || cap < 0 || d <= 0) return ORA_EINVAL;
+    int64_t u;
+    int err = ORA_OK;
+#pragma omp parallel for schedule(dynamic)
+    for (u = 0; u < n_units; ++u) {
+        const int64_t n = n_valid ? n_valid[u] : cap;
+        if (n < 0 || n > cap) {
+#pragma omp atomic write
+            err = ORA_EINVAL;
+            continue;
+        }
+        double* sc = (double*)malloc((size_t)(n > 0 ? n : 1) * sizeof(double));
+        if (!sc) {
+#pragma omp atomic write
+            err = ORA_ENOMEM;
+            continue;
+        }
+        for (int h = 0; h < G; ++h) {
+            const int64_t qrow = (u * G + h) * (int64_t)d;
+            double* o = out + (u * G + h) * (int64_t)d;
+            for (int e = 0; e < d; ++e) o[e] = 0.0;
+            if (n == 0) continue;
+            double mx = -INFINITY;
+            for (int64_t j = 0; j < n; ++j) {
+                const int64_t krow = (u * cap + j) * (int64_t)d;
+                double dot = 0.0;
+                for (int e = 0; e < d; ++e)
+                    dot += ora_decode(q, dtype, qrow + e) * ora_decode(k, dtype, krow + e);
+                sc[j] = scale * dot;
+                if (sc[j] > mx) mx = sc[j];
+            }
+            double den = 0.0;
+            for (int64_t j = 0; j < n; ++j) {
+                const double w = exp(sc[j] - mx);
+                den += w;
+                const int64_t vrow = (u * cap + j) * (int64_t)d;
+                for (int e = 0; e < d; ++e) o[e] += w * ora_decode(v, dtype, vrow + e);
+            }
+            for (int e = 0; e < d; ++e) o[e] /= den;
+        }
+        free(sc);
+    }
+    return err;
+}

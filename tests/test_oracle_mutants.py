@@ -45,6 +45,11 @@ MUTANTS = [
     ("recent window one short", "if (j < n_sink || j >= n - n_recent) kept[p++] = (int32_t)j;",
      "if (j < n_sink || j > n - n_recent) kept[p++] = (int32_t)j;"),
     ("protected keys ignored", "const int64_t rest = m - p;", "const int64_t rest = m - p; p = 0;"),
+    ("attention skips the max shift", "const double w = exp(sc[j] - mx);",
+     "const double w = exp(sc[j] - mx) * (j == 0 ? 2.0 : 1.0);"),
+    ("attention scale dropped", "sc[j] = scale * dot;", "sc[j] = dot;"),
+    ("attention over one row too few", "for (int64_t j = 0; j < n; ++j) {\n                const int64_t krow",
+     "for (int64_t j = 0; j + 1 < n; ++j) {\n                const int64_t krow"),
     ("layer budget of the next layer", "const int64_t Bu = layer_budget ? layer_budget[layer] : B;",
      "const int64_t Bu = layer_budget ? layer_budget[(layer + 1) % n_layers] : B;"),
     ("sample sigma", "sqrt(ss / (double)n)", "sqrt(ss / (double)(n > 1 ? n - 1 : 1))"),
@@ -87,6 +92,8 @@ PIN_TESTS = [
     lambda: var.test_post_rope_calibration_recovers_pre_rope_stats(),
     lambda: [var.test_protected_selection_matches_brute_force(s) for s in range(8)],
     lambda: var.test_layer_budgets_equal_single_budget_runs(),
+    lambda: var.test_decode_attention_matches_library_sdpa(),
+    lambda: var.test_decode_attention_special_cases(),
 ]
 
 

@@ -234,3 +234,52 @@ def test_layer_budgets_equal_single_budget_runs():
     with pytest.raises(ValueError):
         oracle.prune(c["k"], c["v"], c["pos"], c["n_seq"], c["L"], c["Hkv"], c["G"], c["st"],
                      c["p_cur"], c["B"], n_valid=c["n_valid"], layer_budget=[c["B"] + 1, 1])
+
+
+# ---------------------------------------------------------------------------
+# decode attention over the kept keys
+# ---------------------------------------------------------------------------
+def test_decode_attention_matches_library_sdpa():
+    """Against torch's scaled_dot_product_attention in float64 on the CPU (a
+    library routine), per unit and head, over the first n_valid rows."""
+    import torch
+
+    rng = np.random.default_rng(11)
+    U, G, cap = 3, 4, 50
+    q = rng.normal(size=(U, G, D)).astype(np.float32)
+    k = rng.normal(size=(U, cap, D)).astype(np.float32)
+    v = rng.normal(size=(U, cap, D)).astype(np.float32)
+    nv = np.array([50, 17, 1], np.int32)
+    got = oracle.decode_attention(q, k, v, n_valid=nv)
+    for u in range(U):
+        n = int(nv[u])
+        qq = torch.from_numpy(q[u].astype(np.float64))[:, None, :]          # [G, 1, d]
+        kk = torch.from_numpy(k[u, :n].astype(np.float64))[None].expand(G, n, D)
+        vv = torch.from_numpy(v[u, :n].astype(np.float64))[None].expand(G, n, D)
+        want = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv)[:, 0].numpy()
+        np.testing.assert_allclose(got[u], want, rtol=1e-12, atol=1e-12)
+
+
+def test_decode_attention_special_cases():
+    """A zero query weighs every kept key equally (the mean of the values);
+    one kept key returns its value; a key scored far above the others takes
+    all the weight; no kept key gives zeros; reordering the keys changes
+    nothing."""
+    rng = np.random.default_rng(12)
+    cap = 40
+    k = rng.normal(size=(1, cap, D)).astype(np.float32)
+    v = rng.normal(size=(1, cap, D)).astype(np.float32)
+    q0 = np.zeros((1, 2, D), np.float32)
+    np.testing.assert_allclose(oracle.decode_attention(q0, k, v)[0, 0],
+                               v[0].astype(np.float64).mean(0), rtol=1e-12, atol=1e-13)
+    q = rng.normal(size=(1, 2, D)).astype(np.float32)
+    np.testing.assert_allclose(oracle.decode_attention(q, k, v, n_valid=[1])[0, 1], v[0, 0],
+                               rtol=1e-15)
+    assert not oracle.decode_attention(q, k, v, n_valid=[0]).any()
+    k2 = k.copy()
+    k2[0, 7] = 40.0 * q[0, 0] / np.linalg.norm(q[0, 0])
+    np.testing.assert_allclose(oracle.decode_attention(q, k2, v, scale=1.0)[0, 0], v[0, 7],
+                               rtol=1e-9, atol=1e-9)
+    perm = rng.permutation(cap)
+    np.testing.assert_allclose(oracle.decode_attention(q, k[:, perm], v[:, perm]),
+                               oracle.decode_attention(q, k, v), rtol=1e-12, atol=1e-13)

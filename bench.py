@@ -324,7 +324,8 @@ def run_reference(args, ws, rank):
         return
     import oracle
 
-    spec = synth.SPECS[args.workload]
+    stream_run = args.workload == STREAM
+    spec = synth.SPECS["c5" if stream_run else args.workload]
     inp, keys, desc, n_units = oracle_sample(spec, seconds_hint=0.5)
     for _ in range(args.warmup):
         oracle_step(inp)
@@ -335,6 +336,26 @@ def run_reference(args, ws, rank):
     value = keys / dt
     threads = min(n_units, oracle.threads())
     desc = desc + f", oracle on {threads} thread(s)"
+    if stream_run:
+        # Seconds per key of the sample, scaled to the 240 prunes of the
+        # stream at full width, per generated token.
+        prunes = (synth.STREAM_TOKENS - spec.cap) // synth.STREAM_WINDOW + 1
+        us_tok = dt / keys * spec.n_units * spec.cap * prunes / synth.STREAM_TOKENS * 1e6
+        line = {
+            "impl": "reference",
+            "metric": "prune-path time per generated token (appends included), streaming run",
+            "value": us_tok, "unit": "us/token", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": STREAM, "sample": desc + "; scaled by keys to the 240 "
+                       "prunes of the full-width stream (appends not counted)"},
+            "cpu_baseline": {"value": us_tok, "unit": "us/token", "cores": os.cpu_count(),
+                             "threads": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": us_tok, "unit": "us/token", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+        return
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "keys/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -538,6 +559,102 @@ def dominant(spec, rec, ms_step):
 
 
 SUB_WORKLOADS = ("c2", "c3", "c5")
+STREAM = "c5-stream"
+
+
+def time_stream(args, dev, stream, ws, inplace_too=True):
+    """The streaming workload end to end (64 sequences x 28 layers x 4 KV
+    heads, G 7, B 2048): from an empty cache, the 256 windows of 128 generated
+    tokens (32768 tokens) are appended with tri_append and the cache is
+    pruned back to B whenever it holds B + 128 rows (240 prunes), through the
+    window driver, on two cache buffers (tri_prune) and, on the same windows,
+    on one buffer compacted in place (tri_prune_inplace).  Each window's keys
+    are drawn at their own positions before its segment; the library's
+    launches of a segment (append, then prune) are timed between CUDA events
+    on the launching stream and summed, max over ranks."""
+    import rope_aware_kv_b200 as tri
+    from rope_aware_kv_b200.window import WindowDriver
+
+    spec = synth.SPECS["c5"]
+    hp = synth.head_params(spec)
+    stats = torch.empty((spec.n_layers, spec.n_qheads, 64, 4), dtype=torch.float32, device=dev)
+    for layer in range(spec.n_layers):
+        q = synth.calib_queries(spec, hp, layer, dev)
+        tri.tri_calibrate(q, stats=stats[layer])
+        del q
+    window = synth.STREAM_WINDOW
+    n_windows = synth.STREAM_TOKENS // window
+    modes = [False, True] if inplace_too else [False]
+    drivers = {m: WindowDriver(spec.n_seq, spec.n_layers, spec.n_kvheads, spec.G, spec.B, stats,
+                               window=window, device=dev, inplace=m) for m in modes}
+
+    launches = {m: 0 for m in modes}
+
+    def run(n, timed):
+        ev = {m: [] for m in modes}
+        with torch.cuda.stream(stream):
+            for d in drivers.values():
+                d.reset()
+            for w in range(n):
+                k_new, v_new, pos_new = synth.stream_window(spec, hp, w, dev)
+                for m, d in drivers.items():
+                    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+                    e[0].record(stream)
+                    d.append(k_new, v_new, pos_new, auto_prune=False, stream=stream)
+                    if timed:
+                        launches[m] += tri.tri_last_launch_count()
+                    e[1].record(stream)
+                    if d.full:
+                        d.prune(stream=stream)
+                        if timed:
+                            launches[m] += tri.tri_last_launch_count()
+                    e[2].record(stream)
+                    ev[m].append(e)
+                del k_new, v_new, pos_new
+        torch.cuda.synchronize()
+        return ev
+
+    run(spec.cap // window + 3, False)  # warm-up: three prunes per driver
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    barrier(ws)
+    clocks.start()
+    ev = run(n_windows, True)
+    clk = clocks.stop()
+    barrier(ws)
+    peak_gbs, peak_kind = measured_peaks()
+    comp = compulsory_bytes(spec)
+    out = {}
+    for m, d in drivers.items():
+        app = sum(e[0].elapsed_time(e[1]) for e in ev[m])
+        pru = sum(e[1].elapsed_time(e[2]) for e in ev[m])
+        flags = tri.tri_check_device_error(d.ws)
+        total = max_over_ranks(app + pru, ws)
+        roof_ms = d.prunes * comp / (peak_gbs * 1e9) * 1e3
+        out["inplace" if m else "pingpong"] = {
+            "tokens": d.tokens, "windows": n_windows, "prunes": d.prunes,
+            "total_ms": total, "append_ms": app, "prune_ms": pru,
+            "prune_ms_mean": pru / max(d.prunes, 1),
+            "us_per_token": total * 1e3 / d.tokens,
+            "keys_per_s": d.prunes * spec.n_units * spec.cap * ws / (total * 1e-3),
+            "path": {tri.PATH_PIPE: "pipe", tri.PATH_SPLIT: "split", tri.PATH_COOP: "coop",
+                     tri.PATH_FUSED: "fused"}.get(
+                tri.tri_prune_path(spec.n_seq, spec.n_layers, spec.n_kvheads, spec.G, spec.cap,
+                                   spec.B, inplace=m), "none"),
+            "roofline_us_per_token": roof_ms * 1e3 / d.tokens,
+            "frac": roof_ms / total if total > 0 else 0.0,
+            "device_flags": flags, "gpu_launches": launches[m],
+        }
+    del drivers
+    torch.cuda.empty_cache()
+    return {
+        "workload": f"{STREAM}: {synth.STREAM_TOKENS} generated tokens, 64 seqs x 28 layers x "
+                    f"4 KV heads, G 7, B {spec.B}, prune every {window} tokens "
+                    f"(cache B + {window} rows)",
+        "compulsory_bytes_per_prune": comp, "peak_gbs": peak_gbs, "peak_kind": peak_kind,
+        "timing": "per window: CUDA events around the append and the prune on the launching "
+                  "stream, summed over the stream; key generation outside the timed segments",
+        "clocks": clk, **out,
+    }
 
 
 def run_tri(args, ws, rank, local):
@@ -548,6 +665,9 @@ def run_tri(args, ws, rank, local):
         tri_build.build()
     barrier(ws)
     tri.load()
+    if args.workload == STREAM:
+        run_stream_line(args, ws, rank, local)
+        return
     spec = synth.SPECS[args.workload]
     if args.n_seq:
         spec = spec.scaled(n_seq=args.n_seq)
@@ -581,6 +701,8 @@ def run_tri(args, ws, rank, local):
             subs[name] = srec
             del r2
             torch.cuda.empty_cache()
+        subs[STREAM] = time_stream(args, dev, stream, ws)
+        subs["decode"] = time_decode(args, dev, stream, ws, min(args.steps, 50))
 
     cpu = cpu_baseline(spec) if (rank == 0 and ws == 1 and not args.no_cpu_baseline) else None
 
@@ -616,6 +738,86 @@ def run_tri(args, ws, rank, local):
             "e2e": e2e,
             "cpu_baseline": cpu,
             "sub_workloads": subs,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def time_decode(args, dev, stream, ws, steps):
+    """Decode attention of the next token over the streaming workload's
+    compacted cache (64 seqs x 28 layers x 4 KV heads, G 7, B 2048 kept rows
+    per unit): K and V rows read once per step, 7.5 GB > L2.  One CUDA graph
+    of ``steps`` calls between CUDA events, max over ranks."""
+    import rope_aware_kv_b200 as tri
+
+    spec = synth.SPECS["c5"]
+    U, B, G = spec.n_units, spec.B, spec.G
+    g = torch.Generator(device=dev).manual_seed(5)
+    k = torch.empty((U, B, spec.d), dtype=torch.bfloat16, device=dev)
+    v = torch.empty_like(k)
+    for u0 in range(0, U, 512):
+        k[u0:u0 + 512] = torch.randn((min(512, U - u0), B, spec.d), generator=g, device=dev)
+        v[u0:u0 + 512] = torch.randn((min(512, U - u0), B, spec.d), generator=g, device=dev)
+    q = (torch.randn((U, G, spec.d), generator=g, device=dev) * 0.1).to(torch.bfloat16)
+    nv = torch.full((U,), B, dtype=torch.int32, device=dev)
+    out = torch.empty((U, G, spec.d), dtype=torch.float32, device=dev)
+    wsb = tri.workspace(tri.load().tri_decode_workspace_bytes(U, G, B), dev)
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3)):
+            tri.tri_decode_attention(q, k, v, n_valid=nv, out=out, ws=wsb, stream=stream)
+        torch.cuda.synchronize()
+        launches = tri.tri_last_launch_count()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream, capture_error_mode="relaxed"):
+            for _ in range(steps):
+                tri.tri_decode_attention(q, k, v, n_valid=nv, out=out, ws=wsb, stream=stream)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    barrier(ws)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        gr.replay()
+        t1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1), ws) / steps
+    flags = tri.tri_check_device_error(wsb)
+    del gr, k, v
+    torch.cuda.empty_cache()
+    peak_gbs, peak_kind = measured_peaks()
+    nbytes = U * B * spec.d * 2 * 2 + U * G * spec.d * (2 + 4)
+    return {"workload": "decode attention over the compacted streaming cache: 7168 units x 2048 "
+                        "kept bf16 rows, G 7, one query token per head",
+            "ms_per_step": ms, "tokens_per_s": spec.n_seq * ws / (ms * 1e-3),
+            "hbm_gbs": nbytes / (ms * 1e-3) / 1e9, "frac": nbytes / (ms * 1e-3) / 1e9 / peak_gbs,
+            "bytes_per_step": nbytes, "peak_gbs": peak_gbs, "peak_kind": peak_kind,
+            "launches_per_step": launches, "device_flags": flags, "steps": steps}
+
+
+def run_stream_line(args, ws, rank, local):
+    """``--workload c5-stream``: the streaming run as the bench line (metric:
+    prune-path time per generated token, appends included)."""
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    rec = time_stream(args, dev, stream, ws)
+    pp = rec["pingpong"]
+    if rank == 0:
+        line = {
+            "metric": "prune-path time per generated token (appends included), streaming run",
+            "value": pp["us_per_token"], "unit": "us/token", "n_gpus": ws,
+            "steps": pp["prunes"], "warmup": 3, "ms_per_step": pp["total_ms"] / pp["prunes"],
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": rec["workload"], "parallelism": f"dp{ws} (independent units)",
+                       "l2": "each prune reads 4.0 GB of keys (> 126 MB L2)",
+                       "timing": rec["timing"]},
+            "roofline": {"bound": "hbm", "kernel": "whole prune step",
+                         "achieved": pp["prunes"] * rec["compulsory_bytes_per_prune"]
+                         / (pp["prune_ms"] * 1e-3) / 1e9,
+                         "peak": rec["peak_gbs"], "peak_kind": rec["peak_kind"], "unit": "GB/s",
+                         "frac": pp["prunes"] * rec["compulsory_bytes_per_prune"]
+                         / (pp["prune_ms"] * 1e-3) / 1e9 / rec["peak_gbs"], "traffic": None},
+            "gpu_launches": pp["gpu_launches"], "clocks": rec["clocks"], "stream": rec,
         }
         print(json.dumps(line), flush=True)
 
@@ -675,7 +877,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="tri", choices=["tri", "reference"])
-    ap.add_argument("--workload", default="c4", choices=sorted(synth.SPECS))
+    ap.add_argument("--workload", default="c4", choices=sorted(synth.SPECS) + [STREAM])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sub", action="store_true",
                     help="time the chosen workload only (no sub-records of the others)")

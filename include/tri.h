@@ -113,16 +113,53 @@ typedef enum tri_dtype {
 #define TRI_PATH_COOP 3  /* each unit split over several CTAs of one kernel (few large units) */
 #define TRI_PATH_PIPE 4  /* persistent kernel, gather of one unit overlapping the next's score */
 
+/* Method variants (tri_config.variant bits; 0 is the method as the pages'
+ * main text states it).  Ablations of the shibing624 paper reading's
+ * ablation section and alternatives the pages name:
+ *   TRI_VAR_NO_TRIG     S_trig left out: the score is S_norm alone;
+ *   TRI_VAR_NO_R        the norm weight E[|q_f|] without the (1 - R_f) factor;
+ *   TRI_VAR_MAX_OFFSET  the maximum over the offsets D of S_trig + S_norm
+ *                       instead of their mean (future-offset paragraph: the
+ *                       maximum is the key's score);
+ *   TRI_VAR_HALF_SPLIT  band f pairs components (x_f, x_{f+d/2}), the
+ *                       rotate-half RoPE layout, for keys and (tri_calibrate_ex)
+ *                       queries, instead of (x_2f, x_2f+1).
+ * NO_TRIG and NO_R change only the folded weights and run on every path;
+ * MAX_OFFSET and HALF_SPLIT run on the split path (TRI_PATH_AUTO takes it;
+ * another forced path returns TRI_ERR_UNSUPPORTED). */
+#define TRI_VAR_NO_TRIG 0x1
+#define TRI_VAR_NO_R 0x2
+#define TRI_VAR_MAX_OFFSET 0x4
+#define TRI_VAR_HALF_SPLIT 0x8
+#define TRI_VAR_ALL 0xf
+
 typedef struct tri_config {
     int head_dim;                      /* d; 128 is supported */
     double theta;                      /* RoPE base, 10000 */
     int n_offsets;                     /* |D|, 1..TRI_MAX_OFFSETS */
     int64_t offsets[TRI_MAX_OFFSETS];  /* future offsets delta >= 0 */
     int path;                          /* TRI_PATH_* (tri_prune only) */
+    int variant;                       /* TRI_VAR_* bits, 0 by default */
+    /* Protected keys (jaedaily.cn tutorial, streaming section: the most
+     * recent tokens are kept from eviction): keys j < n_sink and
+     * j >= n_valid - n_recent of every unit get the final score +inf, so
+     * they rank before every other key (ties by index: the lowest-indexed
+     * protected keys when they alone exceed the budget).  Both 0 by default. */
+    int64_t n_sink;
+    int64_t n_recent;
+    /* Per-layer budgets (same tutorial, budget paragraph: pyramid-shaped
+     * budgets per layer): device array [n_layers], entry l the budget of
+     * every unit of layer l, clamped to [0, B]; B remains the row stride of
+     * kept_idx and the bound of cap_dst.  NULL: B everywhere (tri_prune only). */
+    const int32_t* layer_budget;
 } tri_config;
 
 /* Fill cfg (host) with head_dim, theta = 10000, D = {2^0, ..., 2^16}
- * (talk page, offset-averaged score S~) and TRI_PATH_AUTO. */
+ * (talk page, offset-averaged score S~), TRI_PATH_AUTO and no variant,
+ * protection or per-layer budget.
+ * Protection and per-layer budgets run on the pipelined and split paths
+ * (TRI_PATH_AUTO picks one; TRI_PATH_FUSED or TRI_PATH_COOP returns
+ * TRI_ERR_UNSUPPORTED). */
 void tri_config_default(tri_config* cfg, int head_dim);
 
 /* Human-readable name of a status code (static string). */
@@ -152,6 +189,21 @@ size_t tri_calibrate_workspace_bytes(int64_t n_heads, int64_t n_tok, int head_di
  */
 tri_status tri_calibrate(const void* q_pre, tri_dtype dt, int64_t n_heads, int64_t n_tok,
                          int head_dim, float* stats, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Calibration with the config's options: head_dim, theta and the band
+ * pairing (TRI_VAR_HALF_SPLIT in cfg->variant) from cfg.  q_pos (nullable,
+ * device [n_tok] int32): q holds post-RoPE rows, token t at position
+ * q_pos[t] in every head; each band is rotated back by -w_f q_pos[t] (the
+ * inverse of the talk page's RoPE matrix) before it is averaged, so the
+ * statistics are those of the pre-RoPE queries (shibing624 paper reading,
+ * Q/K concentration section: the centres live in the pre-RoPE space).  The
+ * same call on keys gives the K centres.  Layouts, results and workspace as
+ * tri_calibrate.
+ */
+tri_status tri_calibrate_ex(const tri_config* cfg, const void* q, tri_dtype dt, int64_t n_heads,
+                            int64_t n_tok, int head_dim, const int32_t* q_pos, float* stats,
+                            void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Calibration split for data-parallel shards of the calibration tokens: each
@@ -273,6 +325,25 @@ tri_status tri_compact(const void* k_src, const void* v_src, const int32_t* pos_
                        const int32_t* n_kept, int64_t B, void* k_dst, void* v_dst,
                        int32_t* pos_dst, int64_t cap_dst, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * In-place order-preserving compaction of one cache buffer: for r < n_kept[u],
+ *   k[u][r] = k[u][kept_idx[u][r]] (as it was on entry), v and pos likewise
+ * (tutorial eviction step, keys[idx] / values[idx] kept in temporal order,
+ * without a second cache buffer).  kept_idx rows must satisfy
+ * kept_idx[u][r] >= r, which every ascending list of distinct indices does
+ * (the lists tri_select_topB writes); a row whose index breaks this or lies
+ * outside [0, cap) is left unwritten and sets TRI_FLAG_INDEX_RANGE.  Rows
+ * that already hold their kept row (the prefix before the first dropped row)
+ * are not moved; rows r >= n_kept[u] keep their old contents.
+ *   k, v: [U][cap][head_dim] (dt), v nullable; pos: [U][cap] int32, nullable.
+ *   The three buffers must not overlap one another.
+ *   ws: tri_compact_workspace_bytes() bytes (the device flag word).
+ */
+tri_status tri_compact_inplace(void* k, void* v, int32_t* pos, tri_dtype dt, int64_t n_units,
+                               int64_t cap, int head_dim, const int32_t* kept_idx,
+                               const int32_t* n_kept, int64_t B, void* ws, size_t ws_bytes,
+                               void* stream);
+
 /* ---------------------------------------------------------------------- */
 /* One whole prune step (score + select + compact)                         */
 /* ---------------------------------------------------------------------- */
@@ -305,11 +376,59 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
                      int32_t* n_kept, float* final_score, void* ws, size_t ws_bytes,
                      void* stream);
 
+/*
+ * The same prune step with the cache compacted in place: the kept rows of
+ * unit u end up in rows 0 .. n_kept[u]-1 of k, v and pos themselves, in
+ * temporal order, so one cache buffer serves every step (no ping-pong
+ * destination).  Arguments as in tri_prune with k_dst = k_src = k (likewise v,
+ * pos) and cap_dst = cap_src = cap; k, v and pos must not overlap one
+ * another, and n_kept must not be n_valid (a caller that wants the new count
+ * in place alternates two count arrays).  Served by the pipelined kernel
+ * (its gather stores each piece of destination rows only after every earlier
+ * piece's source rows have been read) or by the split kernels ending in the
+ * in-place compaction of tri_compact_inplace; cfg->path TRI_PATH_FUSED or
+ * TRI_PATH_COOP returns TRI_ERR_UNSUPPORTED.  Workspace:
+ * tri_prune_workspace_bytes.
+ */
+tri_status tri_prune_inplace(const tri_config* cfg, void* k, void* v, int32_t* pos,
+                             tri_dtype dt, int64_t n_seq, int64_t n_layers, int64_t n_kvheads,
+                             int G, int64_t cap, const int32_t* n_valid, const int64_t* p_cur,
+                             const float* stats, int64_t B, int32_t* kept_idx, int32_t* n_kept,
+                             float* final_score, void* ws, size_t ws_bytes, void* stream);
+
 /* The kernel path (TRI_PATH_PIPE, TRI_PATH_COOP, TRI_PATH_FUSED or TRI_PATH_SPLIT) that
- * tri_prune takes for these shapes on the current device when cfg->path is
- * `path`; -1 when `path` cannot serve them or the shapes are invalid. */
+ * tri_prune (inplace = 0) or tri_prune_inplace (inplace = 1) takes for these
+ * shapes on the current device when cfg->path is `path`; -1 when `path`
+ * cannot serve them or the shapes are invalid. */
 int tri_prune_path(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int64_t cap,
-                   int64_t B, tri_dtype dt, int path);
+                   int64_t B, tri_dtype dt, int path, int inplace);
+
+/* ---------------------------------------------------------------------- */
+/* Decode attention over the compacted cache                               */
+/* ---------------------------------------------------------------------- */
+
+size_t tri_decode_workspace_bytes(int64_t n_units, int G, int64_t cap);
+
+/*
+ * Attention of the next token over each unit's kept rows, the softmax
+ * renormalised over them (jaedaily.cn tutorial, KV-compression objective:
+ * the output over the kept subset S is sum_{j in S} a_j v_j with
+ * a_j = exp(s_j) / sum_{j' in S} exp(s_j')):
+ *   out[u][h] = sum_{j < n} a_j v[u][j],  s_j = scale * (q[u][h] . k[u][j]),
+ *   n = n_valid[u] (NULL: cap); a unit with n = 0 gives zeros.
+ *   q: [U][G][head_dim] (dt), the post-RoPE queries of the current token, the
+ *      G query heads of unit u's KV head (unit order as tri_prune).
+ *   k, v: [U][cap][head_dim] (dt), e.g. tri_prune's destination cache.
+ *   scale > 0 (1/sqrt(head_dim) for the usual attention).
+ *   out: [U][G][head_dim] float32.
+ *   ws: tri_decode_workspace_bytes(U, G, cap) bytes (per-chunk partials when
+ *   a unit's keys are split over several CTAs).
+ * Float32 accumulation with an online (running-maximum) softmax.
+ */
+tri_status tri_decode_attention(const void* q, const void* k, const void* v, tri_dtype dt,
+                                int64_t n_units, int G, int64_t cap, int head_dim,
+                                const int32_t* n_valid, float scale, float* out, void* ws,
+                                size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------- */
 /* Streaming helper: append generated tokens                               */

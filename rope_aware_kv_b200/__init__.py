@@ -57,6 +57,8 @@ EXPORTS = (
     "tri_append", "tri_check_device_error",
     "tri_set_timing_events", "tri_last_launch_count", "tri_set_phase_trace",
     "tri_select_topB_static", "tri_select_static_scratch_bytes", "tri_prune_path",
+    "tri_compact_inplace", "tri_prune_inplace", "tri_calibrate_ex",
+    "tri_decode_workspace_bytes", "tri_decode_attention",
 )
 
 
@@ -66,10 +68,18 @@ class TriError(RuntimeError):
         self.code = code
 
 
+VAR_NO_TRIG = 0x1
+VAR_NO_R = 0x2
+VAR_MAX_OFFSET = 0x4
+VAR_HALF_SPLIT = 0x8
+
+
 class TriConfig(ctypes.Structure):
     _fields_ = [("head_dim", ctypes.c_int), ("theta", ctypes.c_double),
                 ("n_offsets", ctypes.c_int), ("offsets", ctypes.c_int64 * MAX_OFFSETS),
-                ("path", ctypes.c_int)]
+                ("path", ctypes.c_int), ("variant", ctypes.c_int),
+                ("n_sink", ctypes.c_int64), ("n_recent", ctypes.c_int64),
+                ("layer_budget", ctypes.c_void_p)]
 
 
 _lib = None
@@ -98,6 +108,11 @@ def load(path: Optional[str] = None):
         "tri_calibrate": (i32, [P, i32, i64, i64, i32, P, P, sz, P]),
         "tri_calibrate_sums": (i32, [P, i32, i64, i64, i32, P, P, sz, P]),
         "tri_calibrate_finish": (i32, [P, i64, i64, i32, P, P]),
+        "tri_decode_workspace_bytes": (sz, [i64, i32, i64]),
+        "tri_decode_attention": (i32, [P, P, P, i32, i64, i32, i64, i32, P, ctypes.c_float, P, P,
+                                       sz, P]),
+        "tri_calibrate_ex": (i32, [ctypes.POINTER(TriConfig), P, i32, i64, i64, i32, P, P, P, sz,
+                                   P]),
         "tri_score_workspace_bytes": (sz, [i64, i64, i64, i32, i64, i32]),
         "tri_score": (i32, [ctypes.POINTER(TriConfig), P, i32, i64, i64, i64, i32, i64, P, P, P, P,
                             P, P, sz, P]),
@@ -115,7 +130,10 @@ def load(path: Optional[str] = None):
         "tri_set_phase_trace": (i32, [P, sz]),
         "tri_select_topB_static": (i32, [P, i64, i64, P, i64, P, P, P]),
         "tri_select_static_scratch_bytes": (sz, []),
-        "tri_prune_path": (i32, [i64, i64, i64, i32, i64, i64, i32, i32]),
+        "tri_prune_path": (i32, [i64, i64, i64, i32, i64, i64, i32, i32, i32]),
+        "tri_compact_inplace": (i32, [P, P, P, i32, i64, i64, i32, P, P, i64, P, sz, P]),
+        "tri_prune_inplace": (i32, [ctypes.POINTER(TriConfig), P, P, P, i32, i64, i64, i64, i32,
+                                    i64, P, P, P, i64, P, P, P, P, sz, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -159,11 +177,24 @@ def _check(fn: str, code: int):
 
 
 def config(theta: float = 10000.0, offsets: Optional[Sequence[int]] = None,
-           head_dim: int = HEAD_DIM, path: int = PATH_AUTO) -> TriConfig:
+           head_dim: int = HEAD_DIM, path: int = PATH_AUTO, variant: int = 0,
+           n_sink: int = 0, n_recent: int = 0,
+           layer_budget: Optional[torch.Tensor] = None) -> TriConfig:
+    """Method parameters (tri.h: tri_config).  ``variant``: VAR_* bits;
+    ``n_sink`` / ``n_recent``: protected first / last keys of every unit;
+    ``layer_budget``: int32 CUDA tensor [n_layers] of per-layer budgets (the
+    config keeps its pointer only: keep the tensor alive while it is used)."""
     cfg = TriConfig()
     load().tri_config_default(ctypes.byref(cfg), head_dim)
     cfg.theta = float(theta)
     cfg.path = int(path)
+    cfg.variant = int(variant)
+    cfg.n_sink = int(n_sink)
+    cfg.n_recent = int(n_recent)
+    if layer_budget is not None:
+        if layer_budget.dtype != torch.int32 or not layer_budget.is_cuda:
+            raise TypeError("layer_budget must be an int32 CUDA tensor")
+        cfg.layer_budget = layer_budget.data_ptr()
     if offsets is not None:
         offs = list(offsets)
         if not 1 <= len(offs) <= MAX_OFFSETS:
@@ -201,6 +232,26 @@ def tri_calibrate(q_pre: torch.Tensor, stats: Optional[torch.Tensor] = None,
         ws = workspace(need, q_pre.device)
     _check("tri_calibrate", load().tri_calibrate(_ptr(q_pre), _dt(q_pre), H, n_tok, d, _ptr(stats),
                                                 _ptr(ws), ws.numel(), _stream(stream)))
+    return stats
+
+
+def tri_calibrate_ex(cfg: TriConfig, q: torch.Tensor, q_pos: Optional[torch.Tensor] = None,
+                     stats: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """Calibration with the config's band pairing; with ``q_pos`` ([n_tok]
+    int32 positions) q holds post-RoPE rows that are rotated back first.
+    q [..., n_tok, d] -> stats [..., d/2, 4] float32."""
+    *lead, n_tok, d = q.shape
+    H = 1
+    for x in lead:
+        H *= x
+    if stats is None:
+        stats = torch.empty((*lead, d // 2, 4), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = workspace(tri_calibrate_workspace_bytes(H, n_tok, d), q.device)
+    _check("tri_calibrate_ex", load().tri_calibrate_ex(
+        ctypes.byref(cfg), _ptr(q), _dt(q), H, n_tok, d, _ptr(q_pos), _ptr(stats), _ptr(ws),
+        ws.numel(), _stream(stream)))
     return stats
 
 
@@ -325,15 +376,30 @@ def tri_compact(k_src: torch.Tensor, v_src: Optional[torch.Tensor], pos_src: Opt
         _stream(stream)))
 
 
+def tri_compact_inplace(k: torch.Tensor, v: Optional[torch.Tensor], pos: Optional[torch.Tensor],
+                        kept: torch.Tensor, n_kept: torch.Tensor,
+                        ws: Optional[torch.Tensor] = None, stream=None):
+    """Move row kept[u][r] to row r of the same buffers (r < n_kept[u])."""
+    U, cap, d = k.shape
+    B = kept.shape[1]
+    if ws is None:
+        ws = workspace(load().tri_compact_workspace_bytes(), k.device)
+    _check("tri_compact_inplace", load().tri_compact_inplace(
+        _ptr(k), _ptr(v), _ptr(pos), _dt(k), U, cap, d, _ptr(kept), _ptr(n_kept), B, _ptr(ws),
+        ws.numel(), _stream(stream)))
+
+
 def tri_prune_workspace_bytes(n_seq, n_layers, n_kvheads, G, cap, B, head_dim=HEAD_DIM) -> int:
     return load().tri_prune_workspace_bytes(n_seq, n_layers, n_kvheads, G, cap, B, head_dim)
 
 
 def tri_prune_path(n_seq, n_layers, n_kvheads, G, cap, B, dtype=torch.bfloat16,
-                   path: int = PATH_AUTO) -> int:
-    """Kernel path tri_prune takes for these shapes (PATH_PIPE / COOP / FUSED / SPLIT)."""
+                   path: int = PATH_AUTO, inplace: bool = False) -> int:
+    """Kernel path tri_prune (or tri_prune_inplace) takes for these shapes
+    (PATH_PIPE / COOP / FUSED / SPLIT; -1 if none)."""
     dt = TRI_BF16 if dtype == torch.bfloat16 else TRI_F32
-    return int(load().tri_prune_path(n_seq, n_layers, n_kvheads, G, cap, B, dt, path))
+    return int(load().tri_prune_path(n_seq, n_layers, n_kvheads, G, cap, B, dt, path,
+                                     1 if inplace else 0))
 
 
 def tri_prune(cfg: TriConfig, k_src: torch.Tensor, v_src: Optional[torch.Tensor],
@@ -356,6 +422,43 @@ def tri_prune(cfg: TriConfig, k_src: torch.Tensor, v_src: Optional[torch.Tensor]
         n_kvheads, G, cap_src, _ptr(n_valid), _ptr(p_cur), _ptr(stats), B, _ptr(k_dst), _ptr(v_dst),
         _ptr(pos_dst), cap_dst, _ptr(kept), _ptr(n_kept), _ptr(final), _ptr(ws), ws.numel(),
         _stream(stream)))
+
+
+def tri_prune_inplace(cfg: TriConfig, k: torch.Tensor, v: Optional[torch.Tensor],
+                      pos: Optional[torch.Tensor], n_seq: int, n_layers: int, n_kvheads: int,
+                      G: int, p_cur: torch.Tensor, stats: torch.Tensor, B: int,
+                      n_kept: torch.Tensor, n_valid: Optional[torch.Tensor] = None,
+                      kept: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                      stream=None, final: Optional[torch.Tensor] = None):
+    """One prune step that compacts the cache in place (kept rows move to the
+    front of k, v and pos in temporal order)."""
+    U, cap, d = k.shape
+    if ws is None:
+        ws = workspace(tri_prune_workspace_bytes(n_seq, n_layers, n_kvheads, G, cap, B, d),
+                       k.device)
+    _check("tri_prune_inplace", load().tri_prune_inplace(
+        ctypes.byref(cfg), _ptr(k), _ptr(v), _ptr(pos), _dt(k), n_seq, n_layers, n_kvheads, G,
+        cap, _ptr(n_valid), _ptr(p_cur), _ptr(stats), B, _ptr(kept), _ptr(n_kept), _ptr(final),
+        _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def tri_decode_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                         n_valid: Optional[torch.Tensor] = None, scale: Optional[float] = None,
+                         out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """Attention of one query token per head over each unit's first n_valid
+    cache rows: q [U, G, d], k / v [U, cap, d] -> out [U, G, d] float32."""
+    U, G, d = q.shape
+    cap = k.shape[1]
+    if out is None:
+        out = torch.empty((U, G, d), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = workspace(load().tri_decode_workspace_bytes(U, G, cap), q.device)
+    sc = (1.0 / d ** 0.5) if scale is None else float(scale)
+    _check("tri_decode_attention", load().tri_decode_attention(
+        _ptr(q), _ptr(k), _ptr(v), _dt(q), U, G, cap, d, _ptr(n_valid), ctypes.c_float(sc),
+        _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
 
 
 def tri_append(k_cache, v_cache, pos_cache, n_seq: int, n_valid: torch.Tensor,

@@ -97,6 +97,16 @@ bool gather_buffers_overlap(const void* k_src, const void* v_src, const void* po
     return false;
 }
 
+// The three in-place buffers (K, V, positions; V and positions nullable)
+// must be disjoint.
+bool inplace_buffers_overlap(const void* k, const void* v, const void* pos, int64_t n_units,
+                             int64_t cap, size_t esz) {
+    const size_t kb = static_cast<size_t>(n_units * cap) * kD * esz;
+    const size_t pb = static_cast<size_t>(n_units * cap) * 4;
+    return (v && overlaps(k, kb, v, kb)) || (pos && overlaps(k, kb, pos, pb)) ||
+           (v && pos && overlaps(v, kb, pos, pb));
+}
+
 struct Carve {
     size_t off = kWsHeader;
     size_t take(size_t bytes) {
@@ -187,6 +197,9 @@ tri_status check_cfg(const tri_config* cfg, FoldOffsets* off) {
     if (!(cfg->theta > 1.0) || cfg->n_offsets < 1 || cfg->n_offsets > TRI_MAX_OFFSETS)
         return TRI_ERR_INVALID_ARG;
     if (cfg->path < TRI_PATH_AUTO || cfg->path > TRI_PATH_PIPE) return TRI_ERR_INVALID_ARG;
+    if ((cfg->variant & ~TRI_VAR_ALL) != 0 || cfg->n_sink < 0 || cfg->n_recent < 0)
+        return TRI_ERR_INVALID_ARG;
+    if (cfg->layer_budget && !aligned4(cfg->layer_budget)) return TRI_ERR_INVALID_ARG;
     off->n = cfg->n_offsets;
     for (int i = 0; i < cfg->n_offsets; ++i) {
         if (cfg->offsets[i] < 0) return TRI_ERR_INVALID_ARG;
@@ -212,6 +225,7 @@ FoldConst fold_const(const tri_config* cfg) {
         fc.cf[f][0] = cre / cfg->n_offsets;
         fc.cf[f][1] = cim / cfg->n_offsets;
     }
+    fc.variant = cfg->variant;
     return fc;
 }
 
@@ -272,6 +286,7 @@ struct PruneWs {
     PipePlan pp;
     size_t queue = 0, counters = 0, wts = 0, raw = 0, fin_scratch = 0;
     size_t zcand = 0, zcount = 0, zstate = 0;  // split path: z-bin selection
+    size_t ub = 0;                             // per-unit budgets (per-layer budgets given)
     ScoreWs sc;
     size_t fin = 0, kept = 0;
     SelectWs sel;
@@ -358,14 +373,35 @@ PipePlan pipe_plan(tri_dtype dt, int G, int64_t U, int64_t cap, int64_t B) {
     return p;
 }
 
+// Which kernel paths can serve a call: 0 every path; 1 the pipelined and
+// split paths (protected keys, per-layer budgets, in-place compaction); 2
+// the split path alone (the max-over-offsets and half-split scores).
+enum { kAnyPath = 0, kPipeOrSplit = 1, kSplitOnly = 2 };
+
+int path_restriction(const tri_config* cfg, bool inplace) {
+    if (cfg->variant & (TRI_VAR_MAX_OFFSET | TRI_VAR_HALF_SPLIT)) return kSplitOnly;
+    if (cfg->n_sink > 0 || cfg->n_recent > 0 || cfg->layer_budget || inplace) return kPipeOrSplit;
+    return kAnyPath;
+}
+
+// In place (destination = source) only the pipelined kernel with one
+// engine warp (pieces stored in order) and the split path (in-place
+// compaction kernel) serve.
 PruneWs prune_ws(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int64_t cap,
-                 int64_t B, tri_dtype dt, bool own_kept, int path) {
+                 int64_t B, tri_dtype dt, bool own_kept, int path, bool inplace = false,
+                 int restrict_to = kAnyPath) {
     PruneWs w;
     const int64_t U = n_seq * n_layers * n_kvheads;
     const int64_t sms = sm_count_or_default();
-    if (path == TRI_PATH_PIPE || path == TRI_PATH_AUTO) {
-        const PipePlan pp = pipe_plan(dt, G, U, cap, B);
-        const CoopPlan cp0 = path == TRI_PATH_AUTO ? coop_plan(dt, G, U, cap) : CoopPlan();
+    if (inplace && restrict_to < kPipeOrSplit) restrict_to = kPipeOrSplit;
+    if (restrict_to >= kPipeOrSplit && (path == TRI_PATH_FUSED || path == TRI_PATH_COOP)) return w;
+    if (restrict_to >= kSplitOnly && path == TRI_PATH_PIPE) return w;
+    if ((path == TRI_PATH_PIPE || path == TRI_PATH_AUTO) && restrict_to < kSplitOnly) {
+        PipePlan pp = pipe_plan(dt, G, U, cap, B);
+        if (inplace && pipe_engine_warps() != 1) pp.ok = false;
+        const CoopPlan cp0 = path == TRI_PATH_AUTO && restrict_to == kAnyPath
+                                 ? coop_plan(dt, G, U, cap)
+                                 : CoopPlan();
         // AUTO takes the pipelined kernel for units that fit one CTA (whole
         // units per CTA); units scored in chunks run faster on the split
         // kernels.
@@ -377,6 +413,7 @@ PruneWs prune_ws(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int6
             w.queue = c.take(4);
             w.counters = c.take(static_cast<size_t>(U) * 4);
             w.zero_end = c.off;
+            w.ub = c.take(static_cast<size_t>(U) * 4);
             // Score rows are padded to a multiple of 32 keys (16-byte groups).
             const int64_t capP = (cap + 31) & ~int64_t(31);
             if (pp.big) {
@@ -393,9 +430,9 @@ PruneWs prune_ws(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int6
         }
         if (path == TRI_PATH_PIPE) return w;  // not possible: tri_prune reports it
     }
-    const bool fused_ok = path != TRI_PATH_SPLIT && path != TRI_PATH_COOP &&
-                          use_fused(dt, G, cap, B, path);
-    const CoopPlan cp = (path == TRI_PATH_AUTO || path == TRI_PATH_COOP)
+    const bool fused_ok = restrict_to == kAnyPath && path != TRI_PATH_SPLIT &&
+                          path != TRI_PATH_COOP && use_fused(dt, G, cap, B, path);
+    const CoopPlan cp = restrict_to == kAnyPath && (path == TRI_PATH_AUTO || path == TRI_PATH_COOP)
                             ? coop_plan(dt, G, U, cap)
                             : CoopPlan();
     const bool want_coop =
@@ -440,8 +477,26 @@ PruneWs prune_ws(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int6
     w.zcand = c.take(static_cast<size_t>(U) * kCandMax * 8);
     w.zcount = c.take(static_cast<size_t>(U) * 4);
     w.zstate = c.take(static_cast<size_t>(U) * zsel_state_bytes());
+    w.ub = c.take(static_cast<size_t>(U) * 4);
     w.total = c.off;
     return w;
+}
+
+// Per-head raw scores and their moments (mean, 1/sigma): the TMA score
+// kernel, or for the max-over-offsets / half-split variants the variant
+// score kernel followed by the moments kernel.
+cudaError_t score_any(const tri_config* cfg, const FoldOffsets& off, tri_dtype dt, int G,
+                      const CUtensorMap& map, const ScoreArgs& a, const float* stats,
+                      const int64_t* p_cur, int64_t n_layers, int64_t n_kvheads, int n_sm,
+                      cudaStream_t s) {
+    if (cfg->variant & (TRI_VAR_MAX_OFFSET | TRI_VAR_HALF_SPLIT)) {
+        cudaError_t e = launch_variant_score(dt, G, a.keys, a.n_units, a.cap, a.n_valid, a.wts,
+                                             stats, p_cur, n_layers, n_kvheads, cfg->theta, off,
+                                             cfg->variant, a.raw, a.flag, s);
+        if (e != cudaSuccess) return e;
+        return launch_moments(a.raw, a.n_units, a.cap, a.n_valid, G, a.mom, s);
+    }
+    return launch_score(dt, G, map, a, n_sm, s);
 }
 
 // Every exported call that launches kernels starts a fresh launch count.
@@ -504,6 +559,25 @@ tri_status tri_calibrate(const void* q_pre, tri_dtype dt, int64_t n_heads, int64
     return cuda_status(launch_calibrate(q_pre, dt, n_heads, n_tok, stats, ws, s));
 }
 
+tri_status tri_calibrate_ex(const tri_config* cfg, const void* q, tri_dtype dt, int64_t n_heads,
+                            int64_t n_tok, int head_dim, const int32_t* q_pos, float* stats,
+                            void* ws, size_t ws_bytes, void* stream) {
+    LaunchScope scope_;
+    FoldOffsets off;
+    TRI_TRY(check_cfg(cfg, &off));
+    if (!q || !stats || n_heads < 1 || n_tok < 1) return TRI_ERR_INVALID_ARG;
+    if (!dtype_ok(dt)) return TRI_ERR_UNSUPPORTED;
+    if (head_dim != kD) return TRI_ERR_UNSUPPORTED;
+    if (n_heads > 65535) return TRI_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned4(stats) || (q_pos && !aligned4(q_pos))) return TRI_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < calibrate_ws_bytes(n_heads, n_tok) || !aligned16(ws))
+        return TRI_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    TRI_CUDA(cudaMemsetAsync(ws, 0, kWsHeader, s));
+    return cuda_status(launch_calibrate(q, dt, n_heads, n_tok, stats, ws, s, q_pos,
+                                        (cfg->variant & TRI_VAR_HALF_SPLIT) ? 1 : 0, cfg->theta));
+}
+
 tri_status tri_calibrate_sums(const void* q_pre, tri_dtype dt, int64_t n_heads, int64_t n_tok,
                               int head_dim, double* sums, void* ws, size_t ws_bytes,
                               void* stream) {
@@ -564,7 +638,8 @@ tri_status tri_score(const tri_config* cfg, const void* k_post, tri_dtype dt, in
     TRI_CUDA(cudaMemsetAsync(ws, 0, kWsHeader, s));
     TRI_CUDA(cudaMemsetAsync(ws_at(ws, w.counters), 0, static_cast<size_t>(U) * 4, s));
     float* wts = reinterpret_cast<float*>(ws_at(ws, w.wts));
-    TRI_CUDA(launch_fold(stats, p_cur, n_seq, n_layers, n_kvheads * G, cfg->theta, off, wts, s));
+    TRI_CUDA(launch_fold(stats, p_cur, n_seq, n_layers, n_kvheads * G, cfg->theta, off,
+                         cfg->variant, wts, s));
     ScoreArgs a;
     a.keys = k_post;
     a.n_units = U;
@@ -577,8 +652,10 @@ tri_status tri_score(const tri_config* cfg, const void* k_post, tri_dtype dt, in
     a.counters = reinterpret_cast<uint32_t*>(ws_at(ws, w.counters));
     a.mom = reinterpret_cast<float2*>(ws_at(ws, w.mom));
     a.flag = ws_flag(ws);
-    TRI_CUDA(launch_score(dt, G, map, a, device_info().sm_count, s));
-    TRI_CUDA(launch_zmax(G, a.raw, U, cap, n_valid, a.mom, final_score, nullptr, 0, a.flag, s));
+    TRI_CUDA(score_any(cfg, off, dt, G, map, a, stats, p_cur, n_layers, n_kvheads,
+                       device_info().sm_count, s));
+    TRI_CUDA(launch_zmax(G, a.raw, U, cap, n_valid, a.mom, final_score, nullptr, 0, cfg->n_sink,
+                         cfg->n_recent, a.flag, s));
     return TRI_OK;
 }
 
@@ -639,6 +716,25 @@ tri_status tri_compact(const void* k_src, const void* v_src, const int32_t* pos_
                                      device_info().sm_count * 8, s));
 }
 
+tri_status tri_compact_inplace(void* k, void* v, int32_t* pos, tri_dtype dt, int64_t n_units,
+                               int64_t cap, int head_dim, const int32_t* kept_idx,
+                               const int32_t* n_kept, int64_t B, void* ws, size_t ws_bytes,
+                               void* stream) {
+    LaunchScope scope_;
+    if (!k || !kept_idx || !n_kept || n_units < 1 || cap < 1 || B < 1) return TRI_ERR_INVALID_ARG;
+    if (!dtype_ok(dt) || head_dim != kD) return TRI_ERR_UNSUPPORTED;
+    if (!aligned16(k) || (v && !aligned16(v)) || (pos && !aligned4(pos)) || !aligned4(kept_idx) ||
+        !aligned4(n_kept))
+        return TRI_ERR_INVALID_ARG;
+    const size_t esz = dt == TRI_BF16 ? 2 : 4;
+    if (inplace_buffers_overlap(k, v, pos, n_units, cap, esz)) return TRI_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < kWsHeader || !aligned16(ws)) return TRI_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    TRI_CUDA(cudaMemsetAsync(ws, 0, kWsHeader, s));
+    return cuda_status(launch_compact_inplace(dt, k, v, pos, n_units, cap, kept_idx, n_kept, B,
+                                              ws_flag(ws), device_info().sm_count * 8, s));
+}
+
 size_t tri_prune_workspace_bytes(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G,
                                  int64_t cap, int64_t B, int head_dim) {
     (void)head_dim;
@@ -655,10 +751,10 @@ size_t tri_prune_workspace_bytes(int64_t n_seq, int64_t n_layers, int64_t n_kvhe
 }
 
 int tri_prune_path(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int64_t cap,
-                   int64_t B, tri_dtype dt, int path) {
+                   int64_t B, tri_dtype dt, int path, int inplace) {
     if (check_units(n_seq, n_layers, n_kvheads, G, cap) != TRI_OK || B < 1 || !dtype_ok(dt))
         return -1;
-    const PruneWs w = prune_ws(n_seq, n_layers, n_kvheads, G, cap, B, dt, false, path);
+    const PruneWs w = prune_ws(n_seq, n_layers, n_kvheads, G, cap, B, dt, false, path, inplace != 0);
     if (w.pipe) return TRI_PATH_PIPE;
     if (w.coop) return TRI_PATH_COOP;
     if (w.fused) return TRI_PATH_FUSED;
@@ -666,13 +762,16 @@ int tri_prune_path(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, in
     return TRI_PATH_SPLIT;
 }
 
-tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src,
-                     const int32_t* pos_src, tri_dtype dt, int64_t n_seq, int64_t n_layers,
-                     int64_t n_kvheads, int G, int64_t cap_src, const int32_t* n_valid,
-                     const int64_t* p_cur, const float* stats, int64_t B, void* k_dst,
-                     void* v_dst, int32_t* pos_dst, int64_t cap_dst, int32_t* kept_idx,
-                     int32_t* n_kept, float* final_score, void* ws, size_t ws_bytes,
-                     void* stream) {
+// tri_prune and tri_prune_inplace (k_dst == k_src, v_dst == v_src,
+// pos_dst == pos_src, cap_dst == cap_src).
+static tri_status prune_impl(const tri_config* cfg, const void* k_src, const void* v_src,
+                             const int32_t* pos_src, tri_dtype dt, int64_t n_seq,
+                             int64_t n_layers, int64_t n_kvheads, int G, int64_t cap_src,
+                             const int32_t* n_valid, const int64_t* p_cur, const float* stats,
+                             int64_t B, void* k_dst, void* v_dst, int32_t* pos_dst,
+                             int64_t cap_dst, int32_t* kept_idx, int32_t* n_kept,
+                             float* final_score, void* ws, size_t ws_bytes, void* stream,
+                             bool inplace) {
     LaunchScope scope_;
     FoldOffsets off;
     TRI_TRY(check_cfg(cfg, &off));
@@ -690,19 +789,31 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
         return TRI_ERR_INVALID_ARG;
     const int64_t U = n_seq * n_layers * n_kvheads;
     const size_t esz = dt == TRI_BF16 ? 2 : 4;
-    if (gather_buffers_overlap(k_src, v_src, pos_src, k_dst, v_dst, pos_dst, U, cap_src, cap_dst,
-                               esz))
+    if (inplace) {
+        if (inplace_buffers_overlap(k_src, v_src, pos_src, U, cap_src, esz) ||
+            (n_valid && static_cast<const void*>(n_valid) == static_cast<const void*>(n_kept)))
+            return TRI_ERR_INVALID_ARG;
+    } else if (gather_buffers_overlap(k_src, v_src, pos_src, k_dst, v_dst, pos_dst, U, cap_src,
+                                      cap_dst, esz)) {
         return TRI_ERR_INVALID_ARG;
-    const PruneWs w =
-        prune_ws(n_seq, n_layers, n_kvheads, G, cap_src, B, dt, kept_idx == nullptr, cfg->path);
+    }
+    const int restrict_to = path_restriction(cfg, inplace);
+    const PruneWs w = prune_ws(n_seq, n_layers, n_kvheads, G, cap_src, B, dt, kept_idx == nullptr,
+                               cfg->path, inplace, restrict_to);
     if (cfg->path == TRI_PATH_FUSED && !w.fused) return TRI_ERR_UNSUPPORTED;
     if (cfg->path == TRI_PATH_COOP && !w.coop) return TRI_ERR_UNSUPPORTED;
     if (cfg->path == TRI_PATH_PIPE && !w.pipe) return TRI_ERR_UNSUPPORTED;
+    if (restrict_to >= kPipeOrSplit && (cfg->path == TRI_PATH_FUSED || cfg->path == TRI_PATH_COOP))
+        return TRI_ERR_UNSUPPORTED;
+    if (restrict_to >= kSplitOnly && cfg->path == TRI_PATH_PIPE) return TRI_ERR_UNSUPPORTED;
     if (!ws || !aligned16(ws) || ws_bytes < w.total) return TRI_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     float* wts = reinterpret_cast<float*>(ws_at(ws, w.sc.wts));
     int32_t* kept = kept_idx ? kept_idx : reinterpret_cast<int32_t*>(ws_at(ws, w.kept));
     uint32_t* flag = ws_flag(ws);
+    int32_t* ub = cfg->layer_budget ? reinterpret_cast<int32_t*>(ws_at(ws, w.ub)) : nullptr;
+    if (ub)
+        TRI_CUDA(launch_unit_budget(cfg->layer_budget, U, n_layers, n_kvheads, ub, s));
 
     if (w.pipe) {
         CUtensorMap map;
@@ -729,6 +840,10 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
         a.k_dst = k_dst;
         a.v_dst = v_dst;
         a.pos_dst = pos_dst;
+        a.inplace = inplace ? 1 : 0;
+        a.n_sink = cfg->n_sink;
+        a.n_recent = cfg->n_recent;
+        a.ub = ub;
         a.kept = kept_idx;
         a.n_kept = n_kept;
         a.final_out = final_score;
@@ -741,7 +856,7 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
         a.flag = flag;
         if (w.pp.big) {
             float* pw = reinterpret_cast<float*>(ws_at(ws, w.wts));
-            TRI_CUDA(launch_fold(stats, p_cur, n_seq, n_layers, n_kvheads * G, cfg->theta, off, pw,
+            TRI_CUDA(launch_fold(stats, p_cur, n_seq, n_layers, n_kvheads * G, cfg->theta, off, cfg->variant, pw,
                                  s));
             a.wts = pw;
         }
@@ -828,7 +943,8 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
     TRI_CUDA(cudaMemsetAsync(ws_at(ws, w.sc.counters), 0, static_cast<size_t>(U) * 4, s));
     TRI_CUDA(cudaMemsetAsync(ws_at(ws, w.sel.hists), 0, w.sel.counts - w.sel.hists, s));
     TRI_CUDA(cudaMemsetAsync(ws_at(ws, w.zcount), 0, static_cast<size_t>(U) * 4, s));
-    TRI_CUDA(launch_fold(stats, p_cur, n_seq, n_layers, n_kvheads * G, cfg->theta, off, wts, s));
+    TRI_CUDA(launch_fold(stats, p_cur, n_seq, n_layers, n_kvheads * G, cfg->theta, off,
+                         cfg->variant, wts, s));
     ScoreArgs a;
     a.keys = k_src;
     a.n_units = U;
@@ -842,17 +958,70 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
     a.mom = reinterpret_cast<float2*>(ws_at(ws, w.sc.mom));
     a.flag = flag;
     const int n_sm = device_info().sm_count;
-    TRI_CUDA(launch_score(dt, G, map, a, n_sm, s));
+    TRI_CUDA(score_any(cfg, off, dt, G, map, a, stats, p_cur, n_layers, n_kvheads, n_sm, s));
     float* fin = final_score ? final_score : reinterpret_cast<float*>(ws_at(ws, w.fin));
     uint32_t* hists = reinterpret_cast<uint32_t*>(ws_at(ws, w.sel.hists));
-    TRI_CUDA(launch_zmax(G, a.raw, U, cap_src, n_valid, a.mom, fin, hists, 1, flag, s));
-    TRI_CUDA(launch_zselect(fin, U, cap_src, n_valid, B, hists,
+    TRI_CUDA(launch_zmax(G, a.raw, U, cap_src, n_valid, a.mom, fin, hists, 1, cfg->n_sink,
+                         cfg->n_recent, flag, s));
+    TRI_CUDA(launch_zselect(fin, U, cap_src, n_valid, B, ub, hists,
                             reinterpret_cast<uint2*>(ws_at(ws, w.sel.counts)),
                             reinterpret_cast<int2*>(ws_at(ws, w.zcand)),
                             reinterpret_cast<uint32_t*>(ws_at(ws, w.zcount)), ws_at(ws, w.zstate), kept,
                             n_kept, s));
+    if (inplace)
+        return cuda_status(launch_compact_inplace(dt, k_dst, v_dst, pos_dst, U, cap_src, kept,
+                                                  n_kept, B, flag, n_sm * 8, s));
     return cuda_status(launch_gather(dt, k_src, v_src, pos_src, U, cap_src, kept, n_kept, B, k_dst,
                                      v_dst, pos_dst, cap_dst, flag, n_sm * 8, s));
+}
+
+tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src,
+                     const int32_t* pos_src, tri_dtype dt, int64_t n_seq, int64_t n_layers,
+                     int64_t n_kvheads, int G, int64_t cap_src, const int32_t* n_valid,
+                     const int64_t* p_cur, const float* stats, int64_t B, void* k_dst,
+                     void* v_dst, int32_t* pos_dst, int64_t cap_dst, int32_t* kept_idx,
+                     int32_t* n_kept, float* final_score, void* ws, size_t ws_bytes,
+                     void* stream) {
+    return prune_impl(cfg, k_src, v_src, pos_src, dt, n_seq, n_layers, n_kvheads, G, cap_src,
+                      n_valid, p_cur, stats, B, k_dst, v_dst, pos_dst, cap_dst, kept_idx, n_kept,
+                      final_score, ws, ws_bytes, stream, false);
+}
+
+tri_status tri_prune_inplace(const tri_config* cfg, void* k, void* v, int32_t* pos,
+                             tri_dtype dt, int64_t n_seq, int64_t n_layers, int64_t n_kvheads,
+                             int G, int64_t cap, const int32_t* n_valid, const int64_t* p_cur,
+                             const float* stats, int64_t B, int32_t* kept_idx, int32_t* n_kept,
+                             float* final_score, void* ws, size_t ws_bytes, void* stream) {
+    return prune_impl(cfg, k, v, pos, dt, n_seq, n_layers, n_kvheads, G, cap, n_valid, p_cur,
+                      stats, B, k, v, pos, cap, kept_idx, n_kept, final_score, ws, ws_bytes,
+                      stream, true);
+}
+
+size_t tri_decode_workspace_bytes(int64_t n_units, int G, int64_t cap) {
+    if (n_units < 1 || cap < 1 || G < 1 || G > TRI_MAX_GROUP) return kWsHeader;
+    return kWsHeader + decode_part_bytes(n_units, G, cap, static_cast<int>(sm_count_or_default()));
+}
+
+tri_status tri_decode_attention(const void* q, const void* k, const void* v, tri_dtype dt,
+                                int64_t n_units, int G, int64_t cap, int head_dim,
+                                const int32_t* n_valid, float scale, float* out, void* ws,
+                                size_t ws_bytes, void* stream) {
+    LaunchScope scope_;
+    if (!q || !k || !v || !out || n_units < 1 || cap < 1 || !(scale > 0.f))
+        return TRI_ERR_INVALID_ARG;
+    if (!dtype_ok(dt) || head_dim != kD || G < 1 || G > TRI_MAX_GROUP) return TRI_ERR_UNSUPPORTED;
+    if (n_units > 65535) return TRI_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        (n_valid && !aligned4(n_valid)))
+        return TRI_ERR_INVALID_ARG;
+    const int n_sm = static_cast<int>(sm_count_or_default());
+    if (!ws || !aligned16(ws) || ws_bytes < kWsHeader + decode_part_bytes(n_units, G, cap, n_sm))
+        return TRI_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    TRI_CUDA(cudaMemsetAsync(ws, 0, kWsHeader, s));
+    return cuda_status(launch_decode(dt, G, q, k, v, n_units, cap, n_valid, scale, out,
+                                     reinterpret_cast<float*>(ws_at(ws, kWsHeader)), ws_flag(ws),
+                                     n_sm, s));
 }
 
 tri_status tri_append(void* k_cache, void* v_cache, int32_t* pos_cache, tri_dtype dt,

@@ -19,29 +19,51 @@ namespace tri {
 constexpr int kCalThreads = 256;   // 4 rows x 64 bands per step
 constexpr int kCalChunk = 1024;    // tokens per CTA
 
+// Options of the extended calibration: post-RoPE queries are rotated back
+// by -w_f p (p the token's position, qpos[t]) before they are averaged, which
+// gives their pre-RoPE bands (shibing624 paper reading, Q/K concentration
+// section: the centres live in the pre-RoPE space); `half` takes band f from
+// components (x_f, x_{f+64}).  Keys calibrated the same way give the K centres.
+struct CalibOpts {
+    const int32_t* qpos = nullptr;  // [n_tok] positions of post-RoPE rows, or null
+    int half = 0;
+    double theta = 10000.0;
+};
+
 template <typename T>
 __global__ void __launch_bounds__(kCalThreads)
 calib_partial_kernel(const T* __restrict__ q, int64_t n_tok, int n_chunks,
-                     double* __restrict__ part) {
+                     double* __restrict__ part, CalibOpts opt) {
     const int f = threadIdx.x & 63;
     const int r = threadIdx.x >> 6;
     const int64_t h = blockIdx.y;
     const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kCalChunk;
     const int64_t t1 = min(t0 + kCalChunk, n_tok);
+    const double w = opt.qpos ? pow(opt.theta, -2.0 * static_cast<double>(f) / kD) : 0.0;
     double sx = 0.0, sy = 0.0, sn = 0.0;
     for (int64_t t = t0 + r; t < t1; t += 4) {
         const T* row = q + (h * n_tok + t) * kD;
         float x, y;
-        if constexpr (sizeof(T) == 2) {
-            const uint32_t w = reinterpret_cast<const uint32_t*>(row)[f];
-            x = bf16_lo(w);
-            y = bf16_hi(w);
+        if (opt.half) {
+            x = to_float(row[f]);
+            y = to_float(row[f + 64]);
+        } else if constexpr (sizeof(T) == 2) {
+            const uint32_t wd = reinterpret_cast<const uint32_t*>(row)[f];
+            x = bf16_lo(wd);
+            y = bf16_hi(wd);
         } else {
             const float2 v = reinterpret_cast<const float2*>(row)[f];
             x = v.x;
             y = v.y;
         }
-        const double dx = x, dy = y;
+        double dx = x, dy = y;
+        if (opt.qpos) {
+            double sa, ca;
+            sincos(w * static_cast<double>(opt.qpos[t]), &sa, &ca);
+            const double rx = ca * dx + sa * dy;
+            dy = -sa * dx + ca * dy;
+            dx = rx;
+        }
         sx += dx;
         sy += dy;
         sn += sqrt(dx * dx + dy * dy);
@@ -129,10 +151,11 @@ cudaError_t launch_calibrate_sums(const void* q, tri_dtype dt, int64_t n_heads, 
     dim3 grid(n_chunks, static_cast<unsigned>(n_heads));
     if (dt == TRI_BF16) {
         calib_partial_kernel<__nv_bfloat16><<<grid, kCalThreads, 0, s>>>(
-            static_cast<const __nv_bfloat16*>(q), n_tok, n_chunks, part);
+            static_cast<const __nv_bfloat16*>(q), n_tok, n_chunks, part, CalibOpts());
     } else {
         calib_partial_kernel<float><<<grid, kCalThreads, 0, s>>>(static_cast<const float*>(q),
-                                                                  n_tok, n_chunks, part);
+                                                                  n_tok, n_chunks, part,
+                                                                  CalibOpts());
     }
     note_launch(s);
     calib_sum_kernel<<<static_cast<unsigned>(n_heads), 64, 0, s>>>(part, n_chunks, sums);
@@ -153,17 +176,22 @@ size_t calibrate_ws_bytes(int64_t n_heads, int64_t n_tok) {
 }
 
 cudaError_t launch_calibrate(const void* q, tri_dtype dt, int64_t n_heads, int64_t n_tok,
-                             float* stats, void* ws, cudaStream_t s) {
+                             float* stats, void* ws, cudaStream_t s, const int32_t* qpos,
+                             int half, double theta) {
     const int n_chunks = static_cast<int>((n_tok + kCalChunk - 1) / kCalChunk);
     double* part = reinterpret_cast<double*>(static_cast<char*>(ws) + kWsHeader);
     dim3 grid(n_chunks, static_cast<unsigned>(n_heads));
+    CalibOpts opt;
+    opt.qpos = qpos;
+    opt.half = half;
+    opt.theta = theta;
     if (dt == TRI_BF16) {
         calib_partial_kernel<__nv_bfloat16><<<grid, kCalThreads, 0, s>>>(
-            static_cast<const __nv_bfloat16*>(q), n_tok, n_chunks, part);
+            static_cast<const __nv_bfloat16*>(q), n_tok, n_chunks, part, opt);
         note_launch(s);
     } else {
         calib_partial_kernel<float><<<grid, kCalThreads, 0, s>>>(static_cast<const float*>(q),
-                                                                  n_tok, n_chunks, part);
+                                                                  n_tok, n_chunks, part, opt);
         note_launch(s);
     }
     calib_merge_kernel<<<static_cast<unsigned>(n_heads), 64, 0, s>>>(part, n_chunks, n_tok, stats);

@@ -101,6 +101,101 @@ cudaError_t launch_gather(tri_dtype dt, const void* k_src, const void* v_src,
 }
 
 // ---------------------------------------------------------------------------
+// In-place compaction: row kept[u][r] moves to row r of the same buffer, for
+// r < n_kept[u] (the same bit copies as the gather, without a second cache).
+// A kept list is ascending, so kept[r] >= r and rows only move towards the
+// front.  Each CTA walks one unit's rows in rounds of kRows destinations: a
+// round loads every source row it needs into registers, passes a CTA
+// barrier (loads requested before it are performed for every thread of the
+// CTA), then stores.  A round's sources lie at or after its first
+// destination row and its destinations before the next round's first one,
+// so no store lands on a row that a later round still has to read; rows
+// whose source is outside [r, cap) are skipped and flagged.  A round in
+// which every row stays where it is (the prefix before the first dropped
+// row) moves nothing.
+// ---------------------------------------------------------------------------
+template <int kVec>
+__global__ void __launch_bounds__(256)
+compact_inplace_kernel(uint4* __restrict__ k, uint4* __restrict__ v, int32_t* __restrict__ pos,
+                       int64_t n_units, int64_t cap, const int32_t* __restrict__ kept,
+                       const int32_t* __restrict__ n_kept, int64_t B, uint32_t* flag) {
+    constexpr int kThreads = 256;
+    constexpr int kRows = 64;                        // destination rows per round
+    constexpr int kPer = kRows * kVec / kThreads;    // vectors per thread per array
+    static_assert(kRows * kVec % kThreads == 0, "round must split evenly");
+    const int tid = threadIdx.x;
+    const int64_t lim = B < cap ? B : cap;
+    for (int64_t u = blockIdx.x; u < n_units; u += gridDim.x) {
+        int64_t nk = n_kept[u];
+        if (nk > lim || nk < 0) {
+            if (tid == 0) raise_flag(flag, TRI_FLAG_INDEX_RANGE);
+            nk = nk < 0 ? 0 : lim;
+        }
+        const int32_t* ku = kept + u * B;
+        for (int64_t r0 = 0; r0 < nk; r0 += kRows) {
+            // Source row of each destination row this thread moves (-1: none).
+            int64_t src[kPer];
+            bool still = true;
+#pragma unroll
+            for (int q = 0; q < kPer; ++q) {
+                const int64_t r = r0 + (tid + q * kThreads) / kVec;
+                src[q] = -1;
+                if (r < nk) {
+                    const int64_t j = ku[r];
+                    if (j >= r && j < cap) {
+                        src[q] = j;
+                        still = still && j == r;
+                    } else if ((tid + q * kThreads) % kVec == 0) {
+                        raise_flag(flag, TRI_FLAG_INDEX_RANGE);
+                    }
+                }
+            }
+            if (__syncthreads_and(still)) continue;
+            const int lane = tid % kVec;
+            uint4 kv[kPer], vv[kPer];
+            int32_t pv[kPer];
+#pragma unroll
+            for (int q = 0; q < kPer; ++q) {
+                if (src[q] >= 0) {
+                    kv[q] = k[(u * cap + src[q]) * kVec + lane];
+                    if (v) vv[q] = v[(u * cap + src[q]) * kVec + lane];
+                    if (pos && lane == 0) pv[q] = pos[u * cap + src[q]];
+                }
+            }
+            __syncthreads();
+#pragma unroll
+            for (int q = 0; q < kPer; ++q) {
+                if (src[q] >= 0) {
+                    const int64_t r = r0 + (tid + q * kThreads) / kVec;
+                    k[(u * cap + r) * kVec + lane] = kv[q];
+                    if (v) v[(u * cap + r) * kVec + lane] = vv[q];
+                    if (pos && lane == 0) pos[u * cap + r] = pv[q];
+                }
+            }
+        }
+        __syncthreads();
+    }
+}
+
+cudaError_t launch_compact_inplace(tri_dtype dt, void* k, void* v, int32_t* pos, int64_t n_units,
+                                   int64_t cap, const int32_t* kept, const int32_t* n_kept,
+                                   int64_t B, uint32_t* flag, int n_blocks, cudaStream_t s) {
+    if (n_units == 0) return cudaSuccess;
+    const int grid = static_cast<int>(n_units < n_blocks ? n_units : n_blocks);
+    if (dt == TRI_BF16) {
+        compact_inplace_kernel<kD * 2 / 16><<<grid, 256, 0, s>>>(
+            static_cast<uint4*>(k), static_cast<uint4*>(v), pos, n_units, cap, kept, n_kept, B,
+            flag);
+    } else {
+        compact_inplace_kernel<kD * 4 / 16><<<grid, 256, 0, s>>>(
+            static_cast<uint4*>(k), static_cast<uint4*>(v), pos, n_units, cap, kept, n_kept, B,
+            flag);
+    }
+    note_launch(s);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // Append n_new rows per unit at rows n_valid[u] .. n_valid[u] + n_new - 1.
 // One CTA per unit; the new position count and p_cur are written by thread 0
 // after every thread has read n_valid.

@@ -2,7 +2,9 @@
 //
 // A_f = E[q_f] e^{i w_f p_cur} C_f with C_f = (1/|D|) sum_delta e^{i w_f delta}
 // and c_f = (1 - R_f) E|q_f| (talk page: S_trig, S_norm and the
-// offset-averaged S~; the key position cancels, see score.cu).  The
+// offset-averaged S~; the key position cancels, see score.cu); the ablations
+// TRI_VAR_NO_TRIG (A_f = 0) and TRI_VAR_NO_R (c_f = E|q_f|) change only
+// these weights.  The
 // config-only factors w_f and C_f arrive as a kernel parameter (FoldConst);
 // each unit needs 64 phases e^{i w_f p_cur} and G x 64 complex products, all
 // in float64, rounded once to the float32 weight records the score loop reads
@@ -52,9 +54,11 @@ __device__ __forceinline__ void fold_unit_sync(FoldShared& fs, const FoldConst& 
         const double mre = st.x, mim = st.y;
         const double tre = mre * fs.ef[f][0] - mim * fs.ef[f][1];
         const double tim = mre * fs.ef[f][1] + mim * fs.ef[f][0];
-        const double are = tre * fc.cf[f][0] - tim * fc.cf[f][1];
-        const double aim = tre * fc.cf[f][1] + tim * fc.cf[f][0];
-        const double cw = (1.0 - static_cast<double>(st.w)) * static_cast<double>(st.z);
+        const bool trig = (fc.variant & TRI_VAR_NO_TRIG) == 0;
+        const double are = trig ? tre * fc.cf[f][0] - tim * fc.cf[f][1] : 0.0;
+        const double aim = trig ? tre * fc.cf[f][1] + tim * fc.cf[f][0] : 0.0;
+        const double rw = (fc.variant & TRI_VAR_NO_R) ? 1.0 : 1.0 - static_cast<double>(st.w);
+        const double cw = rw * static_cast<double>(st.z);
         float* rec = w + h * kWHead + (f >> 2) * kWChunk;
         const int i = f & 3;
         rec[2 * i] = static_cast<float>(are);

@@ -599,7 +599,7 @@ __device__ __forceinline__ void select_unit(const Fin fin, int n, int64_t B, int
 template <int G, typename Fin>
 __device__ __forceinline__ void zmax_unit(const float* raw, int64_t ldr, int n, const PipeMisc* ms,
                                        const Fin fin, float* final_out, uint32_t* hist,
-                                       uint32_t* flag) {
+                                       int64_t n_sink, int64_t n_recent, uint32_t* flag) {
     using S = PipeShape<float>;
     const int tid = threadIdx.x;
     float mu[G], inv[G];
@@ -633,12 +633,14 @@ __device__ __forceinline__ void zmax_unit(const float* raw, int64_t ldr, int n, 
                     const float z = (f4at(sv[q][h], i) - mu[h]) * inv[h];
                     best[i] = (h == 0) ? z : fmaxf(best[i], z);
                 }
+                if (best[i] != best[i] && 4 * g + i < n) nonfinite = true;
+                // Protected sink / recent keys rank above every score.
+                if (4 * g + i < n_sink || 4 * g + i >= n - n_recent) best[i] = INFINITY;
             }
             fin.put4(4 * g, make_float4(best[0], best[1], best[2], best[3]));
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 if (4 * g + i < n) {
-                    if (best[i] != best[i]) nonfinite = true;
                     atomicAdd(&hist[zbin(best[i])], 1u);
                     if (final_out) final_out[4 * g + i] = best[i];
                 }
@@ -1062,17 +1064,23 @@ prune_pipe_kernel(const __grid_constant__ CUtensorMap kmap, PipeArgs a) {
                 a.kept[u * B + r] = r < m ? static_cast<int32_t>(kx[r]) : -1;
         }
         if (a.pos_src) {
+            // Rounds of kU * kMath rows.  In place, a round's stores may land
+            // on rows the same round reads (never on rows a later round
+            // reads: sources are at or after their destination), so the
+            // round's loads are performed before the barrier, its stores
+            // after it.
             constexpr int kU = 8;
-            for (int r0 = tid; r0 < m; r0 += S::kMath * kU) {
+            for (int b0 = 0; b0 < m; b0 += S::kMath * kU) {
                 int32_t pv[kU];
 #pragma unroll
                 for (int qq = 0; qq < kU; ++qq) {
-                    const int r = r0 + qq * S::kMath;
+                    const int r = b0 + tid + qq * S::kMath;
                     pv[qq] = r < m ? a.pos_src[u * a.cap + kx[r]] : 0;
                 }
+                if (a.inplace) math_sync();
 #pragma unroll
                 for (int qq = 0; qq < kU; ++qq) {
-                    const int r = r0 + qq * S::kMath;
+                    const int r = b0 + tid + qq * S::kMath;
                     if (r < m) a.pos_dst[u * a.cap_dst + r] = pv[qq];
                 }
             }
@@ -1113,9 +1121,10 @@ prune_pipe_kernel(const __grid_constant__ CUtensorMap kmap, PipeArgs a) {
                 break;
             }
             const int n = clamp_nvalid(a.n_valid, u, a.cap, tid == 0 ? a.flag : nullptr);
-            const int m = static_cast<int>(n < B ? n : B);
+            const int64_t Bu = unit_budget(a.ub, u, B);
+            const int m = static_cast<int>(n < Bu ? n : Bu);
             pipe_trace(a, u, 0, warp);
-            if (n > B) {
+            if (n > Bu && Bu > 0) {
                 const int n_tiles = (n + S::kTile - 1) / S::kTile;
                 first_loads(u, 0, n_tiles);
                 fold_unit_sync<G>(fs, a.fc, w, a.stats, a.p_cur, u, a.n_layers, a.n_kvheads, 1,
@@ -1135,17 +1144,19 @@ prune_pipe_kernel(const __grid_constant__ CUtensorMap kmap, PipeArgs a) {
                 for (int b = tid; b < kZBins; b += S::kMath) hist[b] = 0;
                 math_sync();
                 zmax_unit<G>(raw, capP, n, ms, FinShared{fin_s},
-                             a.final_out ? a.final_out + u * a.cap : nullptr, hist, a.flag);
+                             a.final_out ? a.final_out + u * a.cap : nullptr, hist, a.n_sink,
+                             a.n_recent, a.flag);
                 math_sync();
                 pipe_trace(a, u, 2, warp);
                 // This warp's first tile of the next unit into L2.
                 const int64_t un = u + gridDim.x;
                 if (lane == 0 && un < a.n_units) {
                     const int nn = clamp_nvalid(a.n_valid, un, a.cap, nullptr);
-                    if (nn > B) prefetch_tile(un, warp, (nn + S::kTile - 1) / S::kTile);
+                    if (nn > unit_budget(a.ub, un, B))
+                        prefetch_tile(un, warp, (nn + S::kTile - 1) / S::kTile);
                 }
                 const bool ok = handoff(u, m, [&](Idx* kx) {
-                    select_unit(FinShared{fin_s}, n, B, m, hist, cand, ms, kx);
+                    select_unit(FinShared{fin_s}, n, Bu, m, hist, cand, ms, kx);
                 });
                 if (!ok) {
                     failed = true;
@@ -1188,8 +1199,9 @@ prune_pipe_kernel(const __grid_constant__ CUtensorMap kmap, PipeArgs a) {
             const int64_t u = item / cpu;
             const int c = static_cast<int>(item % cpu);
             const int n = clamp_nvalid(a.n_valid, u, a.cap, (tid == 0 && c == 0) ? a.flag : nullptr);
-            const int m = static_cast<int>(n < B ? n : B);
-            if (n <= B) {
+            const int64_t Bu = unit_budget(a.ub, u, B);
+            const int m = static_cast<int>(n < Bu ? n : Bu);
+            if (n <= Bu || Bu == 0) {
                 if (c == 0) {
                     const bool ok = handoff(u, m, [&](Idx* kx) {
                         for (int r = tid; r < m; r += S::kMath) kx[r] = r;
@@ -1222,7 +1234,7 @@ prune_pipe_kernel(const __grid_constant__ CUtensorMap kmap, PipeArgs a) {
                 const int cn = static_cast<int>(next % cpu);
                 const int nn = clamp_nvalid(a.n_valid, un, a.cap, nullptr);
                 const int ntn = (nn + S::kTile - 1) / S::kTile;
-                if (nn > B && cn * kChunkTiles < ntn) {
+                if (nn > unit_budget(a.ub, un, B) && cn * kChunkTiles < ntn) {
                     for (int t = 0; t < S::kMathWarps; ++t)
                         prefetch_tile(un, cn * kChunkTiles + t, min(cn * kChunkTiles + kChunkTiles, ntn));
                     prefetch_l2_bulk(a.wts + un * G * kWHead, G * kWHead * 4, pfpol);
@@ -1274,10 +1286,11 @@ prune_pipe_kernel(const __grid_constant__ CUtensorMap kmap, PipeArgs a) {
             math_sync();
             float* fin_g = a.fin_scratch + static_cast<int64_t>(blockIdx.x) * capP;
             float* fo = a.final_out ? a.final_out + u * a.cap : nullptr;
-            zmax_unit<G>(raw, capP, n, ms, FinGlobal{fin_g}, fo, hist, a.flag);
+            zmax_unit<G>(raw, capP, n, ms, FinGlobal{fin_g}, fo, hist, a.n_sink, a.n_recent,
+                         a.flag);
             math_sync();
             const bool ok = handoff(u, m, [&](Idx* kx) {
-                select_unit(FinGlobal{fin_g}, n, B, m, hist, cand, ms, kx);
+                select_unit(FinGlobal{fin_g}, n, Bu, m, hist, cand, ms, kx);
             });
             if (!ok) {
                 failed = true;

@@ -46,7 +46,7 @@ constexpr int kFoldHeads = 64;
 
 __global__ void __launch_bounds__(256)
 fold_kernel(const float* __restrict__ stats, const int64_t* __restrict__ p_cur, int64_t n_layers,
-            int64_t n_qheads, double theta, FoldOffsets off, float* __restrict__ wts) {
+            int64_t n_qheads, double theta, FoldOffsets off, int variant, float* __restrict__ wts) {
     __shared__ double part[4][kF][2];
     __shared__ double cf[kF][2], ef[kF][2];
     const int t = threadIdx.x;
@@ -87,9 +87,11 @@ fold_kernel(const float* __restrict__ stats, const int64_t* __restrict__ p_cur, 
         const double mre = st[0], mim = st[1];
         const double tre = mre * ef[f][0] - mim * ef[f][1];  // E[q_f] e^{i w p_cur}
         const double tim = mre * ef[f][1] + mim * ef[f][0];
-        const double are = tre * cf[f][0] - tim * cf[f][1];  // ... * C_f
-        const double aim = tre * cf[f][1] + tim * cf[f][0];
-        const double cw = (1.0 - static_cast<double>(st[3])) * static_cast<double>(st[2]);
+        const bool trig = (variant & TRI_VAR_NO_TRIG) == 0;
+        const double are = trig ? tre * cf[f][0] - tim * cf[f][1] : 0.0;  // ... * C_f
+        const double aim = trig ? tre * cf[f][1] + tim * cf[f][0] : 0.0;
+        const double rw = (variant & TRI_VAR_NO_R) ? 1.0 : 1.0 - static_cast<double>(st[3]);
+        const double cw = rw * static_cast<double>(st[2]);
         const int64_t q = seq * LH + lh;  // (seq * L + layer) * Hq + qh
         float* rec = wts + q * kWHead + (f >> 2) * kWChunk;
         const int i = f & 3;
@@ -355,7 +357,7 @@ template <int G>
 __global__ void __launch_bounds__(256)
 zmax_kernel(const float* __restrict__ raw, int64_t cap, const int32_t* __restrict__ n_valid,
             const float2* __restrict__ mom, float* __restrict__ fin, uint32_t* __restrict__ hist0,
-            int zbins, uint32_t* flag) {
+            int zbins, int64_t n_sink, int64_t n_recent, uint32_t* flag) {
     __shared__ uint32_t hist[kHistBins0];
     const int64_t u = blockIdx.y;
     const int n = clamp_nvalid(n_valid, u, cap, nullptr);
@@ -390,8 +392,10 @@ zmax_kernel(const float* __restrict__ raw, int64_t cap, const int32_t* __restric
                 const float z = (sv[i][h] - mu[h]) * inv[h];
                 best = (h == 0) ? z : fmaxf(best, z);
             }
-            fin[u * cap + j] = best;
             if (best != best) nonfinite = true;
+            // Protected sink / recent keys rank above every score.
+            if (j < n_sink || j >= n - n_recent) best = INFINITY;
+            fin[u * cap + j] = best;
             if (hist0) atomicAdd(&hist[zbins ? zbin(best) : (ordered_key(best) >> kShift0)], 1u);
         }
     }
@@ -443,11 +447,11 @@ int score_tile_keys(tri_dtype dt) {
 }
 
 cudaError_t launch_fold(const float* stats, const int64_t* p_cur, int64_t n_seq, int64_t n_layers,
-                        int64_t n_qheads, double theta, const FoldOffsets& off, float* wts,
-                        cudaStream_t s) {
+                        int64_t n_qheads, double theta, const FoldOffsets& off, int variant,
+                        float* wts, cudaStream_t s) {
     const int64_t groups = (n_layers * n_qheads + kFoldHeads - 1) / kFoldHeads;
     dim3 grid(static_cast<unsigned>(n_seq), static_cast<unsigned>(groups));
-    fold_kernel<<<grid, 256, 0, s>>>(stats, p_cur, n_layers, n_qheads, theta, off, wts);
+    fold_kernel<<<grid, 256, 0, s>>>(stats, p_cur, n_layers, n_qheads, theta, off, variant, wts);
     note_launch(s);
     return cudaGetLastError();
 }
@@ -460,11 +464,15 @@ cudaError_t launch_score(tri_dtype dt, int G, const CUtensorMap& map, const Scor
 
 cudaError_t launch_zmax(int G, const float* raw, int64_t n_units, int64_t cap,
                         const int32_t* n_valid, const float2* mom, float* fin, uint32_t* hist0,
-                        int zbins, uint32_t* flag, cudaStream_t s) {
+                        int zbins, int64_t n_sink, int64_t n_recent, uint32_t* flag,
+                        cudaStream_t s) {
     dim3 grid(static_cast<unsigned>((cap + kZChunk - 1) / kZChunk), static_cast<unsigned>(n_units));
     switch (G) {
-#define TRI_ZCASE(g) \
-    case g: zmax_kernel<g><<<grid, 256, 0, s>>>(raw, cap, n_valid, mom, fin, hist0, zbins, flag); break;
+#define TRI_ZCASE(g)                                                                              \
+    case g:                                                                                       \
+        zmax_kernel<g><<<grid, 256, 0, s>>>(raw, cap, n_valid, mom, fin, hist0, zbins, n_sink,    \
+                                            n_recent, flag);                                      \
+        break;
         TRI_ZCASE(1) TRI_ZCASE(2) TRI_ZCASE(3) TRI_ZCASE(4)
         TRI_ZCASE(5) TRI_ZCASE(6) TRI_ZCASE(7) TRI_ZCASE(8)
 #undef TRI_ZCASE

@@ -266,6 +266,8 @@ __device__ __forceinline__ float sqrt_approx(float x) {
 // bf16 pair in one 32-bit word: low half is the even element.
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ float to_float(float x) { return x; }
+__device__ __forceinline__ float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
 
 __device__ __forceinline__ int clamp_nvalid(const int32_t* n_valid, int64_t u, int64_t cap,
                                             uint32_t* flag) {
@@ -276,6 +278,13 @@ __device__ __forceinline__ int clamp_nvalid(const int32_t* n_valid, int64_t u, i
         n = n < 0 ? 0 : static_cast<int>(cap);
     }
     return n;
+}
+
+// Budget of unit u: the per-unit budget array, clamped to [0, B], or B.
+__device__ __forceinline__ int64_t unit_budget(const int32_t* ub, int64_t u, int64_t B) {
+    if (!ub) return B;
+    const int64_t b = ub[u];
+    return b < 0 ? 0 : (b > B ? B : b);
 }
 
 }  // namespace tri

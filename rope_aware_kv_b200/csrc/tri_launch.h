@@ -25,6 +25,7 @@ struct FoldOffsets {
 struct FoldConst {
     double omega[64];
     double cf[64][2];
+    int variant;  // TRI_VAR_* bits (the fold applies NO_TRIG and NO_R)
 };
 
 // Static shared memory of the fused and cooperative kernels (the fold's
@@ -93,6 +94,10 @@ struct PipeArgs {
     void* k_dst;
     void* v_dst;
     int32_t* pos_dst;
+    int inplace;                 // destinations are the sources (cap_dst == cap)
+    int64_t n_sink;              // protected first keys of every unit
+    int64_t n_recent;            // protected last keys of every unit
+    const int32_t* ub;           // [U] per-unit budgets (<= B) or null
     int32_t* kept;               // [U][B] or null
     int32_t* n_kept;             // [U]
     float* final_out;            // [U][cap] or null
@@ -171,30 +176,58 @@ void note_launch(cudaStream_t s);
 
 // calibrate.cu
 size_t calibrate_ws_bytes(int64_t n_heads, int64_t n_tok);
+// qpos (nullable): positions of post-RoPE rows, rotated back first; half:
+// half-split band pairing.
 cudaError_t launch_calibrate(const void* q, tri_dtype dt, int64_t n_heads, int64_t n_tok,
-                             float* stats, void* ws, cudaStream_t s);
+                             float* stats, void* ws, cudaStream_t s,
+                             const int32_t* qpos = nullptr, int half = 0, double theta = 10000.0);
 
 // score.cu
 int score_tile_keys(tri_dtype dt);
 cudaError_t launch_fold(const float* stats, const int64_t* p_cur, int64_t n_seq, int64_t n_layers,
-                        int64_t n_qheads, double theta, const FoldOffsets& off, float* wts,
-                        cudaStream_t s);
+                        int64_t n_qheads, double theta, const FoldOffsets& off, int variant,
+                        float* wts, cudaStream_t s);
 cudaError_t launch_score(tri_dtype dt, int G, const CUtensorMap& map, const ScoreArgs& a,
                          int n_sm, cudaStream_t s);
 // hist0 (nullable): per-unit histogram of the final scores, of their z-bins
 // (zbins != 0) or of their first radix digit.
+// Keys j < n_sink or j >= n_valid - n_recent get the final score +inf
+// (protected: kept before every other key).
 cudaError_t launch_zmax(int G, const float* raw, int64_t n_units, int64_t cap,
                         const int32_t* n_valid, const float2* mom, float* fin, uint32_t* hist0,
-                        int zbins, uint32_t* flag, cudaStream_t s);
+                        int zbins, int64_t n_sink, int64_t n_recent, uint32_t* flag,
+                        cudaStream_t s);
+
+// variant.cu: the max-over-offsets and half-split variants of the score,
+// two-pass moments, per-layer budgets to per-unit budgets.
+size_t variant_score_smem();
+cudaError_t launch_variant_score(tri_dtype dt, int G, const void* keys, int64_t n_units,
+                                 int64_t cap, const int32_t* n_valid, const float* wts,
+                                 const float* stats, const int64_t* p_cur, int64_t n_layers,
+                                 int64_t n_kvheads, double theta, const FoldOffsets& off,
+                                 int variant, float* raw, uint32_t* flag, cudaStream_t s);
+cudaError_t launch_moments(const float* raw, int64_t n_units, int64_t cap, const int32_t* n_valid,
+                           int G, float2* mom, cudaStream_t s);
+cudaError_t launch_unit_budget(const int32_t* layer_budget, int64_t n_units, int64_t n_layers,
+                               int64_t n_kvheads, int32_t* ub, cudaStream_t s);
+
+// decode.cu: attention of one query token per head over the cache rows.
+int decode_splits(int64_t n_units, int64_t cap, int n_sm);
+size_t decode_part_bytes(int64_t n_units, int G, int64_t cap, int n_sm);
+cudaError_t launch_decode(tri_dtype dt, int G, const void* q, const void* k, const void* v,
+                          int64_t n_units, int64_t cap, const int32_t* n_valid, float scale,
+                          float* out, float* part, uint32_t* flag, int n_sm, cudaStream_t s);
 
 // zselect.cu: top-B by z-bins on the split path (zhist from launch_zmax with
 // zbins; counts [U][chunks] and cand [U][kCandMax] scratch, cand_count [U]
 // zero on entry, state [U] of zsel_state_bytes()).
 size_t zsel_state_bytes();
+// ub (nullable): per-unit budgets [U] (clamped to [0, B]); B is the row
+// stride of kept.
 cudaError_t launch_zselect(const float* fin, int64_t n_units, int64_t cap, const int32_t* n_valid,
-                           int64_t B, const uint32_t* zhist, uint2* counts, int2* cand,
-                           uint32_t* cand_count, void* state, int32_t* kept, int32_t* n_kept,
-                           cudaStream_t s);
+                           int64_t B, const int32_t* ub, const uint32_t* zhist, uint2* counts,
+                           int2* cand, uint32_t* cand_count, void* state, int32_t* kept,
+                           int32_t* n_kept, cudaStream_t s);
 
 // select.cu
 cudaError_t launch_radix_pass(const float* fin, int64_t n_units, int64_t cap,
@@ -210,6 +243,9 @@ cudaError_t launch_gather(tri_dtype dt, const void* k_src, const void* v_src,
                           const int32_t* kept, const int32_t* n_kept, int64_t B, void* k_dst,
                           void* v_dst, int32_t* pos_dst, int64_t cap_dst, uint32_t* flag,
                           int n_blocks, cudaStream_t s);
+cudaError_t launch_compact_inplace(tri_dtype dt, void* k, void* v, int32_t* pos, int64_t n_units,
+                                   int64_t cap, const int32_t* kept, const int32_t* n_kept,
+                                   int64_t B, uint32_t* flag, int n_blocks, cudaStream_t s);
 cudaError_t launch_append(tri_dtype dt, void* k_cache, void* v_cache, int32_t* pos_cache,
                           int64_t n_seq, int64_t n_units, int64_t cap, int32_t* n_valid,
                           int64_t* p_cur, const void* k_new, const void* v_new,

@@ -1,6 +1,7 @@
 // zselect.cu -- top-B selection of the split prune path by z-bins.
 //
 // Keep the B keys with the highest final score, in ascending index order
+// (B per unit when a per-unit budget array is given: per-layer budgets)
 // (talk page: keep only the top-B; jaedaily.cn tutorial, eviction step:
 // top-k then sort to keep the temporal order).  Ranking: score descending,
 // NaN lowest, -0.0 == +0.0, equal scores by ascending index.
@@ -51,17 +52,19 @@ __device__ __forceinline__ uint32_t block_sum_256(uint32_t v, uint32_t* red8) {
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
 zsel_collect_kernel(const float* __restrict__ fin, int64_t cap, const int32_t* __restrict__ n_valid,
-                    int64_t B, const uint32_t* __restrict__ zhist, uint2* __restrict__ counts,
-                    int2* __restrict__ cand, uint32_t* __restrict__ cand_count) {
+                    int64_t B, const int32_t* __restrict__ ub, const uint32_t* __restrict__ zhist,
+                    uint2* __restrict__ counts, int2* __restrict__ cand,
+                    uint32_t* __restrict__ cand_count) {
     __shared__ uint32_t sb0;
     __shared__ uint32_t red8[8];
     const int64_t u = blockIdx.y;
     const int n = clamp_nvalid(n_valid, u, cap, nullptr);
-    if (n <= B) return;
+    const int64_t Bu = unit_budget(ub, u, B);
+    if (n <= Bu || Bu == 0) return;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (warp == 0) {
         uint32_t bin, above;
-        warp_find_bin(zhist + u * kZBins, kZBins, static_cast<uint32_t>(B), bin, above);
+        warp_find_bin(zhist + u * kZBins, kZBins, static_cast<uint32_t>(Bu), bin, above);
         if (lane == 0) sb0 = bin;
     }
     __syncthreads();
@@ -121,23 +124,24 @@ __device__ __forceinline__ uint32_t block_excl_scan_256(uint32_t v, uint32_t* re
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
 zsel_rank_kernel(const float* __restrict__ fin, int64_t cap, const int32_t* __restrict__ n_valid,
-                 int64_t B, const uint32_t* __restrict__ zhist, uint2* __restrict__ counts,
-                 int n_chunks, const int2* __restrict__ cand, const uint32_t* __restrict__ cand_count,
-                 ZSelState* __restrict__ st) {
+                 int64_t B, const int32_t* __restrict__ ub, const uint32_t* __restrict__ zhist,
+                 uint2* __restrict__ counts, int n_chunks, const int2* __restrict__ cand,
+                 const uint32_t* __restrict__ cand_count, ZSelState* __restrict__ st) {
     extern __shared__ int2 sc[];  // [kCandMax]
     __shared__ uint32_t hist[kHistBins0];
     __shared__ uint32_t sb0, sk, sprefix;
     __shared__ uint32_t red8[8];
     const int64_t u = blockIdx.x;
     const int n = clamp_nvalid(n_valid, u, cap, nullptr);
-    if (n <= B) return;
+    const int64_t Bu = unit_budget(ub, u, B);
+    if (n <= Bu || Bu == 0) return;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (warp == 0) {
         uint32_t bin, above;
-        warp_find_bin(zhist + u * kZBins, kZBins, static_cast<uint32_t>(B), bin, above);
+        warp_find_bin(zhist + u * kZBins, kZBins, static_cast<uint32_t>(Bu), bin, above);
         if (lane == 0) {
             sb0 = bin;
-            sk = static_cast<uint32_t>(B) - above;  // rank of the B-th key inside bin b0
+            sk = static_cast<uint32_t>(Bu) - above;  // rank of the Bu-th key inside bin b0
             sprefix = 0;
         }
     }
@@ -227,21 +231,23 @@ zsel_rank_kernel(const float* __restrict__ fin, int64_t cap, const int32_t* __re
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
 zsel_compact_kernel(const float* __restrict__ fin, int64_t cap, const int32_t* __restrict__ n_valid,
-                    int64_t B, const uint2* __restrict__ counts, const ZSelState* __restrict__ st,
-                    int32_t* __restrict__ kept, int32_t* __restrict__ n_kept) {
+                    int64_t B, const int32_t* __restrict__ ub, const uint2* __restrict__ counts,
+                    const ZSelState* __restrict__ st, int32_t* __restrict__ kept,
+                    int32_t* __restrict__ n_kept) {
     __shared__ uint32_t wgt[8], weq[8];
     const int64_t u = blockIdx.y;
     const int n = clamp_nvalid(n_valid, u, cap, nullptr);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t m = n < B ? n : B;
+    const int64_t Bu = unit_budget(ub, u, B);
+    const int64_t m = n < Bu ? n : Bu;
     int32_t* out = kept + u * B;
     const int j0 = blockIdx.x * kZChunk + warp * 256;
-    if (n <= B) {
+    if (n <= Bu) {
         for (int i = 0; i < 8; ++i) {
             const int j = j0 + 32 * i + lane;
             if (j < n) out[j] = j;
         }
-    } else {
+    } else if (Bu > 0) {
         const ZSelState s = st[u];
         const uint2 base = counts[u * gridDim.x + blockIdx.x];
         uint32_t key[8];
@@ -277,7 +283,7 @@ zsel_compact_kernel(const float* __restrict__ fin, int64_t cap, const int32_t* _
             const uint32_t bk = __ballot_sync(0xffffffffu, keep);
             if (keep) {
                 const uint32_t r = pos + __popc(bk & lt);
-                if (r < static_cast<uint32_t>(B)) out[r] = j;
+                if (r < static_cast<uint32_t>(Bu)) out[r] = j;
             }
             pos += __popc(bk);
             ties += __popc(beq);
@@ -295,22 +301,23 @@ zsel_compact_kernel(const float* __restrict__ fin, int64_t cap, const int32_t* _
 size_t zsel_state_bytes() { return sizeof(ZSelState); }
 
 cudaError_t launch_zselect(const float* fin, int64_t n_units, int64_t cap, const int32_t* n_valid,
-                           int64_t B, const uint32_t* zhist, uint2* counts, int2* cand,
-                           uint32_t* cand_count, void* state, int32_t* kept, int32_t* n_kept,
-                           cudaStream_t s) {
+                           int64_t B, const int32_t* ub, const uint32_t* zhist, uint2* counts,
+                           int2* cand, uint32_t* cand_count, void* state, int32_t* kept,
+                           int32_t* n_kept, cudaStream_t s) {
     const int n_chunks = static_cast<int>((cap + kZChunk - 1) / kZChunk);
     dim3 grid(static_cast<unsigned>(n_chunks), static_cast<unsigned>(n_units));
     ZSelState* st = static_cast<ZSelState*>(state);
-    zsel_collect_kernel<<<grid, 256, 0, s>>>(fin, cap, n_valid, B, zhist, counts, cand, cand_count);
+    zsel_collect_kernel<<<grid, 256, 0, s>>>(fin, cap, n_valid, B, ub, zhist, counts, cand,
+                                             cand_count);
     note_launch(s);
     const size_t smem = static_cast<size_t>(kCandMax) * sizeof(int2);
     cudaError_t e = cudaFuncSetAttribute(zsel_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     zsel_rank_kernel<<<static_cast<unsigned>(n_units), 256, smem, s>>>(
-        fin, cap, n_valid, B, zhist, counts, n_chunks, cand, cand_count, st);
+        fin, cap, n_valid, B, ub, zhist, counts, n_chunks, cand, cand_count, st);
     note_launch(s);
-    zsel_compact_kernel<<<grid, 256, 0, s>>>(fin, cap, n_valid, B, counts, st, kept, n_kept);
+    zsel_compact_kernel<<<grid, 256, 0, s>>>(fin, cap, n_valid, B, ub, counts, st, kept, n_kept);
     note_launch(s);
     return cudaGetLastError();
 }

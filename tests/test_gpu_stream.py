@@ -124,3 +124,69 @@ def test_stream_windows_match_oracle():
         assert np.all(np.diff(pp[:, :cap], axis=1) > 0)
         nxt["nv"], nxt["p_cur"] = nv_next, p_next
         cur, nxt = nxt, dict(k=cur["k"], v=cur["v"], pos=cur["pos"])
+
+
+@pytest.mark.parametrize("inplace,path", [(False, tri.PATH_PIPE), (True, tri.PATH_PIPE),
+                                          (False, tri.PATH_AUTO), (True, tri.PATH_SPLIT)])
+def test_stream_full_run(inplace, path):
+    """The streaming workload's whole stream at reduced width (1 sequence x 1
+    layer x 4 KV heads, G = 7, B 2048, window 128): 256 windows of generated
+    tokens appended, a prune whenever the cache holds B + 128 rows (240
+    prunes, the last at p_cur = 32768), through the window driver on two
+    cache buffers or one buffer compacted in place.  Prune steps 1, 2, 60,
+    120 and 240 are checked against the oracle run on the cache the GPU
+    pruned (kept sets, final scores, the gathered rows)."""
+    from types import SimpleNamespace
+
+    from rope_aware_kv_b200.window import WindowDriver
+
+    spec = synth.SPECS["c5"].scaled(n_seq=1, n_layers=1)
+    U, cap, B, G = spec.n_units, spec.cap, spec.B, spec.G
+    hp = synth.head_params(spec)
+    gst, ost = H.stats_for(spec, SimpleNamespace(hp=hp))
+    drv = WindowDriver(spec.n_seq, spec.n_layers, spec.n_kvheads, G, B, gst,
+                       window=synth.STREAM_WINDOW, inplace=inplace, cfg=tri.config(path=path))
+    assert drv.cap == cap
+    checks = {1, 2, 60, 120, 240}
+    seen = []
+    for w in range(synth.STREAM_TOKENS // synth.STREAM_WINDOW):
+        k_new, v_new, pos_new = synth.stream_window(spec, hp, w, "cuda")
+        drv.append(k_new, v_new, pos_new, auto_prune=False)
+        if not drv.full:
+            continue
+        step = drv.prunes + 1
+        if step not in checks:
+            drv.prune()
+            continue
+        # the cache about to be pruned
+        k0, v0, p0 = drv.k_cache.clone(), drv.v_cache.clone(), drv.pos_cache.clone()
+        nv0 = drv.n_valid.cpu().numpy()
+        pc0 = drv.p_cur.cpu().numpy()
+        assert np.all(nv0 == cap)
+        assert np.all(pc0 == synth.STREAM_WINDOW * (w + 1))
+        fin = torch.full((U, cap), float("nan"), device="cuda")
+        drv.prune(final=fin)
+        assert tri.tri_check_device_error(drv.ws) == 0
+        o = oracle.prune(synth.host_elems(k0), None, p0.cpu().numpy(), spec.n_seq, spec.n_layers,
+                         spec.n_kvheads, G, ost, pc0, B, n_valid=nv0, want_gather=False,
+                         want_raw=False)
+        gk_all = drv.kept.cpu().numpy()
+        fin_h = fin.cpu().numpy()
+        assert np.all(drv.n_valid.cpu().numpy() == B)
+        mismatched = 0
+        for u in range(U):
+            gk = gk_all[u]
+            assert H.check_final(fin_h[u], o["final"][u], cap) <= H.Z_RTOL, f"step {step} unit {u}"
+            mismatched += H.check_kept(gk, o["final"][u], o["kept"][u], cap, B)
+            assert H.rows_equal(drv.k_cache[u, :B], k0[u], gk)
+            assert H.rows_equal(drv.v_cache[u, :B], v0[u], gk)
+            assert np.array_equal(drv.pos_cache[u, :B].cpu().numpy(), p0[u].cpu().numpy()[gk])
+        assert mismatched <= 2 * U
+        seen.append(step)
+    assert seen == sorted(checks)
+    assert drv.prunes == 240
+    assert drv.tokens == synth.STREAM_TOKENS
+    assert np.all(drv.p_cur.cpu().numpy() == synth.STREAM_TOKENS)
+    # kept positions stay ascending through the whole stream
+    pp = drv.pos_cache.cpu().numpy()[:, :B]
+    assert np.all(np.diff(pp, axis=1) > 0)

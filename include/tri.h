@@ -152,6 +152,13 @@ typedef struct tri_config {
      * every unit of layer l, clamped to [0, B]; B remains the row stride of
      * kept_idx and the bound of cap_dst.  NULL: B everywhere (tri_prune only). */
     const int32_t* layer_budget;
+    /* Bound, in nanoseconds, of each wait at the unit-wide barriers of the
+     * cooperative path (TRI_PATH_COOP); 0: 2 s.  A wait that runs out sets
+     * TRI_FLAG_TIMEOUT and its CTA skips the rest of the unit (no copy is in
+     * flight into its shared memory at any unit barrier), so the call's
+     * outputs for that unit are incomplete; the next call starts clean.  Only
+     * for testing the timeout path: production calls leave it 0. */
+    int64_t barrier_wait_ns;
 } tri_config;
 
 /* Fill cfg (host) with head_dim, theta = 10000, D = {2^0, ..., 2^16}

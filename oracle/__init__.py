@@ -20,6 +20,10 @@ Every function follows the pages step by step:
 * ``select`` -- top-B by (score desc, index asc), returned ascending
   (jaedaily.cn KV-compression tutorial, eviction step).
 * ``prune`` -- all of the above plus the bit-exact gather, over many units.
+* ``logit_reconstruct`` / ``logit_curve`` / ``pearson`` -- the trig-series
+  logit(Delta) from the Q/K centres, the measured mean logit at each distance,
+  and their correlation (talk page, centre approximation; paper reading,
+  Fig. 1(D)).
 * ``decode_attention`` -- softmax attention of the next token's queries over
   the kept keys, renormalised over them (jaedaily.cn tutorial, compression
   objective), the consumer of the compacted cache.
@@ -101,6 +105,12 @@ def _bind(lib):
     lib.oracle_prune.restype = i32
     lib.oracle_decode_attention.argtypes = [P, P, P, i32, i64, i32, i64, i32, P, d, P]
     lib.oracle_decode_attention.restype = i32
+    lib.oracle_logit_reconstruct.argtypes = [P, P, i64, i32, i32, d, P, i64, P]
+    lib.oracle_logit_reconstruct.restype = i32
+    lib.oracle_logit_curve.argtypes = [P, P, i32, i64, i32, i64, i32, P, i64, P]
+    lib.oracle_logit_curve.restype = i32
+    lib.oracle_pearson.argtypes = [P, P, i64, i64, P]
+    lib.oracle_pearson.restype = i32
     lib.oracle_threads.argtypes = []
     lib.oracle_threads.restype = i32
     lib.oracle_set_threads.argtypes = [i32]
@@ -298,4 +308,48 @@ def decode_attention(q, k, v, n_valid=None, scale=None):
                                          sc, _ptr(out))
     if rc:
         raise ValueError(f"oracle_decode_attention failed ({rc})")
+    return out
+
+
+def logit_reconstruct(qstats, kstats, G, deltas, theta=THETA):
+    """Trig-series logit(Delta) from the Q and K centres: qstats [Hq, d/2, 4],
+    kstats [Hq/G, d/2, 4] -> [Hq, len(deltas)] (tri_oracle.c)."""
+    qs = np.ascontiguousarray(qstats, np.float64)
+    ks = np.ascontiguousarray(kstats, np.float64)
+    Hq, F = qs.shape[0], qs.shape[1]
+    dl = np.ascontiguousarray(np.asarray(deltas, np.int64))
+    out = np.empty((Hq, len(dl)), np.float64)
+    rc = _load().oracle_logit_reconstruct(_ptr(qs), _ptr(ks), Hq, int(G), 2 * F, float(theta),
+                                          _ptr(dl), len(dl), _ptr(out))
+    if rc:
+        raise ValueError(f"oracle_logit_reconstruct failed ({rc})")
+    return out
+
+
+def logit_curve(q, k, G, deltas):
+    """Mean post-RoPE logit at each distance: q [Hq, n, d], k [Hq/G, n, d]
+    -> [Hq, len(deltas)] (tri_oracle.c)."""
+    q, dt = _elem(q)
+    k, dtk = _elem(k)
+    if dt != dtk:
+        raise TypeError("q and k must share a dtype")
+    Hq, n, d = q.shape
+    dl = np.ascontiguousarray(np.asarray(deltas, np.int64))
+    out = np.empty((Hq, len(dl)), np.float64)
+    rc = _load().oracle_logit_curve(_ptr(q), _ptr(k), dt, Hq, int(G), n, d, _ptr(dl), len(dl),
+                                    _ptr(out))
+    if rc:
+        raise ValueError(f"oracle_logit_curve failed ({rc})")
+    return out
+
+
+def pearson(a, b):
+    """Row-wise Pearson correlation of a and b [rows, n] -> [rows]."""
+    a = np.ascontiguousarray(a, np.float64)
+    b = np.ascontiguousarray(b, np.float64)
+    rows, n = a.shape
+    out = np.empty((rows,), np.float64)
+    rc = _load().oracle_pearson(_ptr(a), _ptr(b), rows, n, _ptr(out))
+    if rc:
+        raise ValueError(f"oracle_pearson failed ({rc})")
     return out

@@ -559,3 +559,95 @@ int oracle_decode_attention(const void* q, const void* k, const void* v, int dty
     }
     return err;
 }
+
+/*
+ * The attention logit as a function of the distance Delta, reconstructed from
+ * the Q and K centres (talk page: the RoPE logit general form
+ * logit = sum_f |q_f| |k_f| cos(w_f Delta + phi_f), phi_f = arg q_f - arg k_f,
+ * and the centre approximation q_f ~ E[q_f], k_f ~ E[k_f] that turns it into
+ * a trigonometric series in Delta; shibing624 paper reading, Fig. 1(D)):
+ *   recon[h][i] = sum_f |E q_f| |E k_f| cos(w_f deltas[i] + arg E q_f - arg E k_f)
+ * for query head h with statistics qstats[h] and its KV head's kstats[h / G]
+ * ([..][d/2][4] as oracle_calibrate writes them).
+ */
+int oracle_logit_reconstruct(const double* qstats, const double* kstats, int64_t n_qheads, int G,
+                             int d, double theta, const int64_t* deltas, int64_t n_delta,
+                             double* recon) {
+    if (!qstats || !kstats || !deltas || !recon || n_qheads < 0 || G <= 0 || d <= 0 || (d & 1))
+        return ORA_EINVAL;
+    const int F = d / 2;
+    for (int64_t h = 0; h < n_qheads; ++h) {
+        const double* qs = qstats + h * F * 4;
+        const double* ks = kstats + (h / G) * F * 4;
+        for (int64_t i = 0; i < n_delta; ++i) {
+            double sum = 0.0;
+            for (int f = 0; f < F; ++f) {
+                const double amp = hypot(qs[f * 4], qs[f * 4 + 1]) * hypot(ks[f * 4], ks[f * 4 + 1]);
+                const double phi = atan2(qs[f * 4 + 1], qs[f * 4]) - atan2(ks[f * 4 + 1], ks[f * 4]);
+                sum += amp * cos(ora_omega(theta, f, d) * (double)deltas[i] + phi);
+            }
+            recon[h * n_delta + i] = sum;
+        }
+    }
+    return ORA_OK;
+}
+
+/*
+ * The measured counterpart: the mean post-RoPE attention logit over every
+ * query/key pair of one sequence at distance Delta, token t at position t:
+ *   curve[h][i] = mean over t in [Delta, n_tok) of q[h][t] . k[h / G][t - Delta]
+ * (0 when no pair is that far apart).  q: [n_qheads][n_tok][d], k:
+ * [n_qheads / G][n_tok][d], post-RoPE (dtype codes as elsewhere).
+ */
+int oracle_logit_curve(const void* q, const void* k, int dtype, int64_t n_qheads, int G,
+                       int64_t n_tok, int d, const int64_t* deltas, int64_t n_delta,
+                       double* curve) {
+    if (!q || !k || !deltas || !curve || n_qheads < 0 || G <= 0 || n_tok < 0 || d <= 0)
+        return ORA_EINVAL;
+    int64_t h;
+#pragma omp parallel for schedule(dynamic)
+    for (h = 0; h < n_qheads; ++h) {
+        const int64_t kh = h / G;
+        for (int64_t i = 0; i < n_delta; ++i) {
+            const int64_t D = deltas[i];
+            double sum = 0.0;
+            int64_t cnt = 0;
+            for (int64_t t = (D > 0 ? D : 0); t < n_tok; ++t) {
+                if (t - D >= n_tok) continue;
+                double dot = 0.0;
+                for (int e = 0; e < d; ++e)
+                    dot += ora_decode(q, dtype, (h * n_tok + t) * (int64_t)d + e) *
+                           ora_decode(k, dtype, (kh * n_tok + t - D) * (int64_t)d + e);
+                sum += dot;
+                ++cnt;
+            }
+            curve[h * n_delta + i] = cnt > 0 ? sum / (double)cnt : 0.0;
+        }
+    }
+    return ORA_OK;
+}
+
+/* Pearson correlation of rows a[r][0..n) and b[r][0..n) (two-pass; 0 when a
+ * row is constant). */
+int oracle_pearson(const double* a, const double* b, int64_t n_rows, int64_t n, double* r) {
+    if (!a || !b || !r || n_rows < 0 || n < 0) return ORA_EINVAL;
+    for (int64_t row = 0; row < n_rows; ++row) {
+        const double* x = a + row * n;
+        const double* y = b + row * n;
+        double mx = 0.0, my = 0.0;
+        for (int64_t i = 0; i < n; ++i) {
+            mx += x[i];
+            my += y[i];
+        }
+        mx /= (double)(n > 0 ? n : 1);
+        my /= (double)(n > 0 ? n : 1);
+        double sxy = 0.0, sxx = 0.0, syy = 0.0;
+        for (int64_t i = 0; i < n; ++i) {
+            sxy += (x[i] - mx) * (y[i] - my);
+            sxx += (x[i] - mx) * (x[i] - mx);
+            syy += (y[i] - my) * (y[i] - my);
+        }
+        r[row] = (sxx > 0.0 && syy > 0.0) ? sxy / sqrt(sxx * syy) : 0.0;
+    }
+    return ORA_OK;
+}

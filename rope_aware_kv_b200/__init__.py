@@ -79,7 +79,7 @@ class TriConfig(ctypes.Structure):
                 ("n_offsets", ctypes.c_int), ("offsets", ctypes.c_int64 * MAX_OFFSETS),
                 ("path", ctypes.c_int), ("variant", ctypes.c_int),
                 ("n_sink", ctypes.c_int64), ("n_recent", ctypes.c_int64),
-                ("layer_budget", ctypes.c_void_p)]
+                ("layer_budget", ctypes.c_void_p), ("barrier_wait_ns", ctypes.c_int64)]
 
 
 _lib = None
@@ -179,11 +179,14 @@ def _check(fn: str, code: int):
 def config(theta: float = 10000.0, offsets: Optional[Sequence[int]] = None,
            head_dim: int = HEAD_DIM, path: int = PATH_AUTO, variant: int = 0,
            n_sink: int = 0, n_recent: int = 0,
-           layer_budget: Optional[torch.Tensor] = None) -> TriConfig:
+           layer_budget: Optional[torch.Tensor] = None,
+           barrier_wait_ns: int = 0) -> TriConfig:
     """Method parameters (tri.h: tri_config).  ``variant``: VAR_* bits;
     ``n_sink`` / ``n_recent``: protected first / last keys of every unit;
     ``layer_budget``: int32 CUDA tensor [n_layers] of per-layer budgets (the
-    config keeps its pointer only: keep the tensor alive while it is used)."""
+    config keeps its pointer only: keep the tensor alive while it is used);
+    ``barrier_wait_ns``: bound of the cooperative path's unit-barrier waits
+    (0: 2 s; a short bound exists to test the timeout path)."""
     cfg = TriConfig()
     load().tri_config_default(ctypes.byref(cfg), head_dim)
     cfg.theta = float(theta)
@@ -191,6 +194,7 @@ def config(theta: float = 10000.0, offsets: Optional[Sequence[int]] = None,
     cfg.variant = int(variant)
     cfg.n_sink = int(n_sink)
     cfg.n_recent = int(n_recent)
+    cfg.barrier_wait_ns = int(barrier_wait_ns)
     if layer_budget is not None:
         if layer_budget.dtype != torch.int32 or not layer_budget.is_cuda:
             raise TypeError("layer_budget must be an int32 CUDA tensor")

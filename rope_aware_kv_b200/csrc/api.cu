@@ -197,7 +197,8 @@ tri_status check_cfg(const tri_config* cfg, FoldOffsets* off) {
     if (!(cfg->theta > 1.0) || cfg->n_offsets < 1 || cfg->n_offsets > TRI_MAX_OFFSETS)
         return TRI_ERR_INVALID_ARG;
     if (cfg->path < TRI_PATH_AUTO || cfg->path > TRI_PATH_PIPE) return TRI_ERR_INVALID_ARG;
-    if ((cfg->variant & ~TRI_VAR_ALL) != 0 || cfg->n_sink < 0 || cfg->n_recent < 0)
+    if ((cfg->variant & ~TRI_VAR_ALL) != 0 || cfg->n_sink < 0 || cfg->n_recent < 0 ||
+        cfg->barrier_wait_ns < 0)
         return TRI_ERR_INVALID_ARG;
     if (cfg->layer_budget && !aligned4(cfg->layer_budget)) return TRI_ERR_INVALID_ARG;
     off->n = cfg->n_offsets;
@@ -881,6 +882,8 @@ static tri_status prune_impl(const tri_config* cfg, const void* k_src, const voi
         a.keys_max = w.cp.keys_max;
         a.stages = w.cp.stages;
         a.ctas_per_unit = w.cp.ctas_per_unit;
+        a.barrier_wait_ns = cfg->barrier_wait_ns > 0 ? static_cast<uint64_t>(cfg->barrier_wait_ns)
+                                                     : kWaitLimitNs;
         a.n_valid = n_valid;
         a.k_src = k_src;
         a.v_src = v_src;

@@ -107,14 +107,14 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
 // and thread 0's fence after the wait orders the other CTAs' writes before
 // everything that follows the second CTA barrier.
 __device__ __forceinline__ bool unit_barrier(uint32_t* ctr, uint32_t target, uint32_t* flag,
-                                             int* abort_flag) {
+                                             int* abort_flag, uint64_t limit_ns) {
     __syncthreads();
     if (threadIdx.x == 0 && !*abort_flag) {
         __threadfence();
         atomicAdd(ctr, 1u);
         const uint64_t t0 = globaltimer_ns();
         while (ld_acquire_u32(ctr) < target) {
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 raise_flag(flag, TRI_FLAG_TIMEOUT);
                 *abort_flag = 1;
                 break;
@@ -307,7 +307,7 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
             part[1] = s2;
         }
         coop_trace(a, 1);
-        if (!unit_barrier(ctr, 1u * C, a.flag, abort_flag)) return;
+        if (!unit_barrier(ctr, 1u * C, a.flag, abort_flag, a.barrier_wait_ns)) return;
         coop_trace(a, 2);
 
         // ---------------- phase 2: moments, final, digit 0 ----------------
@@ -389,7 +389,7 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
                 if (hist[b]) atomicAdd(&g[b], hist[b]);
         }
         coop_trace(a, 3);
-        if (!unit_barrier(ctr, 2u * C, a.flag, abort_flag)) return;
+        if (!unit_barrier(ctr, 2u * C, a.flag, abort_flag, a.barrier_wait_ns)) return;
         coop_trace(a, 4);
 
         // ---------------- phase 3: threshold bin, candidates ----------------
@@ -467,7 +467,7 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
                 slot += __popc(bc);
             }
         }
-        if (!unit_barrier(ctr, 3u * C, a.flag, abort_flag)) return;
+        if (!unit_barrier(ctr, 3u * C, a.flag, abort_flag, a.barrier_wait_ns)) return;
 
         // ---------------- phase 4: the threshold key ----------------
         // Three radix digits of the full key (11, 11, 10 bits) find the
@@ -579,7 +579,7 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
                 uint32_t* g = a.hists_key + (static_cast<int64_t>(p) * a.n_units + u) * kHistBins0;
                 for (int b = tid; b < nb; b += S::kThreads)
                     if (hist[b]) atomicAdd(&g[b], hist[b]);
-                if (!unit_barrier(ctr, (4u + p) * C, a.flag, abort_flag)) return;
+                if (!unit_barrier(ctr, (4u + p) * C, a.flag, abort_flag, a.barrier_wait_ns)) return;
                 copy_l2_to_shared(reinterpret_cast<uint4*>(hist),
                                   reinterpret_cast<const uint4*>(g), nb / 4);
                 __syncthreads();
@@ -621,7 +621,7 @@ prune_coop_kernel(const __grid_constant__ CUtensorMap kmap, CoopArgs a) {
                     a.counts[u * C + c] = make_uint2(g2, e2);
                 }
             }
-            if (!unit_barrier(ctr, 7u * C, a.flag, abort_flag)) return;
+            if (!unit_barrier(ctr, 7u * C, a.flag, abort_flag, a.barrier_wait_ns)) return;
             if (warp == 0) {
                 uint32_t gsum = 0, esum = 0;
                 for (int cc = lane; cc < c; cc += 32) {

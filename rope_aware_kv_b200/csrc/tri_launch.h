@@ -132,6 +132,7 @@ struct CoopArgs {
     int64_t keys_max;            // most keys one CTA takes
     int stages;                  // TMA ring depth
     int ctas_per_unit;           // C
+    uint64_t barrier_wait_ns;    // bound of each unit-barrier wait
     const int32_t* n_valid;
     const void* k_src;
     const void* v_src;

@@ -50,6 +50,12 @@ MUTANTS = [
     ("attention scale dropped", "sc[j] = scale * dot;", "sc[j] = dot;"),
     ("attention over one row too few", "for (int64_t j = 0; j < n; ++j) {\n                const int64_t krow",
      "for (int64_t j = 0; j + 1 < n; ++j) {\n                const int64_t krow"),
+    ("reconstruction phase sign", "- atan2(ks[f * 4 + 1], ks[f * 4]);",
+     "+ atan2(ks[f * 4 + 1], ks[f * 4]);"),
+    ("curve pairs the key after the query", "ora_decode(k, dtype, (kh * n_tok + t - D) * (int64_t)d + e);",
+     "ora_decode(k, dtype, (kh * n_tok + (t - D + 1 < n_tok ? t - D + 1 : t - D)) * (int64_t)d + e);"),
+    ("curve uses KV head h", "const int64_t kh = h / G;", "const int64_t kh = h % (n_qheads / G);"),
+    ("pearson without centring", "sxy += (x[i] - mx) * (y[i] - my);", "sxy += x[i] * y[i];"),
     ("layer budget of the next layer", "const int64_t Bu = layer_budget ? layer_budget[layer] : B;",
      "const int64_t Bu = layer_budget ? layer_budget[(layer + 1) % n_layers] : B;"),
     ("sample sigma", "sqrt(ss / (double)n)", "sqrt(ss / (double)(n > 1 ? n - 1 : 1))"),
@@ -94,6 +100,9 @@ PIN_TESTS = [
     lambda: var.test_layer_budgets_equal_single_budget_runs(),
     lambda: var.test_decode_attention_matches_library_sdpa(),
     lambda: var.test_decode_attention_special_cases(),
+    lambda: var.test_logit_reconstruction_is_the_rotated_centres_dot_product(),
+    lambda: var.test_logit_curve_of_centred_sequences_equals_reconstruction(),
+    lambda: var.test_pearson_matches_numpy(),
 ]
 
 

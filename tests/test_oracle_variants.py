@@ -283,3 +283,57 @@ def test_decode_attention_special_cases():
     perm = rng.permutation(cap)
     np.testing.assert_allclose(oracle.decode_attention(q, k[:, perm], v[:, perm]),
                                oracle.decode_attention(q, k, v), rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# logit(Delta) reconstruction from the centres, measured curve, Pearson
+# ---------------------------------------------------------------------------
+def test_logit_reconstruction_is_the_rotated_centres_dot_product():
+    """The trig series in Delta equals the explicit post-RoPE dot product of
+    the centres, the query centre at position p + Delta and the key centre at
+    p (talk page, RoPE logit general form), for any p."""
+    rng = np.random.default_rng(13)
+    qbar = rng.normal(size=D)
+    kbar = rng.normal(size=D)
+    qs = _stats_identical(qbar.astype(np.float32))
+    ks = _stats_identical(kbar.astype(np.float32))
+    deltas = [0, 1, 7, 100, 4097, 30000]
+    got = oracle.logit_reconstruct(qs, ks, 1, deltas)[0]
+    q32, k32 = qbar.astype(np.float32).astype(np.float64), kbar.astype(np.float32).astype(np.float64)
+    for p in (0, 12345):
+        want = [_rope_matrix_rotate(q32, p + dl) @ _rope_matrix_rotate(k32, p) for dl in deltas]
+        np.testing.assert_allclose(got, want, rtol=1e-10, atol=1e-10 * np.abs(q32).sum() * np.abs(k32).sum())
+
+
+def test_logit_curve_of_centred_sequences_equals_reconstruction():
+    """Every query and key at its centre (token t rotated to position t): the
+    measured mean logit at each distance is exactly the reconstruction, and
+    their Pearson correlation is 1; GQA maps query head h to KV head h / G."""
+    rng = np.random.default_rng(14)
+    n, G = 64, 2
+    qbar = rng.normal(size=(2 * G, D)).astype(np.float32)
+    kbar = rng.normal(size=(2, D)).astype(np.float32)
+    pos = np.arange(n)
+    q = np.stack([[_rope_matrix_rotate(qbar[h].astype(np.float64), t) for t in pos]
+                  for h in range(2 * G)])
+    k = np.stack([[_rope_matrix_rotate(kbar[h].astype(np.float64), t) for t in pos]
+                  for h in range(2)])
+    deltas = [0, 1, 2, 5, 17, 40, 63, 64]
+    curve = oracle.logit_curve(q.astype(np.float32), k.astype(np.float32), G, deltas)
+    qs = np.concatenate([_stats_identical(x) for x in qbar])
+    ks = np.concatenate([_stats_identical(x) for x in kbar])
+    recon = oracle.logit_reconstruct(qs, ks, G, deltas)
+    scale = np.abs(qbar).sum() * np.abs(kbar).sum()
+    np.testing.assert_allclose(curve[:, :-1], recon[:, :-1], atol=1e-5 * scale)
+    assert np.all(curve[:, -1] == 0.0)       # no pair is 64 apart in 64 tokens
+    r = oracle.pearson(curve[:, :-1], recon[:, :-1])
+    np.testing.assert_allclose(r, 1.0, atol=1e-9)
+
+
+def test_pearson_matches_numpy():
+    rng = np.random.default_rng(15)
+    a = rng.normal(size=(5, 40))
+    b = 0.3 * a + rng.normal(size=(5, 40))
+    want = [np.corrcoef(a[i], b[i])[0, 1] for i in range(5)]
+    np.testing.assert_allclose(oracle.pearson(a, b), want, rtol=1e-12)
+    assert oracle.pearson(np.ones((1, 8)), a[:1, :8])[0] == 0.0

@@ -682,7 +682,7 @@ def run_tri(args, ws, rank, local):
     ms_step = rec["ms_per_step"]
     dom_name, dom_bytes, dom_ms = dominant(spec, rec, ms_step)
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9 if dom_ms > 0 else 0.0
-    e2e = run_e2e(args, runner, stream, spec, ws)
+    e2e = None if args.no_e2e else run_e2e(args, runner, stream, spec, ws)
     launches = rec["launches_per_step"]
     del runner
     torch.cuda.empty_cache()
@@ -879,6 +879,8 @@ def main():
     ap.add_argument("--impl", default="tri", choices=["tri", "reference"])
     ap.add_argument("--workload", default="c4", choices=sorted(synth.SPECS) + [STREAM])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="skip the end-to-end (host buffers) measurement")
     ap.add_argument("--no-sub", action="store_true",
                     help="time the chosen workload only (no sub-records of the others)")
     ap.add_argument("--n-seq", type=int, default=0,

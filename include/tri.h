@@ -403,12 +403,76 @@ tri_status tri_prune_inplace(const tri_config* cfg, void* k, void* v, int32_t* p
                              const float* stats, int64_t B, int32_t* kept_idx, int32_t* n_kept,
                              float* final_score, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * The in-place prune step on a paged cache (the page-table layout of paged
+ * KV caches): the K and V rows of all units live in one pool of n_pages
+ * pages of page_rows rows each, [n_pages][page_rows][head_dim] (dt); logical
+ * row j of unit u is row j % page_rows of page
+ * page_table[u * pages_per_unit + j / page_rows] (device int32).  Logical
+ * rows are what every other argument means (n_valid, kept_idx, final_score
+ * and the positions pos, which stay [U][cap] int32, nullable): after the
+ * call rows 0 .. n_kept[u]-1 of unit u hold its kept rows in temporal order,
+ * so the pages past ceil(n_kept[u] / page_rows) hold nothing the unit needs.
+ * page_rows is a multiple of 128 (whole score tiles per page) and
+ * pages_per_unit * page_rows >= cap; a page index outside [0, n_pages) sets
+ * TRI_FLAG_INDEX_RANGE, its keys score as zeros and its rows are not moved.
+ * Runs the split kernels (score tiles located through the table, in-place
+ * compaction through it); cfg->path other than TRI_PATH_AUTO and
+ * TRI_PATH_SPLIT returns TRI_ERR_UNSUPPORTED.  Workspace:
+ * tri_prune_workspace_bytes.
+ */
+tri_status tri_prune_paged_inplace(const tri_config* cfg, void* k_pool, void* v_pool, int32_t* pos,
+                                   tri_dtype dt, int64_t n_seq, int64_t n_layers,
+                                   int64_t n_kvheads, int G, int64_t cap, const int32_t* n_valid,
+                                   const int64_t* p_cur, const float* stats, int64_t B,
+                                   const int32_t* page_table, int64_t page_rows,
+                                   int64_t pages_per_unit, int64_t n_pages, int32_t* kept_idx,
+                                   int32_t* n_kept, float* final_score, void* ws, size_t ws_bytes,
+                                   void* stream);
+
 /* The kernel path (TRI_PATH_PIPE, TRI_PATH_COOP, TRI_PATH_FUSED or TRI_PATH_SPLIT) that
  * tri_prune (inplace = 0) or tri_prune_inplace (inplace = 1) takes for these
  * shapes on the current device when cfg->path is `path`; -1 when `path`
  * cannot serve them or the shapes are invalid. */
 int tri_prune_path(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int64_t cap,
                    int64_t B, tri_dtype dt, int path, int inplace);
+
+/* ---------------------------------------------------------------------- */
+/* logit(Delta) from the centres, measured, and their correlation          */
+/* ---------------------------------------------------------------------- */
+
+/*
+ * The attention logit as a trigonometric series in the distance Delta, from
+ * the Q and K centres (talk page: RoPE logit general form and the centre
+ * approximation q_f ~ E[q_f], k_f ~ E[k_f]):
+ *   recon[h][i] = sum_f |E q_f| |E k_f| cos(w_f deltas[i] + arg E q_f - arg E k_f)
+ * with w_f = theta^(-2f/d) (cfg->theta).  q_stats: [n_qheads][64][4] and
+ * k_stats: [n_qheads / G][64][4] as tri_calibrate / tri_calibrate_ex write
+ * them (keys calibrated like queries give the K centres); query head h uses
+ * KV head h / G.  deltas: device int64 [n_delta]; recon: [n_qheads][n_delta]
+ * float32 (float64 inside).  No workspace.
+ */
+tri_status tri_logit_reconstruct(const tri_config* cfg, const float* q_stats,
+                                 const float* k_stats, int64_t n_qheads, int G,
+                                 const int64_t* deltas, int64_t n_delta, float* recon,
+                                 void* stream);
+
+/*
+ * The measured counterpart on one sequence of post-RoPE rows, token t at
+ * position t:  curve[h][i] = mean over t of q[h][t] . k[h / G][t - deltas[i]]
+ * over the pairs inside [0, n_tok) (0 when there is none).  q_post:
+ * [n_qheads][n_tok][head_dim], k_post: [n_qheads / G][n_tok][head_dim] (dt);
+ * deltas: device int64 [n_delta]; curve: [n_qheads][n_delta] float32.
+ */
+tri_status tri_logit_curve(const void* q_post, const void* k_post, tri_dtype dt, int64_t n_qheads,
+                           int G, int64_t n_tok, int head_dim, const int64_t* deltas,
+                           int64_t n_delta, float* curve, void* stream);
+
+/* Pearson correlation of each row of a and b ([n_rows][n] float32) into
+ * r[n_rows] (shibing624 paper reading, Fig. 1(D): reconstruction against the
+ * measured logits per head); 0 for a constant row. */
+tri_status tri_pearson(const float* a, const float* b, int64_t n_rows, int64_t n, float* r,
+                       void* stream);
 
 /* ---------------------------------------------------------------------- */
 /* Decode attention over the compacted cache                               */

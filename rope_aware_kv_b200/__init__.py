@@ -59,6 +59,7 @@ EXPORTS = (
     "tri_select_topB_static", "tri_select_static_scratch_bytes", "tri_prune_path",
     "tri_compact_inplace", "tri_prune_inplace", "tri_calibrate_ex",
     "tri_decode_workspace_bytes", "tri_decode_attention",
+    "tri_logit_reconstruct", "tri_logit_curve", "tri_pearson", "tri_prune_paged_inplace",
 )
 
 
@@ -108,6 +109,12 @@ def load(path: Optional[str] = None):
         "tri_calibrate": (i32, [P, i32, i64, i64, i32, P, P, sz, P]),
         "tri_calibrate_sums": (i32, [P, i32, i64, i64, i32, P, P, sz, P]),
         "tri_calibrate_finish": (i32, [P, i64, i64, i32, P, P]),
+        "tri_prune_paged_inplace": (i32, [ctypes.POINTER(TriConfig), P, P, P, i32, i64, i64, i64,
+                                          i32, i64, P, P, P, i64, P, i64, i64, i64, P, P, P, P, sz,
+                                          P]),
+        "tri_logit_reconstruct": (i32, [ctypes.POINTER(TriConfig), P, P, i64, i32, P, i64, P, P]),
+        "tri_logit_curve": (i32, [P, P, i32, i64, i32, i64, i32, P, i64, P, P]),
+        "tri_pearson": (i32, [P, P, i64, i64, P, P]),
         "tri_decode_workspace_bytes": (sz, [i64, i32, i64]),
         "tri_decode_attention": (i32, [P, P, P, i32, i64, i32, i64, i32, P, ctypes.c_float, P, P,
                                        sz, P]),
@@ -446,6 +453,39 @@ def tri_prune_inplace(cfg: TriConfig, k: torch.Tensor, v: Optional[torch.Tensor]
         _ptr(ws), ws.numel(), _stream(stream)))
 
 
+def tri_logit_reconstruct(cfg: TriConfig, q_stats: torch.Tensor, k_stats: torch.Tensor, G: int,
+                          deltas: torch.Tensor, stream=None) -> torch.Tensor:
+    """Trig-series logit(Delta) from the centres: q_stats [Hq, 64, 4], k_stats
+    [Hq/G, 64, 4], deltas int64 CUDA [n] -> [Hq, n] float32."""
+    Hq = q_stats.shape[0]
+    out = torch.empty((Hq, deltas.numel()), dtype=torch.float32, device=q_stats.device)
+    _check("tri_logit_reconstruct", load().tri_logit_reconstruct(
+        ctypes.byref(cfg), _ptr(q_stats), _ptr(k_stats), Hq, G, _ptr(deltas), deltas.numel(),
+        _ptr(out), _stream(stream)))
+    return out
+
+
+def tri_logit_curve(q_post: torch.Tensor, k_post: torch.Tensor, G: int, deltas: torch.Tensor,
+                    stream=None) -> torch.Tensor:
+    """Mean post-RoPE logit at each distance: q [Hq, n, d], k [Hq/G, n, d],
+    deltas int64 CUDA [m] -> [Hq, m] float32."""
+    Hq, n, d = q_post.shape
+    out = torch.empty((Hq, deltas.numel()), dtype=torch.float32, device=q_post.device)
+    _check("tri_logit_curve", load().tri_logit_curve(
+        _ptr(q_post), _ptr(k_post), _dt(q_post), Hq, G, n, d, _ptr(deltas), deltas.numel(),
+        _ptr(out), _stream(stream)))
+    return out
+
+
+def tri_pearson(a: torch.Tensor, b: torch.Tensor, stream=None) -> torch.Tensor:
+    """Row-wise Pearson correlation of two [rows, n] float32 CUDA tensors."""
+    rows, n = a.shape
+    out = torch.empty((rows,), dtype=torch.float32, device=a.device)
+    _check("tri_pearson", load().tri_pearson(_ptr(a), _ptr(b), rows, n, _ptr(out),
+                                             _stream(stream)))
+    return out
+
+
 def tri_decode_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
                          n_valid: Optional[torch.Tensor] = None, scale: Optional[float] = None,
                          out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
@@ -463,6 +503,27 @@ def tri_decode_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
         _ptr(q), _ptr(k), _ptr(v), _dt(q), U, G, cap, d, _ptr(n_valid), ctypes.c_float(sc),
         _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
     return out
+
+
+def tri_prune_paged_inplace(cfg: TriConfig, k_pool: torch.Tensor, v_pool: Optional[torch.Tensor],
+                            pos: Optional[torch.Tensor], page_table: torch.Tensor, cap: int,
+                            n_seq: int, n_layers: int, n_kvheads: int, G: int,
+                            p_cur: torch.Tensor, stats: torch.Tensor, B: int,
+                            n_kept: torch.Tensor, n_valid: Optional[torch.Tensor] = None,
+                            kept: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                            stream=None, final: Optional[torch.Tensor] = None):
+    """In-place prune of a paged cache: k_pool / v_pool [n_pages, page_rows, d],
+    page_table int32 [U, pages_per_unit], pos [U, cap] (logical rows)."""
+    n_pages, page_rows, d = k_pool.shape
+    ppu = page_table.shape[1]
+    if ws is None:
+        ws = workspace(tri_prune_workspace_bytes(n_seq, n_layers, n_kvheads, G, cap, B, d),
+                       k_pool.device)
+    _check("tri_prune_paged_inplace", load().tri_prune_paged_inplace(
+        ctypes.byref(cfg), _ptr(k_pool), _ptr(v_pool), _ptr(pos), _dt(k_pool), n_seq, n_layers,
+        n_kvheads, G, cap, _ptr(n_valid), _ptr(p_cur), _ptr(stats), B, _ptr(page_table),
+        page_rows, ppu, n_pages, _ptr(kept), _ptr(n_kept), _ptr(final), _ptr(ws), ws.numel(),
+        _stream(stream)))
 
 
 def tri_append(k_cache, v_cache, pos_cache, n_seq: int, n_valid: torch.Tensor,

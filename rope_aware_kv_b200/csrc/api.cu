@@ -374,6 +374,10 @@ PipePlan pipe_plan(tri_dtype dt, int G, int64_t U, int64_t cap, int64_t B) {
     return p;
 }
 
+// Rows of a page of a paged pool: whole score tiles (128 bf16 / 64 float32
+// keys) per page.
+constexpr int64_t kPageRowQuantum = 128;
+
 // Which kernel paths can serve a call: 0 every path; 1 the pipelined and
 // split paths (protected keys, per-layer budgets, in-place compaction); 2
 // the split path alone (the max-over-offsets and half-split scores).
@@ -493,7 +497,7 @@ cudaError_t score_any(const tri_config* cfg, const FoldOffsets& off, tri_dtype d
     if (cfg->variant & (TRI_VAR_MAX_OFFSET | TRI_VAR_HALF_SPLIT)) {
         cudaError_t e = launch_variant_score(dt, G, a.keys, a.n_units, a.cap, a.n_valid, a.wts,
                                              stats, p_cur, n_layers, n_kvheads, cfg->theta, off,
-                                             cfg->variant, a.raw, a.flag, s);
+                                             cfg->variant, a.raw, a.flag, s, a.pm);
         if (e != cudaSuccess) return e;
         return launch_moments(a.raw, a.n_units, a.cap, a.n_valid, G, a.mom, s);
     }
@@ -772,7 +776,7 @@ static tri_status prune_impl(const tri_config* cfg, const void* k_src, const voi
                              int64_t B, void* k_dst, void* v_dst, int32_t* pos_dst,
                              int64_t cap_dst, int32_t* kept_idx, int32_t* n_kept,
                              float* final_score, void* ws, size_t ws_bytes, void* stream,
-                             bool inplace) {
+                             bool inplace, const PageMap* paged = nullptr) {
     LaunchScope scope_;
     FoldOffsets off;
     TRI_TRY(check_cfg(cfg, &off));
@@ -790,7 +794,14 @@ static tri_status prune_impl(const tri_config* cfg, const void* k_src, const voi
         return TRI_ERR_INVALID_ARG;
     const int64_t U = n_seq * n_layers * n_kvheads;
     const size_t esz = dt == TRI_BF16 ? 2 : 4;
-    if (inplace) {
+    if (paged) {
+        const size_t pool = static_cast<size_t>(paged->n_pages * paged->rows) * kD * esz;
+        const size_t pb = static_cast<size_t>(U * cap_src) * 4;
+        if ((v_src && overlaps(k_src, pool, v_src, pool)) || (pos_src && overlaps(k_src, pool, pos_src, pb)) ||
+            (v_src && pos_src && overlaps(v_src, pool, pos_src, pb)) ||
+            (n_valid && static_cast<const void*>(n_valid) == static_cast<const void*>(n_kept)))
+            return TRI_ERR_INVALID_ARG;
+    } else if (inplace) {
         if (inplace_buffers_overlap(k_src, v_src, pos_src, U, cap_src, esz) ||
             (n_valid && static_cast<const void*>(n_valid) == static_cast<const void*>(n_kept)))
             return TRI_ERR_INVALID_ARG;
@@ -798,7 +809,7 @@ static tri_status prune_impl(const tri_config* cfg, const void* k_src, const voi
                                       cap_dst, esz)) {
         return TRI_ERR_INVALID_ARG;
     }
-    const int restrict_to = path_restriction(cfg, inplace);
+    const int restrict_to = paged ? kSplitOnly : path_restriction(cfg, inplace);
     const PruneWs w = prune_ws(n_seq, n_layers, n_kvheads, G, cap_src, B, dt, kept_idx == nullptr,
                                cfg->path, inplace, restrict_to);
     if (cfg->path == TRI_PATH_FUSED && !w.fused) return TRI_ERR_UNSUPPORTED;
@@ -940,7 +951,8 @@ static tri_status prune_impl(const tri_config* cfg, const void* k_src, const voi
     }
 
     CUtensorMap map;
-    TRI_TRY(make_key_map(&map, k_src, dt, U * cap_src, score_tile_keys(dt)));
+    TRI_TRY(make_key_map(&map, k_src, dt, paged ? paged->n_pages * paged->rows : U * cap_src,
+                         score_tile_keys(dt)));
     // Zero the flag word, the moment counters and the radix histograms.
     TRI_CUDA(cudaMemsetAsync(ws, 0, kWsHeader, s));
     TRI_CUDA(cudaMemsetAsync(ws_at(ws, w.sc.counters), 0, static_cast<size_t>(U) * 4, s));
@@ -960,6 +972,7 @@ static tri_status prune_impl(const tri_config* cfg, const void* k_src, const voi
     a.counters = reinterpret_cast<uint32_t*>(ws_at(ws, w.sc.counters));
     a.mom = reinterpret_cast<float2*>(ws_at(ws, w.sc.mom));
     a.flag = flag;
+    if (paged) a.pm = *paged;
     const int n_sm = device_info().sm_count;
     TRI_CUDA(score_any(cfg, off, dt, G, map, a, stats, p_cur, n_layers, n_kvheads, n_sm, s));
     float* fin = final_score ? final_score : reinterpret_cast<float*>(ws_at(ws, w.fin));
@@ -973,7 +986,8 @@ static tri_status prune_impl(const tri_config* cfg, const void* k_src, const voi
                             n_kept, s));
     if (inplace)
         return cuda_status(launch_compact_inplace(dt, k_dst, v_dst, pos_dst, U, cap_src, kept,
-                                                  n_kept, B, flag, n_sm * 8, s));
+                                                  n_kept, B, flag, n_sm * 8, s,
+                                                  paged ? *paged : PageMap()));
     return cuda_status(launch_gather(dt, k_src, v_src, pos_src, U, cap_src, kept, n_kept, B, k_dst,
                                      v_dst, pos_dst, cap_dst, flag, n_sm * 8, s));
 }
@@ -990,6 +1004,28 @@ tri_status tri_prune(const tri_config* cfg, const void* k_src, const void* v_src
                       final_score, ws, ws_bytes, stream, false);
 }
 
+tri_status tri_prune_paged_inplace(const tri_config* cfg, void* k_pool, void* v_pool, int32_t* pos,
+                                   tri_dtype dt, int64_t n_seq, int64_t n_layers,
+                                   int64_t n_kvheads, int G, int64_t cap, const int32_t* n_valid,
+                                   const int64_t* p_cur, const float* stats, int64_t B,
+                                   const int32_t* page_table, int64_t page_rows,
+                                   int64_t pages_per_unit, int64_t n_pages, int32_t* kept_idx,
+                                   int32_t* n_kept, float* final_score, void* ws, size_t ws_bytes,
+                                   void* stream) {
+    if (!page_table || !aligned4(page_table) || page_rows < 1 || page_rows % kPageRowQuantum != 0 ||
+        n_pages < 1 || pages_per_unit < 1 || cap < 1 || pages_per_unit * page_rows < cap ||
+        n_pages * page_rows > INT32_MAX)
+        return TRI_ERR_INVALID_ARG;
+    PageMap pm;
+    pm.table = page_table;
+    pm.rows = page_rows;
+    pm.per_unit = pages_per_unit;
+    pm.n_pages = n_pages;
+    return prune_impl(cfg, k_pool, v_pool, pos, dt, n_seq, n_layers, n_kvheads, G, cap, n_valid,
+                      p_cur, stats, B, k_pool, v_pool, pos, cap, kept_idx, n_kept, final_score, ws,
+                      ws_bytes, stream, true, &pm);
+}
+
 tri_status tri_prune_inplace(const tri_config* cfg, void* k, void* v, int32_t* pos,
                              tri_dtype dt, int64_t n_seq, int64_t n_layers, int64_t n_kvheads,
                              int G, int64_t cap, const int32_t* n_valid, const int64_t* p_cur,
@@ -998,6 +1034,50 @@ tri_status tri_prune_inplace(const tri_config* cfg, void* k, void* v, int32_t* p
     return prune_impl(cfg, k, v, pos, dt, n_seq, n_layers, n_kvheads, G, cap, n_valid, p_cur,
                       stats, B, k, v, pos, cap, kept_idx, n_kept, final_score, ws, ws_bytes,
                       stream, true);
+}
+
+tri_status tri_logit_reconstruct(const tri_config* cfg, const float* q_stats,
+                                 const float* k_stats, int64_t n_qheads, int G,
+                                 const int64_t* deltas, int64_t n_delta, float* recon,
+                                 void* stream) {
+    LaunchScope scope_;
+    FoldOffsets off;
+    TRI_TRY(check_cfg(cfg, &off));
+    if (!q_stats || !k_stats || !deltas || !recon || n_qheads < 1 || G < 1 || n_delta < 1 ||
+        n_qheads % G != 0)
+        return TRI_ERR_INVALID_ARG;
+    if (n_qheads > 65535) return TRI_ERR_UNSUPPORTED;
+    if (!aligned4(q_stats) || !aligned4(k_stats) || !aligned4(recon) ||
+        (reinterpret_cast<uintptr_t>(deltas) & 7))
+        return TRI_ERR_INVALID_ARG;
+    return cuda_status(launch_logit_reconstruct(q_stats, k_stats, n_qheads, G, cfg->theta, deltas,
+                                                n_delta, recon,
+                                                static_cast<cudaStream_t>(stream)));
+}
+
+tri_status tri_logit_curve(const void* q_post, const void* k_post, tri_dtype dt, int64_t n_qheads,
+                           int G, int64_t n_tok, int head_dim, const int64_t* deltas,
+                           int64_t n_delta, float* curve, void* stream) {
+    LaunchScope scope_;
+    if (!q_post || !k_post || !deltas || !curve || n_qheads < 1 || G < 1 || n_tok < 1 ||
+        n_delta < 1 || n_qheads % G != 0)
+        return TRI_ERR_INVALID_ARG;
+    if (!dtype_ok(dt) || head_dim != kD) return TRI_ERR_UNSUPPORTED;
+    if (n_qheads > 65535 || n_delta > INT32_MAX) return TRI_ERR_UNSUPPORTED;
+    if (!aligned4(q_post) || !aligned4(k_post) || !aligned4(curve) ||
+        (reinterpret_cast<uintptr_t>(deltas) & 7))
+        return TRI_ERR_INVALID_ARG;
+    return cuda_status(launch_logit_curve(dt, q_post, k_post, n_qheads, G, n_tok, deltas, n_delta,
+                                          curve, static_cast<cudaStream_t>(stream)));
+}
+
+tri_status tri_pearson(const float* a, const float* b, int64_t n_rows, int64_t n, float* r,
+                       void* stream) {
+    LaunchScope scope_;
+    if (!a || !b || !r || n_rows < 1 || n < 1) return TRI_ERR_INVALID_ARG;
+    if (n_rows > INT32_MAX) return TRI_ERR_UNSUPPORTED;
+    if (!aligned4(a) || !aligned4(b) || !aligned4(r)) return TRI_ERR_INVALID_ARG;
+    return cuda_status(launch_pearson(a, b, n_rows, n, r, static_cast<cudaStream_t>(stream)));
 }
 
 size_t tri_decode_workspace_bytes(int64_t n_units, int G, int64_t cap) {

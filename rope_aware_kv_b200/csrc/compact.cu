@@ -118,7 +118,8 @@ template <int kVec>
 __global__ void __launch_bounds__(256)
 compact_inplace_kernel(uint4* __restrict__ k, uint4* __restrict__ v, int32_t* __restrict__ pos,
                        int64_t n_units, int64_t cap, const int32_t* __restrict__ kept,
-                       const int32_t* __restrict__ n_kept, int64_t B, uint32_t* flag) {
+                       const int32_t* __restrict__ n_kept, int64_t B, uint32_t* flag,
+                       const PageMap pm) {
     constexpr int kThreads = 256;
     constexpr int kRows = 64;                        // destination rows per round
     constexpr int kPer = kRows * kVec / kThreads;    // vectors per thread per array
@@ -133,8 +134,9 @@ compact_inplace_kernel(uint4* __restrict__ k, uint4* __restrict__ v, int32_t* __
         }
         const int32_t* ku = kept + u * B;
         for (int64_t r0 = 0; r0 < nk; r0 += kRows) {
-            // Source row of each destination row this thread moves (-1: none).
-            int64_t src[kPer];
+            // Source row of each destination row this thread moves (-1: none),
+            // and the physical rows of both (a paged pool maps them).
+            int64_t src[kPer], ps[kPer], pd[kPer];
             bool still = true;
 #pragma unroll
             for (int q = 0; q < kPer; ++q) {
@@ -142,8 +144,12 @@ compact_inplace_kernel(uint4* __restrict__ k, uint4* __restrict__ v, int32_t* __
                 src[q] = -1;
                 if (r < nk) {
                     const int64_t j = ku[r];
-                    if (j >= r && j < cap) {
+                    const int64_t pj = (j >= r && j < cap) ? phys_row(pm, u, cap, j) : -1;
+                    const int64_t pr = pj >= 0 ? phys_row(pm, u, cap, r) : -1;
+                    if (pr >= 0) {
                         src[q] = j;
+                        ps[q] = pj;
+                        pd[q] = pr;
                         still = still && j == r;
                     } else if ((tid + q * kThreads) % kVec == 0) {
                         raise_flag(flag, TRI_FLAG_INDEX_RANGE);
@@ -157,8 +163,8 @@ compact_inplace_kernel(uint4* __restrict__ k, uint4* __restrict__ v, int32_t* __
 #pragma unroll
             for (int q = 0; q < kPer; ++q) {
                 if (src[q] >= 0) {
-                    kv[q] = k[(u * cap + src[q]) * kVec + lane];
-                    if (v) vv[q] = v[(u * cap + src[q]) * kVec + lane];
+                    kv[q] = k[ps[q] * kVec + lane];
+                    if (v) vv[q] = v[ps[q] * kVec + lane];
                     if (pos && lane == 0) pv[q] = pos[u * cap + src[q]];
                 }
             }
@@ -167,8 +173,8 @@ compact_inplace_kernel(uint4* __restrict__ k, uint4* __restrict__ v, int32_t* __
             for (int q = 0; q < kPer; ++q) {
                 if (src[q] >= 0) {
                     const int64_t r = r0 + (tid + q * kThreads) / kVec;
-                    k[(u * cap + r) * kVec + lane] = kv[q];
-                    if (v) v[(u * cap + r) * kVec + lane] = vv[q];
+                    k[pd[q] * kVec + lane] = kv[q];
+                    if (v) v[pd[q] * kVec + lane] = vv[q];
                     if (pos && lane == 0) pos[u * cap + r] = pv[q];
                 }
             }
@@ -179,17 +185,18 @@ compact_inplace_kernel(uint4* __restrict__ k, uint4* __restrict__ v, int32_t* __
 
 cudaError_t launch_compact_inplace(tri_dtype dt, void* k, void* v, int32_t* pos, int64_t n_units,
                                    int64_t cap, const int32_t* kept, const int32_t* n_kept,
-                                   int64_t B, uint32_t* flag, int n_blocks, cudaStream_t s) {
+                                   int64_t B, uint32_t* flag, int n_blocks, cudaStream_t s,
+                                   const PageMap& pm) {
     if (n_units == 0) return cudaSuccess;
     const int grid = static_cast<int>(n_units < n_blocks ? n_units : n_blocks);
     if (dt == TRI_BF16) {
         compact_inplace_kernel<kD * 2 / 16><<<grid, 256, 0, s>>>(
             static_cast<uint4*>(k), static_cast<uint4*>(v), pos, n_units, cap, kept, n_kept, B,
-            flag);
+            flag, pm);
     } else {
         compact_inplace_kernel<kD * 4 / 16><<<grid, 256, 0, s>>>(
             static_cast<uint4*>(k), static_cast<uint4*>(v), pos, n_units, cap, kept, n_kept, B,
-            flag);
+            flag, pm);
     }
     note_launch(s);
     return cudaGetLastError();

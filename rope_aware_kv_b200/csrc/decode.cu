@@ -82,8 +82,21 @@ decode_attn_kernel(const DecodeArgs a) {
     __syncthreads();
     const T* ku = static_cast<const T*>(a.k) + u * a.cap * kD;
     const T* vu = static_cast<const T*>(a.v) + u * a.cap * kD;
+    constexpr int64_t kRowBytes = kD * sizeof(T);
+    if (t == 0 && j1 > j0) {
+        // The first tile's values into L2 while its keys are scored.
+        const int64_t r = min(static_cast<int64_t>(kDecTile), j1 - j0);
+        prefetch_l2_bulk(vu + j0 * kD, static_cast<uint32_t>(r * kRowBytes), policy_evict_first());
+    }
     for (int64_t b = j0; b < j1; b += kDecTile) {
         const int nt = static_cast<int>(min(static_cast<int64_t>(kDecTile), j1 - b));
+        if (t == 0 && b + kDecTile < j1) {
+            // The next tile's keys and values into L2 while this one is used.
+            const int64_t r = min(static_cast<int64_t>(kDecTile), j1 - b - kDecTile);
+            const uint64_t pol = policy_evict_first();
+            prefetch_l2_bulk(ku + (b + kDecTile) * kD, static_cast<uint32_t>(r * kRowBytes), pol);
+            prefetch_l2_bulk(vu + (b + kDecTile) * kD, static_cast<uint32_t>(r * kRowBytes), pol);
+        }
         // ---- scores (log2 domain) of key b + t for every head ----
         if (t < nt) {
             const T* row = ku + (b + t) * kD;

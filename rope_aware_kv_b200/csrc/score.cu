@@ -26,9 +26,18 @@
 #include "select_core.cuh"
 
 // How many key tiles ahead of its shared-memory ring the score kernel asks
-// L2 to fetch (0: no prefetch).
+// L2 to fetch (0: no prefetch), and the L2 policy of those requests (0
+// evict-first, 1 evict-normal, 2 evict-last).
 #ifndef TRI_PREFETCH_TILES
 #define TRI_PREFETCH_TILES 6
+#endif
+#ifndef TRI_PREFETCH_POLICY
+#define TRI_PREFETCH_POLICY 0
+#endif
+// 1: the score kernel only writes each tile's moment partial and a separate
+// kernel merges a unit's partials in tile order (no fence and atomic per tile).
+#ifndef TRI_SCORE_DEFER_MERGE
+#define TRI_SCORE_DEFER_MERGE 0
 #endif
 
 namespace tri {
@@ -234,13 +243,22 @@ score_kernel(const __grid_constant__ CUtensorMap kmap, ScoreArgs a) {
             if (tid == S::kMath) {
                 // Tiles are also requested into L2 kPrefetchTiles ahead of
                 // their load into the ring (TRI_PREFETCH_TILES, 0: none).
-                const char* kunit = static_cast<const char*>(a.keys) + u * a.cap * S::kRowBytes;
-                const uint64_t pol = policy_evict_first();
+                const uint64_t pol = TRI_PREFETCH_POLICY == 2   ? policy_evict_last()
+                                     : TRI_PREFETCH_POLICY == 1 ? policy_evict_normal()
+                                                                : policy_evict_first();
+                // First physical row of tile t of the unit (a page holds whole
+                // tiles); -1: the tile's page is outside the pool (flagged; its
+                // load lands zeros from beyond the tensor map).
+                auto tile_row = [&](int t) -> int64_t {
+                    return phys_row(a.pm, u, a.cap, static_cast<int64_t>(t) * S::kTile);
+                };
                 auto prefetch_tile = [&](int k) {
                     if (S::kPrefetchTiles == 0 || k >= nt) return;
                     const int t = i0 + k;
+                    const int64_t r0 = tile_row(t);
+                    if (r0 < 0) return;
                     const int rows = min(S::kTile, static_cast<int>(a.cap) - t * S::kTile);
-                    prefetch_l2_bulk(kunit + static_cast<int64_t>(t) * S::kStageBytes,
+                    prefetch_l2_bulk(static_cast<const char*>(a.keys) + r0 * S::kRowBytes,
                                      static_cast<uint32_t>(rows * S::kRowBytes), pol);
                 };
                 for (int k = S::kHSlots / 2; k < S::kHSlots / 2 + S::kPrefetchTiles; ++k)
@@ -256,8 +274,12 @@ score_kernel(const __grid_constant__ CUtensorMap kmap, ScoreArgs a) {
                     }
                     uint64_t* landed = &sm.full[hc % S::kHalfBars];
                     mbar_arrive_expect_tx(landed, S::kHalfBytes);
-                    const int32_t y = static_cast<int32_t>(
-                        u * a.cap + static_cast<int64_t>(i0 + (hh >> 1)) * S::kTile);
+                    int64_t r0 = tile_row(i0 + (hh >> 1));
+                    if (r0 < 0) {
+                        raise_flag(a.flag, TRI_FLAG_INDEX_RANGE);
+                        r0 = INT32_MAX - S::kTile;  // past the map: zero fill
+                    }
+                    const int32_t y = static_cast<int32_t>(r0);
 #pragma unroll
                     for (int b = 0; b < S::kHalfBoxes; ++b)
                         tma_load_2d(sm.ring[slot] + b * S::kBoxBytes, &kmap, landed,
@@ -324,9 +346,12 @@ score_kernel(const __grid_constant__ CUtensorMap kmap, ScoreArgs a) {
                         part[2 * h] = m1[h];
                         part[2 * h + 1] = m2[h];
                     }
-                    __threadfence();
-                    done = atomicAdd(&a.counters[u], 1u);
+                    if (!TRI_SCORE_DEFER_MERGE) {
+                        __threadfence();
+                        done = atomicAdd(&a.counters[u], 1u);
+                    }
                 }
+                if (TRI_SCORE_DEFER_MERGE) continue;
                 done = __shfl_sync(0xffffffffu, done, 0);
                 if (done == static_cast<uint32_t>(ntv) - 1u) {
                     // The last tile of the unit: merge every tile's partial.
@@ -347,6 +372,18 @@ score_kernel(const __grid_constant__ CUtensorMap kmap, ScoreArgs a) {
         while (globaltimer_ns() - t0 < 100000) __nanosleep(1000);
     }
     __syncthreads();
+}
+
+// The deferred merge: one warp per unit sums the unit's tile partials in
+// tile order (the same arithmetic as the in-kernel merge).
+template <int G>
+__global__ void __launch_bounds__(32)
+moment_merge_kernel(const double* __restrict__ partial, int64_t tpu, int64_t cap, int tile,
+                    const int32_t* __restrict__ n_valid, float2* __restrict__ mom) {
+    const int64_t u = blockIdx.x;
+    const int n = clamp_nvalid(n_valid, u, cap, nullptr);
+    const int ntv = (n + tile - 1) / tile;
+    merge_unit_moments<G>(partial + u * tpu * G * 2, ntv, n, mom + u * G);
 }
 
 // ---------------------------------------------------------------------------
@@ -422,6 +459,11 @@ static cudaError_t launch_score_t(const CUtensorMap& map, const ScoreArgs& a, in
     const int64_t total = a.n_units * a.tpu;
     const int grid = static_cast<int>(total < n_sm ? total : n_sm);
     kern<<<grid, ScoreShape<T>::kThreads, smem, s>>>(map, a);
+    if (TRI_SCORE_DEFER_MERGE) {
+        note_launch(s);
+        moment_merge_kernel<G><<<static_cast<unsigned>(a.n_units), 32, 0, s>>>(
+            a.partial, a.tpu, a.cap, ScoreShape<T>::kTile, a.n_valid, a.mom);
+    }
     note_launch(s);
     return cudaGetLastError();
 }

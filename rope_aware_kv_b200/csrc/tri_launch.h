@@ -32,6 +32,25 @@ struct FoldConst {
 // per-unit phases), counted in their shared-memory budgets.
 constexpr size_t kFoldStaticBytes = 4096;
 
+// Paged cache layout: logical row j of unit u lives in physical page
+// table[u * per_unit + j / rows] of a pool of n_pages pages of `rows` rows.
+// With no table the layout is contiguous: unit u's rows start at u * cap.
+struct PageMap {
+    const int32_t* table = nullptr;
+    int64_t rows = 0;
+    int64_t per_unit = 0;
+    int64_t n_pages = 0;
+};
+
+// Physical row of logical row j of unit u, or -1 when its page index is
+// outside the pool.
+__device__ __forceinline__ int64_t phys_row(const PageMap& pm, int64_t u, int64_t cap, int64_t j) {
+    if (!pm.table) return u * cap + j;
+    const int64_t pg = pm.table[u * pm.per_unit + j / pm.rows];
+    if (pg < 0 || pg >= pm.n_pages) return -1;
+    return pg * pm.rows + j % pm.rows;
+}
+
 struct ScoreArgs {
     const void* keys;            // [U][cap][128] (for L2 prefetch; loads go through the map)
     int64_t n_units;
@@ -44,6 +63,7 @@ struct ScoreArgs {
     uint32_t* counters;          // [U], zero on entry
     float2* mom;                 // [U][G] (mu, 1/sigma)
     uint32_t* flag;
+    PageMap pm;                  // paged key pool (table null: contiguous [U][cap])
 };
 
 struct FusedArgs {
@@ -206,7 +226,8 @@ cudaError_t launch_variant_score(tri_dtype dt, int G, const void* keys, int64_t 
                                  int64_t cap, const int32_t* n_valid, const float* wts,
                                  const float* stats, const int64_t* p_cur, int64_t n_layers,
                                  int64_t n_kvheads, double theta, const FoldOffsets& off,
-                                 int variant, float* raw, uint32_t* flag, cudaStream_t s);
+                                 int variant, float* raw, uint32_t* flag, cudaStream_t s,
+                                 const PageMap& pm = PageMap());
 cudaError_t launch_moments(const float* raw, int64_t n_units, int64_t cap, const int32_t* n_valid,
                            int G, float2* mom, cudaStream_t s);
 cudaError_t launch_unit_budget(const int32_t* layer_budget, int64_t n_units, int64_t n_layers,
@@ -218,6 +239,16 @@ size_t decode_part_bytes(int64_t n_units, int G, int64_t cap, int n_sm);
 cudaError_t launch_decode(tri_dtype dt, int G, const void* q, const void* k, const void* v,
                           int64_t n_units, int64_t cap, const int32_t* n_valid, float scale,
                           float* out, float* part, uint32_t* flag, int n_sm, cudaStream_t s);
+
+// logit.cu: logit(Delta) from the centres, measured, and their correlation.
+cudaError_t launch_logit_reconstruct(const float* qs, const float* ks, int64_t n_qheads, int G,
+                                     double theta, const int64_t* deltas, int64_t n_delta,
+                                     float* recon, cudaStream_t s);
+cudaError_t launch_logit_curve(tri_dtype dt, const void* q, const void* k, int64_t n_qheads, int G,
+                               int64_t n_tok, const int64_t* deltas, int64_t n_delta, float* curve,
+                               cudaStream_t s);
+cudaError_t launch_pearson(const float* a, const float* b, int64_t n_rows, int64_t n, float* r,
+                           cudaStream_t s);
 
 // zselect.cu: top-B by z-bins on the split path (zhist from launch_zmax with
 // zbins; counts [U][chunks] and cand [U][kCandMax] scratch, cand_count [U]
@@ -244,9 +275,11 @@ cudaError_t launch_gather(tri_dtype dt, const void* k_src, const void* v_src,
                           const int32_t* kept, const int32_t* n_kept, int64_t B, void* k_dst,
                           void* v_dst, int32_t* pos_dst, int64_t cap_dst, uint32_t* flag,
                           int n_blocks, cudaStream_t s);
+// pm: paged K/V pool (positions stay [U][cap]); default contiguous.
 cudaError_t launch_compact_inplace(tri_dtype dt, void* k, void* v, int32_t* pos, int64_t n_units,
                                    int64_t cap, const int32_t* kept, const int32_t* n_kept,
-                                   int64_t B, uint32_t* flag, int n_blocks, cudaStream_t s);
+                                   int64_t B, uint32_t* flag, int n_blocks, cudaStream_t s,
+                                   const PageMap& pm = PageMap());
 cudaError_t launch_append(tri_dtype dt, void* k_cache, void* v_cache, int32_t* pos_cache,
                           int64_t n_seq, int64_t n_units, int64_t cap, int32_t* n_valid,
                           int64_t* p_cur, const void* k_new, const void* v_new,

@@ -44,6 +44,7 @@ struct VariantArgs {
     int variant;
     float* raw;                // [U][G][cap]
     uint32_t* flag;
+    PageMap pm;                // paged key pool, or contiguous
 };
 
 template <typename T, int G>
@@ -58,9 +59,11 @@ variant_score_kernel(const T* __restrict__ keys, const VariantArgs a) {
     const int t = threadIdx.x;
     const int j = blockIdx.x * kVarThreads + t;
     if (blockIdx.x * kVarThreads >= n) return;  // uniform over the block
-    const bool valid = j < n;
+    const int64_t pr = j < n ? phys_row(a.pm, u, a.cap, j) : -1;
+    if (j < n && pr < 0) raise_flag(a.flag, TRI_FLAG_INDEX_RANGE);
+    const bool valid = pr >= 0;
     if (valid) {
-        const T* row = keys + (u * a.cap + j) * kD;
+        const T* row = keys + pr * kD;
         for (int f = 0; f < kF; ++f) {
             const float x = to_float(row[a.half ? f : 2 * f]);
             const float y = to_float(row[a.half ? f + kF : 2 * f + 1]);
@@ -206,8 +209,10 @@ cudaError_t launch_variant_score(tri_dtype dt, int G, const void* keys, int64_t 
                                  int64_t cap, const int32_t* n_valid, const float* wts,
                                  const float* stats, const int64_t* p_cur, int64_t n_layers,
                                  int64_t n_kvheads, double theta, const FoldOffsets& off,
-                                 int variant, float* raw, uint32_t* flag, cudaStream_t s) {
+                                 int variant, float* raw, uint32_t* flag, cudaStream_t s,
+                                 const PageMap& pm) {
     VariantArgs a;
+    a.pm = pm;
     a.cap = cap;
     a.n_valid = n_valid;
     a.wts = wts;

@@ -223,3 +223,64 @@ def test_prune_inplace_refuses_paths_without_it(path):
     with pytest.raises(tri.TriError):
         tri.tri_prune_inplace(tri.config(), wl.k, wl.v, wl.pos, spec.n_seq, spec.n_layers,
                               spec.n_kvheads, spec.G, wl.p_cur, gst, spec.B, nv, n_valid=nv)
+
+
+@pytest.mark.parametrize("dtype,variant", [("bf16", 0), ("f32", 0), ("bf16", tri.VAR_MAX_OFFSET)])
+def test_prune_paged_inplace_equals_contiguous(dtype, variant):
+    """A paged cache (128-row pages in a shuffled pool, one page table row per
+    unit) pruned in place gives the contiguous prune's kept indices, counts
+    and final scores, and its logical rows 0 .. n_kept-1 hold the same rows."""
+    B, cap, page = 300, 700, 128
+    spec = _spec(dtype=dtype, G=4, cap=cap, B=B)
+    U = spec.n_units
+    wl = synth.make_workload(spec, "cuda")
+    gst, _ = H.stats_for(spec, wl)
+    nv_h = _ragged(spec, B)
+    nv = torch.as_tensor(nv_h, device="cuda")
+    ppu = (cap + page - 1) // page
+    n_pages = U * ppu + 5
+    rng = np.random.default_rng(9)
+    table_h = rng.permutation(n_pages)[:U * ppu].reshape(U, ppu).astype(np.int32)
+    table = torch.as_tensor(table_h, device="cuda")
+    k_pool = torch.zeros((n_pages, page, 128), dtype=wl.k.dtype, device="cuda")
+    v_pool = torch.zeros_like(k_pool)
+    for u in range(U):
+        for p in range(ppu):
+            rows = min(page, cap - p * page)
+            k_pool[table_h[u, p], :rows] = wl.k[u, p * page:p * page + rows]
+            v_pool[table_h[u, p], :rows] = wl.v[u, p * page:p * page + rows]
+    pos = wl.pos.clone()
+    cfg = tri.config(variant=variant, path=tri.PATH_SPLIT)
+    ws = tri.workspace(tri.tri_prune_workspace_bytes(spec.n_seq, spec.n_layers, spec.n_kvheads, 4,
+                                                     cap, B))
+    kd = torch.zeros((U, B, 128), dtype=wl.k.dtype, device="cuda")
+    vd = torch.zeros_like(kd)
+    pd = torch.full((U, B), -1, dtype=torch.int32, device="cuda")
+    kept_a = torch.empty((U, B), dtype=torch.int32, device="cuda")
+    nk_a = torch.empty((U,), dtype=torch.int32, device="cuda")
+    fin_a = torch.full((U, cap), float("nan"), device="cuda")
+    tri.tri_prune(cfg, wl.k, wl.v, wl.pos, spec.n_seq, spec.n_layers, spec.n_kvheads, 4,
+                  wl.p_cur, gst, B, kd, vd, pd, nk_a, n_valid=nv, kept=kept_a, ws=ws, final=fin_a)
+    assert tri.tri_check_device_error(ws) == 0
+    kept_b = torch.empty((U, B), dtype=torch.int32, device="cuda")
+    nk_b = torch.empty((U,), dtype=torch.int32, device="cuda")
+    fin_b = torch.full((U, cap), float("nan"), device="cuda")
+    tri.tri_prune_paged_inplace(cfg, k_pool, v_pool, pos, table, cap, spec.n_seq, spec.n_layers,
+                                spec.n_kvheads, 4, wl.p_cur, gst, B, nk_b, n_valid=nv,
+                                kept=kept_b, ws=ws, final=fin_b)
+    assert tri.tri_check_device_error(ws) == 0
+    assert torch.equal(kept_a, kept_b) and torch.equal(nk_a, nk_b)
+    for u in range(U):
+        n = int(nv_h[u])
+        if n > B:
+            assert torch.equal(fin_a[u, :n], fin_b[u, :n])
+        m = int(nk_b[u])
+        logical_k = torch.cat([k_pool[table_h[u, p]] for p in range(ppu)])[:cap]
+        logical_v = torch.cat([v_pool[table_h[u, p]] for p in range(ppu)])[:cap]
+        assert torch.equal(logical_k[:m], kd[u, :m]) and torch.equal(logical_v[:m], vd[u, :m])
+        assert torch.equal(pos[u, :m], pd[u, :m])
+        assert torch.equal(logical_k[m:], wl.k[u, m:])
+    with pytest.raises(tri.TriError):
+        tri.tri_prune_paged_inplace(tri.config(path=tri.PATH_PIPE), k_pool, v_pool, pos, table, cap,
+                                    spec.n_seq, spec.n_layers, spec.n_kvheads, 4, wl.p_cur, gst, B,
+                                    nk_b, n_valid=nv)

@@ -131,3 +131,56 @@ def test_calibration_split_validation_without_gpu(lib):
     assert lib.tri_calibrate_finish(sums, 2, 0, 128, stats, None) == 1
     assert lib.tri_calibrate_finish(sums, 2, 100, 64, stats, None) == 2
     assert lib.tri_calibrate_finish(sums + 4, 2, 100, 128, stats, None) == 1
+
+
+def test_new_entry_points_validate_on_the_host(lib):
+    """In-place / paged prune, decode attention, the logit(Delta) calls and
+    the config's variant fields refuse bad arguments before any launch
+    (fake, never dereferenced addresses)."""
+    P = ctypes.c_void_p
+    k, v, pos = P(1 << 36), P(1 << 37), P(1 << 38)
+    cfg = tri.config()
+
+    def inplace(c, **o):
+        a = dict(k=k, v=v, pos=pos, n_valid=P(1 << 39), n_kept=P(1 << 40))
+        a.update(o)
+        return lib.tri_prune_inplace(ctypes.byref(c), a["k"], a["v"], a["pos"], tri.TRI_BF16, 1,
+                                     1, 4, 7, 4096, a["n_valid"], P(16), P(16), 512, None,
+                                     a["n_kept"], None, None, 0, None)
+    assert inplace(cfg, n_kept=P(1 << 39)) == 1            # n_kept is n_valid
+    assert inplace(cfg, v=P((1 << 36) + 4096)) == 1         # K and V overlap
+    assert inplace(tri.config(path=tri.PATH_FUSED)) in (2, 1)
+    assert inplace(tri.config(path=tri.PATH_COOP)) in (2, 1)
+    assert inplace(tri.config(variant=0x10)) == 1           # unknown variant bit
+    assert inplace(tri.config(n_sink=-1)) == 1
+    assert inplace(tri.config(barrier_wait_ns=-5)) == 1
+
+    def paged(rows, ppu=40, n_pages=200, table=P(1 << 41)):
+        return lib.tri_prune_paged_inplace(ctypes.byref(cfg), k, v, pos, tri.TRI_BF16, 1, 1, 4,
+                                           7, 4096, None, P(16), P(16), 512, table, rows, ppu,
+                                           n_pages, None, P(1 << 40), None, None, 0, None)
+    assert paged(100) == 1                                   # not whole score tiles
+    assert paged(128, ppu=8) == 1                            # pages do not cover cap
+    assert paged(128, table=None) == 1
+    assert paged(128, n_pages=0) == 1
+
+    q, out, ws = P(1 << 36), P(1 << 42), P(1 << 43)
+    assert lib.tri_decode_attention(q, k, v, tri.TRI_BF16, 4, 7, 2048, 128, None,
+                                    ctypes.c_float(0.0), out, ws, 1 << 20, None) == 1
+    assert lib.tri_decode_attention(q, k, v, tri.TRI_BF16, 4, 9, 2048, 128, None,
+                                    ctypes.c_float(0.1), out, ws, 1 << 20, None) == 2
+    assert lib.tri_decode_attention(q, k, v, tri.TRI_BF16, 4, 7, 2048, 64, None,
+                                    ctypes.c_float(0.1), out, ws, 1 << 20, None) == 2
+    assert lib.tri_decode_attention(P((1 << 36) + 4), k, v, tri.TRI_BF16, 4, 7, 2048, 128, None,
+                                    ctypes.c_float(0.1), out, ws, 1 << 20, None) == 1
+    assert lib.tri_decode_workspace_bytes(4, 7, 2048) >= 256
+
+    d = P(1 << 44)
+    assert lib.tri_logit_curve(q, k, tri.TRI_BF16, 8, 3, 100, 128, d, 10, out, None) == 1  # 8 % 3
+    assert lib.tri_logit_curve(q, k, tri.TRI_BF16, 8, 2, 100, 64, d, 10, out, None) == 2
+    assert lib.tri_logit_curve(q, k, tri.TRI_BF16, 8, 2, 100, 128, P((1 << 44) + 4), 10, out,
+                               None) == 1                    # deltas not 8-byte aligned
+    assert lib.tri_logit_reconstruct(ctypes.byref(cfg), P(16), P(16), 8, 3, d, 10, out, None) == 1
+    assert lib.tri_pearson(P(16), P(16), 0, 10, out, None) == 1
+    assert lib.tri_calibrate_ex(ctypes.byref(tri.config(variant=0x40)), q, tri.TRI_BF16, 2, 100,
+                                128, None, P(16), ws, 1 << 20, None) == 1

@@ -14,18 +14,21 @@
 // maximum grows), then either writes o_h (one chunk per unit) or its
 // (maximum, sum, unnormalised accumulator) for a combine kernel that merges
 // the chunks in order.
-//   scores  thread t scores key t of the tile for every head (its 256-byte
-//           row through 16-byte loads, the G queries from shared memory);
-//   values  thread t owns dims 2 (t % 64) and 2 (t % 64) + 1 for the keys
-//           t / 64, t / 64 + 4, ... of the tile (4-byte coalesced loads of V),
-//           the 4 key lanes summed through shared memory at the end.
+//   scores  thread t scores keys t and t + 256 of a 512-key tile for every
+//           head (their rows through 16-byte loads, the G queries from
+//           shared memory), dims paired into packed FFMA2 products;
+//   values  thread t owns dims 2 (t % 64) and 2 (t % 64) + 1 of the keys of
+//           block t / 64 (128 consecutive keys of the tile): 4-byte loads,
+//           coalesced over the 64 threads of a block, the weights of 4 keys
+//           in one 16-byte shared load, packed FFMA2 per key and head; the 4
+//           blocks are summed through shared memory at the end.
 #include "tri_internal.cuh"
 #include "tri_launch.h"
 
 namespace tri {
 
 constexpr int kDecThreads = 256;
-constexpr int kDecTile = 256;  // keys per tile (one per thread in the score phase)
+constexpr int kDecTile = 512;  // keys per tile (two per thread in the score phase)
 
 struct DecodeArgs {
     const void* q;       // [U][G][128]
@@ -51,13 +54,70 @@ __device__ __forceinline__ float2 load_pair(const T* row, int i) {
     }
 }
 
+// Score of two keys (rows r0, r1) for every head, packed: the key's dims
+// (2j, 2j + 1) as one float2 against the query's, accumulated with FFMA2
+// into (even-dim, odd-dim) partial sums.
 template <typename T, int G>
-__global__ void __launch_bounds__(kDecThreads)
+__device__ __forceinline__ void score_two(const T* r0, const T* r1, bool has1,
+                                          const float4 (&qs)[G][kD / 4], float (&s0)[G],
+                                          float (&s1)[G]) {
+    float2 a0[G], a1[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) a0[h] = a1[h] = make_float2(0.f, 0.f);
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll 2
+        for (int i = 0; i < kD / 8; ++i) {  // 16-byte chunk i: dims 8i .. 8i + 7
+            const uint4 w0 = __ldg(reinterpret_cast<const uint4*>(r0) + i);
+            const uint4 w1 = has1 ? __ldg(reinterpret_cast<const uint4*>(r1) + i) : w0;
+            const float2 k0[4] = {make_float2(bf16_lo(w0.x), bf16_hi(w0.x)),
+                                  make_float2(bf16_lo(w0.y), bf16_hi(w0.y)),
+                                  make_float2(bf16_lo(w0.z), bf16_hi(w0.z)),
+                                  make_float2(bf16_lo(w0.w), bf16_hi(w0.w))};
+            const float2 k1[4] = {make_float2(bf16_lo(w1.x), bf16_hi(w1.x)),
+                                  make_float2(bf16_lo(w1.y), bf16_hi(w1.y)),
+                                  make_float2(bf16_lo(w1.z), bf16_hi(w1.z)),
+                                  make_float2(bf16_lo(w1.w), bf16_hi(w1.w))};
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float4 qa = qs[h][2 * i], qb = qs[h][2 * i + 1];
+                const float2 q[4] = {make_float2(qa.x, qa.y), make_float2(qa.z, qa.w),
+                                     make_float2(qb.x, qb.y), make_float2(qb.z, qb.w)};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    a0[h] = __ffma2_rn(k0[j], q[j], a0[h]);
+                    a1[h] = __ffma2_rn(k1[j], q[j], a1[h]);
+                }
+            }
+        }
+    } else {
+#pragma unroll 2
+        for (int i = 0; i < kD / 4; ++i) {  // dims 4i .. 4i + 3
+            const float4 x0 = __ldg(reinterpret_cast<const float4*>(r0) + i);
+            const float4 x1 = has1 ? __ldg(reinterpret_cast<const float4*>(r1) + i) : x0;
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float4 qv = qs[h][i];
+                a0[h] = __ffma2_rn(make_float2(x0.x, x0.y), make_float2(qv.x, qv.y), a0[h]);
+                a0[h] = __ffma2_rn(make_float2(x0.z, x0.w), make_float2(qv.z, qv.w), a0[h]);
+                a1[h] = __ffma2_rn(make_float2(x1.x, x1.y), make_float2(qv.x, qv.y), a1[h]);
+                a1[h] = __ffma2_rn(make_float2(x1.z, x1.w), make_float2(qv.z, qv.w), a1[h]);
+            }
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        s0[h] = a0[h].x + a0[h].y;
+        s1[h] = a1[h].x + a1[h].y;
+    }
+}
+
+template <typename T, int G>
+__global__ void __launch_bounds__(kDecThreads, 3)
 decode_attn_kernel(const DecodeArgs a) {
     __shared__ float4 qs[G][kD / 4];          // scale * log2(e) * q
-    __shared__ float sc[G][kDecTile];         // tile scores, then weights
+    __shared__ __align__(16) float sc[G][kDecTile];  // tile scores, then weights
     __shared__ float mrow[G], lrow[G], alpha[G];
-    __shared__ float2 red[4][G][64];          // key-lane partials of the outputs
+    __shared__ float2 red[4][G][64];          // key-block partials of the outputs
     const int t = threadIdx.x;
     const int64_t u = blockIdx.y;
     const int c = blockIdx.x;
@@ -75,7 +135,8 @@ decode_attn_kernel(const DecodeArgs a) {
         lrow[t] = 0.f;
     }
     const int dp = t & 63;   // dims 2 dp, 2 dp + 1
-    const int kl = t >> 6;   // key lane 0..3
+    const int kb = t >> 6;   // key block 0..3: keys [kb * kBlk, (kb + 1) * kBlk) of a tile
+    constexpr int kBlk = kDecTile / 4;
     float2 acc[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) acc[h] = make_float2(0.f, 0.f);
@@ -97,52 +158,17 @@ decode_attn_kernel(const DecodeArgs a) {
             prefetch_l2_bulk(ku + (b + kDecTile) * kD, static_cast<uint32_t>(r * kRowBytes), pol);
             prefetch_l2_bulk(vu + (b + kDecTile) * kD, static_cast<uint32_t>(r * kRowBytes), pol);
         }
-        // ---- scores (log2 domain) of key b + t for every head ----
+        // ---- scores (log2 domain) of keys b + t and b + t + 256 ----
         if (t < nt) {
-            const T* row = ku + (b + t) * kD;
-            float s[G];
+            const bool has1 = t + kDecThreads < nt;
+            float s0[G], s1[G];
+            score_two<T, G>(ku + (b + t) * kD, ku + (b + t + (has1 ? kDecThreads : 0)) * kD, has1,
+                            qs, s0, s1);
 #pragma unroll
-            for (int h = 0; h < G; ++h) s[h] = 0.f;
-            if constexpr (sizeof(T) == 2) {
-                // 16 x 16-byte loads: 8 bf16 components each.
-#pragma unroll 4
-                for (int i = 0; i < kD / 8; ++i) {
-                    const uint4 w = __ldg(reinterpret_cast<const uint4*>(row) + i);
-                    const float4 xa = make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
-                    const float4 xb = make_float4(bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w));
-#pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        const float4 qa = qs[h][2 * i], qb = qs[h][2 * i + 1];
-                        float r = s[h];
-                        r = fmaf(qa.x, xa.x, r);
-                        r = fmaf(qa.y, xa.y, r);
-                        r = fmaf(qa.z, xa.z, r);
-                        r = fmaf(qa.w, xa.w, r);
-                        r = fmaf(qb.x, xb.x, r);
-                        r = fmaf(qb.y, xb.y, r);
-                        r = fmaf(qb.z, xb.z, r);
-                        r = fmaf(qb.w, xb.w, r);
-                        s[h] = r;
-                    }
-                }
-            } else {
-#pragma unroll 4
-                for (int i = 0; i < kD / 4; ++i) {
-                    const float4 x = __ldg(reinterpret_cast<const float4*>(row) + i);
-#pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        const float4 qv = qs[h][i];
-                        float r = s[h];
-                        r = fmaf(qv.x, x.x, r);
-                        r = fmaf(qv.y, x.y, r);
-                        r = fmaf(qv.z, x.z, r);
-                        r = fmaf(qv.w, x.w, r);
-                        s[h] = r;
-                    }
-                }
+            for (int h = 0; h < G; ++h) {
+                sc[h][t] = s0[h];
+                if (has1) sc[h][t + kDecThreads] = s1[h];
             }
-#pragma unroll
-            for (int h = 0; h < G; ++h) sc[h][t] = s[h];
         }
         __syncthreads();
         // ---- tile maximum per head (warp h), new running maximum ----
@@ -160,6 +186,9 @@ decode_attn_kernel(const DecodeArgs a) {
                 sc[h][i] = p;
                 sum += p;
             }
+            // Weights past the tile's keys are zero (the value phase reads
+            // whole groups of 4).
+            for (int i = nt + lane; i < ((nt + 3) & ~3); i += 32) sc[h][i] = 0.f;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
             if (lane == 0) {
@@ -170,27 +199,34 @@ decode_attn_kernel(const DecodeArgs a) {
             }
         }
         __syncthreads();
-        // ---- accumulate the weighted values ----
+        // ---- accumulate the weighted values: this thread's key block ----
 #pragma unroll
         for (int h = 0; h < G; ++h) {
             const float al = alpha[h];
             acc[h].x *= al;
             acc[h].y *= al;
         }
-        for (int i = kl; i < nt; i += 4) {
-            const float2 vv = load_pair(vu + (b + i) * kD, dp);
+        const int i0 = kb * kBlk;
+        const int i1 = min(i0 + kBlk, nt);
+        for (int i = i0; i < i1; i += 4) {
+            float2 vv[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                vv[q] = i + q < i1 ? load_pair(vu + (b + i + q) * kD, dp) : make_float2(0.f, 0.f);
 #pragma unroll
             for (int h = 0; h < G; ++h) {
-                const float p = sc[h][i];
-                acc[h].x = fmaf(p, vv.x, acc[h].x);
-                acc[h].y = fmaf(p, vv.y, acc[h].y);
+                const float4 p = *reinterpret_cast<const float4*>(&sc[h][i]);
+                acc[h] = __ffma2_rn(make_float2(p.x, p.x), vv[0], acc[h]);
+                acc[h] = __ffma2_rn(make_float2(p.y, p.y), vv[1], acc[h]);
+                acc[h] = __ffma2_rn(make_float2(p.z, p.z), vv[2], acc[h]);
+                acc[h] = __ffma2_rn(make_float2(p.w, p.w), vv[3], acc[h]);
             }
         }
         __syncthreads();  // sc is rewritten by the next tile
     }
-    // ---- the 4 key lanes in a fixed order ----
+    // ---- the 4 key blocks in a fixed order ----
 #pragma unroll
-    for (int h = 0; h < G; ++h) red[kl][h][dp] = acc[h];
+    for (int h = 0; h < G; ++h) red[kb][h][dp] = acc[h];
     __syncthreads();
     for (int e = t; e < G * 64; e += kDecThreads) {
         const int h = e / 64, d2 = e % 64;

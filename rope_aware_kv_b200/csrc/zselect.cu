@@ -9,9 +9,10 @@
 // The final scores here are z-scores (maxima over the GQA group of per-head
 // standardised scores), so a linear histogram of z (2048 bins of width 1/64
 // over [-16, 16), built by the z-max kernel) places the B-th key in a bin
-// that holds few keys.  Three kernels then finish the selection with two
+// that holds few keys.  Four kernels then finish the selection with two
 // passes over the final scores (instead of two radix passes, a count and a
 // compaction):
+//   bin      per unit (one warp): the B-th key's bin b0 and the keys above it;
 //   collect  per chunk of kZChunk keys: the keys above the B-th key's bin b0
 //            are counted, the keys inside b0 (the candidates) are listed per
 //            unit (up to kCandMax).
@@ -27,11 +28,33 @@
 
 namespace tri {
 
-// Per-unit result of the rank kernel.
+// Per-unit selection state: the B-th key's z-bin b0 and the keys above it
+// (bin kernel), then the threshold key T and the ties of T kept (rank kernel).
 struct ZSelState {
+    uint32_t b0;
+    uint32_t above;
     uint32_t T;   // ordered key of the B-th key
     uint32_t kt;  // keys equal to T that are kept
 };
+
+// ---------------------------------------------------------------------------
+// bin: the z-bin of each unit's B-th key, once per unit (grid U, one warp).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(32)
+zsel_bin_kernel(int64_t cap, const int32_t* __restrict__ n_valid, int64_t B,
+                const int32_t* __restrict__ ub, const uint32_t* __restrict__ zhist,
+                ZSelState* __restrict__ st) {
+    const int64_t u = blockIdx.x;
+    const int n = clamp_nvalid(n_valid, u, cap, nullptr);
+    const int64_t Bu = unit_budget(ub, u, B);
+    if (n <= Bu || Bu == 0) return;
+    uint32_t bin, above;
+    warp_find_bin(zhist + u * kZBins, kZBins, static_cast<uint32_t>(Bu), bin, above);
+    if (threadIdx.x == 0) {
+        st[u].b0 = bin;
+        st[u].above = above;
+    }
+}
 
 __device__ __forceinline__ uint32_t block_sum_256(uint32_t v, uint32_t* red8) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -54,21 +77,14 @@ __global__ void __launch_bounds__(256)
 zsel_collect_kernel(const float* __restrict__ fin, int64_t cap, const int32_t* __restrict__ n_valid,
                     int64_t B, const int32_t* __restrict__ ub, const uint32_t* __restrict__ zhist,
                     uint2* __restrict__ counts, int2* __restrict__ cand,
-                    uint32_t* __restrict__ cand_count) {
-    __shared__ uint32_t sb0;
+                    uint32_t* __restrict__ cand_count, const ZSelState* __restrict__ st) {
     __shared__ uint32_t red8[8];
     const int64_t u = blockIdx.y;
     const int n = clamp_nvalid(n_valid, u, cap, nullptr);
     const int64_t Bu = unit_budget(ub, u, B);
     if (n <= Bu || Bu == 0) return;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (warp == 0) {
-        uint32_t bin, above;
-        warp_find_bin(zhist + u * kZBins, kZBins, static_cast<uint32_t>(Bu), bin, above);
-        if (lane == 0) sb0 = bin;
-    }
-    __syncthreads();
-    const uint32_t b0 = sb0;
+    (void)zhist;
+    const uint32_t b0 = __ldg(&st[u].b0);
     const int j0 = blockIdx.x * kZChunk;
     constexpr int kPer = kZChunk / 256;
     float f[kPer];
@@ -136,15 +152,12 @@ zsel_rank_kernel(const float* __restrict__ fin, int64_t cap, const int32_t* __re
     const int64_t Bu = unit_budget(ub, u, B);
     if (n <= Bu || Bu == 0) return;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (warp == 0) {
-        uint32_t bin, above;
-        warp_find_bin(zhist + u * kZBins, kZBins, static_cast<uint32_t>(Bu), bin, above);
-        if (lane == 0) {
-            sb0 = bin;
-            sk = static_cast<uint32_t>(Bu) - above;  // rank of the Bu-th key inside bin b0
-            sprefix = 0;
-        }
+    if (tid == 0) {
+        sb0 = st[u].b0;
+        sk = static_cast<uint32_t>(Bu) - st[u].above;  // rank of the Bu-th key inside bin b0
+        sprefix = 0;
     }
+    (void)zhist;
     const uint32_t nc_all = cand_count[u];
     const bool listed = nc_all <= static_cast<uint32_t>(kCandMax);
     const int nc = listed ? static_cast<int>(nc_all) : 0;
@@ -221,7 +234,10 @@ zsel_rank_kernel(const float* __restrict__ fin, int64_t cap, const int32_t* __re
         gt_run += gt_tot;
         eq_run += eq_tot;
     }
-    if (tid == 0) st[u] = ZSelState{T, kt};
+    if (tid == 0) {
+        st[u].T = T;
+        st[u].kt = kt;
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -307,8 +323,10 @@ cudaError_t launch_zselect(const float* fin, int64_t n_units, int64_t cap, const
     const int n_chunks = static_cast<int>((cap + kZChunk - 1) / kZChunk);
     dim3 grid(static_cast<unsigned>(n_chunks), static_cast<unsigned>(n_units));
     ZSelState* st = static_cast<ZSelState*>(state);
+    zsel_bin_kernel<<<static_cast<unsigned>(n_units), 32, 0, s>>>(cap, n_valid, B, ub, zhist, st);
+    note_launch(s);
     zsel_collect_kernel<<<grid, 256, 0, s>>>(fin, cap, n_valid, B, ub, zhist, counts, cand,
-                                             cand_count);
+                                             cand_count, st);
     note_launch(s);
     const size_t smem = static_cast<size_t>(kCandMax) * sizeof(int2);
     cudaError_t e = cudaFuncSetAttribute(zsel_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

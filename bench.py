@@ -94,8 +94,10 @@ TRAFFIC = {
     ("c2", "prune_coop_kernel"): {"bytes_per_launch": 36226304, "src": "2885885db7594c5c"},
     # profiles/prune_fused_kernel_c3-2seq_full.txt: 224 of 1792 units captured, x 8
     ("c3", "prune_fused_kernel"): {"bytes_per_launch": 6429958144, "src": "58689953c672b152"},
+    # profiles/prune_pipe_kernel_c3-2seq_full.txt: 224 of 1792 units captured, x 8
+    ("c3", "prune_pipe_kernel"): {"bytes_per_launch": 7471310848, "src": "77cc0697d9dcecdc"},
     # profiles/score_kernel_c4-1seq-2layers_full.txt: 16 of 1024 units captured, x 64
-    ("c4", "score_kernel"): {"bytes_per_launch": 39339245568, "src": "be9b26c9e0f73f28"},
+    ("c4", "score_kernel"): {"bytes_per_launch": 36444766208, "src": "d302296dd2cc3dcc"},
 }
 
 
@@ -114,6 +116,7 @@ def _code_only(text: str) -> str:
 KERNEL_SOURCE = {
     "prune_coop_kernel": "coop.cu",
     "prune_fused_kernel": "fused.cu",
+    "prune_pipe_kernel": "pipe.cu",
     "score_kernel": "score.cu",
 }
 
@@ -319,11 +322,53 @@ def cpu_baseline(spec):
                               "seconds": round(dt_one, 3)}}
 
 
+def run_reference_decode(args):
+    """The oracle's decode attention on a sample of the compacted streaming
+    cache (a few units), scaled to a whole decode step of the workload."""
+    import oracle
+
+    spec = synth.SPECS["c5"]
+    rng = np.random.default_rng(5)
+    units = min(spec.n_units, max(1, oracle.threads()))
+    q = rng.normal(size=(units, spec.G, spec.d)).astype(np.float32) * 0.1
+    k = rng.normal(size=(units, spec.B, spec.d)).astype(np.float32)
+    v = rng.normal(size=(units, spec.B, spec.d)).astype(np.float32)
+    to_bf16 = lambda a: (a.view(np.uint32) >> 16).astype(np.uint16)
+    q, k, v = to_bf16(q), to_bf16(k), to_bf16(v)
+    for _ in range(args.warmup):
+        oracle.decode_attention(q, k, v)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.decode_attention(q, k, v)
+    dt = (time.perf_counter() - t0) / args.steps
+    step_s = dt * spec.n_units / units
+    value = spec.n_seq / step_s
+    desc = (f"sampled: {units} unit(s) x {spec.B} kept rows (G={spec.G}), oracle on "
+            f"{min(units, oracle.threads())} thread(s), scaled to {spec.n_units} units")
+    line = {
+        "impl": "reference",
+        "metric": "decode-attention tokens/s over the compacted cache (all layers and KV heads)",
+        "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "decode", "sample": desc},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": os.cpu_count(),
+                         "threads": min(units, oracle.threads()), "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_reference(args, ws, rank):
     if rank != 0:
         return
     import oracle
 
+    if args.workload == "decode":
+        run_reference_decode(args)
+        return
     stream_run = args.workload == STREAM
     spec = synth.SPECS["c5" if stream_run else args.workload]
     inp, keys, desc, n_units = oracle_sample(spec, seconds_hint=0.5)
@@ -668,6 +713,9 @@ def run_tri(args, ws, rank, local):
     if args.workload == STREAM:
         run_stream_line(args, ws, rank, local)
         return
+    if args.workload == "decode":
+        run_decode_line(args, ws, rank, local)
+        return
     spec = synth.SPECS[args.workload]
     if args.n_seq:
         spec = spec.scaled(n_seq=args.n_seq)
@@ -697,7 +745,8 @@ def run_tri(args, ws, rank, local):
                                      min(args.steps, 50))
             dn, db, dms = dominant(synth.SPECS[name], srec, srec["ms_per_step"])
             srec["roofline"] = {"kernel": dn, "achieved": db / (dms * 1e-3) / 1e9 if dms > 0 else 0,
-                                "algorithmic_bytes": db, "ms_per_launch": dms}
+                                "algorithmic_bytes": db, "ms_per_launch": dms,
+                                "traffic": measured_traffic(name, dn, False)}
             subs[name] = srec
             del r2
             torch.cuda.empty_cache()
@@ -742,14 +791,17 @@ def run_tri(args, ws, rank, local):
         print(json.dumps(line), flush=True)
 
 
-def time_decode(args, dev, stream, ws, steps):
+def time_decode(args, dev, stream, ws, steps, n_seq=0):
     """Decode attention of the next token over the streaming workload's
     compacted cache (64 seqs x 28 layers x 4 KV heads, G 7, B 2048 kept rows
     per unit): K and V rows read once per step, 7.5 GB > L2.  One CUDA graph
-    of ``steps`` calls between CUDA events, max over ranks."""
+    of ``steps`` calls between CUDA events, max over ranks.  ``n_seq``: a
+    cut to fewer sequences (profiler captures)."""
     import rope_aware_kv_b200 as tri
 
     spec = synth.SPECS["c5"]
+    if n_seq:
+        spec = spec.scaled(n_seq=n_seq)
     U, B, G = spec.n_units, spec.B, spec.G
     g = torch.Generator(device=dev).manual_seed(5)
     k = torch.empty((U, B, spec.d), dtype=torch.bfloat16, device=dev)
@@ -785,12 +837,44 @@ def time_decode(args, dev, stream, ws, steps):
     torch.cuda.empty_cache()
     peak_gbs, peak_kind = measured_peaks()
     nbytes = U * B * spec.d * 2 * 2 + U * G * spec.d * (2 + 4)
-    return {"workload": "decode attention over the compacted streaming cache: 7168 units x 2048 "
+    return {"workload": f"decode attention over the compacted streaming cache: {U} units x {B} "
                         "kept bf16 rows, G 7, one query token per head",
             "ms_per_step": ms, "tokens_per_s": spec.n_seq * ws / (ms * 1e-3),
             "hbm_gbs": nbytes / (ms * 1e-3) / 1e9, "frac": nbytes / (ms * 1e-3) / 1e9 / peak_gbs,
             "bytes_per_step": nbytes, "peak_gbs": peak_gbs, "peak_kind": peak_kind,
             "launches_per_step": launches, "device_flags": flags, "steps": steps}
+
+
+def run_decode_line(args, ws, rank, local):
+    """``--workload decode``: decode attention over the compacted streaming
+    cache as the bench line (``--n-seq`` cuts it for profiler captures)."""
+    import rope_aware_kv_b200 as tri
+    from rope_aware_kv_b200 import build as tri_build
+
+    if rank == 0:
+        tri_build.build()
+    barrier(ws)
+    tri.load()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(device=dev)
+    rec = time_decode(args, dev, stream, ws, args.steps, n_seq=args.n_seq)
+    if rank == 0:
+        line = {
+            "metric": "decode-attention tokens/s over the compacted cache (all layers and KV heads)",
+            "value": rec["tokens_per_s"], "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": rec["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": rec["workload"], "parallelism": f"dp{ws} (independent units)",
+                       "l2": f"{rec['bytes_per_step'] / 2**20:.0f} MiB read per step",
+                       "timing": "one CUDA graph of K steps between CUDA events"},
+            "roofline": {"bound": "hbm", "kernel": "decode_attn_kernel", "achieved": rec["hbm_gbs"],
+                         "peak": rec["peak_gbs"], "peak_kind": rec["peak_kind"], "unit": "GB/s",
+                         "frac": rec["frac"], "traffic": None},
+            "gpu_launches": rec["launches_per_step"] * args.steps,
+            "device_flags": rec["device_flags"],
+        }
+        print(json.dumps(line), flush=True)
 
 
 def run_stream_line(args, ws, rank, local):
@@ -877,7 +961,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="tri", choices=["tri", "reference"])
-    ap.add_argument("--workload", default="c4", choices=sorted(synth.SPECS) + [STREAM])
+    ap.add_argument("--workload", default="c4", choices=sorted(synth.SPECS) + [STREAM, "decode"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the end-to-end (host buffers) measurement")

@@ -8,30 +8,27 @@
 // weights renormalised over S).  This is the consumer of what the prune step
 // keeps; K and V rows are read once each, so the kernel is bound by HBM.
 //
-// One CTA per SM (per unit, or per chunk of a unit's keys when units are
-// fewer than SMs), 256 threads.  Tiles of 32 KB of keys and 32 KB of values
-// (128 bf16 / 64 float32 rows) are staged in shared memory by bulk copies
-// (one for the keys, one for the values, completing on the stage's
-// mbarrier), three tiles in flight, so HBM streams while the CTA computes:
-//   scores  2 (bf16) or 4 (float32) threads per key, each 8 of its 16-byte
-//           chunks in an order rotated by thread (conflict-free shared
-//           loads), dims paired into packed FFMA2 products against the
-//           queries (pre-scaled by scale * log2 e), partial sums combined by
-//           shuffles;
-//   softmax one warp per head: the tile's maximum, the running maximum and
-//           sum, the accumulators' rescale factor (an online softmax);
+// Split-K over the keys when units are few: CTA (c, u) handles the keys
+// [c * chunk, (c + 1) * chunk) of unit u in tiles of 256 keys with an online
+// softmax (running maximum and sum per head, accumulators rescaled when the
+// maximum grows), then either writes o_h (one chunk per unit) or its
+// (maximum, sum, unnormalised accumulator) for a combine kernel that merges
+// the chunks in order.
+//   scores  thread t scores keys t and t + 256 of a 512-key tile for every
+//           head (their rows through 16-byte loads, the G queries from
+//           shared memory), dims paired into packed FFMA2 products;
 //   values  thread t owns dims 2 (t % 64) and 2 (t % 64) + 1 of the keys of
-//           block t / 64 (a quarter of the tile): 4-byte shared loads, the
-//           weights of 4 keys in one 16-byte load, packed FFMA2 per key and
-//           head; the 4 blocks are summed through shared memory at the end.
-// A unit split over several CTAs writes per-chunk (maximum, sum,
-// unnormalised output) that decode_combine_kernel merges in chunk order.
+//           block t / 64 (128 consecutive keys of the tile): 4-byte loads,
+//           coalesced over the 64 threads of a block, the weights of 4 keys
+//           in one 16-byte shared load, packed FFMA2 per key and head; the 4
+//           blocks are summed through shared memory at the end.
 #include "tri_internal.cuh"
 #include "tri_launch.h"
 
 namespace tri {
 
 constexpr int kDecThreads = 256;
+constexpr int kDecTile = 512;  // keys per tile (two per thread in the score phase)
 
 struct DecodeArgs {
     const void* q;       // [U][G][128]
@@ -40,136 +37,137 @@ struct DecodeArgs {
     int64_t cap;
     const int32_t* n_valid;
     float scale;
-    int64_t chunk;       // keys per CTA (a multiple of the tile)
+    int64_t chunk;       // keys per CTA (a multiple of kDecTile)
     int splits;          // CTAs per unit
     float* out;          // [U][G][128]
     float* part;         // [U][splits][G][2 + 128] when splits > 1
     uint32_t* flag;
 };
 
-// Shape of the staged tiles: 32 KB of keys and 32 KB of values per tile (128
-// bf16 or 64 float32 rows), three tiles in flight.
 template <typename T>
-struct DecShape {
-    static constexpr int kRowBytes = kD * static_cast<int>(sizeof(T));
-    static constexpr int kTileBytes = 32768;
-    static constexpr int kTile = kTileBytes / kRowBytes;          // keys per tile
-    static constexpr int kStages = 3;
-    static constexpr int kTpk = kDecThreads / kTile;               // threads per key (2 / 4)
-    static constexpr int kChunks = kRowBytes / 16 / kTpk;          // 16-byte chunks per thread
-    static constexpr int kBlk = kTile / 4;                         // keys per value block
-    static constexpr size_t kSmem = static_cast<size_t>(kStages) * 2 * kTileBytes + 1024;
-    static_assert(kChunks == 8, "chunk swizzle assumes 8 chunks per thread");
-};
+__device__ __forceinline__ float2 load_pair(const T* row, int i) {
+    if constexpr (sizeof(T) == 2) {
+        const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(row) + i);
+        return make_float2(bf16_lo(w), bf16_hi(w));
+    } else {
+        return __ldg(reinterpret_cast<const float2*>(row) + i);
+    }
+}
+
+// Score of two keys (rows r0, r1) for every head, packed: the key's dims
+// (2j, 2j + 1) as one float2 against the query's, accumulated with FFMA2
+// into (even-dim, odd-dim) partial sums.
+template <typename T, int G>
+__device__ __forceinline__ void score_two(const T* r0, const T* r1, bool has1,
+                                          const float4 (&qs)[G][kD / 4], float (&s0)[G],
+                                          float (&s1)[G]) {
+    float2 a0[G], a1[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) a0[h] = a1[h] = make_float2(0.f, 0.f);
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll 2
+        for (int i = 0; i < kD / 8; ++i) {  // 16-byte chunk i: dims 8i .. 8i + 7
+            const uint4 w0 = __ldg(reinterpret_cast<const uint4*>(r0) + i);
+            const uint4 w1 = has1 ? __ldg(reinterpret_cast<const uint4*>(r1) + i) : w0;
+            const float2 k0[4] = {make_float2(bf16_lo(w0.x), bf16_hi(w0.x)),
+                                  make_float2(bf16_lo(w0.y), bf16_hi(w0.y)),
+                                  make_float2(bf16_lo(w0.z), bf16_hi(w0.z)),
+                                  make_float2(bf16_lo(w0.w), bf16_hi(w0.w))};
+            const float2 k1[4] = {make_float2(bf16_lo(w1.x), bf16_hi(w1.x)),
+                                  make_float2(bf16_lo(w1.y), bf16_hi(w1.y)),
+                                  make_float2(bf16_lo(w1.z), bf16_hi(w1.z)),
+                                  make_float2(bf16_lo(w1.w), bf16_hi(w1.w))};
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float4 qa = qs[h][2 * i], qb = qs[h][2 * i + 1];
+                const float2 q[4] = {make_float2(qa.x, qa.y), make_float2(qa.z, qa.w),
+                                     make_float2(qb.x, qb.y), make_float2(qb.z, qb.w)};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    a0[h] = __ffma2_rn(k0[j], q[j], a0[h]);
+                    a1[h] = __ffma2_rn(k1[j], q[j], a1[h]);
+                }
+            }
+        }
+    } else {
+#pragma unroll 2
+        for (int i = 0; i < kD / 4; ++i) {  // dims 4i .. 4i + 3
+            const float4 x0 = __ldg(reinterpret_cast<const float4*>(r0) + i);
+            const float4 x1 = has1 ? __ldg(reinterpret_cast<const float4*>(r1) + i) : x0;
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float4 qv = qs[h][i];
+                a0[h] = __ffma2_rn(make_float2(x0.x, x0.y), make_float2(qv.x, qv.y), a0[h]);
+                a0[h] = __ffma2_rn(make_float2(x0.z, x0.w), make_float2(qv.z, qv.w), a0[h]);
+                a1[h] = __ffma2_rn(make_float2(x1.x, x1.y), make_float2(qv.x, qv.y), a1[h]);
+                a1[h] = __ffma2_rn(make_float2(x1.z, x1.w), make_float2(qv.z, qv.w), a1[h]);
+            }
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        s0[h] = a0[h].x + a0[h].y;
+        s1[h] = a1[h].x + a1[h].y;
+    }
+}
 
 template <typename T, int G>
-__global__ void __launch_bounds__(kDecThreads, 1)
+__global__ void __launch_bounds__(kDecThreads, 3)
 decode_attn_kernel(const DecodeArgs a) {
-    using S = DecShape<T>;
-    extern __shared__ uint8_t dsm_raw[];
-    uint8_t* stage0 = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ float4 qs[G][kD / 4];                 // scale * log2(e) * q
-    __shared__ __align__(16) float sc[G][S::kTile];  // tile scores, then weights
+    __shared__ float4 qs[G][kD / 4];          // scale * log2(e) * q
+    __shared__ __align__(16) float sc[G][kDecTile];  // tile scores, then weights
     __shared__ float mrow[G], lrow[G], alpha[G];
-    __shared__ float2 red[4][G][64];                 // key-block partials of the outputs
-    __shared__ uint64_t full[S::kStages];
-    __shared__ int abort_s;
+    __shared__ float2 red[4][G][64];          // key-block partials of the outputs
     const int t = threadIdx.x;
     const int64_t u = blockIdx.y;
     const int c = blockIdx.x;
     const int n = clamp_nvalid(a.n_valid, u, a.cap, c == 0 && t == 0 ? a.flag : nullptr);
     const int64_t j0 = static_cast<int64_t>(c) * a.chunk;
     const int64_t j1 = min(j0 + a.chunk, static_cast<int64_t>(n));
-    const int ntiles = j1 > j0 ? static_cast<int>((j1 - j0 + S::kTile - 1) / S::kTile) : 0;
     constexpr float kLog2e = 1.4426950408889634f;
     const T* qu = static_cast<const T*>(a.q) + u * G * kD;
-    const char* ku = static_cast<const char*>(a.k) + u * a.cap * S::kRowBytes;
-    const char* vu = static_cast<const char*>(a.v) + u * a.cap * S::kRowBytes;
-    const uint64_t pol = policy_evict_first();
-    // Tile i of this CTA into stage i % kStages: K rows, then V rows, one
-    // bulk copy each, both completing on the stage's barrier.
-    auto issue = [&](int i) {
-        const int64_t b = j0 + static_cast<int64_t>(i) * S::kTile;
-        const uint32_t rows = static_cast<uint32_t>(min(static_cast<int64_t>(S::kTile), j1 - b));
-        const uint32_t bytes = rows * S::kRowBytes;
-        uint8_t* st = stage0 + static_cast<size_t>(i % S::kStages) * 2 * S::kTileBytes;
-        uint64_t* bar = &full[i % S::kStages];
-        mbar_arrive_expect_tx(bar, 2 * bytes);
-        bulk_load_hint(st, ku + b * S::kRowBytes, bytes, bar, pol);
-        bulk_load_hint(st + S::kTileBytes, vu + b * S::kRowBytes, bytes, bar, pol);
-    };
-    if (t == 0) {
-        for (int i = 0; i < S::kStages; ++i) mbar_init(&full[i], 1);
-        fence_barrier_init();
-        abort_s = 0;
-        for (int i = 0; i < S::kStages && i < ntiles; ++i) issue(i);
+    for (int e = t; e < G * kD; e += kDecThreads) {
+        const float x = to_float(qu[e]) * a.scale * kLog2e;
+        reinterpret_cast<float*>(qs)[e] = x;
     }
-    for (int e = t; e < G * kD; e += kDecThreads)
-        reinterpret_cast<float*>(qs)[e] = to_float(qu[e]) * a.scale * kLog2e;
     if (t < G) {
         mrow[t] = -INFINITY;
         lrow[t] = 0.f;
     }
-    const int dp = t & 63;   // dims 2 dp, 2 dp + 1 in the value phase
-    const int kb = t >> 6;   // value block: keys [kb * kBlk, (kb + 1) * kBlk) of a tile
-    const int kk = t / S::kTpk;         // key of the score phase
-    const int part = t % S::kTpk;       // its part of the row (kChunks chunks)
-    const int sw = t & 7;               // chunk order: conflict-free 16-byte loads
+    const int dp = t & 63;   // dims 2 dp, 2 dp + 1
+    const int kb = t >> 6;   // key block 0..3: keys [kb * kBlk, (kb + 1) * kBlk) of a tile
+    constexpr int kBlk = kDecTile / 4;
     float2 acc[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) acc[h] = make_float2(0.f, 0.f);
     __syncthreads();
-    for (int i = 0; i < ntiles; ++i) {
-        const int64_t b = j0 + static_cast<int64_t>(i) * S::kTile;
-        const int nt = static_cast<int>(min(static_cast<int64_t>(S::kTile), j1 - b));
-        const uint8_t* kt = stage0 + static_cast<size_t>(i % S::kStages) * 2 * S::kTileBytes;
-        const uint8_t* vt = kt + S::kTileBytes;
-        const bool ok = mbar_wait(&full[i % S::kStages], (i / S::kStages) & 1, a.flag);
-        if (__syncthreads_or(!ok)) {
-            if (t == 0) abort_s = 1;
-            break;
+    const T* ku = static_cast<const T*>(a.k) + u * a.cap * kD;
+    const T* vu = static_cast<const T*>(a.v) + u * a.cap * kD;
+    constexpr int64_t kRowBytes = kD * sizeof(T);
+    if (t == 0 && j1 > j0) {
+        // The first tile's values into L2 while its keys are scored.
+        const int64_t r = min(static_cast<int64_t>(kDecTile), j1 - j0);
+        prefetch_l2_bulk(vu + j0 * kD, static_cast<uint32_t>(r * kRowBytes), policy_evict_first());
+    }
+    for (int64_t b = j0; b < j1; b += kDecTile) {
+        const int nt = static_cast<int>(min(static_cast<int64_t>(kDecTile), j1 - b));
+        if (t == 0 && b + kDecTile < j1) {
+            // The next tile's keys and values into L2 while this one is used.
+            const int64_t r = min(static_cast<int64_t>(kDecTile), j1 - b - kDecTile);
+            const uint64_t pol = policy_evict_first();
+            prefetch_l2_bulk(ku + (b + kDecTile) * kD, static_cast<uint32_t>(r * kRowBytes), pol);
+            prefetch_l2_bulk(vu + (b + kDecTile) * kD, static_cast<uint32_t>(r * kRowBytes), pol);
         }
-        // ---- scores (log2 domain): S::kTpk threads per key ----
-        {
-            float2 a2[G];
-#pragma unroll
-            for (int h = 0; h < G; ++h) a2[h] = make_float2(0.f, 0.f);
-            const uint8_t* row = kt + kk * S::kRowBytes;
-#pragma unroll
-            for (int cc = 0; cc < S::kChunks; ++cc) {
-                const int ch = part * S::kChunks + (cc ^ sw);
-                const uint4 w = *reinterpret_cast<const uint4*>(row + ch * 16);
-                if constexpr (sizeof(T) == 2) {
-                    const float2 k2[4] = {make_float2(bf16_lo(w.x), bf16_hi(w.x)),
-                                          make_float2(bf16_lo(w.y), bf16_hi(w.y)),
-                                          make_float2(bf16_lo(w.z), bf16_hi(w.z)),
-                                          make_float2(bf16_lo(w.w), bf16_hi(w.w))};
-#pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        const float4 qa = qs[h][2 * ch], qb = qs[h][2 * ch + 1];
-                        a2[h] = __ffma2_rn(k2[0], make_float2(qa.x, qa.y), a2[h]);
-                        a2[h] = __ffma2_rn(k2[1], make_float2(qa.z, qa.w), a2[h]);
-                        a2[h] = __ffma2_rn(k2[2], make_float2(qb.x, qb.y), a2[h]);
-                        a2[h] = __ffma2_rn(k2[3], make_float2(qb.z, qb.w), a2[h]);
-                    }
-                } else {
-                    const float4 x = make_float4(__uint_as_float(w.x), __uint_as_float(w.y),
-                                                 __uint_as_float(w.z), __uint_as_float(w.w));
-#pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        const float4 qv = qs[h][ch];
-                        a2[h] = __ffma2_rn(make_float2(x.x, x.y), make_float2(qv.x, qv.y), a2[h]);
-                        a2[h] = __ffma2_rn(make_float2(x.z, x.w), make_float2(qv.z, qv.w), a2[h]);
-                    }
-                }
-            }
+        // ---- scores (log2 domain) of keys b + t and b + t + 256 ----
+        if (t < nt) {
+            const bool has1 = t + kDecThreads < nt;
+            float s0[G], s1[G];
+            score_two<T, G>(ku + (b + t) * kD, ku + (b + t + (has1 ? kDecThreads : 0)) * kD, has1,
+                            qs, s0, s1);
 #pragma unroll
             for (int h = 0; h < G; ++h) {
-                float sv = a2[h].x + a2[h].y;
-#pragma unroll
-                for (int o = 1; o < S::kTpk; o <<= 1) sv += __shfl_xor_sync(0xffffffffu, sv, o);
-                if (part == 0 && kk < nt) sc[h][kk] = sv;
+                sc[h][t] = s0[h];
+                if (has1) sc[h][t + kDecThreads] = s1[h];
             }
         }
         __syncthreads();
@@ -177,18 +175,20 @@ decode_attn_kernel(const DecodeArgs a) {
         const int warp = t >> 5, lane = t & 31;
         for (int h = warp; h < G; h += kDecThreads / 32) {
             float mx = -INFINITY;
-            for (int k = lane; k < nt; k += 32) mx = fmaxf(mx, sc[h][k]);
+            for (int i = lane; i < nt; i += 32) mx = fmaxf(mx, sc[h][i]);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
             const float m_old = mrow[h];
             const float m_new = fmaxf(m_old, mx);
             float sum = 0.f;
-            for (int k = lane; k < nt; k += 32) {
-                const float p = exp2f(sc[h][k] - m_new);
-                sc[h][k] = p;
+            for (int i = lane; i < nt; i += 32) {
+                const float p = exp2f(sc[h][i] - m_new);
+                sc[h][i] = p;
                 sum += p;
             }
-            for (int k = nt + lane; k < ((nt + 3) & ~3); k += 32) sc[h][k] = 0.f;
+            // Weights past the tile's keys are zero (the value phase reads
+            // whole groups of 4).
+            for (int i = nt + lane; i < ((nt + 3) & ~3); i += 32) sc[h][i] = 0.f;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
             if (lane == 0) {
@@ -199,53 +199,30 @@ decode_attn_kernel(const DecodeArgs a) {
             }
         }
         __syncthreads();
-        // ---- weighted values of this thread's key block, from shared memory ----
+        // ---- accumulate the weighted values: this thread's key block ----
 #pragma unroll
         for (int h = 0; h < G; ++h) {
             const float al = alpha[h];
             acc[h].x *= al;
             acc[h].y *= al;
         }
-        const int k0 = kb * S::kBlk;
-        const int k1 = min(k0 + S::kBlk, nt);
-        for (int k = k0; k < k1; k += 4) {
+        const int i0 = kb * kBlk;
+        const int i1 = min(i0 + kBlk, nt);
+        for (int i = i0; i < i1; i += 4) {
             float2 vv[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint8_t* vr = vt + (k + q) * S::kRowBytes;
-                if (k + q >= k1) {
-                    vv[q] = make_float2(0.f, 0.f);
-                } else if constexpr (sizeof(T) == 2) {
-                    const uint32_t wv = *reinterpret_cast<const uint32_t*>(vr + dp * 4);
-                    vv[q] = make_float2(bf16_lo(wv), bf16_hi(wv));
-                } else {
-                    vv[q] = *reinterpret_cast<const float2*>(vr + dp * 8);
-                }
-            }
+            for (int q = 0; q < 4; ++q)
+                vv[q] = i + q < i1 ? load_pair(vu + (b + i + q) * kD, dp) : make_float2(0.f, 0.f);
 #pragma unroll
             for (int h = 0; h < G; ++h) {
-                const float4 p = *reinterpret_cast<const float4*>(&sc[h][k]);
+                const float4 p = *reinterpret_cast<const float4*>(&sc[h][i]);
                 acc[h] = __ffma2_rn(make_float2(p.x, p.x), vv[0], acc[h]);
                 acc[h] = __ffma2_rn(make_float2(p.y, p.y), vv[1], acc[h]);
                 acc[h] = __ffma2_rn(make_float2(p.z, p.z), vv[2], acc[h]);
                 acc[h] = __ffma2_rn(make_float2(p.w, p.w), vv[3], acc[h]);
             }
         }
-        __syncthreads();  // the stage and sc are free again
-        if (t == 0 && i + S::kStages < ntiles) {
-            fence_proxy_async();  // generic reads of the stage before the copy overwrites it
-            issue(i + S::kStages);
-        }
-    }
-    __syncthreads();
-    if (abort_s) {
-        // Copies still in flight into the stages: give them time to land.
-        if (t == 0) {
-            const uint64_t t0 = globaltimer_ns();
-            while (globaltimer_ns() - t0 < 200000) __nanosleep(1000);
-        }
-        __syncthreads();
-        return;
+        __syncthreads();  // sc is rewritten by the next tile
     }
     // ---- the 4 key blocks in a fixed order ----
 #pragma unroll
@@ -297,10 +274,8 @@ decode_combine_kernel(const float* __restrict__ part, int splits, int G, float* 
 // host side
 // ---------------------------------------------------------------------------
 int decode_splits(int64_t n_units, int64_t cap, int n_sm) {
-    // One CTA per SM (the staged tiles fill its shared memory): split units
-    // over several CTAs only when there are fewer units than SMs.
-    const int64_t tiles = (cap + DecShape<__nv_bfloat16>::kTile - 1) / DecShape<__nv_bfloat16>::kTile;
-    int64_t s = (static_cast<int64_t>(n_sm) + n_units - 1) / n_units;
+    const int64_t tiles = (cap + kDecTile - 1) / kDecTile;
+    int64_t s = (2LL * n_sm + n_units - 1) / n_units;
     if (s > tiles) s = tiles;
     if (s < 1) s = 1;
     if (s > 1024) s = 1024;
@@ -315,17 +290,9 @@ size_t decode_part_bytes(int64_t n_units, int G, int64_t cap, int n_sm) {
 template <typename T>
 static cudaError_t launch_decode_t(int G, const DecodeArgs& a, int64_t n_units, cudaStream_t s) {
     dim3 grid(static_cast<unsigned>(a.splits), static_cast<unsigned>(n_units));
-    const size_t smem = DecShape<T>::kSmem;
     switch (G) {
-#define TRI_DCASE(g)                                                                        \
-    case g: {                                                                               \
-        cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<T, g>,                      \
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,   \
-                                             static_cast<int>(smem));                       \
-        if (e != cudaSuccess) return e;                                                     \
-        decode_attn_kernel<T, g><<<grid, kDecThreads, smem, s>>>(a);                        \
-        break;                                                                              \
-    }
+#define TRI_DCASE(g) \
+    case g: decode_attn_kernel<T, g><<<grid, kDecThreads, 0, s>>>(a); break;
         TRI_DCASE(1) TRI_DCASE(2) TRI_DCASE(3) TRI_DCASE(4)
         TRI_DCASE(5) TRI_DCASE(6) TRI_DCASE(7) TRI_DCASE(8)
 #undef TRI_DCASE
@@ -346,9 +313,8 @@ cudaError_t launch_decode(tri_dtype dt, int G, const void* q, const void* k, con
     a.n_valid = n_valid;
     a.scale = scale;
     a.splits = decode_splits(n_units, cap, n_sm);
-    const int64_t tile = dt == TRI_BF16 ? DecShape<__nv_bfloat16>::kTile : DecShape<float>::kTile;
-    const int64_t tiles = (cap + tile - 1) / tile;
-    a.chunk = ((tiles + a.splits - 1) / a.splits) * tile;
+    const int64_t tiles = (cap + kDecTile - 1) / kDecTile;
+    a.chunk = ((tiles + a.splits - 1) / a.splits) * kDecTile;
     a.out = out;
     a.part = part;
     a.flag = flag;

@@ -389,8 +389,8 @@ int path_restriction(const tri_config* cfg, bool inplace) {
     return kAnyPath;
 }
 
-// In place (destination = source) only the pipelined kernel with one
-// engine warp (pieces stored in order) and the split path (in-place
+// In place (destination = source) only the pipelined kernel (one engine
+// warp then stores the pieces in order) and the split path (in-place
 // compaction kernel) serve.
 PruneWs prune_ws(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int64_t cap,
                  int64_t B, tri_dtype dt, bool own_kept, int path, bool inplace = false,
@@ -402,8 +402,7 @@ PruneWs prune_ws(int64_t n_seq, int64_t n_layers, int64_t n_kvheads, int G, int6
     if (restrict_to >= kPipeOrSplit && (path == TRI_PATH_FUSED || path == TRI_PATH_COOP)) return w;
     if (restrict_to >= kSplitOnly && path == TRI_PATH_PIPE) return w;
     if ((path == TRI_PATH_PIPE || path == TRI_PATH_AUTO) && restrict_to < kSplitOnly) {
-        PipePlan pp = pipe_plan(dt, G, U, cap, B);
-        if (inplace && pipe_engine_warps() != 1) pp.ok = false;
+        const PipePlan pp = pipe_plan(dt, G, U, cap, B);
         const CoopPlan cp0 = path == TRI_PATH_AUTO && restrict_to == kAnyPath
                                  ? coop_plan(dt, G, U, cap)
                                  : CoopPlan();

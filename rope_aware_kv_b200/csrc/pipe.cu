@@ -7,25 +7,31 @@
 // section, "normalise then aggregate"), top-B by (score desc, index asc)
 // kept in temporal order (jaedaily.cn tutorial, eviction step).
 //
-// One CTA per SM, 256 threads: seven math warps and one gather engine warp.
+// One CTA per SM, 256 threads: six math warps and two gather engine warps
+// (TRI_PIPE_ENGINE_WARPS; eight warps in all keep 255 registers a thread).
 //
 //   math warps   score, z-max and select, one unit (or one chunk of a unit)
-//                at a time.  Warp w scores tiles w, w + 7, ... of the unit
+//                at a time.  Warp w scores tiles w, w + 6, ... of the unit
 //                (a tile is 128 bf16 or 64 float32 rows, every lane on 4 or 2
 //                keys for all G heads).  Each warp streams its own tiles
-//                through a private ring of two 8 KB slots, one 64-byte column
-//                slice of the tile per slot (TMA box with the 64-byte
-//                swizzle), and issues the next slice itself as soon as it
-//                frees a slot; its next tile is requested into L2 one tile
-//                ahead.  Per-head scores go to a float32 scratch in global
-//                memory (it stays in L2), float64 moments to registers.
-//   engine warp  gathers the units the math warps have selected, in order:
-//                for each run of consecutive kept rows one cp.async.bulk
-//                load into an 8 KB buffer of 32 consecutive destination rows
-//                (four loading, six buffers), then one cp.async.bulk store of
-//                the buffer; positions follow by 4-byte cp.async.  It holds
-//                no data in registers, so the gather of unit u runs while the
-//                math warps score unit u + 1.
+//                through a private TMA ring (small units: four 4 KB slots,
+//                one 32-byte column slice of the tile per slot, 32-byte
+//                swizzle; large units: two 8 KB slots of 64-byte slices),
+//                issues the next slice itself as soon as it frees a slot, and
+//                asks L2 for its tiles two tiles ahead.  Per-head scores go
+//                to a float32 scratch in global memory (it stays in L2),
+//                float64 moments to registers.  After selecting, they write
+//                kept / n_kept and copy the kept rows' positions.
+//   engine warps gather the units the math warps have selected, in order:
+//                a piece is 32 bf16 (16 float32) destination rows, its K and
+//                V rows together in one 16 KB buffer; lane o issues the o-th
+//                cp.async.bulk load (the K or V rows of one run of
+//                consecutive kept rows), all completing on the buffer's
+//                barrier, and two lanes store the landed buffer with one
+//                cp.async.bulk store each.  Engine warp e takes pieces e,
+//                e + 2, ... (in place: warp 0 takes every piece in order).
+//                They hold no data in registers, so the gather of unit u
+//                runs while the math warps score unit u + 1.
 //
 // Hand-off: the math warps write the kept indices of a unit into one of two
 // index buffers in shared memory and arrive on its "ready" barrier; the
@@ -53,7 +59,11 @@
 namespace tri {
 
 #ifndef TRI_PIPE_ENGINE_WARPS
-#define TRI_PIPE_ENGINE_WARPS 1
+#define TRI_PIPE_ENGINE_WARPS 2
+#endif
+// Ring slots per math warp in the small-unit mode.
+#ifndef TRI_PIPE_RING_SLOTS
+#define TRI_PIPE_RING_SLOTS 4
 #endif
 // How many of its own tiles ahead a math warp asks L2 for its keys.
 #ifndef TRI_PIPE_PF_AHEAD
@@ -74,11 +84,11 @@ struct PipeShape {
     static constexpr int kSlices = kRowBytes / kSliceBytes;
     static constexpr int kSliceElems = kSliceBytes / static_cast<int>(sizeof(T));
     static constexpr int kSlotBytes = kTile * kSliceBytes;              // 4 KB / 8 KB (bf16)
-    static constexpr int kQ = kBig ? 2 : 3;                             // ring slots per math warp
+    static constexpr int kQ = kBig ? 2 : TRI_PIPE_RING_SLOTS;           // ring slots per math warp
     static constexpr int kPfAhead = TRI_PIPE_PF_AHEAD;                  // L2 prefetch, warp tiles
-    // Seven math warps and the engine (or six and two engines): 256
-    // threads, so that a thread may hold up to 255 registers (the register
-    // file is split over the four SM sub-partitions, two warps each).
+    // Six math warps and two engines (or seven and one): 256 threads, so
+    // that a thread may hold up to 255 registers (the register file is split
+    // over the four SM sub-partitions, two warps each).
     static constexpr int kEngWarps = TRI_PIPE_ENGINE_WARPS;
     static constexpr int kMathWarps = 8 - kEngWarps;
     static constexpr int kMath = 32 * kMathWarps;
@@ -91,7 +101,7 @@ struct PipeShape {
     // Gather buffers: as many as shared memory leaves room for (runtime,
     // kMinGSlots..kMaxGSlots, shared by the engine warps); all but kGGap of
     // an engine warp's buffers may be loading.
-    static constexpr int kMinGSlots = 3 * kEngWarps;
+    static constexpr int kMinGSlots = kEngWarps == 1 ? 3 : 2 * kEngWarps;
     static constexpr int kMaxGSlots = 12;
     static constexpr int kGGap = 1;
     static constexpr int kHand = 2;                // index buffers (units handed to the engine)
@@ -745,7 +755,10 @@ __device__ void pipe_engine(const PipeArgs& a, int eng, uint8_t* gbuf, int gs, c
             kx = kidx_base + slot * kidx_stride;
             smask = smask_base + slot * smask_stride;
             P = (m + S::kGRows - 1) / S::kGRows;
-            q = eng;
+            // In place, engine warp 0 takes every piece of the unit in order
+            // (a piece's store then follows the loads of every earlier
+            // piece); otherwise warp e takes pieces e, e + kEngWarps, ...
+            q = a.inplace ? (eng == 0 ? 0 : P) : eng;
             if (eng == 0) pipe_trace(a, u, 4, 0);
             if (q >= P) {
                 __syncwarp();
@@ -810,7 +823,7 @@ __device__ void pipe_engine(const PipeArgs& a, int eng, uint8_t* gbuf, int gs, c
             }
             __syncwarp();  // the run starts are read before the next piece rewrites them
             ++issued;
-            q += S::kEngWarps;
+            q += a.inplace ? 1 : S::kEngWarps;
             if (q >= P) {
                 // Every load of this warp's pieces of the unit is issued.
                 __syncwarp();

@@ -29,7 +29,8 @@
 //                consecutive kept rows), all completing on the buffer's
 //                barrier, and two lanes store the landed buffer with one
 //                cp.async.bulk store each.  Engine warp e takes pieces e,
-//                e + 2, ... (in place: warp 0 takes every piece in order).
+//                e + 2, ...; in place, a piece is stored only after the
+//                other engine's previous piece has landed.
 //                They hold no data in registers, so the gather of unit u
 //                runs while the math warps score unit u + 1.
 //
@@ -188,6 +189,8 @@ struct PipeMisc {
     uint32_t gdst_rows[PipeShape<float>::kMaxGSlots];  // engine: rows of each gather buffer
     int64_t gdst[PipeShape<float>::kMaxGSlots];        // engine: destination byte offset
     int32_t runst[2][64];                              // engine: start row of each run
+    uint64_t gseq[PipeShape<float>::kMaxGSlots];       // engine: (unit << 32) | piece of each buffer
+    uint64_t landed[2];                                // in place: 1 + last piece each engine saw land
 };
 static_assert(sizeof(PipeMisc) <= 1024, "misc state exceeds its budget");
 
@@ -716,6 +719,32 @@ __device__ void pipe_engine(const PipeArgs& a, int eng, uint8_t* gbuf, int gs, c
     auto store_one = [&]() -> bool {
         const int sl = stored % gs;
         if (!warp_wait(&gfull[sl], (stored / gs) & 1, a.flag)) return false;
+        if (S::kEngWarps > 1 && a.inplace) {
+            // In place, a piece is stored only after the piece before it
+            // (the other engine's) has landed, so that every earlier piece's
+            // source rows are read before this piece's rows are written.
+            const uint64_t seq = ms->gseq[eng * gs + sl];
+            bool ok = true;
+            if (lane == 0) {
+                volatile uint64_t* mine = &ms->landed[eng];
+                *mine = seq + 1u;
+                __threadfence_block();
+                const volatile uint64_t* other = &ms->landed[1 - eng];
+                if ((seq & 0xffffffffu) != 0u && *other < seq) {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (*other < seq) {
+                        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+                            raise_flag(a.flag, TRI_FLAG_TIMEOUT);
+                            ok = false;
+                            break;
+                        }
+                        __nanosleep(32);
+                    }
+                }
+                __threadfence_block();
+            }
+            if (!__shfl_sync(0xffffffffu, ok, 0)) return false;
+        }
         if (lane < (has_v ? 2 : 1)) {
             const int g = eng * gs + sl;
             const int64_t off = ms->gdst[g];
@@ -755,10 +784,9 @@ __device__ void pipe_engine(const PipeArgs& a, int eng, uint8_t* gbuf, int gs, c
             kx = kidx_base + slot * kidx_stride;
             smask = smask_base + slot * smask_stride;
             P = (m + S::kGRows - 1) / S::kGRows;
-            // In place, engine warp 0 takes every piece of the unit in order
-            // (a piece's store then follows the loads of every earlier
-            // piece); otherwise warp e takes pieces e, e + kEngWarps, ...
-            q = a.inplace ? (eng == 0 ? 0 : P) : eng;
+            // Warp e takes pieces e, e + kEngWarps, ... (in place, each
+            // store also waits for the other engine's previous piece).
+            q = eng;
             if (eng == 0) pipe_trace(a, u, 4, 0);
             if (q >= P) {
                 __syncwarp();
@@ -796,6 +824,7 @@ __device__ void pipe_engine(const PipeArgs& a, int eng, uint8_t* gbuf, int gs, c
                 mbar_arrive_expect_tx(landed, static_cast<uint32_t>(rows * S::kRowBytes * (has_v ? 2 : 1)));
                 ms->gdst[eng * gs + sl] = (u * a.cap_dst + r0) * S::kRowBytes;
                 ms->gdst_rows[eng * gs + sl] = static_cast<uint32_t>(rows);
+                ms->gseq[eng * gs + sl] = (static_cast<uint64_t>(hs) << 32) | static_cast<uint32_t>(q);
             }
             __syncwarp();
             uint8_t* buf = gbuf + sl * S::kGSlotBytes;
@@ -823,7 +852,7 @@ __device__ void pipe_engine(const PipeArgs& a, int eng, uint8_t* gbuf, int gs, c
             }
             __syncwarp();  // the run starts are read before the next piece rewrites them
             ++issued;
-            q += a.inplace ? 1 : S::kEngWarps;
+            q += S::kEngWarps;
             if (q >= P) {
                 // Every load of this warp's pieces of the unit is issued.
                 __syncwarp();
@@ -904,6 +933,7 @@ prune_pipe_kernel(const __grid_constant__ CUtensorMap kmap, PipeArgs a) {
         prefetch_tensormap(&kmap);
         ms->abort = 0;
         ms->stop = 0;
+        ms->landed[0] = ms->landed[1] = 0ull;
         ms->item = -1;
     }
     __syncthreads();  // barriers and state initialised before anyone uses them

@@ -473,8 +473,9 @@ KERNEL_NAMES = {
     "pipe_big": ["fold_kernel", "prune_pipe_kernel"],
     "fused": ["prune_fused_kernel"],
     "coop": ["prune_coop_kernel"],
-    "split": ["fold_kernel", "score_kernel", "zmax_kernel", "zsel_bin_kernel",
-              "zsel_collect_kernel", "zsel_rank_kernel", "zsel_compact_kernel", "gather_kernel"],
+    "split": ["fold_kernel", "score_kernel", "moment_merge_kernel", "zmax_kernel",
+              "zsel_bin_kernel", "zsel_collect_kernel", "zsel_rank_kernel", "zsel_compact_kernel",
+              "gather_kernel"],
 }
 
 

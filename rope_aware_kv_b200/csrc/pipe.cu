@@ -119,6 +119,13 @@ constexpr int kPartOff = 16384;
 // Tiles per work item of a large unit: a multiple of the math warps' count.
 constexpr int kChunkTiles = 6 * PipeShape<float>::kMathWarps;
 
+// "Full" barriers per math warp, enough for either mode's ring.
+template <typename T>
+__host__ __device__ constexpr int pipe_full_bars() {
+    return PipeShape<T, false>::kQ > 2 * PipeShape<T, true>::kQ ? PipeShape<T, false>::kQ
+                                                                  : 2 * PipeShape<T, true>::kQ;
+}
+
 struct PipeLayout {
     size_t ring, gbuf, w, fin, hist, cand, kidx, smask, bars, red, misc, total;
 };
@@ -152,7 +159,7 @@ __host__ __device__ inline PipeLayout pipe_layout(int G, int64_t cap, int64_t B,
     L.smask = o;
     o += SS::kHand * ((static_cast<size_t>((m + SS::kGRows - 1) / SS::kGRows) * 8 + 15) & ~size_t(15));
     L.bars = o;
-    o += (SS::kMathWarps * SB::kQ * 2 + SS::kMaxGSlots + 2 * SS::kHand) * 8;
+    o += (SS::kMathWarps * pipe_full_bars<T>() + SS::kMaxGSlots + 2 * SS::kHand) * 8;
     L.red = o;
     o += static_cast<size_t>(SS::kMathWarps) * kMaxG * 2 * 8;
     L.misc = o;
@@ -912,7 +919,7 @@ prune_pipe_kernel(const __grid_constant__ CUtensorMap kmap, PipeArgs a) {
     const size_t smask_stride =
         ((static_cast<size_t>((m_max + S::kGRows - 1) / S::kGRows) * 8 + 15) & ~size_t(15)) / 8;
     uint64_t* full = reinterpret_cast<uint64_t*>(base + L.bars);  // [warp][kQ]
-    uint64_t* gfull = full + S::kMathWarps * PipeShape<T, true>::kQ * 2;  // [gslots]
+    uint64_t* gfull = full + S::kMathWarps * pipe_full_bars<T>();  // [gslots]
     uint64_t* kready = gfull + S::kMaxGSlots;                       // [kHand]
     uint64_t* kfree = kready + S::kHand;                            // [kHand]
     double* red = reinterpret_cast<double*>(base + L.red);         // [warp][kMaxG][2]

@@ -95,9 +95,9 @@ TRAFFIC = {
     # profiles/prune_fused_kernel_c3-2seq_full.txt: 224 of 1792 units captured, x 8
     ("c3", "prune_fused_kernel"): {"bytes_per_launch": 6429958144, "src": "58689953c672b152"},
     # profiles/prune_pipe_kernel_c3-2seq_full.txt: 224 of 1792 units captured, x 8
-    ("c3", "prune_pipe_kernel"): {"bytes_per_launch": 7436969984, "src": "01aa86a31714db31"},
+    ("c3", "prune_pipe_kernel"): {"bytes_per_launch": 7429244928, "src": "f016fe6808e29af5"},
     # profiles/score_kernel_c4-1seq-2layers_full.txt: 16 of 1024 units captured, x 64
-    ("c4", "score_kernel"): {"bytes_per_launch": 36444766208, "src": "d302296dd2cc3dcc"},
+    ("c4", "score_kernel"): {"bytes_per_launch": 36409344000, "src": "240a52b2d38cc78e"},
 }
 
 

@@ -18,7 +18,8 @@ at 32768 keys; the windowed decode step; the streaming step), each with its
 time per step, keys/s and fraction of the HBM roofline.  Metric: keys
 scored and pruned per second, plus the achieved HBM bandwidth of the step's
 compulsory bytes (read every key, read the kept values, write the kept keys
-and values, indices and positions) against the measured copy peak.
+and values, indices and positions) against the measured copy peak (and,
+as ``hbm_frac_of_nominal``, against the nominal 8 TB/s).
 
 Timing: W warm-up steps, then K steps captured as one CUDA graph and replayed
 between CUDA events on the launching stream, with a barrier and a device
@@ -53,7 +54,11 @@ import torch  # noqa: E402
 import synth  # noqa: E402
 
 L2_BYTES = 126 * 1024 * 1024
-METRIC = "keys scored+pruned/sec and achieved HBM GB/s (% of measured copy peak) per prune step"
+METRIC = "keys scored+pruned/sec and achieved HBM GB/s (% of ~8 TB/s) per prune step"
+# The nominal HBM3e figure the metric's percentage names; the roofline
+# fractions use the measured copy peak instead (MEASURED_PEAKS.json, else the
+# 6650 GB/s fallback), which a plain copy can reach.
+NOMINAL_HBM_GBS = 8000.0
 
 WORKLOAD_TEXT = {
     "c1": "single head fp32, 4096 keys -> 512, G=1",
@@ -92,12 +97,10 @@ def fused_bytes(spec) -> int:
 TRAFFIC = {
     # profiles/prune_coop_kernel_c2_full.txt
     ("c2", "prune_coop_kernel"): {"bytes_per_launch": 36226304, "src": "2885885db7594c5c"},
-    # profiles/prune_fused_kernel_c3-2seq_full.txt: 224 of 1792 units captured, x 8
-    ("c3", "prune_fused_kernel"): {"bytes_per_launch": 6429958144, "src": "58689953c672b152"},
     # profiles/prune_pipe_kernel_c3-2seq_full.txt: 224 of 1792 units captured, x 8
-    ("c3", "prune_pipe_kernel"): {"bytes_per_launch": 7429244928, "src": "f016fe6808e29af5"},
+    ("c3", "prune_pipe_kernel"): {"bytes_per_launch": 7422631936, "src": "91d6d2f340ec24f9"},
     # profiles/score_kernel_c4-1seq-2layers_full.txt: 16 of 1024 units captured, x 64
-    ("c4", "score_kernel"): {"bytes_per_launch": 36409344000, "src": "240a52b2d38cc78e"},
+    ("c4", "score_kernel"): {"bytes_per_launch": 36379787264, "src": "e5c635935b897aaa"},
 }
 
 
@@ -772,6 +775,7 @@ def run_tri(args, ws, rank, local):
                 "timing": "one CUDA graph of K steps between CUDA events, max over ranks",
             },
             "hbm_gbs": rec["hbm_gbs"], "hbm_frac_of_peak": rec["frac"],
+            "hbm_frac_of_nominal": rec["hbm_gbs"] / NOMINAL_HBM_GBS,
             "compulsory_bytes_per_step": rec["compulsory_bytes_per_step"],
             "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": achieved,
                          "peak": peak_gbs, "peak_kind": peak_kind, "unit": "GB/s",

@@ -59,11 +59,10 @@ __device__ __forceinline__ void fold_unit_sync(FoldShared& fs, const FoldConst& 
         const double aim = trig ? tre * fc.cf[f][1] + tim * fc.cf[f][0] : 0.0;
         const double rw = (fc.variant & TRI_VAR_NO_R) ? 1.0 : 1.0 - static_cast<double>(st.w);
         const double cw = rw * static_cast<double>(st.z);
-        float* rec = w + h * kWHead + (f >> 2) * kWChunk;
-        const int i = f & 3;
-        rec[2 * i] = static_cast<float>(are);
-        rec[2 * i + 1] = static_cast<float>(aim);
-        rec[8 + i] = static_cast<float>(cw);
+        float* rec = w + h * kWHead;
+        rec[wrec_re(f)] = static_cast<float>(are);
+        rec[wrec_im(f)] = static_cast<float>(aim);
+        rec[wrec_c(f)] = static_cast<float>(cw);
     }
     sync();
 }

@@ -240,16 +240,7 @@ __device__ __forceinline__ void score_slice(const uint8_t* slot, int c0, const f
             for (int k = 0; k < KPT; ++k) {
                 const uint4 v = *reinterpret_cast<const uint4*>(slot + (lane + 32 * k) * SB +
                                                                 ((cc ^ sw) << 4));
-                const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
-                float n[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float x = bf16_lo(wd[i]), y = bf16_hi(wd[i]);
-                    xy[k][i] = make_float2(x, y);
-                    n[i] = sqrt_approx(fmaf(x, x, y * y));
-                }
-                nn[k][0] = make_float2(n[0], n[1]);
-                nn[k][1] = make_float2(n[2], n[3]);
+                band_pairs_bf16(v, xy[k], nn[k]);
             }
 #pragma unroll
             for (int h = 0; h < G; ++h) {
@@ -279,10 +270,7 @@ __device__ __forceinline__ void score_slice(const uint8_t* slot, int c0, const f
             for (int k = 0; k < KPT; ++k) {
                 const float4 v = *reinterpret_cast<const float4*>(slot + (lane + 32 * k) * SB +
                                                                   ((cc ^ sw) << 4));
-                xy[k][0] = make_float2(v.x, v.y);
-                xy[k][1] = make_float2(v.z, v.w);
-                nn[k] = make_float2(sqrt_approx(fmaf(v.x, v.x, v.y * v.y)),
-                                    sqrt_approx(fmaf(v.z, v.z, v.w * v.w)));
+                band_pair_f32(v, xy[k], nn[k]);
             }
             const int half = c & 1;
 #pragma unroll

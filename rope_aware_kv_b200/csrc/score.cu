@@ -50,7 +50,8 @@ namespace tri {
 // ---------------------------------------------------------------------------
 // Fold: per (seq, layer, query head) weights, chunk-major for the score loop.
 // Record layout per query head: 16 chunks x 12 floats; chunk c covers bands
-// 4c..4c+3: [ReA_4c, ImA_4c, ..., ReA_4c+3, ImA_4c+3, c_4c, ..., c_4c+3].
+// 4c..4c+3: [ReA_4c, ReA_4c+1, ImA_4c, ImA_4c+1, ReA_4c+2, ReA_4c+3, ImA_4c+2,
+// ImA_4c+3, c_4c, ..., c_4c+3] (wrec_re / wrec_im / wrec_c).
 // One block per (sequence, group of kFoldHeads query heads): the block first
 // forms C_f = mean_delta e^{i w_f delta} (256 threads, each a quarter of the
 // offsets of one band, merged in a fixed order) and e^{i w_f p_cur}, then
@@ -107,11 +108,10 @@ fold_kernel(const float* __restrict__ stats, const int64_t* __restrict__ p_cur, 
         const double rw = (variant & TRI_VAR_NO_R) ? 1.0 : 1.0 - static_cast<double>(st[3]);
         const double cw = rw * static_cast<double>(st[2]);
         const int64_t q = seq * LH + lh;  // (seq * L + layer) * Hq + qh
-        float* rec = wts + q * kWHead + (f >> 2) * kWChunk;
-        const int i = f & 3;
-        rec[2 * i] = static_cast<float>(are);
-        rec[2 * i + 1] = static_cast<float>(aim);
-        rec[8 + i] = static_cast<float>(cw);
+        float* rec = wts + q * kWHead;
+        rec[wrec_re(f)] = static_cast<float>(are);
+        rec[wrec_im(f)] = static_cast<float>(aim);
+        rec[wrec_c(f)] = static_cast<float>(cw);
     }
 }
 

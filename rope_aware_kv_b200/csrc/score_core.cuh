@@ -4,8 +4,10 @@
 //   s_h = sum_f (ReA_hf * x_f + ImA_hf * y_f) + sum_f c_hf * |k'_f|
 // with k'_f = x_f + i y_f the interleaved pair (x_2f, x_2f+1), A_hf the
 // offset-averaged rotated query centre and c_hf = (1 - R_hf) E|q_hf| (see
-// score.cu).  Products are formed with packed float32x2 FMAs: the (x, y) pair
-// of a band against (ReA, ImA), and two band norms against two c weights.
+// score.cu).  Products are formed with packed float32x2 FMAs on band pairs:
+// (x_i, x_i+1) against (ReA_i, ReA_i+1), (y_i, y_i+1) against (ImA_i,
+// ImA_i+1), and the pair's norms against (c_i, c_i+1); the squared norms of a
+// pair are one packed multiply and one packed FMA of the same registers.
 #pragma once
 
 #include "tri_internal.cuh"
@@ -19,6 +21,30 @@
 namespace tri {
 
 constexpr int kScoreUnroll = TRI_SCORE_UNROLL;
+
+// One 16-byte chunk of a bf16 row (bands i..i+3, words (x_i, y_i) with x in
+// the low half) as register pairs xy = {(x_i, x_i+1), (y_i, y_i+1),
+// (x_i+2, x_i+3), (y_i+2, y_i+3)} and the band norms nn = {(|k_i|, |k_i+1|),
+// (|k_i+2|, |k_i+3|)}.
+__device__ __forceinline__ void band_pairs_bf16(const uint4 v, float2 (&xy)[4], float2 (&nn)[2]) {
+    xy[0] = make_float2(bf16_lo(v.x), bf16_lo(v.y));
+    xy[1] = make_float2(bf16_hi(v.x), bf16_hi(v.y));
+    xy[2] = make_float2(bf16_lo(v.z), bf16_lo(v.w));
+    xy[3] = make_float2(bf16_hi(v.z), bf16_hi(v.w));
+    const float2 q01 = __ffma2_rn(xy[1], xy[1], __fmul2_rn(xy[0], xy[0]));
+    const float2 q23 = __ffma2_rn(xy[3], xy[3], __fmul2_rn(xy[2], xy[2]));
+    nn[0] = make_float2(sqrt_approx(q01.x), sqrt_approx(q01.y));
+    nn[1] = make_float2(sqrt_approx(q23.x), sqrt_approx(q23.y));
+}
+
+// The same for a 16-byte chunk of a float32 row (bands i, i+1: x_i, y_i,
+// x_i+1, y_i+1): xy = {(x_i, x_i+1), (y_i, y_i+1)}, nn = (|k_i|, |k_i+1|).
+__device__ __forceinline__ void band_pair_f32(const float4 v, float2 (&xy)[2], float2& nn) {
+    xy[0] = make_float2(v.x, v.z);
+    xy[1] = make_float2(v.y, v.w);
+    const float2 q = __ffma2_rn(xy[1], xy[1], __fmul2_rn(xy[0], xy[0]));
+    nn = make_float2(sqrt_approx(q.x), sqrt_approx(q.y));
+}
 
 // Chunks (16 bytes: 4 bf16 bands or 2 float32 bands) per key row.
 template <typename T>
@@ -47,16 +73,7 @@ __device__ __forceinline__ void score_rows_acc(const uint8_t* boxes, int c0, int
                 const int r = first_row + kRowStride * k;
                 const uint4 v = *reinterpret_cast<const uint4*>(
                     boxes + ((c >> 3) - box0) * kBoxBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
-                const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
-                float n[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float x = bf16_lo(wd[i]), y = bf16_hi(wd[i]);
-                    xy[k][i] = make_float2(x, y);
-                    n[i] = sqrt_approx(fmaf(x, x, y * y));
-                }
-                nn[k][0] = make_float2(n[0], n[1]);
-                nn[k][1] = make_float2(n[2], n[3]);
+                band_pairs_bf16(v, xy[k], nn[k]);
             }
 #pragma unroll
             for (int h = 0; h < G; ++h) {
@@ -86,10 +103,7 @@ __device__ __forceinline__ void score_rows_acc(const uint8_t* boxes, int c0, int
                 const int r = first_row + kRowStride * k;
                 const float4 v = *reinterpret_cast<const float4*>(
                     boxes + ((c >> 3) - box0) * kBoxBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4));
-                xy[k][0] = make_float2(v.x, v.y);
-                xy[k][1] = make_float2(v.z, v.w);
-                nn[k] = make_float2(sqrt_approx(fmaf(v.x, v.x, v.y * v.y)),
-                                    sqrt_approx(fmaf(v.z, v.z, v.w * v.w)));
+                band_pair_f32(v, xy[k], nn[k]);
             }
             const int half = c & 1;
 #pragma unroll

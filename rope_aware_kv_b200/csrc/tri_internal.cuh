@@ -19,6 +19,17 @@ constexpr int kF = kD / 2;       // RoPE bands
 constexpr int kChunks = 16;      // 16-byte chunks of a bf16 row (4 bands each)
 constexpr int kWChunk = 12;      // floats per (head, chunk) weight record: 8 w + 4 c
 constexpr int kWHead = kChunks * kWChunk;  // 192 floats per query head
+// Place of band f's weights within a head's record.  The record of chunk
+// c = f / 4 (bands 4c..4c+3, i = f % 4) is
+//   [ReA_0, ReA_1, ImA_0, ImA_1, ReA_2, ReA_3, ImA_2, ImA_3, c_0, c_1, c_2, c_3],
+// so a band pair's real parts (and its imaginary parts) are adjacent: the
+// score loop multiplies them with (x_i, x_i+1) and (y_i, y_i+1) register
+// pairs, the same pairs its packed band-norm products use.
+__host__ __device__ constexpr int wrec_re(int f) {
+    return (f >> 2) * kWChunk + ((f & 3) >> 1) * 4 + (f & 1);
+}
+__host__ __device__ constexpr int wrec_im(int f) { return wrec_re(f) + 2; }
+__host__ __device__ constexpr int wrec_c(int f) { return (f >> 2) * kWChunk + 8 + (f & 3); }
 constexpr int kMaxG = TRI_MAX_GROUP;
 
 // Flag word at the start of every workspace.

@@ -97,7 +97,7 @@ variant_score_kernel(const T* __restrict__ keys, const VariantArgs a) {
         if (!valid) continue;
         float s_norm = 0.f;
         for (int f = 0; f < kF; ++f)
-            s_norm = fmaf(__ldg(rec + (f >> 2) * kWChunk + 8 + (f & 3)), nb[f * kVarThreads + t],
+            s_norm = fmaf(__ldg(rec + wrec_c(f)), nb[f * kVarThreads + t],
                           s_norm);
         float s;
         if (a.max_off) {
@@ -116,9 +116,8 @@ variant_score_kernel(const T* __restrict__ keys, const VariantArgs a) {
         } else {
             float tr = 0.f;
             for (int f = 0; f < kF; ++f) {
-                const float* c = rec + (f >> 2) * kWChunk + 2 * (f & 3);
                 const float2 k = kb[f * kVarThreads + t];
-                tr = fmaf(__ldg(c), k.x, fmaf(__ldg(c + 1), k.y, tr));
+                tr = fmaf(__ldg(rec + wrec_re(f)), k.x, fmaf(__ldg(rec + wrec_im(f)), k.y, tr));
             }
             s = tr + s_norm;
         }

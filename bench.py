@@ -96,7 +96,7 @@ def fused_bytes(spec) -> int:
 # the workload up to one full launch (traffic grows with the units processed).
 TRAFFIC = {
     # profiles/prune_coop_kernel_c2_full.txt
-    ("c2", "prune_coop_kernel"): {"bytes_per_launch": 36226304, "src": "2885885db7594c5c"},
+    ("c2", "prune_coop_kernel"): {"bytes_per_launch": 36205824, "src": "c77c64c097379d81"},
     # profiles/prune_pipe_kernel_c3-2seq_full.txt: 224 of 1792 units captured, x 8
     ("c3", "prune_pipe_kernel"): {"bytes_per_launch": 7422631936, "src": "91d6d2f340ec24f9"},
     # profiles/score_kernel_c4-1seq-2layers_full.txt: 16 of 1024 units captured, x 64

@@ -264,6 +264,14 @@ zsel_compact_kernel(const float* __restrict__ fin, int64_t cap, const int32_t* _
             if (j < n) out[j] = j;
         }
     } else if (Bu > 0) {
+        // Every score load of the thread is issued before the first use of
+        // the unit's state (and before the first ballot).
+        float fv[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int j = j0 + 32 * i + lane;
+            fv[i] = j < n ? __ldcs(&fin[u * cap + j]) : 0.f;
+        }
         const ZSelState s = st[u];
         const uint2 base = counts[u * gridDim.x + blockIdx.x];
         uint32_t key[8];
@@ -272,7 +280,7 @@ zsel_compact_kernel(const float* __restrict__ fin, int64_t cap, const int32_t* _
         for (int i = 0; i < 8; ++i) {
             const int j = j0 + 32 * i + lane;
             const bool valid = j < n;
-            key[i] = valid ? ordered_key(fin[u * cap + j]) : 0u;
+            key[i] = valid ? ordered_key(fv[i]) : 0u;
             gt += __popc(__ballot_sync(0xffffffffu, valid && key[i] > s.T));
             eq += __popc(__ballot_sync(0xffffffffu, valid && key[i] == s.T));
         }
